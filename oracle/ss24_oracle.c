@@ -1,0 +1,648 @@
+/*
+ * ss24 oracle: a plain, slow CPU statement of the online 2:4 prune / compress /
+ * quantize pass and of its error energies.
+ *
+ * TEST INFRASTRUCTURE. Only the test suite, the package smoke check and the
+ * benchmark's CPU-baseline leg load this library. The product path (the CUDA
+ * library and its Python binding) never calls, links or imports it, and this
+ * file includes nothing from the product path.
+ *
+ * Style: every step is a scalar loop, in the order the method states it. A
+ * decision that yields an integer (which elements are kept, which code a value
+ * gets) is taken in IEEE binary32 with round-to-nearest-even and no
+ * contraction, because that is the precision the kernels decide in. Error
+ * energies are accumulated in binary64, row-major, one element at a time.
+ * Build with -ffp-contract=off and without fast-math.
+ *
+ * Sources. "Is 2:4 Sparsity Still Worth It? Semi-Structured Sparsity versus
+ * Quantization in LLM Inference" (English digest on paper-daily.com):
+ *   intro .......... 2:4 keeps two non-zeros of every four along the reduction axis
+ *   §1 ............. online operands are pruned and compressed before every GEMM
+ *   §2 ............. equal bits (a 1-bit index per original element), the
+ *                    magnitude and Wanda scores, round-to-nearest quantization
+ *   §3 ............. the formats: FP8, INT8 with one scale per row, NVFP4
+ *                    (FP8 scale per 16 plus one per tensor), MXFP4 (one
+ *                    power-of-two scale per 32); the fused read-once kernel
+ *   §4 ............. 2:4 energy loss, disjoint pruning / quantization error
+ *                    energies, predicted R
+ *   §6 ............. pairwise 4:8 (keep two of four adjacent pairs per eight)
+ * Where the pages leave a format detail open the oracle follows the OCP 8-bit
+ * Floating Point (OFP8) and OCP Microscaling (MX) v1.0 definitions.
+ *
+ * Readings of points the pages leave open (tie rule, metadata nibble layout,
+ * scales over the compressed row, symmetric integer range, NVFP4 two-level
+ * recipe, MX shared exponent) are stated at the function that takes them.
+ *
+ * Parity status: every function here is pinned by a CPU test against
+ * something other than itself (brute force, a library routine, a closed form
+ * or a figure printed on the pages). None is "parity unpinned".
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* Enumerations. Same numeric values as the product's C header; restated here
+ * because the oracle shares no header with the product. */
+enum { OR_BF16 = 0, OR_F32 = 1 };
+enum { OR_SCORE_MAG = 0, OR_SCORE_WANDA = 1 };
+enum { OR_DENSE = 0, OR_SPARSE_24 = 24, OR_SPARSE_48 = 48 };
+enum { OR_FMT_NONE = 0, OR_FMT_FP8 = 1, OR_FMT_INT = 2, OR_FMT_NVFP4 = 3, OR_FMT_MXFP4 = 4 };
+
+typedef struct {
+    const void *x;        /* operand bytes (bf16 as raw uint16, or fp32)              */
+    int32_t dtype;        /* OR_BF16 / OR_F32                                           */
+    int32_t axis;         /* 1: element (r,c) at x[r*ld + c]; 0: at x[c*ld + r]         */
+    int64_t rows, k, ld;  /* logical operand A[rows][k], reduction along k             */
+    int32_t pattern;      /* OR_DENSE, OR_SPARSE_24, OR_SPARSE_48                       */
+    int32_t score;        /* OR_SCORE_MAG, OR_SCORE_WANDA                               */
+    const float *norms;   /* Wanda per-input-channel norms, length k (or NULL)          */
+    int32_t fmt, bits, group, pack4;
+    const float *tensor_scale_in; /* host pointer to a given per-tensor scale, or NULL   */
+} oracle_args;
+
+typedef struct {
+    void *values;         /* kept values (format NONE) or codes                        */
+    void *scales;         /* INT: fp32 per group; NVFP4: E4M3 bytes; MXFP4: E8M0 bytes  */
+    float *tensor_scale;  /* FP8 / NVFP4: the per-tensor scale used                     */
+    uint8_t *meta;        /* 2:4 / 4:8 position metadata                                */
+} oracle_outputs;
+
+/* ------------------------------------------------------------------------- */
+/* Number formats                                                             */
+/* ------------------------------------------------------------------------- */
+
+/* bf16 is the upper half of a binary32; widening is exact. */
+float oracle_bf16_to_f32(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+/* Exact floor(log2(a)) for finite a > 0, subnormals included (frexpf is exact). */
+int oracle_floor_log2(float a)
+{
+    int e;
+    (void)frexpf(a, &e); /* a = f * 2^e with f in [0.5, 1) */
+    return e - 1;
+}
+
+/* Round a non-negative magnitude to the nearest multiple of `step` (a power of
+ * two), ties to the even multiple. a/step is exact (power-of-two scaling). */
+static float round_to_step(float a, float step)
+{
+    float q = a / step;
+    float n = nearbyintf(q); /* default mode: round half to even */
+    return n * step;
+}
+
+/* OCP FP8 E4M3 ("fn"): 1 sign, 4 exponent bits with bias 7, 3 mantissa bits;
+ * no infinities; S.1111.111 is NaN; largest finite 448 = 1.75 * 2^8; smallest
+ * normal 2^-6; subnormal step 2^-9. */
+float oracle_e4m3_decode(uint8_t c)
+{
+    int s = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    float mag;
+    if (e == 15 && m == 7)
+        return s ? -NAN : NAN;
+    if (e == 0)
+        mag = ldexpf((float)m, -9); /* m/8 * 2^-6 */
+    else
+        mag = ldexpf(1.0f + (float)m / 8.0f, e - 7);
+    return s ? -mag : mag;
+}
+
+/* Encode a binary32 to E4M3 with one rounding, nearest-even, saturating to
+ * +-448 ("satfinite"); NaN stays NaN. The sign of a result that rounds to zero
+ * is kept (so -0 and tiny negatives give 0x80). */
+uint8_t oracle_e4m3_encode(float v)
+{
+    uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    float a = fabsf(v);
+    if (isnan(v))
+        return sign | 0x7F;
+    if (a >= 448.0f)
+        return sign | 0x7E;
+    /* Grid spacing: 2^(E-3) inside binade [2^E, 2^(E+1)) for E >= -6, and the
+     * subnormal spacing 2^-9 below 2^-6. */
+    float step;
+    if (a < ldexpf(1.0f, -6))
+        step = ldexpf(1.0f, -9);
+    else
+        step = ldexpf(1.0f, oracle_floor_log2(a) - 3);
+    float r = round_to_step(a, step); /* may round up into the next binade */
+    if (r > 448.0f)
+        r = 448.0f;
+    if (r == 0.0f)
+        return sign;
+    if (r < ldexpf(1.0f, -6))
+        return sign | (uint8_t)(r / ldexpf(1.0f, -9)); /* subnormal: e = 0 */
+    int E = oracle_floor_log2(r);
+    int m = (int)(ldexpf(r, -E) * 8.0f) - 8; /* r = (1 + m/8) * 2^E */
+    return sign | (uint8_t)(((E + 7) << 3) | m);
+}
+
+/* OCP E2M1 (FP4): 1 sign, 2 exponent bits with bias 1, 1 mantissa bit; the
+ * magnitudes are 0, 0.5, 1, 1.5, 2, 3, 4, 6; no infinities or NaN. */
+float oracle_e2m1_decode(uint8_t c)
+{
+    static const float mag[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+    float m = mag[c & 7];
+    return (c & 8) ? -m : m;
+}
+
+/* Encode to E2M1, nearest-even, saturating to +-6; the sign of zero is kept. */
+uint8_t oracle_e2m1_encode(float v)
+{
+    uint8_t sign = signbit(v) ? 0x8 : 0x0;
+    float a = fabsf(v);
+    if (a >= 6.0f)
+        return sign | 0x7;
+    /* Spacing 0.5 below 2 (subnormal 0..0.5 and binade [1,2)), 1 in [2,4), 2 in [4,8). */
+    float step = (a < 2.0f) ? 0.5f : (a < 4.0f ? 1.0f : 2.0f);
+    float r = round_to_step(a, step);
+    if (r > 6.0f)
+        r = 6.0f;
+    uint8_t code = 0;
+    for (uint8_t c = 0; c < 8; ++c)
+        if (oracle_e2m1_decode(c) == r)
+            code = c;
+    return sign | code;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Selection                                                                  */
+/* ------------------------------------------------------------------------- */
+
+/* Top-2 of a group of 4 scores (intro and §2: keep the two largest of every
+ * four). Tie rule (the pages give none): element i beats element j iff
+ * s_i > s_j, or s_i == s_j and i < j; an element is kept when fewer than two
+ * others beat it. Returns the metadata nibble i0 | i1 << 2 with i0 < i1. */
+int oracle_select24(const float s[4])
+{
+    int kept[2], nk = 0;
+    for (int i = 0; i < 4; ++i) {
+        int beaten = 0;
+        for (int j = 0; j < 4; ++j)
+            if (j != i && (s[j] > s[i] || (s[j] == s[i] && j < i)))
+                beaten++;
+        if (beaten < 2)
+            kept[nk++] = i;
+    }
+    return kept[0] | (kept[1] << 2);
+}
+
+/* Pairwise 4:8 (§6): eight elements form four adjacent pairs; a pair's rank is
+ * its energy e_p = s_{2p}^2 + s_{2p+1}^2 (binary32, multiply then add). The
+ * same beats-rule picks two pairs; returns the nibble p0 | p1 << 2. */
+int oracle_select48(const float s[8])
+{
+    float e[4];
+    for (int p = 0; p < 4; ++p) {
+        float a = s[2 * p] * s[2 * p];
+        float b = s[2 * p + 1] * s[2 * p + 1];
+        e[p] = a + b;
+    }
+    return oracle_select24(e);
+}
+
+/* ------------------------------------------------------------------------- */
+/* Row access and scores                                                      */
+/* ------------------------------------------------------------------------- */
+
+static float element(const oracle_args *a, int64_t r, int64_t c)
+{
+    int64_t off = (a->axis == 0) ? c * a->ld + r : r * a->ld + c;
+    if (a->dtype == OR_BF16)
+        return oracle_bf16_to_f32(((const uint16_t *)a->x)[off]);
+    return ((const float *)a->x)[off];
+}
+
+/* Score of element (r, c) (§2): magnitude |x|, or Wanda |x| * n_c where n_c is
+ * the norm of input channel c (product rounded to binary32). */
+static float score_of(const oracle_args *a, float x, int64_t c)
+{
+    if (a->score == OR_SCORE_WANDA)
+        return fabsf(x) * a->norms[c];
+    return fabsf(x);
+}
+
+/* Prune one row. Writes the kept values (in index order) to kept[k/2], their
+ * source indices to kidx, the metadata bytes to meta_row (when not NULL), and
+ * adds the row's energies: e_total += sum x^2, e_prune += sum over dropped x^2. */
+static void prune_row(const oracle_args *a, const float *xr, float *kept, int64_t *kidx,
+                      uint8_t *meta_row, double *e_total, double *e_prune)
+{
+    int64_t k = a->k;
+    int gsize = (a->pattern == OR_SPARSE_48) ? 8 : 4;
+    int64_t nk = 0;
+    for (int64_t g0 = 0; g0 < k; g0 += gsize) {
+        float s[8];
+        int keep[8] = {0};
+        int nib;
+        for (int i = 0; i < gsize; ++i)
+            s[i] = score_of(a, xr[g0 + i], g0 + i);
+        if (gsize == 4) {
+            nib = oracle_select24(s);
+            keep[nib & 3] = 1;
+            keep[nib >> 2] = 1;
+        } else {
+            nib = oracle_select48(s);
+            int p0 = nib & 3, p1 = nib >> 2;
+            keep[2 * p0] = keep[2 * p0 + 1] = 1;
+            keep[2 * p1] = keep[2 * p1 + 1] = 1;
+        }
+        if (meta_row) {
+            int64_t gi = g0 / gsize; /* group index: two groups share a byte */
+            if (gi % 2 == 0)
+                meta_row[gi / 2] = (uint8_t)nib;
+            else
+                meta_row[gi / 2] |= (uint8_t)(nib << 4);
+        }
+        for (int i = 0; i < gsize; ++i) {
+            double xd = (double)xr[g0 + i];
+            *e_total += xd * xd;
+            if (keep[i]) {
+                kept[nk] = xr[g0 + i];
+                kidx[nk] = g0 + i;
+                nk++;
+            } else {
+                *e_prune += xd * xd;
+            }
+        }
+    }
+}
+
+/* The vector that gets quantized for row r: the kept row (sparse) or the whole
+ * row (dense). Returns its length. */
+static int64_t quantized_row(const oracle_args *a, int64_t r, float *xr, float *v, int64_t *kidx,
+                             uint8_t *meta_row, double *e_total, double *e_prune)
+{
+    for (int64_t c = 0; c < a->k; ++c)
+        xr[c] = element(a, r, c);
+    if (a->pattern == OR_DENSE) {
+        for (int64_t c = 0; c < a->k; ++c) {
+            double xd = (double)xr[c];
+            *e_total += xd * xd;
+            v[c] = xr[c];
+        }
+        return a->k;
+    }
+    prune_row(a, xr, v, kidx, meta_row, e_total, e_prune);
+    return a->k / 2;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Quantizers (round to nearest; §2 "plain round-to-nearest", §3 formats).    */
+/* Each writes codes for one row vector v[n] and its dequantized values.      */
+/* ------------------------------------------------------------------------- */
+
+
+typedef struct {
+    const oracle_args *a;
+    oracle_outputs *o;
+    int64_t n;          /* length of the quantized row (k/2 sparse, k dense) */
+    float tensor_scale; /* FP8 / NVFP4 per-tensor scale */
+} qctx;
+
+/* Symmetric INT-b with one fp32 scale per `group` consecutive values of the
+ * quantized row; group 0 means one scale per row (the "INT8 with a single
+ * scale per row" of §3). Reading: restricted range +-(2^(b-1) - 1);
+ * scale = amax / qmax; code = clamp(round_half_even(v / scale)); a zero scale
+ * gives all-zero codes. Codes are stored as int8 (b <= 8), int16 (b > 8), or,
+ * with pack4 and b <= 4, as two's-complement nibbles two per byte, the lower
+ * index in the low nibble. */
+static void quant_int_row(const qctx *q, int64_t r, const float *v, float *deq)
+{
+    const oracle_args *a = q->a;
+    int64_t n = q->n;
+    int64_t g = a->group ? a->group : n;
+    float qmax = (float)((1 << (a->bits - 1)) - 1);
+    for (int64_t j0 = 0; j0 < n; j0 += g) {
+        float amax = 0.0f;
+        for (int64_t j = j0; j < j0 + g; ++j)
+            if (fabsf(v[j]) > amax)
+                amax = fabsf(v[j]);
+        float scale = amax / qmax;
+        if (q->o->scales)
+            ((float *)q->o->scales)[r * (n / g) + j0 / g] = scale;
+        for (int64_t j = j0; j < j0 + g; ++j) {
+            int code = 0;
+            if (scale != 0.0f) {
+                float t = nearbyintf(v[j] / scale);
+                if (t > qmax)
+                    t = qmax;
+                if (t < -qmax)
+                    t = -qmax;
+                code = (int)t;
+            }
+            deq[j] = (float)code * scale;
+            if (!q->o->values)
+                continue;
+            if (a->pack4) {
+                uint8_t *p = (uint8_t *)q->o->values + r * (n / 2) + j / 2;
+                if (j % 2 == 0)
+                    *p = (uint8_t)(code & 0xF);
+                else
+                    *p |= (uint8_t)((code & 0xF) << 4);
+            } else if (a->bits > 8) {
+                ((int16_t *)q->o->values)[r * n + j] = (int16_t)code;
+            } else {
+                ((int8_t *)q->o->values)[r * n + j] = (int8_t)code;
+            }
+        }
+    }
+}
+
+/* FP8 E4M3 with one scale per tensor (§3 "FP8"; the pages fix no granularity,
+ * per-tensor is the reading): s = amax / 448; code = E4M3(v / s);
+ * deq = decode(code) * s; s == 0 gives zero codes. */
+static void quant_fp8_row(const qctx *q, int64_t r, const float *v, float *deq)
+{
+    float s = q->tensor_scale;
+    for (int64_t j = 0; j < q->n; ++j) {
+        uint8_t code = 0;
+        if (s != 0.0f)
+            code = oracle_e4m3_encode(v[j] / s);
+        deq[j] = oracle_e4m3_decode(code) * s;
+        if (q->o->values)
+            ((uint8_t *)q->o->values)[r * q->n + j] = code;
+    }
+}
+
+/* NVFP4 (§3: 4-bit float, an FP8 scale per 16 elements plus one scale per
+ * tensor). Reading of the two-level recipe: s_t = amax / (6 * 448); for each
+ * block of 16, sb = E4M3((amax_block / 6) / s_t) (two divisions in that
+ * order); denom = decode(sb) * s_t; code = E2M1(v / denom); a zero s_t or
+ * denom gives zero codes. Codes two per byte, lower index in the low nibble. */
+static void quant_nvfp4_row(const qctx *q, int64_t r, const float *v, float *deq)
+{
+    float st = q->tensor_scale;
+    int64_t n = q->n;
+    for (int64_t j0 = 0; j0 < n; j0 += 16) {
+        float amax = 0.0f;
+        for (int64_t j = j0; j < j0 + 16; ++j)
+            if (fabsf(v[j]) > amax)
+                amax = fabsf(v[j]);
+        uint8_t sb = 0;
+        if (st != 0.0f)
+            sb = oracle_e4m3_encode((amax / 6.0f) / st);
+        float denom = oracle_e4m3_decode(sb) * st;
+        if (q->o->scales)
+            ((uint8_t *)q->o->scales)[r * (n / 16) + j0 / 16] = sb;
+        for (int64_t j = j0; j < j0 + 16; ++j) {
+            uint8_t code = 0;
+            if (denom != 0.0f)
+                code = oracle_e2m1_encode(v[j] / denom);
+            deq[j] = oracle_e2m1_decode(code) * denom;
+            if (q->o->values) {
+                uint8_t *p = (uint8_t *)q->o->values + r * (n / 2) + j / 2;
+                if (j % 2 == 0)
+                    *p = code;
+                else
+                    *p |= (uint8_t)(code << 4);
+            }
+        }
+    }
+}
+
+/* MXFP4 (§3: 32 elements share one power-of-two scale). Reading, from OCP MX
+ * v1.0: shared exponent e = floor(log2(amax_block)) - 2 (2 = largest E2M1
+ * exponent), clamped to [-127, 127], stored as the E8M0 byte e + 127;
+ * code = E2M1(v / 2^e); an all-zero block stores byte 0 and zero codes. */
+static void quant_mxfp4_row(const qctx *q, int64_t r, const float *v, float *deq)
+{
+    int64_t n = q->n;
+    for (int64_t j0 = 0; j0 < n; j0 += 32) {
+        float amax = 0.0f;
+        for (int64_t j = j0; j < j0 + 32; ++j)
+            if (fabsf(v[j]) > amax)
+                amax = fabsf(v[j]);
+        uint8_t byte = 0;
+        float scale = 0.0f;
+        if (amax != 0.0f) {
+            int e = oracle_floor_log2(amax) - 2;
+            if (e < -127)
+                e = -127;
+            if (e > 127)
+                e = 127;
+            byte = (uint8_t)(e + 127);
+            scale = ldexpf(1.0f, e);
+        }
+        if (q->o->scales)
+            ((uint8_t *)q->o->scales)[r * (n / 32) + j0 / 32] = byte;
+        for (int64_t j = j0; j < j0 + 32; ++j) {
+            uint8_t code = 0;
+            if (scale != 0.0f)
+                code = oracle_e2m1_encode(v[j] / scale);
+            deq[j] = oracle_e2m1_decode(code) * scale;
+            if (q->o->values) {
+                uint8_t *p = (uint8_t *)q->o->values + r * (n / 2) + j / 2;
+                if (j % 2 == 0)
+                    *p = code;
+                else
+                    *p |= (uint8_t)(code << 4);
+            }
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------- */
+/* The pass                                                                   */
+/* ------------------------------------------------------------------------- */
+
+/* Largest |value| among the values that get quantized: the kept values for a
+ * sparse pattern (reading: a per-tensor scale is taken over what is stored),
+ * every value for the dense pattern. */
+float oracle_amax(const oracle_args *a)
+{
+    int64_t k = a->k;
+    float *xr = malloc(sizeof(float) * k), *v = malloc(sizeof(float) * k);
+    int64_t *kidx = malloc(sizeof(int64_t) * k);
+    double et = 0.0, ep = 0.0;
+    float amax = 0.0f;
+    for (int64_t r = 0; r < a->rows; ++r) {
+        int64_t n = quantized_row(a, r, xr, v, kidx, NULL, &et, &ep);
+        for (int64_t j = 0; j < n; ++j)
+            if (fabsf(v[j]) > amax)
+                amax = fabsf(v[j]);
+    }
+    free(xr);
+    free(v);
+    free(kidx);
+    return amax;
+}
+
+/* Argument checks the oracle needs to run at all (it does not restate the
+ * product's validation). Returns 0 when the arguments are usable. */
+static int check_args(const oracle_args *a)
+{
+    if (!a->x || a->rows < 0 || a->k <= 0)
+        return 1;
+    if (a->pattern == OR_SPARSE_24 && a->k % 8)
+        return 2;
+    if (a->pattern == OR_SPARSE_48 && a->k % 16)
+        return 2;
+    if (a->score == OR_SCORE_WANDA && !a->norms)
+        return 3;
+    int64_t n = a->pattern == OR_DENSE ? a->k : a->k / 2;
+    switch (a->fmt) {
+    case OR_FMT_NONE:
+        return a->pattern == OR_DENSE ? 4 : 0;
+    case OR_FMT_FP8:
+        return 0;
+    case OR_FMT_INT:
+        if (a->bits < 2 || a->bits > 16)
+            return 4;
+        if (a->group && n % a->group)
+            return 4;
+        if (a->pack4 && (a->bits > 4 || n % 2))
+            return 4;
+        return 0;
+    case OR_FMT_NVFP4:
+        return n % 16 ? 4 : 0;
+    case OR_FMT_MXFP4:
+        return n % 32 ? 4 : 0;
+    }
+    return 4;
+}
+
+/* One pass of the method over the operand: score, select, compress (sparse
+ * patterns), quantize the stored values, and the error energies
+ *   energy[0] = E_total = sum over all elements of x^2
+ *   energy[1] = E_prune = sum over dropped elements of x^2
+ *   energy[2] = E_q     = sum over kept elements of (x - deq)^2  (sparse)
+ *   energy[3] = E_q,dense = sum over all elements of (x - deq)^2 (dense)
+ * (§4: dropped elements carry only pruning error, kept ones only quantization
+ * error). Format NONE stores the kept values unchanged and has E_q = 0.
+ * Output layouts (all rows of the logical operand, k contiguous):
+ *   values: NONE -> kept values in the input dtype [rows][k/2];
+ *           FP8 -> u8 [rows][n]; INT -> int8/int16 [rows][n] or packed [rows][n/2];
+ *           NVFP4 / MXFP4 -> u8 [rows][n/2]
+ *   scales: INT fp32 [rows][n/group]; NVFP4 u8 [rows][n/16]; MXFP4 u8 [rows][n/32]
+ *   meta:   2:4 -> u8 [rows][k/8], group g's nibble i0 | i1 << 2 in byte g/2,
+ *           even g in the low nibble; 4:8 -> u8 [rows][k/16], same per octet.
+ * Returns 0 on success, nonzero when the arguments are unusable. */
+int oracle_run(const oracle_args *a, oracle_outputs *o, double *energy)
+{
+    int bad = check_args(a);
+    if (bad)
+        return bad;
+    int64_t k = a->k, n = a->pattern == OR_DENSE ? k : k / 2;
+    qctx q = {a, o, n, 0.0f};
+    if (a->fmt == OR_FMT_FP8 || a->fmt == OR_FMT_NVFP4) {
+        if (a->tensor_scale_in) {
+            q.tensor_scale = *a->tensor_scale_in;
+        } else {
+            float amax = oracle_amax(a);
+            q.tensor_scale = a->fmt == OR_FMT_FP8 ? amax / 448.0f : amax / 2688.0f;
+        }
+        if (o->tensor_scale)
+            *o->tensor_scale = q.tensor_scale;
+    }
+    float *xr = malloc(sizeof(float) * k), *v = malloc(sizeof(float) * k);
+    float *deq = malloc(sizeof(float) * k);
+    int64_t *kidx = malloc(sizeof(int64_t) * k);
+    double e_total = 0.0, e_prune = 0.0, e_q = 0.0;
+    int64_t meta_bytes = a->pattern == OR_SPARSE_48 ? k / 16 : k / 8;
+    for (int64_t r = 0; r < a->rows; ++r) {
+        uint8_t *meta_row = (o->meta && a->pattern != OR_DENSE) ? o->meta + r * meta_bytes : NULL;
+        quantized_row(a, r, xr, v, kidx, meta_row, &e_total, &e_prune);
+        switch (a->fmt) {
+        case OR_FMT_NONE:
+            for (int64_t j = 0; j < n; ++j) {
+                deq[j] = v[j];
+                if (!o->values)
+                    continue;
+                if (a->dtype == OR_BF16) {
+                    /* the kept value is stored bit-for-bit */
+                    int64_t off = a->axis == 0 ? kidx[j] * a->ld + r : r * a->ld + kidx[j];
+                    ((uint16_t *)o->values)[r * n + j] = ((const uint16_t *)a->x)[off];
+                } else {
+                    ((float *)o->values)[r * n + j] = v[j];
+                }
+            }
+            break;
+        case OR_FMT_FP8:
+            quant_fp8_row(&q, r, v, deq);
+            break;
+        case OR_FMT_INT:
+            quant_int_row(&q, r, v, deq);
+            break;
+        case OR_FMT_NVFP4:
+            quant_nvfp4_row(&q, r, v, deq);
+            break;
+        case OR_FMT_MXFP4:
+            quant_mxfp4_row(&q, r, v, deq);
+            break;
+        }
+        for (int64_t j = 0; j < n; ++j) {
+            double d = (double)v[j] - (double)deq[j];
+            e_q += d * d;
+        }
+    }
+    if (energy) {
+        energy[0] = e_total;
+        energy[1] = e_prune;
+        energy[2] = a->pattern == OR_DENSE ? 0.0 : e_q;
+        energy[3] = a->pattern == OR_DENSE ? e_q : 0.0;
+    }
+    free(xr);
+    free(v);
+    free(deq);
+    free(kidx);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Derived quantities (§4) and equal-bit accounting (§2)                      */
+/* ------------------------------------------------------------------------- */
+
+/* From the sparse side's energies (E_total, E_prune, E_q at 2m bits) and the
+ * dense side's (E_q,dense at m+1 bits):
+ *   out[0] = 2:4 energy loss          = E_prune / E_total
+ *   out[1] = sparse relative error    = sqrt((E_prune + E_q) / E_total)
+ *   out[2] = dense relative error     = sqrt(E_q,dense / E_total)
+ *   out[3] = predicted R              = sqrt((E_prune + E_q) / E_q,dense)
+ * E_total is taken from the sparse side (both sides see the same tensor). */
+void oracle_ratio(const double *sparse_e, const double *dense_e, double *out)
+{
+    double et = sparse_e[0], ep = sparse_e[1], eq = sparse_e[2], ed = dense_e[3];
+    out[0] = ep / et;
+    out[1] = sqrt((ep + eq) / et);
+    out[2] = sqrt(ed / et);
+    out[3] = sqrt((ep + eq) / ed);
+}
+
+/* Stored bits per ORIGINAL element (§2: every stored bit is charged, values,
+ * indices and scales). Value bits: NONE -> 16 (bf16); FP8 -> 8; INT -> bits;
+ * NVFP4 / MXFP4 -> 4. A sparse pattern keeps half the values and adds its
+ * position index: 2:4 -> 2 bits per kept value = 1 bit per original element;
+ * 4:8 -> 2 bits per 8 elements = 0.25. Scale bits (with_scales): INT 32 bits
+ * per group (group 0: per row of k_q values), NVFP4 8 per 16 plus 32 per
+ * tensor (ignored, O(1/size)), MXFP4 8 per 32 quantized values. */
+double oracle_bits_per_element(int32_t fmt, int32_t bits, int32_t group, int32_t pattern,
+                               int64_t k, int32_t with_scales)
+{
+    double vb = fmt == OR_FMT_NONE ? 16.0
+              : fmt == OR_FMT_FP8 ? 8.0
+              : fmt == OR_FMT_INT ? (double)bits
+              : 4.0;
+    double kept_frac = pattern == OR_DENSE ? 1.0 : 0.5;
+    double index_bits = pattern == OR_SPARSE_24 ? 1.0 : pattern == OR_SPARSE_48 ? 0.25 : 0.0;
+    double total = kept_frac * vb + index_bits;
+    if (with_scales) {
+        double nq = kept_frac * (double)k; /* quantized values per row */
+        double per_q = 0.0;
+        if (fmt == OR_FMT_INT)
+            per_q = 32.0 / (group ? (double)group : nq);
+        else if (fmt == OR_FMT_NVFP4)
+            per_q = 8.0 / 16.0;
+        else if (fmt == OR_FMT_MXFP4)
+            per_q = 8.0 / 32.0;
+        total += kept_frac * per_q;
+    }
+    return total;
+}
