@@ -1,0 +1,302 @@
+/*
+ * ss24.h — C ABI of the online 2:4 prune / compress / quantize / error-energy
+ * library for NVIDIA B200 (sm_100a).
+ *
+ * What it computes. "Is 2:4 Sparsity Still Worth It? Semi-Structured Sparsity
+ * versus Quantization in LLM Inference" (English digest, paper-daily.com):
+ *   intro  2:4 keeps two non-zeros of every four along a GEMM operand's
+ *          reduction axis.
+ *   §1     operands computed on the fly (activations, Q, K, V, P) must be
+ *          pruned and compressed before every GEMM, and that cost counts.
+ *   §2     the pruners' scores (magnitude; Wanda = |W| times the activation
+ *          size of the input channel), plain round-to-nearest quantization,
+ *          and equal-bit accounting (a 1-bit index per original element).
+ *   §3     the formats (FP8, INT8 with one scale per row, NVFP4, MXFP4) and the
+ *          fused kernel that reads the input once and writes kept values and
+ *          indices once.
+ *   §4     the 2:4 energy loss, the disjoint pruning / quantization error
+ *          energies and the predicted ratio R.
+ *   §6     pairwise 4:8 (keep two of the four adjacent pairs of each eight).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Operand. A logical matrix A[rows][k]; k is the reduction axis, along which
+ * groups of 4 (2:4) or 8 (4:8) consecutive elements are formed. Memory:
+ *   axis = 1: A[r][c] is at x[r * ld + c]   (k contiguous; ld >= k)
+ *   axis = 0: A[r][c] is at x[c * ld + r]   (rows contiguous, e.g. V pruned
+ *             along the key axis; ld >= rows)
+ * Element type bf16 or fp32. Inputs are finite; NaN / Inf give unspecified
+ * codes. Energies are accurate for |x| below 2^60 (binary32 squares).
+ *
+ * Outputs are always row-major with k (or the kept half of it) contiguous,
+ * one row per logical row, no padding. With n = k/2 for a sparse pattern and
+ * n = k for the dense pattern:
+ *   kept values (format NONE)  input dtype [rows][n]
+ *   FP8 E4M3 codes             u8 [rows][n]
+ *   INT codes                  int8 [rows][n] (bits <= 8), int16 [rows][n]
+ *                              (bits > 8), or with pack4 (bits <= 4) u8
+ *                              [rows][n/2], two's-complement nibbles, element
+ *                              2j in the low nibble
+ *   INT scales                 fp32 [rows][n/group] (group 0: [rows][1])
+ *   NVFP4 codes / scales       u8 [rows][n/2] (element 2j in the low nibble) /
+ *                              E4M3 u8 [rows][n/16], plus fp32 tensor scale
+ *   MXFP4 codes / scales       u8 [rows][n/2] / E8M0 u8 [rows][n/32]
+ *   2:4 metadata               u8 [rows][k/8]: group g's nibble i0 | i1 << 2
+ *                              (kept positions, i0 < i1) in byte g/2, even g in
+ *                              the low nibble
+ *   4:8 metadata               u8 [rows][k/16]: octet o's nibble p0 | p1 << 2
+ *                              (kept pairs) in byte o/2, even o in the low nibble
+ * Scales of the kept values are taken over the compressed row: an INT group of
+ * g covers g kept values (2g original positions), an NVFP4 block 16 kept
+ * values, an MXFP4 block 32.
+ *
+ * Selection. Element i beats element j when s_i > s_j, or s_i == s_j and
+ * i < j; the two elements beaten by fewer than two others are kept (ties keep
+ * the lower index). Scores: SS24_SCORE_MAG s = |x|; SS24_SCORE_WANDA
+ * s = |x| * col_norms[c] rounded to binary32 (col_norms: fp32 [k], >= 0).
+ * Pairwise 4:8 ranks pair p by s_{2p}*s_{2p} + s_{2p+1}*s_{2p+1} (binary32,
+ * each product and the sum rounded) with the same rule over the four pairs.
+ *
+ * Quantization (round to nearest, ties to even; every division is an IEEE
+ * binary32 division, every product one binary32 rounding, no contraction):
+ *   FP8    s = amax / 448; code = E4M3satfinite(v / s); deq = E4M3(code) * s
+ *   INT-b  qmax = 2^(b-1) - 1; scale = amax_group / qmax;
+ *          code = clamp(rint(v / scale), -qmax, qmax); deq = code * scale
+ *   NVFP4  s_t = amax / 2688; sb = E4M3satfinite((amax_block / 6) / s_t);
+ *          denom = E4M3(sb) * s_t; code = E2M1satfinite(v / denom);
+ *          deq = E2M1(code) * denom
+ *   MXFP4  e = clamp(floor(log2(amax_block)) - 2, -127, 127); byte = e + 127;
+ *          code = E2M1satfinite(v / 2^e); deq = E2M1(code) * 2^e
+ * A zero scale (or zero block amax for MXFP4, which then stores byte 0) gives
+ * all-zero codes. The per-tensor amax of a sparse pattern is taken over the
+ * kept values (equal to the amax of all values for the magnitude score).
+ *
+ * Energies. ss24_energy holds binary64 sums (§4):
+ *   e_total        sum over all elements of x^2
+ *   e_prune        sum over dropped elements of x^2
+ *   e_quant        sum over kept elements of (x - deq)^2 (sparse side)
+ *   e_quant_dense  sum over all elements of (x - deq)^2 (dense side)
+ * Fields a call does not compute are written as 0. Per-element terms are
+ * formed in binary32 and summed in short binary32 trees before binary64
+ * accumulation; the sums match a binary64 reference to about 5e-7 relative.
+ * Results are deterministic run to run (fixed reduction order, no atomics).
+ *
+ * Memory and ownership. Every pointer argument except the descriptor structs
+ * is DEVICE memory owned by the caller; the library allocates nothing and
+ * keeps no state between calls. The descriptor structs (ss24_operand,
+ * ss24_outputs) are read on the host during the call and may be reused
+ * immediately. Data pointers must be 16-byte aligned and, for axis 1,
+ * ld * sizeof(dtype) must be a multiple of 16 (axis 0: likewise).
+ *
+ * Workspace. Calls take a device workspace of ss24_workspace_bytes() bytes,
+ * 256-byte aligned, that must have been cleared once with
+ * ss24_workspace_init(). Concurrent calls need distinct workspaces.
+ *
+ * Asynchrony and errors. Every call validates its arguments on the host and,
+ * if they are invalid, returns an SS24_ERR_* status and launches nothing.
+ * Otherwise it enqueues its kernels on `stream` (NULL: the legacy default
+ * stream) and returns SS24_OK, or SS24_ERR_CUDA if a launch failed. Results
+ * are valid once the stream is synchronized. Kernels never trap: an internal
+ * wait that exceeds about two seconds records a nonzero code in the
+ * workspace (read with ss24_workspace_error) and the kernel returns.
+ */
+#ifndef SS24_H
+#define SS24_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *ss24_stream;
+
+typedef enum {
+    SS24_OK = 0,
+    SS24_ERR_NULL = 1,      /* a required pointer is NULL                            */
+    SS24_ERR_SHAPE = 2,     /* rows / k / ld do not fit the pattern or format        */
+    SS24_ERR_ALIGN = 3,     /* a pointer or the row stride is not 16-byte aligned    */
+    SS24_ERR_DTYPE = 4,     /* unknown element type                                  */
+    SS24_ERR_FORMAT = 5,    /* unknown format, bits out of range, bad group / pack4  */
+    SS24_ERR_WORKSPACE = 6, /* workspace missing, too small or misaligned            */
+    SS24_ERR_CUDA = 7,      /* a CUDA runtime call or a launch failed                */
+    SS24_ERR_ARG = 8        /* unknown score, axis or pattern                        */
+} ss24_status;
+
+typedef enum { SS24_BF16 = 0, SS24_F32 = 1 } ss24_dtype;
+typedef enum { SS24_SCORE_MAG = 0, SS24_SCORE_WANDA = 1 } ss24_score;
+typedef enum { SS24_DENSE = 0, SS24_SPARSE_24 = 24, SS24_SPARSE_48 = 48 } ss24_pattern;
+typedef enum {
+    SS24_FMT_NONE = 0,     /* kept values stored unchanged (sparse patterns only) */
+    SS24_FMT_FP8_E4M3 = 1, /* per-tensor scale                                    */
+    SS24_FMT_INT = 2,      /* bits 2..16, per-group or per-row fp32 scales        */
+    SS24_FMT_NVFP4 = 3,
+    SS24_FMT_MXFP4 = 4
+} ss24_fmt_kind;
+
+/* Quantization format. `bits`, `group`, `pack4` are read for SS24_FMT_INT only:
+ * bits in [2, 16]; group = 0 (one scale per row) or a power of two g with
+ * 8 <= g * (2 for sparse, 1 for dense) <= 256 dividing the quantized row;
+ * pack4 = 1 packs two codes per byte (bits <= 4). */
+typedef struct {
+    int32_t kind;
+    int32_t bits;
+    int32_t group;
+    int32_t pack4;
+} ss24_format;
+
+typedef struct {
+    const void *x; /* device pointer to the operand                      */
+    int32_t dtype; /* ss24_dtype                                          */
+    int32_t axis;  /* 1: k contiguous; 0: rows contiguous                 */
+    int64_t rows;  /* logical rows (>= 0; 0 is a valid empty operand)     */
+    int64_t k;     /* reduction length (> 0)                              */
+    int64_t ld;    /* elements between consecutive rows (axis 1) or
+                      consecutive k positions (axis 0)                    */
+} ss24_operand;
+
+typedef struct {
+    double e_total, e_prune, e_quant, e_quant_dense;
+} ss24_energy;
+
+typedef struct {
+    double loss;           /* e_prune / e_total                                   */
+    double rel_err_sparse; /* sqrt((e_prune + e_quant) / e_total)                 */
+    double rel_err_dense;  /* sqrt(e_quant_dense / e_total)                       */
+    double r_hat;          /* sqrt((e_prune + e_quant) / e_quant_dense), §4       */
+} ss24_ratio;
+
+typedef struct {
+    void *values;        /* kept values or codes (layout above)                 */
+    void *scales;        /* INT / NVFP4 / MXFP4 scales; NULL for NONE and FP8    */
+    float *tensor_scale; /* FP8 / NVFP4: receives the per-tensor scale used     */
+    uint8_t *meta;       /* metadata (sparse patterns); NULL for dense           */
+} ss24_outputs;
+
+/* ---- workspace ----------------------------------------------------------- */
+
+/* Bytes of device workspace every computing call needs (a constant). */
+size_t ss24_workspace_bytes(void);
+
+/* Clears the workspace's error word (stream-ordered memset). Call once after
+ * allocating the workspace, and again to reset a recorded error. */
+ss24_status ss24_workspace_init(void *ws, size_t ws_bytes, ss24_stream stream);
+
+/* Synchronizes `stream`, then copies the workspace's error word to *code
+ * (0: no kernel gave up on a wait). */
+ss24_status ss24_workspace_error(const void *ws, int32_t *code, ss24_stream stream);
+
+/* ---- the pass -------------------------------------------------------------- */
+
+/* 2:4 prune + compress (intro, §2 scores, §3 fused read-once / write-once
+ * kernel). Writes the kept values in the input dtype to `kept` [rows][k/2] and
+ * the metadata to `meta` [rows][k/8]. `energy` (may be NULL) receives e_total
+ * and e_prune. col_norms is required for SS24_SCORE_WANDA, ignored otherwise.
+ * k must be a multiple of 8. */
+ss24_status ss24_prune24_compress(const ss24_operand *x, ss24_score score, const float *col_norms,
+                                  void *kept, uint8_t *meta, ss24_energy *energy, void *ws,
+                                  size_t ws_bytes, ss24_stream stream);
+
+/* Dense FP8 E4M3 with one scale per tensor (§3). tensor_scale_in: device
+ * pointer to a given scale s, or NULL to compute s = amax / 448 (an extra
+ * read-only pass). out->values u8 [rows][k]; out->tensor_scale receives s.
+ * energy (may be NULL) receives e_total and e_quant_dense. k % 8 == 0. */
+ss24_status ss24_quantize_fp8(const ss24_operand *x, const float *tensor_scale_in,
+                              ss24_outputs *out, ss24_energy *energy, void *ws, size_t ws_bytes,
+                              ss24_stream stream);
+
+/* Dense symmetric INT-b with per-group or per-row scales (§3 "INT8 with a
+ * single scale per row"; §2 equal-bit partners INT3 ... INT9). fmt.kind must be
+ * SS24_FMT_INT. energy receives e_total and e_quant_dense. */
+ss24_status ss24_quantize_int(const ss24_operand *x, ss24_format fmt, ss24_outputs *out,
+                              ss24_energy *energy, void *ws, size_t ws_bytes, ss24_stream stream);
+
+/* Dense NVFP4 (§3: FP8 scale per 16 plus one per tensor). tensor_scale_in as
+ * for FP8 (NULL: s_t = amax / 2688). k % 16 == 0. */
+ss24_status ss24_quantize_nvfp4(const ss24_operand *x, const float *tensor_scale_in,
+                                ss24_outputs *out, ss24_energy *energy, void *ws, size_t ws_bytes,
+                                ss24_stream stream);
+
+/* Dense MXFP4 (§3: one power-of-two scale per 32). k % 32 == 0. */
+ss24_status ss24_quantize_mxfp4(const ss24_operand *x, ss24_outputs *out, ss24_energy *energy,
+                                void *ws, size_t ws_bytes, ss24_stream stream);
+
+/* The fused online pass (§3): one read of the operand, 2:4 selection, and the
+ * kept values written once, quantized to `fmt` (NONE: unchanged), with the
+ * metadata; energy receives e_total, e_prune and e_quant (§4).
+ * tensor_scale_in is read for FP8 / NVFP4 (NULL: computed from the amax of
+ * the kept values by an extra read-only pass). Constraints: k % 8 == 0 and the
+ * format's unit on the kept row (NVFP4 k % 32, MXFP4 k % 64, INT k % (2g)). */
+ss24_status ss24_prune24_quant_fused(const ss24_operand *x, ss24_score score,
+                                     const float *col_norms, ss24_format fmt,
+                                     const float *tensor_scale_in, ss24_outputs *out,
+                                     ss24_energy *energy, void *ws, size_t ws_bytes,
+                                     ss24_stream stream);
+
+/* Pairwise 4:8 variant of the fused pass (§6: keep two of the four adjacent
+ * pairs of each eight, ranked by pair energy). meta is u8 [rows][k/16];
+ * k % 16 == 0. Otherwise as ss24_prune24_quant_fused. */
+ss24_status ss24_prune48_pairwise_quant_fused(const ss24_operand *x, ss24_score score,
+                                              const float *col_norms, ss24_format fmt,
+                                              const float *tensor_scale_in, ss24_outputs *out,
+                                              ss24_energy *energy, void *ws, size_t ws_bytes,
+                                              ss24_stream stream);
+
+/* Read-only analysis pass (§4): in one read of the operand, the energies of
+ * both sides of the comparison — pattern (2:4 or 4:8) with its kept values
+ * quantized to sparse_fmt (2m bits; NONE allowed), and the whole operand
+ * quantized to dense_fmt (m+1 bits; NONE not allowed). Nothing but `energy`
+ * (all four fields) is written. sparse_scale_in / dense_scale_in: given
+ * per-tensor scales, or NULL to compute them in an extra read-only pass. */
+ss24_status ss24_error_energy(const ss24_operand *x, ss24_pattern pattern, ss24_score score,
+                              const float *col_norms, ss24_format sparse_fmt,
+                              ss24_format dense_fmt, const float *sparse_scale_in,
+                              const float *dense_scale_in, ss24_energy *energy, void *ws,
+                              size_t ws_bytes, ss24_stream stream);
+
+/* Largest |value| among the values a pass would quantize (§3 per-tensor
+ * scale): the kept values for a sparse pattern, all values for SS24_DENSE.
+ * Writes one fp32 to the device pointer amax_out. */
+ss24_status ss24_amax(const ss24_operand *x, ss24_pattern pattern, ss24_score score,
+                      const float *col_norms, float *amax_out, void *ws, size_t ws_bytes,
+                      ss24_stream stream);
+
+/* Derived quantities (§4) from a sparse-side energy record (e_total, e_prune,
+ * e_quant) and a dense-side record (e_quant_dense); both device pointers, and
+ * they may be the same record (as ss24_error_energy writes it). One-thread
+ * kernel; writes *out on the device. */
+ss24_status ss24_predicted_ratio(const ss24_energy *sparse_side, const ss24_energy *dense_side,
+                                 ss24_ratio *out, ss24_stream stream);
+
+/* ---- host-only helpers ------------------------------------------------------ */
+
+/* Stored bits per ORIGINAL element (§2: values, indices and, with with_scales,
+ * scales are all charged). Value bits: NONE 16, FP8 8, INT bits, NVFP4 /
+ * MXFP4 4; 2:4 adds 1 index bit per element, 4:8 adds 0.25. Scales: INT 32
+ * bits per group (per row of the quantized length when group is 0), NVFP4
+ * 8 per 16 values, MXFP4 8 per 32; the single NVFP4 / FP8 tensor scale is not
+ * charged. Returns a negative value for an invalid format. */
+double ss24_bits_per_element(ss24_format fmt, ss24_pattern pattern, int64_t k, int32_t with_scales);
+
+/* Static string naming a status. */
+const char *ss24_status_string(ss24_status status);
+
+/* ---- format conversion primitives (the kernels' own converters) ------------ */
+
+/* Encode n binary32 values to E4M3 (nearest-even, satfinite), one byte each. */
+ss24_status ss24_encode_e4m3(const float *in, uint8_t *out, int64_t n, ss24_stream stream);
+/* Decode n E4M3 bytes to binary32. */
+ss24_status ss24_decode_e4m3(const uint8_t *in, float *out, int64_t n, ss24_stream stream);
+/* Encode n binary32 values to E2M1 (nearest-even, satfinite), one code per
+ * byte in the low nibble. */
+ss24_status ss24_encode_e2m1(const float *in, uint8_t *out, int64_t n, ss24_stream stream);
+/* Decode n E2M1 codes (low nibble of each byte) to binary32. */
+ss24_status ss24_decode_e2m1(const uint8_t *in, float *out, int64_t n, ss24_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SS24_H */

@@ -63,6 +63,8 @@ def lib():
         _lib.oracle_run.argtypes = [ctypes.POINTER(_Args), ctypes.POINTER(_Outputs), ctypes.c_void_p]
         _lib.oracle_amax.restype = ctypes.c_float
         _lib.oracle_amax.argtypes = [ctypes.POINTER(_Args)]
+        _lib.oracle_tensor_scale.restype = ctypes.c_float
+        _lib.oracle_tensor_scale.argtypes = [ctypes.POINTER(_Args)]
         _lib.oracle_select24.restype = ctypes.c_int
         _lib.oracle_select24.argtypes = [ctypes.c_void_p]
         _lib.oracle_select48.restype = ctypes.c_int
@@ -161,6 +163,19 @@ def amax(x, *, pattern=SPARSE_24, score=MAG, norms=None, axis=1, rows=None, k=No
         norms = np.ascontiguousarray(norms, dtype=np.float32)
     args = _make_args(x, dtype, rows, k, ld, axis, pattern, score, norms, FMT_NONE, 8, 0, 0, None)
     return float(lib().oracle_amax(ctypes.byref(args)))
+
+
+def tensor_scale(x, fmt, *, pattern=SPARSE_24, score=MAG, norms=None, axis=1, rows=None, k=None, ld=None):
+    """The per-tensor scale (FP8: amax / 448, NVFP4: amax / 2688) a pass over the
+    whole operand derives when none is given."""
+    x = np.ascontiguousarray(x)
+    dtype = BF16 if x.dtype == np.uint16 else F32
+    rows, k, ld = _operand_shape(x, axis, rows, k, ld)
+    if norms is not None:
+        norms = np.ascontiguousarray(norms, dtype=np.float32)
+    fmt_id = _FMT_NAMES[fmt] if isinstance(fmt, str) else fmt
+    args = _make_args(x, dtype, rows, k, ld, axis, pattern, score, norms, fmt_id, 8, 0, 0, None)
+    return float(lib().oracle_tensor_scale(ctypes.byref(args)))
 
 
 def select24(s):

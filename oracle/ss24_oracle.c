@@ -646,3 +646,13 @@ double oracle_bits_per_element(int32_t fmt, int32_t bits, int32_t group, int32_t
     }
     return total;
 }
+
+/* The per-tensor scale a pass derives when none is given (§3): FP8
+ * s = amax / 448, NVFP4 s_t = amax / (6 * 448), over the values that get
+ * quantized. Lets a test check sampled rows of a large operand with the scale
+ * of the whole tensor. */
+float oracle_tensor_scale(const oracle_args *a)
+{
+    float amax = oracle_amax(a);
+    return a->fmt == OR_FMT_FP8 ? amax / 448.0f : amax / 2688.0f;
+}

@@ -1,0 +1,705 @@
+// The C ABI (include/ss24.h): host-side validation, tile geometry, TMA tensor
+// maps and launches. Every check runs before anything is enqueued; a failed
+// check returns its status and launches nothing.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <unordered_map>
+
+#include "../../include/ss24.h"
+#include "internal.cuh"
+
+namespace ss24 {
+const void *tile_kernel_bf16(int pattern, int score, int fmt);
+const void *tile_kernel_f32(int pattern, int score, int fmt);
+const void *row_kernel_bf16(int pattern, int score);
+const void *row_kernel_f32(int pattern, int score);
+} // namespace ss24
+
+using namespace ss24;
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// small helpers
+// ---------------------------------------------------------------------------
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
+int64_t next_pow2(int64_t v)
+{
+    int64_t p = 1;
+    while (p < v)
+        p <<= 1;
+    return p;
+}
+int ilog2(int64_t v)
+{
+    int l = 0;
+    while ((int64_t(1) << l) < v)
+        ++l;
+    return l;
+}
+size_t esize(int dtype) { return dtype == SS24_BF16 ? 2 : 4; }
+
+ss24_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SS24_OK : SS24_ERR_CUDA; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2-D map over the operand's memory: inner dimension = the contiguous one.
+bool make_map(CUtensorMap *map, const ss24_operand *x, int64_t inner, int64_t outer, uint32_t box_inner,
+              uint32_t box_outer)
+{
+    auto fn = encode_fn();
+    if (!fn)
+        return false;
+    const CUtensorMapDataType dt =
+        x->dtype == SS24_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    cuuint64_t gdim[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+    cuuint64_t gstride[1] = {static_cast<cuuint64_t>(x->ld) * esize(x->dtype)};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estride[2] = {1, 1};
+    const CUresult r = fn(map, dt, 2, const_cast<void *>(x->x), gdim, gstride, box, estride,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// Kernel attributes (dynamic shared memory) and occupancy, once per kernel.
+struct KernelInfo {
+    int blocks_per_sm = 0;
+};
+
+std::mutex g_mu;
+std::unordered_map<const void *, KernelInfo> g_info;
+int g_sms = 0;
+
+cudaError_t kernel_info(const void *k, size_t smem, KernelInfo *out)
+{
+    std::lock_guard<std::mutex> lock(g_mu);
+    auto it = g_info.find(k);
+    if (it != g_info.end()) {
+        *out = it->second;
+        return cudaSuccess;
+    }
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess)
+        return e;
+    KernelInfo info;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&info.blocks_per_sm, k, kThreads, smem);
+    if (e != cudaSuccess)
+        return e;
+    if (g_sms == 0) {
+        int dev = 0;
+        e = cudaGetDevice(&dev);
+        if (e == cudaSuccess)
+            e = cudaDeviceGetAttribute(&g_sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess)
+            return e;
+    }
+    g_info[k] = info;
+    *out = info;
+    return cudaSuccess;
+}
+
+cudaError_t launch(const void *k, size_t smem, int64_t n_tiles, const CUtensorMap &map, const PassParams &p,
+                   cudaStream_t stream)
+{
+    KernelInfo info;
+    cudaError_t e = kernel_info(k, smem, &info);
+    if (e != cudaSuccess)
+        return e;
+    int64_t grid = static_cast<int64_t>(g_sms) * (info.blocks_per_sm > 0 ? info.blocks_per_sm : 1);
+    if (grid > kMaxGrid)
+        grid = kMaxGrid;
+    if (grid > n_tiles)
+        grid = n_tiles;
+    CUtensorMap m = map;
+    PassParams pp = p;
+    void *args[2] = {&m, &pp};
+    e = cudaLaunchKernel(k, dim3(static_cast<unsigned>(grid)), dim3(kThreads), args, smem, stream);
+    return e;
+}
+
+// ---------------------------------------------------------------------------
+// validation
+// ---------------------------------------------------------------------------
+
+// An empty operand (rows == 0) may have a NULL data pointer.
+ss24_status check_operand(const ss24_operand *x)
+{
+    if (!x || (!x->x && x->rows != 0))
+        return SS24_ERR_NULL;
+    if (x->dtype != SS24_BF16 && x->dtype != SS24_F32)
+        return SS24_ERR_DTYPE;
+    if (x->axis != 1)
+        return SS24_ERR_ARG;
+    if (x->rows < 0 || x->k <= 0 || x->rows > INT32_MAX || x->k > INT32_MAX)
+        return SS24_ERR_SHAPE;
+    if (x->ld < x->k)
+        return SS24_ERR_SHAPE;
+    if (!aligned16(x->x) || (x->ld * static_cast<int64_t>(esize(x->dtype))) % 16 != 0)
+        return SS24_ERR_ALIGN;
+    return SS24_OK;
+}
+
+ss24_status check_ws(const void *ws, size_t ws_bytes)
+{
+    if (!ws || ws_bytes < kWsBytes || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+        return SS24_ERR_WORKSPACE;
+    return SS24_OK;
+}
+
+ss24_status check_pattern_k(int pattern, int64_t k)
+{
+    if (pattern != SS24_DENSE && pattern != SS24_SPARSE_24 && pattern != SS24_SPARSE_48)
+        return SS24_ERR_ARG;
+    if (k % (pattern == SS24_SPARSE_48 ? 16 : 8) != 0)
+        return SS24_ERR_SHAPE;
+    return SS24_OK;
+}
+
+// Resolved quantization of the values a pass stores (n per row).
+struct Resolved {
+    QuantSpec q;
+    bool row_mode = false;
+};
+
+// Validates `fmt` for rows of n quantized values (n = k/2 sparse, k dense) and
+// fills the kernel's QuantSpec (without the scale pointers).
+ss24_status resolve_format(ss24_format fmt, int pattern, int64_t k, bool allow_none, Resolved *r)
+{
+    const bool sparse = pattern != SS24_DENSE;
+    const int64_t n = sparse ? k / 2 : k;
+    const int vpc = sparse ? 4 : 8;
+    QuantSpec q{};
+    q.fmt = fmt.kind;
+    switch (fmt.kind) {
+    case SS24_FMT_NONE:
+        if (!allow_none || !sparse)
+            return SS24_ERR_FORMAT;
+        break;
+    case SS24_FMT_FP8_E4M3:
+        q.divisor = 448.0f;
+        break;
+    case SS24_FMT_NVFP4:
+        if (n % 16 != 0)
+            return SS24_ERR_SHAPE;
+        q.divisor = 2688.0f;
+        break;
+    case SS24_FMT_MXFP4:
+        if (n % 32 != 0)
+            return SS24_ERR_SHAPE;
+        break;
+    case SS24_FMT_INT: {
+        if (fmt.bits < 2 || fmt.bits > 16)
+            return SS24_ERR_FORMAT;
+        if (fmt.pack4 && fmt.bits > 4)
+            return SS24_ERR_FORMAT;
+        q.bits = fmt.bits;
+        q.qmax = static_cast<float>((1 << (fmt.bits - 1)) - 1);
+        q.store = fmt.pack4 ? kPack4 : (fmt.bits > 8 ? kInt16 : kInt8);
+        if (fmt.group < 0)
+            return SS24_ERR_FORMAT;
+        if (fmt.group == 0) {
+            q.group = static_cast<int32_t>(n);
+            // a whole row fits one warp's span only when k is a power of two <= 256
+            r->row_mode = !(pow2(k) && k <= 256);
+            q.lanes = r->row_mode ? 32 : static_cast<int32_t>(n / vpc);
+        } else {
+            const int64_t g_in = static_cast<int64_t>(fmt.group) * (sparse ? 2 : 1);
+            if (!pow2(fmt.group) || g_in < 8 || g_in > 256)
+                return SS24_ERR_FORMAT;
+            if (n % fmt.group != 0)
+                return SS24_ERR_SHAPE;
+            q.group = fmt.group;
+            q.lanes = fmt.group / vpc;
+        }
+        break;
+    }
+    default:
+        return SS24_ERR_FORMAT;
+    }
+    r->q = q;
+    return SS24_OK;
+}
+
+bool per_tensor(int kind) { return kind == SS24_FMT_FP8_E4M3 || kind == SS24_FMT_NVFP4; }
+
+// ---------------------------------------------------------------------------
+// geometry
+// ---------------------------------------------------------------------------
+
+struct Geometry {
+    int32_t R, W, log2_cpr, cpt;
+    int64_t n_tiles, n_col_tiles;
+    uint32_t tile_bytes;
+};
+
+Geometry tile_geometry(const ss24_operand *x)
+{
+    Geometry g{};
+    const int64_t es = static_cast<int64_t>(esize(x->dtype));
+    g.W = static_cast<int32_t>(x->k >= 256 ? 256 : next_pow2(x->k));
+    const int64_t stage_elems = kStageBytes / es;
+    int64_t R = stage_elems / g.W;
+    if (R > 256)
+        R = 256;
+    g.R = static_cast<int32_t>(R);
+    g.log2_cpr = ilog2(g.W / 8);
+    g.cpt = static_cast<int32_t>((R * g.W / 8) / kConsumers);
+    g.n_col_tiles = (x->k + g.W - 1) / g.W;
+    g.n_tiles = g.n_col_tiles * ((x->rows + R - 1) / R);
+    g.tile_bytes = static_cast<uint32_t>(R * g.W * es);
+    return g;
+}
+
+// Row mode: whole rows, boxes of W = min(256, next_pow2(k)) columns.
+bool row_geometry(const ss24_operand *x, Geometry *g)
+{
+    const int64_t es = static_cast<int64_t>(esize(x->dtype));
+    g->W = static_cast<int32_t>(x->k >= 256 ? 256 : next_pow2(x->k));
+    const int64_t nbox = (x->k + g->W - 1) / g->W;
+    const int64_t row_bytes = nbox * g->W * es;
+    int64_t R = kRowStageBytes / row_bytes;
+    if (R < 1)
+        return false;
+    if (R > 256)
+        R = 256;
+    g->R = static_cast<int32_t>(R);
+    g->log2_cpr = ilog2(g->W / 8);
+    g->cpt = 0;
+    g->n_col_tiles = 1;
+    g->n_tiles = (x->rows + R - 1) / R;
+    g->tile_bytes = static_cast<uint32_t>(R * row_bytes);
+    return true;
+}
+
+PassParams base_params(const ss24_operand *x, const Geometry &g, void *ws, ss24_energy *energy)
+{
+    PassParams p{};
+    p.rows = x->rows;
+    p.k = x->k;
+    p.n_tiles = g.n_tiles;
+    p.n_col_tiles = g.n_col_tiles;
+    p.R = g.R;
+    p.W = g.W;
+    p.log2_cpr = g.log2_cpr;
+    p.cpt = g.cpt;
+    p.tile_bytes = g.tile_bytes;
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    p.err = reinterpret_cast<int32_t *>(w + kWsErrOff);
+    p.energy_ticket = reinterpret_cast<uint32_t *>(w + kWsEnergyTicketOff);
+    p.amax_ticket = reinterpret_cast<uint32_t *>(w + kWsAmaxTicketOff);
+    p.energy_partials = reinterpret_cast<double *>(w + kWsEnergyOff);
+    p.amax_partials = reinterpret_cast<float *>(w + kWsAmaxOff);
+    p.amax_out = reinterpret_cast<float *>(w + kWsAmaxReducedOff);
+    p.energy_out = reinterpret_cast<double *>(energy);
+    return p;
+}
+
+const void *tile_kernel(int dtype, int pattern, int score, int fmt)
+{
+    return dtype == SS24_BF16 ? tile_kernel_bf16(pattern, score, fmt) : tile_kernel_f32(pattern, score, fmt);
+}
+
+// The read-only amax pass; leaves {amax of kept, amax of all} in the workspace.
+// For the magnitude score the kept amax equals the amax of all values, so the
+// cheaper dense form is used.
+cudaError_t run_amax(const ss24_operand *x, int pattern, int score, const float *norms, void *ws,
+                     cudaStream_t stream)
+{
+    const int pat = score == SS24_SCORE_MAG ? SS24_DENSE : pattern;
+    const Geometry g = tile_geometry(x);
+    CUtensorMap map;
+    if (!make_map(&map, x, x->k, x->rows, static_cast<uint32_t>(g.W), static_cast<uint32_t>(g.R)))
+        return cudaErrorInvalidValue;
+    PassParams p = base_params(x, g, ws, nullptr);
+    p.norms = norms;
+    return launch(tile_kernel(x->dtype, pat, score, kAmax), kSmemBytes, g.n_tiles, map, p, stream);
+}
+
+// Zero energy record / scale for an empty operand (nothing to launch).
+ss24_status empty_operand(ss24_energy *energy, const ss24_outputs *out, const float *scale_in,
+                          cudaStream_t stream)
+{
+    cudaError_t e = cudaSuccess;
+    if (energy)
+        e = cudaMemsetAsync(energy, 0, sizeof(ss24_energy), stream);
+    if (e == cudaSuccess && out && out->tensor_scale) {
+        if (scale_in)
+            e = cudaMemcpyAsync(out->tensor_scale, scale_in, sizeof(float), cudaMemcpyDeviceToDevice, stream);
+        else
+            e = cudaMemsetAsync(out->tensor_scale, 0, sizeof(float), stream);
+    }
+    return cuda_status(e);
+}
+
+// The storing pass shared by the quantize / prune entry points.
+ss24_status run_pass(const ss24_operand *x, int pattern, int score, const float *norms, ss24_format fmt,
+                     bool allow_none, const float *scale_in, const ss24_outputs *out, ss24_energy *energy,
+                     void *ws, size_t ws_bytes, cudaStream_t stream)
+{
+    ss24_status st = check_operand(x);
+    if (st != SS24_OK)
+        return st;
+    if ((st = check_pattern_k(pattern, x->k)) != SS24_OK)
+        return st;
+    if (score != SS24_SCORE_MAG && score != SS24_SCORE_WANDA)
+        return SS24_ERR_ARG;
+    if (score == SS24_SCORE_WANDA && pattern != SS24_DENSE && (!norms || !aligned16(norms)))
+        return norms ? SS24_ERR_ALIGN : SS24_ERR_NULL;
+    if ((st = check_ws(ws, ws_bytes)) != SS24_OK)
+        return st;
+    Resolved r;
+    if ((st = resolve_format(fmt, pattern, x->k, allow_none, &r)) != SS24_OK)
+        return st;
+    if (!out)
+        return SS24_ERR_NULL;
+    Geometry g;
+    if (r.row_mode) {
+        if (!row_geometry(x, &g))
+            return SS24_ERR_SHAPE;
+    } else {
+        g = tile_geometry(x);
+    }
+    if (x->rows == 0)
+        return empty_operand(energy, out, per_tensor(fmt.kind) ? scale_in : nullptr, stream);
+    if (!out->values)
+        return SS24_ERR_NULL;
+    if (!aligned16(out->values))
+        return SS24_ERR_ALIGN;
+    const bool needs_scales = fmt.kind == SS24_FMT_INT || fmt.kind == SS24_FMT_NVFP4 || fmt.kind == SS24_FMT_MXFP4;
+    if (needs_scales && !out->scales)
+        return SS24_ERR_NULL;
+    if (needs_scales && !aligned16(out->scales))
+        return SS24_ERR_ALIGN;
+    if (per_tensor(fmt.kind) && !out->tensor_scale)
+        return SS24_ERR_NULL;
+    if (pattern != SS24_DENSE && (!out->meta))
+        return SS24_ERR_NULL;
+    if (pattern != SS24_DENSE && !aligned16(out->meta))
+        return SS24_ERR_ALIGN;
+
+    // ---- launches ----
+    PassParams p = base_params(x, g, ws, energy);
+    p.values = out->values;
+    p.scales = out->scales;
+    p.meta = out->meta;
+    p.norms = norms;
+    p.q = r.q;
+    if (per_tensor(fmt.kind)) {
+        p.q.scale_out = out->tensor_scale;
+        p.q.scale_in = scale_in;
+        if (!scale_in) {
+            cudaError_t e = run_amax(x, pattern, score, norms, ws, stream);
+            if (e != cudaSuccess)
+                return SS24_ERR_CUDA;
+            p.q.amax_reduced = p.amax_out; // [0] = amax of the quantized values
+        }
+    }
+    CUtensorMap map;
+    cudaError_t e;
+    if (r.row_mode) {
+        if (!make_map(&map, x, x->k, x->rows, static_cast<uint32_t>(g.W), static_cast<uint32_t>(g.R)))
+            return SS24_ERR_CUDA;
+        const void *k = x->dtype == SS24_BF16 ? row_kernel_bf16(pattern, score) : row_kernel_f32(pattern, score);
+        e = launch(k, kRowSmemBytes, g.n_tiles, map, p, stream);
+    } else {
+        if (!make_map(&map, x, x->k, x->rows, static_cast<uint32_t>(g.W), static_cast<uint32_t>(g.R)))
+            return SS24_ERR_CUDA;
+        e = launch(tile_kernel(x->dtype, pattern, score, fmt.kind), kSmemBytes, g.n_tiles, map, p, stream);
+    }
+    return cuda_status(e);
+}
+
+} // namespace
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+
+extern "C" {
+
+size_t ss24_workspace_bytes(void) { return kWsBytes; }
+
+ss24_status ss24_workspace_init(void *ws, size_t ws_bytes, ss24_stream stream)
+{
+    ss24_status st = check_ws(ws, ws_bytes);
+    if (st != SS24_OK)
+        return st;
+    return cuda_status(cudaMemsetAsync(ws, 0, 256, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ss24_status ss24_workspace_error(const void *ws, int32_t *code, ss24_stream stream)
+{
+    if (!ws || !code)
+        return SS24_ERR_NULL;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess)
+        e = cudaMemcpy(code, ws, sizeof(int32_t), cudaMemcpyDeviceToHost);
+    return cuda_status(e);
+}
+
+ss24_status ss24_prune24_compress(const ss24_operand *x, ss24_score score, const float *col_norms, void *kept,
+                                  uint8_t *meta, ss24_energy *energy, void *ws, size_t ws_bytes,
+                                  ss24_stream stream)
+{
+    ss24_outputs out{kept, nullptr, nullptr, meta};
+    ss24_format none{SS24_FMT_NONE, 0, 0, 0};
+    return run_pass(x, SS24_SPARSE_24, score, col_norms, none, true, nullptr, &out, energy, ws, ws_bytes,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+ss24_status ss24_quantize_fp8(const ss24_operand *x, const float *tensor_scale_in, ss24_outputs *out,
+                              ss24_energy *energy, void *ws, size_t ws_bytes, ss24_stream stream)
+{
+    ss24_format f{SS24_FMT_FP8_E4M3, 8, 0, 0};
+    return run_pass(x, SS24_DENSE, SS24_SCORE_MAG, nullptr, f, false, tensor_scale_in, out, energy, ws, ws_bytes,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+ss24_status ss24_quantize_int(const ss24_operand *x, ss24_format fmt, ss24_outputs *out, ss24_energy *energy,
+                              void *ws, size_t ws_bytes, ss24_stream stream)
+{
+    if (fmt.kind != SS24_FMT_INT)
+        return SS24_ERR_FORMAT;
+    return run_pass(x, SS24_DENSE, SS24_SCORE_MAG, nullptr, fmt, false, nullptr, out, energy, ws, ws_bytes,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+ss24_status ss24_quantize_nvfp4(const ss24_operand *x, const float *tensor_scale_in, ss24_outputs *out,
+                                ss24_energy *energy, void *ws, size_t ws_bytes, ss24_stream stream)
+{
+    ss24_format f{SS24_FMT_NVFP4, 4, 0, 0};
+    return run_pass(x, SS24_DENSE, SS24_SCORE_MAG, nullptr, f, false, tensor_scale_in, out, energy, ws, ws_bytes,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+ss24_status ss24_quantize_mxfp4(const ss24_operand *x, ss24_outputs *out, ss24_energy *energy, void *ws,
+                                size_t ws_bytes, ss24_stream stream)
+{
+    ss24_format f{SS24_FMT_MXFP4, 4, 0, 0};
+    return run_pass(x, SS24_DENSE, SS24_SCORE_MAG, nullptr, f, false, nullptr, out, energy, ws, ws_bytes,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+ss24_status ss24_prune24_quant_fused(const ss24_operand *x, ss24_score score, const float *col_norms,
+                                     ss24_format fmt, const float *tensor_scale_in, ss24_outputs *out,
+                                     ss24_energy *energy, void *ws, size_t ws_bytes, ss24_stream stream)
+{
+    return run_pass(x, SS24_SPARSE_24, score, col_norms, fmt, true, tensor_scale_in, out, energy, ws, ws_bytes,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+ss24_status ss24_prune48_pairwise_quant_fused(const ss24_operand *x, ss24_score score, const float *col_norms,
+                                              ss24_format fmt, const float *tensor_scale_in, ss24_outputs *out,
+                                              ss24_energy *energy, void *ws, size_t ws_bytes, ss24_stream stream)
+{
+    return run_pass(x, SS24_SPARSE_48, score, col_norms, fmt, true, tensor_scale_in, out, energy, ws, ws_bytes,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+ss24_status ss24_error_energy(const ss24_operand *x, ss24_pattern pattern, ss24_score score, const float *col_norms,
+                              ss24_format sparse_fmt, ss24_format dense_fmt, const float *sparse_scale_in,
+                              const float *dense_scale_in, ss24_energy *energy, void *ws, size_t ws_bytes,
+                              ss24_stream stream)
+{
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    ss24_status st = check_operand(x);
+    if (st != SS24_OK)
+        return st;
+    if (pattern == SS24_DENSE)
+        return SS24_ERR_ARG;
+    if ((st = check_pattern_k(pattern, x->k)) != SS24_OK)
+        return st;
+    if (score != SS24_SCORE_MAG && score != SS24_SCORE_WANDA)
+        return SS24_ERR_ARG;
+    if (score == SS24_SCORE_WANDA && (!col_norms || !aligned16(col_norms)))
+        return col_norms ? SS24_ERR_ALIGN : SS24_ERR_NULL;
+    if ((st = check_ws(ws, ws_bytes)) != SS24_OK)
+        return st;
+    if (!energy)
+        return SS24_ERR_NULL;
+    Resolved rs, rd;
+    if ((st = resolve_format(sparse_fmt, pattern, x->k, true, &rs)) != SS24_OK)
+        return st;
+    if ((st = resolve_format(dense_fmt, SS24_DENSE, x->k, false, &rd)) != SS24_OK)
+        return st;
+    if (rs.row_mode || rd.row_mode)
+        return SS24_ERR_FORMAT; // one scale per long row needs the storing row-mode pass
+    if (x->rows == 0)
+        return empty_operand(energy, nullptr, nullptr, s);
+    const Geometry g = tile_geometry(x);
+    PassParams p = base_params(x, g, ws, energy);
+    p.norms = col_norms;
+    p.q = rs.q;
+    p.qd = rd.q;
+    const bool need_s = per_tensor(sparse_fmt.kind) && !sparse_scale_in;
+    const bool need_d = per_tensor(dense_fmt.kind) && !dense_scale_in;
+    if (need_s || need_d) {
+        if (run_amax(x, pattern, score, col_norms, ws, s) != cudaSuccess)
+            return SS24_ERR_CUDA;
+    }
+    p.q.scale_in = sparse_scale_in;
+    p.q.amax_reduced = p.amax_out;     // [0]: amax of the kept values
+    p.qd.scale_in = dense_scale_in;
+    p.qd.amax_reduced = p.amax_out + 1; // [1]: amax of all values
+    CUtensorMap map;
+    if (!make_map(&map, x, x->k, x->rows, static_cast<uint32_t>(g.W), static_cast<uint32_t>(g.R)))
+        return SS24_ERR_CUDA;
+    return cuda_status(launch(tile_kernel(x->dtype, pattern, score, kEnergy), kSmemBytes, g.n_tiles, map, p, s));
+}
+
+ss24_status ss24_amax(const ss24_operand *x, ss24_pattern pattern, ss24_score score, const float *col_norms,
+                      float *amax_out, void *ws, size_t ws_bytes, ss24_stream stream)
+{
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    ss24_status st = check_operand(x);
+    if (st != SS24_OK)
+        return st;
+    if ((st = check_pattern_k(pattern, x->k)) != SS24_OK)
+        return st;
+    if (score != SS24_SCORE_MAG && score != SS24_SCORE_WANDA)
+        return SS24_ERR_ARG;
+    if (score == SS24_SCORE_WANDA && pattern != SS24_DENSE && (!col_norms || !aligned16(col_norms)))
+        return col_norms ? SS24_ERR_ALIGN : SS24_ERR_NULL;
+    if ((st = check_ws(ws, ws_bytes)) != SS24_OK)
+        return st;
+    if (!amax_out)
+        return SS24_ERR_NULL;
+    if (x->rows == 0)
+        return cuda_status(cudaMemsetAsync(amax_out, 0, sizeof(float), s));
+    if (run_amax(x, pattern, score, col_norms, ws, s) != cudaSuccess)
+        return SS24_ERR_CUDA;
+    const float *red = reinterpret_cast<const float *>(static_cast<uint8_t *>(ws) + kWsAmaxReducedOff);
+    return cuda_status(cudaMemcpyAsync(amax_out, red, sizeof(float), cudaMemcpyDeviceToDevice, s));
+}
+
+ss24_status ss24_predicted_ratio(const ss24_energy *sparse_side, const ss24_energy *dense_side, ss24_ratio *out,
+                                 ss24_stream stream)
+{
+    if (!sparse_side || !dense_side || !out)
+        return SS24_ERR_NULL;
+    return cuda_status(launch_ratio(reinterpret_cast<const double *>(sparse_side),
+                                    reinterpret_cast<const double *>(dense_side), reinterpret_cast<double *>(out),
+                                    reinterpret_cast<cudaStream_t>(stream)));
+}
+
+double ss24_bits_per_element(ss24_format fmt, ss24_pattern pattern, int64_t k, int32_t with_scales)
+{
+    if (pattern != SS24_DENSE && pattern != SS24_SPARSE_24 && pattern != SS24_SPARSE_48)
+        return -1.0;
+    double vb;
+    switch (fmt.kind) {
+    case SS24_FMT_NONE:
+        vb = 16.0;
+        break;
+    case SS24_FMT_FP8_E4M3:
+        vb = 8.0;
+        break;
+    case SS24_FMT_INT:
+        if (fmt.bits < 2 || fmt.bits > 16)
+            return -1.0;
+        vb = fmt.bits;
+        break;
+    case SS24_FMT_NVFP4:
+    case SS24_FMT_MXFP4:
+        vb = 4.0;
+        break;
+    default:
+        return -1.0;
+    }
+    const double kept = pattern == SS24_DENSE ? 1.0 : 0.5;
+    const double index = pattern == SS24_SPARSE_24 ? 1.0 : (pattern == SS24_SPARSE_48 ? 0.25 : 0.0);
+    double bits = kept * vb + index;
+    if (with_scales) {
+        double per_value = 0.0;
+        if (fmt.kind == SS24_FMT_INT)
+            per_value = 32.0 / (fmt.group > 0 ? static_cast<double>(fmt.group) : kept * static_cast<double>(k));
+        else if (fmt.kind == SS24_FMT_NVFP4)
+            per_value = 8.0 / 16.0;
+        else if (fmt.kind == SS24_FMT_MXFP4)
+            per_value = 8.0 / 32.0;
+        bits += kept * per_value;
+    }
+    return bits;
+}
+
+const char *ss24_status_string(ss24_status status)
+{
+    switch (status) {
+    case SS24_OK:
+        return "ok";
+    case SS24_ERR_NULL:
+        return "a required pointer is NULL";
+    case SS24_ERR_SHAPE:
+        return "shape does not fit the pattern or format";
+    case SS24_ERR_ALIGN:
+        return "pointer or row stride not 16-byte aligned";
+    case SS24_ERR_DTYPE:
+        return "unknown element type";
+    case SS24_ERR_FORMAT:
+        return "unsupported quantization format";
+    case SS24_ERR_WORKSPACE:
+        return "workspace missing, too small or misaligned";
+    case SS24_ERR_CUDA:
+        return "CUDA call or launch failed";
+    case SS24_ERR_ARG:
+        return "unknown score, axis or pattern";
+    }
+    return "unknown status";
+}
+
+ss24_status ss24_encode_e4m3(const float *in, uint8_t *out, int64_t n, ss24_stream stream)
+{
+    if ((!in || !out) && n > 0)
+        return SS24_ERR_NULL;
+    if (n < 0)
+        return SS24_ERR_SHAPE;
+    return cuda_status(launch_convert(0, in, out, n, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ss24_status ss24_decode_e4m3(const uint8_t *in, float *out, int64_t n, ss24_stream stream)
+{
+    if ((!in || !out) && n > 0)
+        return SS24_ERR_NULL;
+    if (n < 0)
+        return SS24_ERR_SHAPE;
+    return cuda_status(launch_convert(1, in, out, n, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ss24_status ss24_encode_e2m1(const float *in, uint8_t *out, int64_t n, ss24_stream stream)
+{
+    if ((!in || !out) && n > 0)
+        return SS24_ERR_NULL;
+    if (n < 0)
+        return SS24_ERR_SHAPE;
+    return cuda_status(launch_convert(2, in, out, n, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ss24_status ss24_decode_e2m1(const uint8_t *in, float *out, int64_t n, ss24_stream stream)
+{
+    if ((!in || !out) && n > 0)
+        return SS24_ERR_NULL;
+    if (n < 0)
+        return SS24_ERR_SHAPE;
+    return cuda_status(launch_convert(3, in, out, n, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+} // extern "C"

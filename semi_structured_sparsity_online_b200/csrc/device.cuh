@@ -1,0 +1,232 @@
+// Device building blocks of the ss24 kernels (sm_100a): PTX wrappers for
+// mbarriers and TMA tile loads, bounded waits, the FP8 / FP4 converters, and
+// the 2:4 / 4:8 selection tournaments.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cstdint>
+
+namespace ss24 {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+// ---------------------------------------------------------------------------
+// shared-memory barriers and TMA (PTX ISA: mbarrier, cp.async.bulk.tensor)
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+// Makes barrier initialisation visible to the async (TMA) proxy.
+__device__ __forceinline__ void fence_barrier_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n"
+        " .reg .pred p;\n"
+        " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n"
+        "}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// A wait gives up after this long; the kernel then records an error code and
+// returns instead of spinning forever.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// Waits until the barrier phase with the given parity has completed.
+// Returns false (without having waited forever) if that takes over ~2 s.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+        for (int i = 0; i < 32; ++i)
+            if (mbar_try_wait(bar, parity))
+                return true;
+        if (global_timer_ns() - t0 > kWaitLimitNs)
+            return false;
+    }
+}
+
+// 2-D tiled TMA load of one box into shared memory, completing on `bar`.
+// Coordinates are {inner (contiguous) element index, outer index}.
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int32_t c_inner,
+                                            int32_t c_outer, uint64_t *bar, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c_inner), "r"(c_outer), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+
+// L2 policy for data read exactly once: evict it first.
+__device__ __forceinline__ uint64_t l2_evict_first_policy()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ void named_barrier_sync(int id, int threads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// number formats (PTX cvt forms for e4m3x2 / e2m1x2; rounding is the
+// instruction's own .rn with .satfinite)
+// ---------------------------------------------------------------------------
+
+// Two binary32 -> two E4M3 bytes; `lo` lands in bits 0..7, `hi` in 8..15.
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi)
+{
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Two E4M3 bytes (bits 0..7 and 8..15) -> two binary32 (exact).
+__device__ __forceinline__ float2 e4m3x2_to_f32(uint32_t two_bytes)
+{
+    uint32_t h2;
+    const uint16_t b = static_cast<uint16_t>(two_bytes);
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(b));
+    __half2 h = *reinterpret_cast<__half2 *>(&h2);
+    return __half22float2(h); // .x from the low byte
+}
+
+__device__ __forceinline__ float e4m3_to_f32(uint32_t byte)
+{
+    return e4m3x2_to_f32(byte & 0xffu).x;
+}
+
+// Four binary32 -> four E2M1 nibbles (v0 in bits 0..3, ..., v3 in 12..15).
+__device__ __forceinline__ uint32_t cvt_e2m1x4(float v0, float v1, float v2, float v3)
+{
+    uint16_t r;
+    asm("{\n"
+        " .reg .b8 b0, b1;\n"
+        " cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n"
+        " cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n"
+        " mov.b16 %0, {b0, b1};\n"
+        "}\n"
+        : "=h"(r)
+        : "f"(v0), "f"(v1), "f"(v2), "f"(v3));
+    return r;
+}
+
+// Two E2M1 nibbles (bits 0..3 and 4..7 of `byte`) -> two binary32 (exact).
+__device__ __forceinline__ float2 e2m1x2_to_f32(uint32_t byte)
+{
+    uint32_t h2;
+    asm("{\n"
+        " .reg .b8 b0, b1, b2, b3;\n"
+        " mov.b32 {b0, b1, b2, b3}, %1;\n"
+        " cvt.rn.f16x2.e2m1x2 %0, b0;\n"
+        "}\n"
+        : "=r"(h2)
+        : "r"(byte));
+    __half2 h = *reinterpret_cast<__half2 *>(&h2);
+    return __half22float2(h); // .x from the low nibble
+}
+
+// MXFP4 shared exponent of a block with amax > 0: floor(log2(amax)) - 2,
+// read from the bits of amax (subnormals included), clamped to [-127, 127].
+__device__ __forceinline__ int mx_shared_exponent(float amax)
+{
+    const uint32_t b = __float_as_uint(amax);
+    const int ebits = static_cast<int>(b >> 23);
+    const int fl = ebits ? ebits - 127 : (31 - __clz(static_cast<int>(b))) - 149;
+    return max(-127, min(127, fl - 2));
+}
+
+// 2^e as a binary32 for e in [-127, 127] (2^-127 is subnormal).
+__device__ __forceinline__ float exp2_int(int e)
+{
+    return e >= -126 ? __uint_as_float(static_cast<uint32_t>(e + 127) << 23) : __uint_as_float(0x00400000u);
+}
+
+// ---------------------------------------------------------------------------
+// selection
+// ---------------------------------------------------------------------------
+
+// Top-2 of four by score with ties to the lower index, as a small tournament:
+// the winners of (0,1) and (2,3) meet for first place; second place is the
+// better of the first-place pair's loser and the other pair's winner. A later
+// index wins a comparison only when its score is strictly larger.
+struct Pick {
+    bool p;     // winner of (0,1) is 1
+    bool q;     // winner of (2,3) is 3
+    bool both01; // both kept elements are 0 and 1
+    bool both23; // both kept elements are 2 and 3
+    uint32_t nib;
+};
+
+__device__ __forceinline__ Pick top2_of_4(float s0, float s1, float s2, float s3)
+{
+    Pick k;
+    k.p = s1 > s0;
+    k.q = s3 > s2;
+    const float w01 = k.p ? s1 : s0, l01 = k.p ? s0 : s1;
+    const float w23 = k.q ? s3 : s2, l23 = k.q ? s2 : s3;
+    const bool r = w23 > w01;   // first place comes from pair (2,3)
+    const bool ta = w23 > l01;  // if first is from (0,1): second is (2,3)'s winner
+    const bool tb = l23 > w01;  // if first is from (2,3): second is its loser
+    k.both01 = !r && !ta;
+    k.both23 = r && tb;
+    const uint32_t mixed = static_cast<uint32_t>(k.p) | ((2u + static_cast<uint32_t>(k.q)) << 2);
+    k.nib = k.both01 ? 0x4u : (k.both23 ? 0xEu : mixed);
+    return k;
+}
+
+// Kept and dropped values of one 2:4 group, in index order.
+__device__ __forceinline__ void apply24(const Pick &k, float a, float b, float c, float d, float &k0,
+                                        float &k1, float &d0, float &d1)
+{
+    const float w01 = k.p ? b : a, l01 = k.p ? a : b;
+    const float w23 = k.q ? d : c, l23 = k.q ? c : d;
+    k0 = k.both01 ? a : (k.both23 ? c : w01);
+    k1 = k.both01 ? b : (k.both23 ? d : w23);
+    d0 = k.both01 ? c : (k.both23 ? a : l01);
+    d1 = k.both01 ? d : (k.both23 ? b : l23);
+}
+
+} // namespace ss24

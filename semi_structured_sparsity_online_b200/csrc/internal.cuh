@@ -1,0 +1,85 @@
+// Internal interface between the C ABI layer (abi.cu) and the kernels
+// (pass_impl.cuh, instantiated in pass_bf16.cu / pass_f32.cu; misc.cu).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace ss24 {
+
+enum Pattern { kDense = 0, kSparse24 = 24, kSparse48 = 48 };
+enum Score { kMag = 0, kWanda = 1 };
+// Formats of the pass; kAmax is the read-only amax pass; kEnergy the
+// read-only two-format energy pass.
+enum Fmt { kNone = 0, kFp8 = 1, kInt = 2, kNvfp4 = 3, kMxfp4 = 4, kAmax = 5, kEnergy = 6 };
+enum IntStore { kInt8 = 0, kInt16 = 1, kPack4 = 2 };
+
+// Consumer warps per CTA and the TMA stage ring (each stage 16 KiB).
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumers = kConsumerWarps * 32;
+constexpr int kThreads = kConsumers + 32; // + one producer warp
+constexpr int kStageBytes = 16384;
+constexpr int kStages = 4;
+constexpr int kMaxGrid = 1024;            // bound on CTAs (workspace partials)
+constexpr size_t kSmemBytes = kStages * kStageBytes + 1024;
+
+// Row-mode (one scale per row, long rows): a stage holds whole rows.
+constexpr int kRowStageBytes = 49152;
+constexpr int kRowStages = 3;
+constexpr size_t kRowSmemBytes = kRowStages * kRowStageBytes + 2048;
+
+// Workspace layout (bytes): [0, 256) header: error word at 0, the energy
+// ticket counter at 4, the amax ticket counter at 8 (each left at zero by the
+// CTA that finishes last); [256, 256 + 32 * kMaxGrid) energy partials (4
+// doubles per CTA); then amax partials (2 floats per CTA); then the 2 reduced
+// amax floats (kept values, all values).
+constexpr size_t kWsErrOff = 0;
+constexpr size_t kWsEnergyTicketOff = 4;
+constexpr size_t kWsAmaxTicketOff = 8;
+constexpr size_t kWsEnergyOff = 256;
+constexpr size_t kWsAmaxOff = kWsEnergyOff + 32 * kMaxGrid;
+constexpr size_t kWsAmaxReducedOff = kWsAmaxOff + 8 * kMaxGrid;
+constexpr size_t kWsBytes = kWsAmaxReducedOff + 256;
+
+struct QuantSpec {
+    int32_t fmt;       // Fmt (kNone .. kMxfp4)
+    int32_t bits;      // INT
+    int32_t group;     // INT: quantized values per scale (already resolved, > 0)
+    int32_t lanes;     // lanes (chunks) per scale group
+    int32_t store;     // IntStore
+    float qmax;        // INT
+    float divisor;     // FP8: 448, NVFP4: 2688 (tensor scale = amax / divisor)
+    const float *scale_in;     // given tensor scale (device) or nullptr
+    const float *amax_reduced; // device float holding the amax when the scale is computed
+    float *scale_out;          // where to write the tensor scale used (device) or nullptr
+};
+
+struct PassParams {
+    int64_t rows, k;           // logical operand A[rows][k]
+    int64_t n_tiles, n_col_tiles;
+    int32_t R, W;              // tile rows and width (elements)
+    int32_t log2_cpr;          // log2(chunks of 8 per tile row)
+    int32_t cpt;               // chunks per consumer thread per tile
+    uint32_t tile_bytes;
+    // outputs
+    void *values;
+    void *scales;
+    uint8_t *meta;
+    const float *norms;        // Wanda column norms
+    QuantSpec q;               // the stored format (or the sparse side of kEnergy)
+    QuantSpec qd;              // kEnergy: the dense side
+    double *energy_partials;   // [grid][4] (workspace)
+    double *energy_out;        // caller's ss24_energy (4 doubles) or nullptr: no energies
+    float *amax_partials;      // kAmax: [grid][2] (workspace)
+    float *amax_out;           // kAmax: 2 floats (kept values, all values)
+    uint32_t *energy_ticket;   // last-CTA-done counters (workspace)
+    uint32_t *amax_ticket;
+    int32_t *err;              // workspace error word
+};
+
+cudaError_t launch_ratio(const double *sparse_side, const double *dense_side, double *out,
+                         cudaStream_t stream);
+cudaError_t launch_convert(int op, const void *in, void *out, int64_t n, cudaStream_t stream);
+
+} // namespace ss24

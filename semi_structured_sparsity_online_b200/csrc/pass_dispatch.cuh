@@ -1,0 +1,60 @@
+// Kernel tables for one element type: maps (pattern, score, format) to the
+// instantiated tile-mode or row-mode kernel.
+#pragma once
+
+#include "pass_impl.cuh"
+
+namespace ss24 {
+
+template <typename T, int PAT, int SC> const void *tile_kernel_for_fmt(int fmt)
+{
+    switch (fmt) {
+    case kNone:
+        if constexpr (PAT != kDense)
+            return reinterpret_cast<const void *>(&pass_kernel<T, PAT, SC, kNone>);
+        break;
+    case kFp8:
+        return reinterpret_cast<const void *>(&pass_kernel<T, PAT, SC, kFp8>);
+    case kInt:
+        return reinterpret_cast<const void *>(&pass_kernel<T, PAT, SC, kInt>);
+    case kNvfp4:
+        return reinterpret_cast<const void *>(&pass_kernel<T, PAT, SC, kNvfp4>);
+    case kMxfp4:
+        return reinterpret_cast<const void *>(&pass_kernel<T, PAT, SC, kMxfp4>);
+    case kAmax:
+        return reinterpret_cast<const void *>(&pass_kernel<T, PAT, SC, kAmax>);
+    case kEnergy:
+        if constexpr (PAT != kDense)
+            return reinterpret_cast<const void *>(&pass_kernel<T, PAT, SC, kEnergy>);
+        break;
+    }
+    return nullptr;
+}
+
+template <typename T> const void *tile_kernel(int pattern, int score, int fmt)
+{
+    if (pattern == kDense)
+        return tile_kernel_for_fmt<T, kDense, kMag>(fmt);
+    if (pattern == kSparse24)
+        return score == kWanda ? tile_kernel_for_fmt<T, kSparse24, kWanda>(fmt)
+                               : tile_kernel_for_fmt<T, kSparse24, kMag>(fmt);
+    if (pattern == kSparse48)
+        return score == kWanda ? tile_kernel_for_fmt<T, kSparse48, kWanda>(fmt)
+                               : tile_kernel_for_fmt<T, kSparse48, kMag>(fmt);
+    return nullptr;
+}
+
+template <typename T> const void *row_kernel_ptr(int pattern, int score)
+{
+    if (pattern == kDense)
+        return reinterpret_cast<const void *>(&row_kernel<T, kDense, kMag>);
+    if (pattern == kSparse24)
+        return score == kWanda ? reinterpret_cast<const void *>(&row_kernel<T, kSparse24, kWanda>)
+                               : reinterpret_cast<const void *>(&row_kernel<T, kSparse24, kMag>);
+    if (pattern == kSparse48)
+        return score == kWanda ? reinterpret_cast<const void *>(&row_kernel<T, kSparse48, kWanda>)
+                               : reinterpret_cast<const void *>(&row_kernel<T, kSparse48, kMag>);
+    return nullptr;
+}
+
+} // namespace ss24

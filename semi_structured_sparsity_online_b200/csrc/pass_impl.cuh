@@ -1,0 +1,815 @@
+// The online pass (tile mode): one read of the operand, selection, quantization,
+// stores and error energies, in a persistent warp-specialised kernel.
+//
+// Method: "Is 2:4 Sparsity Still Worth It? Semi-Structured Sparsity versus
+// Quantization in LLM Inference" — intro (2:4 along the reduction axis), §2
+// (scores, round-to-nearest), §3 (formats; a fused kernel that reads the input
+// once and writes kept values and indices once), §4 (disjoint error energies),
+// §6 (pairwise 4:8).
+//
+// Structure. Each CTA owns tiles t = blockIdx.x, blockIdx.x + gridDim.x, ...
+// A tile is a TMA box of R rows x W columns of the operand (W a power of two
+// <= 256 along k, out-of-range parts zero-filled). One producer lane streams
+// tiles into a ring of kStages shared-memory stages (mbarrier full/empty
+// pairs); 8 consumer warps each read 16-byte chunks of 8 consecutive elements
+// from the stage, release it, then select / quantize / store from registers.
+// A warp's 32 lanes hold 32 consecutive chunks of one tile row segment, so a
+// quantization group (at most 256 input elements) is a power-of-two run of
+// lanes reduced with xor shuffles. Energies are summed per chunk in binary32
+// trees, accumulated per thread in binary64, reduced per CTA, and the last CTA
+// to finish (a ticket counter) reduces the per-CTA partials in fixed order.
+#pragma once
+
+#include "device.cuh"
+#include "internal.cuh"
+
+namespace ss24 {
+
+// ---------------------------------------------------------------------------
+// element access: a chunk is 8 consecutive elements of one row
+// ---------------------------------------------------------------------------
+
+template <typename T> struct Elem;
+
+template <> struct Elem<__nv_bfloat16> {
+    struct Raw {
+        uint4 v;
+    };
+    static constexpr int kChunkBytes = 16;
+    __device__ __forceinline__ static Raw load(const uint8_t *tile, int j)
+    {
+        Raw r;
+        r.v = *reinterpret_cast<const uint4 *>(tile + j * 16);
+        return r;
+    }
+    __device__ __forceinline__ static void unpack(const Raw &r, float (&x)[8])
+    {
+        const uint32_t w[4] = {r.v.x, r.v.y, r.v.z, r.v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            x[2 * i] = __uint_as_float(w[i] << 16);
+            x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+};
+
+template <> struct Elem<float> {
+    struct Raw {
+        float4 a, b;
+    };
+    static constexpr int kChunkBytes = 32;
+    __device__ __forceinline__ static Raw load(const uint8_t *tile, int j)
+    {
+        Raw r;
+        r.a = *reinterpret_cast<const float4 *>(tile + j * 32);
+        r.b = *reinterpret_cast<const float4 *>(tile + j * 32 + 16);
+        return r;
+    }
+    __device__ __forceinline__ static void unpack(const Raw &r, float (&x)[8])
+    {
+        x[0] = r.a.x; x[1] = r.a.y; x[2] = r.a.z; x[3] = r.a.w;
+        x[4] = r.b.x; x[5] = r.b.y; x[6] = r.b.z; x[7] = r.b.w;
+    }
+};
+
+__device__ __forceinline__ float sq(float a) { return a * a; }
+
+// ---------------------------------------------------------------------------
+// quantizers of one chunk's values (VPC = 4 kept or 8 dense values); every
+// lane of the warp calls them (group reductions shuffle across lanes)
+// ---------------------------------------------------------------------------
+
+struct QOut {
+    void *values;
+    void *scales;
+    int64_t row, colq, n; // quantized row length n, column of the chunk's first value
+    bool valid;
+    int lane;
+};
+
+template <int VPC> __device__ __forceinline__ float local_amax(const float (&v)[VPC])
+{
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < VPC; ++i)
+        m = fmaxf(m, fabsf(v[i]));
+    return m;
+}
+
+__device__ __forceinline__ float group_amax(float m, int lanes)
+{
+    for (int off = 1; off < lanes; off <<= 1)
+        m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
+    return m;
+}
+
+template <int VPC> __device__ __forceinline__ float err_energy(const float (&v)[VPC], const float (&d)[VPC])
+{
+    float t[VPC];
+#pragma unroll
+    for (int i = 0; i < VPC; ++i)
+        t[i] = sq(v[i] - d[i]);
+#pragma unroll
+    for (int w = VPC / 2; w >= 1; w /= 2)
+#pragma unroll
+        for (int i = 0; i < w; ++i)
+            t[i] = t[i] + t[i + w];
+    return t[0];
+}
+
+// FP8 E4M3, per-tensor scale s: code = E4M3(v / s); deq = E4M3(code) * s.
+template <int VPC, bool STORE>
+__device__ __forceinline__ float quant_fp8(const float (&v)[VPC], float s, const QOut &o)
+{
+    uint32_t c[VPC / 4];
+    float d[VPC];
+    const bool nz = s != 0.0f;
+#pragma unroll
+    for (int t = 0; t < VPC / 4; ++t) {
+        float q[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            q[i] = nz ? __fdiv_rn(v[4 * t + i], s) : 0.0f;
+        c[t] = cvt_e4m3x2(q[0], q[1]) | (cvt_e4m3x2(q[2], q[3]) << 16);
+        const float2 lo = e4m3x2_to_f32(c[t] & 0xffffu), hi = e4m3x2_to_f32(c[t] >> 16);
+        d[4 * t + 0] = __fmul_rn(lo.x, s);
+        d[4 * t + 1] = __fmul_rn(lo.y, s);
+        d[4 * t + 2] = __fmul_rn(hi.x, s);
+        d[4 * t + 3] = __fmul_rn(hi.y, s);
+    }
+    if (STORE && o.valid) {
+        uint8_t *dst = static_cast<uint8_t *>(o.values) + o.row * o.n + o.colq;
+        if constexpr (VPC == 4)
+            *reinterpret_cast<uint32_t *>(dst) = c[0];
+        else
+            *reinterpret_cast<uint2 *>(dst) = make_uint2(c[0], c[1]);
+    }
+    return err_energy<VPC>(v, d);
+}
+
+// Symmetric INT-b, one fp32 scale per q.group quantized values (q.lanes
+// lanes). row_amax >= 0 supplies the group amax (row mode: the whole row) and
+// leaves the scale store to the caller.
+template <int VPC, bool STORE>
+__device__ __forceinline__ float quant_int(const float (&v)[VPC], const QuantSpec &q, const QOut &o,
+                                           float row_amax = -1.0f)
+{
+    const float amax = row_amax >= 0.0f ? row_amax : group_amax(local_amax<VPC>(v), q.lanes);
+    const float scale = __fdiv_rn(amax, q.qmax);
+    const int qm = static_cast<int>(q.qmax);
+    int c[VPC];
+    float d[VPC];
+#pragma unroll
+    for (int i = 0; i < VPC; ++i) {
+        int ci = 0;
+        if (scale != 0.0f)
+            ci = max(-qm, min(qm, __float2int_rn(__fdiv_rn(v[i], scale))));
+        c[i] = ci;
+        d[i] = __fmul_rn(static_cast<float>(ci), scale);
+    }
+    if (STORE && o.valid) {
+        const int64_t off = o.row * o.n + o.colq;
+        if (q.store == kInt8) {
+            uint32_t w[VPC / 4];
+#pragma unroll
+            for (int t = 0; t < VPC / 4; ++t)
+                w[t] = static_cast<uint32_t>(c[4 * t] & 0xff) | (static_cast<uint32_t>(c[4 * t + 1] & 0xff) << 8) |
+                       (static_cast<uint32_t>(c[4 * t + 2] & 0xff) << 16) |
+                       (static_cast<uint32_t>(c[4 * t + 3] & 0xff) << 24);
+            uint8_t *dst = static_cast<uint8_t *>(o.values) + off;
+            if constexpr (VPC == 4)
+                *reinterpret_cast<uint32_t *>(dst) = w[0];
+            else
+                *reinterpret_cast<uint2 *>(dst) = make_uint2(w[0], w[1]);
+        } else if (q.store == kInt16) {
+            uint32_t w[VPC / 2];
+#pragma unroll
+            for (int t = 0; t < VPC / 2; ++t)
+                w[t] = static_cast<uint32_t>(c[2 * t] & 0xffff) | (static_cast<uint32_t>(c[2 * t + 1] & 0xffff) << 16);
+            int16_t *dst = static_cast<int16_t *>(o.values) + off;
+            if constexpr (VPC == 4)
+                *reinterpret_cast<uint2 *>(dst) = make_uint2(w[0], w[1]);
+            else
+                *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+        } else {
+            uint32_t w = 0;
+#pragma unroll
+            for (int i = 0; i < VPC; ++i)
+                w |= static_cast<uint32_t>(c[i] & 0xf) << (4 * i);
+            uint8_t *dst = static_cast<uint8_t *>(o.values) + off / 2;
+            if constexpr (VPC == 4)
+                *reinterpret_cast<uint16_t *>(dst) = static_cast<uint16_t>(w);
+            else
+                *reinterpret_cast<uint32_t *>(dst) = w;
+        }
+        if (row_amax < 0.0f && (o.lane & (q.lanes - 1)) == 0)
+            static_cast<float *>(o.scales)[o.row * (o.n / q.group) + o.colq / q.group] = scale;
+    }
+    return err_energy<VPC>(v, d);
+}
+
+template <int VPC> __device__ __forceinline__ uint32_t pack_e2m1(const float (&q)[VPC])
+{
+    if constexpr (VPC == 4)
+        return cvt_e2m1x4(q[0], q[1], q[2], q[3]);
+    else
+        return cvt_e2m1x4(q[0], q[1], q[2], q[3]) | (cvt_e2m1x4(q[4], q[5], q[6], q[7]) << 16);
+}
+
+template <int VPC>
+__device__ __forceinline__ void unpack_e2m1(uint32_t codes, float mult, float (&d)[VPC])
+{
+#pragma unroll
+    for (int t = 0; t < VPC / 2; ++t) {
+        const float2 f = e2m1x2_to_f32((codes >> (8 * t)) & 0xffu);
+        d[2 * t] = __fmul_rn(f.x, mult);
+        d[2 * t + 1] = __fmul_rn(f.y, mult);
+    }
+}
+
+template <int VPC, bool STORE>
+__device__ __forceinline__ void store_fp4(uint32_t codes, const QOut &o)
+{
+    if (STORE && o.valid) {
+        uint8_t *dst = static_cast<uint8_t *>(o.values) + (o.row * o.n + o.colq) / 2;
+        if constexpr (VPC == 4)
+            *reinterpret_cast<uint16_t *>(dst) = static_cast<uint16_t>(codes);
+        else
+            *reinterpret_cast<uint32_t *>(dst) = codes;
+    }
+}
+
+// NVFP4: block of 16 values (16 / VPC lanes), E4M3 block scale over a fp32
+// tensor scale st.
+template <int VPC, bool STORE>
+__device__ __forceinline__ float quant_nvfp4(const float (&v)[VPC], float st, const QOut &o)
+{
+    constexpr int kLanes = 16 / VPC;
+    const float amax = group_amax(local_amax<VPC>(v), kLanes);
+    uint32_t sb = 0;
+    if (st != 0.0f)
+        sb = cvt_e4m3x2(__fdiv_rn(__fdiv_rn(amax, 6.0f), st), 0.0f) & 0xffu;
+    const float denom = __fmul_rn(e4m3_to_f32(sb), st);
+    float q[VPC], d[VPC];
+#pragma unroll
+    for (int i = 0; i < VPC; ++i)
+        q[i] = denom != 0.0f ? __fdiv_rn(v[i], denom) : 0.0f;
+    const uint32_t codes = pack_e2m1<VPC>(q);
+    unpack_e2m1<VPC>(codes, denom, d);
+    store_fp4<VPC, STORE>(codes, o);
+    if (STORE && o.valid && (o.lane & (kLanes - 1)) == 0)
+        static_cast<uint8_t *>(o.scales)[o.row * (o.n / 16) + o.colq / 16] = static_cast<uint8_t>(sb);
+    return err_energy<VPC>(v, d);
+}
+
+// MXFP4: block of 32 values (32 / VPC lanes), power-of-two scale 2^e stored as
+// the E8M0 byte e + 127; v / 2^e is computed as v * 2^-e (the same correctly
+// rounded value, since both scale factors are exact powers of two).
+template <int VPC, bool STORE>
+__device__ __forceinline__ float quant_mxfp4(const float (&v)[VPC], const QOut &o)
+{
+    constexpr int kLanes = 32 / VPC;
+    const float amax = group_amax(local_amax<VPC>(v), kLanes);
+    uint32_t byte = 0;
+    float inv = 0.0f, mult = 0.0f;
+    if (amax != 0.0f) {
+        const int e = mx_shared_exponent(amax);
+        byte = static_cast<uint32_t>(e + 127);
+        inv = exp2_int(-e);
+        mult = exp2_int(e);
+    }
+    float q[VPC], d[VPC];
+#pragma unroll
+    for (int i = 0; i < VPC; ++i)
+        q[i] = v[i] * inv;
+    const uint32_t codes = pack_e2m1<VPC>(q);
+    unpack_e2m1<VPC>(codes, mult, d);
+    store_fp4<VPC, STORE>(codes, o);
+    if (STORE && o.valid && (o.lane & (kLanes - 1)) == 0)
+        static_cast<uint8_t *>(o.scales)[o.row * (o.n / 32) + o.colq / 32] = static_cast<uint8_t>(byte);
+    return err_energy<VPC>(v, d);
+}
+
+// Runtime-dispatched quantizer without stores (the energy-only pass).
+template <int VPC>
+__device__ __forceinline__ float quant_energy_only(const float (&v)[VPC], const QuantSpec &q, float st)
+{
+    QOut o{nullptr, nullptr, 0, 0, 1, false, 0};
+    switch (q.fmt) {
+    case kFp8:
+        return quant_fp8<VPC, false>(v, st, o);
+    case kInt:
+        return quant_int<VPC, false>(v, q, o);
+    case kNvfp4:
+        return quant_nvfp4<VPC, false>(v, st, o);
+    case kMxfp4:
+        return quant_mxfp4<VPC, false>(v, o);
+    default:
+        return 0.0f;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// one chunk: score, select, quantize, store, energies
+// ---------------------------------------------------------------------------
+
+struct Acc {
+    float et, ep, eq, eqd; // energies of the current tile (binary32)
+    float amax_kept, amax_all;
+};
+
+template <int SCORE>
+__device__ __forceinline__ void scores(const float (&x)[8], const float *norms, int64_t col, bool in_k,
+                                       float (&s)[8])
+{
+    if constexpr (SCORE == kWanda) {
+        float4 n0 = make_float4(0.f, 0.f, 0.f, 0.f), n1 = n0;
+        if (in_k) {
+            n0 = __ldg(reinterpret_cast<const float4 *>(norms + col));
+            n1 = __ldg(reinterpret_cast<const float4 *>(norms + col + 4));
+        }
+        const float n[8] = {n0.x, n0.y, n0.z, n0.w, n1.x, n1.y, n1.z, n1.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            s[i] = __fmul_rn(fabsf(x[i]), n[i]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            s[i] = fabsf(x[i]);
+    }
+}
+
+template <typename T, int PAT, int SCORE, int FMT>
+__device__ __forceinline__ void process_chunk(const PassParams &p, const float (&x)[8], int64_t row,
+                                              int64_t col, int lane, float st, float std_, Acc &acc,
+                                              float row_amax = -1.0f)
+{
+    constexpr int VPC = PAT == kDense ? 8 : 4;
+    const bool in_k = col < p.k;
+    const bool valid = in_k && row < p.rows;
+    float v[VPC];
+    uint32_t meta = 0;
+    float ep = 0.0f;
+
+    if constexpr (PAT == kDense) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            v[i] = x[i];
+    } else {
+        float s[8];
+        scores<SCORE>(x, p.norms, col, in_k, s);
+        float dr[4];
+        if constexpr (PAT == kSparse24) {
+            const Pick g0 = top2_of_4(s[0], s[1], s[2], s[3]);
+            const Pick g1 = top2_of_4(s[4], s[5], s[6], s[7]);
+            apply24(g0, x[0], x[1], x[2], x[3], v[0], v[1], dr[0], dr[1]);
+            apply24(g1, x[4], x[5], x[6], x[7], v[2], v[3], dr[2], dr[3]);
+            meta = g0.nib | (g1.nib << 4);
+        } else {
+            float e[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                e[i] = __fadd_rn(__fmul_rn(s[2 * i], s[2 * i]), __fmul_rn(s[2 * i + 1], s[2 * i + 1]));
+            const Pick g = top2_of_4(e[0], e[1], e[2], e[3]);
+            // first and second elements of the kept pairs, in pair order
+            apply24(g, x[0], x[2], x[4], x[6], v[0], v[2], dr[0], dr[2]);
+            apply24(g, x[1], x[3], x[5], x[7], v[1], v[3], dr[1], dr[3]);
+            meta = g.nib;
+        }
+        ep = (sq(dr[0]) + sq(dr[1])) + (sq(dr[2]) + sq(dr[3]));
+    }
+
+    if constexpr (FMT == kAmax) {
+        acc.amax_all = fmaxf(acc.amax_all, local_amax<8>(x));
+        if constexpr (PAT != kDense)
+            acc.amax_kept = fmaxf(acc.amax_kept, local_amax<4>(v));
+        return;
+    }
+
+    const float et = ((sq(x[0]) + sq(x[1])) + (sq(x[2]) + sq(x[3]))) +
+                     ((sq(x[4]) + sq(x[5])) + (sq(x[6]) + sq(x[7])));
+    acc.et += et;
+    acc.ep += ep;
+
+    // metadata
+    if constexpr (PAT == kSparse24) {
+        if (FMT != kEnergy && valid)
+            p.meta[row * (p.k / 8) + col / 8] = static_cast<uint8_t>(meta);
+    } else if constexpr (PAT == kSparse48) {
+        const uint32_t other = __shfl_down_sync(kFull, meta, 1);
+        if (FMT != kEnergy && valid && (lane & 1) == 0)
+            p.meta[row * (p.k / 16) + col / 16] = static_cast<uint8_t>(meta | (other << 4));
+    }
+
+    const int64_t n = PAT == kDense ? p.k : p.k / 2;
+    const QOut o{p.values, p.scales, row, PAT == kDense ? col : col / 2, n, valid, lane};
+    float eq = 0.0f;
+    if constexpr (FMT == kNone) {
+        if (valid) {
+            if constexpr (sizeof(T) == 2) {
+                const uint32_t w0 = (__float_as_uint(v[0]) >> 16) | (__float_as_uint(v[1]) & 0xffff0000u);
+                const uint32_t w1 = (__float_as_uint(v[2]) >> 16) | (__float_as_uint(v[3]) & 0xffff0000u);
+                *reinterpret_cast<uint2 *>(static_cast<uint16_t *>(p.values) + row * n + col / 2) =
+                    make_uint2(w0, w1);
+            } else {
+                *reinterpret_cast<float4 *>(static_cast<float *>(p.values) + row * n + col / 2) =
+                    make_float4(v[0], v[1], v[2], v[3]);
+            }
+        }
+    } else if constexpr (FMT == kFp8) {
+        eq = quant_fp8<VPC, true>(v, st, o);
+    } else if constexpr (FMT == kInt) {
+        eq = quant_int<VPC, true>(v, p.q, o, row_amax);
+    } else if constexpr (FMT == kNvfp4) {
+        eq = quant_nvfp4<VPC, true>(v, st, o);
+    } else if constexpr (FMT == kMxfp4) {
+        eq = quant_mxfp4<VPC, true>(v, o);
+    } else if constexpr (FMT == kEnergy) {
+        eq = quant_energy_only<VPC>(v, p.q, st);
+        acc.eqd += quant_energy_only<8>(x, p.qd, std_);
+    }
+    if constexpr (PAT == kDense)
+        acc.eqd += eq;
+    else
+        acc.eq += eq;
+}
+
+// ---------------------------------------------------------------------------
+// kernel
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void record_error(int32_t *err, int32_t code)
+{
+    atomicCAS(err, 0, code);
+}
+
+// Tensor scale of a per-tensor format: the given one, or amax / divisor.
+__device__ __forceinline__ float tensor_scale(const QuantSpec &q)
+{
+    if (q.fmt != kFp8 && q.fmt != kNvfp4)
+        return 0.0f;
+    if (q.scale_in)
+        return *q.scale_in;
+    return __fdiv_rn(*q.amax_reduced, q.divisor);
+}
+
+// Grid-wide energy reduction: per-CTA binary64 partials go to the workspace;
+// the CTA that takes the last ticket sums them in fixed order, writes the
+// caller's 4-double record and resets the ticket. Called by all consumers.
+__device__ __forceinline__ void grid_reduce_energy(const PassParams &p, double e_total, double e_prune, double e_q,
+                                                   double e_qd, double *red, uint32_t *flag, int tid, int lane,
+                                                   int warp)
+{
+    double e[4] = {e_total, e_prune, e_q, e_qd};
+#pragma unroll
+    for (int f = 0; f < 4; ++f)
+        for (int off = 16; off >= 1; off >>= 1)
+            e[f] += __shfl_xor_sync(kFull, e[f], off);
+    if (lane == 0)
+#pragma unroll
+        for (int f = 0; f < 4; ++f)
+            red[warp * 4 + f] = e[f];
+    named_barrier_sync(1, kConsumers);
+    if (tid == 0) {
+        double sum[4] = {0.0, 0.0, 0.0, 0.0};
+        for (int w = 0; w < kConsumerWarps; ++w)
+#pragma unroll
+            for (int f = 0; f < 4; ++f)
+                sum[f] += red[w * 4 + f];
+#pragma unroll
+        for (int f = 0; f < 4; ++f)
+            p.energy_partials[blockIdx.x * 4 + f] = sum[f];
+        __threadfence();
+        const uint32_t ticket = atomicAdd(p.energy_ticket, 1u);
+        *flag = ticket == gridDim.x - 1;
+    }
+    named_barrier_sync(1, kConsumers);
+    if (*flag) {
+        __threadfence();
+        // thread tid sums field (tid & 3) over CTAs (tid >> 2), (tid >> 2) + 64, ...
+        const int f = tid & 3;
+        double acc_f = 0.0;
+        for (int i = tid >> 2; i < static_cast<int>(gridDim.x); i += kConsumers / 4)
+            acc_f += __ldcg(p.energy_partials + 4 * i + f);
+        // lanes holding the same field differ in lane bits 2..4
+        for (int off = 16; off >= 4; off >>= 1)
+            acc_f += __shfl_xor_sync(kFull, acc_f, off);
+        named_barrier_sync(1, kConsumers);
+        if (lane < 4)
+            red[warp * 4 + lane] = acc_f;
+        named_barrier_sync(1, kConsumers);
+        if (tid < 4) {
+            double total = 0.0;
+            for (int w = 0; w < kConsumerWarps; ++w)
+                total += red[w * 4 + tid];
+            p.energy_out[tid] = total;
+        }
+        if (tid == 0)
+            *p.energy_ticket = 0;
+    }
+}
+
+__device__ __forceinline__ void producer(const CUtensorMap *map, const PassParams &p, uint8_t *stages,
+                                         uint64_t *full, uint64_t *empty)
+{
+    const uint64_t policy = l2_evict_first_policy();
+    uint32_t it = 0;
+    bool failed = false;
+    for (int64_t t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++it) {
+        const int s = it % kStages;
+        const uint32_t use = it / kStages;
+        if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1)) {
+            record_error(p.err, 1);
+            failed = true;
+            break;
+        }
+        mbar_arrive_expect_tx(&full[s], p.tile_bytes);
+        const int64_t rt = t / p.n_col_tiles, ct = t - rt * p.n_col_tiles;
+        tma_load_2d(stages + s * kStageBytes, map, static_cast<int32_t>(ct * p.W),
+                    static_cast<int32_t>(rt * p.R), &full[s], policy);
+    }
+    if (failed) {
+        // let the copies already issued land before the CTA can exit
+        for (int s = 0; s < kStages && s < static_cast<int>(it); ++s) {
+            const uint32_t last_use = (it - 1 - ((it - 1 - s) % kStages)) / kStages;
+            (void)mbar_wait(&full[s], last_use & 1);
+        }
+    }
+}
+
+template <typename T, int PAT, int SCORE, int FMT>
+__global__ void __launch_bounds__(kThreads, 1) pass_kernel(const __grid_constant__ CUtensorMap map,
+                                                           const PassParams p)
+{
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t *stages = smem;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kStages * kStageBytes);
+    uint64_t *empty = full + kStages;
+    double *red = reinterpret_cast<double *>(empty + kStages); // [kConsumerWarps][4]
+    float *fred = reinterpret_cast<float *>(red + kConsumerWarps * 4); // [kConsumerWarps][2]
+    uint32_t *flag = reinterpret_cast<uint32_t *>(fred + kConsumerWarps * 2);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    if (warp == kConsumerWarps) {
+        if (lane == 0)
+            producer(&map, p, stages, full, empty);
+        return;
+    }
+
+    // ---- consumers ----
+    float st = 0.0f, std_ = 0.0f;
+    if constexpr (FMT == kFp8 || FMT == kNvfp4 || FMT == kEnergy) {
+        st = tensor_scale(p.q);
+        if (blockIdx.x == 0 && tid == 0 && p.q.scale_out)
+            *p.q.scale_out = st;
+    }
+    if constexpr (FMT == kEnergy)
+        std_ = tensor_scale(p.qd);
+
+    using E = Elem<T>;
+    const int cpr_mask = (1 << p.log2_cpr) - 1;
+    const bool energies = p.energy_out != nullptr;
+    double e_total = 0.0, e_prune = 0.0, e_q = 0.0, e_qd = 0.0;
+    Acc acc{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    uint32_t it = 0;
+    for (int64_t t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++it) {
+        const int s = it % kStages;
+        if (!mbar_wait(&full[s], (it / kStages) & 1)) {
+            record_error(p.err, 2);
+            break;
+        }
+        const uint8_t *tile = stages + s * kStageBytes;
+        typename E::Raw raw[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            if (i < p.cpt)
+                raw[i] = E::load(tile, tid + i * kConsumers);
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(&empty[s]);
+
+        const int64_t rt = t / p.n_col_tiles, ct = t - rt * p.n_col_tiles;
+        const int64_t row0 = rt * p.R, col0 = ct * p.W;
+        acc.et = acc.ep = acc.eq = acc.eqd = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            if (i < p.cpt) {
+                const int j = tid + i * kConsumers;
+                const int64_t row = row0 + (j >> p.log2_cpr);
+                const int64_t col = col0 + ((j & cpr_mask) << 3);
+                float x[8];
+                E::unpack(raw[i], x);
+                process_chunk<T, PAT, SCORE, FMT>(p, x, row, col, lane, st, std_, acc);
+            }
+        }
+        if constexpr (FMT != kAmax) {
+            e_total += acc.et;
+            e_prune += acc.ep;
+            e_q += acc.eq;
+            e_qd += acc.eqd;
+        }
+    }
+
+    // ---- grid reductions (last CTA to finish reduces the partials) ----
+    if constexpr (FMT == kAmax) {
+        float a = acc.amax_kept, b = acc.amax_all;
+        for (int off = 16; off >= 1; off >>= 1) {
+            a = fmaxf(a, __shfl_xor_sync(kFull, a, off));
+            b = fmaxf(b, __shfl_xor_sync(kFull, b, off));
+        }
+        if (lane == 0) {
+            fred[warp * 2] = a;
+            fred[warp * 2 + 1] = b;
+        }
+        named_barrier_sync(1, kConsumers);
+        if (tid == 0) {
+            for (int w = 1; w < kConsumerWarps; ++w) {
+                a = fmaxf(a, fred[w * 2]);
+                b = fmaxf(b, fred[w * 2 + 1]);
+            }
+            p.amax_partials[blockIdx.x * 2] = a;
+            p.amax_partials[blockIdx.x * 2 + 1] = b;
+            __threadfence();
+            const uint32_t ticket = atomicAdd(p.amax_ticket, 1u);
+            *flag = ticket == gridDim.x - 1;
+        }
+        named_barrier_sync(1, kConsumers);
+        if (*flag) {
+            __threadfence();
+            float ka = 0.0f, kb = 0.0f;
+            for (int i = tid; i < static_cast<int>(gridDim.x); i += kConsumers) {
+                ka = fmaxf(ka, __ldcg(p.amax_partials + 2 * i));
+                kb = fmaxf(kb, __ldcg(p.amax_partials + 2 * i + 1));
+            }
+            for (int off = 16; off >= 1; off >>= 1) {
+                ka = fmaxf(ka, __shfl_xor_sync(kFull, ka, off));
+                kb = fmaxf(kb, __shfl_xor_sync(kFull, kb, off));
+            }
+            named_barrier_sync(1, kConsumers);
+            if (lane == 0) {
+                fred[warp * 2] = ka;
+                fred[warp * 2 + 1] = kb;
+            }
+            named_barrier_sync(1, kConsumers);
+            if (tid == 0) {
+                for (int w = 1; w < kConsumerWarps; ++w) {
+                    ka = fmaxf(ka, fred[w * 2]);
+                    kb = fmaxf(kb, fred[w * 2 + 1]);
+                }
+                p.amax_out[0] = PAT == kDense ? kb : ka;
+                p.amax_out[1] = kb;
+                *p.amax_ticket = 0;
+            }
+        }
+        return;
+    } else {
+        if (!energies)
+            return;
+        grid_reduce_energy(p, e_total, e_prune, e_q, e_qd, red, flag, tid, lane, warp);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// row mode: INT with one scale per row when a row does not fit one warp's
+// span (k > 256, or k not a power of two). A stage holds R whole rows, loaded
+// as ceil(k / W) TMA boxes of [R rows x W columns] (W = min(256, next power of
+// two >= k)) laid out [box][row][W] in shared memory.
+// Warp w owns rows w, w + 8, ... of the stage: a first sweep over the row takes
+// the amax of the values to quantize, a second sweep quantizes and stores.
+// ---------------------------------------------------------------------------
+
+// Chunk c of row r in a row-mode stage laid out [box][row][W]; zeros past the
+// padded row end (lanes without a chunk still take part in warp shuffles).
+template <typename T>
+__device__ __forceinline__ void load_row_chunk(const uint8_t *tile, int c, int r, int R, int cpb_log2, bool have,
+                                               float (&x)[8])
+{
+    if (have) {
+        const int box = c >> cpb_log2, cc = c & ((1 << cpb_log2) - 1);
+        Elem<T>::unpack(Elem<T>::load(tile, ((box * R + r) << cpb_log2) + cc), x);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            x[i] = 0.0f;
+    }
+}
+
+__device__ __forceinline__ void row_producer(const CUtensorMap *map, const PassParams &p, uint8_t *stages,
+                                             uint64_t *full, uint64_t *empty, int nbox, int esize)
+{
+    const uint64_t policy = l2_evict_first_policy();
+    uint32_t it = 0;
+    bool failed = false;
+    const int box_bytes = p.R * p.W * esize;
+    for (int64_t t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++it) {
+        const int s = it % kRowStages;
+        const uint32_t use = it / kRowStages;
+        if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1)) {
+            record_error(p.err, 3);
+            failed = true;
+            break;
+        }
+        mbar_arrive_expect_tx(&full[s], p.tile_bytes);
+        for (int b = 0; b < nbox; ++b)
+            tma_load_2d(stages + s * kRowStageBytes + b * box_bytes, map, b * p.W,
+                        static_cast<int32_t>(t * p.R), &full[s], policy);
+    }
+    if (failed) {
+        for (int s = 0; s < kRowStages && s < static_cast<int>(it); ++s) {
+            const uint32_t last_use = (it - 1 - ((it - 1 - s) % kRowStages)) / kRowStages;
+            (void)mbar_wait(&full[s], last_use & 1);
+        }
+    }
+}
+
+template <typename T, int PAT, int SCORE>
+__global__ void __launch_bounds__(kThreads, 1) row_kernel(const __grid_constant__ CUtensorMap map,
+                                                          const PassParams p)
+{
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t *stages = smem;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kRowStages * kRowStageBytes);
+    uint64_t *empty = full + kRowStages;
+    double *red = reinterpret_cast<double *>(empty + kRowStages);
+    uint32_t *flag = reinterpret_cast<uint32_t *>(red + kConsumerWarps * 4);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nbox = static_cast<int>((p.k + p.W - 1) / p.W);
+    if (tid == 0) {
+        for (int s = 0; s < kRowStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (warp == kConsumerWarps) {
+        if (lane == 0)
+            row_producer(&map, p, stages, full, empty, nbox, static_cast<int>(sizeof(T)));
+        return;
+    }
+
+    const int cpb_log2 = p.log2_cpr;            // log2(chunks per box row), box width = p.W
+    const int nchunks = nbox << cpb_log2;        // chunks per (padded) row
+    double e_total = 0.0, e_prune = 0.0, e_q = 0.0, e_qd = 0.0;
+    uint32_t it = 0;
+    for (int64_t t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++it) {
+        const int s = it % kRowStages;
+        if (!mbar_wait(&full[s], (it / kRowStages) & 1)) {
+            record_error(p.err, 4);
+            break;
+        }
+        const uint8_t *tile = stages + s * kRowStageBytes;
+        for (int r = warp; r < p.R; r += kConsumerWarps) {
+            const int64_t row = t * p.R + r;
+            // chunk c of row r sits at chunk index (c / 32 * R + r) * 32 + c % 32
+            float amax = 0.0f;
+            for (int c0 = 0; c0 < nchunks; c0 += 32) {
+                const int c = c0 + lane;
+                float x[8];
+                load_row_chunk<T>(tile, c, r, p.R, cpb_log2, c < nchunks, x);
+                if constexpr (PAT == kDense || SCORE == kMag) {
+                    // for the magnitude score the kept amax equals the amax of all
+                    amax = fmaxf(amax, local_amax<8>(x));
+                } else {
+                    Acc a{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    process_chunk<T, PAT, SCORE, kAmax>(p, x, row, static_cast<int64_t>(c) * 8, lane, 0.f, 0.f, a);
+                    amax = fmaxf(amax, a.amax_kept);
+                }
+            }
+            amax = group_amax(amax, 32);
+            Acc acc{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            for (int c0 = 0; c0 < nchunks; c0 += 32) {
+                const int c = c0 + lane;
+                float x[8];
+                load_row_chunk<T>(tile, c, r, p.R, cpb_log2, c < nchunks, x);
+                process_chunk<T, PAT, SCORE, kInt>(p, x, row, static_cast<int64_t>(c) * 8, lane, 0.f, 0.f, acc,
+                                                   amax);
+            }
+            if (lane == 0 && row < p.rows)
+                static_cast<float *>(p.scales)[row] = __fdiv_rn(amax, p.q.qmax);
+            e_total += acc.et;
+            e_prune += acc.ep;
+            e_q += acc.eq;
+            e_qd += acc.eqd;
+        }
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(&empty[s]);
+    }
+
+    if (!p.energy_out)
+        return;
+    grid_reduce_energy(p, e_total, e_prune, e_q, e_qd, red, flag, tid, lane, warp);
+}
+
+} // namespace ss24

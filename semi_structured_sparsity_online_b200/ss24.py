@@ -1,0 +1,302 @@
+"""ctypes binding of ``libss24.so`` (declared in ``include/ss24.h``).
+
+Argument marshalling only: every step of the pass runs in the library's CUDA
+kernels. PyTorch supplies device memory (outputs are allocated as torch
+tensors) and the current CUDA stream. The raw C functions are available as
+``lib().ss24_*``; the helpers below wrap them for torch tensors.
+
+The library must have been built (``semi_structured_sparsity_online_b200.build``
+or ``__graft_entry__.build()``); loading fails loudly otherwise. There is no
+CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libss24.so")
+
+# enums (include/ss24.h)
+OK = 0
+STATUS_NAMES = {0: "SS24_OK", 1: "SS24_ERR_NULL", 2: "SS24_ERR_SHAPE", 3: "SS24_ERR_ALIGN",
+                4: "SS24_ERR_DTYPE", 5: "SS24_ERR_FORMAT", 6: "SS24_ERR_WORKSPACE", 7: "SS24_ERR_CUDA",
+                8: "SS24_ERR_ARG"}
+BF16, F32 = 0, 1
+MAG, WANDA = 0, 1
+DENSE, SPARSE_24, SPARSE_48 = 0, 24, 48
+FMT_NONE, FMT_FP8, FMT_INT, FMT_NVFP4, FMT_MXFP4 = 0, 1, 2, 3, 4
+_FMT = {"none": FMT_NONE, "fp8": FMT_FP8, "int": FMT_INT, "nvfp4": FMT_NVFP4, "mxfp4": FMT_MXFP4}
+_SCORE = {"mag": MAG, "wanda": WANDA}
+
+
+class Format(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("bits", ctypes.c_int32), ("group", ctypes.c_int32),
+                ("pack4", ctypes.c_int32)]
+
+
+class Operand(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("axis", ctypes.c_int32),
+                ("rows", ctypes.c_int64), ("k", ctypes.c_int64), ("ld", ctypes.c_int64)]
+
+
+class Outputs(ctypes.Structure):
+    _fields_ = [("values", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("tensor_scale", ctypes.c_void_p), ("meta", ctypes.c_void_p)]
+
+
+class SS24Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+
+
+_lib = None
+_P = ctypes.c_void_p
+_S = ctypes.c_size_t
+_OP = ctypes.POINTER(Operand)
+_OUT = ctypes.POINTER(Outputs)
+
+_SIGNATURES = {
+    "ss24_workspace_bytes": (ctypes.c_size_t, []),
+    "ss24_workspace_init": (ctypes.c_int, [_P, _S, _P]),
+    "ss24_workspace_error": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int32), _P]),
+    "ss24_prune24_compress": (ctypes.c_int, [_OP, ctypes.c_int, _P, _P, _P, _P, _P, _S, _P]),
+    "ss24_quantize_fp8": (ctypes.c_int, [_OP, _P, _OUT, _P, _P, _S, _P]),
+    "ss24_quantize_int": (ctypes.c_int, [_OP, Format, _OUT, _P, _P, _S, _P]),
+    "ss24_quantize_nvfp4": (ctypes.c_int, [_OP, _P, _OUT, _P, _P, _S, _P]),
+    "ss24_quantize_mxfp4": (ctypes.c_int, [_OP, _OUT, _P, _P, _S, _P]),
+    "ss24_prune24_quant_fused": (ctypes.c_int, [_OP, ctypes.c_int, _P, Format, _P, _OUT, _P, _P, _S, _P]),
+    "ss24_prune48_pairwise_quant_fused": (ctypes.c_int,
+                                          [_OP, ctypes.c_int, _P, Format, _P, _OUT, _P, _P, _S, _P]),
+    "ss24_error_energy": (ctypes.c_int, [_OP, ctypes.c_int, ctypes.c_int, _P, Format, Format, _P, _P, _P, _P,
+                                         _S, _P]),
+    "ss24_amax": (ctypes.c_int, [_OP, ctypes.c_int, ctypes.c_int, _P, _P, _P, _S, _P]),
+    "ss24_predicted_ratio": (ctypes.c_int, [_P, _P, _P, _P]),
+    "ss24_bits_per_element": (ctypes.c_double, [Format, ctypes.c_int, ctypes.c_int64, ctypes.c_int32]),
+    "ss24_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "ss24_encode_e4m3": (ctypes.c_int, [_P, _P, ctypes.c_int64, _P]),
+    "ss24_decode_e4m3": (ctypes.c_int, [_P, _P, ctypes.c_int64, _P]),
+    "ss24_encode_e2m1": (ctypes.c_int, [_P, _P, ctypes.c_int64, _P]),
+    "ss24_decode_e2m1": (ctypes.c_int, [_P, _P, ctypes.c_int64, _P]),
+}
+
+
+def lib():
+    """Load libss24.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build the CUDA library first "
+                               "(python -m semi_structured_sparsity_online_b200.build)")
+        h = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            f = getattr(h, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = h
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != OK:
+        raise SS24Error(status, where)
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def make_format(fmt="none", bits=8, group=0, pack4=False) -> Format:
+    kind = _FMT[fmt] if isinstance(fmt, str) else int(fmt)
+    return Format(kind, int(bits), int(group), int(bool(pack4)))
+
+
+def make_operand(x: torch.Tensor, axis: int = 1, rows=None, k=None) -> Operand:
+    """Operand descriptor of a 2-D CUDA tensor. axis 1: x is [rows, ld] with k
+    contiguous; axis 0: x is [k, ld] holding A[r][c] at x[c][r]."""
+    if x.dtype == torch.bfloat16:
+        dt = BF16
+    elif x.dtype == torch.float32:
+        dt = F32
+    else:
+        raise TypeError("operand must be bfloat16 or float32")
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("operand must be 2-D with a contiguous last dimension")
+    if axis == 1:
+        r = x.shape[0] if rows is None else rows
+        kk = x.shape[1] if k is None else k
+    else:
+        kk = x.shape[0] if k is None else k
+        r = x.shape[1] if rows is None else rows
+    return Operand(x.data_ptr(), dt, axis, r, kk, x.stride(0))
+
+
+class Workspace:
+    """Device workspace for the library's calls (allocated by torch, cleared once)."""
+
+    def __init__(self, device=None, stream=None):
+        n = lib().ss24_workspace_bytes()
+        self.buf = torch.empty(n + 256, dtype=torch.uint8, device=device or "cuda")
+        off = (-self.buf.data_ptr()) % 256
+        self.tensor = self.buf[off:off + n]
+        self.nbytes = n
+        _check(lib().ss24_workspace_init(self.ptr, n, _stream(stream)), "ss24_workspace_init")
+
+    @property
+    def ptr(self):
+        return ctypes.c_void_p(self.tensor.data_ptr())
+
+    def error(self, stream=None) -> int:
+        code = ctypes.c_int32(0)
+        _check(lib().ss24_workspace_error(self.ptr, ctypes.byref(code), _stream(stream)), "ss24_workspace_error")
+        return code.value
+
+
+_default_ws = {}
+
+
+def default_workspace(device=None) -> Workspace:
+    dev = torch.device(device or "cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    if dev not in _default_ws:
+        _default_ws[dev] = Workspace(dev)
+    return _default_ws[dev]
+
+
+def _alloc_outputs(x_rows, k, pattern, fmt: Format, in_dtype, device):
+    sparse = pattern != DENSE
+    n = k // 2 if sparse else k
+    out = {}
+    if fmt.kind == FMT_NONE:
+        out["values"] = torch.empty((x_rows, n), dtype=in_dtype, device=device)
+    elif fmt.kind == FMT_FP8:
+        out["values"] = torch.empty((x_rows, n), dtype=torch.uint8, device=device)
+    elif fmt.kind == FMT_INT:
+        if fmt.pack4:
+            out["values"] = torch.empty((x_rows, n // 2), dtype=torch.uint8, device=device)
+        else:
+            out["values"] = torch.empty((x_rows, n), dtype=torch.int16 if fmt.bits > 8 else torch.int8,
+                                        device=device)
+        g = fmt.group or n
+        out["scales"] = torch.empty((x_rows, n // g), dtype=torch.float32, device=device)
+    elif fmt.kind in (FMT_NVFP4, FMT_MXFP4):
+        out["values"] = torch.empty((x_rows, n // 2), dtype=torch.uint8, device=device)
+        blk = 16 if fmt.kind == FMT_NVFP4 else 32
+        out["scales"] = torch.empty((x_rows, n // blk), dtype=torch.uint8, device=device)
+    if fmt.kind in (FMT_FP8, FMT_NVFP4):
+        out["tensor_scale"] = torch.empty(1, dtype=torch.float32, device=device)
+    if sparse:
+        out["meta"] = torch.empty((x_rows, k // (16 if pattern == SPARSE_48 else 8)), dtype=torch.uint8,
+                                  device=device)
+    return out
+
+
+def run(x: torch.Tensor, pattern=SPARSE_24, fmt="none", bits=8, group=0, pack4=False, score="mag",
+        col_norms=None, tensor_scale=None, energy=True, axis=1, ws=None, stream=None, out=None):
+    """One pass through the matching C entry point. Returns a dict of output
+    tensors (``values``, ``scales``, ``tensor_scale``, ``meta``) and ``energy``
+    (float64[4] on the device: e_total, e_prune, e_quant, e_quant_dense)."""
+    f = make_format(fmt, bits, group, pack4)
+    op = make_operand(x, axis)
+    sc = _SCORE[score] if isinstance(score, str) else int(score)
+    if out is None:
+        out = _alloc_outputs(op.rows, op.k, pattern, f, x.dtype, x.device)
+    e = torch.zeros(4, dtype=torch.float64, device=x.device) if energy is True else energy
+    if e is not None and e is not False:
+        out["energy"] = e
+    else:
+        e = None
+    ws = ws or default_workspace(x.device)
+    o = Outputs(*(_ptr(out.get(key)) for key in ("values", "scales", "tensor_scale", "meta")))
+    s = _stream(stream)
+    L = lib()
+    if pattern == DENSE:
+        if f.kind == FMT_FP8:
+            st = L.ss24_quantize_fp8(ctypes.byref(op), _ptr(tensor_scale), ctypes.byref(o), _ptr(e), ws.ptr,
+                                     ws.nbytes, s)
+        elif f.kind == FMT_INT:
+            st = L.ss24_quantize_int(ctypes.byref(op), f, ctypes.byref(o), _ptr(e), ws.ptr, ws.nbytes, s)
+        elif f.kind == FMT_NVFP4:
+            st = L.ss24_quantize_nvfp4(ctypes.byref(op), _ptr(tensor_scale), ctypes.byref(o), _ptr(e), ws.ptr,
+                                       ws.nbytes, s)
+        elif f.kind == FMT_MXFP4:
+            st = L.ss24_quantize_mxfp4(ctypes.byref(op), ctypes.byref(o), _ptr(e), ws.ptr, ws.nbytes, s)
+        else:
+            raise ValueError("dense pattern needs a quantization format")
+        _check(st, "ss24_quantize")
+    elif pattern == SPARSE_24 and f.kind == FMT_NONE and tensor_scale is None:
+        _check(L.ss24_prune24_compress(ctypes.byref(op), sc, _ptr(col_norms), _ptr(out["values"]),
+                                       _ptr(out["meta"]), _ptr(e), ws.ptr, ws.nbytes, s), "ss24_prune24_compress")
+    else:
+        fn = L.ss24_prune24_quant_fused if pattern == SPARSE_24 else L.ss24_prune48_pairwise_quant_fused
+        _check(fn(ctypes.byref(op), sc, _ptr(col_norms), f, _ptr(tensor_scale), ctypes.byref(o), _ptr(e),
+                  ws.ptr, ws.nbytes, s), "ss24_prune_quant_fused")
+    return out
+
+
+def error_energy(x, pattern=SPARSE_24, sparse_fmt=("none",), dense_fmt=("int", 8, 0), score="mag",
+                 col_norms=None, sparse_scale=None, dense_scale=None, axis=1, ws=None, stream=None, energy=None):
+    """Read-only energy pass; returns float64[4] on the device."""
+    sf = make_format(*sparse_fmt) if isinstance(sparse_fmt, tuple) else sparse_fmt
+    df = make_format(*dense_fmt) if isinstance(dense_fmt, tuple) else dense_fmt
+    op = make_operand(x, axis)
+    e = energy if energy is not None else torch.zeros(4, dtype=torch.float64, device=x.device)
+    ws = ws or default_workspace(x.device)
+    _check(lib().ss24_error_energy(ctypes.byref(op), pattern, _SCORE[score] if isinstance(score, str) else score,
+                                   _ptr(col_norms), sf, df, _ptr(sparse_scale), _ptr(dense_scale), _ptr(e), ws.ptr,
+                                   ws.nbytes, _stream(stream)), "ss24_error_energy")
+    return e
+
+
+def amax(x, pattern=SPARSE_24, score="mag", col_norms=None, axis=1, ws=None, stream=None):
+    op = make_operand(x, axis)
+    out = torch.empty(1, dtype=torch.float32, device=x.device)
+    ws = ws or default_workspace(x.device)
+    _check(lib().ss24_amax(ctypes.byref(op), pattern, _SCORE[score] if isinstance(score, str) else score,
+                           _ptr(col_norms), _ptr(out), ws.ptr, ws.nbytes, _stream(stream)), "ss24_amax")
+    return out
+
+
+def predicted_ratio(sparse_energy, dense_energy, out=None, stream=None):
+    """float64[4] on the device: loss, rel_err_sparse, rel_err_dense, R_hat."""
+    r = out if out is not None else torch.empty(4, dtype=torch.float64, device=sparse_energy.device)
+    _check(lib().ss24_predicted_ratio(_ptr(sparse_energy), _ptr(dense_energy), _ptr(r), _stream(stream)),
+           "ss24_predicted_ratio")
+    return r
+
+
+def bits_per_element(fmt="none", bits=8, group=0, pattern=SPARSE_24, k=4096, with_scales=False) -> float:
+    return lib().ss24_bits_per_element(make_format(fmt, bits, group), pattern, k, int(with_scales))
+
+
+def status_string(status: int) -> str:
+    return lib().ss24_status_string(status).decode()
+
+
+def _convert(name, t_in, out_dtype, stream=None):
+    out = torch.empty(t_in.shape, dtype=out_dtype, device=t_in.device)
+    _check(getattr(lib(), name)(_ptr(t_in), _ptr(out), t_in.numel(), _stream(stream)), name)
+    return out
+
+
+def encode_e4m3(t, stream=None):
+    return _convert("ss24_encode_e4m3", t.contiguous(), torch.uint8, stream)
+
+
+def decode_e4m3(t, stream=None):
+    return _convert("ss24_decode_e4m3", t.contiguous(), torch.float32, stream)
+
+
+def encode_e2m1(t, stream=None):
+    return _convert("ss24_encode_e2m1", t.contiguous(), torch.uint8, stream)
+
+
+def decode_e2m1(t, stream=None):
+    return _convert("ss24_decode_e2m1", t.contiguous(), torch.float32, stream)

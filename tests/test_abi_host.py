@@ -1,0 +1,176 @@
+"""Host-side checks of the C ABI: the library loads, exports every function the
+header declares, and rejects invalid arguments before touching the GPU.
+No test here launches a kernel."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+from semi_structured_sparsity_online_b200 import ss24
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "ss24.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return sorted(set(re.findall(r"\b(ss24_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert len(names) >= 19
+    L = ss24.lib()
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(ss24._SIGNATURES)
+
+
+def test_workspace_bytes_and_status_strings():
+    assert ss24.lib().ss24_workspace_bytes() >= 256 + 32 * 1024
+    for s in range(9):
+        assert ss24.status_string(s)
+    assert ss24.status_string(99) == "unknown status"
+
+
+def test_bits_per_element_matches_oracle_accounting():
+    for fmt, bits, group in [("none", 16, 0), ("fp8", 8, 0), ("int", 3, 0), ("int", 8, 128), ("int", 16, 64),
+                             ("nvfp4", 4, 0), ("mxfp4", 4, 0)]:
+        for pattern in (ss24.DENSE, ss24.SPARSE_24, ss24.SPARSE_48):
+            for ws in (False, True):
+                a = ss24.bits_per_element(fmt, bits, group, pattern, 4096, ws)
+                b = oracle.bits_per_element(fmt, bits, group, pattern, 4096, ws)
+                assert a == b, (fmt, bits, group, pattern, ws)
+    # equal-bit identity: 2:4 on 2m bits == dense m+1 bits
+    for m in range(1, 9):
+        assert ss24.bits_per_element("int", 2 * m) == ss24.bits_per_element("int", m + 1, pattern=ss24.DENSE)
+    assert ss24.bits_per_element("int", 1) < 0
+
+
+# Fake, never-dereferenced pointer values: every call below fails validation,
+# so nothing is launched and no pointer is read.
+ALIGNED = 0x7F0000000000
+MISALIGNED = ALIGNED + 8
+WS_BYTES = None
+
+
+def _ws_bytes():
+    return ss24.lib().ss24_workspace_bytes()
+
+
+def op(x=ALIGNED, dtype=ss24.BF16, axis=1, rows=16, k=64, ld=64):
+    return ss24.Operand(x, dtype, axis, rows, k, ld)
+
+
+def outs(values=ALIGNED, scales=ALIGNED, tscale=ALIGNED, meta=ALIGNED):
+    return ss24.Outputs(values, scales, tscale, meta)
+
+
+def fused(o, fmt=None, ws=ALIGNED, ws_bytes=None, score=ss24.MAG, norms=None, out=None):
+    fmt = fmt or ss24.make_format("nvfp4")
+    out = out or outs()
+    return ss24.lib().ss24_prune24_quant_fused(ctypes.byref(o) if o is not None else None, score, norms, fmt,
+                                               None, ctypes.byref(out), None, ws,
+                                               _ws_bytes() if ws_bytes is None else ws_bytes, None)
+
+
+@pytest.mark.parametrize("case,expected", [
+    ("null_operand", 1), ("null_x", 1), ("bad_dtype", 4), ("bad_axis", 8), ("neg_rows", 2), ("zero_k", 2),
+    ("ld_lt_k", 2), ("misaligned_x", 3), ("odd_ld", 3), ("k_not_mult8", 2), ("nvfp4_k", 2),
+    ("bad_kind", 5), ("int_bits", 5), ("int_pack4", 5), ("int_group_np2", 5), ("int_group_big", 5),
+    ("ws_null", 6), ("ws_small", 6), ("ws_misaligned", 6), ("null_values", 1), ("null_meta", 1),
+    ("null_scales", 1), ("null_tscale", 1), ("wanda_no_norms", 1), ("wanda_misaligned_norms", 3),
+    ("bad_score", 8), ("misaligned_values", 3),
+])
+def test_validation_rejects_before_launch(case, expected):
+    f = None
+    o = op()
+    kw = {}
+    if case == "null_operand":
+        o = None
+    elif case == "null_x":
+        o = op(x=0)
+    elif case == "bad_dtype":
+        o = op(dtype=7)
+    elif case == "bad_axis":
+        o = op(axis=2)
+    elif case == "neg_rows":
+        o = op(rows=-1)
+    elif case == "zero_k":
+        o = op(k=0)
+    elif case == "ld_lt_k":
+        o = op(ld=32)
+    elif case == "misaligned_x":
+        o = op(x=MISALIGNED)
+    elif case == "odd_ld":
+        o = op(ld=68 + 1)
+    elif case == "k_not_mult8":
+        o = op(k=60, ld=64)
+    elif case == "nvfp4_k":
+        o = op(k=48, ld=64)
+    elif case == "bad_kind":
+        f = ss24.Format(9, 8, 0, 0)
+    elif case == "int_bits":
+        f = ss24.make_format("int", 17)
+    elif case == "int_pack4":
+        f = ss24.make_format("int", 8, 0, True)
+    elif case == "int_group_np2":
+        f = ss24.make_format("int", 8, 24)
+    elif case == "int_group_big":
+        f = ss24.make_format("int", 8, 256)
+    elif case == "ws_null":
+        kw["ws"] = None
+    elif case == "ws_small":
+        kw["ws_bytes"] = 64
+    elif case == "ws_misaligned":
+        kw["ws"] = ALIGNED + 16
+    elif case == "null_values":
+        kw["out"] = outs(values=0)
+    elif case == "null_meta":
+        kw["out"] = outs(meta=0)
+    elif case == "null_scales":
+        kw["out"] = outs(scales=0)
+    elif case == "null_tscale":
+        kw["out"] = outs(tscale=0)
+    elif case == "wanda_no_norms":
+        kw["score"] = ss24.WANDA
+    elif case == "wanda_misaligned_norms":
+        kw["score"] = ss24.WANDA
+        kw["norms"] = MISALIGNED
+    elif case == "bad_score":
+        kw["score"] = 5
+    elif case == "misaligned_values":
+        kw["out"] = outs(values=MISALIGNED)
+    assert fused(o, f, **kw) == expected
+
+
+def test_other_entry_points_validate():
+    L = ss24.lib()
+    o = op()
+    out = outs()
+    wsb = _ws_bytes()
+    assert L.ss24_quantize_fp8(ctypes.byref(op(k=12, ld=16)), None, ctypes.byref(out), None, ALIGNED, wsb, None) == 2
+    assert L.ss24_quantize_int(ctypes.byref(o), ss24.make_format("fp8"), ctypes.byref(out), None, ALIGNED, wsb,
+                               None) == 5
+    assert L.ss24_quantize_nvfp4(ctypes.byref(op(k=8, ld=8)), None, ctypes.byref(out), None, ALIGNED, wsb,
+                                 None) == 2
+    assert L.ss24_quantize_mxfp4(ctypes.byref(op(k=16, ld=16)), ctypes.byref(out), None, ALIGNED, wsb, None) == 2
+    assert L.ss24_prune24_compress(ctypes.byref(o), ss24.MAG, None, ALIGNED, None, None, ALIGNED, wsb, None) == 1
+    assert L.ss24_prune48_pairwise_quant_fused(ctypes.byref(op(k=24, ld=24)), ss24.MAG, None,
+                                               ss24.make_format("none"), None, ctypes.byref(out), None, ALIGNED,
+                                               wsb, None) == 2
+    assert L.ss24_error_energy(ctypes.byref(o), ss24.DENSE, ss24.MAG, None, ss24.make_format("none"),
+                               ss24.make_format("int", 5), None, None, ALIGNED, ALIGNED, wsb, None) == 8
+    assert L.ss24_error_energy(ctypes.byref(o), ss24.SPARSE_24, ss24.MAG, None, ss24.make_format("none"),
+                               ss24.make_format("none"), None, None, ALIGNED, ALIGNED, wsb, None) == 5
+    assert L.ss24_error_energy(ctypes.byref(o), ss24.SPARSE_24, ss24.MAG, None, ss24.make_format("none"),
+                               ss24.make_format("int", 5), None, None, None, ALIGNED, wsb, None) == 1
+    assert L.ss24_amax(ctypes.byref(o), ss24.SPARSE_24, ss24.MAG, None, None, ALIGNED, wsb, None) == 1
+    assert L.ss24_predicted_ratio(None, ALIGNED, ALIGNED, None) == 1
+    assert L.ss24_encode_e4m3(None, None, 5, None) == 1
+    assert L.ss24_decode_e2m1(ALIGNED, ALIGNED, -1, None) == 2
+    assert L.ss24_workspace_init(None, wsb, None) == 6
+    assert L.ss24_workspace_error(None, None, None) == 1

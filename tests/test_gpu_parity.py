@@ -1,0 +1,341 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs. Codes, scales, metadata and kept values must match bit for
+bit; energies to 1e-6 relative (the bound the library states for its binary32
+per-element terms summed in binary64)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from semi_structured_sparsity_online_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+RTOL = 1e-6
+
+
+@pytest.fixture(scope="module")
+def ss():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from semi_structured_sparsity_online_b200 import ss24
+    ss24.lib()
+    return ss24
+
+
+@pytest.fixture(scope="module")
+def ws(ss):
+    return ss.Workspace()
+
+
+def to_dev(a):
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(a).cuda()
+
+
+def to_np(t):
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).cpu().numpy().view(np.uint16)
+    return t.cpu().numpy()
+
+
+def bits_equal(a, b):
+    a = np.ascontiguousarray(a)
+    b = np.ascontiguousarray(b)
+    if a.dtype == np.float32:
+        return a.shape == b.shape and np.array_equal(a.view(np.uint32), b.view(np.uint32))
+    return a.shape == b.shape and np.array_equal(a, b)
+
+
+def assert_same(got, ref, what):
+    if not bits_equal(got, ref):
+        bad = np.argwhere(np.asarray(got) != np.asarray(ref))
+        raise AssertionError(f"{what}: {len(bad)} mismatches, first at {bad[:3].tolist()}: "
+                             f"gpu {np.asarray(got)[tuple(bad[0])] if len(bad) else None} "
+                             f"oracle {np.asarray(ref)[tuple(bad[0])] if len(bad) else None}")
+
+
+def assert_energy(got, ref, fields=(0, 1, 2, 3), atol=0.0):
+    g = got.cpu().numpy()
+    for f in fields:
+        assert abs(g[f] - ref[f]) <= RTOL * abs(ref[f]) + atol, (f, g[f], ref[f])
+
+
+def compare(ss, ws, xh, *, pattern, fmt, bits=8, group=0, pack4=False, score="mag", norms=None,
+            tensor_scale=None, k=None):
+    """Run both sides on the host array xh ([rows][ld]; k <= ld) and compare."""
+    x = to_dev(xh)
+    if k is not None and k != xh.shape[1]:
+        xd = x[:, :k]
+    else:
+        xd = x
+    nd = to_dev(norms) if norms is not None else None
+    sd = torch.tensor([tensor_scale], dtype=torch.float32, device="cuda") if tensor_scale is not None else None
+    opat = {0: oracle.DENSE, 24: oracle.SPARSE_24, 48: oracle.SPARSE_48}[pattern]
+    out = ss.run(xd, pattern=pattern, fmt=fmt, bits=bits, group=group, pack4=pack4, score=score, col_norms=nd,
+                 tensor_scale=sd, ws=ws)
+    torch.cuda.synchronize()
+    ref = oracle.run(xh, pattern=opat, fmt=fmt, bits=bits, group=group, pack4=pack4,
+                     score=oracle.WANDA if score == "wanda" else oracle.MAG, norms=norms,
+                     tensor_scale=tensor_scale, k=k)
+    for key in ("values", "scales", "meta", "tensor_scale"):
+        if key in ref:
+            assert_same(to_np(out[key]), ref[key], key)
+    assert_energy(out["energy"], ref["energy"], atol=1e-30)
+    assert ws.error() == 0
+    return out, ref
+
+
+# --------------------------------------------------------------------------
+# converters: the kernels' own cvt-based encoders against the oracle's
+# --------------------------------------------------------------------------
+
+def probe_values(n_random=1 << 22, seed=0):
+    rng = np.random.default_rng(seed)
+    allbf = synth.bf16_to_f32(np.arange(65536, dtype=np.uint16))
+    rnd = rng.integers(0, 2 ** 32, size=n_random, dtype=np.uint64).astype(np.uint32).view(np.float32)
+    small = (rng.standard_normal(n_random) * 4).astype(np.float32)
+    v = np.concatenate([allbf, rnd, small])
+    return v[np.isfinite(v)].astype(np.float32)
+
+
+def oracle_encode_vec(fn, v):
+    return np.fromiter((fn(float(t)) for t in v), dtype=np.uint8, count=len(v))
+
+
+def test_e4m3_encoder_matches_oracle(ss):
+    rng = np.random.default_rng(2)
+    allbf = synth.bf16_to_f32(np.arange(65536, dtype=np.uint16))
+    rnd = probe_values(n_random=1 << 18, seed=2)
+    # midpoints between neighbouring E4M3 values and one ulp either side
+    dec = np.array([oracle.e4m3_decode(c) for c in range(127)], dtype=np.float64)
+    mids = ((dec[1:] + dec[:-1]) / 2).astype(np.float32)
+    ext = np.concatenate([mids, np.nextafter(mids, np.float32(0)), np.nextafter(mids, np.float32(1e9))])
+    v = np.concatenate([allbf, ext, -ext, rng.choice(rnd, 300000)]).astype(np.float32)
+    v = v[np.isfinite(v)]
+    got = ss.encode_e4m3(torch.from_numpy(v).cuda()).cpu().numpy()
+    ref = oracle_encode_vec(oracle.e4m3_encode, v)
+    assert_same(got, ref, "e4m3 encode")
+    codes = np.arange(256, dtype=np.uint8)
+    d = ss.decode_e4m3(torch.from_numpy(codes).cuda()).cpu().numpy()
+    for c in range(256):
+        r = oracle.e4m3_decode(c)
+        if np.isnan(r):
+            assert np.isnan(d[c])
+        else:
+            assert d[c] == r and np.signbit(d[c]) == np.signbit(r)
+
+
+def test_e2m1_encoder_matches_oracle(ss):
+    v = probe_values(n_random=1 << 18, seed=1)
+    grid = np.arange(-8, 8, 0.03125, dtype=np.float32)
+    v = np.concatenate([v, grid, np.nextafter(grid, np.float32(0)),
+                        np.nextafter(grid, np.float32(100))]).astype(np.float32)
+    got = ss.encode_e2m1(torch.from_numpy(v).cuda()).cpu().numpy()
+    ref = oracle_encode_vec(oracle.e2m1_encode, v)
+    assert_same(got, ref, "e2m1 encode")
+    codes = np.arange(16, dtype=np.uint8)
+    d = ss.decode_e2m1(torch.from_numpy(codes).cuda()).cpu().numpy()
+    for c in range(16):
+        assert d[c] == oracle.e2m1_decode(c) and np.signbit(d[c]) == np.signbit(oracle.e2m1_decode(c))
+
+
+# --------------------------------------------------------------------------
+# the pass: every pattern x score x format, ragged shapes
+# --------------------------------------------------------------------------
+
+FORMATS = [("none", 8, 0, False), ("fp8", 8, 0, False), ("int", 8, 64, False), ("int", 4, 32, True),
+           ("int", 12, 128, False), ("int", 3, 16, False), ("nvfp4", 4, 0, False), ("mxfp4", 4, 0, False)]
+
+
+@pytest.mark.parametrize("pattern", [24, 48])
+@pytest.mark.parametrize("score", ["mag", "wanda"])
+@pytest.mark.parametrize("fmt,bits,group,pack4", FORMATS)
+def test_sparse_pass_bf16(ss, ws, pattern, score, fmt, bits, group, pack4):
+    rows, k = 100, 512     # 4 row tiles (ragged), 2 column tiles
+    xh = synth.sweep_operand(rows, k, seed=3 + pattern)
+    norms = np.exp(np.random.default_rng(5).standard_normal(k)).astype(np.float32) if score == "wanda" else None
+    compare(ss, ws, xh, pattern=pattern, fmt=fmt, bits=bits, group=group, pack4=pack4, score=score, norms=norms)
+
+
+@pytest.mark.parametrize("fmt,bits,group,pack4", FORMATS)
+def test_sparse_pass_fp32(ss, ws, fmt, bits, group, pack4):
+    xh = synth.gaussian_f32(37, 1024, seed=0)
+    compare(ss, ws, xh, pattern=24, fmt=fmt, bits=bits, group=group, pack4=pack4)
+
+
+@pytest.mark.parametrize("fmt,bits,group,pack4", [f for f in FORMATS if f[0] != "none"] + [("int", 8, 256, False)])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_dense_pass(ss, ws, fmt, bits, group, pack4, dtype):
+    xh = synth.sweep_operand(70, 768, seed=9) if dtype == "bf16" else synth.gaussian_f32(70, 768, seed=9)
+    compare(ss, ws, xh, pattern=0, fmt=fmt, bits=bits, group=group, pack4=pack4)
+
+
+@pytest.mark.parametrize("pattern", [0, 24, 48])
+@pytest.mark.parametrize("k", [128, 256, 1024, 4096, 96, 400])
+def test_int_one_scale_per_row(ss, ws, pattern, k):
+    """Group 0: one scale per row; tile mode when k is a power of two <= 256,
+    row mode (two sweeps over whole rows) otherwise."""
+    if pattern == 48 and k % 16:
+        pytest.skip("4:8 needs k % 16 == 0")
+    xh, _ = synth.linear_input(45, k, seed=2, n_outlier=min(8, k // 16))
+    compare(ss, ws, xh, pattern=pattern, fmt="int", bits=8, group=0)
+    compare(ss, ws, xh, pattern=pattern, fmt="int", bits=4, group=0, pack4=True)
+
+
+@pytest.mark.parametrize("k", [8, 16, 24, 40, 96, 136, 264])
+@pytest.mark.parametrize("pattern", [0, 24])
+def test_small_and_ragged_k(ss, ws, pattern, k):
+    """k below the tile width (zero-filled box) and k with a partial last tile."""
+    xh = synth.ties_and_specials(33, k, seed=k) if k >= 12 else synth.gaussian_bf16(33, k, seed=k)
+    fmt = "fp8" if pattern == 24 else "int"
+    compare(ss, ws, xh, pattern=pattern, fmt=fmt, bits=8, group=8 if pattern == 0 else 4)
+    if pattern == 24:
+        compare(ss, ws, xh, pattern=24, fmt="none")
+
+
+@pytest.mark.parametrize("rows", [1, 2, 31, 33, 257])
+def test_ragged_rows(ss, ws, rows):
+    xh = synth.gaussian_bf16(rows, 64, seed=rows)
+    compare(ss, ws, xh, pattern=24, fmt="nvfp4")
+    compare(ss, ws, xh, pattern=48, fmt="mxfp4")
+
+
+def test_ties_specials_every_format(ss, ws):
+    xh = synth.ties_and_specials(64, 256, seed=4)
+    for fmt, bits, group, pack4 in FORMATS:
+        compare(ss, ws, xh, pattern=24, fmt=fmt, bits=bits, group=group, pack4=pack4)
+        compare(ss, ws, xh, pattern=48, fmt=fmt, bits=bits, group=group, pack4=pack4)
+
+
+def test_row_stride_larger_than_k(ss, ws):
+    full = synth.sweep_operand(50, 640, seed=12)
+    compare(ss, ws, full, pattern=24, fmt="nvfp4", k=512)
+    compare(ss, ws, full, pattern=0, fmt="int", bits=8, group=0, k=512)
+
+
+def test_given_tensor_scale_and_saturation(ss, ws):
+    xh = synth.sweep_operand(64, 512, seed=13)
+    # a scale 16x too small saturates the largest values to +-448 / +-6
+    s_fp8 = oracle.tensor_scale(xh, "fp8") / 16.0
+    compare(ss, ws, xh, pattern=24, fmt="fp8", tensor_scale=s_fp8)
+    compare(ss, ws, xh, pattern=0, fmt="fp8", tensor_scale=s_fp8)
+    s_nv = oracle.tensor_scale(xh, "nvfp4") / 1e4
+    compare(ss, ws, xh, pattern=24, fmt="nvfp4", tensor_scale=s_nv)
+    compare(ss, ws, xh, pattern=0, fmt="nvfp4", tensor_scale=0.0)
+
+
+def test_all_zero_operand(ss, ws):
+    xh = np.zeros((40, 256), dtype=np.uint16)
+    for fmt, bits, group, pack4 in FORMATS:
+        compare(ss, ws, xh, pattern=24, fmt=fmt, bits=bits, group=group, pack4=pack4)
+    compare(ss, ws, xh, pattern=0, fmt="nvfp4")
+    compare(ss, ws, xh, pattern=0, fmt="mxfp4")
+
+
+def test_empty_operand(ss, ws):
+    x = torch.zeros((0, 64), dtype=torch.bfloat16, device="cuda")
+    out = ss.run(x, pattern=24, fmt="fp8", ws=ws)
+    torch.cuda.synchronize()
+    assert out["energy"].abs().sum().item() == 0.0
+    assert out["tensor_scale"].item() == 0.0
+
+
+def test_amax_and_error_energy_and_ratio(ss, ws):
+    w, norms = synth.linear_weight(96, 512, seed=2)
+    wd, nd = to_dev(w), to_dev(norms)
+    for score, nrm in (("mag", None), ("wanda", norms)):
+        sc = oracle.WANDA if score == "wanda" else oracle.MAG
+        a = ss.amax(wd, pattern=24, score=score, col_norms=nd if nrm is not None else None, ws=ws)
+        assert a.item() == oracle.amax(w, score=sc, norms=nrm)
+        for sfmt, dfmt in [(("int", 8, 128), ("int", 5, 128)), (("fp8",), ("nvfp4",)), (("none",), ("mxfp4",)),
+                           (("nvfp4",), ("fp8",)), (("int", 4, 64, True), ("int", 3, 64))]:
+            e = ss.error_energy(wd, pattern=24, sparse_fmt=sfmt, dense_fmt=dfmt, score=score,
+                                col_norms=nd if nrm is not None else None, ws=ws)
+            sp = oracle.run(w, fmt=sfmt[0], bits=(sfmt[1] if len(sfmt) > 1 else 8),
+                            group=(sfmt[2] if len(sfmt) > 2 else 0), pack4=(len(sfmt) > 3 and sfmt[3]),
+                            score=sc, norms=nrm)["energy"]
+            de = oracle.run(w, pattern=oracle.DENSE, fmt=dfmt[0], bits=(dfmt[1] if len(dfmt) > 1 else 8),
+                            group=(dfmt[2] if len(dfmt) > 2 else 0))["energy"]
+            ref = np.array([sp[0], sp[1], sp[2], de[3]])
+            assert_energy(e, ref)
+            r = ss.predicted_ratio(e, e)
+            rr = oracle.ratio(ref, ref)
+            np.testing.assert_allclose(r.cpu().numpy(), rr, rtol=2e-6)
+    assert ws.error() == 0
+
+
+def test_repeated_calls_are_deterministic(ss, ws):
+    xh, _ = synth.linear_input(300, 1024, seed=1)
+    x = to_dev(xh)
+    outs = [ss.run(x, pattern=24, fmt="fp8", ws=ws) for _ in range(3)]
+    torch.cuda.synchronize()
+    for o in outs[1:]:
+        assert torch.equal(o["values"], outs[0]["values"])
+        assert torch.equal(o["energy"], outs[0]["energy"])
+
+
+# --------------------------------------------------------------------------
+# full-size configurations: sampled rows against the oracle, energies by
+# properties that hold at any size
+# --------------------------------------------------------------------------
+
+def sampled_check(ss, ws, xh, *, pattern, fmt, bits=8, group=0, score="mag", norms=None, n_rows=48, seed=0):
+    x = to_dev(xh)
+    nd = to_dev(norms) if norms is not None else None
+    out = ss.run(x, pattern=pattern, fmt=fmt, bits=bits, group=group, score=score, col_norms=nd, ws=ws)
+    torch.cuda.synchronize()
+    sc = oracle.WANDA if score == "wanda" else oracle.MAG
+    opat = {0: oracle.DENSE, 24: oracle.SPARSE_24, 48: oracle.SPARSE_48}[pattern]
+    ts = None
+    if fmt in ("fp8", "nvfp4"):
+        ts = oracle.tensor_scale(xh, fmt, pattern=opat, score=sc, norms=norms)
+        assert out["tensor_scale"].item() == np.float32(ts)
+    rng = np.random.default_rng(seed)
+    rows = np.unique(np.concatenate([[0, xh.shape[0] - 1], rng.integers(0, xh.shape[0], n_rows)]))
+    ref = oracle.run(xh[rows], pattern=opat, fmt=fmt, bits=bits, group=group, score=sc, norms=norms,
+                     tensor_scale=ts)
+    for key in ("values", "scales", "meta"):
+        if key in ref:
+            assert_same(to_np(out[key][torch.from_numpy(rows).cuda()]), ref[key], key)
+    # E_total of the whole tensor, summed independently in binary64
+    xf = synth.bf16_to_f32(xh).astype(np.float64) if xh.dtype == np.uint16 else xh.astype(np.float64)
+    e = out["energy"].cpu().numpy()
+    et = float(np.einsum("ij,ij->", xf, xf))
+    assert abs(e[0] - et) <= RTOL * et
+    assert ws.error() == 0
+    return e
+
+
+def test_full_linear_input_fp8_and_int8_per_row(ss, ws):
+    xh, _ = synth.linear_input(4096, 4096, seed=1)
+    e = sampled_check(ss, ws, xh, pattern=24, fmt="fp8")
+    assert 0.0 < e[1] / e[0] < 0.5
+    sampled_check(ss, ws, xh, pattern=0, fmt="fp8")
+    sampled_check(ss, ws, xh, pattern=0, fmt="int", bits=8, group=0)
+
+
+def test_full_weight_wanda_int(ss, ws):
+    w, norms = synth.linear_weight(14336, 4096, seed=2)
+    for m in (2, 4, 8):
+        sampled_check(ss, ws, w, pattern=24, fmt="int", bits=2 * m, group=128, score="wanda", norms=norms,
+                      n_rows=16, seed=m)
+        sampled_check(ss, ws, w, pattern=0, fmt="int", bits=m + 1, group=128, n_rows=16, seed=m)
+
+
+def test_full_attention_operands(ss, ws):
+    q = synth.attention_qkv(seed=4)
+    sampled_check(ss, ws, q, pattern=24, fmt="fp8")
+    sampled_check(ss, ws, q, pattern=0, fmt="nvfp4")
+    sampled_check(ss, ws, q, pattern=0, fmt="mxfp4")
+    p = synth.attention_probs(seed=7)
+    sampled_check(ss, ws, p, pattern=24, fmt="fp8", n_rows=16)
+
+
+@pytest.mark.parametrize("tokens,k", [(2048, 4096), (16384, 14336)])
+def test_full_sweep_nvfp4(ss, ws, tokens, k):
+    xh = synth.sweep_operand(tokens, k, seed=8)
+    sampled_check(ss, ws, xh, pattern=24, fmt="nvfp4", n_rows=12)
+    sampled_check(ss, ws, xh, pattern=48, fmt="nvfp4", n_rows=12)
+    sampled_check(ss, ws, xh, pattern=24, fmt="none", n_rows=12)
