@@ -1,0 +1,434 @@
+"""Benchmark of the online 2:4 prune + compress + quantize + error-energy path.
+
+Workload (one step): a batch of B = 8 linear-layer inputs X, each bf16
+4096 x 4096, Student-t (nu = 4, unit variance) with 8 outlier channels x50.
+A step runs every row of the hot path once over the batch, pass by pass, each
+pass visiting all 8 operands before the next pass starts (so each pass reads
+its operand from HBM: the batch is 256 MiB, twice the L2):
+  1. per-tensor FP8 scale of each X (amax pass)            ss24_tensor_scale
+  2. fused 2:4 magnitude prune + compress + FP8 E4M3 of the
+     kept values + energies (E_total, E_prune, E_q)        ss24_prune24_quant_fused
+  3. dense FP8 E4M3 partner (same scale) + energy          ss24_quantize_fp8
+  4. dense INT8, one scale per row, partner + energy       ss24_quantize_int
+  5. predicted R against both partners                     ss24_predicted_ratio x2
+The step is captured as one CUDA graph per pass; CUDA events between the pass
+graphs give per-kernel durations inside the timed region.
+
+Prints ONE JSON line (rank 0). ``--impl reference`` times the CPU oracle on a
+bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "fused 2:4 prune+compress+quant HBM GB/s and % of peak/memcpy; Gelem/s"
+WORKLOAD = ("linear-input X bf16 4096x4096 (Student-t nu=4 /sqrt2, 8 outlier channels x50), batch of 8 per step: "
+            "FP8 tensor scale, fused 2:4 magnitude prune+compress+FP8 E4M3 kept values, dense FP8 and dense INT8 "
+            "per-row partners, energies, predicted R")
+M = K = 4096
+BATCH = 8
+
+
+def algorithmic_bytes(m=M, k=K):
+    """Bytes each pass must move per operand (bf16 in; see the DESIGN notes)."""
+    n = m * k
+    return {
+        "tensor_scale": 2 * n,                         # read X
+        "fused_24_fp8": 2 * n + n // 2 + n // 8,       # read X; write FP8 codes (k/2) + metadata (k/8)
+        "dense_fp8": 2 * n + n,                        # read X; write FP8 codes
+        "dense_int8_row": 2 * n + n + 4 * m,           # read X; write INT8 codes + one fp32 scale per row
+        "ratio": 0,
+    }
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML, read-only)
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {0x2: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle",
+               0x4: "applications_clocks_setting", 0x10: "sync_boost", 0x100: "display_clock_setting"}
+
+    def __init__(self, index):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.02)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.ok:
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# the CUDA path
+# ---------------------------------------------------------------------------
+
+def make_batch(seed0=1):
+    from semi_structured_sparsity_online_b200 import synth
+    xs = []
+    for b in range(BATCH):
+        x, _ = synth.linear_input(M, K, seed=seed0 + b)
+        xs.append(x)
+    return xs
+
+
+class Step:
+    """Device buffers and per-pass CUDA graphs for one step over the batch."""
+
+    def __init__(self, ss, xs_dev, stream):
+        import torch
+        self.ss, self.torch, self.stream = ss, torch, stream
+        self.xs = xs_dev
+        dev = xs_dev[0].device
+        self.ws = ss.Workspace(dev, stream)
+        u8, f32, f64 = torch.uint8, torch.float32, torch.float64
+        self.scale = [torch.empty(1, dtype=f32, device=dev) for _ in range(BATCH)]
+        self.sp = [ss._alloc_outputs(M, K, ss.SPARSE_24, ss.make_format("fp8"), torch.bfloat16, dev)
+                   for _ in range(BATCH)]
+        self.d8 = [ss._alloc_outputs(M, K, ss.DENSE, ss.make_format("fp8"), torch.bfloat16, dev)
+                   for _ in range(BATCH)]
+        self.di = [ss._alloc_outputs(M, K, ss.DENSE, ss.make_format("int", 8, 0), torch.bfloat16, dev)
+                   for _ in range(BATCH)]
+        self.e = torch.zeros((BATCH, 3, 4), dtype=f64, device=dev)    # sparse, dense fp8, dense int8
+        self.r = torch.zeros((BATCH, 2, 4), dtype=f64, device=dev)    # R vs fp8, R vs int8
+        self.passes = ["tensor_scale", "fused_24_fp8", "dense_fp8", "dense_int8_row", "ratio"]
+        self.launches_per_step = BATCH * (1 + 1 + 1 + 1 + 2)
+
+    def run_pass(self, name):
+        ss, s = self.ss, self.stream
+        for b in range(BATCH):
+            x = self.xs[b]
+            if name == "tensor_scale":
+                ss.tensor_scale(x, "fp8", ss.SPARSE_24, ws=self.ws, stream=s, out=self.scale[b])
+            elif name == "fused_24_fp8":
+                ss.run(x, pattern=ss.SPARSE_24, fmt="fp8", tensor_scale=self.scale[b], energy=self.e[b, 0],
+                       ws=self.ws, stream=s, out=self.sp[b])
+            elif name == "dense_fp8":
+                # for the magnitude score the kept amax equals the amax of all values,
+                # so the 2:4 scale is the dense FP8 scale too
+                ss.run(x, pattern=ss.DENSE, fmt="fp8", tensor_scale=self.scale[b], energy=self.e[b, 1],
+                       ws=self.ws, stream=s, out=self.d8[b])
+            elif name == "dense_int8_row":
+                ss.run(x, pattern=ss.DENSE, fmt="int", bits=8, group=0, energy=self.e[b, 2], ws=self.ws,
+                       stream=s, out=self.di[b])
+            elif name == "ratio":
+                ss.predicted_ratio(self.e[b, 0], self.e[b, 1], out=self.r[b, 0], stream=s)
+                ss.predicted_ratio(self.e[b, 0], self.e[b, 2], out=self.r[b, 1], stream=s)
+
+    def run_eager(self):
+        for p in self.passes:
+            self.run_pass(p)
+
+    def capture(self):
+        torch = self.torch
+        self.graphs = {}
+        for p in self.passes:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=self.stream):
+                self.run_pass(p)
+            self.graphs[p] = g
+
+    def replay(self, events=None):
+        for i, p in enumerate(self.passes):
+            self.graphs[p].replay()
+            if events is not None:
+                events[i + 1].record(self.stream)
+
+
+def memcpy_gbps(torch, dev, nbytes=1 << 30, iters=10):
+    a = torch.empty(nbytes // 2, dtype=torch.bfloat16, device=dev)
+    b = torch.empty_like(a)
+    b.copy_(a)
+    torch.cuda.synchronize()
+    best = None
+    for _ in range(iters):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        b.copy_(a)
+        e.record()
+        e.synchronize()
+        t = s.elapsed_time(e) / 1e3
+        best = t if best is None else min(best, t)
+    del a, b
+    return 2 * nbytes / best / 1e9
+
+
+def cpu_baseline_sample(xs_host, rows=96):
+    """The oracle, as it stands, on a bounded sample: the first `rows` rows of
+    every operand of the batch through the same passes (each sample treated as
+    its own operand). Returns (GB/s of algorithmic bytes, seconds, cores)."""
+    import oracle
+    t0 = time.perf_counter()
+    for x in xs_host:
+        xs = np.ascontiguousarray(x[:rows])
+        ts = oracle.tensor_scale(xs, "fp8")
+        sp = oracle.run(xs, pattern=oracle.SPARSE_24, fmt="fp8", tensor_scale=ts)["energy"]
+        d8 = oracle.run(xs, pattern=oracle.DENSE, fmt="fp8", tensor_scale=ts)["energy"]
+        di = oracle.run(xs, pattern=oracle.DENSE, fmt="int", bits=8, group=0)["energy"]
+        oracle.ratio(sp, d8)
+        oracle.ratio(sp, di)
+    dt = time.perf_counter() - t0
+    nbytes = sum(algorithmic_bytes(rows, K).values()) * len(xs_host)
+    return nbytes / dt / 1e9, dt, 1
+
+
+def run_cuda(args):
+    import torch
+    import torch.distributed as dist
+
+    from semi_structured_sparsity_online_b200 import ss24 as ss
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    ss.lib()
+    stream = torch.cuda.Stream(device=dev)
+
+    # each rank draws its own batch (independent problems: weak scaling)
+    xs_host = make_batch(seed0=1 + 100 * rank)
+    xs_pinned = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in xs_host]
+    xs_dev = [torch.empty((M, K), dtype=torch.bfloat16, device=dev) for _ in range(BATCH)]
+    with torch.cuda.stream(stream):
+        for d, h in zip(xs_dev, xs_pinned):
+            d.copy_(h, non_blocking=True)
+    stream.synchronize()
+
+    step = Step(ss, xs_dev, stream)
+    with torch.cuda.stream(stream):
+        step.run_eager()          # first launches: kernel attributes, tensor-map entry point
+    stream.synchronize()
+    step.capture()
+    with torch.cuda.stream(stream):       # graph replays launch on the current stream
+        for _ in range(args.warmup):
+            step.replay()
+    stream.synchronize()
+    if step.ws.error(stream) != 0:
+        raise RuntimeError("a kernel wait timed out during warm-up")
+
+    # ---- timed region ----
+    n_ev = len(step.passes) + 1
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dev.index)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with clocks, torch.cuda.stream(stream):
+        start.record(stream)
+        for i in range(args.steps):
+            evs[i][0].record(stream)
+            step.replay(evs[i])
+        end.record(stream)
+        end.synchronize()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    elapsed_s = start.elapsed_time(end) / 1e3
+    per_pass = {p: 0.0 for p in step.passes}
+    for i in range(args.steps):
+        for j, p in enumerate(step.passes):
+            per_pass[p] += evs[i][j].elapsed_time(evs[i][j + 1]) / 1e3
+    if world > 1:
+        t = torch.tensor([elapsed_s], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_s = t.item()
+    err = step.ws.error(stream)
+    if err != 0:
+        raise RuntimeError(f"a kernel wait timed out (code {err})")
+
+    ab = algorithmic_bytes()
+    step_bytes = BATCH * sum(ab.values())
+    ms_per_step = elapsed_s / args.steps * 1e3
+    value = world * step_bytes * args.steps / elapsed_s / 1e9
+    elems = world * BATCH * M * K * args.steps / elapsed_s / 1e9
+
+    # ---- end to end through the public API with host buffers ----
+    e2e_steps = max(3, min(20, args.steps // 10))
+    r_host = torch.empty((BATCH, 2, 4), dtype=torch.float64).pin_memory()
+    h2d = BATCH * M * K * 2
+    d2h = r_host.numel() * 8
+    with torch.cuda.stream(stream):
+        for d, h in zip(xs_dev, xs_pinned):     # warm-up of the copy path
+            d.copy_(h, non_blocking=True)
+        step.replay()
+        r_host.copy_(step.r, non_blocking=True)
+    stream.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            for d, h in zip(xs_dev, xs_pinned):
+                d.copy_(h, non_blocking=True)
+            step.replay()
+            r_host.copy_(step.r, non_blocking=True)
+        e1.record(stream)
+    e1.synchronize()
+    e2e_s = e0.elapsed_time(e1) / 1e3
+    if world > 1:
+        t = torch.tensor([e2e_s], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_s = t.item()
+    e2e_value = world * step_bytes * e2e_steps / e2e_s / 1e9
+
+    peak, peak_kind = load_peaks()
+    mc = memcpy_gbps(torch, dev)
+
+    # dominant kernel: the pass with the largest device time
+    dom = max((p for p in step.passes if ab[p] > 0), key=lambda p: per_pass[p])
+    dom_us = per_pass[dom] / (args.steps * BATCH) * 1e6
+    achieved = ab[dom] / (dom_us * 1e-6) / 1e9
+    passes = {}
+    for p in step.passes:
+        us = per_pass[p] / (args.steps * BATCH) * 1e6
+        passes[p] = {"us_per_launch": round(us, 3),
+                     "gbps": round(ab[p] / (us * 1e-6) / 1e9, 1) if ab[p] else None,
+                     "bytes_per_launch": ab[p]}
+    traffic = None
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            traffic = json.load(f).get(dom)
+    except Exception:
+        pass
+
+    r = step.r.cpu().numpy()
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "operands_per_step": BATCH, "m": M, "k": K, "input_dtype": "bf16",
+                   "l2": "inputs larger than L2: 8 x 32 MiB per step; each pass visits all 8 operands before "
+                         "the next pass", "parallelism": f"dp{world} (independent batches)"},
+        "gelem_per_s": round(elems, 2),
+        "frac_of_peak": round(value / world / peak, 4),
+        "memcpy_gbps": round(mc, 1),
+        "frac_of_memcpy": round(value / world / mc, 4),
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peak,
+                     "peak_source": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": traffic, "algorithmic_bytes_per_launch": ab[dom]},
+        "passes": passes,
+        "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": step.launches_per_step * args.steps,
+        "clocks": clocks.summary(),
+        "predicted_r": {"vs_dense_fp8": round(float(r[0, 0, 3]), 4), "vs_dense_int8_row": round(float(r[0, 1, 3]), 4),
+                        "energy_loss_24": round(float(r[0, 0, 0]), 5)},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbps, dt, cores = cpu_baseline_sample(xs_host, rows=args.cpu_rows)
+        result["cpu_baseline"] = {"value": round(gbps, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                                  "sample": f"first {args.cpu_rows} rows of each of the 8 operands, all passes "
+                                            f"({dt:.1f} s of CPU work)"}
+    if world > 1:
+        del step
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result))
+
+
+def run_reference(args):
+    """The oracle on the host cores, per step a bounded sample of the workload."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    xs_host = make_batch()
+    rows = args.ref_rows
+    for _ in range(args.warmup):
+        cpu_baseline_sample(xs_host[:1], rows=rows)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        cpu_baseline_sample(xs_host[:1], rows=rows)
+    dt = time.perf_counter() - t0
+    nbytes = sum(algorithmic_bytes(rows, K).values()) * args.steps
+    value = nbytes / dt / 1e9
+    sample = f"per step: first {rows} rows of one 4096x4096 operand through all passes"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample": sample},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ss24", "reference"], default="ss24")
+    ap.add_argument("--cpu-rows", type=int, default=96)
+    ap.add_argument("--ref-rows", type=int, default=8, help="rows of one operand per reference step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_cuda(args)
+
+
+if __name__ == "__main__":
+    main()

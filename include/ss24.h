@@ -263,6 +263,17 @@ ss24_status ss24_amax(const ss24_operand *x, ss24_pattern pattern, ss24_score sc
                       const float *col_norms, float *amax_out, void *ws, size_t ws_bytes,
                       ss24_stream stream);
 
+/* The per-tensor scale a pass derives when it is given none (§3): FP8
+ * s = amax / 448, NVFP4 s_t = amax / 2688, the amax taken over the values the
+ * pass would quantize (kept values for a sparse pattern). One read-only pass;
+ * writes one fp32 to the device pointer scale_out. Computing the scale ahead
+ * of the quantizing pass and passing it as tensor_scale_in gives the same
+ * codes as letting that pass compute it. kind: SS24_FMT_FP8_E4M3 or
+ * SS24_FMT_NVFP4 (anything else: SS24_ERR_FORMAT). */
+ss24_status ss24_tensor_scale(const ss24_operand *x, ss24_pattern pattern, ss24_score score,
+                              const float *col_norms, int32_t kind, float *scale_out, void *ws,
+                              size_t ws_bytes, ss24_stream stream);
+
 /* Derived quantities (§4) from a sparse-side energy record (e_total, e_prune,
  * e_quant) and a dense-side record (e_quant_dense); both device pointers, and
  * they may be the same record (as ss24_error_energy writes it). One-thread

@@ -321,7 +321,7 @@ const void *tile_kernel(int dtype, int pattern, int score, int fmt)
 // For the magnitude score the kept amax equals the amax of all values, so the
 // cheaper dense form is used.
 cudaError_t run_amax(const ss24_operand *x, int pattern, int score, const float *norms, void *ws,
-                     cudaStream_t stream)
+                     cudaStream_t stream, float *scale_out = nullptr, float divisor = 1.0f)
 {
     const int pat = score == SS24_SCORE_MAG ? SS24_DENSE : pattern;
     const Geometry g = tile_geometry(x);
@@ -330,6 +330,8 @@ cudaError_t run_amax(const ss24_operand *x, int pattern, int score, const float 
         return cudaErrorInvalidValue;
     PassParams p = base_params(x, g, ws, nullptr);
     p.norms = norms;
+    p.q.scale_out = scale_out;
+    p.q.divisor = divisor;
     return launch(tile_kernel(x->dtype, pat, score, kAmax), kSmemBytes, g.n_tiles, map, p, stream);
 }
 
@@ -589,6 +591,31 @@ ss24_status ss24_amax(const ss24_operand *x, ss24_pattern pattern, ss24_score sc
         return SS24_ERR_CUDA;
     const float *red = reinterpret_cast<const float *>(static_cast<uint8_t *>(ws) + kWsAmaxReducedOff);
     return cuda_status(cudaMemcpyAsync(amax_out, red, sizeof(float), cudaMemcpyDeviceToDevice, s));
+}
+
+ss24_status ss24_tensor_scale(const ss24_operand *x, ss24_pattern pattern, ss24_score score, const float *col_norms,
+                              int32_t kind, float *scale_out, void *ws, size_t ws_bytes, ss24_stream stream)
+{
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    ss24_status st = check_operand(x);
+    if (st != SS24_OK)
+        return st;
+    if ((st = check_pattern_k(pattern, x->k)) != SS24_OK)
+        return st;
+    if (score != SS24_SCORE_MAG && score != SS24_SCORE_WANDA)
+        return SS24_ERR_ARG;
+    if (score == SS24_SCORE_WANDA && pattern != SS24_DENSE && (!col_norms || !aligned16(col_norms)))
+        return col_norms ? SS24_ERR_ALIGN : SS24_ERR_NULL;
+    if (!per_tensor(kind))
+        return SS24_ERR_FORMAT;
+    if ((st = check_ws(ws, ws_bytes)) != SS24_OK)
+        return st;
+    if (!scale_out)
+        return SS24_ERR_NULL;
+    if (x->rows == 0)
+        return cuda_status(cudaMemsetAsync(scale_out, 0, sizeof(float), s));
+    const float divisor = kind == SS24_FMT_FP8_E4M3 ? 448.0f : 2688.0f;
+    return cuda_status(run_amax(x, pattern, score, col_norms, ws, s, scale_out, divisor));
 }
 
 ss24_status ss24_predicted_ratio(const ss24_energy *sparse_side, const ss24_energy *dense_side, ss24_ratio *out,

@@ -665,8 +665,11 @@ __global__ void __launch_bounds__(kThreads, 1) pass_kernel(const __grid_constant
                     ka = fmaxf(ka, fred[w * 2]);
                     kb = fmaxf(kb, fred[w * 2 + 1]);
                 }
-                p.amax_out[0] = PAT == kDense ? kb : ka;
+                const float a0 = PAT == kDense ? kb : ka;
+                p.amax_out[0] = a0;
                 p.amax_out[1] = kb;
+                if (p.q.scale_out)
+                    *p.q.scale_out = __fdiv_rn(a0, p.q.divisor);
                 *p.amax_ticket = 0;
             }
         }

@@ -1,0 +1,105 @@
+"""Run one pass of the library on one synthetic operand, a few times.
+
+A small, self-contained driver for profiling a single kernel (for example under
+Nsight Compute) or for a quick timing of one configuration:
+
+    python -m semi_structured_sparsity_online_b200.run_case --pass fused_24_fp8 --m 4096 --k 4096 --iters 3
+
+Passes: tensor_scale, fused_24_{none,fp8,nvfp4,mxfp4,int8g128}, fused_48_nvfp4,
+dense_{fp8,nvfp4,mxfp4,int8_row,int8g128}, error_energy. Prints the mean CUDA-event
+time per launch and the GB/s of the pass's algorithmic bytes.
+"""
+from __future__ import annotations
+
+import argparse
+
+import numpy as np
+import torch
+
+from semi_structured_sparsity_online_b200 import ss24, synth
+
+# (pattern, format, bits, group): the stored format of each pass
+PASSES = {
+    "fused_24_none": (ss24.SPARSE_24, "none", 8, 0),
+    "fused_24_fp8": (ss24.SPARSE_24, "fp8", 8, 0),
+    "fused_24_nvfp4": (ss24.SPARSE_24, "nvfp4", 4, 0),
+    "fused_24_mxfp4": (ss24.SPARSE_24, "mxfp4", 4, 0),
+    "fused_24_int8g128": (ss24.SPARSE_24, "int", 8, 128),
+    "fused_48_nvfp4": (ss24.SPARSE_48, "nvfp4", 4, 0),
+    "dense_fp8": (ss24.DENSE, "fp8", 8, 0),
+    "dense_nvfp4": (ss24.DENSE, "nvfp4", 4, 0),
+    "dense_mxfp4": (ss24.DENSE, "mxfp4", 4, 0),
+    "dense_int8_row": (ss24.DENSE, "int", 8, 0),
+    "dense_int8g128": (ss24.DENSE, "int", 8, 128),
+}
+
+
+def pass_bytes(name, m, k):
+    """Algorithmic bytes of one launch on a bf16 [m, k] operand."""
+    n = m * k
+    if name in ("tensor_scale", "error_energy"):
+        return 2 * n
+    pattern, fmt, bits, group = PASSES[name]
+    q = n // 2 if pattern != ss24.DENSE else n
+    meta = n // 8 if pattern == ss24.SPARSE_24 else (n // 16 if pattern == ss24.SPARSE_48 else 0)
+    if fmt == "none":
+        vals, scales = 2 * q, 0
+    elif fmt == "fp8":
+        vals, scales = q, 0
+    elif fmt == "int":
+        vals, scales = q * (2 if bits > 8 else 1), 4 * (m if group == 0 else q // group)
+    elif fmt == "nvfp4":
+        vals, scales = q // 2, q // 16
+    else:
+        vals, scales = q // 2, q // 32
+    return 2 * n + vals + scales + meta
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--pass", dest="name", default="fused_24_fp8", choices=sorted(PASSES) + ["tensor_scale", "error_energy"])
+    ap.add_argument("--m", type=int, default=4096)
+    ap.add_argument("--k", type=int, default=4096)
+    ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--seed", type=int, default=8)
+    args = ap.parse_args()
+    xb = synth.sweep_operand(args.m, args.k, seed=args.seed)
+    x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).cuda()
+    ws = ss24.Workspace()
+    e = torch.zeros(4, dtype=torch.float64, device="cuda")
+    scale = ss24.tensor_scale(x, "fp8", ss24.SPARSE_24, ws=ws)
+    out = None
+    if args.name in PASSES:
+        pattern, fmt, bits, group = PASSES[args.name]
+        out = ss24._alloc_outputs(args.m, args.k, pattern, ss24.make_format(fmt, bits, group), torch.bfloat16, "cuda")
+        if fmt == "nvfp4":
+            scale = ss24.tensor_scale(x, "nvfp4", pattern if pattern != ss24.DENSE else ss24.DENSE, ws=ws)
+
+    def once():
+        if args.name == "tensor_scale":
+            ss24.tensor_scale(x, "fp8", ss24.SPARSE_24, ws=ws, out=scale)
+        elif args.name == "error_energy":
+            ss24.error_energy(x, ss24.SPARSE_24, ("fp8",), ("int", 5, 128), sparse_scale=scale, dense_scale=None,
+                              ws=ws, energy=e)
+        else:
+            pattern, fmt, bits, group = PASSES[args.name]
+            ts = scale if fmt in ("fp8", "nvfp4") else None
+            ss24.run(x, pattern=pattern, fmt=fmt, bits=bits, group=group, tensor_scale=ts, energy=e, ws=ws, out=out)
+
+    once()
+    torch.cuda.synchronize()
+    s, t = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(args.iters):
+        once()
+    t.record()
+    t.synchronize()
+    us = s.elapsed_time(t) / args.iters * 1e3
+    gb = pass_bytes(args.name, args.m, args.k)
+    assert ws.error() == 0
+    print(f"{args.name} m={args.m} k={args.k}: {us:.2f} us/launch, {gb / us / 1e3:.1f} GB/s "
+          f"({gb} algorithmic bytes per launch; warm L2 between launches)")
+
+
+if __name__ == "__main__":
+    main()

@@ -74,6 +74,7 @@ _SIGNATURES = {
     "ss24_error_energy": (ctypes.c_int, [_OP, ctypes.c_int, ctypes.c_int, _P, Format, Format, _P, _P, _P, _P,
                                          _S, _P]),
     "ss24_amax": (ctypes.c_int, [_OP, ctypes.c_int, ctypes.c_int, _P, _P, _P, _S, _P]),
+    "ss24_tensor_scale": (ctypes.c_int, [_OP, ctypes.c_int, ctypes.c_int, _P, ctypes.c_int32, _P, _P, _S, _P]),
     "ss24_predicted_ratio": (ctypes.c_int, [_P, _P, _P, _P]),
     "ss24_bits_per_element": (ctypes.c_double, [Format, ctypes.c_int, ctypes.c_int64, ctypes.c_int32]),
     "ss24_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -261,6 +262,18 @@ def amax(x, pattern=SPARSE_24, score="mag", col_norms=None, axis=1, ws=None, str
     ws = ws or default_workspace(x.device)
     _check(lib().ss24_amax(ctypes.byref(op), pattern, _SCORE[score] if isinstance(score, str) else score,
                            _ptr(col_norms), _ptr(out), ws.ptr, ws.nbytes, _stream(stream)), "ss24_amax")
+    return out
+
+
+def tensor_scale(x, fmt="fp8", pattern=SPARSE_24, score="mag", col_norms=None, axis=1, ws=None, stream=None,
+                 out=None):
+    """The per-tensor scale (FP8: amax / 448, NVFP4: amax / 2688) as a device float32[1]."""
+    op = make_operand(x, axis)
+    out = out if out is not None else torch.empty(1, dtype=torch.float32, device=x.device)
+    ws = ws or default_workspace(x.device)
+    _check(lib().ss24_tensor_scale(ctypes.byref(op), pattern, _SCORE[score] if isinstance(score, str) else score,
+                                   _ptr(col_norms), _FMT[fmt] if isinstance(fmt, str) else fmt, _ptr(out), ws.ptr,
+                                   ws.nbytes, _stream(stream)), "ss24_tensor_scale")
     return out
 
 
