@@ -281,6 +281,38 @@ ss24_status ss24_tensor_scale(const ss24_operand *x, ss24_pattern pattern, ss24_
 ss24_status ss24_predicted_ratio(const ss24_energy *sparse_side, const ss24_energy *dense_side,
                                  ss24_ratio *out, ss24_stream stream);
 
+/* ---- without caller-supplied scratch ----------------------------------------- */
+
+/* The fused 2:4 pass of ss24_prune24_quant_fused (same arguments, same results)
+ * for callers that cannot allocate device memory: code that runs where
+ * cudaMalloc is not allowed (inside a caching allocator's own callbacks, or a
+ * host that hands the library only the operand and the output buffers) and so
+ * cannot provide a workspace. No counterpart in the paper: it exists for such
+ * callers only.
+ *
+ * Scratch. The pass's scratch (per-CTA partial sums, two ticket counters and
+ * an error word, 41,472 bytes: enough for the at most 1024 CTAs the pass
+ * launches, whatever the operand size) lives in a device array owned by the
+ * library: one copy on every GPU that loads the library, kept until the
+ * process exits. The entry point allocates nothing and frees nothing. If the
+ * pass ever needed more scratch than the array holds it returns
+ * SS24_ERR_WORKSPACE. Errors recorded by a timed-out kernel wait are cleared at
+ * the next call and are not reported through this entry point.
+ *
+ * First call on a device: it looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture. Every call then clears the array's counters with a stream-ordered
+ * memset before launching.
+ *
+ * Concurrency. All calls on a device share the one array, which keeps the
+ * last call's contents: calls that overlap on the GPU (on different streams,
+ * or from different host threads without ordering) race and may return wrong
+ * energies. Order them on one stream. */
+ss24_status ss24_prune24_quant_fused_noalloc(const ss24_operand *x, ss24_score score,
+                                             const float *col_norms, ss24_format fmt,
+                                             const float *tensor_scale_in, ss24_outputs *out,
+                                             ss24_energy *energy, ss24_stream stream);
+
 /* ---- host-only helpers ------------------------------------------------------ */
 
 /* Stored bits per ORIGINAL element (§2: values, indices and, with with_scales,

@@ -429,6 +429,45 @@ ss24_status run_pass(const ss24_operand *x, int pattern, int score, const float 
     return cuda_status(e);
 }
 
+// ---------------------------------------------------------------------------
+// Library-owned scratch for callers that cannot allocate device memory
+// ---------------------------------------------------------------------------
+
+// The fused pass keeps a few partial sums per CTA (and an error word and two
+// ticket counters) between its CTAs. For callers that cannot call cudaMalloc,
+// that scratch lives in this file-scope device array: one copy per GPU that
+// loads the library, held until the process exits. The pass needs the same
+// fixed amount whatever the operand size (partials for at most kMaxGrid CTAs).
+constexpr size_t kStaticScratchBytes = kWsBytes;
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+void *g_static_ptr[kMaxDevices] = {};
+
+// Device address of the array on the current device. Host code must not use
+// the symbol's host-side name as a pointer; the address comes from
+// cudaGetSymbolAddress, taken once per device with that device current.
+cudaError_t static_scratch(void **ptr)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if (dev < 0 || dev >= kMaxDevices)
+        return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_static_scratch);
+        if (e != cudaSuccess)
+            return e;
+        g_static_ptr[dev] = p;
+    }
+    *ptr = g_static_ptr[dev];
+    return cudaSuccess;
+}
+
 } // namespace
 
 // ===========================================================================
@@ -727,6 +766,23 @@ ss24_status ss24_decode_e2m1(const uint8_t *in, float *out, int64_t n, ss24_stre
     if (n < 0)
         return SS24_ERR_SHAPE;
     return cuda_status(launch_convert(3, in, out, n, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ss24_status ss24_prune24_quant_fused_noalloc(const ss24_operand *x, ss24_score score, const float *col_norms,
+                                             ss24_format fmt, const float *tensor_scale_in, ss24_outputs *out,
+                                             ss24_energy *energy, ss24_stream stream)
+{
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (ss24_workspace_bytes() > kStaticScratchBytes)
+        return SS24_ERR_WORKSPACE; // the pass would need more scratch than the array holds
+    void *scratch = nullptr;
+    if (static_scratch(&scratch) != cudaSuccess)
+        return SS24_ERR_CUDA;
+    // the error word and the ticket counters must start at zero for this call
+    if (cudaMemsetAsync(scratch, 0, 256, s) != cudaSuccess)
+        return SS24_ERR_CUDA;
+    return run_pass(x, SS24_SPARSE_24, score, col_norms, fmt, true, tensor_scale_in, out, energy, scratch,
+                    kStaticScratchBytes, s);
 }
 
 } // extern "C"

@@ -69,6 +69,7 @@ _SIGNATURES = {
     "ss24_quantize_nvfp4": (ctypes.c_int, [_OP, _P, _OUT, _P, _P, _S, _P]),
     "ss24_quantize_mxfp4": (ctypes.c_int, [_OP, _OUT, _P, _P, _S, _P]),
     "ss24_prune24_quant_fused": (ctypes.c_int, [_OP, ctypes.c_int, _P, Format, _P, _OUT, _P, _P, _S, _P]),
+    "ss24_prune24_quant_fused_noalloc": (ctypes.c_int, [_OP, ctypes.c_int, _P, Format, _P, _OUT, _P, _P]),
     "ss24_prune48_pairwise_quant_fused": (ctypes.c_int,
                                           [_OP, ctypes.c_int, _P, Format, _P, _OUT, _P, _P, _S, _P]),
     "ss24_error_energy": (ctypes.c_int, [_OP, ctypes.c_int, ctypes.c_int, _P, Format, Format, _P, _P, _P, _P,
