@@ -274,12 +274,13 @@ ss24_status ss24_tensor_scale(const ss24_operand *x, ss24_pattern pattern, ss24_
                               const float *col_norms, int32_t kind, float *scale_out, void *ws,
                               size_t ws_bytes, ss24_stream stream);
 
-/* Derived quantities (§4) from a sparse-side energy record (e_total, e_prune,
- * e_quant) and a dense-side record (e_quant_dense); both device pointers, and
- * they may be the same record (as ss24_error_energy writes it). One-thread
- * kernel; writes *out on the device. */
+/* Derived quantities (§4) from sparse-side energy records (e_total, e_prune,
+ * e_quant) and dense-side records (e_quant_dense): count consecutive pairs,
+ * sparse_side[i] with dense_side[i] -> out[i]. Device pointers; the two inputs
+ * may be the same records (as ss24_error_energy writes them). One small
+ * kernel; count 0 enqueues nothing. */
 ss24_status ss24_predicted_ratio(const ss24_energy *sparse_side, const ss24_energy *dense_side,
-                                 ss24_ratio *out, ss24_stream stream);
+                                 ss24_ratio *out, int64_t count, ss24_stream stream);
 
 /* ---- without caller-supplied scratch ----------------------------------------- */
 
@@ -337,6 +338,23 @@ ss24_status ss24_decode_e4m3(const uint8_t *in, float *out, int64_t n, ss24_stre
 ss24_status ss24_encode_e2m1(const float *in, uint8_t *out, int64_t n, ss24_stream stream);
 /* Decode n E2M1 codes (low nibble of each byte) to binary32. */
 ss24_status ss24_decode_e2m1(const uint8_t *in, float *out, int64_t n, ss24_stream stream);
+
+/* ---- self-check of the kernels' division -------------------------------- */
+
+/* The kernels divide by a scale with Markstein's one-step correction of a
+ * reciprocal (P. Markstein, IBM J. Res. Dev. 34(1), 1990) instead of an IEEE
+ * division, for scales in [2^-60, 2^60]; this entry point checks that the two
+ * agree bit for bit on the running GPU. mode 0: b = 1 + (b_first + j) 2^-23
+ * for j < b_count, against every a in [1, 2) (2^23 significands each; b_first +
+ * b_count <= 2^23 — all 2^23 values of b together cover every pair of
+ * significands, which by exact power-of-two scaling covers every a and b the
+ * kernels divide with the correction). mode 1: 2^23 pseudo-random pairs per
+ * unit of b_count, exponents across the corrected range. Adds the number of
+ * mismatches to result[0] and lowers result[1] to the first mismatch
+ * (a bits << 32 | b bits); result is a device array of two uint64 the caller
+ * initialises to {0, UINT64_MAX}. */
+ss24_status ss24_selfcheck_division(int32_t mode, uint32_t b_first, uint32_t b_count,
+                                    unsigned long long *result, ss24_stream stream);
 
 #ifdef __cplusplus
 }

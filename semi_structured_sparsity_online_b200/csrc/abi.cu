@@ -16,6 +16,10 @@ const void *tile_kernel_bf16(int pattern, int score, int fmt);
 const void *tile_kernel_f32(int pattern, int score, int fmt);
 const void *row_kernel_bf16(int pattern, int score);
 const void *row_kernel_f32(int pattern, int score);
+const void *rowreg_kernel_bf16(int pattern, int score, int nch);
+const void *rowreg_kernel_f32(int pattern, int score, int nch);
+const void *axis0_kernel_bf16(int pattern, int score, int fmt);
+const void *axis0_kernel_f32(int pattern, int score, int fmt);
 } // namespace ss24
 
 using namespace ss24;
@@ -88,7 +92,7 @@ std::mutex g_mu;
 std::unordered_map<const void *, KernelInfo> g_info;
 int g_sms = 0;
 
-cudaError_t kernel_info(const void *k, size_t smem, KernelInfo *out)
+cudaError_t kernel_info(const void *k, size_t smem, KernelInfo *out, int threads = kThreads)
 {
     std::lock_guard<std::mutex> lock(g_mu);
     auto it = g_info.find(k);
@@ -100,7 +104,7 @@ cudaError_t kernel_info(const void *k, size_t smem, KernelInfo *out)
     if (e != cudaSuccess)
         return e;
     KernelInfo info;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&info.blocks_per_sm, k, kThreads, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&info.blocks_per_sm, k, threads, smem);
     if (e != cudaSuccess)
         return e;
     if (g_sms == 0) {
@@ -135,6 +139,39 @@ cudaError_t launch(const void *k, size_t smem, int64_t n_tiles, const CUtensorMa
     return e;
 }
 
+// The register-resident row kernel: no tensor map; one warp per row, 8 rows
+// per CTA.
+cudaError_t launch_rowreg(const void *k, const ss24_operand *x, const PassParams &p, cudaStream_t stream)
+{
+    KernelInfo info;
+    cudaError_t e = kernel_info(k, 0, &info, kRegRowThreads);
+    if (e != cudaSuccess)
+        return e;
+    const int64_t rows_per_cta = kRegRowThreads / 32;
+    int64_t grid = static_cast<int64_t>(g_sms) * (info.blocks_per_sm > 0 ? info.blocks_per_sm : 1);
+    if (grid > kMaxGrid)
+        grid = kMaxGrid;
+    const int64_t need = (x->rows + rows_per_cta - 1) / rows_per_cta;
+    if (grid > need)
+        grid = need;
+    const void *xp = x->x;
+    int64_t ld = x->ld;
+    PassParams pp = p;
+    void *args[3] = {&xp, &ld, &pp};
+    return cudaLaunchKernel(k, dim3(static_cast<unsigned>(grid)), dim3(kRegRowThreads), args, 0, stream);
+}
+
+// Chunks of 8 per lane for a register-resident row, or 0 when the row does not
+// fit (bf16 rows up to 4096 elements, fp32 rows up to 2048).
+int rowreg_chunks(const ss24_operand *x)
+{
+    const int64_t per_lane = (x->k + 255) / 256;
+    const int64_t limit = x->dtype == SS24_BF16 ? 16 : 8;
+    if (per_lane > limit)
+        return 0;
+    return per_lane <= 4 ? 4 : (per_lane <= 8 ? 8 : 16);
+}
+
 // ---------------------------------------------------------------------------
 // validation
 // ---------------------------------------------------------------------------
@@ -146,11 +183,11 @@ ss24_status check_operand(const ss24_operand *x)
         return SS24_ERR_NULL;
     if (x->dtype != SS24_BF16 && x->dtype != SS24_F32)
         return SS24_ERR_DTYPE;
-    if (x->axis != 1)
+    if (x->axis != 0 && x->axis != 1)
         return SS24_ERR_ARG;
     if (x->rows < 0 || x->k <= 0 || x->rows > INT32_MAX || x->k > INT32_MAX)
         return SS24_ERR_SHAPE;
-    if (x->ld < x->k)
+    if (x->ld < (x->axis == 1 ? x->k : x->rows))
         return SS24_ERR_SHAPE;
     if (!aligned16(x->x) || (x->ld * static_cast<int64_t>(esize(x->dtype))) % 16 != 0)
         return SS24_ERR_ALIGN;
@@ -212,6 +249,7 @@ ss24_status resolve_format(ss24_format fmt, int pattern, int64_t k, bool allow_n
             return SS24_ERR_FORMAT;
         q.bits = fmt.bits;
         q.qmax = static_cast<float>((1 << (fmt.bits - 1)) - 1);
+        q.qmax_inv = 1.0f / q.qmax; // IEEE binary32 division: RN(1 / qmax)
         q.store = fmt.pack4 ? kPack4 : (fmt.bits > 8 ? kInt16 : kInt8);
         if (fmt.group < 0)
             return SS24_ERR_FORMAT;
@@ -289,6 +327,34 @@ bool row_geometry(const ss24_operand *x, Geometry *g)
     return true;
 }
 
+// Axis 0: a tile is 128 k x (64 bf16 | 32 fp32) rows, transposed in shared memory.
+Geometry axis0_geometry(const ss24_operand *x)
+{
+    Geometry g{};
+    const int64_t R = x->dtype == SS24_BF16 ? 64 : 32;
+    g.W = kAxis0K;
+    g.R = static_cast<int32_t>(R);
+    g.log2_cpr = ilog2(kAxis0K / 8);
+    g.cpt = static_cast<int32_t>((R * kAxis0K / 8) / kConsumers);
+    g.n_col_tiles = (x->k + kAxis0K - 1) / kAxis0K;
+    g.n_tiles = g.n_col_tiles * ((x->rows + R - 1) / R);
+    g.tile_bytes = static_cast<uint32_t>(kStageBytes);
+    return g;
+}
+
+// The largest quantization group, in input elements, an axis-0 tile holds.
+bool axis0_format_ok(const ss24_format &fmt, int pattern, int64_t k)
+{
+    const bool sparse = pattern != SS24_DENSE;
+    if (fmt.kind == SS24_FMT_MXFP4 && sparse)
+        return true; // 64 input elements
+    if (fmt.kind != SS24_FMT_INT)
+        return true;
+    if (fmt.group == 0)
+        return pow2(k) && k <= kAxis0K;
+    return static_cast<int64_t>(fmt.group) * (sparse ? 2 : 1) <= kAxis0K;
+}
+
 PassParams base_params(const ss24_operand *x, const Geometry &g, void *ws, ss24_energy *energy)
 {
     PassParams p{};
@@ -300,6 +366,7 @@ PassParams base_params(const ss24_operand *x, const Geometry &g, void *ws, ss24_
     p.W = g.W;
     p.log2_cpr = g.log2_cpr;
     p.cpt = g.cpt;
+    p.axis = x->axis;
     p.tile_bytes = g.tile_bytes;
     uint8_t *w = static_cast<uint8_t *>(ws);
     p.err = reinterpret_cast<int32_t *>(w + kWsErrOff);
@@ -317,6 +384,28 @@ const void *tile_kernel(int dtype, int pattern, int score, int fmt)
     return dtype == SS24_BF16 ? tile_kernel_bf16(pattern, score, fmt) : tile_kernel_f32(pattern, score, fmt);
 }
 
+// Tile geometry, tensor map and kernel for a tile-mode pass along either axis.
+struct TilePlan {
+    Geometry g;
+    CUtensorMap map;
+    const void *kernel;
+    size_t smem;
+};
+
+bool plan_tile(const ss24_operand *x, int pattern, int score, int mode, TilePlan *t)
+{
+    if (x->axis == 1) {
+        t->g = tile_geometry(x);
+        t->kernel = tile_kernel(x->dtype, pattern, score, mode);
+        t->smem = kSmemBytes;
+        return make_map(&t->map, x, x->k, x->rows, static_cast<uint32_t>(t->g.W), static_cast<uint32_t>(t->g.R));
+    }
+    t->g = axis0_geometry(x);
+    t->kernel = x->dtype == SS24_BF16 ? axis0_kernel_bf16(pattern, score, mode) : axis0_kernel_f32(pattern, score, mode);
+    t->smem = kAxis0SmemBytes;
+    return make_map(&t->map, x, x->rows, x->k, static_cast<uint32_t>(t->g.R), static_cast<uint32_t>(t->g.W));
+}
+
 // The read-only amax pass; leaves {amax of kept, amax of all} in the workspace.
 // For the magnitude score the kept amax equals the amax of all values, so the
 // cheaper dense form is used.
@@ -324,15 +413,14 @@ cudaError_t run_amax(const ss24_operand *x, int pattern, int score, const float 
                      cudaStream_t stream, float *scale_out = nullptr, float divisor = 1.0f)
 {
     const int pat = score == SS24_SCORE_MAG ? SS24_DENSE : pattern;
-    const Geometry g = tile_geometry(x);
-    CUtensorMap map;
-    if (!make_map(&map, x, x->k, x->rows, static_cast<uint32_t>(g.W), static_cast<uint32_t>(g.R)))
+    TilePlan t;
+    if (!plan_tile(x, pat, score, kAmax, &t))
         return cudaErrorInvalidValue;
-    PassParams p = base_params(x, g, ws, nullptr);
+    PassParams p = base_params(x, t.g, ws, nullptr);
     p.norms = norms;
     p.q.scale_out = scale_out;
     p.q.divisor = divisor;
-    return launch(tile_kernel(x->dtype, pat, score, kAmax), kSmemBytes, g.n_tiles, map, p, stream);
+    return launch(t.kernel, t.smem, t.g.n_tiles, t.map, p, stream);
 }
 
 // Zero energy record / scale for an empty operand (nothing to launch).
@@ -372,8 +460,13 @@ ss24_status run_pass(const ss24_operand *x, int pattern, int score, const float 
         return st;
     if (!out)
         return SS24_ERR_NULL;
+    if (x->axis == 0 && !axis0_format_ok(fmt, pattern, x->k))
+        return SS24_ERR_FORMAT; // a group longer than the 128-element axis-0 tile
     Geometry g;
-    if (r.row_mode) {
+    if (x->axis == 0) {
+        r.row_mode = false;
+        g = axis0_geometry(x);
+    } else if (r.row_mode) {
         if (!row_geometry(x, &g))
             return SS24_ERR_SHAPE;
     } else {
@@ -416,15 +509,21 @@ ss24_status run_pass(const ss24_operand *x, int pattern, int score, const float 
     }
     CUtensorMap map;
     cudaError_t e;
-    if (r.row_mode) {
+    if (r.row_mode && rowreg_chunks(x) > 0) {
+        const int nch = rowreg_chunks(x);
+        const void *k = x->dtype == SS24_BF16 ? rowreg_kernel_bf16(pattern, score, nch)
+                                              : rowreg_kernel_f32(pattern, score, nch);
+        e = launch_rowreg(k, x, p, stream);
+    } else if (r.row_mode) {
         if (!make_map(&map, x, x->k, x->rows, static_cast<uint32_t>(g.W), static_cast<uint32_t>(g.R)))
             return SS24_ERR_CUDA;
         const void *k = x->dtype == SS24_BF16 ? row_kernel_bf16(pattern, score) : row_kernel_f32(pattern, score);
         e = launch(k, kRowSmemBytes, g.n_tiles, map, p, stream);
     } else {
-        if (!make_map(&map, x, x->k, x->rows, static_cast<uint32_t>(g.W), static_cast<uint32_t>(g.R)))
+        TilePlan t;
+        if (!plan_tile(x, pattern, score, fmt.kind, &t))
             return SS24_ERR_CUDA;
-        e = launch(tile_kernel(x->dtype, pattern, score, fmt.kind), kSmemBytes, g.n_tiles, map, p, stream);
+        e = launch(t.kernel, t.smem, t.g.n_tiles, t.map, p, stream);
     }
     return cuda_status(e);
 }
@@ -582,12 +681,16 @@ ss24_status ss24_error_energy(const ss24_operand *x, ss24_pattern pattern, ss24_
         return st;
     if ((st = resolve_format(dense_fmt, SS24_DENSE, x->k, false, &rd)) != SS24_OK)
         return st;
-    if (rs.row_mode || rd.row_mode)
+    if (x->axis == 1 && (rs.row_mode || rd.row_mode))
         return SS24_ERR_FORMAT; // one scale per long row needs the storing row-mode pass
+    if (x->axis == 0 && (!axis0_format_ok(sparse_fmt, pattern, x->k) || !axis0_format_ok(dense_fmt, SS24_DENSE, x->k)))
+        return SS24_ERR_FORMAT;
     if (x->rows == 0)
         return empty_operand(energy, nullptr, nullptr, s);
-    const Geometry g = tile_geometry(x);
-    PassParams p = base_params(x, g, ws, energy);
+    TilePlan t;
+    if (!plan_tile(x, pattern, score, kEnergy, &t))
+        return SS24_ERR_CUDA;
+    PassParams p = base_params(x, t.g, ws, energy);
     p.norms = col_norms;
     p.q = rs.q;
     p.qd = rd.q;
@@ -601,10 +704,7 @@ ss24_status ss24_error_energy(const ss24_operand *x, ss24_pattern pattern, ss24_
     p.q.amax_reduced = p.amax_out;     // [0]: amax of the kept values
     p.qd.scale_in = dense_scale_in;
     p.qd.amax_reduced = p.amax_out + 1; // [1]: amax of all values
-    CUtensorMap map;
-    if (!make_map(&map, x, x->k, x->rows, static_cast<uint32_t>(g.W), static_cast<uint32_t>(g.R)))
-        return SS24_ERR_CUDA;
-    return cuda_status(launch(tile_kernel(x->dtype, pattern, score, kEnergy), kSmemBytes, g.n_tiles, map, p, s));
+    return cuda_status(launch(t.kernel, t.smem, t.g.n_tiles, t.map, p, s));
 }
 
 ss24_status ss24_amax(const ss24_operand *x, ss24_pattern pattern, ss24_score score, const float *col_norms,
@@ -658,13 +758,15 @@ ss24_status ss24_tensor_scale(const ss24_operand *x, ss24_pattern pattern, ss24_
 }
 
 ss24_status ss24_predicted_ratio(const ss24_energy *sparse_side, const ss24_energy *dense_side, ss24_ratio *out,
-                                 ss24_stream stream)
+                                 int64_t count, ss24_stream stream)
 {
-    if (!sparse_side || !dense_side || !out)
+    if (count < 0)
+        return SS24_ERR_SHAPE;
+    if (count > 0 && (!sparse_side || !dense_side || !out))
         return SS24_ERR_NULL;
     return cuda_status(launch_ratio(reinterpret_cast<const double *>(sparse_side),
                                     reinterpret_cast<const double *>(dense_side), reinterpret_cast<double *>(out),
-                                    reinterpret_cast<cudaStream_t>(stream)));
+                                    count, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 double ss24_bits_per_element(ss24_format fmt, ss24_pattern pattern, int64_t k, int32_t with_scales)
@@ -730,6 +832,20 @@ const char *ss24_status_string(ss24_status status)
         return "unknown score, axis or pattern";
     }
     return "unknown status";
+}
+
+ss24_status ss24_selfcheck_division(int32_t mode, uint32_t b_first, uint32_t b_count, unsigned long long *result,
+                                    ss24_stream stream)
+{
+    if (!result)
+        return SS24_ERR_NULL;
+    if (mode != 0 && mode != 1)
+        return SS24_ERR_ARG;
+    if (mode == 0 && (b_first >= (1u << 23) || b_count > (1u << 23) - b_first))
+        return SS24_ERR_SHAPE;
+    if (b_count > 65535u * 32u)
+        return SS24_ERR_SHAPE;
+    return cuda_status(launch_selfcheck_division(mode, b_first, b_count, result, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 ss24_status ss24_encode_e4m3(const float *in, uint8_t *out, int64_t n, ss24_stream stream)

@@ -185,6 +185,104 @@ __device__ __forceinline__ float exp2_int(int e)
 }
 
 // ---------------------------------------------------------------------------
+// packed binary32 pairs (sm_100 f32x2 arithmetic, each lane rounded to nearest)
+// ---------------------------------------------------------------------------
+
+typedef unsigned long long f32x2;
+
+__device__ __forceinline__ f32x2 pack2(float lo, float hi)
+{
+    f32x2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+// element 0 of a pair is its low 32 bits
+__device__ __forceinline__ float lo2(f32x2 v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float hi2(f32x2 v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b)
+{
+    f32x2 d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b)
+{
+    f32x2 d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ f32x2 sub2(f32x2 a, f32x2 b)
+{
+    f32x2 d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c)
+{
+    f32x2 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+// ---------------------------------------------------------------------------
+// division by a scale
+// ---------------------------------------------------------------------------
+
+// Quotients a / b rounded to nearest-even, as an IEEE binary32 division gives
+// them. For a scale b in [2^-60, 2^60] the library uses Markstein's one-step
+// correction (P. Markstein, "Computation of elementary functions on the IBM
+// RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990): with
+// y = RN(1/b), q0 = RN(a y), r = a - q0 b (exact through the fused
+// multiply-add), q = RN(q0 + r y). Both significands range over [1, 2) without
+// loss of generality (power-of-two factors scale every step exactly while
+// operands and intermediates stay normal); ss24_selfcheck_division compares
+// this against IEEE division for every pair of significands. With b in the
+// range, y, q0 and the residual stay normal whenever |a / b| >= 2^-40, so the
+// result is exact there; below that the residual may lose bits, but every
+// format's code of such a quotient is the signed zero either way, and the sign
+// is kept. A quotient that overflows is ruled out by the callers (a group,
+// block or chunk amax times y stays below 2^126). Outside the range, IEEE
+// division is used.
+struct Recip {
+    float b, y, nb; // scale, RN(1/b), -b
+    bool fast;
+};
+
+__device__ __forceinline__ Recip make_recip(float b)
+{
+    Recip r;
+    r.b = b;
+    r.nb = -b;
+    r.y = __frcp_rn(b);
+    r.fast = b >= 0x1p-60f && b <= 0x1p60f;
+    return r;
+}
+
+// The sign of a / b for b > 0 is the sign of a. The correction step can lose
+// it for a signed zero (-0 * y - (-0) * b rounds to +0), so it is copied back.
+__device__ __forceinline__ float with_sign_of(float q, float a)
+{
+    return __uint_as_float((__float_as_uint(q) & 0x7fffffffu) | (__float_as_uint(a) & 0x80000000u));
+}
+
+__device__ __forceinline__ float div_fast(float a, const Recip &r)
+{
+    const float q0 = __fmul_rn(a, r.y);
+    const float res = __fmaf_rn(q0, r.nb, a);
+    return with_sign_of(__fmaf_rn(res, r.y, q0), a);
+}
+
+// Two quotients with packed arithmetic (the sign is restored by the caller
+// through with_sign_of on each half).
+__device__ __forceinline__ f32x2 div_fast2(f32x2 a, const Recip &r)
+{
+    const f32x2 y2 = pack2(r.y, r.y), nb2 = pack2(r.nb, r.nb);
+    const f32x2 q0 = mul2(a, y2);
+    const f32x2 res = fma2(q0, nb2, a);
+    return fma2(res, y2, q0);
+}
+
+// ---------------------------------------------------------------------------
 // selection
 // ---------------------------------------------------------------------------
 
@@ -217,16 +315,58 @@ __device__ __forceinline__ Pick top2_of_4(float s0, float s1, float s2, float s3
     return k;
 }
 
-// Kept and dropped values of one 2:4 group, in index order.
-__device__ __forceinline__ void apply24(const Pick &k, float a, float b, float c, float d, float &k0,
-                                        float &k1, float &d0, float &d1)
+// One 2:4 group: the kept values in index order, the dropped values, the
+// group's energy, the energy of its dropped pair and the metadata nibble. With
+// kAbs the scores are the magnitudes of the values themselves (compared
+// through |.|); otherwise s0..s3 are the scores.
+struct Group24 {
+    float k0, k1, d0, d1, e_all, e_drop;
+    uint32_t nib;
+};
+
+template <bool kAbs>
+__device__ __forceinline__ Group24 group24(float x0, float x1, float x2, float x3, float s0, float s1, float s2,
+                                           float s3)
 {
-    const float w01 = k.p ? b : a, l01 = k.p ? a : b;
-    const float w23 = k.q ? d : c, l23 = k.q ? c : d;
-    k0 = k.both01 ? a : (k.both23 ? c : w01);
-    k1 = k.both01 ? b : (k.both23 ? d : w23);
-    d0 = k.both01 ? c : (k.both23 ? a : l01);
-    d1 = k.both01 ? d : (k.both23 ? b : l23);
+    bool p, q, r, ta, tb;
+    float w01, l01, w23, l23;
+    if constexpr (kAbs) {
+        p = fabsf(x1) > fabsf(x0);
+        q = fabsf(x3) > fabsf(x2);
+        w01 = p ? x1 : x0;
+        l01 = p ? x0 : x1;
+        w23 = q ? x3 : x2;
+        l23 = q ? x2 : x3;
+        r = fabsf(w23) > fabsf(w01);
+        ta = fabsf(w23) > fabsf(l01);
+        tb = fabsf(l23) > fabsf(w01);
+    } else {
+        p = s1 > s0;
+        q = s3 > s2;
+        w01 = p ? x1 : x0;
+        l01 = p ? x0 : x1;
+        w23 = q ? x3 : x2;
+        l23 = q ? x2 : x3;
+        const float sw01 = p ? s1 : s0, sl01 = p ? s0 : s1;
+        const float sw23 = q ? s3 : s2, sl23 = q ? s2 : s3;
+        r = sw23 > sw01;
+        ta = sw23 > sl01;
+        tb = sl23 > sw01;
+    }
+    const bool both01 = !r && !ta, both23 = r && tb;
+    Group24 g;
+    g.k0 = both01 ? x0 : (both23 ? x2 : w01);
+    g.k1 = both01 ? x1 : (both23 ? x3 : w23);
+    g.d0 = both01 ? x2 : (both23 ? x0 : l01);
+    g.d1 = both01 ? x3 : (both23 ? x1 : l23);
+    const f32x2 e = fma2(pack2(x1, x3), pack2(x1, x3), mul2(pack2(x0, x2), pack2(x0, x2)));
+    const float e01 = lo2(e), e23 = hi2(e);
+    const float el = __fmaf_rn(l23, l23, l01 * l01);
+    g.e_all = e01 + e23;
+    g.e_drop = both01 ? e23 : (both23 ? e01 : el);
+    const uint32_t mixed = (p ? 1u : 0u) + (q ? 12u : 8u);
+    g.nib = both01 ? 0x4u : (both23 ? 0xEu : mixed);
+    return g;
 }
 
 } // namespace ss24

@@ -24,6 +24,18 @@ constexpr int kStages = 4;
 constexpr int kMaxGrid = 1024;            // bound on CTAs (workspace partials)
 constexpr size_t kSmemBytes = kStages * kStageBytes + 1024;
 
+// Register-resident rows (one scale per row, rows of at most 4096 bf16 / 2048
+// fp32 elements): one warp per row, 8 warps per CTA.
+constexpr int kRegRowThreads = 256;
+
+// Strided reduction axis (axis 0: rows contiguous in memory). A stage holds a
+// TMA box of 128 k x (64 bf16 | 32 fp32) rows, 16 KiB; consumers transpose it
+// into a row-major buffer (row pitch 128 + 8 bf16 / 128 + 4 fp32 elements =
+// 272 / 528 bytes) and process it like an axis-1 tile of width 128.
+constexpr int kAxis0K = 128;
+constexpr size_t kAxis0TBytes = 64 * 136 * 2; // >= 32 * 132 * 4
+constexpr size_t kAxis0SmemBytes = kStages * kStageBytes + kAxis0TBytes + 1024;
+
 // Row-mode (one scale per row, long rows): a stage holds whole rows.
 constexpr int kRowStageBytes = 49152;
 constexpr int kRowStages = 3;
@@ -49,6 +61,7 @@ struct QuantSpec {
     int32_t lanes;     // lanes (chunks) per scale group
     int32_t store;     // IntStore
     float qmax;        // INT
+    float qmax_inv;    // INT: RN(1 / qmax)
     float divisor;     // FP8: 448, NVFP4: 2688 (tensor scale = amax / divisor)
     const float *scale_in;     // given tensor scale (device) or nullptr
     const float *amax_reduced; // device float holding the amax when the scale is computed
@@ -61,6 +74,7 @@ struct PassParams {
     int32_t R, W;              // tile rows and width (elements)
     int32_t log2_cpr;          // log2(chunks of 8 per tile row)
     int32_t cpt;               // chunks per consumer thread per tile
+    int32_t axis;              // 1: k is the contiguous (TMA inner) dimension; 0: rows are
     uint32_t tile_bytes;
     // outputs
     void *values;
@@ -78,8 +92,10 @@ struct PassParams {
     int32_t *err;              // workspace error word
 };
 
-cudaError_t launch_ratio(const double *sparse_side, const double *dense_side, double *out,
+cudaError_t launch_ratio(const double *sparse_side, const double *dense_side, double *out, int64_t count,
                          cudaStream_t stream);
+cudaError_t launch_selfcheck_division(int mode, uint32_t b_first, uint32_t b_count, unsigned long long *result,
+                                      cudaStream_t stream);
 cudaError_t launch_convert(int op, const void *in, void *out, int64_t n, cudaStream_t stream);
 
 } // namespace ss24

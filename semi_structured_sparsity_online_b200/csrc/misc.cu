@@ -5,19 +5,28 @@
 namespace ss24 {
 
 // §4 of "Is 2:4 Sparsity Still Worth It?": loss = E_prune / E_total, the two
-// relative errors, and R_hat = sqrt((E_prune + E_q,2m) / E_q,m+1).
-__global__ void ratio_kernel(const double *sp, const double *de, double *out)
+// relative errors, and R_hat = sqrt((E_prune + E_q,2m) / E_q,m+1), for `count`
+// consecutive pairs of energy records.
+__global__ void ratio_kernel(const double *sp, const double *de, double *out, int64_t count)
 {
-    const double et = sp[0], ep = sp[1], eq = sp[2], ed = de[3];
-    out[0] = ep / et;
-    out[1] = sqrt((ep + eq) / et);
-    out[2] = sqrt(ed / et);
-    out[3] = sqrt((ep + eq) / ed);
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < count;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const double et = sp[4 * i], ep = sp[4 * i + 1], eq = sp[4 * i + 2], ed = de[4 * i + 3];
+        out[4 * i] = ep / et;
+        out[4 * i + 1] = sqrt((ep + eq) / et);
+        out[4 * i + 2] = sqrt(ed / et);
+        out[4 * i + 3] = sqrt((ep + eq) / ed);
+    }
 }
 
-cudaError_t launch_ratio(const double *sparse_side, const double *dense_side, double *out, cudaStream_t stream)
+cudaError_t launch_ratio(const double *sparse_side, const double *dense_side, double *out, int64_t count,
+                         cudaStream_t stream)
 {
-    ratio_kernel<<<1, 1, 0, stream>>>(sparse_side, dense_side, out);
+    if (count <= 0)
+        return cudaSuccess;
+    const int64_t blocks = (count + 127) / 128;
+    ratio_kernel<<<static_cast<unsigned>(blocks < 1024 ? blocks : 1024), 128, 0, stream>>>(sparse_side, dense_side,
+                                                                                          out, count);
     return cudaGetLastError();
 }
 
@@ -44,6 +53,77 @@ __global__ void convert_kernel(int op, const void *in, void *out, int64_t n)
             break;
         }
     }
+}
+
+// Markstein's correction (device.cuh, div_fast) against IEEE division.
+// mode 0: b = 1 + (b_first + blockIdx.x) * 2^-23 against every a in [1, 2)
+//         (all 2^23 significands); the full sweep over b covers every pair of
+//         significands.
+// mode 1: pseudo-random pairs with b in [2^-60, 2^60] and |a / b| in
+//         [2^-40, 2^100] (the range where the kernels use the correction),
+//         2^23 per block, from a counter-based hash of (block, index).
+// result[0] += mismatches; result[1] = first mismatch as (a bits << 32 | b bits).
+__device__ __forceinline__ uint32_t hash32(uint32_t x)
+{
+    x ^= x >> 16;
+    x *= 0x7feb352du;
+    x ^= x >> 15;
+    x *= 0x846ca68bu;
+    x ^= x >> 16;
+    return x;
+}
+
+__global__ void selfcheck_division_kernel(int mode, uint32_t b_first, unsigned long long *result)
+{
+    unsigned long long bad = 0, first = ~0ull;
+    if (mode == 0) {
+        const float b = __uint_as_float(0x3f800000u | (b_first + blockIdx.x));
+        const Recip rc = make_recip(b);
+        for (uint32_t i = threadIdx.x; i < (1u << 23); i += blockDim.x) {
+            const float a = __uint_as_float(0x3f800000u | i);
+            const float q = div_fast(a, rc), ref = __fdiv_rn(a, b);
+            if (__float_as_uint(q) != __float_as_uint(ref)) {
+                ++bad;
+                first = min(first, (static_cast<unsigned long long>(__float_as_uint(a)) << 32) | __float_as_uint(b));
+            }
+        }
+    } else {
+        for (uint32_t i = threadIdx.x; i < (1u << 23); i += blockDim.x) {
+            const uint32_t h1 = hash32(((b_first + blockIdx.x) << 23) ^ i), h2 = hash32(h1 ^ 0x9e3779b9u);
+            const uint32_t h3 = hash32(h2 + 0x632be5abu);
+            const int eb = static_cast<int>(h1 % 121u) - 60;            // b exponent in [-60, 60]
+            const int eq = static_cast<int>(h2 % 141u) - 40;            // quotient exponent in [-40, 100]
+            const float b = __uint_as_float((static_cast<uint32_t>(eb + 127) << 23) | (h3 & 0x7fffffu));
+            int ea = eb + eq;
+            if (ea > 127 || ea < -126)
+                continue;
+            const float a = __uint_as_float((h2 & 0x80000000u) | (static_cast<uint32_t>(ea + 127) << 23) |
+                                            (hash32(h3) & 0x7fffffu));
+            const Recip rc = make_recip(b);
+            const float q = div_fast(a, rc), ref = __fdiv_rn(a, b);
+            if (__float_as_uint(q) != __float_as_uint(ref)) {
+                ++bad;
+                first = min(first, (static_cast<unsigned long long>(__float_as_uint(a)) << 32) | __float_as_uint(b));
+            }
+        }
+    }
+    for (int off = 16; off >= 1; off >>= 1) {
+        bad += __shfl_xor_sync(kFull, bad, off);
+        first = min(first, __shfl_xor_sync(kFull, first, off));
+    }
+    if ((threadIdx.x & 31) == 0 && bad) {
+        atomicAdd(result, bad);
+        atomicMin(result + 1, first);
+    }
+}
+
+cudaError_t launch_selfcheck_division(int mode, uint32_t b_first, uint32_t b_count, unsigned long long *result,
+                                      cudaStream_t stream)
+{
+    if (b_count == 0)
+        return cudaSuccess;
+    selfcheck_division_kernel<<<b_count, 256, 0, stream>>>(mode, b_first, result);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_convert(int op, const void *in, void *out, int64_t n, cudaStream_t stream)

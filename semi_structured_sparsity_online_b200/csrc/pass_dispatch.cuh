@@ -57,4 +57,66 @@ template <typename T> const void *row_kernel_ptr(int pattern, int score)
     return nullptr;
 }
 
+template <typename T, int PAT, int SC> const void *axis0_for_fmt(int fmt)
+{
+    switch (fmt) {
+    case kNone:
+        if constexpr (PAT != kDense)
+            return reinterpret_cast<const void *>(&axis0_kernel<T, PAT, SC, kNone>);
+        break;
+    case kFp8:
+        return reinterpret_cast<const void *>(&axis0_kernel<T, PAT, SC, kFp8>);
+    case kInt:
+        return reinterpret_cast<const void *>(&axis0_kernel<T, PAT, SC, kInt>);
+    case kNvfp4:
+        return reinterpret_cast<const void *>(&axis0_kernel<T, PAT, SC, kNvfp4>);
+    case kMxfp4:
+        return reinterpret_cast<const void *>(&axis0_kernel<T, PAT, SC, kMxfp4>);
+    case kAmax:
+        return reinterpret_cast<const void *>(&axis0_kernel<T, PAT, SC, kAmax>);
+    case kEnergy:
+        if constexpr (PAT != kDense)
+            return reinterpret_cast<const void *>(&axis0_kernel<T, PAT, SC, kEnergy>);
+        break;
+    }
+    return nullptr;
+}
+
+template <typename T> const void *axis0_kernel_ptr(int pattern, int score, int fmt)
+{
+    if (pattern == kDense)
+        return axis0_for_fmt<T, kDense, kMag>(fmt);
+    if (pattern == kSparse24)
+        return score == kWanda ? axis0_for_fmt<T, kSparse24, kWanda>(fmt) : axis0_for_fmt<T, kSparse24, kMag>(fmt);
+    if (pattern == kSparse48)
+        return score == kWanda ? axis0_for_fmt<T, kSparse48, kWanda>(fmt) : axis0_for_fmt<T, kSparse48, kMag>(fmt);
+    return nullptr;
+}
+
+template <typename T, int PAT, int SC> const void *rowreg_for_nch(int nch)
+{
+    switch (nch) {
+    case 4:
+        return reinterpret_cast<const void *>(&rowreg_kernel<T, PAT, SC, 4>);
+    case 8:
+        return reinterpret_cast<const void *>(&rowreg_kernel<T, PAT, SC, 8>);
+    case 16:
+        if constexpr (sizeof(T) == 2)
+            return reinterpret_cast<const void *>(&rowreg_kernel<T, PAT, SC, 16>);
+        break;
+    }
+    return nullptr;
+}
+
+template <typename T> const void *rowreg_kernel_ptr(int pattern, int score, int nch)
+{
+    if (pattern == kDense)
+        return rowreg_for_nch<T, kDense, kMag>(nch);
+    if (pattern == kSparse24)
+        return score == kWanda ? rowreg_for_nch<T, kSparse24, kWanda>(nch) : rowreg_for_nch<T, kSparse24, kMag>(nch);
+    if (pattern == kSparse48)
+        return score == kWanda ? rowreg_for_nch<T, kSparse48, kWanda>(nch) : rowreg_for_nch<T, kSparse48, kMag>(nch);
+    return nullptr;
+}
+
 } // namespace ss24

@@ -76,9 +76,10 @@ _SIGNATURES = {
                                          _S, _P]),
     "ss24_amax": (ctypes.c_int, [_OP, ctypes.c_int, ctypes.c_int, _P, _P, _P, _S, _P]),
     "ss24_tensor_scale": (ctypes.c_int, [_OP, ctypes.c_int, ctypes.c_int, _P, ctypes.c_int32, _P, _P, _S, _P]),
-    "ss24_predicted_ratio": (ctypes.c_int, [_P, _P, _P, _P]),
+    "ss24_predicted_ratio": (ctypes.c_int, [_P, _P, _P, ctypes.c_int64, _P]),
     "ss24_bits_per_element": (ctypes.c_double, [Format, ctypes.c_int, ctypes.c_int64, ctypes.c_int32]),
     "ss24_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "ss24_selfcheck_division": (ctypes.c_int, [ctypes.c_int32, ctypes.c_uint32, ctypes.c_uint32, _P, _P]),
     "ss24_encode_e4m3": (ctypes.c_int, [_P, _P, ctypes.c_int64, _P]),
     "ss24_decode_e4m3": (ctypes.c_int, [_P, _P, ctypes.c_int64, _P]),
     "ss24_encode_e2m1": (ctypes.c_int, [_P, _P, ctypes.c_int64, _P]),
@@ -279,9 +280,11 @@ def tensor_scale(x, fmt="fp8", pattern=SPARSE_24, score="mag", col_norms=None, a
 
 
 def predicted_ratio(sparse_energy, dense_energy, out=None, stream=None):
-    """float64[4] on the device: loss, rel_err_sparse, rel_err_dense, R_hat."""
-    r = out if out is not None else torch.empty(4, dtype=torch.float64, device=sparse_energy.device)
-    _check(lib().ss24_predicted_ratio(_ptr(sparse_energy), _ptr(dense_energy), _ptr(r), _stream(stream)),
+    """float64[..., 4] on the device: loss, rel_err_sparse, rel_err_dense, R_hat,
+    for each pair of energy records (float64[..., 4], contiguous)."""
+    count = sparse_energy.numel() // 4
+    r = out if out is not None else torch.empty_like(sparse_energy)
+    _check(lib().ss24_predicted_ratio(_ptr(sparse_energy), _ptr(dense_energy), _ptr(r), count, _stream(stream)),
            "ss24_predicted_ratio")
     return r
 
@@ -292,6 +295,17 @@ def bits_per_element(fmt="none", bits=8, group=0, pattern=SPARSE_24, k=4096, wit
 
 def status_string(status: int) -> str:
     return lib().ss24_status_string(status).decode()
+
+
+def selfcheck_division(mode=0, b_first=0, b_count=1 << 23, chunk=1 << 16, stream=None):
+    """Mismatches between the kernels' corrected division and IEEE division
+    (see ss24_selfcheck_division); returns (count, first mismatch or None)."""
+    res = torch.tensor([0, -1], dtype=torch.int64, device="cuda")
+    for b0 in range(b_first, b_first + b_count, chunk):
+        n = min(chunk, b_first + b_count - b0)
+        _check(lib().ss24_selfcheck_division(mode, b0, n, _ptr(res), _stream(stream)), "ss24_selfcheck_division")
+    r = res.cpu().numpy().view("uint64")
+    return int(r[0]), (None if r[1] == 0xFFFFFFFFFFFFFFFF else (int(r[1]) >> 32, int(r[1]) & 0xFFFFFFFF))
 
 
 def _convert(name, t_in, out_dtype, stream=None):

@@ -169,7 +169,11 @@ def test_other_entry_points_validate():
     assert L.ss24_error_energy(ctypes.byref(o), ss24.SPARSE_24, ss24.MAG, None, ss24.make_format("none"),
                                ss24.make_format("int", 5), None, None, None, ALIGNED, wsb, None) == 1
     assert L.ss24_amax(ctypes.byref(o), ss24.SPARSE_24, ss24.MAG, None, None, ALIGNED, wsb, None) == 1
-    assert L.ss24_predicted_ratio(None, ALIGNED, ALIGNED, None) == 1
+    assert L.ss24_predicted_ratio(None, ALIGNED, ALIGNED, 1, None) == 1
+    assert L.ss24_predicted_ratio(ALIGNED, ALIGNED, ALIGNED, -1, None) == 2
+    assert L.ss24_selfcheck_division(2, 0, 1, ALIGNED, None) == 8
+    assert L.ss24_selfcheck_division(0, 1 << 23, 1, ALIGNED, None) == 2
+    assert L.ss24_selfcheck_division(0, 0, 1, None, None) == 1
     assert L.ss24_encode_e4m3(None, None, 5, None) == 1
     assert L.ss24_decode_e2m1(ALIGNED, ALIGNED, -1, None) == 2
     assert L.ss24_workspace_init(None, wsb, None) == 6

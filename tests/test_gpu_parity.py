@@ -63,22 +63,25 @@ def assert_energy(got, ref, fields=(0, 1, 2, 3), atol=0.0):
 
 
 def compare(ss, ws, xh, *, pattern, fmt, bits=8, group=0, pack4=False, score="mag", norms=None,
-            tensor_scale=None, k=None):
-    """Run both sides on the host array xh ([rows][ld]; k <= ld) and compare."""
+            tensor_scale=None, k=None, axis=1, rows=None):
+    """Run both sides on the host array xh and compare: axis 1, xh is [rows][ld]
+    (k <= ld); axis 0, xh is [k][ld] holding A[r][c] at xh[c][r] (rows <= ld)."""
     x = to_dev(xh)
-    if k is not None and k != xh.shape[1]:
+    if axis == 1 and k is not None and k != xh.shape[1]:
         xd = x[:, :k]
+    elif axis == 0 and rows is not None and rows != xh.shape[1]:
+        xd = x[:, :rows]
     else:
         xd = x
     nd = to_dev(norms) if norms is not None else None
     sd = torch.tensor([tensor_scale], dtype=torch.float32, device="cuda") if tensor_scale is not None else None
     opat = {0: oracle.DENSE, 24: oracle.SPARSE_24, 48: oracle.SPARSE_48}[pattern]
     out = ss.run(xd, pattern=pattern, fmt=fmt, bits=bits, group=group, pack4=pack4, score=score, col_norms=nd,
-                 tensor_scale=sd, ws=ws)
+                 tensor_scale=sd, ws=ws, axis=axis)
     torch.cuda.synchronize()
     ref = oracle.run(xh, pattern=opat, fmt=fmt, bits=bits, group=group, pack4=pack4,
                      score=oracle.WANDA if score == "wanda" else oracle.MAG, norms=norms,
-                     tensor_scale=tensor_scale, k=k)
+                     tensor_scale=tensor_scale, k=k, axis=axis, rows=rows)
     for key in ("values", "scales", "meta", "tensor_scale"):
         if key in ref:
             assert_same(to_np(out[key]), ref[key], key)
@@ -184,6 +187,76 @@ def test_int_one_scale_per_row(ss, ws, pattern, k):
     compare(ss, ws, xh, pattern=pattern, fmt="int", bits=4, group=0, pack4=True)
 
 
+AXIS0_FORMATS = [("none", 8, 0, False), ("fp8", 8, 0, False), ("int", 8, 32, False), ("int", 4, 16, True),
+                 ("int", 12, 64, False), ("nvfp4", 4, 0, False), ("mxfp4", 4, 0, False)]
+
+
+@pytest.mark.parametrize("pattern", [24, 48])
+@pytest.mark.parametrize("fmt,bits,group,pack4", AXIS0_FORMATS)
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_strided_axis(ss, ws, pattern, fmt, bits, group, pack4, dtype):
+    """Reduction axis strided in memory (rows contiguous): k = 512 spans four
+    128-wide tiles, 104 rows are ragged against the 64 / 32-row tile."""
+    xh = synth.sweep_operand(512, 104, seed=31) if dtype == "bf16" else synth.gaussian_f32(512, 104, seed=31)
+    compare(ss, ws, xh, pattern=pattern, fmt=fmt, bits=bits, group=group, pack4=pack4, axis=0)
+    norms = np.exp(np.random.default_rng(2).standard_normal(512)).astype(np.float32)
+    compare(ss, ws, xh, pattern=pattern, fmt=fmt, bits=bits, group=group, pack4=pack4, axis=0, score="wanda",
+            norms=norms)
+
+
+@pytest.mark.parametrize("fmt,bits,group", [("fp8", 8, 0), ("int", 8, 128), ("int", 5, 0), ("nvfp4", 4, 0),
+                                            ("mxfp4", 4, 0)])
+def test_strided_axis_dense_and_v_along_keys(ss, ws, fmt, bits, group):
+    """Dense partner along the strided axis, and V (keys x d, row-major) pruned
+    along the key axis of P.V: the logical operand is A[d][keys]."""
+    v = synth.attention_qkv(heads=1, seq=2048, d=128, seed=6)      # [keys, d]
+    if fmt == "int" and group == 0:
+        with pytest.raises(ss.SS24Error):                              # a 2048-long row does not fit a tile
+            ss.run(to_dev(v), pattern=0, fmt="int", bits=bits, group=0, axis=0, ws=ws)
+    else:
+        compare(ss, ws, v, pattern=0, fmt=fmt, bits=bits, group=group, axis=0)
+    compare(ss, ws, v, pattern=24, fmt="fp8", axis=0)
+    compare(ss, ws, v[:, :96].copy(), pattern=24, fmt="nvfp4", axis=0)      # 96 rows: ragged tile
+
+
+def test_strided_axis_limits_and_energy_pass(ss, ws):
+    x = to_dev(synth.gaussian_bf16(512, 64, seed=3))
+    with pytest.raises(ss.SS24Error) as e:
+        ss.run(x, pattern=24, fmt="int", bits=8, group=128, axis=0, ws=ws)   # 256-element groups
+    assert e.value.status == 5
+    with pytest.raises(ss.SS24Error):
+        ss.run(x, pattern=0, fmt="int", bits=8, group=0, axis=0, ws=ws)       # one scale per 512-long row
+    xh = synth.sweep_operand(256, 80, seed=4)
+    xd = to_dev(xh)
+    e_gpu = ss.error_energy(xd, pattern=24, sparse_fmt=("nvfp4",), dense_fmt=("int", 3, 64), axis=0, ws=ws)
+    sp = oracle.run(xh, fmt="nvfp4", axis=0)["energy"]
+    de = oracle.run(xh, pattern=oracle.DENSE, fmt="int", bits=3, group=64, axis=0)["energy"]
+    assert_energy(e_gpu, np.array([sp[0], sp[1], sp[2], de[3]]))
+    w = synth.gaussian_bf16(256, 64, seed=5, std=0.02)               # k = 256, 64 rows
+    norms = np.exp(np.random.default_rng(6).standard_normal(256)).astype(np.float32)
+    a = ss.amax(to_dev(w), pattern=24, score="wanda", col_norms=to_dev(norms), axis=0, ws=ws)
+    assert a.item() == oracle.amax(w, score=oracle.WANDA, norms=norms, axis=0)
+
+
+def test_int_one_scale_per_long_row(ss, ws):
+    """Rows too long for the register-resident kernel use the shared-memory row kernel."""
+    for pattern in (0, 24, 48):
+        xh, _ = synth.linear_input(21, 4352, seed=5)
+        compare(ss, ws, xh, pattern=pattern, fmt="int", bits=8, group=0)
+        xf = synth.gaussian_f32(13, 3072, seed=6)
+        compare(ss, ws, xf, pattern=pattern, fmt="int", bits=6, group=0)
+
+
+def test_division_matches_ieee_for_every_significand_pair(ss):
+    """The kernels' corrected-reciprocal division against IEEE division: every
+    pair of significands (2^46 quotients), then pairs spread over the exponent
+    range where the kernels use it."""
+    bad, first = ss.selfcheck_division(mode=0)
+    assert bad == 0, f"first mismatch a, b bits = {first}"
+    bad, first = ss.selfcheck_division(mode=1, b_count=1 << 12, chunk=1 << 12)
+    assert bad == 0, f"first mismatch a, b bits = {first}"
+
+
 @pytest.mark.parametrize("k", [8, 16, 24, 40, 96, 136, 264])
 @pytest.mark.parametrize("pattern", [0, 24])
 def test_small_and_ragged_k(ss, ws, pattern, k):
@@ -226,6 +299,30 @@ def test_given_tensor_scale_and_saturation(ss, ws):
     compare(ss, ws, xh, pattern=0, fmt="nvfp4", tensor_scale=0.0)
 
 
+def test_int_with_tiny_and_subnormal_scales(ss, ws):
+    """Groups whose amax is tiny give subnormal scales: the IEEE-division path
+    and the clamp of the definition."""
+    rng = np.random.default_rng(17)
+    x = rng.standard_normal((16, 256)).astype(np.float32)
+    x[0::2] *= np.float32(2.0 ** -135)        # subnormal values, subnormal scales
+    x[1::4] *= np.float32(2.0 ** -100)        # tiny normal values
+    for pattern in (0, 24):
+        compare(ss, ws, x, pattern=pattern, fmt="int", bits=8, group=32 if pattern == 0 else 16)
+        compare(ss, ws, x, pattern=pattern, fmt="int", bits=4, group=0)
+        compare(ss, ws, x, pattern=pattern, fmt="mxfp4")
+
+
+def test_signed_zeros_keep_their_sign(ss, ws):
+    """-0 and +0 quantize to the signed-zero codes IEEE division gives them."""
+    x = np.zeros((8, 64), dtype=np.uint16)
+    x[:, 0::3] = 0x8000                       # -0
+    x[:, 1::5] = synth.bf16_bits(np.float32([[1.5]]))[0, 0]
+    x[:, 2::7] = synth.bf16_bits(np.float32([[-3.0]]))[0, 0]
+    for fmt in ("fp8", "nvfp4", "int", "mxfp4"):
+        compare(ss, ws, x, pattern=24, fmt=fmt, bits=8, group=16)
+        compare(ss, ws, x, pattern=0, fmt=fmt, bits=8, group=16)
+
+
 def test_all_zero_operand(ss, ws):
     xh = np.zeros((40, 256), dtype=np.uint16)
     for fmt, bits, group, pack4 in FORMATS:
@@ -262,6 +359,8 @@ def test_amax_and_error_energy_and_ratio(ss, ws):
             assert_energy(e, ref)
             r = ss.predicted_ratio(e, e)
             rr = oracle.ratio(ref, ref)
+            r2 = ss.predicted_ratio(torch.stack([e, e]), torch.stack([e, e]))
+            assert torch.equal(r2[0], r) and torch.equal(r2[1], r)
             np.testing.assert_allclose(r.cpu().numpy(), rr, rtol=2e-6)
     assert ws.error() == 0
 
