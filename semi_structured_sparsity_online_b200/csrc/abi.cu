@@ -120,6 +120,24 @@ cudaError_t kernel_info(const void *k, size_t smem, KernelInfo *out, int threads
     return cudaSuccess;
 }
 
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the previous kernel on the stream finishes; it waits for it
+// (griddepcontrol.wait) before touching global memory.
+cudaError_t launch_pdl(const void *k, unsigned grid, unsigned threads, size_t smem, cudaStream_t stream, void **args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelExC(&cfg, k, args);
+}
+
 cudaError_t launch(const void *k, size_t smem, int64_t n_tiles, const CUtensorMap &map, const PassParams &p,
                    cudaStream_t stream)
 {
@@ -135,8 +153,7 @@ cudaError_t launch(const void *k, size_t smem, int64_t n_tiles, const CUtensorMa
     CUtensorMap m = map;
     PassParams pp = p;
     void *args[2] = {&m, &pp};
-    e = cudaLaunchKernel(k, dim3(static_cast<unsigned>(grid)), dim3(kThreads), args, smem, stream);
-    return e;
+    return launch_pdl(k, static_cast<unsigned>(grid), kThreads, smem, stream, args);
 }
 
 // The register-resident row kernel: no tensor map; one warp per row, 8 rows
@@ -158,7 +175,7 @@ cudaError_t launch_rowreg(const void *k, const ss24_operand *x, const PassParams
     int64_t ld = x->ld;
     PassParams pp = p;
     void *args[3] = {&xp, &ld, &pp};
-    return cudaLaunchKernel(k, dim3(static_cast<unsigned>(grid)), dim3(kRegRowThreads), args, 0, stream);
+    return launch_pdl(k, static_cast<unsigned>(grid), kRegRowThreads, 0, stream, args);
 }
 
 // Chunks of 8 per lane for a register-resident row, or 0 when the row does not

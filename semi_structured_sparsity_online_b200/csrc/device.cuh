@@ -105,6 +105,21 @@ __device__ __forceinline__ uint64_t l2_evict_first_policy()
     return p;
 }
 
+// Programmatic dependent launch (PTX griddepcontrol): a kernel launched with
+// programmatic stream serialization may start while the previous kernel on the
+// stream is finishing; it must wait for that kernel's completion (and memory)
+// before touching global memory. Every pass kernel waits right after its
+// shared-memory set-up, so only launch latency and set-up overlap.
+__device__ __forceinline__ void grid_dependency_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+// Lets the next kernel on the stream be scheduled (it still waits as above).
+__device__ __forceinline__ void grid_dependents_launch()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void named_barrier_sync(int id, int threads)
 {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");

@@ -9,6 +9,7 @@ namespace ss24 {
 // consecutive pairs of energy records.
 __global__ void ratio_kernel(const double *sp, const double *de, double *out, int64_t count)
 {
+    grid_dependency_wait();
     for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < count;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const double et = sp[4 * i], ep = sp[4 * i + 1], eq = sp[4 * i + 2], ed = de[4 * i + 3];
@@ -34,6 +35,7 @@ cudaError_t launch_ratio(const double *sparse_side, const double *dense_side, do
 // 3: E2M1 (low nibble) -> f32.
 __global__ void convert_kernel(int op, const void *in, void *out, int64_t n)
 {
+    grid_dependency_wait();
     for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         switch (op) {

@@ -753,6 +753,8 @@ __global__ void __launch_bounds__(kThreads, 1) pass_kernel(const __grid_constant
         fence_barrier_init();
     }
     __syncthreads();
+    grid_dependency_wait();
+    grid_dependents_launch();
 
     if (warp == kConsumerWarps) {
         if (lane == 0)
@@ -900,6 +902,8 @@ __global__ void __launch_bounds__(kThreads, 1) row_kernel(const __grid_constant_
         fence_barrier_init();
     }
     __syncthreads();
+    grid_dependency_wait();
+    grid_dependents_launch();
     if (warp == kConsumerWarps) {
         if (lane == 0)
             row_producer(&map, p, stages, full, empty, nbox, static_cast<int>(sizeof(T)));
@@ -1005,6 +1009,8 @@ __global__ void __launch_bounds__(kRegRowThreads) rowreg_kernel(const T *__restr
     __shared__ double red[kConsumerWarps * 4];
     __shared__ uint32_t flag;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    grid_dependency_wait();
+    grid_dependents_launch();
     const int nchunks = static_cast<int>(p.k / 8);
     const Recip no_recip = make_recip(0.0f);
     double e_total = 0.0, e_prune = 0.0, e_q = 0.0, e_qd = 0.0;
@@ -1179,6 +1185,8 @@ __global__ void __launch_bounds__(kThreads, 1) axis0_kernel(const __grid_constan
         fence_barrier_init();
     }
     __syncthreads();
+    grid_dependency_wait();
+    grid_dependents_launch();
     if (warp == kConsumerWarps) {
         if (lane == 0)
             producer(&map, p, stages, full, empty);
