@@ -50,6 +50,16 @@
  * g covers g kept values (2g original positions), an NVFP4 block 16 kept
  * values, an MXFP4 block 32.
  *
+ * Batches. An operand descriptor with batch = B > 1 describes B operands of the
+ * same shape, operand b at x + b * batch_stride. One call then processes all
+ * of them (one launch per kernel instead of B), each exactly as a call on that
+ * operand alone would: per-tensor scales, amaxes and energies are per operand.
+ * Every output holds the B operands' outputs one after the other (the
+ * per-operand layouts above, packed): values, scales and metadata as
+ * [B][rows][...], tensor scales as float[B], tensor_scale_in as float[B],
+ * energy records as ss24_energy[B], amax outputs as float[B]. col_norms is
+ * shared by all operands.
+ *
  * Selection. Element i beats element j when s_i > s_j, or s_i == s_j and
  * i < j; the two elements beaten by fewer than two others are kept (ties keep
  * the lower index). Scores: SS24_SCORE_MAG s = |x|; SS24_SCORE_WANDA
@@ -148,13 +158,16 @@ typedef struct {
 } ss24_format;
 
 typedef struct {
-    const void *x; /* device pointer to the operand                      */
-    int32_t dtype; /* ss24_dtype                                          */
-    int32_t axis;  /* 1: k contiguous; 0: rows contiguous                 */
-    int64_t rows;  /* logical rows (>= 0; 0 is a valid empty operand)     */
-    int64_t k;     /* reduction length (> 0)                              */
-    int64_t ld;    /* elements between consecutive rows (axis 1) or
-                      consecutive k positions (axis 0)                    */
+    const void *x;        /* device pointer to the (first) operand                */
+    int32_t dtype;        /* ss24_dtype                                            */
+    int32_t axis;         /* 1: k contiguous; 0: rows contiguous                   */
+    int64_t rows;         /* logical rows (>= 0; 0 is a valid empty operand)       */
+    int64_t k;            /* reduction length (> 0)                                */
+    int64_t ld;           /* elements between consecutive rows (axis 1) or
+                             consecutive k positions (axis 0)                      */
+    int64_t batch;        /* operands in the call: 0 or 1 for one, up to 1024      */
+    int64_t batch_stride; /* elements from one operand to the next (batch > 1);
+                             at least rows * ld (axis 1) or k * ld (axis 0)       */
 } ss24_operand;
 
 typedef struct {
@@ -180,8 +193,9 @@ typedef struct {
 /* Bytes of device workspace every computing call needs (a constant). */
 size_t ss24_workspace_bytes(void);
 
-/* Clears the workspace's error word (stream-ordered memset). Call once after
- * allocating the workspace, and again to reset a recorded error. */
+/* Clears the workspace's error word and ticket counters (a stream-ordered
+ * memset of its first 8,448 bytes). Call once after allocating the workspace,
+ * and again to reset a recorded error. */
 ss24_status ss24_workspace_init(void *ws, size_t ws_bytes, ss24_stream stream);
 
 /* Synchronizes `stream`, then copies the workspace's error word to *code
@@ -292,7 +306,7 @@ ss24_status ss24_predicted_ratio(const ss24_energy *sparse_side, const ss24_ener
  * callers only.
  *
  * Scratch. The pass's scratch (per-CTA partial sums, two ticket counters and
- * an error word, 41,472 bytes: enough for the at most 1024 CTAs the pass
+ * an error word, 57,600 bytes: enough for the at most 1024 CTAs the pass
  * launches, whatever the operand size) lives in a device array owned by the
  * library: one copy on every GPU that loads the library, kept until the
  * process exits. The entry point allocates nothing and frees nothing. If the

@@ -14,10 +14,8 @@
 namespace ss24 {
 const void *tile_kernel_bf16(int pattern, int score, int fmt);
 const void *tile_kernel_f32(int pattern, int score, int fmt);
-const void *row_kernel_bf16(int pattern, int score);
-const void *row_kernel_f32(int pattern, int score);
-const void *rowreg_kernel_bf16(int pattern, int score, int nch);
-const void *rowreg_kernel_f32(int pattern, int score, int nch);
+const void *rowsweep_kernel_bf16(int pattern, int score);
+const void *rowsweep_kernel_f32(int pattern, int score);
 const void *axis0_kernel_bf16(int pattern, int score, int fmt);
 const void *axis0_kernel_f32(int pattern, int score, int fmt);
 } // namespace ss24
@@ -64,7 +62,17 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
     return fn;
 }
 
-// 2-D map over the operand's memory: inner dimension = the contiguous one.
+// Operands in a batch (batch 0 reads as 1) and the element stride between them.
+int64_t nbatch(const ss24_operand *x) { return x->batch > 1 ? x->batch : 1; }
+int64_t bstride_elems(const ss24_operand *x)
+{
+    if (x->batch > 1)
+        return x->batch_stride;
+    return (x->axis == 1 ? x->rows : x->k) * x->ld; // unused: one operand
+}
+
+// 3-D map over the operands' memory: {contiguous dimension, the other one,
+// operand of the batch}.
 bool make_map(CUtensorMap *map, const ss24_operand *x, int64_t inner, int64_t outer, uint32_t box_inner,
               uint32_t box_outer)
 {
@@ -73,11 +81,16 @@ bool make_map(CUtensorMap *map, const ss24_operand *x, int64_t inner, int64_t ou
         return false;
     const CUtensorMapDataType dt =
         x->dtype == SS24_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-    cuuint64_t gdim[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
-    cuuint64_t gstride[1] = {static_cast<cuuint64_t>(x->ld) * esize(x->dtype)};
-    cuuint32_t box[2] = {box_inner, box_outer};
-    cuuint32_t estride[2] = {1, 1};
-    const CUresult r = fn(map, dt, 2, const_cast<void *>(x->x), gdim, gstride, box, estride,
+    const cuuint64_t es = esize(x->dtype);
+    int64_t bs = bstride_elems(x);
+    if (bs < 1)
+        bs = x->ld; // an empty single operand never gets here; keep the stride valid
+    cuuint64_t gdim[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer),
+                          static_cast<cuuint64_t>(nbatch(x))};
+    cuuint64_t gstride[2] = {static_cast<cuuint64_t>(x->ld) * es, static_cast<cuuint64_t>(bs) * es};
+    cuuint32_t box[3] = {box_inner, box_outer, 1};
+    cuuint32_t estride[3] = {1, 1, 1};
+    const CUresult r = fn(map, dt, 3, const_cast<void *>(x->x), gdim, gstride, box, estride,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -138,6 +151,20 @@ cudaError_t launch_pdl(const void *k, unsigned grid, unsigned threads, size_t sm
     return cudaLaunchKernelExC(&cfg, k, args);
 }
 
+// CTAs per operand: the persistent grid (SMs x resident CTAs, at most
+// kMaxGrid) shared among the operands of the batch, at most one CTA per unit
+// of work of an operand.
+int64_t ctas_per_operand(const KernelInfo &info, int64_t batch, int64_t units)
+{
+    int64_t total = static_cast<int64_t>(g_sms) * (info.blocks_per_sm > 0 ? info.blocks_per_sm : 1);
+    if (total > kMaxGrid)
+        total = kMaxGrid;
+    int64_t per = total / batch;
+    if (per > units)
+        per = units;
+    return per < 1 ? 1 : per;
+}
+
 cudaError_t launch(const void *k, size_t smem, int64_t n_tiles, const CUtensorMap &map, const PassParams &p,
                    cudaStream_t stream)
 {
@@ -145,48 +172,27 @@ cudaError_t launch(const void *k, size_t smem, int64_t n_tiles, const CUtensorMa
     cudaError_t e = kernel_info(k, smem, &info);
     if (e != cudaSuccess)
         return e;
-    int64_t grid = static_cast<int64_t>(g_sms) * (info.blocks_per_sm > 0 ? info.blocks_per_sm : 1);
-    if (grid > kMaxGrid)
-        grid = kMaxGrid;
-    if (grid > n_tiles)
-        grid = n_tiles;
-    CUtensorMap m = map;
     PassParams pp = p;
+    pp.ctas_per_op = static_cast<int32_t>(ctas_per_operand(info, p.batch, n_tiles));
+    CUtensorMap m = map;
     void *args[2] = {&m, &pp};
-    return launch_pdl(k, static_cast<unsigned>(grid), kThreads, smem, stream, args);
+    return launch_pdl(k, static_cast<unsigned>(p.batch * pp.ctas_per_op), kThreads, smem, stream, args);
 }
 
-// The register-resident row kernel: no tensor map; one warp per row, 8 rows
-// per CTA.
-cudaError_t launch_rowreg(const void *k, const ss24_operand *x, const PassParams &p, cudaStream_t stream)
+// The one-scale-per-row kernel: no tensor map; one warp per row, 8 rows per CTA.
+cudaError_t launch_rowsweep(const void *k, const ss24_operand *x, const PassParams &p, cudaStream_t stream)
 {
     KernelInfo info;
-    cudaError_t e = kernel_info(k, 0, &info, kRegRowThreads);
+    cudaError_t e = kernel_info(k, 0, &info, kRowThreads);
     if (e != cudaSuccess)
         return e;
-    const int64_t rows_per_cta = kRegRowThreads / 32;
-    int64_t grid = static_cast<int64_t>(g_sms) * (info.blocks_per_sm > 0 ? info.blocks_per_sm : 1);
-    if (grid > kMaxGrid)
-        grid = kMaxGrid;
-    const int64_t need = (x->rows + rows_per_cta - 1) / rows_per_cta;
-    if (grid > need)
-        grid = need;
+    const int64_t rows_per_cta = kRowThreads / 32;
+    PassParams pp = p;
+    pp.ctas_per_op = static_cast<int32_t>(ctas_per_operand(info, p.batch, (x->rows + rows_per_cta - 1) / rows_per_cta));
     const void *xp = x->x;
     int64_t ld = x->ld;
-    PassParams pp = p;
     void *args[3] = {&xp, &ld, &pp};
-    return launch_pdl(k, static_cast<unsigned>(grid), kRegRowThreads, 0, stream, args);
-}
-
-// Chunks of 8 per lane for a register-resident row, or 0 when the row does not
-// fit (bf16 rows up to 4096 elements, fp32 rows up to 2048).
-int rowreg_chunks(const ss24_operand *x)
-{
-    const int64_t per_lane = (x->k + 255) / 256;
-    const int64_t limit = x->dtype == SS24_BF16 ? 16 : 8;
-    if (per_lane > limit)
-        return 0;
-    return per_lane <= 4 ? 4 : (per_lane <= 8 ? 8 : 16);
+    return launch_pdl(k, static_cast<unsigned>(p.batch * pp.ctas_per_op), kRowThreads, 0, stream, args);
 }
 
 // ---------------------------------------------------------------------------
@@ -208,6 +214,15 @@ ss24_status check_operand(const ss24_operand *x)
         return SS24_ERR_SHAPE;
     if (!aligned16(x->x) || (x->ld * static_cast<int64_t>(esize(x->dtype))) % 16 != 0)
         return SS24_ERR_ALIGN;
+    if (x->batch < 0 || x->batch > kMaxGrid)
+        return SS24_ERR_SHAPE;
+    if (x->batch > 1) {
+        // operands must not overlap
+        if (x->batch_stride < (x->axis == 1 ? x->rows : x->k) * x->ld)
+            return SS24_ERR_SHAPE;
+        if ((x->batch_stride * static_cast<int64_t>(esize(x->dtype))) % 16 != 0)
+            return SS24_ERR_ALIGN;
+    }
     return SS24_OK;
 }
 
@@ -323,27 +338,6 @@ Geometry tile_geometry(const ss24_operand *x)
     return g;
 }
 
-// Row mode: whole rows, boxes of W = min(256, next_pow2(k)) columns.
-bool row_geometry(const ss24_operand *x, Geometry *g)
-{
-    const int64_t es = static_cast<int64_t>(esize(x->dtype));
-    g->W = static_cast<int32_t>(x->k >= 256 ? 256 : next_pow2(x->k));
-    const int64_t nbox = (x->k + g->W - 1) / g->W;
-    const int64_t row_bytes = nbox * g->W * es;
-    int64_t R = kRowStageBytes / row_bytes;
-    if (R < 1)
-        return false;
-    if (R > 256)
-        R = 256;
-    g->R = static_cast<int32_t>(R);
-    g->log2_cpr = ilog2(g->W / 8);
-    g->cpt = 0;
-    g->n_col_tiles = 1;
-    g->n_tiles = (x->rows + R - 1) / R;
-    g->tile_bytes = static_cast<uint32_t>(R * row_bytes);
-    return true;
-}
-
 // Axis 0: a tile is 128 k x (64 bf16 | 32 fp32) rows, transposed in shared memory.
 Geometry axis0_geometry(const ss24_operand *x)
 {
@@ -393,7 +387,39 @@ PassParams base_params(const ss24_operand *x, const Geometry &g, void *ws, ss24_
     p.amax_partials = reinterpret_cast<float *>(w + kWsAmaxOff);
     p.amax_out = reinterpret_cast<float *>(w + kWsAmaxReducedOff);
     p.energy_out = reinterpret_cast<double *>(energy);
+    p.batch = static_cast<int32_t>(nbatch(x));
+    p.x_bstride = bstride_elems(x);
     return p;
+}
+
+// Per-operand byte strides of the outputs of a pass storing `fmt` (outputs of
+// a batch are packed one operand after the other).
+void output_strides(const ss24_operand *x, int pattern, ss24_format fmt, PassParams *p)
+{
+    const bool sparse = pattern != SS24_DENSE;
+    const int64_t n = sparse ? x->k / 2 : x->k, rows = x->rows;
+    switch (fmt.kind) {
+    case SS24_FMT_NONE:
+        p->values_bstride = rows * n * static_cast<int64_t>(esize(x->dtype));
+        break;
+    case SS24_FMT_FP8_E4M3:
+        p->values_bstride = rows * n;
+        break;
+    case SS24_FMT_INT:
+        p->values_bstride = fmt.pack4 ? rows * n / 2 : rows * n * (fmt.bits > 8 ? 2 : 1);
+        p->scales_bstride = rows * (fmt.group ? n / fmt.group : 1) * 4;
+        break;
+    case SS24_FMT_NVFP4:
+        p->values_bstride = rows * n / 2;
+        p->scales_bstride = rows * n / 16;
+        break;
+    case SS24_FMT_MXFP4:
+        p->values_bstride = rows * n / 2;
+        p->scales_bstride = rows * n / 32;
+        break;
+    }
+    if (sparse)
+        p->meta_bstride = rows * x->k / (pattern == SS24_SPARSE_48 ? 16 : 8);
 }
 
 const void *tile_kernel(int dtype, int pattern, int score, int fmt)
@@ -427,7 +453,8 @@ bool plan_tile(const ss24_operand *x, int pattern, int score, int mode, TilePlan
 // For the magnitude score the kept amax equals the amax of all values, so the
 // cheaper dense form is used.
 cudaError_t run_amax(const ss24_operand *x, int pattern, int score, const float *norms, void *ws,
-                     cudaStream_t stream, float *scale_out = nullptr, float divisor = 1.0f)
+                     cudaStream_t stream, float *scale_out = nullptr, float divisor = 1.0f,
+                     float *amax_user = nullptr)
 {
     const int pat = score == SS24_SCORE_MAG ? SS24_DENSE : pattern;
     TilePlan t;
@@ -437,21 +464,23 @@ cudaError_t run_amax(const ss24_operand *x, int pattern, int score, const float 
     p.norms = norms;
     p.q.scale_out = scale_out;
     p.q.divisor = divisor;
+    p.amax_user = amax_user;
     return launch(t.kernel, t.smem, t.g.n_tiles, t.map, p, stream);
 }
 
-// Zero energy record / scale for an empty operand (nothing to launch).
-ss24_status empty_operand(ss24_energy *energy, const ss24_outputs *out, const float *scale_in,
+// Zero energy records / scales for empty operands (nothing to launch).
+ss24_status empty_operand(const ss24_operand *x, ss24_energy *energy, const ss24_outputs *out, const float *scale_in,
                           cudaStream_t stream)
 {
+    const size_t nb = static_cast<size_t>(nbatch(x));
     cudaError_t e = cudaSuccess;
     if (energy)
-        e = cudaMemsetAsync(energy, 0, sizeof(ss24_energy), stream);
+        e = cudaMemsetAsync(energy, 0, nb * sizeof(ss24_energy), stream);
     if (e == cudaSuccess && out && out->tensor_scale) {
         if (scale_in)
-            e = cudaMemcpyAsync(out->tensor_scale, scale_in, sizeof(float), cudaMemcpyDeviceToDevice, stream);
+            e = cudaMemcpyAsync(out->tensor_scale, scale_in, nb * sizeof(float), cudaMemcpyDeviceToDevice, stream);
         else
-            e = cudaMemsetAsync(out->tensor_scale, 0, sizeof(float), stream);
+            e = cudaMemsetAsync(out->tensor_scale, 0, nb * sizeof(float), stream);
     }
     return cuda_status(e);
 }
@@ -483,14 +512,11 @@ ss24_status run_pass(const ss24_operand *x, int pattern, int score, const float 
     if (x->axis == 0) {
         r.row_mode = false;
         g = axis0_geometry(x);
-    } else if (r.row_mode) {
-        if (!row_geometry(x, &g))
-            return SS24_ERR_SHAPE;
     } else {
-        g = tile_geometry(x);
+        g = tile_geometry(x); // (row mode uses only rows / k of it)
     }
     if (x->rows == 0)
-        return empty_operand(energy, out, per_tensor(fmt.kind) ? scale_in : nullptr, stream);
+        return empty_operand(x, energy, out, per_tensor(fmt.kind) ? scale_in : nullptr, stream);
     if (!out->values)
         return SS24_ERR_NULL;
     if (!aligned16(out->values))
@@ -509,6 +535,7 @@ ss24_status run_pass(const ss24_operand *x, int pattern, int score, const float 
 
     // ---- launches ----
     PassParams p = base_params(x, g, ws, energy);
+    output_strides(x, pattern, fmt, &p);
     p.values = out->values;
     p.scales = out->scales;
     p.meta = out->meta;
@@ -524,18 +551,10 @@ ss24_status run_pass(const ss24_operand *x, int pattern, int score, const float 
             p.q.amax_reduced = p.amax_out; // [0] = amax of the quantized values
         }
     }
-    CUtensorMap map;
     cudaError_t e;
-    if (r.row_mode && rowreg_chunks(x) > 0) {
-        const int nch = rowreg_chunks(x);
-        const void *k = x->dtype == SS24_BF16 ? rowreg_kernel_bf16(pattern, score, nch)
-                                              : rowreg_kernel_f32(pattern, score, nch);
-        e = launch_rowreg(k, x, p, stream);
-    } else if (r.row_mode) {
-        if (!make_map(&map, x, x->k, x->rows, static_cast<uint32_t>(g.W), static_cast<uint32_t>(g.R)))
-            return SS24_ERR_CUDA;
-        const void *k = x->dtype == SS24_BF16 ? row_kernel_bf16(pattern, score) : row_kernel_f32(pattern, score);
-        e = launch(k, kRowSmemBytes, g.n_tiles, map, p, stream);
+    if (r.row_mode) {
+        const void *k = x->dtype == SS24_BF16 ? rowsweep_kernel_bf16(pattern, score) : rowsweep_kernel_f32(pattern, score);
+        e = launch_rowsweep(k, x, p, stream);
     } else {
         TilePlan t;
         if (!plan_tile(x, pattern, score, fmt.kind, &t))
@@ -599,7 +618,7 @@ ss24_status ss24_workspace_init(void *ws, size_t ws_bytes, ss24_stream stream)
     ss24_status st = check_ws(ws, ws_bytes);
     if (st != SS24_OK)
         return st;
-    return cuda_status(cudaMemsetAsync(ws, 0, 256, reinterpret_cast<cudaStream_t>(stream)));
+    return cuda_status(cudaMemsetAsync(ws, 0, kWsClearBytes, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 ss24_status ss24_workspace_error(const void *ws, int32_t *code, ss24_stream stream)
@@ -703,7 +722,7 @@ ss24_status ss24_error_energy(const ss24_operand *x, ss24_pattern pattern, ss24_
     if (x->axis == 0 && (!axis0_format_ok(sparse_fmt, pattern, x->k) || !axis0_format_ok(dense_fmt, SS24_DENSE, x->k)))
         return SS24_ERR_FORMAT;
     if (x->rows == 0)
-        return empty_operand(energy, nullptr, nullptr, s);
+        return empty_operand(x, energy, nullptr, nullptr, s);
     TilePlan t;
     if (!plan_tile(x, pattern, score, kEnergy, &t))
         return SS24_ERR_CUDA;
@@ -742,11 +761,8 @@ ss24_status ss24_amax(const ss24_operand *x, ss24_pattern pattern, ss24_score sc
     if (!amax_out)
         return SS24_ERR_NULL;
     if (x->rows == 0)
-        return cuda_status(cudaMemsetAsync(amax_out, 0, sizeof(float), s));
-    if (run_amax(x, pattern, score, col_norms, ws, s) != cudaSuccess)
-        return SS24_ERR_CUDA;
-    const float *red = reinterpret_cast<const float *>(static_cast<uint8_t *>(ws) + kWsAmaxReducedOff);
-    return cuda_status(cudaMemcpyAsync(amax_out, red, sizeof(float), cudaMemcpyDeviceToDevice, s));
+        return cuda_status(cudaMemsetAsync(amax_out, 0, nbatch(x) * sizeof(float), s));
+    return cuda_status(run_amax(x, pattern, score, col_norms, ws, s, nullptr, 1.0f, amax_out));
 }
 
 ss24_status ss24_tensor_scale(const ss24_operand *x, ss24_pattern pattern, ss24_score score, const float *col_norms,
@@ -769,7 +785,7 @@ ss24_status ss24_tensor_scale(const ss24_operand *x, ss24_pattern pattern, ss24_
     if (!scale_out)
         return SS24_ERR_NULL;
     if (x->rows == 0)
-        return cuda_status(cudaMemsetAsync(scale_out, 0, sizeof(float), s));
+        return cuda_status(cudaMemsetAsync(scale_out, 0, nbatch(x) * sizeof(float), s));
     const float divisor = kind == SS24_FMT_FP8_E4M3 ? 448.0f : 2688.0f;
     return cuda_status(run_amax(x, pattern, score, col_norms, ws, s, scale_out, divisor));
 }
@@ -912,7 +928,7 @@ ss24_status ss24_prune24_quant_fused_noalloc(const ss24_operand *x, ss24_score s
     if (static_scratch(&scratch) != cudaSuccess)
         return SS24_ERR_CUDA;
     // the error word and the ticket counters must start at zero for this call
-    if (cudaMemsetAsync(scratch, 0, 256, s) != cudaSuccess)
+    if (cudaMemsetAsync(scratch, 0, kWsClearBytes, s) != cudaSuccess)
         return SS24_ERR_CUDA;
     return run_pass(x, SS24_SPARSE_24, score, col_norms, fmt, true, tensor_scale_in, out, energy, scratch,
                     kStaticScratchBytes, s);

@@ -22,11 +22,10 @@ constexpr int kThreads = kConsumers + 32; // + one producer warp
 constexpr int kStageBytes = 16384;
 constexpr int kStages = 4;
 constexpr int kMaxGrid = 1024;            // bound on CTAs (workspace partials)
-constexpr size_t kSmemBytes = kStages * kStageBytes + 1024;
+constexpr size_t kSmemBytes = kStages * kStageBytes + 4096;
 
-// Register-resident rows (one scale per row, rows of at most 4096 bf16 / 2048
-// fp32 elements): one warp per row, 8 warps per CTA.
-constexpr int kRegRowThreads = 256;
+// One scale per long row: one warp per row, 8 warps per CTA.
+constexpr int kRowThreads = 256;
 
 // Strided reduction axis (axis 0: rows contiguous in memory). A stage holds a
 // TMA box of 128 k x (64 bf16 | 32 fp32) rows, 16 KiB; consumers transpose it
@@ -34,25 +33,25 @@ constexpr int kRegRowThreads = 256;
 // 272 / 528 bytes) and process it like an axis-1 tile of width 128.
 constexpr int kAxis0K = 128;
 constexpr size_t kAxis0TBytes = 64 * 136 * 2; // >= 32 * 132 * 4
-constexpr size_t kAxis0SmemBytes = kStages * kStageBytes + kAxis0TBytes + 1024;
+constexpr size_t kAxis0SmemBytes = kStages * kStageBytes + kAxis0TBytes + 4096;
 
-// Row-mode (one scale per row, long rows): a stage holds whole rows.
-constexpr int kRowStageBytes = 49152;
-constexpr int kRowStages = 3;
-constexpr size_t kRowSmemBytes = kRowStages * kRowStageBytes + 2048;
-
-// Workspace layout (bytes): [0, 256) header: error word at 0, the energy
-// ticket counter at 4, the amax ticket counter at 8 (each left at zero by the
-// CTA that finishes last); [256, 256 + 32 * kMaxGrid) energy partials (4
-// doubles per CTA); then amax partials (2 floats per CTA); then the 2 reduced
-// amax floats (kept values, all values).
+// Workspace layout (bytes):
+//   [0, 256)                 header: the error word at 0
+//   energy tickets           kMaxGrid uint32, one per operand of a batch
+//   amax tickets             kMaxGrid uint32, one per operand
+//   energy partials          kMaxGrid x 4 doubles (one slot per CTA)
+//   amax partials            kMaxGrid x 2 floats (one slot per CTA)
+//   reduced amax             kMaxGrid x 2 floats per operand (kept values, all values)
+// Tickets are left at zero by the CTA that finishes last; the header and the
+// tickets (the first kWsClearBytes) must be zero before the first call.
 constexpr size_t kWsErrOff = 0;
-constexpr size_t kWsEnergyTicketOff = 4;
-constexpr size_t kWsAmaxTicketOff = 8;
-constexpr size_t kWsEnergyOff = 256;
+constexpr size_t kWsEnergyTicketOff = 256;
+constexpr size_t kWsAmaxTicketOff = kWsEnergyTicketOff + 4 * kMaxGrid;
+constexpr size_t kWsClearBytes = kWsAmaxTicketOff + 4 * kMaxGrid;
+constexpr size_t kWsEnergyOff = kWsClearBytes;
 constexpr size_t kWsAmaxOff = kWsEnergyOff + 32 * kMaxGrid;
 constexpr size_t kWsAmaxReducedOff = kWsAmaxOff + 8 * kMaxGrid;
-constexpr size_t kWsBytes = kWsAmaxReducedOff + 256;
+constexpr size_t kWsBytes = kWsAmaxReducedOff + 8 * kMaxGrid;
 
 struct QuantSpec {
     int32_t fmt;       // Fmt (kNone .. kMxfp4)
@@ -69,8 +68,8 @@ struct QuantSpec {
 };
 
 struct PassParams {
-    int64_t rows, k;           // logical operand A[rows][k]
-    int64_t n_tiles, n_col_tiles;
+    int64_t rows, k;           // logical operand A[rows][k] (each operand of a batch)
+    int64_t n_tiles, n_col_tiles; // per operand
     int32_t R, W;              // tile rows and width (elements)
     int32_t log2_cpr;          // log2(chunks of 8 per tile row)
     int32_t cpt;               // chunks per consumer thread per tile
@@ -84,12 +83,21 @@ struct PassParams {
     QuantSpec q;               // the stored format (or the sparse side of kEnergy)
     QuantSpec qd;              // kEnergy: the dense side
     double *energy_partials;   // [grid][4] (workspace)
-    double *energy_out;        // caller's ss24_energy (4 doubles) or nullptr: no energies
+    double *energy_out;        // caller's ss24_energy records [batch] or nullptr: no energies
     float *amax_partials;      // kAmax: [grid][2] (workspace)
-    float *amax_out;           // kAmax: 2 floats (kept values, all values)
-    uint32_t *energy_ticket;   // last-CTA-done counters (workspace)
+    float *amax_out;           // kAmax: [batch][2] (kept values, all values)
+    float *amax_user;          // kAmax: caller's [batch] amax of the quantized values, or nullptr
+    uint32_t *energy_ticket;   // last-CTA-done counters, one per operand (workspace)
     uint32_t *amax_ticket;
     int32_t *err;              // workspace error word
+    // batch of operands: CTAs [b * ctas_per_op, (b + 1) * ctas_per_op) serve
+    // operand b, whose input starts x_bstride elements after operand b - 1's
+    // and whose outputs start the given byte strides after operand b - 1's
+    int32_t batch, ctas_per_op;
+    int64_t x_bstride, values_bstride, scales_bstride, meta_bstride;
+    // set per CTA by operand_view(): the operand served and the CTA's index
+    // among that operand's CTAs
+    int32_t op, cta;
 };
 
 cudaError_t launch_ratio(const double *sparse_side, const double *dense_side, double *out, int64_t count,

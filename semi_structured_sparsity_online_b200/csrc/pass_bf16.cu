@@ -6,13 +6,9 @@ const void *tile_kernel_bf16(int pattern, int score, int fmt)
 {
     return tile_kernel<__nv_bfloat16>(pattern, score, fmt);
 }
-const void *row_kernel_bf16(int pattern, int score)
+const void *rowsweep_kernel_bf16(int pattern, int score)
 {
-    return row_kernel_ptr<__nv_bfloat16>(pattern, score);
-}
-const void *rowreg_kernel_bf16(int pattern, int score, int nch)
-{
-    return rowreg_kernel_ptr<__nv_bfloat16>(pattern, score, nch);
+    return rowsweep_kernel_ptr<__nv_bfloat16>(pattern, score);
 }
 const void *axis0_kernel_bf16(int pattern, int score, int fmt)
 {

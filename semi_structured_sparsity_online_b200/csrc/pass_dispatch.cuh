@@ -44,16 +44,16 @@ template <typename T> const void *tile_kernel(int pattern, int score, int fmt)
     return nullptr;
 }
 
-template <typename T> const void *row_kernel_ptr(int pattern, int score)
+template <typename T> const void *rowsweep_kernel_ptr(int pattern, int score)
 {
     if (pattern == kDense)
-        return reinterpret_cast<const void *>(&row_kernel<T, kDense, kMag>);
+        return reinterpret_cast<const void *>(&rowsweep_kernel<T, kDense, kMag>);
     if (pattern == kSparse24)
-        return score == kWanda ? reinterpret_cast<const void *>(&row_kernel<T, kSparse24, kWanda>)
-                               : reinterpret_cast<const void *>(&row_kernel<T, kSparse24, kMag>);
+        return score == kWanda ? reinterpret_cast<const void *>(&rowsweep_kernel<T, kSparse24, kWanda>)
+                               : reinterpret_cast<const void *>(&rowsweep_kernel<T, kSparse24, kMag>);
     if (pattern == kSparse48)
-        return score == kWanda ? reinterpret_cast<const void *>(&row_kernel<T, kSparse48, kWanda>)
-                               : reinterpret_cast<const void *>(&row_kernel<T, kSparse48, kMag>);
+        return score == kWanda ? reinterpret_cast<const void *>(&rowsweep_kernel<T, kSparse48, kWanda>)
+                               : reinterpret_cast<const void *>(&rowsweep_kernel<T, kSparse48, kMag>);
     return nullptr;
 }
 
@@ -90,32 +90,6 @@ template <typename T> const void *axis0_kernel_ptr(int pattern, int score, int f
         return score == kWanda ? axis0_for_fmt<T, kSparse24, kWanda>(fmt) : axis0_for_fmt<T, kSparse24, kMag>(fmt);
     if (pattern == kSparse48)
         return score == kWanda ? axis0_for_fmt<T, kSparse48, kWanda>(fmt) : axis0_for_fmt<T, kSparse48, kMag>(fmt);
-    return nullptr;
-}
-
-template <typename T, int PAT, int SC> const void *rowreg_for_nch(int nch)
-{
-    switch (nch) {
-    case 4:
-        return reinterpret_cast<const void *>(&rowreg_kernel<T, PAT, SC, 4>);
-    case 8:
-        return reinterpret_cast<const void *>(&rowreg_kernel<T, PAT, SC, 8>);
-    case 16:
-        if constexpr (sizeof(T) == 2)
-            return reinterpret_cast<const void *>(&rowreg_kernel<T, PAT, SC, 16>);
-        break;
-    }
-    return nullptr;
-}
-
-template <typename T> const void *rowreg_kernel_ptr(int pattern, int score, int nch)
-{
-    if (pattern == kDense)
-        return rowreg_for_nch<T, kDense, kMag>(nch);
-    if (pattern == kSparse24)
-        return score == kWanda ? rowreg_for_nch<T, kSparse24, kWanda>(nch) : rowreg_for_nch<T, kSparse24, kMag>(nch);
-    if (pattern == kSparse48)
-        return score == kWanda ? rowreg_for_nch<T, kSparse48, kWanda>(nch) : rowreg_for_nch<T, kSparse48, kMag>(nch);
     return nullptr;
 }
 

@@ -6,13 +6,9 @@ const void *tile_kernel_f32(int pattern, int score, int fmt)
 {
     return tile_kernel<float>(pattern, score, fmt);
 }
-const void *row_kernel_f32(int pattern, int score)
+const void *rowsweep_kernel_f32(int pattern, int score)
 {
-    return row_kernel_ptr<float>(pattern, score);
-}
-const void *rowreg_kernel_f32(int pattern, int score, int nch)
-{
-    return rowreg_kernel_ptr<float>(pattern, score, nch);
+    return rowsweep_kernel_ptr<float>(pattern, score);
 }
 const void *axis0_kernel_f32(int pattern, int score, int fmt)
 {

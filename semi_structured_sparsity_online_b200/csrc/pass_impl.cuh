@@ -7,8 +7,8 @@
 // once and writes kept values and indices once), §4 (disjoint error energies),
 // §6 (pairwise 4:8).
 //
-// Structure. Each CTA owns tiles t = blockIdx.x, blockIdx.x + gridDim.x, ...
-// A tile is a TMA box of R rows x W columns of the operand (W a power of two
+// Structure. The CTAs serving one operand of a batch own its tiles t = cta,
+// cta + ctas_per_op, ... A tile is a TMA box of R rows x W columns of the operand (W a power of two
 // <= 256 along k, out-of-range parts zero-filled). One producer lane streams
 // tiles into a ring of kStages shared-memory stages (mbarrier full/empty
 // pairs); 8 consumer warps each read 16-byte chunks of 8 consecutive elements
@@ -326,8 +326,25 @@ __device__ __forceinline__ void store_fp4(uint32_t codes, const QOut &o)
 
 // NVFP4: block of 16 values (16 / VPC lanes), E4M3 block scale over a fp32
 // tensor scale st.
+// Per-CTA NVFP4 table over the 128 non-negative E4M3 block-scale codes c:
+// den[c] = E4M3(c) * s_t (the block's divisor) and inv[c] = RN(1 / den[c]).
+struct NvTable {
+    const float *den, *inv;
+};
+
+// Fills den / inv (256 floats at `t`) for tensor scale st; threads 0..127.
+__device__ __forceinline__ void build_nv_table(float *t, float st, int tid)
+{
+    if (tid < 128) {
+        const float d = __fmul_rn(e4m3_to_f32(static_cast<uint32_t>(tid)), st);
+        t[tid] = d;
+        t[128 + tid] = d != 0.0f ? __frcp_rn(d) : 0.0f;
+    }
+}
+
 template <int VPC, bool STORE>
-__device__ __forceinline__ float quant_nvfp4(const float (&v)[VPC], const Recip &rst, const QOut &o)
+__device__ __forceinline__ float quant_nvfp4(const float (&v)[VPC], const Recip &rst, const QOut &o,
+                                             const NvTable &tb)
 {
     constexpr int kLanes = 16 / VPC;
     const float st = rst.b;
@@ -346,9 +363,14 @@ __device__ __forceinline__ float quant_nvfp4(const float (&v)[VPC], const Recip 
                              : __fdiv_rn(a6, st);
         sb = cvt_e4m3x2(bs, 0.0f) & 0xffu;
     }
-    const float denom = __fmul_rn(e4m3_to_f32(sb), st);
+    Recip rd;
+    rd.b = tb.den[sb];
+    rd.nb = -rd.b;
+    rd.y = tb.inv[sb];
+    rd.fast = rd.b >= 0x1p-60f && rd.b <= 0x1p60f;
+    const float denom = rd.b;
     float q[VPC], d[VPC];
-    quotients<VPC>(v, make_recip(denom), amax, q);
+    quotients<VPC>(v, rd, amax, q);
     const uint32_t codes = pack_e2m1<VPC>(q);
     unpack_e2m1<VPC>(codes, denom, d);
     store_fp4<VPC, STORE>(codes, o);
@@ -385,7 +407,8 @@ __device__ __forceinline__ float quant_mxfp4(const float (&v)[VPC], const QOut &
 
 // Runtime-dispatched quantizer without stores (the energy-only pass).
 template <int VPC>
-__device__ __forceinline__ float quant_energy_only(const float (&v)[VPC], const QuantSpec &q, const Recip &rst)
+__device__ __forceinline__ float quant_energy_only(const float (&v)[VPC], const QuantSpec &q, const Recip &rst,
+                                                   const NvTable &tb)
 {
     QOut o{nullptr, nullptr, 0, 0, 1, false, 0};
     switch (q.fmt) {
@@ -394,7 +417,7 @@ __device__ __forceinline__ float quant_energy_only(const float (&v)[VPC], const 
     case kInt:
         return quant_int<VPC, false>(v, q, o);
     case kNvfp4:
-        return quant_nvfp4<VPC, false>(v, rst, o);
+        return quant_nvfp4<VPC, false>(v, rst, o, tb);
     case kMxfp4:
         return quant_mxfp4<VPC, false>(v, o);
     default:
@@ -435,7 +458,9 @@ __device__ __forceinline__ void scores(const float (&x)[8], const float *norms, 
 template <typename T, int PAT, int SCORE, int FMT>
 __device__ __forceinline__ void process_chunk(const PassParams &p, const float (&x)[8], int64_t row,
                                               int64_t col, int lane, const Recip &rst, const Recip &rstd,
-                                              Acc &acc, float row_amax = -1.0f, const RowScale *rs = nullptr)
+                                              Acc &acc, float row_amax = -1.0f, const RowScale *rs = nullptr,
+                                              const NvTable &tb = NvTable{nullptr, nullptr},
+                                              const NvTable &tbd = NvTable{nullptr, nullptr})
 {
     constexpr int VPC = PAT == kDense ? 8 : 4;
     const bool in_k = col < p.k;
@@ -551,12 +576,12 @@ __device__ __forceinline__ void process_chunk(const PassParams &p, const float (
     } else if constexpr (FMT == kInt) {
         eq = quant_int<VPC, true>(v, p.q, o, row_amax, rs);
     } else if constexpr (FMT == kNvfp4) {
-        eq = quant_nvfp4<VPC, true>(v, rst, o);
+        eq = quant_nvfp4<VPC, true>(v, rst, o, tb);
     } else if constexpr (FMT == kMxfp4) {
         eq = quant_mxfp4<VPC, true>(v, o);
     } else if constexpr (FMT == kEnergy) {
-        eq = quant_energy_only<VPC>(v, p.q, rst);
-        acc.eqd += quant_energy_only<8>(x, p.qd, rstd);
+        eq = quant_energy_only<VPC>(v, p.q, rst, tb);
+        acc.eqd += quant_energy_only<8>(x, p.qd, rstd, tbd);
     }
     if constexpr (PAT == kDense)
         acc.eqd += eq;
@@ -573,6 +598,42 @@ __device__ __forceinline__ void record_error(int32_t *err, int32_t code)
     atomicCAS(err, 0, code);
 }
 
+// The parameters as seen by the CTAs serving one operand of a batch: every
+// per-operand pointer offset to that operand, and the CTA's index among the
+// operand's CTAs.
+__device__ __forceinline__ PassParams operand_view(const PassParams &p)
+{
+    PassParams q = p;
+    const int b = static_cast<int>(blockIdx.x) / p.ctas_per_op;
+    q.op = b;
+    q.cta = static_cast<int>(blockIdx.x) - b * p.ctas_per_op;
+    if (p.values)
+        q.values = static_cast<uint8_t *>(p.values) + b * p.values_bstride;
+    if (p.scales)
+        q.scales = static_cast<uint8_t *>(p.scales) + b * p.scales_bstride;
+    if (p.meta)
+        q.meta = p.meta + b * p.meta_bstride;
+    if (p.energy_out)
+        q.energy_out = p.energy_out + 4 * b;
+    if (p.amax_user)
+        q.amax_user = p.amax_user + b;
+    q.energy_partials = p.energy_partials + 4 * static_cast<int64_t>(b) * p.ctas_per_op;
+    q.amax_partials = p.amax_partials + 2 * static_cast<int64_t>(b) * p.ctas_per_op;
+    q.amax_out = p.amax_out + 2 * b;
+    q.energy_ticket = p.energy_ticket + b;
+    q.amax_ticket = p.amax_ticket + b;
+    QuantSpec *qs[2] = {&q.q, &q.qd};
+    for (int i = 0; i < 2; ++i) {
+        if (qs[i]->scale_in)
+            qs[i]->scale_in += b;
+        if (qs[i]->scale_out)
+            qs[i]->scale_out += b;
+        if (qs[i]->amax_reduced)
+            qs[i]->amax_reduced += 2 * b;
+    }
+    return q;
+}
+
 // Tensor scale of a per-tensor format: the given one, or amax / divisor.
 __device__ __forceinline__ float tensor_scale(const QuantSpec &q)
 {
@@ -583,9 +644,10 @@ __device__ __forceinline__ float tensor_scale(const QuantSpec &q)
     return __fdiv_rn(*q.amax_reduced, q.divisor);
 }
 
-// Grid-wide energy reduction: per-CTA binary64 partials go to the workspace;
-// the CTA that takes the last ticket sums them in fixed order, writes the
-// caller's 4-double record and resets the ticket. Called by all consumers.
+// Energy reduction over the CTAs of one operand: per-CTA binary64 partials go
+// to the workspace; the CTA that takes the operand's last ticket sums them in
+// fixed order, writes the caller's 4-double record and resets the ticket.
+// Called by all consumers, with the operand's view of the parameters.
 __device__ __forceinline__ void grid_reduce_energy(const PassParams &p, double e_total, double e_prune, double e_q,
                                                    double e_qd, double *red, uint32_t *flag, int tid, int lane,
                                                    int warp)
@@ -608,10 +670,10 @@ __device__ __forceinline__ void grid_reduce_energy(const PassParams &p, double e
                 sum[f] += red[w * 4 + f];
 #pragma unroll
         for (int f = 0; f < 4; ++f)
-            p.energy_partials[blockIdx.x * 4 + f] = sum[f];
+            p.energy_partials[p.cta * 4 + f] = sum[f];
         __threadfence();
         const uint32_t ticket = atomicAdd(p.energy_ticket, 1u);
-        *flag = ticket == gridDim.x - 1;
+        *flag = ticket == static_cast<uint32_t>(p.ctas_per_op - 1);
     }
     named_barrier_sync(1, kConsumers);
     if (*flag) {
@@ -619,7 +681,7 @@ __device__ __forceinline__ void grid_reduce_energy(const PassParams &p, double e
         // thread tid sums field (tid & 3) over CTAs (tid >> 2), (tid >> 2) + 64, ...
         const int f = tid & 3;
         double acc_f = 0.0;
-        for (int i = tid >> 2; i < static_cast<int>(gridDim.x); i += kConsumers / 4)
+        for (int i = tid >> 2; i < p.ctas_per_op; i += kConsumers / 4)
             acc_f += __ldcg(p.energy_partials + 4 * i + f);
         // lanes holding the same field differ in lane bits 2..4
         for (int off = 16; off >= 4; off >>= 1)
@@ -639,10 +701,10 @@ __device__ __forceinline__ void grid_reduce_energy(const PassParams &p, double e
     }
 }
 
-// Grid-wide amax reduction of the kept values (a) and of all values (b): the
-// same last-CTA scheme as the energies. Writes amax_out[0] (the amax of the
-// values the pass quantizes), amax_out[1] (all values) and, when asked, the
-// per-tensor scale amax_out[0] / divisor. Called by all consumers.
+// Amax reduction over the CTAs of one operand, of the kept values (a) and of
+// all values (b): the same last-CTA scheme as the energies. Writes amax_out[0]
+// (the amax of the values the pass quantizes), amax_out[1] (all values) and,
+// when asked, the caller's amax and the per-tensor scale amax / divisor.
 template <int PAT>
 __device__ __forceinline__ void grid_reduce_amax(const PassParams &p, float a, float b, float *fred, uint32_t *flag,
                                                  int tid, int lane, int warp)
@@ -661,17 +723,17 @@ __device__ __forceinline__ void grid_reduce_amax(const PassParams &p, float a, f
             a = fmaxf(a, fred[w * 2]);
             b = fmaxf(b, fred[w * 2 + 1]);
         }
-        p.amax_partials[blockIdx.x * 2] = a;
-        p.amax_partials[blockIdx.x * 2 + 1] = b;
+        p.amax_partials[p.cta * 2] = a;
+        p.amax_partials[p.cta * 2 + 1] = b;
         __threadfence();
         const uint32_t ticket = atomicAdd(p.amax_ticket, 1u);
-        *flag = ticket == gridDim.x - 1;
+        *flag = ticket == static_cast<uint32_t>(p.ctas_per_op - 1);
     }
     named_barrier_sync(1, kConsumers);
     if (*flag) {
         __threadfence();
         float ka = 0.0f, kb = 0.0f;
-        for (int i = tid; i < static_cast<int>(gridDim.x); i += kConsumers) {
+        for (int i = tid; i < p.ctas_per_op; i += kConsumers) {
             ka = fmaxf(ka, __ldcg(p.amax_partials + 2 * i));
             kb = fmaxf(kb, __ldcg(p.amax_partials + 2 * i + 1));
         }
@@ -693,6 +755,8 @@ __device__ __forceinline__ void grid_reduce_amax(const PassParams &p, float a, f
             const float a0 = PAT == kDense ? kb : ka;
             p.amax_out[0] = a0;
             p.amax_out[1] = kb;
+            if (p.amax_user)
+                *p.amax_user = a0;
             if (p.q.scale_out)
                 *p.q.scale_out = __fdiv_rn(a0, p.q.divisor);
             *p.amax_ticket = 0;
@@ -706,7 +770,7 @@ __device__ __forceinline__ void producer(const CUtensorMap *map, const PassParam
     const uint64_t policy = l2_evict_first_policy();
     uint32_t it = 0;
     bool failed = false;
-    for (int64_t t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++it) {
+    for (int64_t t = p.cta; t < p.n_tiles; t += p.ctas_per_op, ++it) {
         const int s = it % kStages;
         const uint32_t use = it / kStages;
         if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1)) {
@@ -717,11 +781,11 @@ __device__ __forceinline__ void producer(const CUtensorMap *map, const PassParam
         mbar_arrive_expect_tx(&full[s], p.tile_bytes);
         const int64_t rt = t / p.n_col_tiles, ct = t - rt * p.n_col_tiles;
         const int32_t ck = static_cast<int32_t>(ct * p.W), cr = static_cast<int32_t>(rt * p.R);
-        // TMA coordinates are {inner (contiguous), outer}
+        // TMA coordinates are {inner (contiguous), outer, operand}
         if (p.axis == 1)
-            tma_load_2d(stages + s * kStageBytes, map, ck, cr, &full[s], policy);
+            tma_load_3d(stages + s * kStageBytes, map, ck, cr, p.op, &full[s], policy);
         else
-            tma_load_2d(stages + s * kStageBytes, map, cr, ck, &full[s], policy);
+            tma_load_3d(stages + s * kStageBytes, map, cr, ck, p.op, &full[s], policy);
     }
     if (failed) {
         // let the copies already issued land before the CTA can exit
@@ -733,9 +797,10 @@ __device__ __forceinline__ void producer(const CUtensorMap *map, const PassParam
 }
 
 template <typename T, int PAT, int SCORE, int FMT>
-__global__ void __launch_bounds__(kThreads, 1) pass_kernel(const __grid_constant__ CUtensorMap map,
-                                                           const PassParams p)
+__global__ void __launch_bounds__(kThreads, 3) pass_kernel(const __grid_constant__ CUtensorMap map,
+                                                           const PassParams pk)
 {
+    const PassParams p = operand_view(pk);
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t *stages = smem;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + kStages * kStageBytes);
@@ -766,12 +831,19 @@ __global__ void __launch_bounds__(kThreads, 1) pass_kernel(const __grid_constant
     float st = 0.0f, std_ = 0.0f;
     if constexpr (FMT == kFp8 || FMT == kNvfp4 || FMT == kEnergy) {
         st = tensor_scale(p.q);
-        if (blockIdx.x == 0 && tid == 0 && p.q.scale_out)
+        if (p.cta == 0 && tid == 0 && p.q.scale_out)
             *p.q.scale_out = st;
     }
     if constexpr (FMT == kEnergy)
         std_ = tensor_scale(p.qd);
     const Recip rst = make_recip(st), rstd = make_recip(std_);
+    float *nvt = reinterpret_cast<float *>(flag + 4); // 2 x 256 floats
+    if constexpr (FMT == kNvfp4 || FMT == kEnergy) {
+        build_nv_table(nvt, st, tid);
+        build_nv_table(nvt + 256, std_, tid);
+        named_barrier_sync(1, kConsumers);
+    }
+    const NvTable tb{nvt, nvt + 128}, tbd{nvt + 256, nvt + 384};
 
     using E = Elem<T>;
     const int cpr_mask = (1 << p.log2_cpr) - 1;
@@ -779,7 +851,7 @@ __global__ void __launch_bounds__(kThreads, 1) pass_kernel(const __grid_constant
     double e_total = 0.0, e_prune = 0.0, e_q = 0.0, e_qd = 0.0;
     Acc acc{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     uint32_t it = 0;
-    for (int64_t t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++it) {
+    for (int64_t t = p.cta; t < p.n_tiles; t += p.ctas_per_op, ++it) {
         const int s = it % kStages;
         if (!mbar_wait(&full[s], (it / kStages) & 1)) {
             record_error(p.err, 2);
@@ -806,7 +878,7 @@ __global__ void __launch_bounds__(kThreads, 1) pass_kernel(const __grid_constant
                 const int64_t col = col0 + ((j & cpr_mask) << 3);
                 float x[8];
                 E::unpack(raw[i], x);
-                process_chunk<T, PAT, SCORE, FMT>(p, x, row, col, lane, rst, rstd, acc);
+                process_chunk<T, PAT, SCORE, FMT>(p, x, row, col, lane, rst, rstd, acc, -1.0f, nullptr, tb, tbd);
             }
         }
         if constexpr (FMT != kAmax) {
@@ -829,158 +901,21 @@ __global__ void __launch_bounds__(kThreads, 1) pass_kernel(const __grid_constant
 }
 
 // ---------------------------------------------------------------------------
-// row mode: INT with one scale per row when a row does not fit one warp's
-// span (k > 256, or k not a power of two). A stage holds R whole rows, loaded
-// as ceil(k / W) TMA boxes of [R rows x W columns] (W = min(256, next power of
-// two >= k)) laid out [box][row][W] in shared memory.
-// Warp w owns rows w, w + 8, ... of the stage: a first sweep over the row takes
-// the amax of the values to quantize, a second sweep quantizes and stores.
+// one scale per row (INT with group 0) when a row does not fit one warp's
+// 256-element span. One warp per row, two sweeps over the row in global
+// memory: the first streams it through L1-caching loads (eight 16-byte chunks
+// per lane in flight) and takes the amax of the values to quantize; the second
+// reads it again (from L1 or L2; HBM sees one read) and quantizes with the
+// row's scale. The code stays small and registers few, so many warps are
+// resident to cover the load latency.
 // ---------------------------------------------------------------------------
 
-// Chunk c of row r in a row-mode stage laid out [box][row][W]; zeros past the
-// padded row end (lanes without a chunk still take part in warp shuffles).
-template <typename T>
-__device__ __forceinline__ void load_row_chunk(const uint8_t *tile, int c, int r, int R, int cpb_log2, bool have,
-                                               float (&x)[8])
-{
-    if (have) {
-        const int box = c >> cpb_log2, cc = c & ((1 << cpb_log2) - 1);
-        Elem<T>::unpack(Elem<T>::load(tile, ((box * R + r) << cpb_log2) + cc), x);
-    } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            x[i] = 0.0f;
-    }
-}
-
-__device__ __forceinline__ void row_producer(const CUtensorMap *map, const PassParams &p, uint8_t *stages,
-                                             uint64_t *full, uint64_t *empty, int nbox, int esize)
-{
-    const uint64_t policy = l2_evict_first_policy();
-    uint32_t it = 0;
-    bool failed = false;
-    const int box_bytes = p.R * p.W * esize;
-    for (int64_t t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++it) {
-        const int s = it % kRowStages;
-        const uint32_t use = it / kRowStages;
-        if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1)) {
-            record_error(p.err, 3);
-            failed = true;
-            break;
-        }
-        mbar_arrive_expect_tx(&full[s], p.tile_bytes);
-        for (int b = 0; b < nbox; ++b)
-            tma_load_2d(stages + s * kRowStageBytes + b * box_bytes, map, b * p.W,
-                        static_cast<int32_t>(t * p.R), &full[s], policy);
-    }
-    if (failed) {
-        for (int s = 0; s < kRowStages && s < static_cast<int>(it); ++s) {
-            const uint32_t last_use = (it - 1 - ((it - 1 - s) % kRowStages)) / kRowStages;
-            (void)mbar_wait(&full[s], last_use & 1);
-        }
-    }
-}
-
-template <typename T, int PAT, int SCORE>
-__global__ void __launch_bounds__(kThreads, 1) row_kernel(const __grid_constant__ CUtensorMap map,
-                                                          const PassParams p)
-{
-    extern __shared__ __align__(1024) uint8_t smem[];
-    uint8_t *stages = smem;
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kRowStages * kRowStageBytes);
-    uint64_t *empty = full + kRowStages;
-    double *red = reinterpret_cast<double *>(empty + kRowStages);
-    uint32_t *flag = reinterpret_cast<uint32_t *>(red + kConsumerWarps * 4);
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int nbox = static_cast<int>((p.k + p.W - 1) / p.W);
-    if (tid == 0) {
-        for (int s = 0; s < kRowStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kConsumerWarps);
-        }
-        fence_barrier_init();
-    }
-    __syncthreads();
-    grid_dependency_wait();
-    grid_dependents_launch();
-    if (warp == kConsumerWarps) {
-        if (lane == 0)
-            row_producer(&map, p, stages, full, empty, nbox, static_cast<int>(sizeof(T)));
-        return;
-    }
-
-    const Recip no_recip = make_recip(0.0f);
-    const int cpb_log2 = p.log2_cpr;            // log2(chunks per box row), box width = p.W
-    const int nchunks = nbox << cpb_log2;        // chunks per (padded) row
-    double e_total = 0.0, e_prune = 0.0, e_q = 0.0, e_qd = 0.0;
-    uint32_t it = 0;
-    for (int64_t t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++it) {
-        const int s = it % kRowStages;
-        if (!mbar_wait(&full[s], (it / kRowStages) & 1)) {
-            record_error(p.err, 4);
-            break;
-        }
-        const uint8_t *tile = stages + s * kRowStageBytes;
-        for (int r = warp; r < p.R; r += kConsumerWarps) {
-            const int64_t row = t * p.R + r;
-            // chunk c of row r sits at chunk index (c / 32 * R + r) * 32 + c % 32
-            float amax = 0.0f;
-            for (int c0 = 0; c0 < nchunks; c0 += 32) {
-                const int c = c0 + lane;
-                float x[8];
-                load_row_chunk<T>(tile, c, r, p.R, cpb_log2, c < nchunks, x);
-                if constexpr (PAT == kDense || SCORE == kMag) {
-                    // for the magnitude score the kept amax equals the amax of all
-                    amax = fmaxf(amax, local_amax<8>(x));
-                } else {
-                    Acc a{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                    process_chunk<T, PAT, SCORE, kAmax>(p, x, row, static_cast<int64_t>(c) * 8, lane, no_recip,
-                                                        no_recip, a);
-                    amax = fmaxf(amax, a.amax_kept);
-                }
-            }
-            amax = group_amax(amax, 32);
-            Acc acc{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            for (int c0 = 0; c0 < nchunks; c0 += 32) {
-                const int c = c0 + lane;
-                float x[8];
-                load_row_chunk<T>(tile, c, r, p.R, cpb_log2, c < nchunks, x);
-                process_chunk<T, PAT, SCORE, kInt>(p, x, row, static_cast<int64_t>(c) * 8, lane, no_recip, no_recip, acc,
-                                                   amax);
-            }
-            if (lane == 0 && row < p.rows)
-                static_cast<float *>(p.scales)[row] = __fdiv_rn(amax, p.q.qmax);
-            e_total += acc.et;
-            e_prune += acc.ep;
-            e_q += acc.eq;
-            e_qd += acc.eqd;
-        }
-        __syncwarp();
-        if (lane == 0)
-            mbar_arrive(&empty[s]);
-    }
-
-    if (!p.energy_out)
-        return;
-    grid_reduce_energy(p, e_total, e_prune, e_q, e_qd, red, flag, tid, lane, warp);
-}
-
-// ---------------------------------------------------------------------------
-// register-resident rows: INT with one scale per row for rows that fit in a
-// warp's registers (k <= 32 * 8 * NCH). One warp per row: every lane loads its
-// NCH chunks (lane, lane + 32, ...) with streaming 16-byte loads, all in
-// flight at once; the row amax is a warp reduction over registers; the codes
-// are computed from the same registers. No shared-memory staging and no second
-// read of the row.
-// ---------------------------------------------------------------------------
-
-template <typename T> struct RegChunk;
-template <> struct RegChunk<__nv_bfloat16> {
+template <typename T> struct RowChunk;
+template <> struct RowChunk<__nv_bfloat16> {
     uint4 v;
     __device__ __forceinline__ void load(const void *row, int c)
     {
-        v = __ldcs(reinterpret_cast<const uint4 *>(row) + c);
+        v = __ldg(reinterpret_cast<const uint4 *>(row) + c);
     }
     __device__ __forceinline__ void unpack(float (&x)[8]) const
     {
@@ -988,12 +923,12 @@ template <> struct RegChunk<__nv_bfloat16> {
         Elem<__nv_bfloat16>::unpack(r, x);
     }
 };
-template <> struct RegChunk<float> {
+template <> struct RowChunk<float> {
     float4 a, b;
     __device__ __forceinline__ void load(const void *row, int c)
     {
-        a = __ldcs(reinterpret_cast<const float4 *>(row) + 2 * c);
-        b = __ldcs(reinterpret_cast<const float4 *>(row) + 2 * c + 1);
+        a = __ldg(reinterpret_cast<const float4 *>(row) + 2 * c);
+        b = __ldg(reinterpret_cast<const float4 *>(row) + 2 * c + 1);
     }
     __device__ __forceinline__ void unpack(float (&x)[8]) const
     {
@@ -1002,10 +937,11 @@ template <> struct RegChunk<float> {
     }
 };
 
-template <typename T, int PAT, int SCORE, int NCH>
-__global__ void __launch_bounds__(kRegRowThreads) rowreg_kernel(const T *__restrict__ x, int64_t ld,
-                                                                const PassParams p)
+template <typename T, int PAT, int SCORE>
+__global__ void __launch_bounds__(kRowThreads) rowsweep_kernel(const T *__restrict__ x, int64_t ld,
+                                                               const PassParams pk)
 {
+    const PassParams p = operand_view(pk);
     __shared__ double red[kConsumerWarps * 4];
     __shared__ uint32_t flag;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1014,30 +950,32 @@ __global__ void __launch_bounds__(kRegRowThreads) rowreg_kernel(const T *__restr
     const int nchunks = static_cast<int>(p.k / 8);
     const Recip no_recip = make_recip(0.0f);
     double e_total = 0.0, e_prune = 0.0, e_q = 0.0, e_qd = 0.0;
-    for (int64_t row = static_cast<int64_t>(blockIdx.x) * kConsumerWarps + warp; row < p.rows;
-         row += static_cast<int64_t>(gridDim.x) * kConsumerWarps) {
-        const T *xr = x + row * ld;
-        RegChunk<T> buf[NCH];
-#pragma unroll
-        for (int j = 0; j < NCH; ++j)
-            if (lane + 32 * j < nchunks)
-                buf[j].load(xr, lane + 32 * j);
-        // the row amax of the values to quantize (for the magnitude score the
-        // kept amax equals the amax of all values)
+    for (int64_t row = static_cast<int64_t>(p.cta) * kConsumerWarps + warp; row < p.rows;
+         row += static_cast<int64_t>(p.ctas_per_op) * kConsumerWarps) {
+        const T *xr = x + p.op * p.x_bstride + row * ld;
+        // sweep 1: the row amax of the values to quantize (for the magnitude
+        // score the kept amax equals the amax of all values)
         float amax = 0.0f;
+        for (int c0 = 0; c0 < nchunks; c0 += 256) {
+            RowChunk<T> buf[8];
 #pragma unroll
-        for (int j = 0; j < NCH; ++j) {
-            const int c = lane + 32 * j;
-            if (c < nchunks) {
-                float xv[8];
-                buf[j].unpack(xv);
-                if constexpr (PAT == kDense || SCORE == kMag) {
-                    amax = fmaxf(amax, local_amax<8>(xv));
-                } else {
-                    Acc a{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                    process_chunk<T, PAT, SCORE, kAmax>(p, xv, row, static_cast<int64_t>(c) * 8, lane, no_recip,
-                                                        no_recip, a);
-                    amax = fmaxf(amax, a.amax_kept);
+            for (int u = 0; u < 8; ++u)
+                if (c0 + 32 * u + lane < nchunks)
+                    buf[u].load(xr, c0 + 32 * u + lane);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int c = c0 + 32 * u + lane;
+                if (c < nchunks) {
+                    float xv[8];
+                    buf[u].unpack(xv);
+                    if constexpr (PAT == kDense || SCORE == kMag) {
+                        amax = fmaxf(amax, local_amax<8>(xv));
+                    } else {
+                        Acc a{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                        process_chunk<T, PAT, SCORE, kAmax>(p, xv, row, static_cast<int64_t>(c) * 8, lane,
+                                                            no_recip, no_recip, a);
+                        amax = fmaxf(amax, a.amax_kept);
+                    }
                 }
             }
         }
@@ -1047,16 +985,26 @@ __global__ void __launch_bounds__(kRegRowThreads) rowreg_kernel(const T *__restr
         rs.amax = amax;
         rs.scale = int_scale(amax, p.q);
         rs.rc = make_recip(rs.scale);
+        // sweep 2: codes, metadata and energies; every lane takes part in each
+        // step (4:8 metadata pairs lanes through a shuffle)
         Acc acc{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int c0 = 0; c0 < nchunks; c0 += 64) {
+            RowChunk<T> buf[2];
 #pragma unroll
-        for (int j = 0; j < NCH; ++j) {
-            const int c = lane + 32 * j;
-            // every lane takes part (4:8 metadata pairs lanes through a shuffle)
-            float xv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            if (c < nchunks)
-                buf[j].unpack(xv);
-            process_chunk<T, PAT, SCORE, kInt>(p, xv, row, static_cast<int64_t>(c) * 8, lane, no_recip, no_recip,
-                                               acc, amax, &rs);
+            for (int u = 0; u < 2; ++u)
+                if (c0 + 32 * u + lane < nchunks)
+                    buf[u].load(xr, c0 + 32 * u + lane);
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int c = c0 + 32 * u + lane;
+                if (c0 + 32 * u < nchunks) {
+                    float xv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    if (c < nchunks)
+                        buf[u].unpack(xv);
+                    process_chunk<T, PAT, SCORE, kInt>(p, xv, row, static_cast<int64_t>(c) * 8, lane, no_recip,
+                                                       no_recip, acc, amax, &rs);
+                }
+            }
         }
         if (lane == 0)
             static_cast<float *>(p.scales)[row] = rs.scale;
@@ -1164,8 +1112,9 @@ template <> struct Axis0<float> {
 
 template <typename T, int PAT, int SCORE, int FMT>
 __global__ void __launch_bounds__(kThreads, 1) axis0_kernel(const __grid_constant__ CUtensorMap map,
-                                                            const PassParams p)
+                                                            const PassParams pk)
 {
+    const PassParams p = operand_view(pk);
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t *stages = smem;
     uint8_t *Tb = smem + kStages * kStageBytes;
@@ -1196,17 +1145,24 @@ __global__ void __launch_bounds__(kThreads, 1) axis0_kernel(const __grid_constan
     float st = 0.0f, std_ = 0.0f;
     if constexpr (FMT == kFp8 || FMT == kNvfp4 || FMT == kEnergy) {
         st = tensor_scale(p.q);
-        if (blockIdx.x == 0 && tid == 0 && p.q.scale_out)
+        if (p.cta == 0 && tid == 0 && p.q.scale_out)
             *p.q.scale_out = st;
     }
     if constexpr (FMT == kEnergy)
         std_ = tensor_scale(p.qd);
     const Recip rst = make_recip(st), rstd = make_recip(std_);
+    float *nvt = reinterpret_cast<float *>(ready + 4); // 2 x 256 floats
+    if constexpr (FMT == kNvfp4 || FMT == kEnergy) {
+        build_nv_table(nvt, st, tid);
+        build_nv_table(nvt + 256, std_, tid);
+        named_barrier_sync(1, kConsumers);
+    }
+    const NvTable tb{nvt, nvt + 128}, tbd{nvt + 256, nvt + 384};
     using A0 = Axis0<T>;
     double e_total = 0.0, e_prune = 0.0, e_q = 0.0, e_qd = 0.0;
     Acc acc{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     uint32_t it = 0;
-    for (int64_t t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++it) {
+    for (int64_t t = p.cta; t < p.n_tiles; t += p.ctas_per_op, ++it) {
         const int s = it % kStages;
         // one thread waits for the stage and tells the others, so that every
         // consumer leaves the loop together if the wait gives up
@@ -1241,7 +1197,7 @@ __global__ void __launch_bounds__(kThreads, 1) axis0_kernel(const __grid_constan
                 float x[8];
                 Elem<T>::unpack(raw[i], x);
                 process_chunk<T, PAT, SCORE, FMT>(p, x, row0 + (j >> 4), col0 + ((j & 15) << 3), lane, rst,
-                                                  rstd, acc);
+                                                  rstd, acc, -1.0f, nullptr, tb, tbd);
             }
         }
         if constexpr (FMT != kAmax) {

@@ -39,7 +39,8 @@ class Format(ctypes.Structure):
 
 class Operand(ctypes.Structure):
     _fields_ = [("x", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("axis", ctypes.c_int32),
-                ("rows", ctypes.c_int64), ("k", ctypes.c_int64), ("ld", ctypes.c_int64)]
+                ("rows", ctypes.c_int64), ("k", ctypes.c_int64), ("ld", ctypes.c_int64),
+                ("batch", ctypes.c_int64), ("batch_stride", ctypes.c_int64)]
 
 
 class Outputs(ctypes.Structure):
@@ -123,23 +124,26 @@ def make_format(fmt="none", bits=8, group=0, pack4=False) -> Format:
 
 
 def make_operand(x: torch.Tensor, axis: int = 1, rows=None, k=None) -> Operand:
-    """Operand descriptor of a 2-D CUDA tensor. axis 1: x is [rows, ld] with k
-    contiguous; axis 0: x is [k, ld] holding A[r][c] at x[c][r]."""
+    """Operand descriptor of a CUDA tensor. 2-D: one operand; axis 1: x is
+    [rows, ld] with k contiguous; axis 0: x is [k, ld] holding A[r][c] at
+    x[c][r]. 3-D [B, ., .]: a batch of B such operands (x.stride(0) apart)."""
     if x.dtype == torch.bfloat16:
         dt = BF16
     elif x.dtype == torch.float32:
         dt = F32
     else:
         raise TypeError("operand must be bfloat16 or float32")
-    if x.dim() != 2 or x.stride(1) != 1:
-        raise ValueError("operand must be 2-D with a contiguous last dimension")
+    if x.dim() not in (2, 3) or x.stride(-1) != 1:
+        raise ValueError("operand must be 2-D or 3-D with a contiguous last dimension")
+    batch, bstride = (x.shape[0], x.stride(0)) if x.dim() == 3 else (1, 0)
+    m = x[0] if x.dim() == 3 else x
     if axis == 1:
-        r = x.shape[0] if rows is None else rows
-        kk = x.shape[1] if k is None else k
+        r = m.shape[0] if rows is None else rows
+        kk = m.shape[1] if k is None else k
     else:
-        kk = x.shape[0] if k is None else k
-        r = x.shape[1] if rows is None else rows
-    return Operand(x.data_ptr(), dt, axis, r, kk, x.stride(0))
+        kk = m.shape[0] if k is None else k
+        r = m.shape[1] if rows is None else rows
+    return Operand(x.data_ptr(), dt, axis, r, kk, m.stride(0), batch, bstride)
 
 
 class Workspace:
@@ -173,45 +177,61 @@ def default_workspace(device=None) -> Workspace:
     return _default_ws[dev]
 
 
-def _alloc_outputs(x_rows, k, pattern, fmt: Format, in_dtype, device):
+def _alloc_outputs(x_rows, k, pattern, fmt: Format, in_dtype, device, batch=None):
+    """Output tensors of a pass; with `batch` every output gets a leading
+    [batch] dimension (the per-operand outputs packed one after the other)."""
     sparse = pattern != DENSE
     n = k // 2 if sparse else k
+    lead = () if batch is None else (batch,)
     out = {}
+
+    def empty(shape, dtype):
+        return torch.empty(lead + shape, dtype=dtype, device=device)
+
     if fmt.kind == FMT_NONE:
-        out["values"] = torch.empty((x_rows, n), dtype=in_dtype, device=device)
+        out["values"] = empty((x_rows, n), in_dtype)
     elif fmt.kind == FMT_FP8:
-        out["values"] = torch.empty((x_rows, n), dtype=torch.uint8, device=device)
+        out["values"] = empty((x_rows, n), torch.uint8)
     elif fmt.kind == FMT_INT:
         if fmt.pack4:
-            out["values"] = torch.empty((x_rows, n // 2), dtype=torch.uint8, device=device)
+            out["values"] = empty((x_rows, n // 2), torch.uint8)
         else:
-            out["values"] = torch.empty((x_rows, n), dtype=torch.int16 if fmt.bits > 8 else torch.int8,
-                                        device=device)
+            out["values"] = empty((x_rows, n), torch.int16 if fmt.bits > 8 else torch.int8)
         g = fmt.group or n
-        out["scales"] = torch.empty((x_rows, n // g), dtype=torch.float32, device=device)
+        out["scales"] = empty((x_rows, n // g), torch.float32)
     elif fmt.kind in (FMT_NVFP4, FMT_MXFP4):
-        out["values"] = torch.empty((x_rows, n // 2), dtype=torch.uint8, device=device)
+        out["values"] = empty((x_rows, n // 2), torch.uint8)
         blk = 16 if fmt.kind == FMT_NVFP4 else 32
-        out["scales"] = torch.empty((x_rows, n // blk), dtype=torch.uint8, device=device)
+        out["scales"] = empty((x_rows, n // blk), torch.uint8)
     if fmt.kind in (FMT_FP8, FMT_NVFP4):
-        out["tensor_scale"] = torch.empty(1, dtype=torch.float32, device=device)
+        out["tensor_scale"] = empty((1,), torch.float32) if batch is None else torch.empty(
+            (batch,), dtype=torch.float32, device=device)
     if sparse:
-        out["meta"] = torch.empty((x_rows, k // (16 if pattern == SPARSE_48 else 8)), dtype=torch.uint8,
-                                  device=device)
+        out["meta"] = empty((x_rows, k // (16 if pattern == SPARSE_48 else 8)), torch.uint8)
     return out
+
+
+def _lead(op):
+    return None if op.batch <= 1 and op.batch_stride == 0 else op.batch
+
+
+def _energy(op, device):
+    b = _lead(op)
+    return torch.zeros((4,) if b is None else (b, 4), dtype=torch.float64, device=device)
 
 
 def run(x: torch.Tensor, pattern=SPARSE_24, fmt="none", bits=8, group=0, pack4=False, score="mag",
         col_norms=None, tensor_scale=None, energy=True, axis=1, ws=None, stream=None, out=None):
     """One pass through the matching C entry point. Returns a dict of output
     tensors (``values``, ``scales``, ``tensor_scale``, ``meta``) and ``energy``
-    (float64[4] on the device: e_total, e_prune, e_quant, e_quant_dense)."""
+    (float64[4] on the device: e_total, e_prune, e_quant, e_quant_dense). A
+    3-D x is a batch: every output and the energies get a leading [B]."""
     f = make_format(fmt, bits, group, pack4)
     op = make_operand(x, axis)
     sc = _SCORE[score] if isinstance(score, str) else int(score)
     if out is None:
-        out = _alloc_outputs(op.rows, op.k, pattern, f, x.dtype, x.device)
-    e = torch.zeros(4, dtype=torch.float64, device=x.device) if energy is True else energy
+        out = _alloc_outputs(op.rows, op.k, pattern, f, x.dtype, x.device, _lead(op))
+    e = _energy(op, x.device) if energy is True else energy
     if e is not None and e is not False:
         out["energy"] = e
     else:
@@ -246,11 +266,11 @@ def run(x: torch.Tensor, pattern=SPARSE_24, fmt="none", bits=8, group=0, pack4=F
 
 def error_energy(x, pattern=SPARSE_24, sparse_fmt=("none",), dense_fmt=("int", 8, 0), score="mag",
                  col_norms=None, sparse_scale=None, dense_scale=None, axis=1, ws=None, stream=None, energy=None):
-    """Read-only energy pass; returns float64[4] on the device."""
+    """Read-only energy pass; returns float64[4] (or [B, 4]) on the device."""
     sf = make_format(*sparse_fmt) if isinstance(sparse_fmt, tuple) else sparse_fmt
     df = make_format(*dense_fmt) if isinstance(dense_fmt, tuple) else dense_fmt
     op = make_operand(x, axis)
-    e = energy if energy is not None else torch.zeros(4, dtype=torch.float64, device=x.device)
+    e = energy if energy is not None else _energy(op, x.device)
     ws = ws or default_workspace(x.device)
     _check(lib().ss24_error_energy(ctypes.byref(op), pattern, _SCORE[score] if isinstance(score, str) else score,
                                    _ptr(col_norms), sf, df, _ptr(sparse_scale), _ptr(dense_scale), _ptr(e), ws.ptr,
@@ -260,7 +280,7 @@ def error_energy(x, pattern=SPARSE_24, sparse_fmt=("none",), dense_fmt=("int", 8
 
 def amax(x, pattern=SPARSE_24, score="mag", col_norms=None, axis=1, ws=None, stream=None):
     op = make_operand(x, axis)
-    out = torch.empty(1, dtype=torch.float32, device=x.device)
+    out = torch.empty(max(op.batch, 1), dtype=torch.float32, device=x.device)
     ws = ws or default_workspace(x.device)
     _check(lib().ss24_amax(ctypes.byref(op), pattern, _SCORE[score] if isinstance(score, str) else score,
                            _ptr(col_norms), _ptr(out), ws.ptr, ws.nbytes, _stream(stream)), "ss24_amax")
@@ -269,9 +289,10 @@ def amax(x, pattern=SPARSE_24, score="mag", col_norms=None, axis=1, ws=None, str
 
 def tensor_scale(x, fmt="fp8", pattern=SPARSE_24, score="mag", col_norms=None, axis=1, ws=None, stream=None,
                  out=None):
-    """The per-tensor scale (FP8: amax / 448, NVFP4: amax / 2688) as a device float32[1]."""
+    """The per-tensor scale (FP8: amax / 448, NVFP4: amax / 2688) as a device
+    float32[1] (float32[B] for a batch)."""
     op = make_operand(x, axis)
-    out = out if out is not None else torch.empty(1, dtype=torch.float32, device=x.device)
+    out = out if out is not None else torch.empty(max(op.batch, 1), dtype=torch.float32, device=x.device)
     ws = ws or default_workspace(x.device)
     _check(lib().ss24_tensor_scale(ctypes.byref(op), pattern, _SCORE[score] if isinstance(score, str) else score,
                                    _ptr(col_norms), _FMT[fmt] if isinstance(fmt, str) else fmt, _ptr(out), ws.ptr,

@@ -61,8 +61,8 @@ def _ws_bytes():
     return ss24.lib().ss24_workspace_bytes()
 
 
-def op(x=ALIGNED, dtype=ss24.BF16, axis=1, rows=16, k=64, ld=64):
-    return ss24.Operand(x, dtype, axis, rows, k, ld)
+def op(x=ALIGNED, dtype=ss24.BF16, axis=1, rows=16, k=64, ld=64, batch=0, batch_stride=0):
+    return ss24.Operand(x, dtype, axis, rows, k, ld, batch, batch_stride)
 
 
 def outs(values=ALIGNED, scales=ALIGNED, tscale=ALIGNED, meta=ALIGNED):
@@ -83,7 +83,8 @@ def fused(o, fmt=None, ws=ALIGNED, ws_bytes=None, score=ss24.MAG, norms=None, ou
     ("bad_kind", 5), ("int_bits", 5), ("int_pack4", 5), ("int_group_np2", 5), ("int_group_big", 5),
     ("ws_null", 6), ("ws_small", 6), ("ws_misaligned", 6), ("null_values", 1), ("null_meta", 1),
     ("null_scales", 1), ("null_tscale", 1), ("wanda_no_norms", 1), ("wanda_misaligned_norms", 3),
-    ("bad_score", 8), ("misaligned_values", 3),
+    ("bad_score", 8), ("misaligned_values", 3), ("neg_batch", 2), ("huge_batch", 2), ("overlapping_batch", 2),
+    ("misaligned_batch_stride", 3),
 ])
 def test_validation_rejects_before_launch(case, expected):
     f = None
@@ -144,6 +145,14 @@ def test_validation_rejects_before_launch(case, expected):
         kw["score"] = 5
     elif case == "misaligned_values":
         kw["out"] = outs(values=MISALIGNED)
+    elif case == "neg_batch":
+        o = op(batch=-1)
+    elif case == "huge_batch":
+        o = op(batch=1025, batch_stride=16 * 64)
+    elif case == "overlapping_batch":
+        o = op(batch=2, batch_stride=16 * 64 - 8)
+    elif case == "misaligned_batch_stride":
+        o = op(batch=2, batch_stride=16 * 64 + 4)
     assert fused(o, f, **kw) == expected
 
 

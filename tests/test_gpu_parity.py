@@ -238,6 +238,78 @@ def test_strided_axis_limits_and_energy_pass(ss, ws):
     assert a.item() == oracle.amax(w, score=oracle.WANDA, norms=norms, axis=0)
 
 
+# --------------------------------------------------------------------------
+# batches: B same-shaped operands in one call, each exactly as alone
+# --------------------------------------------------------------------------
+
+def compare_batch(ss, ws, xs, *, pattern, fmt, bits=8, group=0, pack4=False, axis=1, pad_rows=0, tensor_scale=None):
+    """xs: host arrays of one shape; they are placed pad_rows apart (a strided
+    batch when pad_rows > 0) and processed in one call; each operand's outputs
+    are compared with the oracle run on that operand alone."""
+    B = len(xs)
+    shape = xs[0].shape
+    full = np.zeros((B, shape[0] + pad_rows, shape[1]), dtype=xs[0].dtype)
+    for b in range(B):
+        full[b, :shape[0]] = xs[b]
+    xd = to_dev(full)[:, :shape[0]]
+    sd = torch.tensor(tensor_scale, dtype=torch.float32, device="cuda") if tensor_scale is not None else None
+    out = ss.run(xd, pattern=pattern, fmt=fmt, bits=bits, group=group, pack4=pack4, axis=axis, tensor_scale=sd,
+                 ws=ws)
+    torch.cuda.synchronize()
+    opat = {0: oracle.DENSE, 24: oracle.SPARSE_24, 48: oracle.SPARSE_48}[pattern]
+    for b in range(B):
+        ref = oracle.run(xs[b], pattern=opat, fmt=fmt, bits=bits, group=group, pack4=pack4, axis=axis,
+                         tensor_scale=None if tensor_scale is None else tensor_scale[b])
+        for key in ("values", "scales", "meta"):
+            if key in ref:
+                assert_same(to_np(out[key][b]), ref[key], f"{key}[{b}]")
+        if "tensor_scale" in ref:
+            assert_same(to_np(out["tensor_scale"][b:b + 1]), ref["tensor_scale"], f"tensor_scale[{b}]")
+        assert_energy(out["energy"][b], ref["energy"], atol=1e-30)
+    assert ws.error() == 0
+
+
+@pytest.mark.parametrize("pattern,fmt,bits,group", [(24, "fp8", 8, 0), (24, "nvfp4", 4, 0), (48, "mxfp4", 4, 0),
+                                                    (24, "int", 8, 64), (24, "none", 8, 0), (0, "fp8", 8, 0),
+                                                    (0, "int", 8, 0), (24, "int", 4, 0), (0, "int", 8, 0)])
+@pytest.mark.parametrize("pad_rows", [0, 5])
+def test_batch_of_operands(ss, ws, pattern, fmt, bits, group, pad_rows):
+    xs = [synth.sweep_operand(100, 1024, seed=40 + b) for b in range(3)]  # distinct operands and scales
+    compare_batch(ss, ws, xs, pattern=pattern, fmt=fmt, bits=bits, group=group, pad_rows=pad_rows)
+
+
+def test_batch_given_scales_axis0_and_long_rows(ss, ws):
+    xs = [synth.sweep_operand(64, 512, seed=50 + b) for b in range(4)]
+    scales = [oracle.tensor_scale(x, "fp8") * (1 + b) for b, x in enumerate(xs)]
+    compare_batch(ss, ws, xs, pattern=24, fmt="fp8", tensor_scale=scales)
+    xa = [synth.sweep_operand(256, 72, seed=60 + b) for b in range(3)]        # axis 0: [k][rows]
+    compare_batch(ss, ws, xa, pattern=24, fmt="nvfp4", axis=0)
+    compare_batch(ss, ws, xa, pattern=0, fmt="int", bits=8, group=32, axis=0)
+    xl = [synth.linear_input(20, 5120, seed=70 + b, n_outlier=8)[0] for b in range(2)]
+    compare_batch(ss, ws, xl, pattern=24, fmt="int", bits=8, group=0, pad_rows=3)
+
+
+def test_batch_amax_scale_energy_and_empty(ss, ws):
+    xs = [synth.gaussian_bf16(40, 256, seed=80 + b, std=1.0 + b) for b in range(5)]
+    xd = to_dev(np.stack(xs))
+    a = ss.amax(xd, pattern=24, ws=ws).cpu().numpy()
+    t = ss.tensor_scale(xd, "nvfp4", ss.SPARSE_24, ws=ws).cpu().numpy()
+    e = ss.error_energy(xd, pattern=24, sparse_fmt=("fp8",), dense_fmt=("int", 5, 32), ws=ws).cpu().numpy()
+    for b, x in enumerate(xs):
+        assert a[b] == np.float32(oracle.amax(x))
+        assert t[b] == np.float32(oracle.tensor_scale(x, "nvfp4"))
+        sp = oracle.run(x, fmt="fp8")["energy"]
+        de = oracle.run(x, pattern=oracle.DENSE, fmt="int", bits=5, group=32)["energy"]
+        g = e[b]
+        for f, r in zip(range(4), [sp[0], sp[1], sp[2], de[3]]):
+            assert abs(g[f] - r) <= RTOL * abs(r)
+    empty = torch.zeros((3, 0, 64), dtype=torch.bfloat16, device="cuda")
+    out = ss.run(empty, pattern=24, fmt="fp8", ws=ws)
+    torch.cuda.synchronize()
+    assert out["energy"].shape == (3, 4) and out["energy"].abs().sum().item() == 0.0
+    assert ws.error() == 0
+
+
 def test_int_one_scale_per_long_row(ss, ws):
     """Rows too long for the register-resident kernel use the shared-memory row kernel."""
     for pattern in (0, 24, 48):
