@@ -357,8 +357,10 @@ ss24_status ss24_decode_e2m1(const uint8_t *in, float *out, int64_t n, ss24_stre
 
 /* The kernels divide by a scale with Markstein's one-step correction of a
  * reciprocal (P. Markstein, IBM J. Res. Dev. 34(1), 1990) instead of an IEEE
- * division, for scales in [2^-60, 2^60]; this entry point checks that the two
- * agree bit for bit on the running GPU. mode 0: b = 1 + (b_first + j) 2^-23
+ * division, for scales in [2^-60, 2^60]: as a / b, and in a packed form that
+ * yields -(a / b) directly (the correction run with -1/b) so that codes come out
+ * with their signs flipped back exactly. This entry point checks that both
+ * forms agree bit for bit with IEEE division on the running GPU. mode 0: b = 1 + (b_first + j) 2^-23
  * for j < b_count, against every a in [1, 2) (2^23 significands each; b_first +
  * b_count <= 2^23 — all 2^23 values of b together cover every pair of
  * significands, which by exact power-of-two scaling covers every a and b the

@@ -12,8 +12,8 @@
 #include "internal.cuh"
 
 namespace ss24 {
-const void *tile_kernel_bf16(int pattern, int score, int fmt);
-const void *tile_kernel_f32(int pattern, int score, int fmt);
+const void *stream_kernel_bf16(int pattern, int score, int fmt, bool fw);
+const void *stream_kernel_f32(int pattern, int score, int fmt, bool fw);
 const void *rowsweep_kernel_bf16(int pattern, int score);
 const void *rowsweep_kernel_f32(int pattern, int score);
 const void *axis0_kernel_bf16(int pattern, int score, int fmt);
@@ -169,6 +169,16 @@ cudaError_t launch(const void *k, size_t smem, int64_t n_tiles, const CUtensorMa
                    cudaStream_t stream)
 {
     KernelInfo info;
+    if (p.axis == 1) {
+        // the stream kernel: no tensor map, no dynamic shared memory
+        cudaError_t e = kernel_info(k, 0, &info, kStreamThreads);
+        if (e != cudaSuccess)
+            return e;
+        PassParams pp = p;
+        pp.ctas_per_op = static_cast<int32_t>(ctas_per_operand(info, p.batch, n_tiles));
+        void *args[1] = {&pp};
+        return launch_pdl(k, static_cast<unsigned>(p.batch * pp.ctas_per_op), kStreamThreads, 0, stream, args);
+    }
     cudaError_t e = kernel_info(k, smem, &info);
     if (e != cudaSuccess)
         return e;
@@ -316,25 +326,43 @@ bool per_tensor(int kind) { return kind == SS24_FMT_FP8_E4M3 || kind == SS24_FMT
 
 struct Geometry {
     int32_t R, W, log2_cpr, cpt;
-    int64_t n_tiles, n_col_tiles;
+    int64_t n_tiles, n_col_tiles; // axis 1: n_tiles = work items of 8 units (one per warp of a CTA)
     uint32_t tile_bytes;
+    int32_t units_a, units_b, unit_rows, unit_cols, step_rows, step_cols;
 };
 
-Geometry tile_geometry(const ss24_operand *x)
+// Axis 1 (stream kernel). A slot is a row segment of W = min(256,
+// next_pow2(k)) columns for 256 / W rows (one 16-byte chunk per lane); a unit
+// is four slots. Four consecutive segments of the same rows when a row has at
+// least 4 segments and a ragged last quad wastes little (nseg a multiple of 4
+// or at least 16); otherwise the same segment of four consecutive row groups.
+Geometry stream_geometry(const ss24_operand *x)
 {
     Geometry g{};
-    const int64_t es = static_cast<int64_t>(esize(x->dtype));
     g.W = static_cast<int32_t>(x->k >= 256 ? 256 : next_pow2(x->k));
-    const int64_t stage_elems = kStageBytes / es;
-    int64_t R = stage_elems / g.W;
-    if (R > 256)
-        R = 256;
-    g.R = static_cast<int32_t>(R);
     g.log2_cpr = ilog2(g.W / 8);
-    g.cpt = static_cast<int32_t>((R * g.W / 8) / kConsumers);
-    g.n_col_tiles = (x->k + g.W - 1) / g.W;
-    g.n_tiles = g.n_col_tiles * ((x->rows + R - 1) / R);
-    g.tile_bytes = static_cast<uint32_t>(R * g.W * es);
+    const int64_t rps = 256 / g.W;
+    const int64_t nseg = (x->k + g.W - 1) / g.W;
+    const int64_t n_rg = (x->rows + rps - 1) / rps;
+    int64_t ua, ub;
+    if (nseg >= 4 && (nseg % 4 == 0 || nseg >= 16)) {
+        g.unit_rows = static_cast<int32_t>(rps);
+        g.unit_cols = 4 * g.W;
+        g.step_rows = 0;
+        g.step_cols = g.W;
+        ua = n_rg;
+        ub = (nseg + 3) / 4;
+    } else {
+        g.unit_rows = static_cast<int32_t>(4 * rps);
+        g.unit_cols = g.W;
+        g.step_rows = static_cast<int32_t>(rps);
+        g.step_cols = 0;
+        ua = (n_rg + 3) / 4;
+        ub = nseg;
+    }
+    g.units_a = static_cast<int32_t>(ua);
+    g.units_b = static_cast<int32_t>(ub);
+    g.n_tiles = (ua * ub + kStreamWarps - 1) / kStreamWarps;
     return g;
 }
 
@@ -379,6 +407,14 @@ PassParams base_params(const ss24_operand *x, const Geometry &g, void *ws, ss24_
     p.cpt = g.cpt;
     p.axis = x->axis;
     p.tile_bytes = g.tile_bytes;
+    p.x = x->x;
+    p.ld = x->ld;
+    p.units_a = g.units_a;
+    p.units_b = g.units_b;
+    p.unit_rows = g.unit_rows;
+    p.unit_cols = g.unit_cols;
+    p.step_rows = g.step_rows;
+    p.step_cols = g.step_cols;
     uint8_t *w = static_cast<uint8_t *>(ws);
     p.err = reinterpret_cast<int32_t *>(w + kWsErrOff);
     p.energy_ticket = reinterpret_cast<uint32_t *>(w + kWsEnergyTicketOff);
@@ -422,9 +458,10 @@ void output_strides(const ss24_operand *x, int pattern, ss24_format fmt, PassPar
         p->meta_bstride = rows * x->k / (pattern == SS24_SPARSE_48 ? 16 : 8);
 }
 
-const void *tile_kernel(int dtype, int pattern, int score, int fmt)
+const void *stream_kernel(int dtype, int pattern, int score, int fmt, bool fw)
 {
-    return dtype == SS24_BF16 ? tile_kernel_bf16(pattern, score, fmt) : tile_kernel_f32(pattern, score, fmt);
+    return dtype == SS24_BF16 ? stream_kernel_bf16(pattern, score, fmt, fw)
+                              : stream_kernel_f32(pattern, score, fmt, fw);
 }
 
 // Tile geometry, tensor map and kernel for a tile-mode pass along either axis.
@@ -438,10 +475,11 @@ struct TilePlan {
 bool plan_tile(const ss24_operand *x, int pattern, int score, int mode, TilePlan *t)
 {
     if (x->axis == 1) {
-        t->g = tile_geometry(x);
-        t->kernel = tile_kernel(x->dtype, pattern, score, mode);
-        t->smem = kSmemBytes;
-        return make_map(&t->map, x, x->k, x->rows, static_cast<uint32_t>(t->g.W), static_cast<uint32_t>(t->g.R));
+        t->g = stream_geometry(x);
+        // full width: W = 256 with four segments per unit
+        t->kernel = stream_kernel(x->dtype, pattern, score, mode, t->g.W == 256 && t->g.step_cols == 256);
+        t->smem = 0;
+        return t->kernel != nullptr;
     }
     t->g = axis0_geometry(x);
     t->kernel = x->dtype == SS24_BF16 ? axis0_kernel_bf16(pattern, score, mode) : axis0_kernel_f32(pattern, score, mode);
@@ -513,7 +551,7 @@ ss24_status run_pass(const ss24_operand *x, int pattern, int score, const float 
         r.row_mode = false;
         g = axis0_geometry(x);
     } else {
-        g = tile_geometry(x); // (row mode uses only rows / k of it)
+        g = stream_geometry(x); // (row mode uses only rows / k of it)
     }
     if (x->rows == 0)
         return empty_operand(x, energy, out, per_tensor(fmt.kind) ? scale_in : nullptr, stream);

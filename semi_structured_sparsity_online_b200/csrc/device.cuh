@@ -308,6 +308,19 @@ __device__ __forceinline__ f32x2 div_fast2(f32x2 a, const Recip &r)
     return fma2(res, y2, q0);
 }
 
+// Negated quotients -(a / b) of two values: Markstein's correction run with
+// -y in place of y (q0 = RN(a (-y)), r = a + q0 b exact, RN(q0 + r (-y))).
+// Because rounding to nearest is symmetric this is exactly -RN(a / b) where
+// div_fast is exact, with the signed zeros right as well: a = -0 gives +0 and
+// a = +0 gives -0, so no sign fix-up is needed.
+__device__ __forceinline__ f32x2 neg_div_fast2(f32x2 a, const Recip &r)
+{
+    const f32x2 ny2 = pack2(-r.y, -r.y), b2 = pack2(r.b, r.b);
+    const f32x2 q0 = mul2(a, ny2);
+    const f32x2 res = fma2(q0, b2, a);
+    return fma2(res, ny2, q0);
+}
+
 // ---------------------------------------------------------------------------
 // selection
 // ---------------------------------------------------------------------------

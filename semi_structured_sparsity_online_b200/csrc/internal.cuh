@@ -24,6 +24,11 @@ constexpr int kStages = 4;
 constexpr int kMaxGrid = 1024;            // bound on CTAs (workspace partials)
 constexpr size_t kSmemBytes = kStages * kStageBytes + 4096;
 
+// The axis-1 stream kernel: 8 warps per CTA, no shared-memory stages. The
+// block reductions assume the same warp count as the tile kernels' consumers.
+constexpr int kStreamWarps = kConsumerWarps;
+constexpr int kStreamThreads = kStreamWarps * 32;
+
 // One scale per long row: one warp per row, 8 warps per CTA.
 constexpr int kRowThreads = 256;
 
@@ -75,6 +80,12 @@ struct PassParams {
     int32_t cpt;               // chunks per consumer thread per tile
     int32_t axis;              // 1: k is the contiguous (TMA inner) dimension; 0: rows are
     uint32_t tile_bytes;
+    // axis-1 stream kernel: the operand (elements ld apart between rows), the
+    // unit grid units_a x units_b, a unit's extent (rows, columns) and the
+    // step between its four slots (rows, columns)
+    const void *x;
+    int64_t ld;
+    int32_t units_a, units_b, unit_rows, unit_cols, step_rows, step_cols;
     // outputs
     void *values;
     void *scales;

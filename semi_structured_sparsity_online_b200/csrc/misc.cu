@@ -57,7 +57,9 @@ __global__ void convert_kernel(int op, const void *in, void *out, int64_t n)
     }
 }
 
-// Markstein's correction (device.cuh, div_fast) against IEEE division.
+// Markstein's correction against IEEE division, in both forms the kernels
+// use: div_fast (a / b) and the packed negated form neg_div_fast2, whose two
+// lanes are checked as -(a / b) (negated back) and -(-a) / b.
 // mode 0: b = 1 + (b_first + blockIdx.x) * 2^-23 against every a in [1, 2)
 //         (all 2^23 significands); the full sweep over b covers every pair of
 //         significands.
@@ -84,7 +86,9 @@ __global__ void selfcheck_division_kernel(int mode, uint32_t b_first, unsigned l
         for (uint32_t i = threadIdx.x; i < (1u << 23); i += blockDim.x) {
             const float a = __uint_as_float(0x3f800000u | i);
             const float q = div_fast(a, rc), ref = __fdiv_rn(a, b);
-            if (__float_as_uint(q) != __float_as_uint(ref)) {
+            const float qn = lo2(neg_div_fast2(pack2(a, -a), rc)), qp = hi2(neg_div_fast2(pack2(a, -a), rc));
+            if (__float_as_uint(q) != __float_as_uint(ref) || __float_as_uint(-qn) != __float_as_uint(ref) ||
+                __float_as_uint(qp) != __float_as_uint(ref)) {
                 ++bad;
                 first = min(first, (static_cast<unsigned long long>(__float_as_uint(a)) << 32) | __float_as_uint(b));
             }
@@ -103,7 +107,9 @@ __global__ void selfcheck_division_kernel(int mode, uint32_t b_first, unsigned l
                                             (hash32(h3) & 0x7fffffu));
             const Recip rc = make_recip(b);
             const float q = div_fast(a, rc), ref = __fdiv_rn(a, b);
-            if (__float_as_uint(q) != __float_as_uint(ref)) {
+            const f32x2 nq = neg_div_fast2(pack2(a, -a), rc);
+            if (__float_as_uint(q) != __float_as_uint(ref) || __float_as_uint(-lo2(nq)) != __float_as_uint(ref) ||
+                __float_as_uint(hi2(nq)) != __float_as_uint(ref)) {
                 ++bad;
                 first = min(first, (static_cast<unsigned long long>(__float_as_uint(a)) << 32) | __float_as_uint(b));
             }

@@ -1,47 +1,52 @@
 // Kernel tables for one element type: maps (pattern, score, format) to the
-// instantiated tile-mode or row-mode kernel.
+// instantiated stream (axis 1), row-sweep or axis-0 kernel.
 #pragma once
 
 #include "pass_impl.cuh"
 
 namespace ss24 {
 
-template <typename T, int PAT, int SC> const void *tile_kernel_for_fmt(int fmt)
+template <typename T, int PAT, int SC, bool FW> const void *stream_kernel_for_fmt(int fmt)
 {
     switch (fmt) {
     case kNone:
         if constexpr (PAT != kDense)
-            return reinterpret_cast<const void *>(&pass_kernel<T, PAT, SC, kNone>);
+            return reinterpret_cast<const void *>(&stream_kernel<T, PAT, SC, kNone, FW>);
         break;
     case kFp8:
-        return reinterpret_cast<const void *>(&pass_kernel<T, PAT, SC, kFp8>);
+        return reinterpret_cast<const void *>(&stream_kernel<T, PAT, SC, kFp8, FW>);
     case kInt:
-        return reinterpret_cast<const void *>(&pass_kernel<T, PAT, SC, kInt>);
+        return reinterpret_cast<const void *>(&stream_kernel<T, PAT, SC, kInt, FW>);
     case kNvfp4:
-        return reinterpret_cast<const void *>(&pass_kernel<T, PAT, SC, kNvfp4>);
+        return reinterpret_cast<const void *>(&stream_kernel<T, PAT, SC, kNvfp4, FW>);
     case kMxfp4:
-        return reinterpret_cast<const void *>(&pass_kernel<T, PAT, SC, kMxfp4>);
+        return reinterpret_cast<const void *>(&stream_kernel<T, PAT, SC, kMxfp4, FW>);
     case kAmax:
-        return reinterpret_cast<const void *>(&pass_kernel<T, PAT, SC, kAmax>);
+        return reinterpret_cast<const void *>(&stream_kernel<T, PAT, SC, kAmax, FW>);
     case kEnergy:
         if constexpr (PAT != kDense)
-            return reinterpret_cast<const void *>(&pass_kernel<T, PAT, SC, kEnergy>);
+            return reinterpret_cast<const void *>(&stream_kernel<T, PAT, SC, kEnergy, FW>);
         break;
     }
     return nullptr;
 }
 
-template <typename T> const void *tile_kernel(int pattern, int score, int fmt)
+template <typename T, bool FW> const void *stream_kernel_pat(int pattern, int score, int fmt)
 {
     if (pattern == kDense)
-        return tile_kernel_for_fmt<T, kDense, kMag>(fmt);
+        return stream_kernel_for_fmt<T, kDense, kMag, FW>(fmt);
     if (pattern == kSparse24)
-        return score == kWanda ? tile_kernel_for_fmt<T, kSparse24, kWanda>(fmt)
-                               : tile_kernel_for_fmt<T, kSparse24, kMag>(fmt);
+        return score == kWanda ? stream_kernel_for_fmt<T, kSparse24, kWanda, FW>(fmt)
+                               : stream_kernel_for_fmt<T, kSparse24, kMag, FW>(fmt);
     if (pattern == kSparse48)
-        return score == kWanda ? tile_kernel_for_fmt<T, kSparse48, kWanda>(fmt)
-                               : tile_kernel_for_fmt<T, kSparse48, kMag>(fmt);
+        return score == kWanda ? stream_kernel_for_fmt<T, kSparse48, kWanda, FW>(fmt)
+                               : stream_kernel_for_fmt<T, kSparse48, kMag, FW>(fmt);
     return nullptr;
+}
+
+template <typename T> const void *stream_kernel_ptr(int pattern, int score, int fmt, bool fw)
+{
+    return fw ? stream_kernel_pat<T, true>(pattern, score, fmt) : stream_kernel_pat<T, false>(pattern, score, fmt);
 }
 
 template <typename T> const void *rowsweep_kernel_ptr(int pattern, int score)

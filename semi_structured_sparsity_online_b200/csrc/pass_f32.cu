@@ -2,9 +2,9 @@
 #include "pass_dispatch.cuh"
 
 namespace ss24 {
-const void *tile_kernel_f32(int pattern, int score, int fmt)
+const void *stream_kernel_f32(int pattern, int score, int fmt, bool fw)
 {
-    return tile_kernel<float>(pattern, score, fmt);
+    return stream_kernel_ptr<float>(pattern, score, fmt, fw);
 }
 const void *rowsweep_kernel_f32(int pattern, int score)
 {

@@ -79,10 +79,14 @@ __device__ __forceinline__ float sq(float a) { return a * a; }
 // lane of the warp calls them (group reductions shuffle across lanes)
 // ---------------------------------------------------------------------------
 
-struct QOut {
-    void *values;
-    void *scales;
-    int64_t row, colq, n; // quantized row length n, column of the chunk's first value
+// Where one chunk's results go: its first output value, its group's scale
+// entry, its metadata byte (4:8: the byte of its pair of chunks, written by the
+// even lane) and, for the Wanda score, the norms of its eight columns.
+struct ChunkOut {
+    uint8_t *val;
+    uint8_t *scale;
+    uint8_t *meta;
+    const float *norms;
     bool valid;
     int lane;
 };
@@ -121,23 +125,31 @@ template <int VPC> __device__ __forceinline__ float err_energy(const float (&v)[
     return lo2(t[0]) + hi2(t[0]);
 }
 
-// Quotients v / s of a chunk: Markstein's correction when the scale is in the
-// fast range and no quotient can overflow (max|v| * y < 2^126), IEEE division
-// otherwise; zero scale gives zero quotients.
-template <int VPC>
-__device__ __forceinline__ void quotients(const float (&v)[VPC], const Recip &rc, float vmax, float (&q)[VPC])
+// True when the fast division applies to every value of a chunk or group
+// whose largest magnitude is vmax: the scale is in [2^-60, 2^60] and no
+// quotient can overflow (vmax * y < 2^126).
+__device__ __forceinline__ bool quot_fast(const Recip &rc, float vmax)
 {
-    if (rc.fast && __fmul_rn(vmax, rc.y) < 0x1p126f) {
+    return rc.fast && __fmul_rn(vmax, rc.y) < 0x1p126f;
+}
+
+// Negated quotients -v / s of a chunk: neg_div_fast2 on the fast path,
+// otherwise IEEE division; a zero scale gives negated zero quotients. Callers encode -q and flip the sign of the codes,
+// which is exact because every rounding to a format is symmetric.
+template <int VPC>
+__device__ __forceinline__ void neg_quotients(const float (&v)[VPC], const Recip &rc, bool fast, float (&qn)[VPC])
+{
+    if (fast) {
 #pragma unroll
         for (int i = 0; i < VPC / 2; ++i) {
-            const f32x2 qq = div_fast2(pack2(v[2 * i], v[2 * i + 1]), rc);
-            q[2 * i] = with_sign_of(lo2(qq), v[2 * i]);
-            q[2 * i + 1] = with_sign_of(hi2(qq), v[2 * i + 1]);
+            const f32x2 qq = neg_div_fast2(pack2(v[2 * i], v[2 * i + 1]), rc);
+            qn[2 * i] = lo2(qq);
+            qn[2 * i + 1] = hi2(qq);
         }
     } else {
 #pragma unroll
         for (int i = 0; i < VPC; ++i)
-            q[i] = rc.b != 0.0f ? __fdiv_rn(v[i], rc.b) : 0.0f;
+            qn[i] = rc.b != 0.0f ? __fdiv_rn(-v[i], rc.b) : -0.0f;
     }
 }
 
@@ -155,15 +167,21 @@ __device__ __forceinline__ void scale_values(const float (&c)[VPC], float s, flo
 }
 
 // FP8 E4M3, per-tensor scale s: code = E4M3(v / s); deq = E4M3(code) * s.
+// With `guard` false the caller knows that no quotient can overflow (the scale
+// was derived from the amax of the values quantized).
 template <int VPC, bool STORE>
-__device__ __forceinline__ float quant_fp8(const float (&v)[VPC], const Recip &rc, const QOut &o)
+__device__ __forceinline__ float quant_fp8(const float (&v)[VPC], const Recip &rc, bool guard, const ChunkOut &o)
 {
-    float q[VPC], dec[VPC], d[VPC];
-    quotients<VPC>(v, rc, local_amax<VPC>(v), q);
+    bool fast = rc.fast;
+    if (guard)
+        fast = quot_fast(rc, local_amax<VPC>(v));
+    float qn[VPC], dec[VPC], d[VPC];
+    neg_quotients<VPC>(v, rc, fast, qn);
     uint32_t c[VPC / 4];
 #pragma unroll
     for (int t = 0; t < VPC / 4; ++t) {
-        c[t] = cvt_e4m3x2(q[4 * t], q[4 * t + 1]) | (cvt_e4m3x2(q[4 * t + 2], q[4 * t + 3]) << 16);
+        c[t] = (cvt_e4m3x2(qn[4 * t], qn[4 * t + 1]) | (cvt_e4m3x2(qn[4 * t + 2], qn[4 * t + 3]) << 16)) ^
+               0x80808080u;
         const float2 lo = e4m3x2_to_f32(c[t] & 0xffffu), hi = e4m3x2_to_f32(c[t] >> 16);
         dec[4 * t + 0] = lo.x;
         dec[4 * t + 1] = lo.y;
@@ -172,11 +190,10 @@ __device__ __forceinline__ float quant_fp8(const float (&v)[VPC], const Recip &r
     }
     scale_values<VPC>(dec, rc.b, d);
     if (STORE && o.valid) {
-        uint8_t *dst = static_cast<uint8_t *>(o.values) + o.row * o.n + o.colq;
         if constexpr (VPC == 4)
-            *reinterpret_cast<uint32_t *>(dst) = c[0];
+            *reinterpret_cast<uint32_t *>(o.val) = c[0];
         else
-            *reinterpret_cast<uint2 *>(dst) = make_uint2(c[0], c[1]);
+            *reinterpret_cast<uint2 *>(o.val) = make_uint2(c[0], c[1]);
     }
     return err_energy<VPC>(v, d);
 }
@@ -212,7 +229,7 @@ struct RowScale {
 };
 
 template <int VPC, bool STORE>
-__device__ __forceinline__ float quant_int(const float (&v)[VPC], const QuantSpec &q, const QOut &o,
+__device__ __forceinline__ float quant_int(const float (&v)[VPC], const QuantSpec &q, const ChunkOut &o,
                                            float row_amax = -1.0f, const RowScale *rs = nullptr)
 {
     float amax, scale;
@@ -226,20 +243,23 @@ __device__ __forceinline__ float quant_int(const float (&v)[VPC], const QuantSpe
         scale = int_scale(amax, q);
         rc = make_recip(scale);
     }
-    float qv[VPC];
-    quotients<VPC>(v, rc, amax, qv);
-    if (!rc.fast) {
+    const bool fast = quot_fast(rc, amax);
+    float qn[VPC];
+    neg_quotients<VPC>(v, rc, fast, qn);
+    if (!fast) {
         // a scale outside [2^-60, 2^60] (e.g. subnormal) can put |v / scale|
         // above qmax: apply the clamp of the definition
 #pragma unroll
         for (int i = 0; i < VPC; ++i)
-            qv[i] = fminf(fmaxf(qv[i], -q.qmax), q.qmax);
+            qn[i] = fminf(fmaxf(qn[i], -q.qmax), q.qmax);
     }
+    // M - (-q) = M + q rounds q to an integer (ties to even) held in the low
+    // bits of the sum; (M + q) - M is that integer exactly
     float t[VPC], cf[VPC], d[VPC];
     const f32x2 m2 = pack2(kMagic, kMagic);
 #pragma unroll
     for (int i = 0; i < VPC / 2; ++i) {
-        const f32x2 tt = add2(pack2(qv[2 * i], qv[2 * i + 1]), m2);
+        const f32x2 tt = sub2(m2, pack2(qn[2 * i], qn[2 * i + 1]));
         const f32x2 cc = sub2(tt, m2);
         t[2 * i] = lo2(tt);
         t[2 * i + 1] = hi2(tt);
@@ -248,8 +268,7 @@ __device__ __forceinline__ float quant_int(const float (&v)[VPC], const QuantSpe
     }
     scale_values<VPC>(cf, scale, d);
     if (STORE && o.valid) {
-        const int64_t off = o.row * o.n + o.colq;
-        uint32_t b[VPC]; // low bits of q + M hold the two's-complement code
+        uint32_t b[VPC]; // low bits of M + q hold the two's-complement code
 #pragma unroll
         for (int i = 0; i < VPC; ++i)
             b[i] = __float_as_uint(t[i]);
@@ -259,34 +278,31 @@ __device__ __forceinline__ float quant_int(const float (&v)[VPC], const QuantSpe
             for (int k = 0; k < VPC / 4; ++k)
                 w[k] = __byte_perm(__byte_perm(b[4 * k], b[4 * k + 1], 0x0040), __byte_perm(b[4 * k + 2], b[4 * k + 3], 0x0040),
                                    0x5410);
-            uint8_t *dst = static_cast<uint8_t *>(o.values) + off;
             if constexpr (VPC == 4)
-                *reinterpret_cast<uint32_t *>(dst) = w[0];
+                *reinterpret_cast<uint32_t *>(o.val) = w[0];
             else
-                *reinterpret_cast<uint2 *>(dst) = make_uint2(w[0], w[1]);
+                *reinterpret_cast<uint2 *>(o.val) = make_uint2(w[0], w[1]);
         } else if (q.store == kInt16) {
             uint32_t w[VPC / 2];
 #pragma unroll
             for (int k = 0; k < VPC / 2; ++k)
                 w[k] = __byte_perm(b[2 * k], b[2 * k + 1], 0x5410);
-            int16_t *dst = static_cast<int16_t *>(o.values) + off;
             if constexpr (VPC == 4)
-                *reinterpret_cast<uint2 *>(dst) = make_uint2(w[0], w[1]);
+                *reinterpret_cast<uint2 *>(o.val) = make_uint2(w[0], w[1]);
             else
-                *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+                *reinterpret_cast<uint4 *>(o.val) = make_uint4(w[0], w[1], w[2], w[3]);
         } else {
             uint32_t w = 0;
 #pragma unroll
             for (int i = 0; i < VPC; ++i)
                 w |= (b[i] & 0xfu) << (4 * i);
-            uint8_t *dst = static_cast<uint8_t *>(o.values) + off / 2;
             if constexpr (VPC == 4)
-                *reinterpret_cast<uint16_t *>(dst) = static_cast<uint16_t>(w);
+                *reinterpret_cast<uint16_t *>(o.val) = static_cast<uint16_t>(w);
             else
-                *reinterpret_cast<uint32_t *>(dst) = w;
+                *reinterpret_cast<uint32_t *>(o.val) = w;
         }
         if (row_amax < 0.0f && !(rs && rs->given) && (o.lane & (q.lanes - 1)) == 0)
-            static_cast<float *>(o.scales)[o.row * (o.n / q.group) + o.colq / q.group] = scale;
+            *reinterpret_cast<float *>(o.scale) = scale;
     }
     return err_energy<VPC>(v, d);
 }
@@ -313,14 +329,13 @@ __device__ __forceinline__ void unpack_e2m1(uint32_t codes, float mult, float (&
 }
 
 template <int VPC, bool STORE>
-__device__ __forceinline__ void store_fp4(uint32_t codes, const QOut &o)
+__device__ __forceinline__ void store_fp4(uint32_t codes, const ChunkOut &o)
 {
     if (STORE && o.valid) {
-        uint8_t *dst = static_cast<uint8_t *>(o.values) + (o.row * o.n + o.colq) / 2;
         if constexpr (VPC == 4)
-            *reinterpret_cast<uint16_t *>(dst) = static_cast<uint16_t>(codes);
+            *reinterpret_cast<uint16_t *>(o.val) = static_cast<uint16_t>(codes);
         else
-            *reinterpret_cast<uint32_t *>(dst) = codes;
+            *reinterpret_cast<uint32_t *>(o.val) = codes;
     }
 }
 
@@ -343,7 +358,7 @@ __device__ __forceinline__ void build_nv_table(float *t, float st, int tid)
 }
 
 template <int VPC, bool STORE>
-__device__ __forceinline__ float quant_nvfp4(const float (&v)[VPC], const Recip &rst, const QOut &o,
+__device__ __forceinline__ float quant_nvfp4(const float (&v)[VPC], const Recip &rst, const ChunkOut &o,
                                              const NvTable &tb)
 {
     constexpr int kLanes = 16 / VPC;
@@ -369,13 +384,13 @@ __device__ __forceinline__ float quant_nvfp4(const float (&v)[VPC], const Recip 
     rd.y = tb.inv[sb];
     rd.fast = rd.b >= 0x1p-60f && rd.b <= 0x1p60f;
     const float denom = rd.b;
-    float q[VPC], d[VPC];
-    quotients<VPC>(v, rd, amax, q);
-    const uint32_t codes = pack_e2m1<VPC>(q);
+    float qn[VPC], d[VPC];
+    neg_quotients<VPC>(v, rd, quot_fast(rd, amax), qn);
+    const uint32_t codes = pack_e2m1<VPC>(qn) ^ (VPC == 4 ? 0x8888u : 0x88888888u);
     unpack_e2m1<VPC>(codes, denom, d);
     store_fp4<VPC, STORE>(codes, o);
     if (STORE && o.valid && (o.lane & (kLanes - 1)) == 0)
-        static_cast<uint8_t *>(o.scales)[o.row * (o.n / 16) + o.colq / 16] = static_cast<uint8_t>(sb);
+        *o.scale = static_cast<uint8_t>(sb);
     return err_energy<VPC>(v, d);
 }
 
@@ -383,7 +398,7 @@ __device__ __forceinline__ float quant_nvfp4(const float (&v)[VPC], const Recip 
 // the E8M0 byte e + 127; v / 2^e is computed as v * 2^-e (the same correctly
 // rounded value, since both scale factors are exact powers of two).
 template <int VPC, bool STORE>
-__device__ __forceinline__ float quant_mxfp4(const float (&v)[VPC], const QOut &o)
+__device__ __forceinline__ float quant_mxfp4(const float (&v)[VPC], const ChunkOut &o)
 {
     constexpr int kLanes = 32 / VPC;
     const float amax = group_amax(local_amax<VPC>(v), kLanes);
@@ -401,19 +416,19 @@ __device__ __forceinline__ float quant_mxfp4(const float (&v)[VPC], const QOut &
     unpack_e2m1<VPC>(codes, mult, d);
     store_fp4<VPC, STORE>(codes, o);
     if (STORE && o.valid && (o.lane & (kLanes - 1)) == 0)
-        static_cast<uint8_t *>(o.scales)[o.row * (o.n / 32) + o.colq / 32] = static_cast<uint8_t>(byte);
+        *o.scale = static_cast<uint8_t>(byte);
     return err_energy<VPC>(v, d);
 }
 
 // Runtime-dispatched quantizer without stores (the energy-only pass).
 template <int VPC>
 __device__ __forceinline__ float quant_energy_only(const float (&v)[VPC], const QuantSpec &q, const Recip &rst,
-                                                   const NvTable &tb)
+                                                   bool guard, const NvTable &tb)
 {
-    QOut o{nullptr, nullptr, 0, 0, 1, false, 0};
+    const ChunkOut o{nullptr, nullptr, nullptr, nullptr, false, 0};
     switch (q.fmt) {
     case kFp8:
-        return quant_fp8<VPC, false>(v, rst, o);
+        return quant_fp8<VPC, false>(v, rst, guard, o);
     case kInt:
         return quant_int<VPC, false>(v, q, o);
     case kNvfp4:
@@ -434,15 +449,23 @@ struct Acc {
     float amax_kept, amax_all;
 };
 
+// Per-CTA constants of a pass: the tensor scales (as reciprocals), the NVFP4
+// tables, and whether a per-tensor FP8 quotient must be checked for overflow
+// (a scale the caller gave; a scale derived from the amax never overflows).
+struct PassConsts {
+    Recip rst, rstd;
+    NvTable tb, tbd;
+    bool guard, guardd;
+};
+
 template <int SCORE>
-__device__ __forceinline__ void scores(const float (&x)[8], const float *norms, int64_t col, bool in_k,
-                                       float (&s)[8])
+__device__ __forceinline__ void scores(const float (&x)[8], const ChunkOut &o, float (&s)[8])
 {
     if constexpr (SCORE == kWanda) {
         float4 n0 = make_float4(0.f, 0.f, 0.f, 0.f), n1 = n0;
-        if (in_k) {
-            n0 = __ldg(reinterpret_cast<const float4 *>(norms + col));
-            n1 = __ldg(reinterpret_cast<const float4 *>(norms + col + 4));
+        if (o.valid) {
+            n0 = __ldg(reinterpret_cast<const float4 *>(o.norms));
+            n1 = __ldg(reinterpret_cast<const float4 *>(o.norms + 4));
         }
         const float n[8] = {n0.x, n0.y, n0.z, n0.w, n1.x, n1.y, n1.z, n1.w};
 #pragma unroll
@@ -456,15 +479,11 @@ __device__ __forceinline__ void scores(const float (&x)[8], const float *norms, 
 }
 
 template <typename T, int PAT, int SCORE, int FMT>
-__device__ __forceinline__ void process_chunk(const PassParams &p, const float (&x)[8], int64_t row,
-                                              int64_t col, int lane, const Recip &rst, const Recip &rstd,
-                                              Acc &acc, float row_amax = -1.0f, const RowScale *rs = nullptr,
-                                              const NvTable &tb = NvTable{nullptr, nullptr},
-                                              const NvTable &tbd = NvTable{nullptr, nullptr})
+__device__ __forceinline__ void process_chunk(const PassParams &p, const float (&x)[8], const ChunkOut &o,
+                                              const PassConsts &c, Acc &acc, float row_amax = -1.0f,
+                                              const RowScale *rs = nullptr)
 {
     constexpr int VPC = PAT == kDense ? 8 : 4;
-    const bool in_k = col < p.k;
-    const bool valid = in_k && row < p.rows;
     float v[VPC];
     uint32_t meta = 0;
     float et, ep = 0.0f;
@@ -483,7 +502,7 @@ __device__ __forceinline__ void process_chunk(const PassParams &p, const float (
         Group24 g0, g1;
         if constexpr (SCORE == kWanda) {
             float s[8];
-            scores<SCORE>(x, p.norms, col, in_k, s);
+            scores<SCORE>(x, o, s);
             g0 = group24<false>(x[0], x[1], x[2], x[3], s[0], s[1], s[2], s[3]);
             g1 = group24<false>(x[4], x[5], x[6], x[7], s[4], s[5], s[6], s[7]);
         } else {
@@ -511,7 +530,7 @@ __device__ __forceinline__ void process_chunk(const PassParams &p, const float (
         float rank[4] = {e[0], e[1], e[2], e[3]};
         if constexpr (SCORE == kWanda) {
             float s[8];
-            scores<SCORE>(x, p.norms, col, in_k, s);
+            scores<SCORE>(x, o, s);
             a = mul2(pack2(s[0], s[2]), pack2(s[0], s[2]));
             b = mul2(pack2(s[1], s[3]), pack2(s[1], s[3]));
             const f32x2 r01 = add2(a, b);
@@ -548,40 +567,36 @@ __device__ __forceinline__ void process_chunk(const PassParams &p, const float (
 
     // metadata
     if constexpr (PAT == kSparse24) {
-        if (FMT != kEnergy && valid)
-            p.meta[row * (p.k / 8) + col / 8] = static_cast<uint8_t>(meta);
+        if (FMT != kEnergy && o.valid)
+            *o.meta = static_cast<uint8_t>(meta);
     } else if constexpr (PAT == kSparse48) {
         const uint32_t other = __shfl_down_sync(kFull, meta, 1);
-        if (FMT != kEnergy && valid && (lane & 1) == 0)
-            p.meta[row * (p.k / 16) + col / 16] = static_cast<uint8_t>(meta | (other << 4));
+        if (FMT != kEnergy && o.valid && (o.lane & 1) == 0)
+            *o.meta = static_cast<uint8_t>(meta | (other << 4));
     }
 
-    const int64_t n = PAT == kDense ? p.k : p.k / 2;
-    const QOut o{p.values, p.scales, row, PAT == kDense ? col : col / 2, n, valid, lane};
     float eq = 0.0f;
     if constexpr (FMT == kNone) {
-        if (valid) {
+        if (o.valid) {
             if constexpr (sizeof(T) == 2) {
                 const uint32_t w0 = (__float_as_uint(v[0]) >> 16) | (__float_as_uint(v[1]) & 0xffff0000u);
                 const uint32_t w1 = (__float_as_uint(v[2]) >> 16) | (__float_as_uint(v[3]) & 0xffff0000u);
-                *reinterpret_cast<uint2 *>(static_cast<uint16_t *>(p.values) + row * n + col / 2) =
-                    make_uint2(w0, w1);
+                *reinterpret_cast<uint2 *>(o.val) = make_uint2(w0, w1);
             } else {
-                *reinterpret_cast<float4 *>(static_cast<float *>(p.values) + row * n + col / 2) =
-                    make_float4(v[0], v[1], v[2], v[3]);
+                *reinterpret_cast<float4 *>(o.val) = make_float4(v[0], v[1], v[2], v[3]);
             }
         }
     } else if constexpr (FMT == kFp8) {
-        eq = quant_fp8<VPC, true>(v, rst, o);
+        eq = quant_fp8<VPC, true>(v, c.rst, c.guard, o);
     } else if constexpr (FMT == kInt) {
         eq = quant_int<VPC, true>(v, p.q, o, row_amax, rs);
     } else if constexpr (FMT == kNvfp4) {
-        eq = quant_nvfp4<VPC, true>(v, rst, o, tb);
+        eq = quant_nvfp4<VPC, true>(v, c.rst, o, c.tb);
     } else if constexpr (FMT == kMxfp4) {
         eq = quant_mxfp4<VPC, true>(v, o);
     } else if constexpr (FMT == kEnergy) {
-        eq = quant_energy_only<VPC>(v, p.q, rst, tb);
-        acc.eqd += quant_energy_only<8>(x, p.qd, rstd, tbd);
+        eq = quant_energy_only<VPC>(v, p.q, c.rst, c.guard, c.tb);
+        acc.eqd += quant_energy_only<8>(x, p.qd, c.rstd, c.guardd, c.tbd);
     }
     if constexpr (PAT == kDense)
         acc.eqd += eq;
@@ -796,38 +811,46 @@ __device__ __forceinline__ void producer(const CUtensorMap *map, const PassParam
     }
 }
 
-template <typename T, int PAT, int SCORE, int FMT>
-__global__ void __launch_bounds__(kThreads, 3) pass_kernel(const __grid_constant__ CUtensorMap map,
-                                                           const PassParams pk)
+// Output pointers of the chunk at (row, col) (col: first input column of the
+// chunk); nothing is dereferenced unless `valid`.
+template <typename T, int PAT, int FMT>
+__device__ __forceinline__ ChunkOut make_out(const PassParams &p, int64_t row, int64_t col, bool valid, int lane)
 {
-    const PassParams p = operand_view(pk);
-    extern __shared__ __align__(1024) uint8_t smem[];
-    uint8_t *stages = smem;
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kStages * kStageBytes);
-    uint64_t *empty = full + kStages;
-    double *red = reinterpret_cast<double *>(empty + kStages); // [kConsumerWarps][4]
-    float *fred = reinterpret_cast<float *>(red + kConsumerWarps * 4); // [kConsumerWarps][2]
-    uint32_t *flag = reinterpret_cast<uint32_t *>(fred + kConsumerWarps * 2);
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kConsumerWarps);
-        }
-        fence_barrier_init();
+    const int64_t n = PAT == kDense ? p.k : p.k / 2;
+    const int64_t colq = PAT == kDense ? col : col / 2;
+    const int64_t off = row * n + colq; // index of the chunk's first quantized value
+    uint8_t *vals = static_cast<uint8_t *>(p.values);
+    uint8_t *sc = static_cast<uint8_t *>(p.scales);
+    ChunkOut o{nullptr, nullptr, nullptr, nullptr, valid, lane};
+    if constexpr (FMT == kNone) {
+        o.val = vals + off * static_cast<int64_t>(sizeof(T));
+    } else if constexpr (FMT == kFp8) {
+        o.val = vals + off;
+    } else if constexpr (FMT == kInt) {
+        o.val = vals + (p.q.store == kInt8 ? off : (p.q.store == kInt16 ? 2 * off : off / 2));
+        const int lg = __ffs(p.q.group) - 1; // tile-mode groups are powers of two
+        o.scale = sc + 4 * (row * (n >> lg) + (colq >> lg));
+    } else if constexpr (FMT == kNvfp4) {
+        o.val = vals + off / 2;
+        o.scale = sc + row * (n / 16) + colq / 16;
+    } else if constexpr (FMT == kMxfp4) {
+        o.val = vals + off / 2;
+        o.scale = sc + row * (n / 32) + colq / 32;
     }
-    __syncthreads();
-    grid_dependency_wait();
-    grid_dependents_launch();
+    if constexpr (PAT == kSparse24 && FMT != kAmax && FMT != kEnergy)
+        o.meta = p.meta + row * (p.k / 8) + col / 8;
+    else if constexpr (PAT == kSparse48 && FMT != kAmax && FMT != kEnergy)
+        o.meta = p.meta + row * (p.k / 16) + col / 16;
+    if (p.norms)
+        o.norms = p.norms + col;
+    return o;
+}
 
-    if (warp == kConsumerWarps) {
-        if (lane == 0)
-            producer(&map, p, stages, full, empty);
-        return;
-    }
-
-    // ---- consumers ----
+// Tensor scales, reciprocals and NVFP4 tables of a pass (every thread of the
+// CTA calls it; `nvt` is 512 floats of shared memory for the tables).
+template <int FMT>
+__device__ __forceinline__ PassConsts make_consts(const PassParams &p, int tid, int nthreads, float *nvt)
+{
     float st = 0.0f, std_ = 0.0f;
     if constexpr (FMT == kFp8 || FMT == kNvfp4 || FMT == kEnergy) {
         st = tensor_scale(p.q);
@@ -836,67 +859,185 @@ __global__ void __launch_bounds__(kThreads, 3) pass_kernel(const __grid_constant
     }
     if constexpr (FMT == kEnergy)
         std_ = tensor_scale(p.qd);
-    const Recip rst = make_recip(st), rstd = make_recip(std_);
-    float *nvt = reinterpret_cast<float *>(flag + 4); // 2 x 256 floats
+    PassConsts c;
+    c.rst = make_recip(st);
+    c.rstd = make_recip(std_);
+    c.guard = p.q.scale_in != nullptr;
+    c.guardd = p.qd.scale_in != nullptr;
+    c.tb = NvTable{nvt, nvt + 128};
+    c.tbd = NvTable{nvt + 256, nvt + 384};
     if constexpr (FMT == kNvfp4 || FMT == kEnergy) {
         build_nv_table(nvt, st, tid);
         build_nv_table(nvt + 256, std_, tid);
-        named_barrier_sync(1, kConsumers);
+        named_barrier_sync(1, nthreads);
     }
-    const NvTable tb{nvt, nvt + 128}, tbd{nvt + 256, nvt + 384};
+    return c;
+}
 
+// 16-byte global load that bypasses L1 (each input byte is read once).
+__device__ __forceinline__ uint4 ld_stream(const void *p)
+{
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+template <typename T> struct Stream;
+template <> struct Stream<__nv_bfloat16> {
+    __device__ __forceinline__ static Elem<__nv_bfloat16>::Raw load(const __nv_bfloat16 *p, bool ok)
+    {
+        Elem<__nv_bfloat16>::Raw r;
+        r.v = ok ? ld_stream(p) : make_uint4(0u, 0u, 0u, 0u);
+        return r;
+    }
+};
+template <> struct Stream<float> {
+    __device__ __forceinline__ static Elem<float>::Raw load(const float *p, bool ok)
+    {
+        Elem<float>::Raw r;
+        const uint4 a = ok ? ld_stream(p) : make_uint4(0u, 0u, 0u, 0u);
+        const uint4 b = ok ? ld_stream(p + 4) : make_uint4(0u, 0u, 0u, 0u);
+        r.a = make_float4(__uint_as_float(a.x), __uint_as_float(a.y), __uint_as_float(a.z), __uint_as_float(a.w));
+        r.b = make_float4(__uint_as_float(b.x), __uint_as_float(b.y), __uint_as_float(b.z), __uint_as_float(b.w));
+        return r;
+    }
+};
+
+// Resident CTAs per SM the stream kernel is compiled for (register budget).
+template <typename T, int PAT, int SCORE, int FMT> struct StreamOcc {
+    static constexpr int value = (FMT == kAmax || FMT == kNone) ? 4 : 3;
+};
+
+// Byte advance of each output between consecutive slots of a full-width unit
+// (slots 256 input columns apart); -1 where it depends on runtime fields (INT
+// code width and group).
+template <typename T, int PAT, int FMT> struct FwStep {
+    static constexpr int64_t q = PAT == kDense ? 256 : 128; // quantized values per slot
+    static constexpr int64_t val = FMT == kNone   ? q * static_cast<int64_t>(sizeof(T))
+                                   : FMT == kFp8  ? q
+                                   : (FMT == kNvfp4 || FMT == kMxfp4) ? q / 2
+                                                  : -1;
+    static constexpr int64_t scale = FMT == kNvfp4 ? q / 16 : FMT == kMxfp4 ? q / 32 : -1;
+    static constexpr int64_t meta = PAT == kSparse24 ? 32 : PAT == kSparse48 ? 16 : 0;
+};
+
+// One unit: four 16-byte loads per lane first, then the four chunks. FULL:
+// every chunk of the unit lies inside the operand (no per-chunk checks).
+template <typename T, int PAT, int SCORE, int FMT, bool FULL>
+__device__ __forceinline__ void stream_unit(const PassParams &p, const PassConsts &c, const T *xp, int64_t step_x,
+                                            int64_t step_c, const ChunkOut &o, int64_t dval, int64_t dscale,
+                                            int64_t dmeta, int64_t row0, int64_t col0, Acc &acc)
+{
     using E = Elem<T>;
-    const int cpr_mask = (1 << p.log2_cpr) - 1;
-    const bool energies = p.energy_out != nullptr;
+    typename E::Raw raw[4];
+    bool ok[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        ok[i] = FULL || (row0 + i * p.step_rows < p.rows && col0 + i * p.step_cols < p.k);
+        raw[i] = Stream<T>::load(xp + i * step_x, ok[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        ChunkOut oi = o;
+        oi.val += i * dval;
+        oi.scale += i * dscale;
+        oi.meta += i * dmeta;
+        if constexpr (SCORE == kWanda)
+            oi.norms = o.norms + i * step_c;
+        oi.valid = ok[i];
+        float xv[8];
+        E::unpack(raw[i], xv);
+        process_chunk<T, PAT, SCORE, FMT>(p, xv, oi, c, acc);
+    }
+}
+
+// The pass along axis 1 (k contiguous). A slot is 32 chunks, one per lane: a
+// row segment of W = 8 * cpr columns for each of 32 / cpr rows (lane = row
+// offset * cpr + chunk). A unit is four slots, either four consecutive
+// segments of the same rows (step_cols = W) or the same segment of four
+// consecutive row groups (step_rows = 32 / cpr); a warp loads the unit's
+// four chunks per lane (16-byte loads, 512 contiguous bytes per slot) before
+// processing them. The warps serving an operand take units u = warp index,
+// warp index + number of warps, ... The CTA count per operand and the layout
+// are chosen by the host. FW: the full-width case W = 256 with four segments
+// per unit, where the slot offsets are compile-time constants and a unit
+// wholly inside the operand skips the per-chunk checks.
+template <typename T, int PAT, int SCORE, int FMT, bool FW>
+__global__ void __launch_bounds__(kStreamThreads, (StreamOcc<T, PAT, SCORE, FMT>::value))
+    stream_kernel(const PassParams pk)
+{
+    const PassParams p = operand_view(pk);
+    __shared__ double red[kStreamWarps * 4];
+    __shared__ float fred[kStreamWarps * 2];
+    __shared__ uint32_t flag;
+    __shared__ float nvt[(FMT == kNvfp4 || FMT == kEnergy) ? 512 : 4];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    grid_dependency_wait();
+    grid_dependents_launch();
+    const PassConsts c = make_consts<FMT>(p, tid, kStreamThreads, nvt);
+
+    const T *x = static_cast<const T *>(p.x) + p.op * p.x_bstride;
+    const int log2_cpr = FW ? 5 : p.log2_cpr;
+    const int lrow = lane >> log2_cpr;
+    const int lcol = (lane & ((1 << log2_cpr) - 1)) << 3;
+    const int64_t step_x = FW ? 256 : static_cast<int64_t>(p.step_rows) * p.ld + p.step_cols;
+    const int64_t step_c = FW ? 256 : p.step_cols;
+    // pointer advance per slot of a unit (the output offsets are linear in
+    // row and column, and a step never splits a scale group)
+    const ChunkOut z0 = make_out<T, PAT, FMT>(p, 0, 0, false, lane);
+    const ChunkOut z1 = make_out<T, PAT, FMT>(p, FW ? 0 : p.step_rows, FW ? 256 : p.step_cols, false, lane);
+    using FS = FwStep<T, PAT, FMT>;
+    const int64_t dval = (FW && FS::val >= 0) ? FS::val : z1.val - z0.val;
+    const int64_t dscale = (FW && FS::scale >= 0) ? FS::scale : z1.scale - z0.scale;
+    const int64_t dmeta = FW ? FS::meta : z1.meta - z0.meta;
+    const int unit_rows = FW ? 1 : p.unit_rows;
+    const int unit_cols = FW ? 1024 : p.unit_cols;
+
+    const int tw = p.ctas_per_op * kStreamWarps;
+    const int u0 = p.cta * kStreamWarps + warp;
+    int ua = u0 / p.units_b, ub = u0 - ua * p.units_b;
+    const int sa = tw / p.units_b, sb = tw - sa * p.units_b;
     double e_total = 0.0, e_prune = 0.0, e_q = 0.0, e_qd = 0.0;
     Acc acc{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    uint32_t it = 0;
-    for (int64_t t = p.cta; t < p.n_tiles; t += p.ctas_per_op, ++it) {
-        const int s = it % kStages;
-        if (!mbar_wait(&full[s], (it / kStages) & 1)) {
-            record_error(p.err, 2);
-            break;
-        }
-        const uint8_t *tile = stages + s * kStageBytes;
-        typename E::Raw raw[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            if (i < p.cpt)
-                raw[i] = E::load(tile, tid + i * kConsumers);
-        __syncwarp();
-        if (lane == 0)
-            mbar_arrive(&empty[s]);
-
-        const int64_t rt = t / p.n_col_tiles, ct = t - rt * p.n_col_tiles;
-        const int64_t row0 = rt * p.R, col0 = ct * p.W;
+    while (ua < p.units_a) {
+        const int64_t row0 = static_cast<int64_t>(ua) * unit_rows + lrow;
+        const int64_t col0 = static_cast<int64_t>(ub) * unit_cols + lcol;
+        const T *xp = x + row0 * p.ld + col0;
+        const ChunkOut o = make_out<T, PAT, FMT>(p, row0, col0, true, lane);
         acc.et = acc.ep = acc.eq = acc.eqd = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            if (i < p.cpt) {
-                const int j = tid + i * kConsumers;
-                const int64_t row = row0 + (j >> p.log2_cpr);
-                const int64_t col = col0 + ((j & cpr_mask) << 3);
-                float x[8];
-                E::unpack(raw[i], x);
-                process_chunk<T, PAT, SCORE, FMT>(p, x, row, col, lane, rst, rstd, acc, -1.0f, nullptr, tb, tbd);
-            }
-        }
-        if constexpr (FMT != kAmax) {
+        // full-width units lie inside the operand except in the last quad
+        // of a row (rows are whole: one row per unit)
+        if (FW && static_cast<int64_t>(ub + 1) * 1024 <= p.k)
+            stream_unit<T, PAT, SCORE, FMT, true>(p, c, xp, step_x, step_c, o, dval, dscale, dmeta, row0, col0,
+                                                  acc);
+        else
+            stream_unit<T, PAT, SCORE, FMT, false>(p, c, xp, step_x, step_c, o, dval, dscale, dmeta, row0, col0,
+                                                   acc);
+        // only the energies this pass produces (the others stay zero)
+        if constexpr (FMT != kAmax)
             e_total += acc.et;
+        if constexpr (FMT != kAmax && PAT != kDense)
             e_prune += acc.ep;
+        if constexpr (FMT != kAmax && FMT != kNone && PAT != kDense)
             e_q += acc.eq;
+        if constexpr (FMT != kAmax && FMT != kNone && (PAT == kDense || FMT == kEnergy))
             e_qd += acc.eqd;
+        ua += sa;
+        ub += sb;
+        if (ub >= p.units_b) {
+            ub -= p.units_b;
+            ++ua;
         }
     }
 
-    // ---- grid reductions (last CTA to finish reduces the partials) ----
     if constexpr (FMT == kAmax) {
-        grid_reduce_amax<PAT>(p, acc.amax_kept, acc.amax_all, fred, flag, tid, lane, warp);
-        return;
+        grid_reduce_amax<PAT>(p, acc.amax_kept, acc.amax_all, fred, &flag, tid, lane, warp);
     } else {
-        if (!energies)
+        if (!p.energy_out)
             return;
-        grid_reduce_energy(p, e_total, e_prune, e_q, e_qd, red, flag, tid, lane, warp);
+        grid_reduce_energy(p, e_total, e_prune, e_q, e_qd, red, &flag, tid, lane, warp);
     }
 }
 
@@ -948,7 +1089,8 @@ __global__ void __launch_bounds__(kRowThreads) rowsweep_kernel(const T *__restri
     grid_dependency_wait();
     grid_dependents_launch();
     const int nchunks = static_cast<int>(p.k / 8);
-    const Recip no_recip = make_recip(0.0f);
+    const PassConsts nc{make_recip(0.0f), make_recip(0.0f), NvTable{nullptr, nullptr}, NvTable{nullptr, nullptr},
+                        false, false};
     double e_total = 0.0, e_prune = 0.0, e_q = 0.0, e_qd = 0.0;
     for (int64_t row = static_cast<int64_t>(p.cta) * kConsumerWarps + warp; row < p.rows;
          row += static_cast<int64_t>(p.ctas_per_op) * kConsumerWarps) {
@@ -972,8 +1114,8 @@ __global__ void __launch_bounds__(kRowThreads) rowsweep_kernel(const T *__restri
                         amax = fmaxf(amax, local_amax<8>(xv));
                     } else {
                         Acc a{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                        process_chunk<T, PAT, SCORE, kAmax>(p, xv, row, static_cast<int64_t>(c) * 8, lane,
-                                                            no_recip, no_recip, a);
+                        process_chunk<T, PAT, SCORE, kAmax>(
+                            p, xv, make_out<T, PAT, kAmax>(p, row, static_cast<int64_t>(c) * 8, true, lane), nc, a);
                         amax = fmaxf(amax, a.amax_kept);
                     }
                 }
@@ -1001,8 +1143,9 @@ __global__ void __launch_bounds__(kRowThreads) rowsweep_kernel(const T *__restri
                     float xv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
                     if (c < nchunks)
                         buf[u].unpack(xv);
-                    process_chunk<T, PAT, SCORE, kInt>(p, xv, row, static_cast<int64_t>(c) * 8, lane, no_recip,
-                                                       no_recip, acc, amax, &rs);
+                    process_chunk<T, PAT, SCORE, kInt>(
+                        p, xv, make_out<T, PAT, kInt>(p, row, static_cast<int64_t>(c) * 8, c < nchunks, lane), nc,
+                        acc, amax, &rs);
                 }
             }
         }
@@ -1142,22 +1285,8 @@ __global__ void __launch_bounds__(kThreads, 1) axis0_kernel(const __grid_constan
         return;
     }
 
-    float st = 0.0f, std_ = 0.0f;
-    if constexpr (FMT == kFp8 || FMT == kNvfp4 || FMT == kEnergy) {
-        st = tensor_scale(p.q);
-        if (p.cta == 0 && tid == 0 && p.q.scale_out)
-            *p.q.scale_out = st;
-    }
-    if constexpr (FMT == kEnergy)
-        std_ = tensor_scale(p.qd);
-    const Recip rst = make_recip(st), rstd = make_recip(std_);
     float *nvt = reinterpret_cast<float *>(ready + 4); // 2 x 256 floats
-    if constexpr (FMT == kNvfp4 || FMT == kEnergy) {
-        build_nv_table(nvt, st, tid);
-        build_nv_table(nvt + 256, std_, tid);
-        named_barrier_sync(1, kConsumers);
-    }
-    const NvTable tb{nvt, nvt + 128}, tbd{nvt + 256, nvt + 384};
+    const PassConsts c = make_consts<FMT>(p, tid, kConsumers, nvt);
     using A0 = Axis0<T>;
     double e_total = 0.0, e_prune = 0.0, e_q = 0.0, e_qd = 0.0;
     Acc acc{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -1196,8 +1325,9 @@ __global__ void __launch_bounds__(kThreads, 1) axis0_kernel(const __grid_constan
                 const int j = tid + i * kConsumers;
                 float x[8];
                 Elem<T>::unpack(raw[i], x);
-                process_chunk<T, PAT, SCORE, FMT>(p, x, row0 + (j >> 4), col0 + ((j & 15) << 3), lane, rst,
-                                                  rstd, acc, -1.0f, nullptr, tb, tbd);
+                const int64_t row = row0 + (j >> 4), col = col0 + ((j & 15) << 3);
+                process_chunk<T, PAT, SCORE, FMT>(
+                    p, x, make_out<T, PAT, FMT>(p, row, col, row < p.rows && col < p.k, lane), c, acc);
             }
         }
         if constexpr (FMT != kAmax) {

@@ -5,6 +5,9 @@ Nsight Compute) or for a quick timing of one configuration:
 
     python -m semi_structured_sparsity_online_b200.run_case --pass fused_24_fp8 --m 4096 --k 4096 --iters 3
 
+With --batch B the pass runs as one batched launch over B operands of that
+shape (a [B, m, k] tensor).
+
 Passes: tensor_scale, fused_24_{none,fp8,nvfp4,mxfp4,int8g128}, fused_48_nvfp4,
 dense_{fp8,nvfp4,mxfp4,int8_row,int8g128}, error_energy. Prints the mean CUDA-event
 time per launch and the GB/s of the pass's algorithmic bytes.
@@ -62,16 +65,24 @@ def main():
     ap.add_argument("--k", type=int, default=4096)
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--seed", type=int, default=8)
+    ap.add_argument("--batch", type=int, default=0, help="0: one 2-D operand; B: one launch over B operands")
     args = ap.parse_args()
-    xb = synth.sweep_operand(args.m, args.k, seed=args.seed)
+    nb = max(args.batch, 1)
+    xb = np.stack([synth.sweep_operand(args.m, args.k, seed=args.seed + i) for i in range(nb)])
     x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).cuda()
+    if args.batch == 0:
+        x = x[0]
+    lead = None if args.batch == 0 else args.batch
     ws = ss24.Workspace()
-    e = torch.zeros(4, dtype=torch.float64, device="cuda")
+    e = torch.zeros((nb, 4), dtype=torch.float64, device="cuda")
+    if args.batch == 0:
+        e = e[0]
     scale = ss24.tensor_scale(x, "fp8", ss24.SPARSE_24, ws=ws)
     out = None
     if args.name in PASSES:
         pattern, fmt, bits, group = PASSES[args.name]
-        out = ss24._alloc_outputs(args.m, args.k, pattern, ss24.make_format(fmt, bits, group), torch.bfloat16, "cuda")
+        out = ss24._alloc_outputs(args.m, args.k, pattern, ss24.make_format(fmt, bits, group), torch.bfloat16, "cuda",
+                                  lead)
         if fmt == "nvfp4":
             scale = ss24.tensor_scale(x, "nvfp4", pattern if pattern != ss24.DENSE else ss24.DENSE, ws=ws)
 
@@ -95,9 +106,9 @@ def main():
     t.record()
     t.synchronize()
     us = s.elapsed_time(t) / args.iters * 1e3
-    gb = pass_bytes(args.name, args.m, args.k)
+    gb = nb * pass_bytes(args.name, args.m, args.k)
     assert ws.error() == 0
-    print(f"{args.name} m={args.m} k={args.k}: {us:.2f} us/launch, {gb / us / 1e3:.1f} GB/s "
+    print(f"{args.name} m={args.m} k={args.k} batch={args.batch}: {us:.2f} us/launch, {gb / us / 1e3:.1f} GB/s "
           f"({gb} algorithmic bytes per launch; warm L2 between launches)")
 
 
