@@ -365,7 +365,13 @@ ss24_status ss24_decode_e2m1(const uint8_t *in, float *out, int64_t n, ss24_stre
  * b_count <= 2^23 — all 2^23 values of b together cover every pair of
  * significands, which by exact power-of-two scaling covers every a and b the
  * kernels divide with the correction). mode 1: 2^23 pseudo-random pairs per
- * unit of b_count, exponents across the corrected range. Adds the number of
+ * unit of b_count, exponents across the corrected range. mode 2 checks the
+ * packed bf16 operations the 2:4 selection and the amax use (magnitude
+ * comparison through a rounded bf16 difference, magnitude maximum, bf16 to
+ * binary32 conversion and squares on the multiply-add unit) for the magnitude
+ * bits a = b_first + j, j < b_count (b_first + b_count <= 2^15), against every
+ * magnitude b < 2^15, finite values only, both signs; a mismatch is reported as
+ * (a << 32 | b). Adds the number of
  * mismatches to result[0] and lowers result[1] to the first mismatch
  * (a bits << 32 | b bits); result is a device array of two uint64 the caller
  * initialises to {0, UINT64_MAX}. */

@@ -16,6 +16,8 @@ const void *stream_kernel_bf16(int pattern, int score, int fmt, bool fw);
 const void *stream_kernel_f32(int pattern, int score, int fmt, bool fw);
 const void *rowsweep_kernel_bf16(int pattern, int score);
 const void *rowsweep_kernel_f32(int pattern, int score);
+const void *rowblock_kernel_bf16(int pattern, int score, int cpt);
+const void *rowblock_kernel_f32(int pattern, int score, int cpt);
 const void *axis0_kernel_bf16(int pattern, int score, int fmt);
 const void *axis0_kernel_f32(int pattern, int score, int fmt);
 } // namespace ss24
@@ -202,6 +204,46 @@ cudaError_t launch_rowsweep(const void *k, const ss24_operand *x, const PassPara
     const void *xp = x->x;
     int64_t ld = x->ld;
     void *args[3] = {&xp, &ld, &pp};
+    return launch_pdl(k, static_cast<unsigned>(p.batch * pp.ctas_per_op), kRowThreads, 0, stream, args);
+}
+
+// One scale per row with the row in registers: cpt chunks per thread, tpr
+// threads per row (a power of two in [32, 256]), 256 / tpr rows per CTA step.
+// Rows longer than 2048 chunks (k > 16384) take the two-sweep kernel instead.
+bool rowblock_plan(int64_t k, int *cpt, int *log2_tpr)
+{
+    const int64_t nchunks = k / 8;
+    int c;
+    if (nchunks <= 32)
+        c = 1;
+    else if (nchunks <= 1024)
+        c = 4;
+    else if (nchunks <= 2048)
+        c = 8;
+    else
+        return false;
+    int64_t tpr = 32;
+    while (tpr * c < nchunks)
+        tpr *= 2;
+    *cpt = c;
+    *log2_tpr = ilog2(tpr);
+    return true;
+}
+
+cudaError_t launch_rowblock(const void *k, const ss24_operand *x, int log2_tpr, const PassParams &p,
+                            cudaStream_t stream)
+{
+    KernelInfo info;
+    cudaError_t e = kernel_info(k, 0, &info, kRowThreads);
+    if (e != cudaSuccess)
+        return e;
+    const int64_t rows_per_cta = kRowThreads >> log2_tpr;
+    PassParams pp = p;
+    pp.ctas_per_op = static_cast<int32_t>(ctas_per_operand(info, p.batch, (x->rows + rows_per_cta - 1) / rows_per_cta));
+    const void *xp = x->x;
+    int64_t ld = x->ld;
+    int32_t lt = log2_tpr;
+    void *args[4] = {&xp, &ld, &lt, &pp};
     return launch_pdl(k, static_cast<unsigned>(p.batch * pp.ctas_per_op), kRowThreads, 0, stream, args);
 }
 
@@ -590,7 +632,12 @@ ss24_status run_pass(const ss24_operand *x, int pattern, int score, const float 
         }
     }
     cudaError_t e;
-    if (r.row_mode) {
+    int cpt = 0, log2_tpr = 0;
+    if (r.row_mode && rowblock_plan(x->k, &cpt, &log2_tpr)) {
+        const void *k = x->dtype == SS24_BF16 ? rowblock_kernel_bf16(pattern, score, cpt)
+                                              : rowblock_kernel_f32(pattern, score, cpt);
+        e = launch_rowblock(k, x, log2_tpr, p, stream);
+    } else if (r.row_mode) {
         const void *k = x->dtype == SS24_BF16 ? rowsweep_kernel_bf16(pattern, score) : rowsweep_kernel_f32(pattern, score);
         e = launch_rowsweep(k, x, p, stream);
     } else {
@@ -910,9 +957,11 @@ ss24_status ss24_selfcheck_division(int32_t mode, uint32_t b_first, uint32_t b_c
 {
     if (!result)
         return SS24_ERR_NULL;
-    if (mode != 0 && mode != 1)
+    if (mode < 0 || mode > 2)
         return SS24_ERR_ARG;
     if (mode == 0 && (b_first >= (1u << 23) || b_count > (1u << 23) - b_first))
+        return SS24_ERR_SHAPE;
+    if (mode == 2 && (b_first >= (1u << 15) || b_count > (1u << 15) - b_first))
         return SS24_ERR_SHAPE;
     if (b_count > 65535u * 32u)
         return SS24_ERR_SHAPE;

@@ -251,6 +251,69 @@ __device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c)
 }
 
 // ---------------------------------------------------------------------------
+// packed bf16 pairs (two 16-bit lanes of a 32-bit word, lane 0 in the low half)
+// ---------------------------------------------------------------------------
+
+// bf16 lane -> binary32 (exact) computed on the FMA pipe: a mixed-precision
+// add of -0, which leaves every value (signed zeros included) unchanged.
+__device__ __forceinline__ float bf16_lo(uint32_t w)
+{
+    float r;
+    asm("{ .reg .b16 l, h; mov.b32 {l, h}, %1; add.rn.f32.bf16 %0, l, 0f80000000; }" : "=f"(r) : "r"(w));
+    return r;
+}
+__device__ __forceinline__ float bf16_hi(uint32_t w)
+{
+    float r;
+    asm("{ .reg .b16 l, h; mov.b32 {l, h}, %1; add.rn.f32.bf16 %0, h, 0f80000000; }" : "=f"(r) : "r"(w));
+    return r;
+}
+// RN(l * l + c) and RN(h * h + c) for the lanes of w (products of bf16 values
+// are exact in binary32, so these equal the binary32 fused multiply-add)
+__device__ __forceinline__ float bf16_sq_lo(uint32_t w, float c)
+{
+    float r;
+    asm("{ .reg .b16 l, h; mov.b32 {l, h}, %1; fma.rn.f32.bf16 %0, l, l, %2; }" : "=f"(r) : "r"(w), "f"(c));
+    return r;
+}
+__device__ __forceinline__ float bf16_sq_hi(uint32_t w, float c)
+{
+    float r;
+    asm("{ .reg .b16 l, h; mov.b32 {l, h}, %1; fma.rn.f32.bf16 %0, h, h, %2; }" : "=f"(r) : "r"(w), "f"(c));
+    return r;
+}
+
+// Per lane: a value whose magnitude is max(|a|, |b|) (its sign is not
+// meaningful). Exact: a maximum selects one of its inputs.
+__device__ __forceinline__ uint32_t bf16x2_maxabs(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+// The larger magnitude of the two lanes as binary32 (magnitude bit patterns
+// of non-NaN values order like the values).
+__device__ __forceinline__ float bf16x2_hmax(uint32_t m)
+{
+    return __uint_as_float(max(m & 0x7fffu, (m >> 16) & 0x7fffu) << 16);
+}
+
+// Per lane: all ones where |b| > |a|, else zero. |a| - |b| is computed in
+// bf16 with rounding to nearest, which keeps the sign of the exact difference
+// and is zero (+0) only when the magnitudes are equal (gradual underflow);
+// the sign bit of each lane is then replicated across it (prmt sign mode).
+__device__ __forceinline__ uint32_t bf16x2_gt_abs(uint32_t b, uint32_t a)
+{
+    uint32_t d, m;
+    asm("{ .reg .b32 aa, bb; abs.bf16x2 aa, %1; abs.bf16x2 bb, %2; sub.rn.bf16x2 %0, aa, bb; }"
+        : "=r"(d)
+        : "r"(a), "r"(b));
+    asm("prmt.b32 %0, %1, 0, 0xBB99;" : "=r"(m) : "r"(d));
+    return m;
+}
+__device__ __forceinline__ uint32_t sel_mask(uint32_t m, uint32_t a, uint32_t b) { return (a & m) | (b & ~m); }
+
+// ---------------------------------------------------------------------------
 // division by a scale
 // ---------------------------------------------------------------------------
 
@@ -405,6 +468,47 @@ __device__ __forceinline__ Group24 group24(float x0, float x1, float x2, float x
     g.e_drop = both01 ? e23 : (both23 ? e01 : el);
     const uint32_t mixed = (p ? 1u : 0u) + (q ? 12u : 8u);
     g.nib = both01 ? 0x4u : (both23 ? 0xEu : mixed);
+    return g;
+}
+
+// The two 2:4 groups of a chunk of eight bf16 values (words w0..w3, element
+// 2i in the low half of word i) by magnitude, both at once: lane 0 of every
+// packed word below is group 0, lane 1 group 1. The same tournament as
+// group24, with the comparisons from bf16x2_gt_abs and the choices as bit
+// selects. Results: kept values k0 (lower index) and k1 per lane, the
+// metadata byte (group 0 in the low nibble), the chunk's energy and the
+// energy of its dropped values, summed in the same order as group24.
+struct Pair24 {
+    uint32_t k0, k1, meta;
+    float e_all, e_drop;
+};
+
+__device__ __forceinline__ Pair24 pair24_bf16(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3)
+{
+    const uint32_t A = __byte_perm(w0, w2, 0x5410), B = __byte_perm(w0, w2, 0x7632); // x0 | x4, x1 | x5
+    const uint32_t C = __byte_perm(w1, w3, 0x5410), D = __byte_perm(w1, w3, 0x7632); // x2 | x6, x3 | x7
+    const uint32_t mp = bf16x2_gt_abs(B, A);            // p: |x1| > |x0|
+    const uint32_t mq = bf16x2_gt_abs(D, C);            // q: |x3| > |x2|
+    const uint32_t w01 = sel_mask(mp, B, A), l01 = sel_mask(mp, A, B);
+    const uint32_t w23 = sel_mask(mq, D, C), l23 = sel_mask(mq, C, D);
+    const uint32_t mr = bf16x2_gt_abs(w23, w01);        // r: first place from pair (2,3)
+    const uint32_t ma = bf16x2_gt_abs(w23, l01);        // ta
+    const uint32_t mb = bf16x2_gt_abs(l23, w01);        // tb
+    const uint32_t m01 = ~(mr | ma), m23 = mr & mb;     // both kept from (0,1) / from (2,3)
+    Pair24 g;
+    g.k0 = sel_mask(m01, A, sel_mask(m23, C, w01));
+    g.k1 = sel_mask(m01, B, sel_mask(m23, D, w23));
+    const uint32_t d0 = sel_mask(m01, C, sel_mask(m23, A, l01));
+    const uint32_t d1 = sel_mask(m01, D, sel_mask(m23, B, l23));
+    // nibble i0 | i1 << 2: (0,1) -> 4, (2,3) -> 14, otherwise p | (2 + q) << 2
+    const uint32_t mixed = 0x00080008u | (mp & 0x00010001u) | (mq & 0x00040004u);
+    const uint32_t nib = sel_mask(m01, 0x00040004u, sel_mask(m23, 0x000E000Eu, mixed));
+    g.meta = (nib | (nib >> 12)) & 0xffu;
+    // energies: (x0^2 + x1^2) + (x2^2 + x3^2) per group, dropped d0^2 + d1^2
+    const float e01a = bf16_sq_lo(B, bf16_sq_lo(A, -0.0f)), e23a = bf16_sq_lo(D, bf16_sq_lo(C, -0.0f));
+    const float e01b = bf16_sq_hi(B, bf16_sq_hi(A, -0.0f)), e23b = bf16_sq_hi(D, bf16_sq_hi(C, -0.0f));
+    g.e_all = (e01a + e23a) + (e01b + e23b);
+    g.e_drop = bf16_sq_lo(d1, bf16_sq_lo(d0, -0.0f)) + bf16_sq_hi(d1, bf16_sq_hi(d0, -0.0f));
     return g;
 }
 

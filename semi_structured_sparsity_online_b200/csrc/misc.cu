@@ -93,7 +93,7 @@ __global__ void selfcheck_division_kernel(int mode, uint32_t b_first, unsigned l
                 first = min(first, (static_cast<unsigned long long>(__float_as_uint(a)) << 32) | __float_as_uint(b));
             }
         }
-    } else {
+    } else if (mode == 1) {
         for (uint32_t i = threadIdx.x; i < (1u << 23); i += blockDim.x) {
             const uint32_t h1 = hash32(((b_first + blockIdx.x) << 23) ^ i), h2 = hash32(h1 ^ 0x9e3779b9u);
             const uint32_t h3 = hash32(h2 + 0x632be5abu);
@@ -112,6 +112,33 @@ __global__ void selfcheck_division_kernel(int mode, uint32_t b_first, unsigned l
                 __float_as_uint(hi2(nq)) != __float_as_uint(ref)) {
                 ++bad;
                 first = min(first, (static_cast<unsigned long long>(__float_as_uint(a)) << 32) | __float_as_uint(b));
+            }
+        }
+    } else {
+        // mode 2: the packed bf16 operations of the selection and the amax,
+        // for a = b_first + blockIdx.x against every b (magnitude bits < 2^15,
+        // finite), signs taken from the low bits of the other operand
+        const uint32_t a = b_first + blockIdx.x;
+        for (uint32_t b = threadIdx.x; b < 32768u; b += blockDim.x) {
+            if (((a >> 7) & 0xffu) == 0xffu || ((b >> 7) & 0xffu) == 0xffu)
+                continue;
+            const uint32_t sa = (b & 1u) << 15, sb = (a & 1u) << 15;
+            const uint32_t ha = a | sa, hb = b | sb;
+            const uint32_t u = ha | (hb << 16), v = hb | (ha << 16);   // lanes (a, b) and (b, a)
+            const uint32_t gt = bf16x2_gt_abs(v, u);                    // lane 0: |b| > |a|; lane 1: |a| > |b|
+            const uint32_t mx = bf16x2_maxabs(u, v);
+            const float fa = __uint_as_float(ha << 16), fb = __uint_as_float(hb << 16);
+            bool ok = gt == ((b > a ? 0xffffu : 0u) | (a > b ? 0xffff0000u : 0u));
+            ok = ok && (mx & 0x7fffu) == max(a, b) && ((mx >> 16) & 0x7fffu) == max(a, b);
+            ok = ok && bf16x2_hmax(u) == fmaxf(fabsf(fa), fabsf(fb));
+            ok = ok && __float_as_uint(bf16_lo(u)) == __float_as_uint(fa) &&
+                 __float_as_uint(bf16_hi(u)) == __float_as_uint(fb);
+            const float c = __uint_as_float(hash32(a * 32768u + b) & 0xbf7fffffu);   // finite addend
+            ok = ok && __float_as_uint(bf16_sq_lo(u, c)) == __float_as_uint(__fmaf_rn(fa, fa, c)) &&
+                 __float_as_uint(bf16_sq_hi(u, c)) == __float_as_uint(__fmaf_rn(fb, fb, c));
+            if (!ok) {
+                ++bad;
+                first = min(first, (static_cast<unsigned long long>(a) << 32) | b);
             }
         }
     }

@@ -14,4 +14,8 @@ const void *axis0_kernel_bf16(int pattern, int score, int fmt)
 {
     return axis0_kernel_ptr<__nv_bfloat16>(pattern, score, fmt);
 }
+const void *rowblock_kernel_bf16(int pattern, int score, int cpt)
+{
+    return rowblock_kernel_ptr<__nv_bfloat16>(pattern, score, cpt);
+}
 } // namespace ss24

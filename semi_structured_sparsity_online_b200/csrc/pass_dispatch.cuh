@@ -62,6 +62,30 @@ template <typename T> const void *rowsweep_kernel_ptr(int pattern, int score)
     return nullptr;
 }
 
+template <typename T, int PAT, int SC> const void *rowblock_for_cpt(int cpt)
+{
+    switch (cpt) {
+    case 1:
+        return reinterpret_cast<const void *>(&rowblock_kernel<T, PAT, SC, 1>);
+    case 4:
+        return reinterpret_cast<const void *>(&rowblock_kernel<T, PAT, SC, 4>);
+    case 8:
+        return reinterpret_cast<const void *>(&rowblock_kernel<T, PAT, SC, 8>);
+    }
+    return nullptr;
+}
+
+template <typename T> const void *rowblock_kernel_ptr(int pattern, int score, int cpt)
+{
+    if (pattern == kDense)
+        return rowblock_for_cpt<T, kDense, kMag>(cpt);
+    if (pattern == kSparse24)
+        return score == kWanda ? rowblock_for_cpt<T, kSparse24, kWanda>(cpt) : rowblock_for_cpt<T, kSparse24, kMag>(cpt);
+    if (pattern == kSparse48)
+        return score == kWanda ? rowblock_for_cpt<T, kSparse48, kWanda>(cpt) : rowblock_for_cpt<T, kSparse48, kMag>(cpt);
+    return nullptr;
+}
+
 template <typename T, int PAT, int SC> const void *axis0_for_fmt(int fmt)
 {
     switch (fmt) {

@@ -14,4 +14,8 @@ const void *axis0_kernel_f32(int pattern, int score, int fmt)
 {
     return axis0_kernel_ptr<float>(pattern, score, fmt);
 }
+const void *rowblock_kernel_f32(int pattern, int score, int cpt)
+{
+    return rowblock_kernel_ptr<float>(pattern, score, cpt);
+}
 } // namespace ss24

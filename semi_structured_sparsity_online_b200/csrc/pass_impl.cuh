@@ -47,8 +47,8 @@ template <> struct Elem<__nv_bfloat16> {
         const uint32_t w[4] = {r.v.x, r.v.y, r.v.z, r.v.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            x[2 * i] = __uint_as_float(w[i] << 16);
-            x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+            x[2 * i] = bf16_lo(w[i]);
+            x[2 * i + 1] = bf16_hi(w[i]);
         }
     }
 };
@@ -170,11 +170,12 @@ __device__ __forceinline__ void scale_values(const float (&c)[VPC], float s, flo
 // With `guard` false the caller knows that no quotient can overflow (the scale
 // was derived from the amax of the values quantized).
 template <int VPC, bool STORE>
-__device__ __forceinline__ float quant_fp8(const float (&v)[VPC], const Recip &rc, bool guard, const ChunkOut &o)
+__device__ __forceinline__ float quant_fp8(const float (&v)[VPC], float vmax, const Recip &rc, bool guard,
+                                           const ChunkOut &o)
 {
     bool fast = rc.fast;
     if (guard)
-        fast = quot_fast(rc, local_amax<VPC>(v));
+        fast = quot_fast(rc, vmax);
     float qn[VPC], dec[VPC], d[VPC];
     neg_quotients<VPC>(v, rc, fast, qn);
     uint32_t c[VPC / 4];
@@ -229,7 +230,7 @@ struct RowScale {
 };
 
 template <int VPC, bool STORE>
-__device__ __forceinline__ float quant_int(const float (&v)[VPC], const QuantSpec &q, const ChunkOut &o,
+__device__ __forceinline__ float quant_int(const float (&v)[VPC], float vmax, const QuantSpec &q, const ChunkOut &o,
                                            float row_amax = -1.0f, const RowScale *rs = nullptr)
 {
     float amax, scale;
@@ -239,7 +240,7 @@ __device__ __forceinline__ float quant_int(const float (&v)[VPC], const QuantSpe
         scale = rs->scale;
         rc = rs->rc;
     } else {
-        amax = row_amax >= 0.0f ? row_amax : group_amax(local_amax<VPC>(v), q.lanes);
+        amax = row_amax >= 0.0f ? row_amax : group_amax(vmax, q.lanes);
         scale = int_scale(amax, q);
         rc = make_recip(scale);
     }
@@ -358,12 +359,12 @@ __device__ __forceinline__ void build_nv_table(float *t, float st, int tid)
 }
 
 template <int VPC, bool STORE>
-__device__ __forceinline__ float quant_nvfp4(const float (&v)[VPC], const Recip &rst, const ChunkOut &o,
-                                             const NvTable &tb)
+__device__ __forceinline__ float quant_nvfp4(const float (&v)[VPC], float vmax, const Recip &rst,
+                                             const ChunkOut &o, const NvTable &tb)
 {
     constexpr int kLanes = 16 / VPC;
     const float st = rst.b;
-    const float amax = group_amax(local_amax<VPC>(v), kLanes);
+    const float amax = group_amax(vmax, kLanes);
     uint32_t sb = 0;
     if (st != 0.0f) {
         // (amax / 6) / st: two correctly rounded divisions
@@ -398,10 +399,10 @@ __device__ __forceinline__ float quant_nvfp4(const float (&v)[VPC], const Recip 
 // the E8M0 byte e + 127; v / 2^e is computed as v * 2^-e (the same correctly
 // rounded value, since both scale factors are exact powers of two).
 template <int VPC, bool STORE>
-__device__ __forceinline__ float quant_mxfp4(const float (&v)[VPC], const ChunkOut &o)
+__device__ __forceinline__ float quant_mxfp4(const float (&v)[VPC], float vmax, const ChunkOut &o)
 {
     constexpr int kLanes = 32 / VPC;
-    const float amax = group_amax(local_amax<VPC>(v), kLanes);
+    const float amax = group_amax(vmax, kLanes);
     uint32_t byte = 0;
     float inv = 0.0f, mult = 0.0f;
     if (amax != 0.0f) {
@@ -422,19 +423,19 @@ __device__ __forceinline__ float quant_mxfp4(const float (&v)[VPC], const ChunkO
 
 // Runtime-dispatched quantizer without stores (the energy-only pass).
 template <int VPC>
-__device__ __forceinline__ float quant_energy_only(const float (&v)[VPC], const QuantSpec &q, const Recip &rst,
-                                                   bool guard, const NvTable &tb)
+__device__ __forceinline__ float quant_energy_only(const float (&v)[VPC], float vmax, const QuantSpec &q,
+                                                   const Recip &rst, bool guard, const NvTable &tb)
 {
     const ChunkOut o{nullptr, nullptr, nullptr, nullptr, false, 0};
     switch (q.fmt) {
     case kFp8:
-        return quant_fp8<VPC, false>(v, rst, guard, o);
+        return quant_fp8<VPC, false>(v, vmax, rst, guard, o);
     case kInt:
-        return quant_int<VPC, false>(v, q, o);
+        return quant_int<VPC, false>(v, vmax, q, o);
     case kNvfp4:
-        return quant_nvfp4<VPC, false>(v, rst, o, tb);
+        return quant_nvfp4<VPC, false>(v, vmax, rst, o, tb);
     case kMxfp4:
-        return quant_mxfp4<VPC, false>(v, o);
+        return quant_mxfp4<VPC, false>(v, vmax, o);
     default:
         return 0.0f;
     }
@@ -478,26 +479,59 @@ __device__ __forceinline__ void scores(const float (&x)[8], const ChunkOut &o, f
     }
 }
 
+// The largest magnitude of a chunk's eight input values: packed bf16 lanes for
+// bf16 operands, else from the unpacked values.
+template <typename T>
+__device__ __forceinline__ float chunk_amax(const typename Elem<T>::Raw &raw, const float (&x)[8])
+{
+    if constexpr (sizeof(T) == 2) {
+        const uint4 w = raw.v;
+        return bf16x2_hmax(bf16x2_maxabs(bf16x2_maxabs(w.x, w.y), bf16x2_maxabs(w.z, w.w)));
+    } else {
+        return local_amax<8>(x);
+    }
+}
+
 template <typename T, int PAT, int SCORE, int FMT>
-__device__ __forceinline__ void process_chunk(const PassParams &p, const float (&x)[8], const ChunkOut &o,
-                                              const PassConsts &c, Acc &acc, float row_amax = -1.0f,
-                                              const RowScale *rs = nullptr)
+__device__ __forceinline__ void process_chunk(const PassParams &p, const typename Elem<T>::Raw &raw,
+                                              const ChunkOut &o, const PassConsts &c, Acc &acc,
+                                              float row_amax = -1.0f, const RowScale *rs = nullptr)
 {
     constexpr int VPC = PAT == kDense ? 8 : 4;
+    // two groups of bf16 values selected by magnitude with packed lanes
+    constexpr bool kPair = sizeof(T) == 2 && PAT == kSparse24 && SCORE == kMag;
+    float x[8]; // (unused values are not computed)
+    Elem<T>::unpack(raw, x);
     float v[VPC];
+    float vmax;   // max |v| over the chunk's values to quantize
     uint32_t meta = 0;
+    uint32_t kept_bits[2] = {0u, 0u}; // kPair: kept values as bf16x2 (group 0, group 1)
     float et, ep = 0.0f;
 
     if constexpr (PAT == kDense) {
 #pragma unroll
         for (int i = 0; i < 8; ++i)
             v[i] = x[i];
+        vmax = chunk_amax<T>(raw, x);
         f32x2 t[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
             t[i] = mul2(pack2(x[2 * i], x[2 * i + 1]), pack2(x[2 * i], x[2 * i + 1]));
         t[0] = add2(add2(t[0], t[1]), add2(t[2], t[3]));
         et = lo2(t[0]) + hi2(t[0]);
+    } else if constexpr (kPair) {
+        const uint4 w = raw.v;
+        const Pair24 g = pair24_bf16(w.x, w.y, w.z, w.w);
+        v[0] = bf16_lo(g.k0);
+        v[1] = bf16_lo(g.k1);
+        v[2] = bf16_hi(g.k0);
+        v[3] = bf16_hi(g.k1);
+        vmax = bf16x2_hmax(bf16x2_maxabs(g.k0, g.k1));
+        kept_bits[0] = __byte_perm(g.k0, g.k1, 0x5410);
+        kept_bits[1] = __byte_perm(g.k0, g.k1, 0x7632);
+        meta = g.meta;
+        et = g.e_all;
+        ep = g.e_drop;
     } else if constexpr (PAT == kSparse24) {
         Group24 g0, g1;
         if constexpr (SCORE == kWanda) {
@@ -513,6 +547,7 @@ __device__ __forceinline__ void process_chunk(const PassParams &p, const float (
         v[1] = g0.k1;
         v[2] = g1.k0;
         v[3] = g1.k1;
+        vmax = local_amax<4>(v);
         meta = g0.nib | (g1.nib << 4);
         et = g0.e_all + g1.e_all;
         ep = g0.e_drop + g1.e_drop;
@@ -554,12 +589,14 @@ __device__ __forceinline__ void process_chunk(const PassParams &p, const float (
         meta = f.nib;
         et = (e[0] + e[1]) + (e[2] + e[3]);
         ep = en.d0 + en.d1;
+        vmax = local_amax<4>(v);
     }
 
+
     if constexpr (FMT == kAmax) {
-        acc.amax_all = fmaxf(acc.amax_all, local_amax<8>(x));
+        acc.amax_all = fmaxf(acc.amax_all, chunk_amax<T>(raw, x));
         if constexpr (PAT != kDense)
-            acc.amax_kept = fmaxf(acc.amax_kept, local_amax<4>(v));
+            acc.amax_kept = fmaxf(acc.amax_kept, vmax);
         return;
     }
     acc.et += et;
@@ -578,7 +615,9 @@ __device__ __forceinline__ void process_chunk(const PassParams &p, const float (
     float eq = 0.0f;
     if constexpr (FMT == kNone) {
         if (o.valid) {
-            if constexpr (sizeof(T) == 2) {
+            if constexpr (kPair) {
+                *reinterpret_cast<uint2 *>(o.val) = make_uint2(kept_bits[0], kept_bits[1]);
+            } else if constexpr (sizeof(T) == 2) {
                 const uint32_t w0 = (__float_as_uint(v[0]) >> 16) | (__float_as_uint(v[1]) & 0xffff0000u);
                 const uint32_t w1 = (__float_as_uint(v[2]) >> 16) | (__float_as_uint(v[3]) & 0xffff0000u);
                 *reinterpret_cast<uint2 *>(o.val) = make_uint2(w0, w1);
@@ -587,16 +626,16 @@ __device__ __forceinline__ void process_chunk(const PassParams &p, const float (
             }
         }
     } else if constexpr (FMT == kFp8) {
-        eq = quant_fp8<VPC, true>(v, c.rst, c.guard, o);
+        eq = quant_fp8<VPC, true>(v, vmax, c.rst, c.guard, o);
     } else if constexpr (FMT == kInt) {
-        eq = quant_int<VPC, true>(v, p.q, o, row_amax, rs);
+        eq = quant_int<VPC, true>(v, vmax, p.q, o, row_amax, rs);
     } else if constexpr (FMT == kNvfp4) {
-        eq = quant_nvfp4<VPC, true>(v, c.rst, o, c.tb);
+        eq = quant_nvfp4<VPC, true>(v, vmax, c.rst, o, c.tb);
     } else if constexpr (FMT == kMxfp4) {
-        eq = quant_mxfp4<VPC, true>(v, o);
+        eq = quant_mxfp4<VPC, true>(v, vmax, o);
     } else if constexpr (FMT == kEnergy) {
-        eq = quant_energy_only<VPC>(v, p.q, c.rst, c.guard, c.tb);
-        acc.eqd += quant_energy_only<8>(x, p.qd, c.rstd, c.guardd, c.tbd);
+        eq = quant_energy_only<VPC>(v, vmax, p.q, c.rst, c.guard, c.tb);
+        acc.eqd += quant_energy_only<8>(x, chunk_amax<T>(raw, x), p.qd, c.rstd, c.guardd, c.tbd);
     }
     if constexpr (PAT == kDense)
         acc.eqd += eq;
@@ -906,8 +945,13 @@ template <> struct Stream<float> {
 };
 
 // Resident CTAs per SM the stream kernel is compiled for (register budget).
+// (Four CTAs where the kernel fits 64 registers without spilling, else three;
+// two for the energy pass.)
 template <typename T, int PAT, int SCORE, int FMT> struct StreamOcc {
-    static constexpr int value = (FMT == kAmax || FMT == kNone) ? 4 : 3;
+    static constexpr bool light = FMT == kAmax || (sizeof(T) == 2 && SCORE == kMag && PAT != kSparse48 &&
+                                                   FMT != kEnergy && FMT != kNvfp4 &&
+                                                   !(PAT != kDense && FMT == kFp8));
+    static constexpr int value = FMT == kEnergy ? 2 : light ? 4 : 3; // the energy pass: two formats live
 };
 
 // Byte advance of each output between consecutive slots of a full-width unit
@@ -947,9 +991,7 @@ __device__ __forceinline__ void stream_unit(const PassParams &p, const PassConst
         if constexpr (SCORE == kWanda)
             oi.norms = o.norms + i * step_c;
         oi.valid = ok[i];
-        float xv[8];
-        E::unpack(raw[i], xv);
-        process_chunk<T, PAT, SCORE, FMT>(p, xv, oi, c, acc);
+        process_chunk<T, PAT, SCORE, FMT>(p, raw[i], oi, c, acc);
     }
 }
 
@@ -1051,30 +1093,25 @@ __global__ void __launch_bounds__(kStreamThreads, (StreamOcc<T, PAT, SCORE, FMT>
 // resident to cover the load latency.
 // ---------------------------------------------------------------------------
 
+// Chunk c of a row through the read-only cache path (the row is read again in
+// the second sweep, from L1 or L2); zeros when !ok.
 template <typename T> struct RowChunk;
 template <> struct RowChunk<__nv_bfloat16> {
-    uint4 v;
-    __device__ __forceinline__ void load(const void *row, int c)
+    __device__ __forceinline__ static Elem<__nv_bfloat16>::Raw load(const void *row, int c, bool ok)
     {
-        v = __ldg(reinterpret_cast<const uint4 *>(row) + c);
-    }
-    __device__ __forceinline__ void unpack(float (&x)[8]) const
-    {
-        Elem<__nv_bfloat16>::Raw r{v};
-        Elem<__nv_bfloat16>::unpack(r, x);
+        Elem<__nv_bfloat16>::Raw r;
+        r.v = ok ? __ldg(reinterpret_cast<const uint4 *>(row) + c) : make_uint4(0u, 0u, 0u, 0u);
+        return r;
     }
 };
 template <> struct RowChunk<float> {
-    float4 a, b;
-    __device__ __forceinline__ void load(const void *row, int c)
+    __device__ __forceinline__ static Elem<float>::Raw load(const void *row, int c, bool ok)
     {
-        a = __ldg(reinterpret_cast<const float4 *>(row) + 2 * c);
-        b = __ldg(reinterpret_cast<const float4 *>(row) + 2 * c + 1);
-    }
-    __device__ __forceinline__ void unpack(float (&x)[8]) const
-    {
-        Elem<float>::Raw r{a, b};
-        Elem<float>::unpack(r, x);
+        Elem<float>::Raw r;
+        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+        r.a = ok ? __ldg(reinterpret_cast<const float4 *>(row) + 2 * c) : z;
+        r.b = ok ? __ldg(reinterpret_cast<const float4 *>(row) + 2 * c + 1) : z;
+        return r;
     }
 };
 
@@ -1099,23 +1136,23 @@ __global__ void __launch_bounds__(kRowThreads) rowsweep_kernel(const T *__restri
         // score the kept amax equals the amax of all values)
         float amax = 0.0f;
         for (int c0 = 0; c0 < nchunks; c0 += 256) {
-            RowChunk<T> buf[8];
+            typename Elem<T>::Raw buf[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u)
-                if (c0 + 32 * u + lane < nchunks)
-                    buf[u].load(xr, c0 + 32 * u + lane);
+                buf[u] = RowChunk<T>::load(xr, c0 + 32 * u + lane, c0 + 32 * u + lane < nchunks);
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int c = c0 + 32 * u + lane;
                 if (c < nchunks) {
-                    float xv[8];
-                    buf[u].unpack(xv);
                     if constexpr (PAT == kDense || SCORE == kMag) {
-                        amax = fmaxf(amax, local_amax<8>(xv));
+                        float xv[8];
+                        Elem<T>::unpack(buf[u], xv);
+                        amax = fmaxf(amax, chunk_amax<T>(buf[u], xv));
                     } else {
                         Acc a{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
                         process_chunk<T, PAT, SCORE, kAmax>(
-                            p, xv, make_out<T, PAT, kAmax>(p, row, static_cast<int64_t>(c) * 8, true, lane), nc, a);
+                            p, buf[u], make_out<T, PAT, kAmax>(p, row, static_cast<int64_t>(c) * 8, true, lane), nc,
+                            a);
                         amax = fmaxf(amax, a.amax_kept);
                     }
                 }
@@ -1131,25 +1168,118 @@ __global__ void __launch_bounds__(kRowThreads) rowsweep_kernel(const T *__restri
         // step (4:8 metadata pairs lanes through a shuffle)
         Acc acc{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         for (int c0 = 0; c0 < nchunks; c0 += 64) {
-            RowChunk<T> buf[2];
+            typename Elem<T>::Raw buf[2];
 #pragma unroll
             for (int u = 0; u < 2; ++u)
-                if (c0 + 32 * u + lane < nchunks)
-                    buf[u].load(xr, c0 + 32 * u + lane);
+                buf[u] = RowChunk<T>::load(xr, c0 + 32 * u + lane, c0 + 32 * u + lane < nchunks);
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
                 const int c = c0 + 32 * u + lane;
-                if (c0 + 32 * u < nchunks) {
-                    float xv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                    if (c < nchunks)
-                        buf[u].unpack(xv);
+                if (c0 + 32 * u < nchunks)
                     process_chunk<T, PAT, SCORE, kInt>(
-                        p, xv, make_out<T, PAT, kInt>(p, row, static_cast<int64_t>(c) * 8, c < nchunks, lane), nc,
+                        p, buf[u], make_out<T, PAT, kInt>(p, row, static_cast<int64_t>(c) * 8, c < nchunks, lane), nc,
                         acc, amax, &rs);
-                }
             }
         }
         if (lane == 0)
+            static_cast<float *>(p.scales)[row] = rs.scale;
+        e_total += acc.et;
+        e_prune += acc.ep;
+        e_q += acc.eq;
+        e_qd += acc.eqd;
+    }
+    if (!p.energy_out)
+        return;
+    grid_reduce_energy(p, e_total, e_prune, e_q, e_qd, red, &flag, tid, lane, warp);
+}
+
+// ---------------------------------------------------------------------------
+// one scale per row with the row held in registers (k <= 8 * 256 * CPT):
+// tpr threads (a power of two, 32..256) share a row, each holding CPT chunks
+// (chunk c = t + j * tpr of the row, so a warp's loads are contiguous); a CTA
+// of 256 threads takes 256 / tpr rows per step. The row amax is reduced with
+// shuffles and, across the row's warps, through shared memory (one CTA
+// barrier per step, the buffer alternating between steps); the codes are then
+// computed from the registers, so the operand is read once.
+// ---------------------------------------------------------------------------
+
+// Resident CTAs per SM the row-block kernel is compiled for (register budget:
+// the row's CPT chunks per thread stay in registers).
+template <typename T, int PAT, int SCORE, int CPT> struct RowblockOcc {
+    static constexpr bool light = sizeof(T) == 2 && (PAT == kDense || (PAT == kSparse24 && SCORE == kMag));
+    static constexpr int value = CPT == 1 ? 4 : CPT == 4 ? (light ? 4 : 3) : 2;
+};
+
+template <typename T, int PAT, int SCORE, int CPT>
+__global__ void __launch_bounds__(kRowThreads, (RowblockOcc<T, PAT, SCORE, CPT>::value))
+    rowblock_kernel(const T *__restrict__ x, int64_t ld, int32_t log2_tpr, const PassParams pk)
+{
+    const PassParams p = operand_view(pk);
+    __shared__ double red[kConsumerWarps * 4];
+    __shared__ float wmax[2][kConsumerWarps];
+    __shared__ uint32_t flag;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    grid_dependency_wait();
+    grid_dependents_launch();
+    const int tpr = 1 << log2_tpr, rpc = kRowThreads >> log2_tpr;
+    const int t = tid & (tpr - 1), rin = tid >> log2_tpr;
+    const int wpr = tpr >> 5 > 0 ? tpr >> 5 : 1; // warps per row
+    const int w0 = (rin * tpr) >> 5;               // first warp of this thread's row
+    const int nchunks = static_cast<int>(p.k / 8);
+    const PassConsts nc{make_recip(0.0f), make_recip(0.0f), NvTable{nullptr, nullptr}, NvTable{nullptr, nullptr},
+                        false, false};
+    const T *xo = x + p.op * p.x_bstride;
+    double e_total = 0.0, e_prune = 0.0, e_q = 0.0, e_qd = 0.0;
+    int buf = 0;
+    for (int64_t base = static_cast<int64_t>(p.cta) * rpc; base < p.rows;
+         base += static_cast<int64_t>(p.ctas_per_op) * rpc, buf ^= 1) {
+        const int64_t row = base + rin;
+        const bool rv = row < p.rows;
+        const T *xr = xo + row * ld;
+        typename Elem<T>::Raw raw[CPT];
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) {
+            const int c = t + j * tpr;
+            raw[j] = Stream<T>::load(xr + 8 * c, rv && c < nchunks);
+        }
+        // the row amax of the values to quantize (for the magnitude score the
+        // kept amax equals the amax of all values)
+        float m = 0.0f;
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) {
+            if constexpr (PAT == kDense || SCORE == kMag) {
+                float xv[8];
+                Elem<T>::unpack(raw[j], xv);
+                m = fmaxf(m, chunk_amax<T>(raw[j], xv));
+            } else {
+                const int c = t + j * tpr;
+                Acc a{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                process_chunk<T, PAT, SCORE, kAmax>(
+                    p, raw[j], make_out<T, PAT, kAmax>(p, row, static_cast<int64_t>(c) * 8, rv && c < nchunks, lane),
+                    nc, a);
+                m = fmaxf(m, a.amax_kept);
+            }
+        }
+        m = group_amax(m, tpr < 32 ? tpr : 32);
+        if (lane == 0)
+            wmax[buf][warp] = m;
+        __syncthreads();
+        for (int w = 0; w < wpr; ++w)
+            m = fmaxf(m, wmax[buf][w0 + w]);
+        RowScale rs;
+        rs.given = true;
+        rs.amax = m;
+        rs.scale = int_scale(m, p.q);
+        rs.rc = make_recip(rs.scale);
+        Acc acc{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) {
+            const int c = t + j * tpr;
+            process_chunk<T, PAT, SCORE, kInt>(
+                p, raw[j], make_out<T, PAT, kInt>(p, row, static_cast<int64_t>(c) * 8, rv && c < nchunks, lane), nc,
+                acc, m, &rs);
+        }
+        if (rv && t == 0)
             static_cast<float *>(p.scales)[row] = rs.scale;
         e_total += acc.et;
         e_prune += acc.ep;
@@ -1323,11 +1453,9 @@ __global__ void __launch_bounds__(kThreads, 1) axis0_kernel(const __grid_constan
         for (int i = 0; i < 4; ++i) {
             if (i < p.cpt) {
                 const int j = tid + i * kConsumers;
-                float x[8];
-                Elem<T>::unpack(raw[i], x);
                 const int64_t row = row0 + (j >> 4), col = col0 + ((j & 15) << 3);
                 process_chunk<T, PAT, SCORE, FMT>(
-                    p, x, make_out<T, PAT, FMT>(p, row, col, row < p.rows && col < p.k, lane), c, acc);
+                    p, raw[i], make_out<T, PAT, FMT>(p, row, col, row < p.rows && col < p.k, lane), c, acc);
             }
         }
         if constexpr (FMT != kAmax) {

@@ -180,7 +180,9 @@ def test_other_entry_points_validate():
     assert L.ss24_amax(ctypes.byref(o), ss24.SPARSE_24, ss24.MAG, None, None, ALIGNED, wsb, None) == 1
     assert L.ss24_predicted_ratio(None, ALIGNED, ALIGNED, 1, None) == 1
     assert L.ss24_predicted_ratio(ALIGNED, ALIGNED, ALIGNED, -1, None) == 2
-    assert L.ss24_selfcheck_division(2, 0, 1, ALIGNED, None) == 8
+    assert L.ss24_selfcheck_division(3, 0, 1, ALIGNED, None) == 8
+    assert L.ss24_selfcheck_division(2, 1 << 15, 1, ALIGNED, None) == 2
+    assert L.ss24_selfcheck_division(2, 100, (1 << 15) - 99, ALIGNED, None) == 2
     assert L.ss24_selfcheck_division(0, 1 << 23, 1, ALIGNED, None) == 2
     assert L.ss24_selfcheck_division(0, 0, 1, None, None) == 1
     assert L.ss24_encode_e4m3(None, None, 5, None) == 1

@@ -310,8 +310,22 @@ def test_batch_amax_scale_energy_and_empty(ss, ws):
     assert ws.error() == 0
 
 
+@pytest.mark.parametrize("k", [14336, 16400])
+def test_int_one_scale_per_very_long_row(ss, ws, k):
+    """k = 14336: eight chunks per thread of a 256-thread row block; k = 16400
+    (over 2048 chunks): the two-sweep warp-per-row kernel."""
+    for pattern in (0, 24, 48):
+        xh, _ = synth.linear_input(7, k, seed=8)
+        compare(ss, ws, xh, pattern=pattern, fmt="int", bits=8, group=0)
+        xf = synth.gaussian_f32(5, k, seed=9)
+        compare(ss, ws, xf, pattern=pattern, fmt="int", bits=5, group=0)
+    xh, _ = synth.linear_input(6, k, seed=10)
+    norms = synth.linear_weight(1, k, seed=11)[1]
+    compare(ss, ws, xh, pattern=24, fmt="int", bits=4, group=0, pack4=True, score="wanda", norms=norms)
+
+
 def test_int_one_scale_per_long_row(ss, ws):
-    """Rows too long for the register-resident kernel use the shared-memory row kernel."""
+    """Rows of several hundred chunks: the row-block kernel with 256 threads per row."""
     for pattern in (0, 24, 48):
         xh, _ = synth.linear_input(21, 4352, seed=5)
         compare(ss, ws, xh, pattern=pattern, fmt="int", bits=8, group=0)
@@ -327,6 +341,13 @@ def test_division_matches_ieee_for_every_significand_pair(ss):
     assert bad == 0, f"first mismatch a, b bits = {first}"
     bad, first = ss.selfcheck_division(mode=1, b_count=1 << 12, chunk=1 << 12)
     assert bad == 0, f"first mismatch a, b bits = {first}"
+
+
+def test_packed_bf16_operations_for_every_pair_of_magnitudes(ss):
+    """The packed comparison, maximum, conversion and squares behind the bf16
+    2:4 selection and amax, for every pair of finite bf16 magnitudes."""
+    bad, first = ss.selfcheck_division(mode=2, b_first=0, b_count=1 << 15, chunk=1 << 15)
+    assert bad == 0, f"first mismatch (a, b) = {first}"
 
 
 @pytest.mark.parametrize("k", [8, 16, 24, 40, 96, 136, 264])
