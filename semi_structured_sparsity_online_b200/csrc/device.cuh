@@ -150,13 +150,25 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi)
 }
 
 // Two E4M3 bytes (bits 0..7 and 8..15) -> two binary32 (exact).
+// Two fp16 lanes -> two binary32 (exact), on the multiply-add pipe: a
+// mixed-precision add of -0, which leaves every value unchanged.
+__device__ __forceinline__ float2 f16x2_to_f32(uint32_t h2)
+{
+    float lo, hi;
+    asm("{ .reg .b16 l, h; mov.b32 {l, h}, %2;\n"
+        " add.rn.f32.f16 %0, l, 0f80000000;\n"
+        " add.rn.f32.f16 %1, h, 0f80000000; }"
+        : "=f"(lo), "=f"(hi)
+        : "r"(h2));
+    return make_float2(lo, hi);
+}
+
 __device__ __forceinline__ float2 e4m3x2_to_f32(uint32_t two_bytes)
 {
     uint32_t h2;
     const uint16_t b = static_cast<uint16_t>(two_bytes);
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(b));
-    __half2 h = *reinterpret_cast<__half2 *>(&h2);
-    return __half22float2(h); // .x from the low byte
+    return f16x2_to_f32(h2); // .x from the low byte
 }
 
 __device__ __forceinline__ float e4m3_to_f32(uint32_t byte)
@@ -190,8 +202,7 @@ __device__ __forceinline__ float2 e2m1x2_to_f32(uint32_t byte)
         "}\n"
         : "=r"(h2)
         : "r"(byte));
-    __half2 h = *reinterpret_cast<__half2 *>(&h2);
-    return __half22float2(h); // .x from the low nibble
+    return f16x2_to_f32(h2); // .x from the low nibble
 }
 
 // MXFP4 shared exponent of a block with amax > 0: floor(log2(amax)) - 2,

@@ -852,14 +852,29 @@ __device__ __forceinline__ void producer(const CUtensorMap *map, const PassParam
 
 // Output pointers of the chunk at (row, col) (col: first input column of the
 // chunk); nothing is dereferenced unless `valid`.
+// Output base pointers of one operand of a batch.
+struct OutBase {
+    uint8_t *values, *scales, *meta;
+};
+
+__device__ __forceinline__ OutBase out_base(const PassParams &pk, int op)
+{
+    OutBase b;
+    b.values = static_cast<uint8_t *>(pk.values) + op * pk.values_bstride;
+    b.scales = static_cast<uint8_t *>(pk.scales) + op * pk.scales_bstride;
+    b.meta = pk.meta + op * pk.meta_bstride;
+    return b;
+}
+
 template <typename T, int PAT, int FMT>
-__device__ __forceinline__ ChunkOut make_out(const PassParams &p, int64_t row, int64_t col, bool valid, int lane)
+__device__ __forceinline__ ChunkOut make_out(const PassParams &p, const OutBase &ob, int64_t row, int64_t col,
+                                             bool valid, int lane)
 {
     const int64_t n = PAT == kDense ? p.k : p.k / 2;
     const int64_t colq = PAT == kDense ? col : col / 2;
     const int64_t off = row * n + colq; // index of the chunk's first quantized value
-    uint8_t *vals = static_cast<uint8_t *>(p.values);
-    uint8_t *sc = static_cast<uint8_t *>(p.scales);
+    uint8_t *vals = ob.values;
+    uint8_t *sc = ob.scales;
     ChunkOut o{nullptr, nullptr, nullptr, nullptr, valid, lane};
     if constexpr (FMT == kNone) {
         o.val = vals + off * static_cast<int64_t>(sizeof(T));
@@ -877,12 +892,20 @@ __device__ __forceinline__ ChunkOut make_out(const PassParams &p, int64_t row, i
         o.scale = sc + row * (n / 32) + colq / 32;
     }
     if constexpr (PAT == kSparse24 && FMT != kAmax && FMT != kEnergy)
-        o.meta = p.meta + row * (p.k / 8) + col / 8;
+        o.meta = ob.meta + row * (p.k / 8) + col / 8;
     else if constexpr (PAT == kSparse48 && FMT != kAmax && FMT != kEnergy)
-        o.meta = p.meta + row * (p.k / 16) + col / 16;
+        o.meta = ob.meta + row * (p.k / 16) + col / 16;
     if (p.norms)
         o.norms = p.norms + col;
     return o;
+}
+
+// make_out for kernels whose parameters are already an operand's view.
+template <typename T, int PAT, int FMT>
+__device__ __forceinline__ ChunkOut make_out(const PassParams &p, int64_t row, int64_t col, bool valid, int lane)
+{
+    const OutBase ob{static_cast<uint8_t *>(p.values), static_cast<uint8_t *>(p.scales), p.meta};
+    return make_out<T, PAT, FMT>(p, ob, row, col, valid, lane);
 }
 
 // Tensor scales, reciprocals and NVFP4 tables of a pass (every thread of the
@@ -947,10 +970,10 @@ template <> struct Stream<float> {
 // Resident CTAs per SM the stream kernel is compiled for (register budget).
 // (Four CTAs where the kernel fits 64 registers without spilling, else three;
 // two for the energy pass.)
-template <typename T, int PAT, int SCORE, int FMT> struct StreamOcc {
+template <typename T, int PAT, int SCORE, int FMT, bool FW> struct StreamOcc {
     static constexpr bool light = FMT == kAmax || (sizeof(T) == 2 && SCORE == kMag && PAT != kSparse48 &&
                                                    FMT != kEnergy && FMT != kNvfp4 &&
-                                                   !(PAT != kDense && FMT == kFp8));
+                                                   (FW || !(PAT != kDense && FMT == kFp8)));
     static constexpr int value = FMT == kEnergy ? 2 : light ? 4 : 3; // the energy pass: two formats live
 };
 
@@ -1007,10 +1030,15 @@ __device__ __forceinline__ void stream_unit(const PassParams &p, const PassConst
 // per unit, where the slot offsets are compile-time constants and a unit
 // wholly inside the operand skips the per-chunk checks.
 template <typename T, int PAT, int SCORE, int FMT, bool FW>
-__global__ void __launch_bounds__(kStreamThreads, (StreamOcc<T, PAT, SCORE, FMT>::value))
-    stream_kernel(const PassParams pk)
+__global__ void __launch_bounds__(kStreamThreads, (StreamOcc<T, PAT, SCORE, FMT, FW>::value))
+    stream_kernel(const __grid_constant__ PassParams pk)
 {
-    const PassParams p = operand_view(pk);
+    // the loop reads the (operand-independent) parameters in place and keeps
+    // only this operand's output bases; the operand's full view is built for
+    // the constants and again for the final reductions
+    const PassParams &p = pk;
+    const int op = static_cast<int>(blockIdx.x) / pk.ctas_per_op;
+    const int cta = static_cast<int>(blockIdx.x) - op * pk.ctas_per_op;
     __shared__ double red[kStreamWarps * 4];
     __shared__ float fred[kStreamWarps * 2];
     __shared__ uint32_t flag;
@@ -1018,9 +1046,10 @@ __global__ void __launch_bounds__(kStreamThreads, (StreamOcc<T, PAT, SCORE, FMT>
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     grid_dependency_wait();
     grid_dependents_launch();
-    const PassConsts c = make_consts<FMT>(p, tid, kStreamThreads, nvt);
+    const PassConsts c = make_consts<FMT>(operand_view(pk), tid, kStreamThreads, nvt);
+    const OutBase ob = out_base(pk, op);
 
-    const T *x = static_cast<const T *>(p.x) + p.op * p.x_bstride;
+    const T *x = static_cast<const T *>(p.x) + op * p.x_bstride;
     const int log2_cpr = FW ? 5 : p.log2_cpr;
     const int lrow = lane >> log2_cpr;
     const int lcol = (lane & ((1 << log2_cpr) - 1)) << 3;
@@ -1028,8 +1057,8 @@ __global__ void __launch_bounds__(kStreamThreads, (StreamOcc<T, PAT, SCORE, FMT>
     const int64_t step_c = FW ? 256 : p.step_cols;
     // pointer advance per slot of a unit (the output offsets are linear in
     // row and column, and a step never splits a scale group)
-    const ChunkOut z0 = make_out<T, PAT, FMT>(p, 0, 0, false, lane);
-    const ChunkOut z1 = make_out<T, PAT, FMT>(p, FW ? 0 : p.step_rows, FW ? 256 : p.step_cols, false, lane);
+    const ChunkOut z0 = make_out<T, PAT, FMT>(p, ob, 0, 0, false, lane);
+    const ChunkOut z1 = make_out<T, PAT, FMT>(p, ob, FW ? 0 : p.step_rows, FW ? 256 : p.step_cols, false, lane);
     using FS = FwStep<T, PAT, FMT>;
     const int64_t dval = (FW && FS::val >= 0) ? FS::val : z1.val - z0.val;
     const int64_t dscale = (FW && FS::scale >= 0) ? FS::scale : z1.scale - z0.scale;
@@ -1038,7 +1067,7 @@ __global__ void __launch_bounds__(kStreamThreads, (StreamOcc<T, PAT, SCORE, FMT>
     const int unit_cols = FW ? 1024 : p.unit_cols;
 
     const int tw = p.ctas_per_op * kStreamWarps;
-    const int u0 = p.cta * kStreamWarps + warp;
+    const int u0 = cta * kStreamWarps + warp;
     int ua = u0 / p.units_b, ub = u0 - ua * p.units_b;
     const int sa = tw / p.units_b, sb = tw - sa * p.units_b;
     double e_total = 0.0, e_prune = 0.0, e_q = 0.0, e_qd = 0.0;
@@ -1047,7 +1076,7 @@ __global__ void __launch_bounds__(kStreamThreads, (StreamOcc<T, PAT, SCORE, FMT>
         const int64_t row0 = static_cast<int64_t>(ua) * unit_rows + lrow;
         const int64_t col0 = static_cast<int64_t>(ub) * unit_cols + lcol;
         const T *xp = x + row0 * p.ld + col0;
-        const ChunkOut o = make_out<T, PAT, FMT>(p, row0, col0, true, lane);
+        const ChunkOut o = make_out<T, PAT, FMT>(p, ob, row0, col0, true, lane);
         acc.et = acc.ep = acc.eq = acc.eqd = 0.0f;
         // full-width units lie inside the operand except in the last quad
         // of a row (rows are whole: one row per unit)
@@ -1074,12 +1103,13 @@ __global__ void __launch_bounds__(kStreamThreads, (StreamOcc<T, PAT, SCORE, FMT>
         }
     }
 
+    const PassParams v = operand_view(pk);
     if constexpr (FMT == kAmax) {
-        grid_reduce_amax<PAT>(p, acc.amax_kept, acc.amax_all, fred, &flag, tid, lane, warp);
+        grid_reduce_amax<PAT>(v, acc.amax_kept, acc.amax_all, fred, &flag, tid, lane, warp);
     } else {
-        if (!p.energy_out)
+        if (!v.energy_out)
             return;
-        grid_reduce_energy(p, e_total, e_prune, e_q, e_qd, red, &flag, tid, lane, warp);
+        grid_reduce_energy(v, e_total, e_prune, e_q, e_qd, red, &flag, tid, lane, warp);
     }
 }
 

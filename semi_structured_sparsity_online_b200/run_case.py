@@ -66,6 +66,8 @@ def main():
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--seed", type=int, default=8)
     ap.add_argument("--batch", type=int, default=0, help="0: one 2-D operand; B: one launch over B operands")
+    ap.add_argument("--derive-scale", action="store_true",
+                    help="FP8 / NVFP4: let the pass compute its tensor scale (an amax launch precedes it)")
     args = ap.parse_args()
     nb = max(args.batch, 1)
     xb = np.stack([synth.sweep_operand(args.m, args.k, seed=args.seed + i) for i in range(nb)])
@@ -94,7 +96,7 @@ def main():
                               ws=ws, energy=e)
         else:
             pattern, fmt, bits, group = PASSES[args.name]
-            ts = scale if fmt in ("fp8", "nvfp4") else None
+            ts = scale if fmt in ("fp8", "nvfp4") and not args.derive_scale else None
             ss24.run(x, pattern=pattern, fmt=fmt, bits=bits, group=group, tensor_scale=ts, energy=e, ws=ws, out=out)
 
     once()
