@@ -365,20 +365,23 @@ __device__ __forceinline__ float quant_nvfp4(const float (&v)[VPC], float vmax, 
     constexpr int kLanes = 16 / VPC;
     const float st = rst.b;
     const float amax = group_amax(vmax, kLanes);
-    uint32_t sb = 0;
-    if (st != 0.0f) {
-        // (amax / 6) / st: two correctly rounded divisions
-        Recip r6;
-        r6.b = 6.0f;
-        r6.nb = -6.0f;
-        r6.y = 0x1.555556p-3f; // RN(1/6)
-        r6.fast = true;
-        const float a6 = amax >= 0x1p-30f ? div_fast(amax, r6) : __fdiv_rn(amax, 6.0f);
-        const float bs = (rst.fast && a6 >= 0x1p-40f * st && __fmul_rn(a6, rst.y) < 0x1p126f)
-                             ? div_fast(a6, rst)
-                             : __fdiv_rn(a6, st);
-        sb = cvt_e4m3x2(bs, 0.0f) & 0xffu;
+    // the block scale E4M3((amax / 6) / st): two correctly rounded divisions,
+    // by Markstein's correction when both are in its exact range (zero amax
+    // included), else by IEEE division; one branch in the common case
+    Recip r6;
+    r6.b = 6.0f;
+    r6.nb = -6.0f;
+    r6.y = 0x1.555556p-3f; // RN(1/6)
+    r6.fast = true;
+    float a6 = div_fast(amax, r6);
+    float bs = div_fast(a6, rst);
+    const bool ok = (amax == 0.0f || amax >= 0x1p-30f) && rst.fast &&
+                    (a6 == 0.0f || (a6 >= 0x1p-40f * st && __fmul_rn(a6, rst.y) < 0x1p126f));
+    if (!ok) {
+        a6 = __fdiv_rn(amax, 6.0f);
+        bs = st != 0.0f ? __fdiv_rn(a6, st) : 0.0f;
     }
+    const uint32_t sb = cvt_e4m3x2(bs, 0.0f) & 0xffu;
     Recip rd;
     rd.b = tb.den[sb];
     rd.nb = -rd.b;
@@ -1242,9 +1245,11 @@ template <typename T, int PAT, int SCORE, int CPT> struct RowblockOcc {
 
 template <typename T, int PAT, int SCORE, int CPT>
 __global__ void __launch_bounds__(kRowThreads, (RowblockOcc<T, PAT, SCORE, CPT>::value))
-    rowblock_kernel(const T *__restrict__ x, int64_t ld, int32_t log2_tpr, const PassParams pk)
+    rowblock_kernel(const T *__restrict__ x, int64_t ld, int32_t log2_tpr, const __grid_constant__ PassParams pk)
 {
-    const PassParams p = operand_view(pk);
+    const PassParams &p = pk;
+    const int op = static_cast<int>(blockIdx.x) / pk.ctas_per_op;
+    const int cta = static_cast<int>(blockIdx.x) - op * pk.ctas_per_op;
     __shared__ double red[kConsumerWarps * 4];
     __shared__ float wmax[2][kConsumerWarps];
     __shared__ uint32_t flag;
@@ -1258,10 +1263,17 @@ __global__ void __launch_bounds__(kRowThreads, (RowblockOcc<T, PAT, SCORE, CPT>:
     const int nchunks = static_cast<int>(p.k / 8);
     const PassConsts nc{make_recip(0.0f), make_recip(0.0f), NvTable{nullptr, nullptr}, NvTable{nullptr, nullptr},
                         false, false};
-    const T *xo = x + p.op * p.x_bstride;
+    const OutBase ob = out_base(pk, op);
+    const T *xo = x + op * p.x_bstride;
+    // output offsets are linear in the column: the advance of each pointer
+    // per chunk step (tpr chunks)
+    const ChunkOut z = make_out<T, PAT, kInt>(p, ob, 0, 8 * t, true, lane);
+    const ChunkOut zc = make_out<T, PAT, kInt>(p, ob, 0, 8 * (t + tpr), true, lane);
+    const int64_t cval = zc.val - z.val, cmeta = zc.meta - z.meta;
+    float *scales = reinterpret_cast<float *>(ob.scales); // one per row
     double e_total = 0.0, e_prune = 0.0, e_q = 0.0, e_qd = 0.0;
     int buf = 0;
-    for (int64_t base = static_cast<int64_t>(p.cta) * rpc; base < p.rows;
+    for (int64_t base = static_cast<int64_t>(cta) * rpc; base < p.rows;
          base += static_cast<int64_t>(p.ctas_per_op) * rpc, buf ^= 1) {
         const int64_t row = base + rin;
         const bool rv = row < p.rows;
@@ -1272,6 +1284,7 @@ __global__ void __launch_bounds__(kRowThreads, (RowblockOcc<T, PAT, SCORE, CPT>:
             const int c = t + j * tpr;
             raw[j] = Stream<T>::load(xr + 8 * c, rv && c < nchunks);
         }
+        const ChunkOut o = make_out<T, PAT, kInt>(p, ob, row, 8 * t, rv, lane);
         // the row amax of the values to quantize (for the magnitude score the
         // kept amax equals the amax of all values)
         float m = 0.0f;
@@ -1282,15 +1295,15 @@ __global__ void __launch_bounds__(kRowThreads, (RowblockOcc<T, PAT, SCORE, CPT>:
                 Elem<T>::unpack(raw[j], xv);
                 m = fmaxf(m, chunk_amax<T>(raw[j], xv));
             } else {
-                const int c = t + j * tpr;
+                ChunkOut oj = o;
+                oj.norms = o.norms + 8 * j * tpr;
+                oj.valid = rv && t + j * tpr < nchunks;
                 Acc a{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                process_chunk<T, PAT, SCORE, kAmax>(
-                    p, raw[j], make_out<T, PAT, kAmax>(p, row, static_cast<int64_t>(c) * 8, rv && c < nchunks, lane),
-                    nc, a);
+                process_chunk<T, PAT, SCORE, kAmax>(p, raw[j], oj, nc, a);
                 m = fmaxf(m, a.amax_kept);
             }
         }
-        m = group_amax(m, tpr < 32 ? tpr : 32);
+        m = group_amax(m, 32);
         if (lane == 0)
             wmax[buf][warp] = m;
         __syncthreads();
@@ -1304,21 +1317,28 @@ __global__ void __launch_bounds__(kRowThreads, (RowblockOcc<T, PAT, SCORE, CPT>:
         Acc acc{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int j = 0; j < CPT; ++j) {
-            const int c = t + j * tpr;
-            process_chunk<T, PAT, SCORE, kInt>(
-                p, raw[j], make_out<T, PAT, kInt>(p, row, static_cast<int64_t>(c) * 8, rv && c < nchunks, lane), nc,
-                acc, m, &rs);
+            ChunkOut oj = o;
+            oj.val += j * cval;
+            oj.meta += j * cmeta;
+            if constexpr (SCORE == kWanda)
+                oj.norms = o.norms + 8 * j * tpr;
+            oj.valid = rv && t + j * tpr < nchunks;
+            process_chunk<T, PAT, SCORE, kInt>(p, raw[j], oj, nc, acc, m, &rs);
         }
         if (rv && t == 0)
-            static_cast<float *>(p.scales)[row] = rs.scale;
+            scales[row] = rs.scale;
         e_total += acc.et;
-        e_prune += acc.ep;
-        e_q += acc.eq;
-        e_qd += acc.eqd;
+        if constexpr (PAT != kDense) {
+            e_prune += acc.ep;
+            e_q += acc.eq;
+        } else {
+            e_qd += acc.eqd;
+        }
     }
-    if (!p.energy_out)
+    const PassParams v = operand_view(pk);
+    if (!v.energy_out)
         return;
-    grid_reduce_energy(p, e_total, e_prune, e_q, e_qd, red, &flag, tid, lane, warp);
+    grid_reduce_energy(v, e_total, e_prune, e_q, e_qd, red, &flag, tid, lane, warp);
 }
 
 // ---------------------------------------------------------------------------
