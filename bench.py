@@ -52,6 +52,31 @@ def algorithmic_bytes(m=M, k=K):
     }
 
 
+def kernel_source_sha():
+    """Hash of the CUDA sources (the ncu traffic figures are valid for one)."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    src = os.path.join(ROOT, "semi_structured_sparsity_online_b200", "csrc")
+    for f in sorted(glob.glob(os.path.join(src, "*.cu")) + glob.glob(os.path.join(src, "*.cuh"))):
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(pass_name):
+    """DRAM bytes per launch of a pass from the committed ncu capture, or None
+    when the kernels changed since it was taken."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if t.get("source_sha") != kernel_source_sha():
+        return None
+    return t.get(pass_name)
+
+
 def load_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -337,12 +362,7 @@ def run_cuda(args):
         passes[p] = {"us_per_step": round(us, 3),
                      "gbps": round(BATCH * ab[p] / (us * 1e-6) / 1e9, 1) if ab[p] else None,
                      "bytes_per_launch": BATCH * ab[p]}
-    traffic = None
-    try:
-        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
-            traffic = json.load(f).get(dom)
-    except Exception:
-        pass
+    traffic = measured_traffic(dom)
 
     r = step.r.cpu().numpy()
     result = {
