@@ -227,6 +227,7 @@ struct RowScale {
     bool given;
     float amax, scale;
     Recip rc;
+    bool fast; // quot_fast(rc, amax)
 };
 
 template <int VPC, bool STORE>
@@ -235,16 +236,18 @@ __device__ __forceinline__ float quant_int(const float (&v)[VPC], float vmax, co
 {
     float amax, scale;
     Recip rc;
+    bool fast;
     if (rs && rs->given) {
         amax = rs->amax;
         scale = rs->scale;
         rc = rs->rc;
+        fast = rs->fast;
     } else {
         amax = row_amax >= 0.0f ? row_amax : group_amax(vmax, q.lanes);
         scale = int_scale(amax, q);
         rc = make_recip(scale);
+        fast = quot_fast(rc, amax);
     }
-    const bool fast = quot_fast(rc, amax);
     float qn[VPC];
     neg_quotients<VPC>(v, rc, fast, qn);
     if (!fast) {
@@ -939,13 +942,18 @@ __device__ __forceinline__ PassConsts make_consts(const PassParams &p, int tid, 
     return c;
 }
 
-// 16-byte global load that bypasses L1 (each input byte is read once).
-__device__ __forceinline__ uint4 ld_stream(const void *p)
+// 16-byte global load that bypasses L1 (each input byte is read once),
+// predicated: zeros and no memory access when !ok (no branch).
+__device__ __forceinline__ uint4 ld_stream(const void *p, bool ok)
 {
-    uint4 r;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
+    uint4 r = make_uint4(0u, 0u, 0u, 0u);
+    asm volatile("{\n"
+                 " .reg .pred q;\n"
+                 " setp.ne.b32 q, %5, 0;\n"
+                 " @q ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];\n"
+                 "}\n"
+                 : "+r"(r.x), "+r"(r.y), "+r"(r.z), "+r"(r.w)
+                 : "l"(p), "r"(static_cast<int>(ok)));
     return r;
 }
 
@@ -954,7 +962,7 @@ template <> struct Stream<__nv_bfloat16> {
     __device__ __forceinline__ static Elem<__nv_bfloat16>::Raw load(const __nv_bfloat16 *p, bool ok)
     {
         Elem<__nv_bfloat16>::Raw r;
-        r.v = ok ? ld_stream(p) : make_uint4(0u, 0u, 0u, 0u);
+        r.v = ld_stream(p, ok);
         return r;
     }
 };
@@ -962,8 +970,8 @@ template <> struct Stream<float> {
     __device__ __forceinline__ static Elem<float>::Raw load(const float *p, bool ok)
     {
         Elem<float>::Raw r;
-        const uint4 a = ok ? ld_stream(p) : make_uint4(0u, 0u, 0u, 0u);
-        const uint4 b = ok ? ld_stream(p + 4) : make_uint4(0u, 0u, 0u, 0u);
+        const uint4 a = ld_stream(p, ok);
+        const uint4 b = ld_stream(p + 4, ok);
         r.a = make_float4(__uint_as_float(a.x), __uint_as_float(a.y), __uint_as_float(a.z), __uint_as_float(a.w));
         r.b = make_float4(__uint_as_float(b.x), __uint_as_float(b.y), __uint_as_float(b.z), __uint_as_float(b.w));
         return r;
@@ -1197,6 +1205,7 @@ __global__ void __launch_bounds__(kRowThreads) rowsweep_kernel(const T *__restri
         rs.amax = amax;
         rs.scale = int_scale(amax, p.q);
         rs.rc = make_recip(rs.scale);
+        rs.fast = quot_fast(rs.rc, amax);
         // sweep 2: codes, metadata and energies; every lane takes part in each
         // step (4:8 metadata pairs lanes through a shuffle)
         Acc acc{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -1235,6 +1244,80 @@ __global__ void __launch_bounds__(kRowThreads) rowsweep_kernel(const T *__restri
 // barrier per step, the buffer alternating between steps); the codes are then
 // computed from the registers, so the operand is read once.
 // ---------------------------------------------------------------------------
+
+// Dense INT-b codes of one chunk with its row's scale, straight-line on
+// binary32 pairs: the same operations, roundings and summation order as
+// quant_int / err_energy and the dense energy in process_chunk, with the code
+// width (STORE) and the fast-division decision (FAST, one per row) fixed.
+template <typename T, int STORE, bool FAST>
+__device__ __forceinline__ void dense_int_chunk(const typename Elem<T>::Raw &raw, const RowScale &rs, float qmax,
+                                                uint8_t *val, bool valid, Acc &acc)
+{
+    float x[8];
+    Elem<T>::unpack(raw, x);
+    f32x2 x2[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        x2[i] = pack2(x[2 * i], x[2 * i + 1]);
+    f32x2 t[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        t[i] = mul2(x2[i], x2[i]);
+    t[0] = add2(add2(t[0], t[1]), add2(t[2], t[3]));
+    acc.et += lo2(t[0]) + hi2(t[0]);
+    const f32x2 m2 = pack2(kMagic, kMagic), s2 = pack2(rs.scale, rs.scale);
+    f32x2 tt[4], e[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f32x2 qn;
+        if constexpr (FAST) {
+            qn = neg_div_fast2(x2[i], rs.rc);
+        } else {
+            float a = rs.rc.b != 0.0f ? __fdiv_rn(-x[2 * i], rs.rc.b) : -0.0f;
+            float b = rs.rc.b != 0.0f ? __fdiv_rn(-x[2 * i + 1], rs.rc.b) : -0.0f;
+            qn = pack2(fminf(fmaxf(a, -qmax), qmax), fminf(fmaxf(b, -qmax), qmax));
+        }
+        tt[i] = sub2(m2, qn);
+        const f32x2 d = mul2(sub2(tt[i], m2), s2);
+        const f32x2 df = sub2(x2[i], d);
+        e[i] = mul2(df, df);
+    }
+    e[0] = add2(add2(e[0], e[2]), add2(e[1], e[3]));
+    acc.eqd += lo2(e[0]) + hi2(e[0]);
+    if (valid) {
+        uint32_t b[8]; // low bits of M + q hold the two's-complement code
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            b[2 * i] = __float_as_uint(lo2(tt[i]));
+            b[2 * i + 1] = __float_as_uint(hi2(tt[i]));
+        }
+        if constexpr (STORE == kInt8) {
+            *reinterpret_cast<uint2 *>(val) =
+                make_uint2(__byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410),
+                           __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410));
+        } else if constexpr (STORE == kInt16) {
+            *reinterpret_cast<uint4 *>(val) = make_uint4(__byte_perm(b[0], b[1], 0x5410), __byte_perm(b[2], b[3], 0x5410),
+                                                         __byte_perm(b[4], b[5], 0x5410), __byte_perm(b[6], b[7], 0x5410));
+        } else {
+            uint32_t w = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                w |= (b[i] & 0xfu) << (4 * i);
+            *reinterpret_cast<uint32_t *>(val) = w;
+        }
+    }
+}
+
+// The CPT chunks of a thread in one row (dense operand), chunk j at val0 + j * cval.
+template <typename T, int CPT, int STORE, bool FAST>
+__device__ __forceinline__ void dense_int_row(const typename Elem<T>::Raw (&raw)[CPT], const RowScale &rs, float qmax,
+                                              uint8_t *val0, int64_t cval, int t, int tpr, int nchunks, bool rv,
+                                              Acc &acc)
+{
+#pragma unroll
+    for (int j = 0; j < CPT; ++j)
+        dense_int_chunk<T, STORE, FAST>(raw[j], rs, qmax, val0 + j * cval, rv && t + j * tpr < nchunks, acc);
+}
 
 // Resident CTAs per SM the row-block kernel is compiled for (register budget:
 // the row's CPT chunks per thread stay in registers).
@@ -1314,16 +1397,37 @@ __global__ void __launch_bounds__(kRowThreads, (RowblockOcc<T, PAT, SCORE, CPT>:
         rs.amax = m;
         rs.scale = int_scale(m, p.q);
         rs.rc = make_recip(rs.scale);
+        rs.fast = quot_fast(rs.rc, m);
         Acc acc{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if constexpr (PAT == kDense) {
+            const float qm = p.q.qmax;
+            const int st = p.q.store;
+            if (rs.fast) {
+                if (st == kInt8)
+                    dense_int_row<T, CPT, kInt8, true>(raw, rs, qm, o.val, cval, t, tpr, nchunks, rv, acc);
+                else if (st == kInt16)
+                    dense_int_row<T, CPT, kInt16, true>(raw, rs, qm, o.val, cval, t, tpr, nchunks, rv, acc);
+                else
+                    dense_int_row<T, CPT, kPack4, true>(raw, rs, qm, o.val, cval, t, tpr, nchunks, rv, acc);
+            } else {
+                if (st == kInt8)
+                    dense_int_row<T, CPT, kInt8, false>(raw, rs, qm, o.val, cval, t, tpr, nchunks, rv, acc);
+                else if (st == kInt16)
+                    dense_int_row<T, CPT, kInt16, false>(raw, rs, qm, o.val, cval, t, tpr, nchunks, rv, acc);
+                else
+                    dense_int_row<T, CPT, kPack4, false>(raw, rs, qm, o.val, cval, t, tpr, nchunks, rv, acc);
+            }
+        } else {
 #pragma unroll
-        for (int j = 0; j < CPT; ++j) {
-            ChunkOut oj = o;
-            oj.val += j * cval;
-            oj.meta += j * cmeta;
-            if constexpr (SCORE == kWanda)
-                oj.norms = o.norms + 8 * j * tpr;
-            oj.valid = rv && t + j * tpr < nchunks;
-            process_chunk<T, PAT, SCORE, kInt>(p, raw[j], oj, nc, acc, m, &rs);
+            for (int j = 0; j < CPT; ++j) {
+                ChunkOut oj = o;
+                oj.val += j * cval;
+                oj.meta += j * cmeta;
+                if constexpr (SCORE == kWanda)
+                    oj.norms = o.norms + 8 * j * tpr;
+                oj.valid = rv && t + j * tpr < nchunks;
+                process_chunk<T, PAT, SCORE, kInt>(p, raw[j], oj, nc, acc, m, &rs);
+            }
         }
         if (rv && t == 0)
             scales[row] = rs.scale;
