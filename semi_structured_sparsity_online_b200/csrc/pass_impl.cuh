@@ -1240,9 +1240,10 @@ __global__ void __launch_bounds__(kRowThreads) rowsweep_kernel(const T *__restri
 // tpr threads (a power of two, 32..256) share a row, each holding CPT chunks
 // (chunk c = t + j * tpr of the row, so a warp's loads are contiguous); a CTA
 // of 256 threads takes 256 / tpr rows per step. The row amax is reduced with
-// shuffles and, across the row's warps, through shared memory (one CTA
-// barrier per step, the buffer alternating between steps); the codes are then
-// computed from the registers, so the operand is read once.
+// shuffles and, across the row's warps, through shared memory (one named
+// barrier per row and step, over that row's warps only; the buffer alternates
+// between steps); the codes are then computed from the registers, so the
+// operand is read once.
 // ---------------------------------------------------------------------------
 
 // Dense INT-b codes of one chunk with its row's scale, straight-line on
@@ -1387,11 +1388,15 @@ __global__ void __launch_bounds__(kRowThreads, (RowblockOcc<T, PAT, SCORE, CPT>:
             }
         }
         m = group_amax(m, 32);
-        if (lane == 0)
-            wmax[buf][warp] = m;
-        __syncthreads();
-        for (int w = 0; w < wpr; ++w)
-            m = fmaxf(m, wmax[buf][w0 + w]);
+        if (wpr > 1) {
+            // the row's warps only: a named barrier per row, ids 2.. (id 1
+            // belongs to the CTA-wide reduction at the end)
+            if (lane == 0)
+                wmax[buf][warp] = m;
+            named_barrier_sync(2 + rin, tpr);
+            for (int w = 0; w < wpr; ++w)
+                m = fmaxf(m, wmax[buf][w0 + w]);
+        }
         RowScale rs;
         rs.given = true;
         rs.amax = m;
