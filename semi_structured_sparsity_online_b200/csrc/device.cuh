@@ -163,6 +163,21 @@ __device__ __forceinline__ float2 f16x2_to_f32(uint32_t h2)
     return make_float2(lo, hi);
 }
 
+// Two E4M3 codes in a 16-bit register -> two binary32 (exact).
+__device__ __forceinline__ float2 e4m3x2h_to_f32(uint16_t h)
+{
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(h));
+    return f16x2_to_f32(h2);
+}
+// Two binary32 -> two E4M3 codes (lo in the low byte), saturating, in a 16-bit register.
+__device__ __forceinline__ uint16_t cvt_e4m3x2h(float lo, float hi)
+{
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
 __device__ __forceinline__ float2 e4m3x2_to_f32(uint32_t two_bytes)
 {
     uint32_t h2;

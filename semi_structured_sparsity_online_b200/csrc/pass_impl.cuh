@@ -125,6 +125,24 @@ template <int VPC> __device__ __forceinline__ float err_energy(const float (&v)[
     return lo2(t[0]) + hi2(t[0]);
 }
 
+// The same with the dequantized values given negated (dn = -d): the terms
+// v + dn equal v - d, rounding included.
+template <int VPC> __device__ __forceinline__ float err_energy_neg(const float (&v)[VPC], const float (&dn)[VPC])
+{
+    f32x2 t[VPC / 2];
+#pragma unroll
+    for (int i = 0; i < VPC / 2; ++i) {
+        const f32x2 e = add2(pack2(v[2 * i], v[2 * i + 1]), pack2(dn[2 * i], dn[2 * i + 1]));
+        t[i] = mul2(e, e);
+    }
+#pragma unroll
+    for (int w = VPC / 4; w >= 1; w /= 2)
+#pragma unroll
+        for (int i = 0; i < w; ++i)
+            t[i] = add2(t[i], t[i + w]);
+    return lo2(t[0]) + hi2(t[0]);
+}
+
 // True when the fast division applies to every value of a chunk or group
 // whose largest magnitude is vmax: the scale is in [2^-60, 2^60] and no
 // quotient can overflow (vmax * y < 2^126).
@@ -176,27 +194,29 @@ __device__ __forceinline__ float quant_fp8(const float (&v)[VPC], float vmax, co
     bool fast = rc.fast;
     if (guard)
         fast = quot_fast(rc, vmax);
-    float qn[VPC], dec[VPC], d[VPC];
+    float qn[VPC], decn[VPC], dn[VPC];
     neg_quotients<VPC>(v, rc, fast, qn);
-    uint32_t c[VPC / 4];
+    // codes of -q, decoded as they come from the conversion: dn = -deq exactly
+    uint16_t h[VPC / 2];
 #pragma unroll
-    for (int t = 0; t < VPC / 4; ++t) {
-        c[t] = (cvt_e4m3x2(qn[4 * t], qn[4 * t + 1]) | (cvt_e4m3x2(qn[4 * t + 2], qn[4 * t + 3]) << 16)) ^
-               0x80808080u;
-        const float2 lo = e4m3x2_to_f32(c[t] & 0xffffu), hi = e4m3x2_to_f32(c[t] >> 16);
-        dec[4 * t + 0] = lo.x;
-        dec[4 * t + 1] = lo.y;
-        dec[4 * t + 2] = hi.x;
-        dec[4 * t + 3] = hi.y;
+    for (int t = 0; t < VPC / 2; ++t) {
+        h[t] = cvt_e4m3x2h(qn[2 * t], qn[2 * t + 1]);
+        const float2 f = e4m3x2h_to_f32(h[t]);
+        decn[2 * t] = f.x;
+        decn[2 * t + 1] = f.y;
     }
-    scale_values<VPC>(dec, rc.b, d);
+    scale_values<VPC>(decn, rc.b, dn);
+    uint32_t c[VPC / 4]; // the codes of q: the sign bits flipped back
+#pragma unroll
+    for (int t = 0; t < VPC / 4; ++t)
+        c[t] = (static_cast<uint32_t>(h[2 * t]) | (static_cast<uint32_t>(h[2 * t + 1]) << 16)) ^ 0x80808080u;
     if (STORE && o.valid) {
         if constexpr (VPC == 4)
             *reinterpret_cast<uint32_t *>(o.val) = c[0];
         else
             *reinterpret_cast<uint2 *>(o.val) = make_uint2(c[0], c[1]);
     }
-    return err_energy<VPC>(v, d);
+    return err_energy_neg<VPC>(v, dn);
 }
 
 // Integer rounding by the magic constant 1.5 * 2^23: for |q| < 2^22 the sum
