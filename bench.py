@@ -11,8 +11,12 @@ pass reads its operands from HBM (the batch is 256 MiB, twice the L2):
   3. dense FP8 E4M3 partner (same scale) + energy          ss24_quantize_fp8
   4. dense INT8, one scale per row, partner + energy       ss24_quantize_int
   5. predicted R against both partners (one launch each)   ss24_predicted_ratio
-The step is captured as one CUDA graph per pass; CUDA events between the pass
-graphs give per-kernel durations inside the timed region.
+The whole step is one CUDA graph, the passes chained by programmatic dependent
+launch. Every 8th step of the timed region instead replays a copy of that graph
+with an event-record node at every pass boundary, the nodes pointed at that
+step's own events: the per-kernel durations are CUDA events on the launching
+stream inside the timed region (an event node ends the overlap of the launches
+it separates, so those steps are a little slower, and are counted).
 
 Prints ONE JSON line (rank 0). ``--impl reference`` times the CPU oracle on a
 bounded sample of the same workload instead.
@@ -38,6 +42,7 @@ WORKLOAD = ("linear-input X bf16 4096x4096 (Student-t nu=4 /sqrt2, 8 outlier cha
             "per-row partners, energies, predicted R")
 M = K = 4096
 BATCH = 8
+EVENT_EVERY = 8   # steps per evented step in the timed region
 
 
 def algorithmic_bytes(m=M, k=K):
@@ -151,6 +156,59 @@ def make_batch(seed0=1):
     return xs
 
 
+class Cudart:
+    """The few runtime calls torch does not expose: event-record nodes in a
+    captured graph, repointed to fresh events before every replay."""
+    EVENT_RECORD_EXTERNAL = 0x1
+    NODE_TYPE_EVENT_RECORD = 7
+
+    def __init__(self):
+        import ctypes
+        self.c = ctypes
+        self.rt = ctypes.CDLL("libcudart.so.12")
+
+    def check(self, err, what):
+        if err != 0:
+            raise RuntimeError(f"{what} failed with CUDA error {err}")
+
+    def event_create(self):
+        ev = self.c.c_void_p()
+        self.check(self.rt.cudaEventCreate(self.c.byref(ev)), "cudaEventCreate")
+        return ev
+
+    def record_external(self, ev, stream):
+        self.check(self.rt.cudaEventRecordWithFlags(ev, self.c.c_void_p(stream), self.EVENT_RECORD_EXTERNAL),
+                   "cudaEventRecordWithFlags")
+
+    def elapsed_ms(self, a, b):
+        ms = self.c.c_float()
+        self.check(self.rt.cudaEventElapsedTime(self.c.byref(ms), a, b), "cudaEventElapsedTime")
+        return ms.value
+
+    def event_nodes(self, graph):
+        """{event handle value: node} for the event-record nodes of a graph."""
+        c = self.c
+        n = c.c_size_t(0)
+        g = c.c_void_p(graph)
+        self.check(self.rt.cudaGraphGetNodes(g, None, c.byref(n)), "cudaGraphGetNodes")
+        nodes = (c.c_void_p * n.value)()
+        self.check(self.rt.cudaGraphGetNodes(g, nodes, c.byref(n)), "cudaGraphGetNodes")
+        out = {}
+        for i in range(n.value):
+            t = c.c_int()
+            self.check(self.rt.cudaGraphNodeGetType(c.c_void_p(nodes[i]), c.byref(t)), "cudaGraphNodeGetType")
+            if t.value == self.NODE_TYPE_EVENT_RECORD:
+                ev = c.c_void_p()
+                self.check(self.rt.cudaGraphEventRecordNodeGetEvent(c.c_void_p(nodes[i]), c.byref(ev)),
+                           "cudaGraphEventRecordNodeGetEvent")
+                out[ev.value] = c.c_void_p(nodes[i])
+        return out
+
+    def set_node_event(self, graph_exec, node, ev):
+        self.check(self.rt.cudaGraphExecEventRecordNodeSetEvent(self.c.c_void_p(graph_exec), node, ev),
+                   "cudaGraphExecEventRecordNodeSetEvent")
+
+
 class Step:
     """Device buffers and per-pass CUDA graphs for one step over the batch.
     Each pass is one batched call (one kernel launch over all 8 operands)."""
@@ -193,20 +251,40 @@ class Step:
         for p in self.passes:
             self.run_pass(p)
 
-    def capture(self):
+    def capture(self, rt):
+        """The whole step as one CUDA graph (the passes chained by
+        programmatic dependent launch), with an event-record node before each
+        pass and after the last one. Before each replay the nodes are pointed
+        at that step's own events, so every step's pass boundaries are timed
+        with CUDA events on the launching stream."""
         torch = self.torch
-        self.graphs = {}
-        for p in self.passes:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=self.stream):
+        self.rt = rt
+        marks = [rt.event_create() for _ in range(len(self.passes) + 1)]
+        self.graph = torch.cuda.CUDAGraph(keep_graph=True)
+        with torch.cuda.graph(self.graph, stream=self.stream):
+            for i, p in enumerate(self.passes):
+                rt.record_external(marks[i], self.stream.cuda_stream)
                 self.run_pass(p)
-            self.graphs[p] = g
+            rt.record_external(marks[-1], self.stream.cuda_stream)
+        nodes = rt.event_nodes(self.graph.raw_cuda_graph())
+        self.nodes = [nodes[m.value] for m in marks]
+        self.graph.instantiate()
+        self.exec = self.graph.raw_cuda_graph_exec()
+        # the same step without event nodes: every pass boundary stays a
+        # programmatic (overlapping) launch
+        self.plain = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.plain, stream=self.stream):
+            self.run_eager()
 
     def replay(self, events=None):
-        for i, p in enumerate(self.passes):
-            self.graphs[p].replay()
-            if events is not None:
-                events[i + 1].record(self.stream)
+        """One step. With events (len(passes) + 1 fresh events) the evented
+        graph runs and records the pass boundaries; else the plain graph."""
+        if events is None:
+            self.plain.replay()
+            return
+        for node, ev in zip(self.nodes, events):
+            self.rt.set_node_event(self.exec, node, ev)
+        self.graph.replay()
 
 
 def memcpy_gbps(torch, dev, nbytes=1 << 30, iters=10):
@@ -275,17 +353,21 @@ def run_cuda(args):
     with torch.cuda.stream(stream):
         step.run_eager()          # first launches: kernel attributes, tensor-map entry point
     stream.synchronize()
-    step.capture()
+    rt = Cudart()
+    step.capture(rt)
     with torch.cuda.stream(stream):       # graph replays launch on the current stream
         for _ in range(args.warmup):
             step.replay()
+        step.replay([rt.event_create() for _ in range(len(step.passes) + 1)])   # the evented graph too
     stream.synchronize()
     if step.ws.error(stream) != 0:
         raise RuntimeError("a kernel wait timed out during warm-up")
 
-    # ---- timed region ----
+    # ---- timed region: K steps; every EVENT_EVERY-th step runs the evented
+    # graph (its pass boundaries timed by CUDA events), the others the plain one ----
     n_ev = len(step.passes) + 1
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    timed = [i for i in range(args.steps) if i % EVENT_EVERY == 0]
+    evs = {i: [rt.event_create() for _ in range(n_ev)] for i in timed}
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(dev.index)
     if world > 1:
@@ -294,8 +376,7 @@ def run_cuda(args):
     with clocks, torch.cuda.stream(stream):
         start.record(stream)
         for i in range(args.steps):
-            evs[i][0].record(stream)
-            step.replay(evs[i])
+            step.replay(evs.get(i))
         end.record(stream)
         end.synchronize()
     torch.cuda.synchronize()
@@ -303,9 +384,9 @@ def run_cuda(args):
         dist.barrier()
     elapsed_s = start.elapsed_time(end) / 1e3
     per_pass = {p: 0.0 for p in step.passes}
-    for i in range(args.steps):
+    for i in timed:
         for j, p in enumerate(step.passes):
-            per_pass[p] += evs[i][j].elapsed_time(evs[i][j + 1]) / 1e3
+            per_pass[p] += rt.elapsed_ms(evs[i][j], evs[i][j + 1]) / 1e3
     if world > 1:
         t = torch.tensor([elapsed_s], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -354,11 +435,11 @@ def run_cuda(args):
     # dominant kernel: the pass with the largest device time
     dom = max((p for p in step.passes if ab[p] > 0), key=lambda p: per_pass[p])
     # one launch per pass covers the whole batch (the ratio pass is two tiny launches)
-    dom_us = per_pass[dom] / args.steps * 1e6
+    dom_us = per_pass[dom] / len(timed) * 1e6
     achieved = BATCH * ab[dom] / (dom_us * 1e-6) / 1e9
     passes = {}
     for p in step.passes:
-        us = per_pass[p] / args.steps * 1e6
+        us = per_pass[p] / len(timed) * 1e6
         passes[p] = {"us_per_step": round(us, 3),
                      "gbps": round(BATCH * ab[p] / (us * 1e-6) / 1e9, 1) if ab[p] else None,
                      "bytes_per_launch": BATCH * ab[p]}
