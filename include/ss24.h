@@ -378,6 +378,24 @@ ss24_status ss24_decode_e2m1(const uint8_t *in, float *out, int64_t n, ss24_stre
 ss24_status ss24_selfcheck_division(int32_t mode, uint32_t b_first, uint32_t b_count,
                                     unsigned long long *result, ss24_stream stream);
 
+/* ---- self-check of the kernels' encoders ------------------------------- */
+
+/* The E4M3 (kind SS24_FMT_FP8_E4M3) or E2M1 (kind SS24_FMT_NVFP4 or
+ * SS24_FMT_MXFP4) encoder the kernels use (round to nearest even,
+ * saturating to the largest finite code) against a step table, for every fp32
+ * bit pattern (hi << 16) | lo with hi in [hi_first, hi_first + hi_count) and
+ * every lo, NaN and infinity excluded. bounds (device, ascending, 126 values
+ * for E4M3, 7 for E2M1): bounds[i] is the smallest magnitude bit pattern whose
+ * code is i + 1; the expected code of x is the number of bounds <= |x|'s bits,
+ * with the sign bit (0x80, E2M1 0x8) set when x is negative (-0 included).
+ * The caller derives the table from an independent encoder. Adds the number of
+ * mismatches to result[0] and lowers result[1] to the first mismatching bit
+ * pattern; result is a device array of two uint64 the caller initialises to
+ * {0, UINT64_MAX}. Errors: SS24_ERR_NULL, SS24_ERR_FORMAT (other kinds),
+ * SS24_ERR_SHAPE (wrong table length or hi range beyond 2^16). */
+ss24_status ss24_selfcheck_encoder(int32_t kind, const uint32_t *bounds, int32_t n_bounds, uint32_t hi_first,
+                                   uint32_t hi_count, unsigned long long *result, ss24_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

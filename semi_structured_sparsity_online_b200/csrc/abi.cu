@@ -968,6 +968,26 @@ ss24_status ss24_selfcheck_division(int32_t mode, uint32_t b_first, uint32_t b_c
     return cuda_status(launch_selfcheck_division(mode, b_first, b_count, result, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+ss24_status ss24_selfcheck_encoder(int32_t kind, const uint32_t *bounds, int32_t n_bounds, uint32_t hi_first,
+                                   uint32_t hi_count, unsigned long long *result, ss24_stream stream)
+{
+    if (!bounds || !result)
+        return SS24_ERR_NULL;
+    int e2m1;
+    if (kind == SS24_FMT_FP8_E4M3)
+        e2m1 = 0;
+    else if (kind == SS24_FMT_NVFP4 || kind == SS24_FMT_MXFP4)
+        e2m1 = 1;
+    else
+        return SS24_ERR_FORMAT;
+    if (n_bounds != (e2m1 ? 7 : 126))
+        return SS24_ERR_SHAPE;
+    if (hi_first >= 65536u || hi_count > 65536u - hi_first)
+        return SS24_ERR_SHAPE;
+    return cuda_status(launch_selfcheck_encoder(e2m1, bounds, n_bounds, hi_first, hi_count, result,
+                                                reinterpret_cast<cudaStream_t>(stream)));
+}
+
 ss24_status ss24_encode_e4m3(const float *in, uint8_t *out, int64_t n, ss24_stream stream)
 {
     if ((!in || !out) && n > 0)

@@ -116,5 +116,7 @@ cudaError_t launch_ratio(const double *sparse_side, const double *dense_side, do
 cudaError_t launch_selfcheck_division(int mode, uint32_t b_first, uint32_t b_count, unsigned long long *result,
                                       cudaStream_t stream);
 cudaError_t launch_convert(int op, const void *in, void *out, int64_t n, cudaStream_t stream);
+cudaError_t launch_selfcheck_encoder(int e2m1, const uint32_t *bounds, int n_bounds, uint32_t hi_first,
+                                     uint32_t hi_count, unsigned long long *result, cudaStream_t stream);
 
 } // namespace ss24

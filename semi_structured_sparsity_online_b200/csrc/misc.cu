@@ -161,6 +161,67 @@ cudaError_t launch_selfcheck_division(int mode, uint32_t b_first, uint32_t b_cou
     return cudaGetLastError();
 }
 
+// The kernels' encoders (cvt ... satfinite) against a step table: for the
+// fp32 bit patterns (hi << 16) | lo, hi = hi_first + blockIdx.x, every lo,
+// finite values only, the expected code of |x| is the number of bounds <= the
+// magnitude bits (bounds ascending: bounds[i] is the smallest magnitude whose
+// code is i + 1), with the sign bit (0x80 / 0x8) set for negative x, -0
+// included. e2m1: 0 = E4M3 (126 bounds), 1 = E2M1 (7 bounds).
+__global__ void selfcheck_encoder_kernel(int e2m1, const uint32_t *bounds, int n_bounds, uint32_t hi_first,
+                                         unsigned long long *result)
+{
+    __shared__ uint32_t b[128];
+    for (int i = threadIdx.x; i < n_bounds; i += blockDim.x)
+        b[i] = bounds[i];
+    __syncthreads();
+    unsigned long long bad = 0, first = ~0ull;
+    const uint32_t hi = hi_first + blockIdx.x;
+    for (uint32_t lo = threadIdx.x; lo < 65536u; lo += blockDim.x) {
+        const uint32_t bits = (hi << 16) | lo;
+        if (((bits >> 23) & 0xffu) == 0xffu)
+            continue;
+        const uint32_t mag = bits & 0x7fffffffu;
+        int lo_i = 0, hi_i = n_bounds; // count of bounds <= mag (upper bound search)
+        while (lo_i < hi_i) {
+            const int mid = (lo_i + hi_i) >> 1;
+            if (b[mid] <= mag)
+                lo_i = mid + 1;
+            else
+                hi_i = mid;
+        }
+        const float x = __uint_as_float(bits);
+        uint32_t want, got;
+        if (e2m1) {
+            want = static_cast<uint32_t>(lo_i) | ((bits >> 31) << 3);
+            got = cvt_e2m1x4(x, 0.0f, 0.0f, 0.0f) & 0xfu;
+        } else {
+            want = static_cast<uint32_t>(lo_i) | ((bits >> 31) << 7);
+            got = cvt_e4m3x2(x, 0.0f) & 0xffu;
+        }
+        if (want != got) {
+            ++bad;
+            first = min(first, static_cast<unsigned long long>(bits));
+        }
+    }
+    for (int off = 16; off >= 1; off >>= 1) {
+        bad += __shfl_xor_sync(kFull, bad, off);
+        first = min(first, __shfl_xor_sync(kFull, first, off));
+    }
+    if ((threadIdx.x & 31) == 0 && bad) {
+        atomicAdd(result, bad);
+        atomicMin(result + 1, first);
+    }
+}
+
+cudaError_t launch_selfcheck_encoder(int e2m1, const uint32_t *bounds, int n_bounds, uint32_t hi_first,
+                                     uint32_t hi_count, unsigned long long *result, cudaStream_t stream)
+{
+    if (hi_count == 0)
+        return cudaSuccess;
+    selfcheck_encoder_kernel<<<hi_count, 256, 0, stream>>>(e2m1, bounds, n_bounds, hi_first, result);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_convert(int op, const void *in, void *out, int64_t n, cudaStream_t stream)
 {
     if (n <= 0)

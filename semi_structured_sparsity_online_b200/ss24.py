@@ -14,6 +14,7 @@ from __future__ import annotations
 import ctypes
 import os
 
+import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -81,6 +82,8 @@ _SIGNATURES = {
     "ss24_bits_per_element": (ctypes.c_double, [Format, ctypes.c_int, ctypes.c_int64, ctypes.c_int32]),
     "ss24_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "ss24_selfcheck_division": (ctypes.c_int, [ctypes.c_int32, ctypes.c_uint32, ctypes.c_uint32, _P, _P]),
+    "ss24_selfcheck_encoder": (ctypes.c_int, [ctypes.c_int32, _P, ctypes.c_int32, ctypes.c_uint32, ctypes.c_uint32,
+                                              _P, _P]),
     "ss24_encode_e4m3": (ctypes.c_int, [_P, _P, ctypes.c_int64, _P]),
     "ss24_decode_e4m3": (ctypes.c_int, [_P, _P, ctypes.c_int64, _P]),
     "ss24_encode_e2m1": (ctypes.c_int, [_P, _P, ctypes.c_int64, _P]),
@@ -327,6 +330,21 @@ def selfcheck_division(mode=0, b_first=0, b_count=1 << 23, chunk=1 << 16, stream
         _check(lib().ss24_selfcheck_division(mode, b0, n, _ptr(res), _stream(stream)), "ss24_selfcheck_division")
     r = res.cpu().numpy().view("uint64")
     return int(r[0]), (None if r[1] == 0xFFFFFFFFFFFFFFFF else (int(r[1]) >> 32, int(r[1]) & 0xFFFFFFFF))
+
+
+def selfcheck_encoder(kind, bounds, chunk=1 << 12, stream=None):
+    """Mismatches between the kernels' E4M3 ("fp8") or E2M1 ("nvfp4") encoder
+    and the step table `bounds` (see ss24_selfcheck_encoder) over every finite
+    fp32 bit pattern; returns (count, first mismatching bit pattern or None)."""
+    k = _FMT[kind] if isinstance(kind, str) else int(kind)
+    b = torch.as_tensor(np.asarray(bounds, dtype=np.uint32).view(np.int32)).cuda()
+    res = torch.tensor([0, -1], dtype=torch.int64, device="cuda")
+    for h0 in range(0, 1 << 16, chunk):
+        n = min(chunk, (1 << 16) - h0)
+        _check(lib().ss24_selfcheck_encoder(k, _ptr(b), b.numel(), h0, n, _ptr(res), _stream(stream)),
+               "ss24_selfcheck_encoder")
+    r = res.cpu().numpy().view("uint64")
+    return int(r[0]), (None if r[1] == 0xFFFFFFFFFFFFFFFF else int(r[1]))
 
 
 def _convert(name, t_in, out_dtype, stream=None):

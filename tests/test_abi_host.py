@@ -181,6 +181,10 @@ def test_other_entry_points_validate():
     assert L.ss24_predicted_ratio(None, ALIGNED, ALIGNED, 1, None) == 1
     assert L.ss24_predicted_ratio(ALIGNED, ALIGNED, ALIGNED, -1, None) == 2
     assert L.ss24_selfcheck_division(3, 0, 1, ALIGNED, None) == 8
+    assert L.ss24_selfcheck_encoder(1, None, 126, 0, 1, ALIGNED, None) == 1            # null table
+    assert L.ss24_selfcheck_encoder(2, ALIGNED, 126, 0, 1, ALIGNED, None) == 5         # INT: no encoder
+    assert L.ss24_selfcheck_encoder(1, ALIGNED, 7, 0, 1, ALIGNED, None) == 2           # E4M3 wants 126
+    assert L.ss24_selfcheck_encoder(3, ALIGNED, 7, 65535, 2, ALIGNED, None) == 2       # hi range
     assert L.ss24_selfcheck_division(2, 1 << 15, 1, ALIGNED, None) == 2
     assert L.ss24_selfcheck_division(2, 100, (1 << 15) - 99, ALIGNED, None) == 2
     assert L.ss24_selfcheck_division(0, 1 << 23, 1, ALIGNED, None) == 2

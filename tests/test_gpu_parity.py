@@ -144,6 +144,15 @@ def test_e2m1_encoder_matches_oracle(ss):
         assert d[c] == oracle.e2m1_decode(c) and np.signbit(d[c]) == np.signbit(oracle.e2m1_decode(c))
 
 
+def test_encoders_match_the_oracle_on_every_fp32_pattern(ss):
+    """The kernels' E4M3 and E2M1 encoders against the oracle's step tables for
+    all 2^32 fp32 bit patterns (NaN and infinity excluded)."""
+    import encoder_bounds as eb
+    for kind, bounds in (("fp8", eb.e4m3_bounds()), ("nvfp4", eb.e2m1_bounds())):
+        bad, first = ss.selfcheck_encoder(kind, bounds)
+        assert bad == 0, f"{kind}: {bad} mismatches, first bit pattern {first:#010x}"
+
+
 # --------------------------------------------------------------------------
 # the pass: every pattern x score x format, ragged shapes
 # --------------------------------------------------------------------------

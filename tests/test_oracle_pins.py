@@ -498,3 +498,20 @@ def test_amax_of_kept_equals_amax_of_all_for_magnitude():
     assert oracle.amax(x) == oracle.amax(x, pattern=oracle.DENSE)
     w, n = synth.linear_weight(64, 512)
     assert oracle.amax(w, score=oracle.WANDA, norms=n) <= oracle.amax(w, pattern=oracle.DENSE)
+
+
+def test_encoder_step_tables_are_round_to_nearest_even_midpoints():
+    """The bisected step tables (used to check the GPU encoders over all fp32
+    patterns) sit exactly at the midpoints between neighbouring codes, the
+    midpoint itself going to the code with an even significand."""
+    import encoder_bounds as eb
+    for bounds, decode, n in ((eb.e4m3_bounds(), oracle.e4m3_decode, 127),
+                              (eb.e2m1_bounds(), oracle.e2m1_decode, 8)):
+        vals = [decode(c) for c in range(n)]
+        assert np.all(np.diff(bounds.astype(np.int64)) > 0)
+        for i in range(n - 1):
+            mid = np.float32((vals[i] + vals[i + 1]) / 2)          # exact: a few significant bits
+            assert float(mid) == (vals[i] + vals[i + 1]) / 2
+            mbits = int(np.array([mid], dtype=np.float32).view(np.uint32)[0])
+            want = mbits if (i + 1) % 2 == 0 else mbits + 1         # tie goes to the even code
+            assert int(bounds[i]) == want, (n, i)
