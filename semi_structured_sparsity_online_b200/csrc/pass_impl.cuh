@@ -252,7 +252,8 @@ struct RowScale {
 
 template <int VPC, bool STORE>
 __device__ __forceinline__ float quant_int(const float (&v)[VPC], float vmax, const QuantSpec &q, const ChunkOut &o,
-                                           float row_amax = -1.0f, const RowScale *rs = nullptr)
+                                           float row_amax = -1.0f, const RowScale *rs = nullptr,
+                                           float gamax = -1.0f)
 {
     float amax, scale;
     Recip rc;
@@ -263,7 +264,7 @@ __device__ __forceinline__ float quant_int(const float (&v)[VPC], float vmax, co
         rc = rs->rc;
         fast = rs->fast;
     } else {
-        amax = row_amax >= 0.0f ? row_amax : group_amax(vmax, q.lanes);
+        amax = row_amax >= 0.0f ? row_amax : (gamax >= 0.0f ? gamax : group_amax(vmax, q.lanes));
         scale = int_scale(amax, q);
         rc = make_recip(scale);
         fast = quot_fast(rc, amax);
@@ -383,11 +384,11 @@ __device__ __forceinline__ void build_nv_table(float *t, float st, int tid)
 
 template <int VPC, bool STORE>
 __device__ __forceinline__ float quant_nvfp4(const float (&v)[VPC], float vmax, const Recip &rst,
-                                             const ChunkOut &o, const NvTable &tb)
+                                             const ChunkOut &o, const NvTable &tb, float gamax = -1.0f)
 {
     constexpr int kLanes = 16 / VPC;
     const float st = rst.b;
-    const float amax = group_amax(vmax, kLanes);
+    const float amax = gamax >= 0.0f ? gamax : group_amax(vmax, kLanes);
     // the block scale E4M3((amax / 6) / st): two correctly rounded divisions,
     // by Markstein's correction when both are in its exact range (zero amax
     // included), else by IEEE division; one branch in the common case
@@ -425,10 +426,11 @@ __device__ __forceinline__ float quant_nvfp4(const float (&v)[VPC], float vmax, 
 // the E8M0 byte e + 127; v / 2^e is computed as v * 2^-e (the same correctly
 // rounded value, since both scale factors are exact powers of two).
 template <int VPC, bool STORE>
-__device__ __forceinline__ float quant_mxfp4(const float (&v)[VPC], float vmax, const ChunkOut &o)
+__device__ __forceinline__ float quant_mxfp4(const float (&v)[VPC], float vmax, const ChunkOut &o,
+                                             float gamax = -1.0f)
 {
     constexpr int kLanes = 32 / VPC;
-    const float amax = group_amax(vmax, kLanes);
+    const float amax = gamax >= 0.0f ? gamax : group_amax(vmax, kLanes);
     uint32_t byte = 0;
     float inv = 0.0f, mult = 0.0f;
     if (amax != 0.0f) {
@@ -518,10 +520,20 @@ __device__ __forceinline__ float chunk_amax(const typename Elem<T>::Raw &raw, co
     }
 }
 
-template <typename T, int PAT, int SCORE, int FMT>
-__device__ __forceinline__ void process_chunk(const PassParams &p, const typename Elem<T>::Raw &raw,
-                                              const ChunkOut &o, const PassConsts &c, Acc &acc,
-                                              float row_amax = -1.0f, const RowScale *rs = nullptr)
+// The selection half of a chunk: scores, the kept values (all values for the
+// dense pattern), their largest magnitude, the metadata and the chunk's
+// energies E_total and E_prune.
+template <int VPC> struct Sel {
+    float v[VPC];
+    float vmax;
+    uint32_t meta;
+    uint32_t kept_bits[2]; // bf16 2:4 by magnitude: kept values as bf16x2 (group 0, group 1)
+    float et, ep;
+};
+
+template <typename T, int PAT, int SCORE>
+__device__ __forceinline__ Sel<PAT == kDense ? 8 : 4> select_chunk(const typename Elem<T>::Raw &raw,
+                                                                   const ChunkOut &o)
 {
     constexpr int VPC = PAT == kDense ? 8 : 4;
     // two groups of bf16 values selected by magnitude with packed lanes
@@ -531,7 +543,7 @@ __device__ __forceinline__ void process_chunk(const PassParams &p, const typenam
     float v[VPC];
     float vmax;   // max |v| over the chunk's values to quantize
     uint32_t meta = 0;
-    uint32_t kept_bits[2] = {0u, 0u}; // kPair: kept values as bf16x2 (group 0, group 1)
+    uint32_t kept_bits[2] = {0u, 0u};
     float et, ep = 0.0f;
 
     if constexpr (PAT == kDense) {
@@ -619,6 +631,41 @@ __device__ __forceinline__ void process_chunk(const PassParams &p, const typenam
     }
 
 
+    Sel<VPC> r;
+#pragma unroll
+    for (int i = 0; i < VPC; ++i)
+        r.v[i] = v[i];
+    r.vmax = vmax;
+    r.meta = meta;
+    r.kept_bits[0] = kept_bits[0];
+    r.kept_bits[1] = kept_bits[1];
+    r.et = et;
+    r.ep = ep;
+    return r;
+}
+
+// The rest of a chunk: metadata and value stores, quantization, energies.
+// gamax >= 0: the group / block amax of the values to quantize, already
+// reduced across the group's lanes by the caller.
+template <typename T, int PAT, int SCORE, int FMT>
+__device__ __forceinline__ void finish_chunk(const PassParams &p, const typename Elem<T>::Raw &raw,
+                                             const Sel<PAT == kDense ? 8 : 4> &sl, const ChunkOut &o,
+                                             const PassConsts &c, Acc &acc, float row_amax = -1.0f,
+                                             const RowScale *rs = nullptr, float gamax = -1.0f)
+{
+    constexpr int VPC = PAT == kDense ? 8 : 4;
+    constexpr bool kPair = sizeof(T) == 2 && PAT == kSparse24 && SCORE == kMag;
+    float x[8]; // (unused values are not computed)
+    Elem<T>::unpack(raw, x);
+    float v[VPC];
+#pragma unroll
+    for (int i = 0; i < VPC; ++i)
+        v[i] = sl.v[i];
+    const float vmax = sl.vmax;
+    const uint32_t meta = sl.meta;
+    const uint32_t kept_bits[2] = {sl.kept_bits[0], sl.kept_bits[1]};
+    const float et = sl.et, ep = sl.ep;
+
     if constexpr (FMT == kAmax) {
         acc.amax_all = fmaxf(acc.amax_all, chunk_amax<T>(raw, x));
         if constexpr (PAT != kDense)
@@ -654,11 +701,11 @@ __device__ __forceinline__ void process_chunk(const PassParams &p, const typenam
     } else if constexpr (FMT == kFp8) {
         eq = quant_fp8<VPC, true>(v, vmax, c.rst, c.guard, o);
     } else if constexpr (FMT == kInt) {
-        eq = quant_int<VPC, true>(v, vmax, p.q, o, row_amax, rs);
+        eq = quant_int<VPC, true>(v, vmax, p.q, o, row_amax, rs, gamax);
     } else if constexpr (FMT == kNvfp4) {
-        eq = quant_nvfp4<VPC, true>(v, vmax, c.rst, o, c.tb);
+        eq = quant_nvfp4<VPC, true>(v, vmax, c.rst, o, c.tb, gamax);
     } else if constexpr (FMT == kMxfp4) {
-        eq = quant_mxfp4<VPC, true>(v, vmax, o);
+        eq = quant_mxfp4<VPC, true>(v, vmax, o, gamax);
     } else if constexpr (FMT == kEnergy) {
         eq = quant_energy_only<VPC>(v, vmax, p.q, c.rst, c.guard, c.tb);
         acc.eqd += quant_energy_only<8>(x, chunk_amax<T>(raw, x), p.qd, c.rstd, c.guardd, c.tbd);
@@ -667,6 +714,15 @@ __device__ __forceinline__ void process_chunk(const PassParams &p, const typenam
         acc.eqd += eq;
     else
         acc.eq += eq;
+}
+
+template <typename T, int PAT, int SCORE, int FMT>
+__device__ __forceinline__ void process_chunk(const PassParams &p, const typename Elem<T>::Raw &raw,
+                                              const ChunkOut &o, const PassConsts &c, Acc &acc,
+                                              float row_amax = -1.0f, const RowScale *rs = nullptr)
+{
+    const auto sl = select_chunk<T, PAT, SCORE>(raw, o);
+    finish_chunk<T, PAT, SCORE, FMT>(p, raw, sl, o, c, acc, row_amax, rs);
 }
 
 // ---------------------------------------------------------------------------
@@ -1002,9 +1058,10 @@ template <> struct Stream<float> {
 // (Four CTAs where the kernel fits 64 registers without spilling, else three;
 // two for the energy pass.)
 template <typename T, int PAT, int SCORE, int FMT, bool FW> struct StreamOcc {
-    static constexpr bool light = FMT == kAmax || (sizeof(T) == 2 && SCORE == kMag && PAT != kSparse48 &&
-                                                   FMT != kEnergy && FMT != kNvfp4 &&
-                                                   (FW || !(PAT != kDense && FMT == kFp8)));
+    // (INT holds four selected chunks across its group reduction)
+    static constexpr bool light =
+        FMT == kAmax || (sizeof(T) == 2 && SCORE == kMag && PAT != kSparse48 &&
+                         (FMT == kNone || FMT == kMxfp4 || (FMT == kFp8 && (FW || PAT == kDense))));
     static constexpr int value = FMT == kEnergy ? 2 : light ? 4 : 3; // the energy pass: two formats live
 };
 
@@ -1036,8 +1093,7 @@ __device__ __forceinline__ void stream_unit(const PassParams &p, const PassConst
         ok[i] = FULL || (row0 + i * p.step_rows < p.rows && col0 + i * p.step_cols < p.k);
         raw[i] = Stream<T>::load(xp + i * step_x, ok[i]);
     }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    auto out_i = [&](int i) {
         ChunkOut oi = o;
         oi.val += i * dval;
         oi.scale += i * dscale;
@@ -1045,7 +1101,33 @@ __device__ __forceinline__ void stream_unit(const PassParams &p, const PassConst
         if constexpr (SCORE == kWanda)
             oi.norms = o.norms + i * step_c;
         oi.valid = ok[i];
-        process_chunk<T, PAT, SCORE, FMT>(p, raw[i], oi, c, acc);
+        return oi;
+    };
+    if constexpr (FMT == kInt) {
+        // INT groups (up to 32 lanes): select all four chunks, then reduce
+        // their group amaxes across lanes together (four independent shuffle
+        // chains instead of four dependent ones), then quantize. The short
+        // NVFP4 / MXFP4 reductions gain less than the registers cost.
+        constexpr int VPC = PAT == kDense ? 8 : 4;
+        Sel<VPC> sl[4];
+        float g[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            sl[i] = select_chunk<T, PAT, SCORE>(raw[i], out_i(i));
+            g[i] = sl[i].vmax;
+        }
+        const int lanes = p.q.lanes;
+        for (int off = 1; off < lanes; off <<= 1)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                g[i] = fmaxf(g[i], __shfl_xor_sync(kFull, g[i], off));
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            finish_chunk<T, PAT, SCORE, FMT>(p, raw[i], sl[i], out_i(i), c, acc, -1.0f, nullptr, g[i]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            process_chunk<T, PAT, SCORE, FMT>(p, raw[i], out_i(i), c, acc);
     }
 }
 
