@@ -5,11 +5,12 @@ Workload (one step): a batch of B = 8 linear-layer inputs X, each bf16
 A step runs every row of the hot path once over the batch, pass by pass; each
 pass is one batched call over all 8 operands (one kernel launch), so each
 pass reads its operands from HBM (the batch is 256 MiB, twice the L2):
-  1. per-tensor FP8 scale of each X (amax pass)            ss24_tensor_scale
+  1. per-tensor FP8 scale and per-row amax of each X       ss24_amax_rows
   2. fused 2:4 magnitude prune + compress + FP8 E4M3 of the
      kept values + energies (E_total, E_prune, E_q)        ss24_prune24_quant_fused
   3. dense FP8 E4M3 partner (same scale) + energy          ss24_quantize_fp8
-  4. dense INT8, one scale per row, partner + energy       ss24_quantize_int
+  4. dense INT8, one scale per row (from the row amax),
+     partner + energy                                      ss24_quantize_int_rows
   5. predicted R against both partners (one launch each)   ss24_predicted_ratio
 The whole step is one CUDA graph, the passes chained by programmatic dependent
 launch. Every 8th step of the timed region instead replays a copy of that graph
@@ -49,10 +50,10 @@ def algorithmic_bytes(m=M, k=K):
     """Bytes each pass must move per operand (bf16 in; see the DESIGN notes)."""
     n = m * k
     return {
-        "tensor_scale": 2 * n,                         # read X
+        "tensor_scale": 2 * n + 4 * m,                 # read X; write the row amax
         "fused_24_fp8": 2 * n + n // 2 + n // 8,       # read X; write FP8 codes (k/2) + metadata (k/8)
         "dense_fp8": 2 * n + n,                        # read X; write FP8 codes
-        "dense_int8_row": 2 * n + n + 4 * m,           # read X; write INT8 codes + one fp32 scale per row
+        "dense_int8_row": 2 * n + 4 * m + n + 4 * m,   # read X and the row amax; write INT8 codes + row scales
         "ratio": 0,
     }
 
@@ -220,6 +221,7 @@ class Step:
         dev = x_dev.device
         self.ws = ss.Workspace(dev, stream)
         self.scale = torch.empty(BATCH, dtype=torch.float32, device=dev)
+        self.row_amax = torch.empty((BATCH, M), dtype=torch.float32, device=dev)
         self.sp = ss._alloc_outputs(M, K, ss.SPARSE_24, ss.make_format("fp8"), torch.bfloat16, dev, BATCH)
         self.d8 = ss._alloc_outputs(M, K, ss.DENSE, ss.make_format("fp8"), torch.bfloat16, dev, BATCH)
         self.di = ss._alloc_outputs(M, K, ss.DENSE, ss.make_format("int", 8, 0), torch.bfloat16, dev, BATCH)
@@ -231,7 +233,10 @@ class Step:
     def run_pass(self, name):
         ss, s, x = self.ss, self.stream, self.x
         if name == "tensor_scale":
-            ss.tensor_scale(x, "fp8", ss.SPARSE_24, ws=self.ws, stream=s, out=self.scale)
+            # the FP8 tensor scale and the per-row amax of the INT8 partner in
+            # one read (magnitude score: the kept amax equals the amax of all)
+            ss.amax_rows(x, pattern=ss.DENSE, scale_fmt="fp8", ws=self.ws, stream=s, out=self.row_amax,
+                         scale_out=self.scale)
         elif name == "fused_24_fp8":
             ss.run(x, pattern=ss.SPARSE_24, fmt="fp8", tensor_scale=self.scale, energy=self.e[0], ws=self.ws,
                    stream=s, out=self.sp)
@@ -241,8 +246,8 @@ class Step:
             ss.run(x, pattern=ss.DENSE, fmt="fp8", tensor_scale=self.scale, energy=self.e[1], ws=self.ws,
                    stream=s, out=self.d8)
         elif name == "dense_int8_row":
-            ss.run(x, pattern=ss.DENSE, fmt="int", bits=8, group=0, energy=self.e[2], ws=self.ws, stream=s,
-                   out=self.di)
+            ss.run_int_rows(x, self.row_amax, pattern=ss.DENSE, bits=8, energy=self.e[2], ws=self.ws, stream=s,
+                            out=self.di)
         elif name == "ratio":
             ss.predicted_ratio(self.e[0], self.e[1], out=self.r[0], stream=s)
             ss.predicted_ratio(self.e[0], self.e[2], out=self.r[1], stream=s)

@@ -288,6 +288,34 @@ ss24_status ss24_tensor_scale(const ss24_operand *x, ss24_pattern pattern, ss24_
                               const float *col_norms, int32_t kind, float *scale_out, void *ws,
                               size_t ws_bytes, ss24_stream stream);
 
+/* Per-row amax in the same read as the per-tensor scale (§3: INT with one
+ * scale per row needs the amax of each row before its codes; a pass that reads
+ * the operand for the tensor scale can produce them at no extra read). Writes
+ * row_amax[b * rows + r] = max |value| over the values of row r of operand b
+ * that a pass with this pattern and score quantizes (the kept values for a
+ * sparse pattern). row_amax: device, batch x rows fp32, 4-byte aligned (NULL
+ * allowed when rows is 0); the call clears it first (it is reduced by atomic
+ * maxima). If scale_out is not
+ * NULL it also writes the per-tensor scale of kind (SS24_FMT_FP8_E4M3 or
+ * SS24_FMT_NVFP4) as ss24_tensor_scale does. Axis 1 only (SS24_ERR_ARG
+ * otherwise). */
+ss24_status ss24_amax_rows(const ss24_operand *x, ss24_pattern pattern, ss24_score score, const float *col_norms,
+                           float *row_amax, int32_t kind, float *scale_out, void *ws, size_t ws_bytes,
+                           ss24_stream stream);
+
+/* INT-b with one scale per row (fmt.kind SS24_FMT_INT, fmt.group 0) from a
+ * given per-row amax, as ss24_amax_rows writes it for the same pattern and
+ * score: scale = amax / qmax per row, then the codes, metadata, scales and
+ * energies of ss24_prune24_quant_fused / ss24_prune48_pairwise_quant_fused
+ * (sparse patterns) or ss24_quantize_int (SS24_DENSE), identical to them when
+ * row_amax holds the rows' amax. One streaming pass (the rows need not fit a
+ * block of threads). row_amax: device, batch x rows fp32, 4-byte aligned.
+ * Axis 1 only. */
+ss24_status ss24_quantize_int_rows(const ss24_operand *x, ss24_pattern pattern, ss24_score score,
+                                   const float *col_norms, ss24_format fmt, const float *row_amax,
+                                   ss24_outputs *out, ss24_energy *energy, void *ws, size_t ws_bytes,
+                                   ss24_stream stream);
+
 /* Derived quantities (§4) from sparse-side energy records (e_total, e_prune,
  * e_quant) and dense-side records (e_quant_dense): count consecutive pairs,
  * sparse_side[i] with dense_side[i] -> out[i]. Device pointers; the two inputs

@@ -534,7 +534,7 @@ bool plan_tile(const ss24_operand *x, int pattern, int score, int mode, TilePlan
 // cheaper dense form is used.
 cudaError_t run_amax(const ss24_operand *x, int pattern, int score, const float *norms, void *ws,
                      cudaStream_t stream, float *scale_out = nullptr, float divisor = 1.0f,
-                     float *amax_user = nullptr)
+                     float *amax_user = nullptr, float *row_amax = nullptr)
 {
     const int pat = score == SS24_SCORE_MAG ? SS24_DENSE : pattern;
     TilePlan t;
@@ -545,6 +545,7 @@ cudaError_t run_amax(const ss24_operand *x, int pattern, int score, const float 
     p.q.scale_out = scale_out;
     p.q.divisor = divisor;
     p.amax_user = amax_user;
+    p.row_amax = row_amax;
     return launch(t.kernel, t.smem, t.g.n_tiles, t.map, p, stream);
 }
 
@@ -568,7 +569,7 @@ ss24_status empty_operand(const ss24_operand *x, ss24_energy *energy, const ss24
 // The storing pass shared by the quantize / prune entry points.
 ss24_status run_pass(const ss24_operand *x, int pattern, int score, const float *norms, ss24_format fmt,
                      bool allow_none, const float *scale_in, const ss24_outputs *out, ss24_energy *energy,
-                     void *ws, size_t ws_bytes, cudaStream_t stream)
+                     void *ws, size_t ws_bytes, cudaStream_t stream, const float *row_amax_in = nullptr)
 {
     ss24_status st = check_operand(x);
     if (st != SS24_OK)
@@ -621,6 +622,9 @@ ss24_status run_pass(const ss24_operand *x, int pattern, int score, const float 
     p.meta = out->meta;
     p.norms = norms;
     p.q = r.q;
+    p.q.row_amax_in = row_amax_in;
+    if (row_amax_in)
+        r.row_mode = false; // the stream kernel, with the rows' scales from the given amax
     if (per_tensor(fmt.kind)) {
         p.q.scale_out = out->tensor_scale;
         p.q.scale_in = scale_in;
@@ -642,7 +646,7 @@ ss24_status run_pass(const ss24_operand *x, int pattern, int score, const float 
         e = launch_rowsweep(k, x, p, stream);
     } else {
         TilePlan t;
-        if (!plan_tile(x, pattern, score, fmt.kind, &t))
+        if (!plan_tile(x, pattern, score, row_amax_in ? static_cast<int>(kIntRows) : fmt.kind, &t))
             return SS24_ERR_CUDA;
         e = launch(t.kernel, t.smem, t.g.n_tiles, t.map, p, stream);
     }
@@ -848,6 +852,60 @@ ss24_status ss24_amax(const ss24_operand *x, ss24_pattern pattern, ss24_score sc
     if (x->rows == 0)
         return cuda_status(cudaMemsetAsync(amax_out, 0, nbatch(x) * sizeof(float), s));
     return cuda_status(run_amax(x, pattern, score, col_norms, ws, s, nullptr, 1.0f, amax_out));
+}
+
+ss24_status ss24_amax_rows(const ss24_operand *x, ss24_pattern pattern, ss24_score score, const float *col_norms,
+                           float *row_amax, int32_t kind, float *scale_out, void *ws, size_t ws_bytes,
+                           ss24_stream stream)
+{
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    ss24_status st = check_operand(x);
+    if (st != SS24_OK)
+        return st;
+    if (x->axis != 1)
+        return SS24_ERR_ARG;
+    if ((st = check_pattern_k(pattern, x->k)) != SS24_OK)
+        return st;
+    if (score != SS24_SCORE_MAG && score != SS24_SCORE_WANDA)
+        return SS24_ERR_ARG;
+    if (score == SS24_SCORE_WANDA && pattern != SS24_DENSE && (!col_norms || !aligned16(col_norms)))
+        return col_norms ? SS24_ERR_ALIGN : SS24_ERR_NULL;
+    if (scale_out && !per_tensor(kind))
+        return SS24_ERR_FORMAT;
+    if ((st = check_ws(ws, ws_bytes)) != SS24_OK)
+        return st;
+    if (!row_amax && x->rows != 0) // an empty operand may give a NULL row array
+        return SS24_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(row_amax) & 3u) != 0)
+        return SS24_ERR_ALIGN;
+    const size_t nb = static_cast<size_t>(nbatch(x));
+    if (x->rows == 0)
+        return scale_out ? cuda_status(cudaMemsetAsync(scale_out, 0, nb * sizeof(float), s)) : SS24_OK;
+    cudaError_t e = cudaMemsetAsync(row_amax, 0, nb * static_cast<size_t>(x->rows) * sizeof(float), s);
+    if (e != cudaSuccess)
+        return SS24_ERR_CUDA;
+    const float divisor = kind == SS24_FMT_FP8_E4M3 ? 448.0f : 2688.0f;
+    return cuda_status(run_amax(x, pattern, score, col_norms, ws, s, scale_out, scale_out ? divisor : 1.0f, nullptr,
+                                row_amax));
+}
+
+ss24_status ss24_quantize_int_rows(const ss24_operand *x, ss24_pattern pattern, ss24_score score,
+                                   const float *col_norms, ss24_format fmt, const float *row_amax,
+                                   ss24_outputs *out, ss24_energy *energy, void *ws, size_t ws_bytes,
+                                   ss24_stream stream)
+{
+    if (fmt.kind != SS24_FMT_INT || fmt.group != 0)
+        return SS24_ERR_FORMAT;
+    if (!x)
+        return SS24_ERR_NULL;
+    if (x->axis != 1)
+        return SS24_ERR_ARG;
+    if (!row_amax && x->rows != 0)
+        return SS24_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(row_amax) & 3u) != 0)
+        return SS24_ERR_ALIGN;
+    return run_pass(x, pattern, score, col_norms, fmt, false, nullptr, out, energy, ws, ws_bytes,
+                    reinterpret_cast<cudaStream_t>(stream), row_amax);
 }
 
 ss24_status ss24_tensor_scale(const ss24_operand *x, ss24_pattern pattern, ss24_score score, const float *col_norms,

@@ -11,8 +11,9 @@ namespace ss24 {
 enum Pattern { kDense = 0, kSparse24 = 24, kSparse48 = 48 };
 enum Score { kMag = 0, kWanda = 1 };
 // Formats of the pass; kAmax is the read-only amax pass; kEnergy the
-// read-only two-format energy pass.
-enum Fmt { kNone = 0, kFp8 = 1, kInt = 2, kNvfp4 = 3, kMxfp4 = 4, kAmax = 5, kEnergy = 6 };
+// read-only two-format energy pass; kIntRows is INT with one scale per row
+// from a given per-row amax (the stream kernel).
+enum Fmt { kNone = 0, kFp8 = 1, kInt = 2, kNvfp4 = 3, kMxfp4 = 4, kAmax = 5, kEnergy = 6, kIntRows = 7 };
 enum IntStore { kInt8 = 0, kInt16 = 1, kPack4 = 2 };
 
 // Consumer warps per CTA and the TMA stage ring (each stage 16 KiB).
@@ -69,6 +70,8 @@ struct QuantSpec {
     float divisor;     // FP8: 448, NVFP4: 2688 (tensor scale = amax / divisor)
     const float *scale_in;     // given tensor scale (device) or nullptr
     const float *amax_reduced; // device float holding the amax when the scale is computed
+    const float *row_amax_in;  // INT, one scale per row: the given amax of each row's quantized
+                               // values, [batch][rows] (device), or nullptr
     float *scale_out;          // where to write the tensor scale used (device) or nullptr
 };
 
@@ -98,6 +101,8 @@ struct PassParams {
     float *amax_partials;      // kAmax: [grid][2] (workspace)
     float *amax_out;           // kAmax: [batch][2] (kept values, all values)
     float *amax_user;          // kAmax: caller's [batch] amax of the quantized values, or nullptr
+    float *row_amax;           // kAmax: the amax of each row's quantized values, [batch][rows]
+                               // (device, zero before the launch; atomic max), or nullptr
     uint32_t *energy_ticket;   // last-CTA-done counters, one per operand (workspace)
     uint32_t *amax_ticket;
     int32_t *err;              // workspace error word

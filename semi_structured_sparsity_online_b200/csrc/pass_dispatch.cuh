@@ -17,6 +17,8 @@ template <typename T, int PAT, int SC, bool FW> const void *stream_kernel_for_fm
         return reinterpret_cast<const void *>(&stream_kernel<T, PAT, SC, kFp8, FW>);
     case kInt:
         return reinterpret_cast<const void *>(&stream_kernel<T, PAT, SC, kInt, FW>);
+    case kIntRows:
+        return reinterpret_cast<const void *>(&stream_kernel<T, PAT, SC, kIntRows, FW>);
     case kNvfp4:
         return reinterpret_cast<const void *>(&stream_kernel<T, PAT, SC, kNvfp4, FW>);
     case kMxfp4:

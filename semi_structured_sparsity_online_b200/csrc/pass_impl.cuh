@@ -20,6 +20,8 @@
 // to finish (a ticket counter) reduces the per-CTA partials in fixed order.
 #pragma once
 
+#include <type_traits>
+
 #include "device.cuh"
 #include "internal.cuh"
 
@@ -700,7 +702,7 @@ __device__ __forceinline__ void finish_chunk(const PassParams &p, const typename
         }
     } else if constexpr (FMT == kFp8) {
         eq = quant_fp8<VPC, true>(v, vmax, c.rst, c.guard, o);
-    } else if constexpr (FMT == kInt) {
+    } else if constexpr (FMT == kInt || FMT == kIntRows) {
         eq = quant_int<VPC, true>(v, vmax, p.q, o, row_amax, rs, gamax);
     } else if constexpr (FMT == kNvfp4) {
         eq = quant_nvfp4<VPC, true>(v, vmax, c.rst, o, c.tb, gamax);
@@ -723,6 +725,80 @@ __device__ __forceinline__ void process_chunk(const PassParams &p, const typenam
 {
     const auto sl = select_chunk<T, PAT, SCORE>(raw, o);
     finish_chunk<T, PAT, SCORE, FMT>(p, raw, sl, o, c, acc, row_amax, rs);
+}
+
+// Dense INT-b codes of one chunk with its row's scale, straight-line on
+// binary32 pairs: the same operations, roundings and summation order as
+// quant_int / err_energy and the dense energy in process_chunk, with the code
+// width (STORE) and the fast-division decision (FAST, one per row) fixed.
+template <typename T, int STORE, bool FAST>
+__device__ __forceinline__ void dense_int_chunk(const typename Elem<T>::Raw &raw, const RowScale &rs, float qmax,
+                                                uint8_t *val, bool valid, Acc &acc)
+{
+    float x[8];
+    Elem<T>::unpack(raw, x);
+    f32x2 x2[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        x2[i] = pack2(x[2 * i], x[2 * i + 1]);
+    f32x2 t[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        t[i] = mul2(x2[i], x2[i]);
+    t[0] = add2(add2(t[0], t[1]), add2(t[2], t[3]));
+    acc.et += lo2(t[0]) + hi2(t[0]);
+    const f32x2 m2 = pack2(kMagic, kMagic), s2 = pack2(rs.scale, rs.scale);
+    f32x2 tt[4], e[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f32x2 qn;
+        if constexpr (FAST) {
+            qn = neg_div_fast2(x2[i], rs.rc);
+        } else {
+            float a = rs.rc.b != 0.0f ? __fdiv_rn(-x[2 * i], rs.rc.b) : -0.0f;
+            float b = rs.rc.b != 0.0f ? __fdiv_rn(-x[2 * i + 1], rs.rc.b) : -0.0f;
+            qn = pack2(fminf(fmaxf(a, -qmax), qmax), fminf(fmaxf(b, -qmax), qmax));
+        }
+        tt[i] = sub2(m2, qn);
+        const f32x2 d = mul2(sub2(tt[i], m2), s2);
+        const f32x2 df = sub2(x2[i], d);
+        e[i] = mul2(df, df);
+    }
+    e[0] = add2(add2(e[0], e[2]), add2(e[1], e[3]));
+    acc.eqd += lo2(e[0]) + hi2(e[0]);
+    if (valid) {
+        uint32_t b[8]; // low bits of M + q hold the two's-complement code
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            b[2 * i] = __float_as_uint(lo2(tt[i]));
+            b[2 * i + 1] = __float_as_uint(hi2(tt[i]));
+        }
+        if constexpr (STORE == kInt8) {
+            *reinterpret_cast<uint2 *>(val) =
+                make_uint2(__byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410),
+                           __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410));
+        } else if constexpr (STORE == kInt16) {
+            *reinterpret_cast<uint4 *>(val) = make_uint4(__byte_perm(b[0], b[1], 0x5410), __byte_perm(b[2], b[3], 0x5410),
+                                                         __byte_perm(b[4], b[5], 0x5410), __byte_perm(b[6], b[7], 0x5410));
+        } else {
+            uint32_t w = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                w |= (b[i] & 0xfu) << (4 * i);
+            *reinterpret_cast<uint32_t *>(val) = w;
+        }
+    }
+}
+
+// The CPT chunks of a thread in one row (dense operand), chunk j at val0 + j * cval.
+template <typename T, int CPT, int STORE, bool FAST>
+__device__ __forceinline__ void dense_int_row(const typename Elem<T>::Raw (&raw)[CPT], const RowScale &rs, float qmax,
+                                              uint8_t *val0, int64_t cval, int t, int tpr, int nchunks, bool rv,
+                                              Acc &acc)
+{
+#pragma unroll
+    for (int j = 0; j < CPT; ++j)
+        dense_int_chunk<T, STORE, FAST>(raw[j], rs, qmax, val0 + j * cval, rv && t + j * tpr < nchunks, acc);
 }
 
 // ---------------------------------------------------------------------------
@@ -962,7 +1038,7 @@ __device__ __forceinline__ ChunkOut make_out(const PassParams &p, const OutBase 
         o.val = vals + off * static_cast<int64_t>(sizeof(T));
     } else if constexpr (FMT == kFp8) {
         o.val = vals + off;
-    } else if constexpr (FMT == kInt) {
+    } else if constexpr (FMT == kInt || FMT == kIntRows) {
         o.val = vals + (p.q.store == kInt8 ? off : (p.q.store == kInt16 ? 2 * off : off / 2));
         const int lg = __ffs(p.q.group) - 1; // tile-mode groups are powers of two
         o.scale = sc + 4 * (row * (n >> lg) + (colq >> lg));
@@ -1083,7 +1159,9 @@ template <typename T, int PAT, int FMT> struct FwStep {
 template <typename T, int PAT, int SCORE, int FMT, bool FULL>
 __device__ __forceinline__ void stream_unit(const PassParams &p, const PassConsts &c, const T *xp, int64_t step_x,
                                             int64_t step_c, const ChunkOut &o, int64_t dval, int64_t dscale,
-                                            int64_t dmeta, int64_t row0, int64_t col0, Acc &acc)
+                                            int64_t dmeta, int64_t row0, int64_t col0, Acc &acc,
+                                            float *rowa = nullptr, const float *rowa_in = nullptr,
+                                            float *rscales = nullptr)
 {
     using E = Elem<T>;
     typename E::Raw raw[4];
@@ -1103,6 +1181,75 @@ __device__ __forceinline__ void stream_unit(const PassParams &p, const PassConst
         oi.valid = ok[i];
         return oi;
     };
+    const int lane = static_cast<int>(threadIdx.x & 31);
+    if constexpr (FMT == kIntRows) {
+        {
+            // one scale per row from the given row amax: the chunks' rows are
+            // row0 + i * step_rows; the first lane of a row's first segment
+            // stores the row's scale
+            if constexpr (PAT == kDense) {
+                if (p.step_rows == 0) {
+                    // one row for the whole unit: one scale, the straight-line
+                    // chunk quantizer with the code width fixed
+                    const bool rv = row0 < p.rows;
+                    RowScale rs;
+                    rs.given = true;
+                    rs.amax = rv ? rowa_in[row0] : 0.0f;
+                    rs.scale = int_scale(rs.amax, p.q);
+                    rs.rc = make_recip(rs.scale);
+                    rs.fast = quot_fast(rs.rc, rs.amax);
+                    const float qm = p.q.qmax;
+                    auto run = [&](auto store_tag, auto fast_tag) {
+                        constexpr int S = decltype(store_tag)::value;
+                        constexpr bool F = decltype(fast_tag)::value;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            dense_int_chunk<T, S, F>(raw[i], rs, qm, o.val + i * dval, ok[i], acc);
+                    };
+                    using I8 = std::integral_constant<int, kInt8>;
+                    using I16 = std::integral_constant<int, kInt16>;
+                    using P4 = std::integral_constant<int, kPack4>;
+                    using Y = std::true_type;
+                    using N = std::false_type;
+                    const int st = p.q.store;
+                    if (rs.fast) {
+                        if (st == kInt8)
+                            run(I8{}, Y{});
+                        else if (st == kInt16)
+                            run(I16{}, Y{});
+                        else
+                            run(P4{}, Y{});
+                    } else {
+                        if (st == kInt8)
+                            run(I8{}, N{});
+                        else if (st == kInt16)
+                            run(I16{}, N{});
+                        else
+                            run(P4{}, N{});
+                    }
+                    if (rv && col0 == 0)
+                        rscales[row0] = rs.scale;
+                    return;
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int64_t row = row0 + i * p.step_rows;
+                const bool rv = row < p.rows;
+                RowScale rs;
+                rs.given = true;
+                rs.amax = rv ? rowa_in[row] : 0.0f;
+                rs.scale = int_scale(rs.amax, p.q);
+                rs.rc = make_recip(rs.scale);
+                rs.fast = quot_fast(rs.rc, rs.amax);
+                const ChunkOut oi = out_i(i);
+                process_chunk<T, PAT, SCORE, FMT>(p, raw[i], oi, c, acc, rs.amax, &rs);
+                if (rv && col0 + i * p.step_cols == 0)
+                    rscales[row] = rs.scale;
+            }
+            return;
+        }
+    }
     if constexpr (FMT == kInt) {
         // INT groups (up to 32 lanes): select all four chunks, then reduce
         // their group amaxes across lanes together (four independent shuffle
@@ -1128,6 +1275,40 @@ __device__ __forceinline__ void stream_unit(const PassParams &p, const PassConst
 #pragma unroll
         for (int i = 0; i < 4; ++i)
             process_chunk<T, PAT, SCORE, FMT>(p, raw[i], out_i(i), c, acc);
+        if constexpr (FMT == kAmax) {
+            if (rowa) {
+                // per-row amax of the values to quantize: reduced over the
+                // lanes sharing a row segment, then an atomic max (non-negative
+                // floats order like their bit patterns)
+                const int lcpr = p.log2_cpr, segl = 1 << lcpr;
+                float cm[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    if constexpr (PAT == kDense || SCORE == kMag) {
+                        float xv[8];
+                        Elem<T>::unpack(raw[i], xv);
+                        cm[i] = chunk_amax<T>(raw[i], xv);
+                    } else {
+                        cm[i] = select_chunk<T, PAT, SCORE>(raw[i], out_i(i)).vmax;
+                    }
+                }
+                if (p.step_rows == 0) {
+                    // the four chunks share the lane's row
+                    float m = fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3]));
+                    m = group_amax(m, segl);
+                    if ((lane & (segl - 1)) == 0 && row0 < p.rows)
+                        atomicMax(reinterpret_cast<int *>(rowa + row0), __float_as_int(m));
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float m = group_amax(cm[i], segl);
+                        const int64_t row = row0 + i * p.step_rows;
+                        if ((lane & (segl - 1)) == 0 && row < p.rows)
+                            atomicMax(reinterpret_cast<int *>(rowa + row), __float_as_int(m));
+                    }
+                }
+            }
+        }
     }
 }
 
@@ -1161,6 +1342,10 @@ __global__ void __launch_bounds__(kStreamThreads, (StreamOcc<T, PAT, SCORE, FMT,
     grid_dependents_launch();
     const PassConsts c = make_consts<FMT>(operand_view(pk), tid, kStreamThreads, nvt);
     const OutBase ob = out_base(pk, op);
+    // per-row amax out (amax pass) or in (INT with one scale per row)
+    float *rowa = FMT == kAmax && p.row_amax ? p.row_amax + op * p.rows : nullptr;
+    const float *rowa_in = FMT == kIntRows ? p.q.row_amax_in + op * p.rows : nullptr;
+    float *rscales = reinterpret_cast<float *>(ob.scales);
 
     const T *x = static_cast<const T *>(p.x) + op * p.x_bstride;
     const int log2_cpr = FW ? 5 : p.log2_cpr;
@@ -1195,10 +1380,10 @@ __global__ void __launch_bounds__(kStreamThreads, (StreamOcc<T, PAT, SCORE, FMT,
         // of a row (rows are whole: one row per unit)
         if (FW && static_cast<int64_t>(ub + 1) * 1024 <= p.k)
             stream_unit<T, PAT, SCORE, FMT, true>(p, c, xp, step_x, step_c, o, dval, dscale, dmeta, row0, col0,
-                                                  acc);
+                                                  acc, rowa, rowa_in, rscales);
         else
             stream_unit<T, PAT, SCORE, FMT, false>(p, c, xp, step_x, step_c, o, dval, dscale, dmeta, row0, col0,
-                                                   acc);
+                                                   acc, rowa, rowa_in, rscales);
         // only the energies this pass produces (the others stay zero)
         if constexpr (FMT != kAmax)
             e_total += acc.et;
@@ -1347,80 +1532,6 @@ __global__ void __launch_bounds__(kRowThreads) rowsweep_kernel(const T *__restri
 // between steps); the codes are then computed from the registers, so the
 // operand is read once.
 // ---------------------------------------------------------------------------
-
-// Dense INT-b codes of one chunk with its row's scale, straight-line on
-// binary32 pairs: the same operations, roundings and summation order as
-// quant_int / err_energy and the dense energy in process_chunk, with the code
-// width (STORE) and the fast-division decision (FAST, one per row) fixed.
-template <typename T, int STORE, bool FAST>
-__device__ __forceinline__ void dense_int_chunk(const typename Elem<T>::Raw &raw, const RowScale &rs, float qmax,
-                                                uint8_t *val, bool valid, Acc &acc)
-{
-    float x[8];
-    Elem<T>::unpack(raw, x);
-    f32x2 x2[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-        x2[i] = pack2(x[2 * i], x[2 * i + 1]);
-    f32x2 t[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-        t[i] = mul2(x2[i], x2[i]);
-    t[0] = add2(add2(t[0], t[1]), add2(t[2], t[3]));
-    acc.et += lo2(t[0]) + hi2(t[0]);
-    const f32x2 m2 = pack2(kMagic, kMagic), s2 = pack2(rs.scale, rs.scale);
-    f32x2 tt[4], e[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        f32x2 qn;
-        if constexpr (FAST) {
-            qn = neg_div_fast2(x2[i], rs.rc);
-        } else {
-            float a = rs.rc.b != 0.0f ? __fdiv_rn(-x[2 * i], rs.rc.b) : -0.0f;
-            float b = rs.rc.b != 0.0f ? __fdiv_rn(-x[2 * i + 1], rs.rc.b) : -0.0f;
-            qn = pack2(fminf(fmaxf(a, -qmax), qmax), fminf(fmaxf(b, -qmax), qmax));
-        }
-        tt[i] = sub2(m2, qn);
-        const f32x2 d = mul2(sub2(tt[i], m2), s2);
-        const f32x2 df = sub2(x2[i], d);
-        e[i] = mul2(df, df);
-    }
-    e[0] = add2(add2(e[0], e[2]), add2(e[1], e[3]));
-    acc.eqd += lo2(e[0]) + hi2(e[0]);
-    if (valid) {
-        uint32_t b[8]; // low bits of M + q hold the two's-complement code
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            b[2 * i] = __float_as_uint(lo2(tt[i]));
-            b[2 * i + 1] = __float_as_uint(hi2(tt[i]));
-        }
-        if constexpr (STORE == kInt8) {
-            *reinterpret_cast<uint2 *>(val) =
-                make_uint2(__byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410),
-                           __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410));
-        } else if constexpr (STORE == kInt16) {
-            *reinterpret_cast<uint4 *>(val) = make_uint4(__byte_perm(b[0], b[1], 0x5410), __byte_perm(b[2], b[3], 0x5410),
-                                                         __byte_perm(b[4], b[5], 0x5410), __byte_perm(b[6], b[7], 0x5410));
-        } else {
-            uint32_t w = 0;
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                w |= (b[i] & 0xfu) << (4 * i);
-            *reinterpret_cast<uint32_t *>(val) = w;
-        }
-    }
-}
-
-// The CPT chunks of a thread in one row (dense operand), chunk j at val0 + j * cval.
-template <typename T, int CPT, int STORE, bool FAST>
-__device__ __forceinline__ void dense_int_row(const typename Elem<T>::Raw (&raw)[CPT], const RowScale &rs, float qmax,
-                                              uint8_t *val0, int64_t cval, int t, int tpr, int nchunks, bool rv,
-                                              Acc &acc)
-{
-#pragma unroll
-    for (int j = 0; j < CPT; ++j)
-        dense_int_chunk<T, STORE, FAST>(raw[j], rs, qmax, val0 + j * cval, rv && t + j * tpr < nchunks, acc);
-}
 
 // Resident CTAs per SM the row-block kernel is compiled for (register budget:
 // the row's CPT chunks per thread stay in registers).

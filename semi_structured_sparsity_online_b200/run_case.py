@@ -8,8 +8,10 @@ Nsight Compute) or for a quick timing of one configuration:
 With --batch B the pass runs as one batched launch over B operands of that
 shape (a [B, m, k] tensor).
 
-Passes: tensor_scale, fused_24_{none,fp8,nvfp4,mxfp4,int8g128}, fused_48_nvfp4,
-dense_{fp8,nvfp4,mxfp4,int8_row,int8g128}, error_energy. Prints the mean CUDA-event
+Passes: tensor_scale, amax_rows (tensor scale and per-row amax),
+fused_24_{none,fp8,nvfp4,mxfp4,int8g128}, fused_48_nvfp4,
+dense_{fp8,nvfp4,mxfp4,int8_row,int8g128}, dense_int8_given_rows (one scale per
+row from a given row amax), error_energy. Prints the mean CUDA-event
 time per launch and the GB/s of the pass's algorithmic bytes.
 """
 from __future__ import annotations
@@ -42,6 +44,10 @@ def pass_bytes(name, m, k):
     n = m * k
     if name in ("tensor_scale", "error_energy"):
         return 2 * n
+    if name == "amax_rows":
+        return 2 * n + 4 * m
+    if name == "dense_int8_given_rows":
+        return 2 * n + 8 * m + n
     pattern, fmt, bits, group = PASSES[name]
     q = n // 2 if pattern != ss24.DENSE else n
     meta = n // 8 if pattern == ss24.SPARSE_24 else (n // 16 if pattern == ss24.SPARSE_48 else 0)
@@ -60,7 +66,8 @@ def pass_bytes(name, m, k):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--pass", dest="name", default="fused_24_fp8", choices=sorted(PASSES) + ["tensor_scale", "error_energy"])
+    ap.add_argument("--pass", dest="name", default="fused_24_fp8", choices=sorted(PASSES) + ["tensor_scale", "error_energy", "amax_rows",
+                                                                       "dense_int8_given_rows"])
     ap.add_argument("--m", type=int, default=4096)
     ap.add_argument("--k", type=int, default=4096)
     ap.add_argument("--iters", type=int, default=3)
@@ -88,8 +95,17 @@ def main():
         if fmt == "nvfp4":
             scale = ss24.tensor_scale(x, "nvfp4", pattern if pattern != ss24.DENSE else ss24.DENSE, ws=ws)
 
+    row_amax, _ = ss24.amax_rows(x, ws=ws)
+    if args.name == "dense_int8_given_rows":
+        out = ss24._alloc_outputs(args.m, args.k, ss24.DENSE, ss24.make_format("int", 8, 0), torch.bfloat16, "cuda",
+                                  lead)
+
     def once():
-        if args.name == "tensor_scale":
+        if args.name == "amax_rows":
+            ss24.amax_rows(x, scale_fmt="fp8", ws=ws, out=row_amax, scale_out=scale)
+        elif args.name == "dense_int8_given_rows":
+            ss24.run_int_rows(x, row_amax, bits=8, energy=e, ws=ws, out=out)
+        elif args.name == "tensor_scale":
             ss24.tensor_scale(x, "fp8", ss24.SPARSE_24, ws=ws, out=scale)
         elif args.name == "error_energy":
             ss24.error_energy(x, ss24.SPARSE_24, ("fp8",), ("int", 5, 128), sparse_scale=scale, dense_scale=None,

@@ -82,6 +82,9 @@ _SIGNATURES = {
     "ss24_bits_per_element": (ctypes.c_double, [Format, ctypes.c_int, ctypes.c_int64, ctypes.c_int32]),
     "ss24_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "ss24_selfcheck_division": (ctypes.c_int, [ctypes.c_int32, ctypes.c_uint32, ctypes.c_uint32, _P, _P]),
+    "ss24_amax_rows": (ctypes.c_int, [_OP, ctypes.c_int, ctypes.c_int, _P, _P, ctypes.c_int32, _P, _P, _S, _P]),
+    "ss24_quantize_int_rows": (ctypes.c_int, [_OP, ctypes.c_int, ctypes.c_int, _P, Format, _P, _OUT, _P, _P, _S,
+                                              _P]),
     "ss24_selfcheck_encoder": (ctypes.c_int, [ctypes.c_int32, _P, ctypes.c_int32, ctypes.c_uint32, ctypes.c_uint32,
                                               _P, _P]),
     "ss24_encode_e4m3": (ctypes.c_int, [_P, _P, ctypes.c_int64, _P]),
@@ -300,6 +303,46 @@ def tensor_scale(x, fmt="fp8", pattern=SPARSE_24, score="mag", col_norms=None, a
     _check(lib().ss24_tensor_scale(ctypes.byref(op), pattern, _SCORE[score] if isinstance(score, str) else score,
                                    _ptr(col_norms), _FMT[fmt] if isinstance(fmt, str) else fmt, _ptr(out), ws.ptr,
                                    ws.nbytes, _stream(stream)), "ss24_tensor_scale")
+    return out
+
+
+def amax_rows(x, pattern=DENSE, score="mag", col_norms=None, scale_fmt=None, ws=None, stream=None, out=None,
+              scale_out=None):
+    """Per-row amax of the values a pass with this pattern / score quantizes,
+    float32 [rows] (or [B, rows]) on the device, and, with scale_fmt ("fp8" or
+    "nvfp4"), the per-tensor scale from the same read: returns (rows, scale)."""
+    op = make_operand(x, 1)
+    lead = _lead(op)
+    shape = (op.rows,) if lead is None else (lead, op.rows)
+    out = out if out is not None else torch.empty(shape, dtype=torch.float32, device=x.device)
+    if scale_fmt is not None and scale_out is None:
+        scale_out = torch.empty(max(op.batch, 1), dtype=torch.float32, device=x.device)
+    kind = 0 if scale_fmt is None else (_FMT[scale_fmt] if isinstance(scale_fmt, str) else int(scale_fmt))
+    ws = ws or default_workspace(x.device)
+    _check(lib().ss24_amax_rows(ctypes.byref(op), pattern, _SCORE[score] if isinstance(score, str) else score,
+                                _ptr(col_norms), _ptr(out), kind, _ptr(scale_out), ws.ptr, ws.nbytes,
+                                _stream(stream)), "ss24_amax_rows")
+    return out, scale_out
+
+
+def run_int_rows(x, row_amax, pattern=DENSE, bits=8, pack4=False, score="mag", col_norms=None, energy=True,
+                 ws=None, stream=None, out=None):
+    """INT-b with one scale per row from a given per-row amax (ss24_quantize_int_rows);
+    returns the same dict as run()."""
+    f = make_format("int", bits, 0, pack4)
+    op = make_operand(x, 1)
+    if out is None:
+        out = _alloc_outputs(op.rows, op.k, pattern, f, x.dtype, x.device, _lead(op))
+    e = _energy(op, x.device) if energy is True else energy
+    if e is not None and e is not False:
+        out["energy"] = e
+    else:
+        e = None
+    ws = ws or default_workspace(x.device)
+    o = Outputs(*(_ptr(out.get(key)) for key in ("values", "scales", "tensor_scale", "meta")))
+    _check(lib().ss24_quantize_int_rows(ctypes.byref(op), pattern, _SCORE[score] if isinstance(score, str) else score,
+                                        _ptr(col_norms), f, _ptr(row_amax), ctypes.byref(o), _ptr(e), ws.ptr,
+                                        ws.nbytes, _stream(stream)), "ss24_quantize_int_rows")
     return out
 
 

@@ -178,6 +178,18 @@ def test_other_entry_points_validate():
     assert L.ss24_error_energy(ctypes.byref(o), ss24.SPARSE_24, ss24.MAG, None, ss24.make_format("none"),
                                ss24.make_format("int", 5), None, None, None, ALIGNED, wsb, None) == 1
     assert L.ss24_amax(ctypes.byref(o), ss24.SPARSE_24, ss24.MAG, None, None, ALIGNED, wsb, None) == 1
+    assert L.ss24_amax_rows(ctypes.byref(o), ss24.DENSE, ss24.MAG, None, None, 0, None, ALIGNED, wsb, None) == 1
+    assert L.ss24_amax_rows(ctypes.byref(o), ss24.DENSE, ss24.MAG, None, ALIGNED, 2, ALIGNED, ALIGNED, wsb,
+                            None) == 5                                        # INT has no tensor scale
+    assert L.ss24_amax_rows(ctypes.byref(op(axis=0)), ss24.DENSE, ss24.MAG, None, ALIGNED, 0, None, ALIGNED, wsb,
+                            None) == 8
+    assert L.ss24_quantize_int_rows(ctypes.byref(o), ss24.DENSE, ss24.MAG, None, ss24.make_format("int", 8, 32),
+                                    ALIGNED, ctypes.byref(out), None, ALIGNED, wsb, None) == 5   # group must be 0
+    assert L.ss24_quantize_int_rows(ctypes.byref(o), ss24.DENSE, ss24.MAG, None, ss24.make_format("int", 8, 0),
+                                    None, ctypes.byref(out), None, ALIGNED, wsb, None) == 1
+    assert L.ss24_quantize_int_rows(ctypes.byref(op(axis=0)), ss24.DENSE, ss24.MAG, None,
+                                    ss24.make_format("int", 8, 0), ALIGNED, ctypes.byref(out), None, ALIGNED, wsb,
+                                    None) == 8
     assert L.ss24_predicted_ratio(None, ALIGNED, ALIGNED, 1, None) == 1
     assert L.ss24_predicted_ratio(ALIGNED, ALIGNED, ALIGNED, -1, None) == 2
     assert L.ss24_selfcheck_division(3, 0, 1, ALIGNED, None) == 8

@@ -333,6 +333,60 @@ def test_int_one_scale_per_very_long_row(ss, ws, k):
     compare(ss, ws, xh, pattern=24, fmt="int", bits=4, group=0, pack4=True, score="wanda", norms=norms)
 
 
+ROWS_CASES = [("linear", 45, 4096), ("linear", 13, 1000), ("linear", 33, 96), ("gauss32", 9, 5120),
+              ("linear", 7, 14336)]
+
+
+@pytest.mark.parametrize("pattern,score", [(0, "mag"), (24, "mag"), (24, "wanda"), (48, "mag")])
+@pytest.mark.parametrize("case", ROWS_CASES)
+def test_row_amax_and_int_from_given_row_amax(ss, ws, pattern, score, case):
+    """ss24_amax_rows (per-row amax and the tensor scale in one read) and
+    ss24_quantize_int_rows (one scale per row from that amax) against the oracle."""
+    kind, rows, k = case
+    if pattern == 48 and k % 16:
+        pytest.skip("4:8 needs k % 16 == 0")
+    xh = synth.linear_input(rows, k, seed=12, n_outlier=min(8, k // 16))[0] if kind == "linear" \
+        else synth.gaussian_f32(rows, k, seed=13)
+    norms = synth.linear_weight(1, k, seed=14)[1] if score == "wanda" else None
+    opat = {0: oracle.DENSE, 24: oracle.SPARSE_24, 48: oracle.SPARSE_48}[pattern]
+    osc = oracle.WANDA if score == "wanda" else oracle.MAG
+    x, nd = to_dev(xh), (to_dev(norms) if norms is not None else None)
+    ra, sc = ss.amax_rows(x, pattern=pattern, score=score, col_norms=nd, scale_fmt="fp8", ws=ws)
+    torch.cuda.synchronize()
+    want = np.array([oracle.amax(np.ascontiguousarray(xh[r:r + 1]), pattern=opat, score=osc, norms=norms)
+                     for r in range(rows)], dtype=np.float32)
+    assert_same(to_np(ra), want, "row amax")
+    assert_same(to_np(sc), np.array([oracle.tensor_scale(xh, "fp8", pattern=opat, score=osc, norms=norms)],
+                                    dtype=np.float32), "tensor scale")
+    for bits, pack4 in ((8, False), (4, True)):
+        out = ss.run_int_rows(x, ra, pattern=pattern, bits=bits, pack4=pack4, score=score, col_norms=nd, ws=ws)
+        torch.cuda.synchronize()
+        ref = oracle.run(xh, pattern=opat, fmt="int", bits=bits, group=0, pack4=pack4, score=osc, norms=norms)
+        for key in ("values", "scales", "meta"):
+            if key in ref:
+                assert_same(to_np(out[key]), ref[key], key)
+        assert_energy(out["energy"], ref["energy"], atol=1e-30)
+    assert ws.error() == 0
+
+
+def test_row_amax_batch_and_empty(ss, ws):
+    xs = [synth.sweep_operand(40, 2048, seed=80 + b) for b in range(3)]
+    x = torch.stack([to_dev(v) for v in xs])
+    ra, _ = ss.amax_rows(x, ws=ws)
+    out = ss.run_int_rows(x, ra, bits=8, ws=ws)
+    torch.cuda.synchronize()
+    for b, xh in enumerate(xs):
+        ref = oracle.run(xh, pattern=oracle.DENSE, fmt="int", bits=8, group=0)
+        assert_same(to_np(out["values"][b]), ref["values"], "values")
+        assert_same(to_np(out["scales"][b]), ref["scales"], "scales")
+        assert_energy(out["energy"][b], ref["energy"], atol=1e-30)
+    empty = torch.zeros((0, 64), dtype=torch.bfloat16, device="cuda")
+    ra0, sc0 = ss.amax_rows(empty, scale_fmt="fp8", ws=ws)
+    torch.cuda.synchronize()
+    assert ra0.numel() == 0 and sc0.item() == 0.0
+    assert ws.error() == 0
+
+
 def test_int_one_scale_per_long_row(ss, ws):
     """Rows of several hundred chunks: the row-block kernel with 256 threads per row."""
     for pattern in (0, 24, 48):
