@@ -294,8 +294,7 @@ ss24_status ss24_tensor_scale(const ss24_operand *x, ss24_pattern pattern, ss24_
  * row_amax[b * rows + r] = max |value| over the values of row r of operand b
  * that a pass with this pattern and score quantizes (the kept values for a
  * sparse pattern). row_amax: device, batch x rows fp32, 4-byte aligned (NULL
- * allowed when rows is 0); the call clears it first (it is reduced by atomic
- * maxima). If scale_out is not
+ * allowed when rows is 0); every entry is written. If scale_out is not
  * NULL it also writes the per-tensor scale of kind (SS24_FMT_FP8_E4M3 or
  * SS24_FMT_NVFP4) as ss24_tensor_scale does. Axis 1 only (SS24_ERR_ARG
  * otherwise). */

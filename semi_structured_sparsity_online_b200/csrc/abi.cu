@@ -881,9 +881,14 @@ ss24_status ss24_amax_rows(const ss24_operand *x, ss24_pattern pattern, ss24_sco
     const size_t nb = static_cast<size_t>(nbatch(x));
     if (x->rows == 0)
         return scale_out ? cuda_status(cudaMemsetAsync(scale_out, 0, nb * sizeof(float), s)) : SS24_OK;
-    cudaError_t e = cudaMemsetAsync(row_amax, 0, nb * static_cast<size_t>(x->rows) * sizeof(float), s);
-    if (e != cudaSuccess)
-        return SS24_ERR_CUDA;
+    // full-width rows are each reduced by one warp and stored; other shapes
+    // reduce row segments with atomic maxima into a cleared array
+    const Geometry g = stream_geometry(x);
+    if (!(g.W == 256 && g.step_cols == 256)) {
+        cudaError_t e = cudaMemsetAsync(row_amax, 0, nb * static_cast<size_t>(x->rows) * sizeof(float), s);
+        if (e != cudaSuccess)
+            return SS24_ERR_CUDA;
+    }
     const float divisor = kind == SS24_FMT_FP8_E4M3 ? 448.0f : 2688.0f;
     return cuda_status(run_amax(x, pattern, score, col_norms, ws, s, scale_out, scale_out ? divisor : 1.0f, nullptr,
                                 row_amax));

@@ -1154,6 +1154,51 @@ template <typename T, int PAT, int FMT> struct FwStep {
     static constexpr int64_t meta = PAT == kSparse24 ? 32 : PAT == kSparse48 ? 16 : 0;
 };
 
+// The largest magnitude among a chunk's values a pass quantizes (all values
+// for the dense pattern, the kept ones otherwise).
+template <typename T, int PAT, int SCORE>
+__device__ __forceinline__ float quantized_amax(const typename Elem<T>::Raw &raw, const ChunkOut &o)
+{
+    if constexpr (PAT == kDense || SCORE == kMag) {
+        float xv[8];
+        Elem<T>::unpack(raw, xv);
+        return chunk_amax<T>(raw, xv);
+    } else {
+        return select_chunk<T, PAT, SCORE>(raw, o).vmax;
+    }
+}
+
+// A full-width unit of the amax pass, wholly inside the operand: the amax of
+// all values and of the kept values into acc, and the lane's largest
+// quantized magnitude returned (for the row amax).
+template <typename T, int PAT, int SCORE>
+__device__ __forceinline__ float amax_unit_fw(const T *xp, const ChunkOut &o, Acc &acc)
+{
+    typename Elem<T>::Raw raw[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        raw[i] = Stream<T>::load(xp + i * 256, true);
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float xv[8];
+        Elem<T>::unpack(raw[i], xv);
+        const float all = chunk_amax<T>(raw[i], xv);
+        acc.amax_all = fmaxf(acc.amax_all, all);
+        if constexpr (PAT == kDense) {
+            m = fmaxf(m, all);
+        } else {
+            ChunkOut oi = o;
+            if constexpr (SCORE == kWanda)
+                oi.norms = o.norms + i * 256;
+            const float kept = SCORE == kMag ? all : select_chunk<T, PAT, SCORE>(raw[i], oi).vmax;
+            acc.amax_kept = fmaxf(acc.amax_kept, kept);
+            m = fmaxf(m, kept);
+        }
+    }
+    return m;
+}
+
 // One unit: four 16-byte loads per lane first, then the four chunks. FULL:
 // every chunk of the unit lies inside the operand (no per-chunk checks).
 template <typename T, int PAT, int SCORE, int FMT, bool FULL>
@@ -1280,18 +1325,11 @@ __device__ __forceinline__ void stream_unit(const PassParams &p, const PassConst
                 // per-row amax of the values to quantize: reduced over the
                 // lanes sharing a row segment, then an atomic max (non-negative
                 // floats order like their bit patterns)
-                const int lcpr = p.log2_cpr, segl = 1 << lcpr;
+                const int segl = 1 << p.log2_cpr;
                 float cm[4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    if constexpr (PAT == kDense || SCORE == kMag) {
-                        float xv[8];
-                        Elem<T>::unpack(raw[i], xv);
-                        cm[i] = chunk_amax<T>(raw[i], xv);
-                    } else {
-                        cm[i] = select_chunk<T, PAT, SCORE>(raw[i], out_i(i)).vmax;
-                    }
-                }
+                for (int i = 0; i < 4; ++i)
+                    cm[i] = quantized_amax<T, PAT, SCORE>(raw[i], out_i(i));
                 if (p.step_rows == 0) {
                     // the four chunks share the lane's row
                     float m = fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3]));
@@ -1370,6 +1408,35 @@ __global__ void __launch_bounds__(kStreamThreads, (StreamOcc<T, PAT, SCORE, FMT,
     const int sa = tw / p.units_b, sb = tw - sa * p.units_b;
     double e_total = 0.0, e_prune = 0.0, e_q = 0.0, e_qd = 0.0;
     Acc acc{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if constexpr (FMT == kAmax && FW) {
+        if (rowa) {
+            // whole rows per warp (rows = units_a here): the row amax is the
+            // warp's own, stored without atomics; units wholly inside the
+            // operand take the fast path, the last partial quad the general one
+            for (int64_t row = u0; row < p.units_a; row += tw) {
+                float rm = 0.0f;
+                for (int b = 0; b < p.units_b; ++b) {
+                    const int64_t col0 = static_cast<int64_t>(b) * 1024 + lcol;
+                    const T *xp = x + row * p.ld + col0;
+                    const ChunkOut o = make_out<T, PAT, FMT>(p, ob, row, col0, true, lane);
+                    if (static_cast<int64_t>(b + 1) * 1024 <= p.k) {
+                        rm = fmaxf(rm, amax_unit_fw<T, PAT, SCORE>(xp, o, acc));
+                    } else {
+                        Acc a{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                        stream_unit<T, PAT, SCORE, FMT, false>(p, c, xp, step_x, step_c, o, dval, dscale, dmeta, row,
+                                                               col0, a);
+                        acc.amax_all = fmaxf(acc.amax_all, a.amax_all);
+                        acc.amax_kept = fmaxf(acc.amax_kept, a.amax_kept);
+                        rm = fmaxf(rm, PAT == kDense ? a.amax_all : a.amax_kept);
+                    }
+                }
+                rm = group_amax(rm, 32);
+                if (lane == 0)
+                    rowa[row] = rm;
+            }
+            ua = p.units_a; // skip the unit loop
+        }
+    }
     while (ua < p.units_a) {
         const int64_t row0 = static_cast<int64_t>(ua) * unit_rows + lrow;
         const int64_t col0 = static_cast<int64_t>(ub) * unit_cols + lcol;
