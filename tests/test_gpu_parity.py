@@ -455,6 +455,20 @@ def test_given_tensor_scale_and_saturation(ss, ws):
     compare(ss, ws, xh, pattern=0, fmt="nvfp4", tensor_scale=0.0)
 
 
+def test_fp8_given_scale_overflow_guard(ss, ws):
+    """Given FP8 scales tiny enough that v / s leaves the binary32 range for
+    part of the values: the per-chunk guard (a bf16 threshold for bf16 input)
+    must send exactly those chunks to IEEE division."""
+    rng = np.random.default_rng(21)
+    mag = np.exp2(rng.uniform(-10.0, 20.0, size=(40, 512))).astype(np.float32)
+    xf = (mag * rng.choice([-1.0, 1.0], size=mag.shape)).astype(np.float32)
+    xh = synth.bf16_bits(xf)
+    for s in (2.0 ** -120, 2.0 ** -108, 2.0 ** -100, 2.0 ** -61, 2.0 ** -59, 3.0, 5.0):
+        compare(ss, ws, xh, pattern=24, fmt="fp8", tensor_scale=s)
+        compare(ss, ws, xh, pattern=0, fmt="fp8", tensor_scale=s)
+    compare(ss, ws, xf, pattern=24, fmt="fp8", tensor_scale=2.0 ** -110)
+
+
 def test_int_with_tiny_and_subnormal_scales(ss, ws):
     """Groups whose amax is tiny give subnormal scales: the IEEE-division path
     and the clamp of the definition."""
