@@ -384,16 +384,13 @@ __device__ __forceinline__ void build_nv_table(float *t, float st, int tid)
     }
 }
 
-template <int VPC, bool STORE>
-__device__ __forceinline__ float quant_nvfp4(const float (&v)[VPC], float vmax, const Recip &rst,
-                                             const ChunkOut &o, const NvTable &tb, float gamax = -1.0f)
+// The E4M3 code of an NVFP4 block scale, E4M3((amax / 6) / st): two
+// correctly rounded divisions, by Markstein's correction when both are in its
+// exact range (zero amax included), else by IEEE division; one branch in the
+// common case.
+__device__ __forceinline__ uint32_t nv_block_code(float amax, const Recip &rst)
 {
-    constexpr int kLanes = 16 / VPC;
     const float st = rst.b;
-    const float amax = gamax >= 0.0f ? gamax : group_amax(vmax, kLanes);
-    // the block scale E4M3((amax / 6) / st): two correctly rounded divisions,
-    // by Markstein's correction when both are in its exact range (zero amax
-    // included), else by IEEE division; one branch in the common case
     Recip r6;
     r6.b = 6.0f;
     r6.nb = -6.0f;
@@ -407,11 +404,33 @@ __device__ __forceinline__ float quant_nvfp4(const float (&v)[VPC], float vmax, 
         a6 = __fdiv_rn(amax, 6.0f);
         bs = st != 0.0f ? __fdiv_rn(a6, st) : 0.0f;
     }
-    const uint32_t sb = cvt_e4m3x2(bs, 0.0f) & 0xffu;
+    return cvt_e4m3x2(bs, 0.0f) & 0xffu;
+}
+
+// A block's divisor and its reciprocal, when the caller computed them (the
+// block scale byte is then stored by the caller too).
+struct NvBlock {
+    float den, inv;
+};
+
+template <int VPC, bool STORE>
+__device__ __forceinline__ float quant_nvfp4(const float (&v)[VPC], float vmax, const Recip &rst,
+                                             const ChunkOut &o, const NvTable &tb, float gamax = -1.0f,
+                                             const NvBlock *blk = nullptr)
+{
+    constexpr int kLanes = 16 / VPC;
+    const float amax = gamax >= 0.0f ? gamax : group_amax(vmax, kLanes);
+    uint32_t sb = 0;
     Recip rd;
-    rd.b = tb.den[sb];
+    if (blk) {
+        rd.b = blk->den;
+        rd.y = blk->inv;
+    } else {
+        sb = nv_block_code(amax, rst);
+        rd.b = tb.den[sb];
+        rd.y = tb.inv[sb];
+    }
     rd.nb = -rd.b;
-    rd.y = tb.inv[sb];
     rd.fast = rd.b >= 0x1p-60f && rd.b <= 0x1p60f;
     const float denom = rd.b;
     float qn[VPC], d[VPC];
@@ -419,7 +438,7 @@ __device__ __forceinline__ float quant_nvfp4(const float (&v)[VPC], float vmax, 
     const uint32_t codes = pack_e2m1<VPC>(qn) ^ (VPC == 4 ? 0x8888u : 0x88888888u);
     unpack_e2m1<VPC>(codes, denom, d);
     store_fp4<VPC, STORE>(codes, o);
-    if (STORE && o.valid && (o.lane & (kLanes - 1)) == 0)
+    if (STORE && !blk && o.valid && (o.lane & (kLanes - 1)) == 0)
         *o.scale = static_cast<uint8_t>(sb);
     return err_energy<VPC>(v, d);
 }
@@ -653,7 +672,8 @@ template <typename T, int PAT, int SCORE, int FMT>
 __device__ __forceinline__ void finish_chunk(const PassParams &p, const typename Elem<T>::Raw &raw,
                                              const Sel<PAT == kDense ? 8 : 4> &sl, const ChunkOut &o,
                                              const PassConsts &c, Acc &acc, float row_amax = -1.0f,
-                                             const RowScale *rs = nullptr, float gamax = -1.0f)
+                                             const RowScale *rs = nullptr, float gamax = -1.0f,
+                                             const NvBlock *blk = nullptr)
 {
     constexpr int VPC = PAT == kDense ? 8 : 4;
     constexpr bool kPair = sizeof(T) == 2 && PAT == kSparse24 && SCORE == kMag;
@@ -705,7 +725,7 @@ __device__ __forceinline__ void finish_chunk(const PassParams &p, const typename
     } else if constexpr (FMT == kInt || FMT == kIntRows) {
         eq = quant_int<VPC, true>(v, vmax, p.q, o, row_amax, rs, gamax);
     } else if constexpr (FMT == kNvfp4) {
-        eq = quant_nvfp4<VPC, true>(v, vmax, c.rst, o, c.tb, gamax);
+        eq = quant_nvfp4<VPC, true>(v, vmax, c.rst, o, c.tb, gamax, blk);
     } else if constexpr (FMT == kMxfp4) {
         eq = quant_mxfp4<VPC, true>(v, vmax, o, gamax);
     } else if constexpr (FMT == kEnergy) {
@@ -1316,6 +1336,49 @@ __device__ __forceinline__ void stream_unit(const PassParams &p, const PassConst
 #pragma unroll
         for (int i = 0; i < 4; ++i)
             finish_chunk<T, PAT, SCORE, FMT>(p, raw[i], sl[i], out_i(i), c, acc, -1.0f, nullptr, g[i]);
+    } else if (FMT == kNvfp4 && PAT != kDense && p.step_rows == 0) {
+        // 2:4 / 4:8 + NVFP4: a unit holds 4 chunks x 8 blocks of 16 kept
+        // values = 32 blocks; lane L computes the scale of block L % 8 of
+        // chunk L / 8 once (instead of each chunk's lanes computing their
+        // block's) and stores its byte; the chunks' lanes fetch the divisor
+        // and its reciprocal. (Full-width units: one row per slot, so block
+        // j's scale byte is j - lane / 4 bytes from this lane's own.)
+        constexpr int VPC = PAT == kDense ? 8 : 4;
+        Sel<VPC> sl[4];
+        float g[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            sl[i] = select_chunk<T, PAT, SCORE>(raw[i], out_i(i));
+            g[i] = sl[i].vmax;
+        }
+#pragma unroll
+        for (int off = 1; off < 4; off <<= 1)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                g[i] = fmaxf(g[i], __shfl_xor_sync(kFull, g[i], off));
+        const int bs_ = lane >> 3, bj = lane & 7;
+        float t[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            t[i] = __shfl_sync(kFull, g[i], 4 * bj);
+        const float am = bs_ == 0 ? t[0] : bs_ == 1 ? t[1] : bs_ == 2 ? t[2] : t[3];
+        const uint32_t sb = nv_block_code(am, c.rst);
+        const float den = c.tb.den[sb], inv = c.tb.inv[sb];
+        {
+            // the block's scale byte: block bj of chunk bs_, 8 bytes per chunk slot
+            const ChunkOut ob_ = out_i(bs_);
+            const bool bvalid = FULL || col0 - 8 * lane + bs_ * step_c + 32 * bj < p.k;
+            if (bvalid && row0 + bs_ * p.step_rows < p.rows)
+                ob_.scale[bj - (lane >> 2)] = static_cast<uint8_t>(sb);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            NvBlock b;
+            const int src = 8 * i + (lane >> 2);
+            b.den = __shfl_sync(kFull, den, src);
+            b.inv = __shfl_sync(kFull, inv, src);
+            finish_chunk<T, PAT, SCORE, FMT>(p, raw[i], sl[i], out_i(i), c, acc, -1.0f, nullptr, g[i], &b);
+        }
     } else {
 #pragma unroll
         for (int i = 0; i < 4; ++i)

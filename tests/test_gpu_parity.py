@@ -171,6 +171,24 @@ def test_sparse_pass_bf16(ss, ws, pattern, score, fmt, bits, group, pack4):
     compare(ss, ws, xh, pattern=pattern, fmt=fmt, bits=bits, group=group, pack4=pack4, score=score, norms=norms)
 
 
+@pytest.mark.parametrize("k", [2048, 4608])
+@pytest.mark.parametrize("pattern", [24, 48])
+@pytest.mark.parametrize("score", ["mag", "wanda"])
+@pytest.mark.parametrize("fmt,bits,group,pack4", FORMATS)
+def test_sparse_pass_full_width(ss, ws, pattern, score, fmt, bits, group, pack4, k):
+    """k >= 1024: units of 1024 columns of one row (k = 4608: a ragged last unit)."""
+    xh = synth.sweep_operand(37, k, seed=6 + pattern)
+    norms = np.exp(np.random.default_rng(7).standard_normal(k)).astype(np.float32) if score == "wanda" else None
+    compare(ss, ws, xh, pattern=pattern, fmt=fmt, bits=bits, group=group, pack4=pack4, score=score, norms=norms)
+
+
+@pytest.mark.parametrize("k", [2048, 4608])
+@pytest.mark.parametrize("fmt,bits,group,pack4", [f for f in FORMATS if f[0] != "none"])
+def test_dense_pass_full_width(ss, ws, fmt, bits, group, pack4, k):
+    xh = synth.linear_input(29, k, seed=9, n_outlier=8)[0]
+    compare(ss, ws, xh, pattern=0, fmt=fmt, bits=bits, group=group, pack4=pack4)
+
+
 @pytest.mark.parametrize("fmt,bits,group,pack4", FORMATS)
 def test_sparse_pass_fp32(ss, ws, fmt, bits, group, pack4):
     xh = synth.gaussian_f32(37, 1024, seed=0)
