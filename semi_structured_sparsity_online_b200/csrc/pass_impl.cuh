@@ -1151,14 +1151,13 @@ template <> struct Stream<float> {
 };
 
 // Resident CTAs per SM the stream kernel is compiled for (register budget).
-// (Four CTAs where the kernel fits 64 registers without spilling, else three;
-// two for the energy pass.)
+// (Four CTAs where the kernel fits 64 registers without spilling, else three.)
 template <typename T, int PAT, int SCORE, int FMT, bool FW> struct StreamOcc {
     // (INT holds four selected chunks across its group reduction)
     static constexpr bool light =
         FMT == kAmax || (sizeof(T) == 2 && SCORE == kMag && PAT != kSparse48 &&
                          (FMT == kNone || FMT == kMxfp4 || (FMT == kFp8 && (FW || PAT == kDense))));
-    static constexpr int value = FMT == kEnergy ? 2 : light ? 4 : 3; // the energy pass: two formats live
+    static constexpr int value = light ? 4 : 3;
 };
 
 // Byte advance of each output between consecutive slots of a full-width unit
