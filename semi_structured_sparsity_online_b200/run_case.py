@@ -95,7 +95,7 @@ def main():
         if fmt == "nvfp4":
             scale = ss24.tensor_scale(x, "nvfp4", pattern if pattern != ss24.DENSE else ss24.DENSE, ws=ws)
 
-    row_amax, _ = ss24.amax_rows(x, ws=ws)
+    row_amax = ss24.amax_rows(x, ws=ws)[0] if args.name in ("amax_rows", "dense_int8_given_rows") else None
     if args.name == "dense_int8_given_rows":
         out = ss24._alloc_outputs(args.m, args.k, ss24.DENSE, ss24.make_format("int", 8, 0), torch.bfloat16, "cuda",
                                   lead)
