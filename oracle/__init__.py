@@ -61,6 +61,8 @@ def lib():
         _lib = ctypes.CDLL(build())
         _lib.oracle_run.restype = ctypes.c_int
         _lib.oracle_run.argtypes = [ctypes.POINTER(_Args), ctypes.POINTER(_Outputs), ctypes.c_void_p]
+        _lib.oracle_dequantize.restype = ctypes.c_int
+        _lib.oracle_dequantize.argtypes = [ctypes.POINTER(_Args), ctypes.POINTER(_Outputs), ctypes.c_void_p]
         _lib.oracle_amax.restype = ctypes.c_float
         _lib.oracle_amax.argtypes = [ctypes.POINTER(_Args)]
         _lib.oracle_tensor_scale.restype = ctypes.c_float
@@ -152,6 +154,22 @@ def run(x, *, pattern=SPARSE_24, score=MAG, norms=None, fmt="none", bits=8, grou
         raise ValueError(f"oracle_run rejected its arguments (code {rc})")
     out["energy"] = energy
     return out
+
+
+def dequantize(out, *, rows, k, pattern=SPARSE_24, fmt="none", bits=8, group=0, pack4=False, dtype=BF16):
+    """The dense float32 operand [rows][k] that the outputs of a pass (a dict as
+    run() returns it) stand for: dequantized values on kept positions, zero on
+    dropped ones."""
+    fmt_id = _FMT_NAMES[fmt] if isinstance(fmt, str) else fmt
+    dummy = np.zeros(1, dtype=np.uint16 if dtype == BF16 else np.float32)
+    args = _make_args(dummy, dtype, rows, k, k, 1, pattern, MAG, None, fmt_id, bits, group, int(pack4), None)
+    keep = {key: np.ascontiguousarray(out[key]) for key in ("values", "scales", "tensor_scale", "meta") if key in out}
+    outs = _Outputs(_ptr(keep.get("values")), _ptr(keep.get("scales")), _ptr(keep.get("tensor_scale")),
+                    _ptr(keep.get("meta")))
+    xhat = np.zeros((rows, k), dtype=np.float32)
+    if lib().oracle_dequantize(ctypes.byref(args), ctypes.byref(outs), xhat.ctypes.data) != 0:
+        raise ValueError("oracle_dequantize rejected its arguments")
+    return xhat
 
 
 def amax(x, *, pattern=SPARSE_24, score=MAG, norms=None, axis=1, rows=None, k=None, ld=None):

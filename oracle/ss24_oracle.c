@@ -656,3 +656,91 @@ float oracle_tensor_scale(const oracle_args *a)
     float amax = oracle_amax(a);
     return a->fmt == OR_FMT_FP8 ? amax / 448.0f : amax / 2688.0f;
 }
+
+/* ------------------------------------------------------------------------- */
+/* Dequantization: the stored outputs back to a dense operand                 */
+/* ------------------------------------------------------------------------- */
+
+/* The dequantized value of entry j of quantized row r, from the stored codes
+ * and scales, formed exactly as the pass forms it (decode(code) * scale, one
+ * binary32 product); format NONE returns the kept value itself. */
+static float dequant_entry(const oracle_args *a, const oracle_outputs *o, int64_t r, int64_t n, int64_t j)
+{
+    switch (a->fmt) {
+    case OR_FMT_NONE:
+        if (a->dtype == OR_BF16)
+            return oracle_bf16_to_f32(((const uint16_t *)o->values)[r * n + j]);
+        return ((const float *)o->values)[r * n + j];
+    case OR_FMT_FP8:
+        return oracle_e4m3_decode(((const uint8_t *)o->values)[r * n + j]) * o->tensor_scale[0];
+    case OR_FMT_INT: {
+        int64_t g = a->group ? a->group : n;
+        int code;
+        if (a->pack4) {
+            int nib = (((const uint8_t *)o->values)[(r * n + j) / 2] >> (4 * ((r * n + j) % 2))) & 0xF;
+            code = nib >= 8 ? nib - 16 : nib; /* two's-complement nibble */
+        } else if (a->bits > 8) {
+            code = ((const int16_t *)o->values)[r * n + j];
+        } else {
+            code = ((const int8_t *)o->values)[r * n + j];
+        }
+        return (float)code * ((const float *)o->scales)[r * (n / g) + j / g];
+    }
+    case OR_FMT_NVFP4: {
+        uint8_t sb = ((const uint8_t *)o->scales)[r * (n / 16) + j / 16];
+        float denom = oracle_e4m3_decode(sb) * o->tensor_scale[0];
+        uint8_t code = (((const uint8_t *)o->values)[(r * n + j) / 2] >> (4 * ((r * n + j) % 2))) & 0xF;
+        return oracle_e2m1_decode(code) * denom;
+    }
+    default: { /* OR_FMT_MXFP4 */
+        uint8_t byte = ((const uint8_t *)o->scales)[r * (n / 32) + j / 32];
+        float scale = ldexpf(1.0f, (int)byte - 127);
+        uint8_t code = (((const uint8_t *)o->values)[(r * n + j) / 2] >> (4 * ((r * n + j) % 2))) & 0xF;
+        return oracle_e2m1_decode(code) * scale;
+    }
+    }
+}
+
+/* The dense operand the stored outputs stand for (§4: the 2:4 error of an
+ * element is x - x_hat, with x_hat the dequantized value on kept positions and
+ * 0 on dropped ones): xhat[r * k + c] for the operand's rows and columns (row
+ * major, axis-1 layout). Sparse patterns place the quantized row's entries at
+ * the positions the metadata records (2:4: nibble i0 | i1 << 2 per group of 4,
+ * two groups per byte, even group low; 4:8: nibble p0 | p1 << 2 per 8, the
+ * pairs 2p, 2p + 1). Returns 0, or -1 for arguments it does not support. */
+int oracle_dequantize(const oracle_args *a, const oracle_outputs *o, float *xhat)
+{
+    if (!a || !o || !xhat || a->rows < 0 || a->k <= 0)
+        return -1;
+    int sparse = a->pattern != OR_DENSE;
+    int64_t k = a->k, n = sparse ? k / 2 : k;
+    for (int64_t r = 0; r < a->rows; ++r) {
+        float *row = xhat + r * k;
+        for (int64_t c = 0; c < k; ++c)
+            row[c] = 0.0f;
+        if (!sparse) {
+            for (int64_t c = 0; c < k; ++c)
+                row[c] = dequant_entry(a, o, r, n, c);
+            continue;
+        }
+        int gsize = a->pattern == OR_SPARSE_48 ? 8 : 4;
+        int64_t mrow = k / (2 * gsize); /* metadata bytes per row */
+        for (int64_t gi = 0; gi < k / gsize; ++gi) {
+            uint8_t byte = o->meta[r * mrow + gi / 2];
+            int nib = (gi % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+            int64_t j = gi * 2 * (gsize / 4); /* first quantized entry of the group */
+            int64_t c0 = gi * gsize;
+            if (gsize == 4) {
+                row[c0 + (nib & 3)] = dequant_entry(a, o, r, n, j);
+                row[c0 + (nib >> 2)] = dequant_entry(a, o, r, n, j + 1);
+            } else {
+                int p0 = nib & 3, p1 = nib >> 2;
+                row[c0 + 2 * p0] = dequant_entry(a, o, r, n, j);
+                row[c0 + 2 * p0 + 1] = dequant_entry(a, o, r, n, j + 1);
+                row[c0 + 2 * p1] = dequant_entry(a, o, r, n, j + 2);
+                row[c0 + 2 * p1 + 1] = dequant_entry(a, o, r, n, j + 3);
+            }
+        }
+    }
+    return 0;
+}

@@ -515,3 +515,33 @@ def test_encoder_step_tables_are_round_to_nearest_even_midpoints():
             mbits = int(np.array([mid], dtype=np.float32).view(np.uint32)[0])
             want = mbits if (i + 1) % 2 == 0 else mbits + 1         # tie goes to the even code
             assert int(bounds[i]) == want, (n, i)
+
+
+DEQ_FORMATS = [("none", 8, 0, False), ("fp8", 8, 0, False), ("int", 8, 16, False), ("int", 4, 0, True),
+               ("int", 12, 32, False), ("nvfp4", 4, 0, False), ("mxfp4", 4, 0, False)]
+
+
+@pytest.mark.parametrize("pattern", [oracle.DENSE, oracle.SPARSE_24, oracle.SPARSE_48])
+@pytest.mark.parametrize("fmt,bits,group,pack4", DEQ_FORMATS)
+def test_dequantize_reproduces_the_error_energies(pattern, fmt, bits, group, pack4):
+    """x_hat from the stored outputs: sum (x - x_hat)^2 is E_prune + E_q (sparse)
+    or E_q,dense (dense), the energies the pass accumulated element by element
+    (§4: the two errors land on disjoint elements). A wrong position, code,
+    scale or product shows up as a different sum."""
+    if fmt == "none" and pattern == oracle.DENSE:
+        pytest.skip("format NONE is the plain 2:4 compression")
+    xh = synth.linear_input(24, 256, seed=31, n_outlier=4)[0]
+    out = oracle.run(xh, pattern=pattern, fmt=fmt, bits=bits, group=group, pack4=pack4)
+    xhat = oracle.dequantize(out, rows=24, k=256, pattern=pattern, fmt=fmt, bits=bits, group=group, pack4=pack4)
+    x = synth.bf16_to_f32(xh).astype(np.float64)
+    err = float(np.sum((x - xhat.astype(np.float64)) ** 2))
+    e = out["energy"]
+    want = e[3] if pattern == oracle.DENSE else e[1] + e[2]
+    assert abs(err - want) <= 1e-12 * want
+    if pattern != oracle.DENSE:
+        per_group = 4 if pattern == oracle.SPARSE_24 else 8
+        nz = (xhat.reshape(24, -1, per_group) != 0).sum(axis=2)
+        assert nz.max() <= per_group // 2      # at most the kept half of each group is non-zero
+    if fmt == "none":
+        kept = xhat != 0
+        assert np.array_equal(xhat[kept], x[kept].astype(np.float32))
