@@ -380,6 +380,23 @@ ss24_status ss24_encode_e2m1(const float *in, uint8_t *out, int64_t n, ss24_stre
 /* Decode n E2M1 codes (low nibble of each byte) to binary32. */
 ss24_status ss24_decode_e2m1(const uint8_t *in, float *out, int64_t n, ss24_stream stream);
 
+/* ---- dequantization ------------------------------------------------------ */
+
+/* The dense operand the outputs of a pass stand for (§4: the 2:4 error of an
+ * element is x - x_hat, x_hat being the dequantized value on kept positions
+ * and 0 on dropped ones). Writes xhat[b][r][c] (fp32, row major, batch x rows x
+ * k, 16-byte aligned) from the outputs `in` that a pass with this pattern and
+ * format wrote for an operand of x's shape (x->rows, x->k, x->batch; x->dtype
+ * is the type of the kept values for SS24_FMT_NONE; x->x and the strides are
+ * not read). Dequantized values are decode(code) * scale rounded once, the
+ * products the pass forms, so sum (x - xhat)^2 reproduces the pass's
+ * E_prune + E_quant (sparse) or E_quant_dense (dense). Layouts: those the
+ * pass writes (see ss24_outputs), the operands of a batch packed one after the
+ * other. Errors: SS24_ERR_NULL for a missing buffer the format needs, and the
+ * shape / format checks of the passes. */
+ss24_status ss24_dequantize(const ss24_operand *x, ss24_pattern pattern, ss24_format fmt, const ss24_outputs *in,
+                            float *xhat, ss24_stream stream);
+
 /* ---- self-check of the kernels' division -------------------------------- */
 
 /* The kernels divide by a scale with Markstein's one-step correction of a

@@ -938,6 +938,43 @@ ss24_status ss24_tensor_scale(const ss24_operand *x, ss24_pattern pattern, ss24_
     return cuda_status(run_amax(x, pattern, score, col_norms, ws, s, scale_out, divisor));
 }
 
+ss24_status ss24_dequantize(const ss24_operand *x, ss24_pattern pattern, ss24_format fmt, const ss24_outputs *in,
+                            float *xhat, ss24_stream stream)
+{
+    if (!x || !in)
+        return SS24_ERR_NULL;
+    if (x->dtype != SS24_BF16 && x->dtype != SS24_F32)
+        return SS24_ERR_DTYPE;
+    if (x->rows < 0 || x->k <= 0 || x->rows > INT32_MAX || x->k > INT32_MAX)
+        return SS24_ERR_SHAPE;
+    if (x->batch < 0 || x->batch > kMaxGrid)
+        return SS24_ERR_SHAPE;
+    ss24_status st = check_pattern_k(pattern, x->k);
+    if (st != SS24_OK)
+        return st;
+    Resolved r;
+    if ((st = resolve_format(fmt, pattern, x->k, true, &r)) != SS24_OK)
+        return st;
+    if (x->rows == 0)
+        return SS24_OK;
+    const bool needs_scales = fmt.kind == SS24_FMT_INT || fmt.kind == SS24_FMT_NVFP4 || fmt.kind == SS24_FMT_MXFP4;
+    if (!in->values || !xhat || (needs_scales && !in->scales) || (per_tensor(fmt.kind) && !in->tensor_scale) ||
+        (pattern != SS24_DENSE && !in->meta))
+        return SS24_ERR_NULL;
+    if (!aligned16(xhat) || !aligned16(in->values))
+        return SS24_ERR_ALIGN;
+    // the outputs of a batch are packed operand after operand (as the pass writes them)
+    PassParams strides{};
+    output_strides(x, pattern, fmt, &strides);
+    int32_t lg = -1; // INT: log2 of the group of quantized values; one scale per row: -1
+    if (fmt.kind == SS24_FMT_INT && fmt.group != 0)
+        lg = ilog2(fmt.group);
+    return cuda_status(launch_dequant(pattern, fmt.kind, r.q.store, lg, x->dtype == SS24_F32 ? 1 : 0, x->rows, x->k,
+                                      static_cast<int32_t>(nbatch(x)), in->values, in->scales, in->tensor_scale,
+                                      in->meta, xhat, strides.values_bstride, strides.scales_bstride,
+                                      strides.meta_bstride, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 ss24_status ss24_predicted_ratio(const ss24_energy *sparse_side, const ss24_energy *dense_side, ss24_ratio *out,
                                  int64_t count, ss24_stream stream)
 {

@@ -73,6 +73,8 @@ def main():
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--seed", type=int, default=8)
     ap.add_argument("--batch", type=int, default=0, help="0: one 2-D operand; B: one launch over B operands")
+    ap.add_argument("--dequant", action="store_true",
+                    help="time the reconstruction of the pass's outputs (ss24_dequantize) instead of the pass")
     ap.add_argument("--derive-scale", action="store_true",
                     help="FP8 / NVFP4: let the pass compute its tensor scale (an amax launch precedes it)")
     args = ap.parse_args()
@@ -117,6 +119,19 @@ def main():
 
     once()
     torch.cuda.synchronize()
+    gb = nb * pass_bytes(args.name, args.m, args.k)
+    if args.dequant:
+        pattern, fmt, bits, group = PASSES[args.name]
+        xhat = torch.empty(x.shape, dtype=torch.float32, device="cuda")
+        # reads the stored outputs, writes fp32 x_hat: the pass's bytes less its input, plus 4 per element
+        gb = gb - nb * 2 * args.m * args.k + nb * 4 * args.m * args.k
+
+        def once():
+            ss24.dequantize(out, args.m, args.k, pattern=pattern, fmt=fmt, bits=bits, group=group, batch=lead,
+                            xhat=xhat)
+
+        once()
+        torch.cuda.synchronize()
     s, t = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     s.record()
     for _ in range(args.iters):
@@ -124,9 +139,8 @@ def main():
     t.record()
     t.synchronize()
     us = s.elapsed_time(t) / args.iters * 1e3
-    gb = nb * pass_bytes(args.name, args.m, args.k)
     assert ws.error() == 0
-    print(f"{args.name} m={args.m} k={args.k} batch={args.batch}: {us:.2f} us/launch, {gb / us / 1e3:.1f} GB/s "
+    print(f"{args.name}{' dequant' if args.dequant else ''} m={args.m} k={args.k} batch={args.batch}: {us:.2f} us/launch, {gb / us / 1e3:.1f} GB/s "
           f"({gb} algorithmic bytes per launch; warm L2 between launches)")
 
 

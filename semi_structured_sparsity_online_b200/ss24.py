@@ -85,6 +85,7 @@ _SIGNATURES = {
     "ss24_amax_rows": (ctypes.c_int, [_OP, ctypes.c_int, ctypes.c_int, _P, _P, ctypes.c_int32, _P, _P, _S, _P]),
     "ss24_quantize_int_rows": (ctypes.c_int, [_OP, ctypes.c_int, ctypes.c_int, _P, Format, _P, _OUT, _P, _P, _S,
                                               _P]),
+    "ss24_dequantize": (ctypes.c_int, [_OP, ctypes.c_int, Format, _OUT, _P, _P]),
     "ss24_selfcheck_encoder": (ctypes.c_int, [ctypes.c_int32, _P, ctypes.c_int32, ctypes.c_uint32, ctypes.c_uint32,
                                               _P, _P]),
     "ss24_encode_e4m3": (ctypes.c_int, [_P, _P, ctypes.c_int64, _P]),
@@ -344,6 +345,22 @@ def run_int_rows(x, row_amax, pattern=DENSE, bits=8, pack4=False, score="mag", c
                                         _ptr(col_norms), f, _ptr(row_amax), ctypes.byref(o), _ptr(e), ws.ptr,
                                         ws.nbytes, _stream(stream)), "ss24_quantize_int_rows")
     return out
+
+
+def dequantize(out, rows, k, pattern=SPARSE_24, fmt="none", bits=8, group=0, pack4=False, dtype=torch.bfloat16,
+               batch=None, stream=None, xhat=None):
+    """The dense float32 operand [rows, k] (or [B, rows, k]) that the outputs of a
+    pass (the dict run() returns) stand for: dequantized values on kept
+    positions, zero on dropped ones."""
+    f = make_format(fmt, bits, group, pack4)
+    dev = out["values"].device
+    op = Operand(None, BF16 if dtype == torch.bfloat16 else F32, 1, rows, k, k, batch or 0, 0)
+    shape = (rows, k) if batch is None else (batch, rows, k)
+    xhat = xhat if xhat is not None else torch.empty(shape, dtype=torch.float32, device=dev)
+    o = Outputs(*(_ptr(out.get(key)) for key in ("values", "scales", "tensor_scale", "meta")))
+    _check(lib().ss24_dequantize(ctypes.byref(op), pattern, f, ctypes.byref(o), _ptr(xhat), _stream(stream)),
+           "ss24_dequantize")
+    return xhat
 
 
 def predicted_ratio(sparse_energy, dense_energy, out=None, stream=None):

@@ -405,6 +405,72 @@ def test_row_amax_batch_and_empty(ss, ws):
     assert ws.error() == 0
 
 
+DEQ_FORMATS = [("none", 8, 0, False), ("fp8", 8, 0, False), ("int", 8, 64, False), ("int", 4, 0, True),
+               ("int", 12, 32, False), ("int", 5, 0, False), ("nvfp4", 4, 0, False), ("mxfp4", 4, 0, False)]
+
+
+@pytest.mark.parametrize("pattern", [0, 24, 48])
+@pytest.mark.parametrize("fmt,bits,group,pack4", DEQ_FORMATS)
+@pytest.mark.parametrize("shape", [(37, 512), (9, 2048)])
+def test_dequantize_matches_oracle(ss, ws, pattern, fmt, bits, group, pack4, shape):
+    """ss24_dequantize of the pass's own outputs against the oracle's
+    reconstruction, bit for bit (fp32 and bf16 kept values for format NONE)."""
+    if fmt == "none" and pattern == 0:
+        pytest.skip("format NONE is the plain 2:4 compression")
+    rows, k = shape
+    opat = {0: oracle.DENSE, 24: oracle.SPARSE_24, 48: oracle.SPARSE_48}[pattern]
+    for xh in ((synth.sweep_operand(rows, k, seed=40),) if fmt != "none"
+               else (synth.sweep_operand(rows, k, seed=40), synth.gaussian_f32(rows, k, seed=41))):
+        out, ref = compare(ss, ws, xh, pattern=pattern, fmt=fmt, bits=bits, group=group, pack4=pack4)
+        dt = torch.bfloat16 if xh.dtype == np.uint16 else torch.float32
+        got = ss.dequantize(out, rows, k, pattern=pattern, fmt=fmt, bits=bits, group=group, pack4=pack4, dtype=dt)
+        torch.cuda.synchronize()
+        want = oracle.dequantize(ref, rows=rows, k=k, pattern=opat, fmt=fmt, bits=bits, group=group, pack4=pack4,
+                                 dtype=oracle.BF16 if xh.dtype == np.uint16 else oracle.F32)
+        assert_same(to_np(got), want, "x_hat")
+
+
+def test_dequantize_batch(ss, ws):
+    xs = [synth.sweep_operand(20, 1024, seed=90 + b) for b in range(3)]
+    x = torch.stack([to_dev(v) for v in xs])
+    out = ss.run(x, pattern=24, fmt="nvfp4", ws=ws)
+    got = ss.dequantize(out, 20, 1024, pattern=24, fmt="nvfp4", batch=3)
+    torch.cuda.synchronize()
+    for b, xh in enumerate(xs):
+        ref = oracle.run(xh, pattern=oracle.SPARSE_24, fmt="nvfp4")
+        want = oracle.dequantize(ref, rows=20, k=1024, pattern=oracle.SPARSE_24, fmt="nvfp4")
+        assert_same(to_np(got[b]), want, "x_hat")
+
+
+@pytest.mark.parametrize("sparse,dense", [(("fp8",), ("int", 5, 128)), (("nvfp4",), ("mxfp4",)),
+                                          (("int", 8, 0), ("int", 5, 0))])
+def test_measured_ratio_against_oracle_and_prediction(ss, ws, sparse, dense):
+    """Operator-level R (errors of X_hat W^T): the GPU value against the same
+    quantity built from the oracle's outputs in fp64, and against R_hat, which
+    it matches in expectation for a weight with i.i.d. entries."""
+    from semi_structured_sparsity_online_b200 import operator_error
+    xh = synth.linear_input(256, 1024, seed=51, n_outlier=8)[0]
+    wf = synth.gaussian_f32(512, 1024, seed=52)
+    got = operator_error.measured_ratio(to_dev(xh), torch.from_numpy(wf).cuda(), sparse=sparse, dense=dense, ws=ws)
+
+    def side(pattern, spec):
+        fmt, bits, group = (spec + (8, 0))[:3]
+        ref = oracle.run(xh, pattern=pattern, fmt=fmt, bits=bits, group=group)
+        xhat = oracle.dequantize(ref, rows=256, k=1024, pattern=pattern, fmt=fmt, bits=bits, group=group)
+        return xhat.astype(np.float64), ref["energy"]
+
+    x = synth.bf16_to_f32(xh).astype(np.float64)
+    y = x @ wf.astype(np.float64).T
+    xs, es = side(oracle.SPARSE_24, sparse)
+    xd, ed = side(oracle.DENSE, dense)
+    err_s = np.linalg.norm((xs - x) @ wf.astype(np.float64).T) / np.linalg.norm(y)
+    err_d = np.linalg.norm((xd - x) @ wf.astype(np.float64).T) / np.linalg.norm(y)
+    assert abs(got["err_sparse"] / err_s - 1) < 1e-3 and abs(got["err_dense"] / err_d - 1) < 1e-3
+    r_hat = oracle.ratio(es, ed)[3]
+    assert abs(got["r_predicted"] / r_hat - 1) < 1e-6
+    assert abs(got["r_measured"] / got["r_predicted"] - 1) < 0.1
+
+
 def test_int_one_scale_per_long_row(ss, ws):
     """Rows of several hundred chunks: the row-block kernel with 256 threads per row."""
     for pattern in (0, 24, 48):
