@@ -963,16 +963,14 @@ ss24_status ss24_dequantize(const ss24_operand *x, ss24_pattern pattern, ss24_fo
         return SS24_ERR_NULL;
     if (!aligned16(xhat) || !aligned16(in->values))
         return SS24_ERR_ALIGN;
-    // the outputs of a batch are packed operand after operand (as the pass writes them)
-    PassParams strides{};
-    output_strides(x, pattern, fmt, &strides);
+    // the outputs of a batch are packed operand after operand, each the exact size
+    // of one operand's outputs (as the pass writes them)
     int32_t lg = -1; // INT: log2 of the group of quantized values; one scale per row: -1
     if (fmt.kind == SS24_FMT_INT && fmt.group != 0)
         lg = ilog2(fmt.group);
     return cuda_status(launch_dequant(pattern, fmt.kind, r.q.store, lg, x->dtype == SS24_F32 ? 1 : 0, x->rows, x->k,
                                       static_cast<int32_t>(nbatch(x)), in->values, in->scales, in->tensor_scale,
-                                      in->meta, xhat, strides.values_bstride, strides.scales_bstride,
-                                      strides.meta_bstride, reinterpret_cast<cudaStream_t>(stream)));
+                                      in->meta, xhat, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 ss24_status ss24_predicted_ratio(const ss24_energy *sparse_side, const ss24_energy *dense_side, ss24_ratio *out,

@@ -210,13 +210,14 @@ __device__ __forceinline__ uint32_t cvt_e2m1x4(float v0, float v1, float v2, flo
 __device__ __forceinline__ float2 e2m1x2_to_f32(uint32_t byte)
 {
     uint32_t h2;
+    const uint16_t h = static_cast<uint16_t>(byte & 0xffu);
     asm("{\n"
-        " .reg .b8 b0, b1, b2, b3;\n"
-        " mov.b32 {b0, b1, b2, b3}, %1;\n"
-        " cvt.rn.f16x2.e2m1x2 %0, b0;\n"
+        " .reg .b8 lo, hi;\n"
+        " mov.b16 {lo, hi}, %1;\n"
+        " cvt.rn.f16x2.e2m1x2 %0, lo;\n"
         "}\n"
         : "=r"(h2)
-        : "r"(byte));
+        : "h"(h));
     return f16x2_to_f32(h2); // .x from the low nibble
 }
 

@@ -123,8 +123,7 @@ cudaError_t launch_selfcheck_division(int mode, uint32_t b_first, uint32_t b_cou
 cudaError_t launch_convert(int op, const void *in, void *out, int64_t n, cudaStream_t stream);
 cudaError_t launch_dequant(int pattern, int fmt, int32_t store, int32_t lg, int32_t none_f32, int64_t rows,
                            int64_t k, int32_t batch, const void *values, const void *scales, const float *tscale,
-                           const uint8_t *meta, float *xhat, int64_t values_bstride, int64_t scales_bstride,
-                           int64_t meta_bstride, cudaStream_t stream);
+                           const uint8_t *meta, float *xhat, cudaStream_t stream);
 cudaError_t launch_selfcheck_encoder(int e2m1, const uint32_t *bounds, int n_bounds, uint32_t hi_first,
                                      uint32_t hi_count, unsigned long long *result, cudaStream_t stream);
 

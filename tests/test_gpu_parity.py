@@ -411,7 +411,7 @@ DEQ_FORMATS = [("none", 8, 0, False), ("fp8", 8, 0, False), ("int", 8, 64, False
 
 @pytest.mark.parametrize("pattern", [0, 24, 48])
 @pytest.mark.parametrize("fmt,bits,group,pack4", DEQ_FORMATS)
-@pytest.mark.parametrize("shape", [(37, 512), (9, 2048)])
+@pytest.mark.parametrize("shape", [(37, 512), (9, 2048), (13, 1536)])
 def test_dequantize_matches_oracle(ss, ws, pattern, fmt, bits, group, pack4, shape):
     """ss24_dequantize of the pass's own outputs against the oracle's
     reconstruction, bit for bit (fp32 and bf16 kept values for format NONE)."""
@@ -430,16 +430,28 @@ def test_dequantize_matches_oracle(ss, ws, pattern, fmt, bits, group, pack4, sha
         assert_same(to_np(got), want, "x_hat")
 
 
-def test_dequantize_batch(ss, ws):
-    xs = [synth.sweep_operand(20, 1024, seed=90 + b) for b in range(3)]
+@pytest.mark.parametrize("pattern", [0, 24, 48])
+@pytest.mark.parametrize("fmt,bits,group,pack4", [("fp8", 8, 0, False), ("nvfp4", 4, 0, False),
+                                                  ("int", 8, 0, False), ("int", 4, 0, True), ("mxfp4", 4, 0, False)])
+@pytest.mark.parametrize("rows,k,batch", [(20, 1024, 3), (3, 64, 7), (1, 8, 5)])
+def test_dequantize_batch(ss, ws, pattern, fmt, bits, group, pack4, rows, k, batch):
+    """Batches: one tensor scale per operand (FP8, NVFP4) and one INT scale per
+    row, including operands much smaller than the kernel's unit of work."""
+    if k % 16 and pattern == 48:
+        pytest.skip("4:8 needs k % 16 == 0")
+    n = k // 2 if pattern else k
+    if (fmt == "nvfp4" and n % 16) or (fmt == "mxfp4" and n % 32):
+        pytest.skip("block longer than the row")
+    opat = {0: oracle.DENSE, 24: oracle.SPARSE_24, 48: oracle.SPARSE_48}[pattern]
+    xs = [synth.sweep_operand(rows, k, seed=90 + b) for b in range(batch)]
     x = torch.stack([to_dev(v) for v in xs])
-    out = ss.run(x, pattern=24, fmt="nvfp4", ws=ws)
-    got = ss.dequantize(out, 20, 1024, pattern=24, fmt="nvfp4", batch=3)
+    out = ss.run(x, pattern=pattern, fmt=fmt, bits=bits, group=group, pack4=pack4, ws=ws)
+    got = ss.dequantize(out, rows, k, pattern=pattern, fmt=fmt, bits=bits, group=group, pack4=pack4, batch=batch)
     torch.cuda.synchronize()
     for b, xh in enumerate(xs):
-        ref = oracle.run(xh, pattern=oracle.SPARSE_24, fmt="nvfp4")
-        want = oracle.dequantize(ref, rows=20, k=1024, pattern=oracle.SPARSE_24, fmt="nvfp4")
-        assert_same(to_np(got[b]), want, "x_hat")
+        ref = oracle.run(xh, pattern=opat, fmt=fmt, bits=bits, group=group, pack4=pack4)
+        want = oracle.dequantize(ref, rows=rows, k=k, pattern=opat, fmt=fmt, bits=bits, group=group, pack4=pack4)
+        assert_same(to_np(got[b]), want, f"x_hat[{b}]")
 
 
 @pytest.mark.parametrize("sparse,dense", [(("fp8",), ("int", 5, 128)), (("nvfp4",), ("mxfp4",)),
