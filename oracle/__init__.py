@@ -64,6 +64,11 @@ def lib():
         _lib.oracle_dequantize.restype = ctypes.c_int
         _lib.oracle_dequantize.argtypes = [ctypes.POINTER(_Args), ctypes.POINTER(_Outputs), ctypes.c_void_p]
         _lib.oracle_amax.restype = ctypes.c_float
+        _lib.oracle_scale_tiles_bytes.restype = ctypes.c_int64
+        _lib.oracle_scale_tiles_bytes.argtypes = [ctypes.c_int64, ctypes.c_int64]
+        _lib.oracle_scale_tiles.restype = ctypes.c_int
+        _lib.oracle_scale_tiles.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                            ctypes.c_void_p]
         _lib.oracle_amax.argtypes = [ctypes.POINTER(_Args)]
         _lib.oracle_tensor_scale.restype = ctypes.c_float
         _lib.oracle_tensor_scale.argtypes = [ctypes.POINTER(_Args)]
@@ -224,6 +229,19 @@ def e2m1_decode(c):
 
 def floor_log2(a):
     return lib().oracle_floor_log2(float(a))
+
+
+def scale_tiles(scales, rows, cols, batch=1):
+    """Scale bytes [batch, rows, cols] (or [rows, cols]) in the block-scaled MMA's
+    128 x 4 tile layout (see oracle_scale_tiles): uint8[batch * tiles_bytes]."""
+    src = np.ascontiguousarray(scales, dtype=np.uint8).reshape(-1)
+    if src.size != batch * rows * cols:
+        raise ValueError("scales do not hold batch * rows * cols bytes")
+    per = lib().oracle_scale_tiles_bytes(rows, cols)
+    out = np.empty(batch * per, dtype=np.uint8)
+    if lib().oracle_scale_tiles(src.ctypes.data if src.size else None, rows, cols, batch, out.ctypes.data) != 0:
+        raise ValueError("oracle_scale_tiles rejected its arguments")
+    return out
 
 
 def ratio(sparse_energy, dense_energy):

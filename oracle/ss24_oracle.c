@@ -744,3 +744,46 @@ int oracle_dequantize(const oracle_args *a, const oracle_outputs *o, float *xhat
     }
     return 0;
 }
+
+/* Block-scale tiles: the layout in which the tensor cores' block-scaled MMA
+ * takes its scale factors (one byte each, E4M3 for NVFP4, E8M0 for MXFP4).
+ * This is not in the pages: it is the layout NVIDIA documents for block-scaled
+ * GEMM operands (cuBLAS library documentation, "1D block scaling factors
+ * layout"). The scale matrix of rows x cols bytes (cols = scale blocks along
+ * the reduction axis) is padded with zero bytes to a multiple of 128 rows and
+ * 4 columns and cut into 128 x 4 tiles. Tiles are stored row-tile major
+ * (column tiles inner), 512 bytes each. Inside a tile, row r = 32 a + b and
+ * column j go to byte 16 b + 4 a + j.
+ * A batch is stored operand after operand, the input packed (rows * cols
+ * bytes per operand), the output tiles_bytes(rows, cols) per operand.
+ * Returns 0, or -1 for arguments it does not support. */
+int64_t oracle_scale_tiles_bytes(int64_t rows, int64_t cols)
+{
+    if (rows < 0 || cols < 0)
+        return -1;
+    int64_t rt = (rows + 127) / 128, ct = (cols + 3) / 4;
+    return rt * ct * 512;
+}
+
+int oracle_scale_tiles(const uint8_t *in, int64_t rows, int64_t cols, int64_t batch, uint8_t *out)
+{
+    if (rows < 0 || cols < 0 || batch < 1 || (!in && rows * cols > 0) || !out)
+        return -1;
+    int64_t ct = (cols + 3) / 4;
+    int64_t per_op = oracle_scale_tiles_bytes(rows, cols);
+    for (int64_t b = 0; b < batch; ++b) {
+        const uint8_t *src = in ? in + b * rows * cols : NULL;
+        uint8_t *dst = out + b * per_op;
+        for (int64_t i = 0; i < per_op; ++i)
+            dst[i] = 0;
+        for (int64_t r = 0; r < rows; ++r) {
+            for (int64_t c = 0; c < cols; ++c) {
+                int64_t tile = (r / 128) * ct + c / 4;
+                int64_t rr = r % 128;
+                int64_t within = 16 * (rr % 32) + 4 * (rr / 32) + c % 4;
+                dst[tile * 512 + within] = src[r * cols + c];
+            }
+        }
+    }
+    return 0;
+}

@@ -545,3 +545,50 @@ def test_dequantize_reproduces_the_error_energies(pattern, fmt, bits, group, pac
     if fmt == "none":
         kept = xhat != 0
         assert np.array_equal(xhat[kept], x[kept].astype(np.float32))
+
+
+def _golden_scale_tiles(name):
+    pts, total = [], None
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            if line.startswith("# total_bytes"):
+                total = int(line.split()[2])
+            elif line.strip() and not line.startswith("#"):
+                pts.append(tuple(int(v) for v in line.split()))
+    return total, pts
+
+
+def test_scale_tiles_golden_offsets():
+    """Hand-computed byte offsets of the block-scale tile layout."""
+    total, pts = _golden_scale_tiles("scale_tiles_130x5.txt")
+    assert oracle.lib().oracle_scale_tiles_bytes(130, 5) == total
+    for r, c, off in pts:
+        src = np.zeros((130, 5), dtype=np.uint8)
+        src[r, c] = 0xA5
+        out = oracle.scale_tiles(src, 130, 5)
+        assert out.size == total
+        assert np.flatnonzero(out).tolist() == [off], (r, c)
+
+
+def test_scale_tiles_reshape_statement_and_padding():
+    """The oracle's index arithmetic against the layout stated as tensor
+    reshapes (pad, split rows into tiles of 4 x 32, swap the 4 and the 32),
+    plus: zero padding, and every input byte stored exactly once."""
+    rng = np.random.default_rng(5)
+    for rows, cols, batch in ((1, 1, 1), (128, 4, 1), (130, 5, 2), (300, 17, 3), (7, 64, 1)):
+        src = rng.integers(1, 256, size=(batch, rows, cols), dtype=np.uint8)
+        got = oracle.scale_tiles(src, rows, cols, batch)
+        rp, cp = -(-rows // 128) * 128, -(-cols // 4) * 4
+        pad = np.zeros((batch, rp, cp), dtype=np.uint8)
+        pad[:, :rows, :cols] = src
+        t = pad.reshape(batch, rp // 128, 4, 32, cp // 4, 4)      # [b, rt, a, b32, ct, j]
+        t = t.transpose(0, 1, 4, 3, 2, 5)                          # [b, rt, ct, b32, a, j]
+        assert np.array_equal(got, t.reshape(-1)), (rows, cols, batch)
+        assert np.count_nonzero(got) == src.size
+        assert sorted(got[got != 0].tolist()) == sorted(src.reshape(-1).tolist())
+
+
+def test_scale_tiles_rejects_bad_arguments():
+    assert oracle.lib().oracle_scale_tiles_bytes(-1, 4) == -1
+    assert oracle.lib().oracle_scale_tiles(None, 4, 4, 1, None) == -1
+    assert oracle.lib().oracle_scale_tiles_bytes(0, 7) == 0
