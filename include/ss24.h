@@ -440,6 +440,29 @@ ss24_status ss24_selfcheck_division(int32_t mode, uint32_t b_first, uint32_t b_c
 ss24_status ss24_selfcheck_encoder(int32_t kind, const uint32_t *bounds, int32_t n_bounds, uint32_t hi_first,
                                    uint32_t hi_count, unsigned long long *result, ss24_stream stream);
 
+/* ---- consumer layouts ------------------------------------------------------ */
+
+/* Bytes of the block-scale tiles of a rows x cols scale matrix (one operand):
+ * ceil(rows / 128) * ceil(cols / 4) * 512; -1 for negative sizes. */
+int64_t ss24_scale_tiles_bytes(int64_t rows, int64_t cols);
+
+/* The NVFP4 (E4M3) or MXFP4 (E8M0) scale bytes a pass wrote, rearranged into
+ * the layout in which the tensor cores' block-scaled MMA takes its scale
+ * factors (NVIDIA's documented "1D block scaling factors layout"; the pages
+ * give no layout, §3 only the scale granularity). `scales` holds batch
+ * operands packed one after the other, each rows x cols bytes row major
+ * (cols = scale blocks per row: n / 16 for NVFP4, n / 32 for MXFP4, n the
+ * quantized row length), on the device. `tiles` (device, 16-byte aligned)
+ * receives ss24_scale_tiles_bytes(rows, cols) bytes per operand: the matrix
+ * padded with zero bytes to multiples of 128 rows and 4 columns, cut into
+ * 128 x 4 tiles of 512 bytes stored row tile by row tile (column tiles
+ * inner); inside a tile, row 32 a + b and column j sit at byte 16 b + 4 a + j.
+ * Every byte of `tiles` is written. batch: 0 or 1 for one operand, up to
+ * 1024. Errors: SS24_ERR_NULL, SS24_ERR_SHAPE (negative sizes, batch out of
+ * range), SS24_ERR_ALIGN (tiles not 16-byte aligned). */
+ss24_status ss24_scale_tiles(const uint8_t *scales, int64_t rows, int64_t cols, int64_t batch, uint8_t *tiles,
+                             ss24_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

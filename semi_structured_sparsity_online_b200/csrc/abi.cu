@@ -973,6 +973,26 @@ ss24_status ss24_dequantize(const ss24_operand *x, ss24_pattern pattern, ss24_fo
                                       in->meta, xhat, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int64_t ss24_scale_tiles_bytes(int64_t rows, int64_t cols)
+{
+    return scale_tiles_bytes(rows, cols);
+}
+
+ss24_status ss24_scale_tiles(const uint8_t *scales, int64_t rows, int64_t cols, int64_t batch, uint8_t *tiles,
+                             ss24_stream stream)
+{
+    if (rows < 0 || cols < 0 || batch < 0 || batch > kMaxGrid)
+        return SS24_ERR_SHAPE;
+    const int64_t nb = batch > 1 ? batch : 1;
+    if (scale_tiles_bytes(rows, cols) == 0)
+        return SS24_OK;
+    if (!tiles || (!scales && rows * cols > 0))
+        return SS24_ERR_NULL;
+    if (!aligned16(tiles))
+        return SS24_ERR_ALIGN;
+    return cuda_status(launch_scale_tiles(scales, rows, cols, nb, tiles, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 ss24_status ss24_predicted_ratio(const ss24_energy *sparse_side, const ss24_energy *dense_side, ss24_ratio *out,
                                  int64_t count, ss24_stream stream)
 {

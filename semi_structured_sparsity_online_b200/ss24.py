@@ -86,6 +86,8 @@ _SIGNATURES = {
     "ss24_quantize_int_rows": (ctypes.c_int, [_OP, ctypes.c_int, ctypes.c_int, _P, Format, _P, _OUT, _P, _P, _S,
                                               _P]),
     "ss24_dequantize": (ctypes.c_int, [_OP, ctypes.c_int, Format, _OUT, _P, _P]),
+    "ss24_scale_tiles_bytes": (ctypes.c_int64, [ctypes.c_int64, ctypes.c_int64]),
+    "ss24_scale_tiles": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, _P, _P]),
     "ss24_selfcheck_encoder": (ctypes.c_int, [ctypes.c_int32, _P, ctypes.c_int32, ctypes.c_uint32, ctypes.c_uint32,
                                               _P, _P]),
     "ss24_encode_e4m3": (ctypes.c_int, [_P, _P, ctypes.c_int64, _P]),
@@ -361,6 +363,20 @@ def dequantize(out, rows, k, pattern=SPARSE_24, fmt="none", bits=8, group=0, pac
     _check(lib().ss24_dequantize(ctypes.byref(op), pattern, f, ctypes.byref(o), _ptr(xhat), _stream(stream)),
            "ss24_dequantize")
     return xhat
+
+
+def scale_tiles(scales, rows, cols, batch=None, out=None, stream=None):
+    """NVFP4 / MXFP4 scale bytes (uint8 [rows, cols] or [B, rows, cols] on the
+    device, packed) in the block-scaled MMA's 128 x 4 tile layout
+    (ss24_scale_tiles): uint8 [B * ss24_scale_tiles_bytes(rows, cols)]."""
+    nb = batch or 1
+    per = lib().ss24_scale_tiles_bytes(rows, cols)
+    if per < 0:
+        raise ValueError("negative scale matrix size")
+    out = out if out is not None else torch.empty(nb * per, dtype=torch.uint8, device=scales.device)
+    _check(lib().ss24_scale_tiles(_ptr(scales), rows, cols, batch or 0, _ptr(out), _stream(stream)),
+           "ss24_scale_tiles")
+    return out
 
 
 def predicted_ratio(sparse_energy, dense_energy, out=None, stream=None):

@@ -205,3 +205,16 @@ def test_other_entry_points_validate():
     assert L.ss24_decode_e2m1(ALIGNED, ALIGNED, -1, None) == 2
     assert L.ss24_workspace_init(None, wsb, None) == 6
     assert L.ss24_workspace_error(None, None, None) == 1
+
+
+def test_scale_tiles_validation():
+    L = ss24.lib()
+    assert L.ss24_scale_tiles_bytes(130, 5) == oracle.lib().oracle_scale_tiles_bytes(130, 5) == 2048
+    assert L.ss24_scale_tiles_bytes(0, 5) == 0 and L.ss24_scale_tiles_bytes(5, 0) == 0
+    assert L.ss24_scale_tiles_bytes(-1, 5) == -1
+    assert L.ss24_scale_tiles(None, -1, 4, 0, ALIGNED, None) == 2          # SS24_ERR_SHAPE
+    assert L.ss24_scale_tiles(ALIGNED, 4, 4, 1025, ALIGNED, None) == 2     # batch beyond 1024
+    assert L.ss24_scale_tiles(None, 4, 4, 0, ALIGNED, None) == 1           # SS24_ERR_NULL
+    assert L.ss24_scale_tiles(ALIGNED, 4, 4, 0, None, None) == 1
+    assert L.ss24_scale_tiles(ALIGNED, 4, 4, 0, MISALIGNED, None) == 3     # SS24_ERR_ALIGN
+    assert L.ss24_scale_tiles(None, 0, 4, 0, None, None) == 0              # empty: nothing to write

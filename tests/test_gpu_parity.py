@@ -454,6 +454,41 @@ def test_dequantize_batch(ss, ws, pattern, fmt, bits, group, pack4, rows, k, bat
         assert_same(to_np(got[b]), want, f"x_hat[{b}]")
 
 
+@pytest.mark.parametrize("pattern", [0, 24, 48])
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4"])
+@pytest.mark.parametrize("rows,k,batch", [(37, 512, 0), (130, 1536, 0), (20, 1024, 3), (1, 64, 2)])
+def test_scale_tiles_of_pass_scales(ss, ws, pattern, fmt, rows, k, batch):
+    """The pass's own block scales, rearranged into the block-scaled MMA's tiles,
+    against the oracle's rearrangement of the oracle's scales, byte for byte."""
+    n = k // 2 if pattern else k
+    blk = 16 if fmt == "nvfp4" else 32
+    if n % blk:
+        pytest.skip("block longer than the row")
+    cols = n // blk
+    opat = {0: oracle.DENSE, 24: oracle.SPARSE_24, 48: oracle.SPARSE_48}[pattern]
+    nb = max(batch, 1)
+    xs = [synth.sweep_operand(rows, k, seed=60 + b) for b in range(nb)]
+    x = torch.stack([to_dev(v) for v in xs]) if batch else to_dev(xs[0])
+    out = ss.run(x, pattern=pattern, fmt=fmt, ws=ws)
+    got = ss.scale_tiles(out["scales"], rows, cols, batch=batch or None)
+    torch.cuda.synchronize()
+    want = np.concatenate([oracle.scale_tiles(oracle.run(xh, pattern=opat, fmt=fmt)["scales"], rows, cols)
+                           for xh in xs])
+    assert np.array_equal(got.cpu().numpy(), want)
+
+
+@pytest.mark.parametrize("rows,cols,batch", [(1, 1, 0), (300, 17, 0), (129, 5, 4), (128, 4, 0), (4096, 256, 2)])
+def test_scale_tiles_random_bytes(ss, rows, cols, batch):
+    """Every byte value, ragged rows and columns, and zero padding written."""
+    nb = max(batch, 1)
+    src = np.random.default_rng(rows + cols).integers(0, 256, size=(nb, rows, cols), dtype=np.uint8)
+    per = oracle.lib().oracle_scale_tiles_bytes(rows, cols)
+    out = torch.full((nb * per,), 0x5A, dtype=torch.uint8, device="cuda")   # stale bytes must be overwritten
+    got = ss.scale_tiles(torch.from_numpy(src).cuda(), rows, cols, batch=batch or None, out=out)
+    torch.cuda.synchronize()
+    assert np.array_equal(got.cpu().numpy(), oracle.scale_tiles(src, rows, cols, nb))
+
+
 @pytest.mark.parametrize("sparse,dense", [(("fp8",), ("int", 5, 128)), (("nvfp4",), ("mxfp4",)),
                                           (("int", 8, 0), ("int", 5, 0))])
 def test_measured_ratio_against_oracle_and_prediction(ss, ws, sparse, dense):
