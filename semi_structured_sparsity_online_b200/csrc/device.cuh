@@ -325,17 +325,15 @@ __device__ __forceinline__ float bf16x2_hmax(uint32_t m)
     return __uint_as_float(max(m & 0x7fffu, (m >> 16) & 0x7fffu) << 16);
 }
 
-// Per lane: all ones where |b| > |a|, else zero. |a| - |b| is computed in
-// bf16 with rounding to nearest, which keeps the sign of the exact difference
-// and is zero (+0) only when the magnitudes are equal (gradual underflow);
-// the sign bit of each lane is then replicated across it (prmt sign mode).
+// Per lane: all ones where |b| > |a|, else zero: a packed bf16 comparison of
+// the magnitudes whose unsigned result is a 16-bit mask per lane (|-0| = |+0|
+// is not greater; subnormals compare by value).
 __device__ __forceinline__ uint32_t bf16x2_gt_abs(uint32_t b, uint32_t a)
 {
-    uint32_t d, m;
-    asm("{ .reg .b32 aa, bb; abs.bf16x2 aa, %1; abs.bf16x2 bb, %2; sub.rn.bf16x2 %0, aa, bb; }"
-        : "=r"(d)
+    uint32_t m;
+    asm("{ .reg .b32 aa, bb; abs.bf16x2 aa, %1; abs.bf16x2 bb, %2; set.gt.u32.bf16x2 %0, bb, aa; }"
+        : "=r"(m)
         : "r"(a), "r"(b));
-    asm("prmt.b32 %0, %1, 0, 0xBB99;" : "=r"(m) : "r"(d));
     return m;
 }
 __device__ __forceinline__ uint32_t sel_mask(uint32_t m, uint32_t a, uint32_t b) { return (a & m) | (b & ~m); }
@@ -415,10 +413,11 @@ __device__ __forceinline__ f32x2 neg_div_fast2(f32x2 a, const Recip &r)
 // selection
 // ---------------------------------------------------------------------------
 
-// Top-2 of four by score with ties to the lower index, as a small tournament:
-// the winners of (0,1) and (2,3) meet for first place; second place is the
-// better of the first-place pair's loser and the other pair's winner. A later
-// index wins a comparison only when its score is strictly larger.
+// Top-2 of four by score with ties to the lower index. After the pairs (0,1)
+// and (2,3) are decided, the kept pair is (0,1) when (0,1)'s loser beats
+// (2,3)'s winner, (2,3) when (2,3)'s loser beats (0,1)'s winner, and the two
+// winners otherwise: four comparisons in all. A later index wins a comparison
+// only when its score is strictly larger.
 struct Pick {
     bool p;     // winner of (0,1) is 1
     bool q;     // winner of (2,3) is 3
@@ -434,11 +433,10 @@ __device__ __forceinline__ Pick top2_of_4(float s0, float s1, float s2, float s3
     k.q = s3 > s2;
     const float w01 = k.p ? s1 : s0, l01 = k.p ? s0 : s1;
     const float w23 = k.q ? s3 : s2, l23 = k.q ? s2 : s3;
-    const bool r = w23 > w01;   // first place comes from pair (2,3)
-    const bool ta = w23 > l01;  // if first is from (0,1): second is (2,3)'s winner
-    const bool tb = l23 > w01;  // if first is from (2,3): second is its loser
-    k.both01 = !r && !ta;
-    k.both23 = r && tb;
+    const bool ta = w23 > l01;  // (0,1)'s loser does not beat (2,3)'s winner
+    const bool tb = l23 > w01;  // (2,3)'s loser beats (0,1)'s winner
+    k.both01 = !ta;
+    k.both23 = tb;
     const uint32_t mixed = static_cast<uint32_t>(k.p) | ((2u + static_cast<uint32_t>(k.q)) << 2);
     k.nib = k.both01 ? 0x4u : (k.both23 ? 0xEu : mixed);
     return k;
@@ -457,7 +455,7 @@ template <bool kAbs>
 __device__ __forceinline__ Group24 group24(float x0, float x1, float x2, float x3, float s0, float s1, float s2,
                                            float s3)
 {
-    bool p, q, r, ta, tb;
+    bool p, q, ta, tb;
     float w01, l01, w23, l23;
     if constexpr (kAbs) {
         p = fabsf(x1) > fabsf(x0);
@@ -466,7 +464,6 @@ __device__ __forceinline__ Group24 group24(float x0, float x1, float x2, float x
         l01 = p ? x0 : x1;
         w23 = q ? x3 : x2;
         l23 = q ? x2 : x3;
-        r = fabsf(w23) > fabsf(w01);
         ta = fabsf(w23) > fabsf(l01);
         tb = fabsf(l23) > fabsf(w01);
     } else {
@@ -478,11 +475,12 @@ __device__ __forceinline__ Group24 group24(float x0, float x1, float x2, float x
         l23 = q ? x2 : x3;
         const float sw01 = p ? s1 : s0, sl01 = p ? s0 : s1;
         const float sw23 = q ? s3 : s2, sl23 = q ? s2 : s3;
-        r = sw23 > sw01;
         ta = sw23 > sl01;
         tb = sl23 > sw01;
     }
-    const bool both01 = !r && !ta, both23 = r && tb;
+    // ties keep the lower index: l01 beats w23 exactly when both kept values
+    // come from (0, 1); l23 beats w01 exactly when both come from (2, 3)
+    const bool both01 = !ta, both23 = tb;
     Group24 g;
     g.k0 = both01 ? x0 : (both23 ? x2 : w01);
     g.k1 = both01 ? x1 : (both23 ? x3 : w23);
@@ -500,8 +498,8 @@ __device__ __forceinline__ Group24 group24(float x0, float x1, float x2, float x
 
 // The two 2:4 groups of a chunk of eight bf16 values (words w0..w3, element
 // 2i in the low half of word i) by magnitude, both at once: lane 0 of every
-// packed word below is group 0, lane 1 group 1. The same tournament as
-// group24, with the comparisons from bf16x2_gt_abs and the choices as bit
+// packed word below is group 0, lane 1 group 1. The same top-2 as group24
+// (ties keep the lower index), from four comparisons (bf16x2_gt_abs) and bit
 // selects. Results: kept values k0 (lower index) and k1 per lane, the
 // metadata byte (group 0 in the low nibble), the chunk's energy and the
 // energy of its dropped values, summed in the same order as group24.
@@ -518,18 +516,20 @@ __device__ __forceinline__ Pair24 pair24_bf16(uint32_t w0, uint32_t w1, uint32_t
     const uint32_t mq = bf16x2_gt_abs(D, C);            // q: |x3| > |x2|
     const uint32_t w01 = sel_mask(mp, B, A), l01 = sel_mask(mp, A, B);
     const uint32_t w23 = sel_mask(mq, D, C), l23 = sel_mask(mq, C, D);
-    const uint32_t mr = bf16x2_gt_abs(w23, w01);        // r: first place from pair (2,3)
-    const uint32_t ma = bf16x2_gt_abs(w23, l01);        // ta
-    const uint32_t mb = bf16x2_gt_abs(l23, w01);        // tb
-    const uint32_t m01 = ~(mr | ma), m23 = mr & mb;     // both kept from (0,1) / from (2,3)
+    // With the tie rule (the lower index wins), l01 beats w23 exactly when both
+    // kept values come from (0, 1), and l23 beats w01 exactly when both come
+    // from (2, 3); otherwise w01 and w23 are kept (already in index order). The
+    // winners' own comparison is implied and not needed.
+    const uint32_t ta = bf16x2_gt_abs(w23, l01);        // not both from (0, 1)
+    const uint32_t tb = bf16x2_gt_abs(l23, w01);        // both from (2, 3)
     Pair24 g;
-    g.k0 = sel_mask(m01, A, sel_mask(m23, C, w01));
-    g.k1 = sel_mask(m01, B, sel_mask(m23, D, w23));
-    const uint32_t d0 = sel_mask(m01, C, sel_mask(m23, A, l01));
-    const uint32_t d1 = sel_mask(m01, D, sel_mask(m23, B, l23));
+    g.k0 = sel_mask(ta, sel_mask(tb, C, w01), A);
+    g.k1 = sel_mask(ta, sel_mask(tb, D, w23), B);
+    const uint32_t d0 = sel_mask(ta, sel_mask(tb, A, l01), C);
+    const uint32_t d1 = sel_mask(ta, sel_mask(tb, B, l23), D);
     // nibble i0 | i1 << 2: (0,1) -> 4, (2,3) -> 14, otherwise p | (2 + q) << 2
     const uint32_t mixed = 0x00080008u | (mp & 0x00010001u) | (mq & 0x00040004u);
-    const uint32_t nib = sel_mask(m01, 0x00040004u, sel_mask(m23, 0x000E000Eu, mixed));
+    const uint32_t nib = sel_mask(ta, sel_mask(tb, 0x000E000Eu, mixed), 0x00040004u);
     g.meta = (nib | (nib >> 12)) & 0xffu;
     // energies: (x0^2 + x1^2) + (x2^2 + x3^2) per group, dropped d0^2 + d1^2
     const float e01a = bf16_sq_lo(B, bf16_sq_lo(A, -0.0f)), e23a = bf16_sq_lo(D, bf16_sq_lo(C, -0.0f));
