@@ -502,7 +502,7 @@ __device__ __forceinline__ Group24 group24(float x0, float x1, float x2, float x
 // (ties keep the lower index), from four comparisons (bf16x2_gt_abs) and bit
 // selects. Results: kept values k0 (lower index) and k1 per lane, the
 // metadata byte (group 0 in the low nibble), the chunk's energy and the
-// energy of its dropped values, summed in the same order as group24.
+// energy of its dropped values.
 struct Pair24 {
     uint32_t k0, k1, meta;
     float e_all, e_drop;
@@ -531,11 +531,11 @@ __device__ __forceinline__ Pair24 pair24_bf16(uint32_t w0, uint32_t w1, uint32_t
     const uint32_t mixed = 0x00080008u | (mp & 0x00010001u) | (mq & 0x00040004u);
     const uint32_t nib = sel_mask(ta, sel_mask(tb, 0x000E000Eu, mixed), 0x00040004u);
     g.meta = (nib | (nib >> 12)) & 0xffu;
-    // energies: (x0^2 + x1^2) + (x2^2 + x3^2) per group, dropped d0^2 + d1^2
-    const float e01a = bf16_sq_lo(B, bf16_sq_lo(A, -0.0f)), e23a = bf16_sq_lo(D, bf16_sq_lo(C, -0.0f));
-    const float e01b = bf16_sq_hi(B, bf16_sq_hi(A, -0.0f)), e23b = bf16_sq_hi(D, bf16_sq_hi(C, -0.0f));
-    g.e_all = (e01a + e23a) + (e01b + e23b);
-    g.e_drop = bf16_sq_lo(d1, bf16_sq_lo(d0, -0.0f)) + bf16_sq_hi(d1, bf16_sq_hi(d0, -0.0f));
+    // energies: the dropped values' squares, and the chunk's energy as the kept
+    // values' squares plus the dropped ones (binary32 chains of fused
+    // multiply-adds; the energies are sums, compared within 1e-6 relative)
+    g.e_drop = bf16_sq_hi(d1, bf16_sq_hi(d0, bf16_sq_lo(d1, bf16_sq_lo(d0, -0.0f))));
+    g.e_all = bf16_sq_hi(g.k1, bf16_sq_hi(g.k0, bf16_sq_lo(g.k1, bf16_sq_lo(g.k0, g.e_drop))));
     return g;
 }
 

@@ -109,40 +109,37 @@ __device__ __forceinline__ float group_amax(float m, int lanes)
     return m;
 }
 
-// Sum of (v - d)^2 over a chunk's values: packed differences and squares,
-// summed as a binary tree (each term and each partial sum rounded once).
+// Sum of the squares of N packed pairs: one packed multiply, then packed fused
+// multiply-adds, then the two lanes (binary32; the energies are sums compared
+// within 1e-6 relative, and each term and partial sum is rounded once).
+template <int N> __device__ __forceinline__ float sq_sum2(const f32x2 (&e)[N])
+{
+    f32x2 t = mul2(e[0], e[0]);
+#pragma unroll
+    for (int i = 1; i < N; ++i)
+        t = fma2(e[i], e[i], t);
+    return lo2(t) + hi2(t);
+}
+
+// Sum of (v - d)^2 over a chunk's values (packed differences, sq_sum2).
 template <int VPC> __device__ __forceinline__ float err_energy(const float (&v)[VPC], const float (&d)[VPC])
 {
-    f32x2 t[VPC / 2];
+    f32x2 e[VPC / 2];
 #pragma unroll
-    for (int i = 0; i < VPC / 2; ++i) {
-        const f32x2 e = sub2(pack2(v[2 * i], v[2 * i + 1]), pack2(d[2 * i], d[2 * i + 1]));
-        t[i] = mul2(e, e);
-    }
-#pragma unroll
-    for (int w = VPC / 4; w >= 1; w /= 2)
-#pragma unroll
-        for (int i = 0; i < w; ++i)
-            t[i] = add2(t[i], t[i + w]);
-    return lo2(t[0]) + hi2(t[0]);
+    for (int i = 0; i < VPC / 2; ++i)
+        e[i] = sub2(pack2(v[2 * i], v[2 * i + 1]), pack2(d[2 * i], d[2 * i + 1]));
+    return sq_sum2<VPC / 2>(e);
 }
 
 // The same with the dequantized values given negated (dn = -d): the terms
 // v + dn equal v - d, rounding included.
 template <int VPC> __device__ __forceinline__ float err_energy_neg(const float (&v)[VPC], const float (&dn)[VPC])
 {
-    f32x2 t[VPC / 2];
+    f32x2 e[VPC / 2];
 #pragma unroll
-    for (int i = 0; i < VPC / 2; ++i) {
-        const f32x2 e = add2(pack2(v[2 * i], v[2 * i + 1]), pack2(dn[2 * i], dn[2 * i + 1]));
-        t[i] = mul2(e, e);
-    }
-#pragma unroll
-    for (int w = VPC / 4; w >= 1; w /= 2)
-#pragma unroll
-        for (int i = 0; i < w; ++i)
-            t[i] = add2(t[i], t[i + w]);
-    return lo2(t[0]) + hi2(t[0]);
+    for (int i = 0; i < VPC / 2; ++i)
+        e[i] = add2(pack2(v[2 * i], v[2 * i + 1]), pack2(dn[2 * i], dn[2 * i + 1]));
+    return sq_sum2<VPC / 2>(e);
 }
 
 // True when the fast division applies to every value of a chunk or group
@@ -575,9 +572,8 @@ __device__ __forceinline__ Sel<PAT == kDense ? 8 : 4> select_chunk(const typenam
         f32x2 t[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-            t[i] = mul2(pack2(x[2 * i], x[2 * i + 1]), pack2(x[2 * i], x[2 * i + 1]));
-        t[0] = add2(add2(t[0], t[1]), add2(t[2], t[3]));
-        et = lo2(t[0]) + hi2(t[0]);
+            t[i] = pack2(x[2 * i], x[2 * i + 1]);
+        et = sq_sum2<4>(t);
     } else if constexpr (kPair) {
         const uint4 w = raw.v;
         const Pair24 g = pair24_bf16(w.x, w.y, w.z, w.w);
@@ -749,7 +745,7 @@ __device__ __forceinline__ void process_chunk(const PassParams &p, const typenam
 
 // Dense INT-b codes of one chunk with its row's scale, straight-line on
 // binary32 pairs: the same operations, roundings and summation order as
-// quant_int / err_energy and the dense energy in process_chunk, with the code
+// quant_int / err_energy and the dense energy in select_chunk, with the code
 // width (STORE) and the fast-division decision (FAST, one per row) fixed.
 template <typename T, int STORE, bool FAST>
 __device__ __forceinline__ void dense_int_chunk(const typename Elem<T>::Raw &raw, const RowScale &rs, float qmax,
@@ -761,12 +757,7 @@ __device__ __forceinline__ void dense_int_chunk(const typename Elem<T>::Raw &raw
 #pragma unroll
     for (int i = 0; i < 4; ++i)
         x2[i] = pack2(x[2 * i], x[2 * i + 1]);
-    f32x2 t[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-        t[i] = mul2(x2[i], x2[i]);
-    t[0] = add2(add2(t[0], t[1]), add2(t[2], t[3]));
-    acc.et += lo2(t[0]) + hi2(t[0]);
+    acc.et += sq_sum2<4>(x2);
     const f32x2 m2 = pack2(kMagic, kMagic), s2 = pack2(rs.scale, rs.scale);
     f32x2 tt[4], e[4];
 #pragma unroll
@@ -781,11 +772,9 @@ __device__ __forceinline__ void dense_int_chunk(const typename Elem<T>::Raw &raw
         }
         tt[i] = sub2(m2, qn);
         const f32x2 d = mul2(sub2(tt[i], m2), s2);
-        const f32x2 df = sub2(x2[i], d);
-        e[i] = mul2(df, df);
+        e[i] = sub2(x2[i], d);
     }
-    e[0] = add2(add2(e[0], e[2]), add2(e[1], e[3]));
-    acc.eqd += lo2(e[0]) + hi2(e[0]);
+    acc.eqd += sq_sum2<4>(e);
     if (valid) {
         uint32_t b[8]; // low bits of M + q hold the two's-complement code
 #pragma unroll
