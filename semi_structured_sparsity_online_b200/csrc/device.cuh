@@ -338,6 +338,18 @@ __device__ __forceinline__ uint32_t bf16x2_gt_abs(uint32_t b, uint32_t a)
 }
 __device__ __forceinline__ uint32_t sel_mask(uint32_t m, uint32_t a, uint32_t b) { return (a & m) | (b & ~m); }
 
+// True when some lane of a or b has a magnitude >= the bf16 value lim (both
+// lanes of lim2 hold it): two packed comparisons.
+__device__ __forceinline__ bool bf16x2_any_ge_abs(uint32_t a, uint32_t b, uint32_t lim2)
+{
+    uint32_t m;
+    asm("{ .reg .b32 aa, bb, ma, mb; abs.bf16x2 aa, %1; abs.bf16x2 bb, %2;\n"
+        " set.ge.u32.bf16x2 ma, aa, %3; set.ge.u32.bf16x2 mb, bb, %3; or.b32 %0, ma, mb; }"
+        : "=r"(m)
+        : "r"(a), "r"(b), "r"(lim2));
+    return m != 0u;
+}
+
 // ---------------------------------------------------------------------------
 // division by a scale
 // ---------------------------------------------------------------------------

@@ -187,12 +187,23 @@ __device__ __forceinline__ void scale_values(const float (&c)[VPC], float s, flo
 // With `guard` false the caller knows that no quotient can overflow (the scale
 // was derived from the amax of the values quantized).
 template <int VPC, bool STORE>
+__device__ __forceinline__ float quant_fp8_as(const float (&v)[VPC], bool fast, const Recip &rc, const ChunkOut &o);
+
+template <int VPC, bool STORE>
 __device__ __forceinline__ float quant_fp8(const float (&v)[VPC], float vmax, const Recip &rc, bool guard,
                                            const ChunkOut &o)
 {
     bool fast = rc.fast;
     if (guard)
         fast = quot_fast(rc, vmax);
+    return quant_fp8_as<VPC, STORE>(v, fast, rc, o);
+}
+
+// quant_fp8 with the division path decided by the caller (fast: every
+// quotient of the chunk is in range for neg_div_fast2).
+template <int VPC, bool STORE>
+__device__ __forceinline__ float quant_fp8_as(const float (&v)[VPC], bool fast, const Recip &rc, const ChunkOut &o)
+{
     float qn[VPC], decn[VPC], dn[VPC];
     neg_quotients<VPC>(v, rc, fast, qn);
     // codes of -q, decoded as they come from the conversion: dn = -deq exactly
@@ -503,7 +514,25 @@ struct PassConsts {
     Recip rst, rstd;
     NvTable tb, tbd;
     bool guard, guardd;
+    uint32_t lim2; // FP8 with a given scale: bf16x2 of fast_limit(rst), see fp8_fast_limit
 };
+
+// The smallest bf16 magnitude m with RN(m * y) >= 2^126 for the reciprocal y
+// of a per-tensor scale (+inf when no finite bf16 reaches it). RN(m * y) is
+// non-decreasing in m, so a chunk's quotients all suit neg_div_fast2 (see
+// quot_fast) exactly when every kept magnitude is below this limit.
+__device__ __forceinline__ uint32_t fp8_fast_limit(const Recip &rc)
+{
+    uint32_t lo = 0u, hi = 0x7f80u; // f(lo) false, the answer in (lo, hi]
+    while (hi - lo > 1u) {
+        const uint32_t mid = (lo + hi) >> 1;
+        if (__fmul_rn(__uint_as_float(mid << 16), rc.y) >= 0x1p126f)
+            hi = mid;
+        else
+            lo = mid;
+    }
+    return hi | (hi << 16);
+}
 
 template <int SCORE>
 __device__ __forceinline__ void scores(const float (&x)[8], const ChunkOut &o, float (&s)[8])
@@ -546,6 +575,7 @@ template <int VPC> struct Sel {
     float vmax;
     uint32_t meta;
     uint32_t kept_bits[2]; // bf16 2:4 by magnitude: kept values as bf16x2 (group 0, group 1)
+    uint32_t k0, k1;       // the same values as selected: lower-index kept value of each group, then the other
     float et, ep;
 };
 
@@ -562,6 +592,7 @@ __device__ __forceinline__ Sel<PAT == kDense ? 8 : 4> select_chunk(const typenam
     float vmax;   // max |v| over the chunk's values to quantize
     uint32_t meta = 0;
     uint32_t kept_bits[2] = {0u, 0u};
+    uint32_t kw0 = 0u, kw1 = 0u;
     float et, ep = 0.0f;
 
     if constexpr (PAT == kDense) {
@@ -584,6 +615,8 @@ __device__ __forceinline__ Sel<PAT == kDense ? 8 : 4> select_chunk(const typenam
         vmax = bf16x2_hmax(bf16x2_maxabs(g.k0, g.k1));
         kept_bits[0] = __byte_perm(g.k0, g.k1, 0x5410);
         kept_bits[1] = __byte_perm(g.k0, g.k1, 0x7632);
+        kw0 = g.k0;
+        kw1 = g.k1;
         meta = g.meta;
         et = g.e_all;
         ep = g.e_drop;
@@ -656,6 +689,8 @@ __device__ __forceinline__ Sel<PAT == kDense ? 8 : 4> select_chunk(const typenam
     r.meta = meta;
     r.kept_bits[0] = kept_bits[0];
     r.kept_bits[1] = kept_bits[1];
+    r.k0 = kw0;
+    r.k1 = kw1;
     r.et = et;
     r.ep = ep;
     return r;
@@ -717,7 +752,14 @@ __device__ __forceinline__ void finish_chunk(const PassParams &p, const typename
             }
         }
     } else if constexpr (FMT == kFp8) {
-        eq = quant_fp8<VPC, true>(v, vmax, c.rst, c.guard, o);
+        if constexpr (kPair) {
+            // the overflow guard as two packed comparisons of the kept values
+            // with the CTA's limit (equivalent to quot_fast on their maximum)
+            const bool fast = c.rst.fast && !(c.guard && bf16x2_any_ge_abs(sl.k0, sl.k1, c.lim2));
+            eq = quant_fp8_as<VPC, true>(v, fast, c.rst, o);
+        } else {
+            eq = quant_fp8<VPC, true>(v, vmax, c.rst, c.guard, o);
+        }
     } else if constexpr (FMT == kInt || FMT == kIntRows) {
         eq = quant_int<VPC, true>(v, vmax, p.q, o, row_amax, rs, gamax);
     } else if constexpr (FMT == kNvfp4) {
@@ -1093,6 +1135,10 @@ __device__ __forceinline__ PassConsts make_consts(const PassParams &p, int tid, 
     c.rstd = make_recip(std_);
     c.guard = p.q.scale_in != nullptr;
     c.guardd = p.qd.scale_in != nullptr;
+    c.lim2 = 0x7f807f80u;
+    if constexpr (FMT == kFp8)
+        if (c.guard)
+            c.lim2 = fp8_fast_limit(c.rst);
     c.tb = NvTable{nvt, nvt + 128};
     c.tbd = NvTable{nvt + 256, nvt + 384};
     if constexpr (FMT == kNvfp4 || FMT == kEnergy) {
