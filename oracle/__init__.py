@@ -69,6 +69,11 @@ def lib():
         _lib.oracle_scale_tiles.restype = ctypes.c_int
         _lib.oracle_scale_tiles.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                             ctypes.c_void_p]
+        _lib.oracle_hadamard_scale.restype = ctypes.c_float
+        _lib.oracle_hadamard_scale.argtypes = [ctypes.c_int32]
+        _lib.oracle_hadamard.restype = ctypes.c_int
+        _lib.oracle_hadamard.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                         ctypes.c_int32, ctypes.c_void_p]
         _lib.oracle_amax.argtypes = [ctypes.POINTER(_Args)]
         _lib.oracle_tensor_scale.restype = ctypes.c_float
         _lib.oracle_tensor_scale.argtypes = [ctypes.POINTER(_Args)]
@@ -229,6 +234,24 @@ def e2m1_decode(c):
 
 def floor_log2(a):
     return lib().oracle_floor_log2(float(a))
+
+
+def hadamard(x, block):
+    """Block Hadamard rotation along k (see oracle_hadamard) of an operand given
+    as bf16 bits (uint16) or float32, [rows, k] or [batch, rows, k]: float32 of
+    the same shape."""
+    a = np.asarray(x)
+    if a.dtype == np.uint16:
+        f = (a.astype(np.uint32) << 16).view(np.float32)   # bf16 bits widened exactly
+    else:
+        f = a.astype(np.float32)
+    f = np.ascontiguousarray(f, dtype=np.float32)
+    k = f.shape[-1]
+    rows = f.size // k if k else 0
+    out = np.empty_like(f)
+    if f.size and lib().oracle_hadamard(f.ctypes.data, rows, k, k, int(block), out.ctypes.data) != 0:
+        raise ValueError("oracle_hadamard rejected its arguments")
+    return out
 
 
 def scale_tiles(scales, rows, cols, batch=1):

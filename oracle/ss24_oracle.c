@@ -787,3 +787,48 @@ int oracle_scale_tiles(const uint8_t *in, int64_t rows, int64_t cols, int64_t ba
     }
     return 0;
 }
+
+/* Block Hadamard rotation along the reduction axis. The pages (§4) note that
+ * tensors are often multiplied by a Hadamard matrix (an orthogonal matrix of
+ * +-1 entries, rescaled) before low-bit quantization, which spreads outliers
+ * over many elements and, by their analysis, raises R. They do not fix the
+ * block size. Reading taken: block-diagonal along k with block size b (a power
+ * of two from 2 to 256 dividing k); each block of b consecutive elements of a
+ * row is multiplied by the Sylvester matrix H_b (H_1 = [1],
+ * H_2m = [[H_m, H_m], [H_m, -H_m]]) and by 1/sqrt(b).
+ * Arithmetic, binary32: the fast Walsh-Hadamard butterflies in stage order
+ * h = 1, 2, 4, ..., b/2, each pair (y_i, y_i+h) with (i & h) == 0 becoming
+ * (y_i + y_i+h, y_i - y_i+h), each result rounded; then every element times
+ * c_b = RN(1/sqrt(b)) (exact when b is a power of 4).
+ * x: rows x k values with row stride ld (>= k); out: rows x k, packed.
+ * Returns 0, or -1 for arguments it does not support. */
+float oracle_hadamard_scale(int32_t b)
+{
+    return (float)(1.0 / sqrt((double)b));
+}
+
+int oracle_hadamard(const float *x, int64_t rows, int64_t k, int64_t ld, int32_t b, float *out)
+{
+    if (!x || !out || rows < 0 || k <= 0 || ld < k || b < 2 || b > 256 || (b & (b - 1)) != 0 || k % b != 0)
+        return -1;
+    float y[256];
+    const float cb = oracle_hadamard_scale(b);
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t c0 = 0; c0 < k; c0 += b) {
+            for (int32_t i = 0; i < b; ++i)
+                y[i] = x[r * ld + c0 + i];
+            for (int32_t h = 1; h < b; h *= 2) {
+                for (int32_t i = 0; i < b; ++i) {
+                    if (i & h)
+                        continue;
+                    float a = y[i], c = y[i + h];
+                    y[i] = a + c;
+                    y[i + h] = a - c;
+                }
+            }
+            for (int32_t i = 0; i < b; ++i)
+                out[r * k + c0 + i] = y[i] * cb;
+        }
+    }
+    return 0;
+}

@@ -592,3 +592,52 @@ def test_scale_tiles_rejects_bad_arguments():
     assert oracle.lib().oracle_scale_tiles_bytes(-1, 4) == -1
     assert oracle.lib().oracle_scale_tiles(None, 4, 4, 1, None) == -1
     assert oracle.lib().oracle_scale_tiles_bytes(0, 7) == 0
+
+
+HADAMARD_BLOCKS = [2, 4, 8, 16, 32, 64, 128, 256]
+
+
+@pytest.mark.parametrize("b", HADAMARD_BLOCKS)
+def test_hadamard_unit_vectors_closed_form(b):
+    """Each unit vector maps to a column of the Sylvester matrix, whose entry
+    (j, i) is (-1)^popcount(i & j), times RN(1/sqrt(b)); other blocks stay 0."""
+    k = 2 * b
+    cb = np.float32(1.0 / math.sqrt(b))
+    assert oracle.lib().oracle_hadamard_scale(b) == cb
+    for i in sorted({0, 1, b // 2, b - 1, b, k - 1}):
+        x = np.zeros((1, k), dtype=np.float32)
+        x[0, i] = 1.0
+        got = oracle.hadamard(x, b)[0]
+        blk = (i // b) * b
+        want = np.zeros(k, dtype=np.float32)
+        for j in range(b):
+            want[blk + j] = cb if bin((i - blk) & j).count("1") % 2 == 0 else -cb
+        assert np.array_equal(got, want), (b, i)
+
+
+@pytest.mark.parametrize("b", HADAMARD_BLOCKS)
+def test_hadamard_against_library_matrix(b):
+    """Against scipy.linalg.hadamard in binary64, within the rounding bound of
+    log2(b) butterfly stages and the final scaling; and energy preserved."""
+    from scipy.linalg import hadamard
+    xh, _ = synth.linear_input(16, 1024, seed=71)
+    x = ((xh.astype(np.uint32) << 16).view(np.float32)).astype(np.float64)
+    got = oracle.hadamard(xh, b).astype(np.float64)
+    H = hadamard(b).astype(np.float64) / math.sqrt(b)
+    want = (x.reshape(16, -1, b) @ H.T).reshape(16, 1024)
+    absx = np.abs(x).reshape(16, -1, b).sum(axis=2, keepdims=True) / math.sqrt(b)
+    bound = ((math.log2(b) + 2) * 2.0 ** -24 * np.broadcast_to(absx, (16, 1024 // b, b))).reshape(16, 1024)
+    assert np.all(np.abs(got - want) <= bound + 1e-45)
+    assert abs((got ** 2).sum() / (x ** 2).sum() - 1) < 1e-5
+
+
+def test_hadamard_is_an_involution_and_rejects_bad_blocks():
+    xf = synth.gaussian_f32(8, 512, seed=72)
+    for b in (8, 128):
+        twice = oracle.hadamard(oracle.hadamard(xf, b), b)
+        assert np.allclose(twice, xf, rtol=0, atol=1e-5 * np.abs(xf).max())
+    for b in (0, 1, 3, 512):
+        with pytest.raises(ValueError):
+            oracle.hadamard(xf, b)
+    with pytest.raises(ValueError):
+        oracle.hadamard(synth.gaussian_f32(2, 24, seed=1), 16)   # k not a multiple of b
