@@ -440,6 +440,25 @@ ss24_status ss24_selfcheck_division(int32_t mode, uint32_t b_first, uint32_t b_c
 ss24_status ss24_selfcheck_encoder(int32_t kind, const uint32_t *bounds, int32_t n_bounds, uint32_t hi_first,
                                    uint32_t hi_count, unsigned long long *result, ss24_stream stream);
 
+/* ---- rotation ----------------------------------------------------------------- */
+
+/* Block Hadamard rotation along k (§4: a Hadamard matrix, orthogonal with
+ * +-1 entries rescaled, applied before low-bit quantization spreads outliers
+ * and, by the pages' analysis, raises R; they do not fix the block size).
+ * Every block of `block` consecutive elements of a row (block a power of two
+ * from 2 to 256 dividing k; k a multiple of 8) is multiplied by the Sylvester
+ * matrix H_b (H_1 = [1], H_2m = [[H_m, H_m], [H_m, -H_m]]) and by
+ * RN(1/sqrt(block)). Arithmetic in binary32: fast Walsh-Hadamard butterflies
+ * in stage order h = 1, 2, 4, ..., block/2, the pair (y_i, y_i+h) with
+ * (i & h) == 0 becoming (y_i + y_i+h, y_i - y_i+h), each rounded, then one
+ * rounded multiplication. x: bf16 or fp32, axis 1 only (ld >= k, batch as for
+ * the passes). out (device, 16-byte aligned, owned by the caller): fp32,
+ * packed [batch][rows][k]; it is the operand to hand to the passes (as fp32)
+ * for a rotated pass. Errors: the operand checks of the passes, SS24_ERR_ARG
+ * (axis 0, block not a power of two in [2, 256]), SS24_ERR_SHAPE (k not a
+ * multiple of 8 and of block), SS24_ERR_NULL, SS24_ERR_ALIGN. */
+ss24_status ss24_hadamard(const ss24_operand *x, int32_t block, float *out, ss24_stream stream);
+
 /* ---- consumer layouts ------------------------------------------------------ */
 
 /* Bytes of the block-scale tiles of a rows x cols scale matrix (one operand):

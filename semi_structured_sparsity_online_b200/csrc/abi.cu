@@ -973,6 +973,28 @@ ss24_status ss24_dequantize(const ss24_operand *x, ss24_pattern pattern, ss24_fo
                                       in->meta, xhat, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+ss24_status ss24_hadamard(const ss24_operand *x, int32_t block, float *out, ss24_stream stream)
+{
+    ss24_status st = check_operand(x);
+    if (st != SS24_OK)
+        return st;
+    if (x->axis != 1)
+        return SS24_ERR_ARG;
+    if (block < 2 || block > 256 || (block & (block - 1)) != 0)
+        return SS24_ERR_ARG;
+    if (x->k % 8 != 0 || x->k % block != 0)
+        return SS24_ERR_SHAPE;
+    if (x->rows == 0)
+        return SS24_OK;
+    if (!out)
+        return SS24_ERR_NULL;
+    if (!aligned16(out))
+        return SS24_ERR_ALIGN;
+    return cuda_status(launch_hadamard(x->x, x->dtype == SS24_BF16 ? 1 : 0, x->rows, x->k, x->ld,
+                                       nbatch(x) > 1 ? x->batch_stride : 0, nbatch(x), block, out,
+                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int64_t ss24_scale_tiles_bytes(int64_t rows, int64_t cols)
 {
     return scale_tiles_bytes(rows, cols);

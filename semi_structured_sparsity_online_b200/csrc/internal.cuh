@@ -124,6 +124,8 @@ cudaError_t launch_convert(int op, const void *in, void *out, int64_t n, cudaStr
 cudaError_t launch_dequant(int pattern, int fmt, int32_t store, int32_t lg, int32_t none_f32, int64_t rows,
                            int64_t k, int32_t batch, const void *values, const void *scales, const float *tscale,
                            const uint8_t *meta, float *xhat, cudaStream_t stream);
+cudaError_t launch_hadamard(const void *x, int bf16, int64_t rows, int64_t k, int64_t ld, int64_t bstride,
+                            int64_t batch, int32_t block, float *out, cudaStream_t stream);
 int64_t scale_tiles_bytes(int64_t rows, int64_t cols);
 cudaError_t launch_scale_tiles(const uint8_t *in, int64_t rows, int64_t cols, int64_t batch, uint8_t *out,
                                cudaStream_t stream);

@@ -44,6 +44,8 @@ def pass_bytes(name, m, k):
     n = m * k
     if name in ("tensor_scale", "error_energy"):
         return 2 * n
+    if name == "hadamard128":
+        return 2 * n + 4 * n
     if name == "amax_rows":
         return 2 * n + 4 * m
     if name == "dense_int8_given_rows":
@@ -66,7 +68,7 @@ def pass_bytes(name, m, k):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--pass", dest="name", default="fused_24_fp8", choices=sorted(PASSES) + ["tensor_scale", "error_energy", "amax_rows",
+    ap.add_argument("--pass", dest="name", default="fused_24_fp8", choices=sorted(PASSES) + ["tensor_scale", "error_energy", "amax_rows", "hadamard128",
                                                                        "dense_int8_given_rows"])
     ap.add_argument("--m", type=int, default=4096)
     ap.add_argument("--k", type=int, default=4096)
@@ -102,11 +104,15 @@ def main():
         out = ss24._alloc_outputs(args.m, args.k, ss24.DENSE, ss24.make_format("int", 8, 0), torch.bfloat16, "cuda",
                                   lead)
 
+    rot = torch.empty(x.shape, dtype=torch.float32, device="cuda") if args.name == "hadamard128" else None
+
     def once():
         if args.name == "amax_rows":
             ss24.amax_rows(x, scale_fmt="fp8", ws=ws, out=row_amax, scale_out=scale)
         elif args.name == "dense_int8_given_rows":
             ss24.run_int_rows(x, row_amax, bits=8, energy=e, ws=ws, out=out)
+        elif args.name == "hadamard128":
+            ss24.hadamard(x, 128, out=rot)
         elif args.name == "tensor_scale":
             ss24.tensor_scale(x, "fp8", ss24.SPARSE_24, ws=ws, out=scale)
         elif args.name == "error_energy":

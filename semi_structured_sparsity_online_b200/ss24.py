@@ -86,6 +86,7 @@ _SIGNATURES = {
     "ss24_quantize_int_rows": (ctypes.c_int, [_OP, ctypes.c_int, ctypes.c_int, _P, Format, _P, _OUT, _P, _P, _S,
                                               _P]),
     "ss24_dequantize": (ctypes.c_int, [_OP, ctypes.c_int, Format, _OUT, _P, _P]),
+    "ss24_hadamard": (ctypes.c_int, [_OP, ctypes.c_int32, _P, _P]),
     "ss24_scale_tiles_bytes": (ctypes.c_int64, [ctypes.c_int64, ctypes.c_int64]),
     "ss24_scale_tiles": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, _P, _P]),
     "ss24_selfcheck_encoder": (ctypes.c_int, [ctypes.c_int32, _P, ctypes.c_int32, ctypes.c_uint32, ctypes.c_uint32,
@@ -363,6 +364,15 @@ def dequantize(out, rows, k, pattern=SPARSE_24, fmt="none", bits=8, group=0, pac
     _check(lib().ss24_dequantize(ctypes.byref(op), pattern, f, ctypes.byref(o), _ptr(xhat), _stream(stream)),
            "ss24_dequantize")
     return xhat
+
+
+def hadamard(x: torch.Tensor, block: int, out=None, stream=None):
+    """Block Hadamard rotation of x [rows, k] or [B, rows, k] (bf16 or fp32,
+    k contiguous) along k (ss24_hadamard): fp32 of the same shape, packed."""
+    op = make_operand(x, 1)
+    out = out if out is not None else torch.empty(x.shape, dtype=torch.float32, device=x.device)
+    _check(lib().ss24_hadamard(ctypes.byref(op), int(block), _ptr(out), _stream(stream)), "ss24_hadamard")
+    return out
 
 
 def scale_tiles(scales, rows, cols, batch=None, out=None, stream=None):

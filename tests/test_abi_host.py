@@ -218,3 +218,18 @@ def test_scale_tiles_validation():
     assert L.ss24_scale_tiles(ALIGNED, 4, 4, 0, None, None) == 1
     assert L.ss24_scale_tiles(ALIGNED, 4, 4, 0, MISALIGNED, None) == 3     # SS24_ERR_ALIGN
     assert L.ss24_scale_tiles(None, 0, 4, 0, None, None) == 0              # empty: nothing to write
+
+
+def test_hadamard_validation():
+    L = ss24.lib()
+
+    def op(rows=4, k=64, ld=None, axis=1, ptr=ALIGNED, dtype=ss24.BF16):
+        return ss24.Operand(ptr, dtype, axis, rows, k, ld or k, 0, 0)
+    call = lambda o, b, out=ALIGNED: L.ss24_hadamard(ctypes.byref(o), b, out, None)
+    assert call(op(), 3) == 8 and call(op(), 1) == 8 and call(op(), 512) == 8       # SS24_ERR_ARG
+    assert call(op(axis=0, ld=8), 16) == 8
+    assert call(op(k=48), 32) == 2                                                 # k % block
+    assert call(op(k=4, ld=8), 2) == 2                                             # k % 8
+    assert call(op(), 16, None) == 1                                               # SS24_ERR_NULL
+    assert call(op(), 16, MISALIGNED) == 3                                         # SS24_ERR_ALIGN
+    assert call(op(rows=0, ptr=None), 16, None) == 0                               # empty operand

@@ -489,6 +489,68 @@ def test_scale_tiles_random_bytes(ss, rows, cols, batch):
     assert np.array_equal(got.cpu().numpy(), oracle.scale_tiles(src, rows, cols, nb))
 
 
+@pytest.mark.parametrize("b", [2, 4, 8, 16, 32, 64, 128, 256])
+def test_hadamard_matches_oracle(ss, b):
+    """Rotation bit for bit: bf16 and fp32 inputs, several rows, a ragged last
+    warp, rows with ld > k, and a batch."""
+    for rows, k in ((37, 512), (5, 256), (3, 768)):
+        if k % b:
+            continue
+        for xh in (synth.sweep_operand(rows, k, seed=80 + b), synth.gaussian_f32(rows, k, seed=81 + b)):
+            got = ss.hadamard(to_dev(xh), b)
+            torch.cuda.synchronize()
+            assert_same(to_np(got), oracle.hadamard(xh, b), f"rot b={b} {rows}x{k}")
+    xh = synth.sweep_operand(9, 512, seed=82)
+    wide = torch.zeros((9, 640), dtype=torch.bfloat16, device="cuda")
+    wide[:, :512] = to_dev(xh)
+    got = ss.hadamard(wide[:, :512], b)
+    torch.cuda.synchronize()
+    assert_same(to_np(got), oracle.hadamard(xh, b), "rot ld > k")
+    xs = [synth.sweep_operand(6, 256, seed=83 + i) for i in range(3)]
+    got = ss.hadamard(torch.stack([to_dev(v) for v in xs]), b)
+    torch.cuda.synchronize()
+    for i, v in enumerate(xs):
+        assert_same(to_np(got[i]), oracle.hadamard(v, b), f"rot batch {i}")
+
+
+@pytest.mark.parametrize("fmt,bits,group", [("fp8", 8, 0), ("nvfp4", 4, 0), ("int", 8, 0)])
+def test_rotated_pass_matches_oracle(ss, ws, fmt, bits, group):
+    """A rotated pass: the rotation on the GPU feeding a fused 2:4 pass on the
+    rotated fp32 operand, against the oracle's pass on its own rotation."""
+    xh = synth.linear_input(64, 1024, seed=84)[0]
+    rot = ss.hadamard(to_dev(xh), 128)
+    out = ss.run(rot, pattern=24, fmt=fmt, bits=bits, group=group, ws=ws)
+    torch.cuda.synchronize()
+    ref = oracle.run(oracle.hadamard(xh, 128), pattern=oracle.SPARSE_24, fmt=fmt, bits=bits, group=group)
+    assert_same(to_np(out["values"]), ref["values"], "values")
+    assert_same(to_np(out["meta"]), ref["meta"], "meta")
+    assert_energy(out["energy"], ref["energy"])
+
+
+def test_rotation_raises_predicted_ratio(ss, ws):
+    """The pages' direction (§4): on a linear input with outlier channels,
+    rotation makes 2:4 relatively worse (R_hat grows), for 2:4 + FP8 against
+    dense FP8 and for 2:4 INT8 against dense INT5 (one scale per row)."""
+    x = to_dev(synth.linear_input(512, 4096, seed=85)[0])
+    rot = ss.hadamard(x, 128)
+    for sp, de in ((("fp8", 8), ("fp8", 8)), (("int", 8), ("int", 5))):
+        r = []
+        for inp in (x, rot):
+            es = ss.run(inp, pattern=24, fmt=sp[0], bits=sp[1], ws=ws)["energy"]
+            ed = ss.run(inp, pattern=0, fmt=de[0], bits=de[1], ws=ws)["energy"]
+            r.append(ss.predicted_ratio(es, ed)[3].item())
+        assert r[1] > r[0], (sp, de, r)
+    # i.i.d. Gaussian data is rotation invariant in distribution: R_hat unchanged
+    g = to_dev(synth.gaussian_bf16(32768, 128, seed=86))
+    for inp_pair in ((g, ss.hadamard(g, 128)),):
+        r = []
+        for inp in inp_pair:
+            es = ss.run(inp, pattern=24, fmt="fp8", ws=ws)["energy"]
+            ed = ss.run(inp, pattern=0, fmt="int", bits=5, ws=ws)["energy"]
+            r.append(ss.predicted_ratio(es, ed)[3].item())
+        assert abs(r[1] / r[0] - 1) < 0.02, r
+
+
 @pytest.mark.parametrize("sparse,dense", [(("fp8",), ("int", 5, 128)), (("nvfp4",), ("mxfp4",)),
                                           (("int", 8, 0), ("int", 5, 0))])
 def test_measured_ratio_against_oracle_and_prediction(ss, ws, sparse, dense):
