@@ -14,8 +14,11 @@
 // in lane ^ (h / 8) of the same warp: strides 1, 2, 4 run in registers and
 // strides 8..128 through warp shuffles, the lower lane taking own + partner
 // and the upper lane partner - own (the pair's y_i - y_i+h). The output is
-// fp32, packed [batch, rows, k]. The launch reads 2 (bf16) or 4 (fp32) and
+// fp32, packed [batch, rows, k], each lane's 32 bytes in one 256-bit store when
+// the output is 32-byte aligned. The launch reads 2 (bf16) or 4 (fp32) and
 // writes 4 bytes per element: HBM-bound.
+#include <type_traits>
+
 #include "device.cuh"
 #include "internal.cuh"
 
@@ -36,14 +39,16 @@ struct RotParams {
     float cb;
 };
 
-__device__ __forceinline__ void bfly(float &a, float &c)
+// One 32-byte store of 8 floats (sm_100 256-bit vector store; dst 32-byte aligned).
+__device__ __forceinline__ void st_v8(float *dst, const float (&v)[8])
 {
-    const float s = __fadd_rn(a, c), d = __fsub_rn(a, c);
-    a = s;
-    c = d;
+    asm volatile("st.global.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "f"(v[0]), "f"(v[1]),
+                 "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7])
+                 : "memory");
 }
 
-template <bool BF16> __global__ void __launch_bounds__(kRotThreads) hadamard_kernel(const __grid_constant__ RotParams p)
+template <bool BF16, bool V8, bool LIN>
+__global__ void __launch_bounds__(kRotThreads) hadamard_kernel(const __grid_constant__ RotParams p)
 {
     grid_dependency_wait();
     grid_dependents_launch();
@@ -56,9 +61,15 @@ template <bool BF16> __global__ void __launch_bounds__(kRotThreads) hadamard_ker
         const bool ok = c < p.chunks;
         float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         if (ok) {
-            const int64_t grow = c / p.cpr, c8 = c - grow * p.cpr;
-            const int64_t op = grow / p.rows, r = grow - op * p.rows;
-            const uint8_t *src = p.x + (op * p.bstride + r * p.ld + 8 * c8) * p.esize;
+            // LIN: rows packed (ld == k) and operands packed, so chunk c starts
+            // at element 8c; otherwise row and operand come from c
+            int64_t e = 8 * c;
+            if constexpr (!LIN) {
+                const int64_t grow = c / p.cpr, c8 = c - grow * p.cpr;
+                const int64_t op = grow / p.rows, r = grow - op * p.rows;
+                e = op * p.bstride + r * p.ld + 8 * c8;
+            }
+            const uint8_t *src = p.x + e * p.esize;
             if constexpr (BF16) {
                 const uint4 w = *reinterpret_cast<const uint4 *>(src);
                 const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
@@ -74,33 +85,54 @@ template <bool BF16> __global__ void __launch_bounds__(kRotThreads) hadamard_ker
                 y[4] = b.x, y[5] = b.y, y[6] = b.z, y[7] = b.w;
             }
         }
-        // strides 1, 2, 4 inside the chunk
+        // strides 1, 2, 4 inside the chunk: two butterflies per packed add and subtract
 #pragma unroll
         for (int s = 0; s < 3; ++s) {
             if (s >= p.log2b)
                 break;
             const int h = 1 << s;
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                if ((i & h) == 0)
-                    bfly(y[i], y[i + h]);
+            for (int i0 = 0; i0 < 8; i0 += 2 * h) {
+                if (h == 1 && (i0 & 2))
+                    continue; // (stride 1 pairs two butterflies 2 apart)
+#pragma unroll
+                for (int j = 0; j < (h == 1 ? 1 : h); j += 2) {
+                    // butterflies (a, a + h) and (b, b + h), a and b the pair's lower indices
+                    const int a = h == 1 ? i0 : i0 + j, b = h == 1 ? i0 + 2 : i0 + j + 1;
+                    const f32x2 lo = pack2(y[a], y[b]), hi = pack2(y[a + h], y[b + h]);
+                    const f32x2 sm = add2(lo, hi), df = sub2(lo, hi);
+                    y[a] = lo2(sm), y[b] = hi2(sm), y[a + h] = lo2(df), y[b + h] = hi2(df);
+                }
+            }
         }
-        // strides 8 .. b/2 across lanes (the whole warp takes part)
+        // strides 8 .. b/2 across lanes (the whole warp takes part): own * (+-1)
+        // + partner is exactly the rounded own + partner (lower lane) or
+        // partner - own (upper lane), one packed fused multiply-add per pair
         for (int s = 3; s < p.log2b; ++s) {
             const int m = 1 << (s - 3);
-            const bool upper = (lane & m) != 0;
+            const float sg = (lane & m) ? -1.0f : 1.0f;
+            const f32x2 sg2 = pack2(sg, sg);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float o = __shfl_xor_sync(0xffffffffu, y[i], m);
-                y[i] = upper ? __fsub_rn(o, y[i]) : __fadd_rn(y[i], o);
+            for (int i = 0; i < 8; i += 2) {
+                const float o0 = __shfl_xor_sync(0xffffffffu, y[i], m);
+                const float o1 = __shfl_xor_sync(0xffffffffu, y[i + 1], m);
+                const f32x2 r = fma2(pack2(y[i], y[i + 1]), sg2, pack2(o0, o1));
+                y[i] = lo2(r), y[i + 1] = hi2(r);
             }
         }
         if (ok) {
-            float4 *dst = reinterpret_cast<float4 *>(p.out + 8 * c);
-            dst[0] = make_float4(__fmul_rn(y[0], p.cb), __fmul_rn(y[1], p.cb), __fmul_rn(y[2], p.cb),
-                                 __fmul_rn(y[3], p.cb));
-            dst[1] = make_float4(__fmul_rn(y[4], p.cb), __fmul_rn(y[5], p.cb), __fmul_rn(y[6], p.cb),
-                                 __fmul_rn(y[7], p.cb));
+            float o[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                o[i] = __fmul_rn(y[i], p.cb);
+            if constexpr (V8) {
+                // a warp's 32 stores cover 1 KB of contiguous output
+                st_v8(p.out + 8 * c, o);
+            } else {
+                float4 *dst = reinterpret_cast<float4 *>(p.out + 8 * c);
+                dst[0] = make_float4(o[0], o[1], o[2], o[3]);
+                dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+            }
         }
     }
 }
@@ -141,8 +173,20 @@ cudaError_t launch_hadamard(const void *x, int bf16, int64_t rows, int64_t k, in
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     void *args[1] = {&p};
-    const void *kern = bf16 ? reinterpret_cast<const void *>(&hadamard_kernel<true>)
-                            : reinterpret_cast<const void *>(&hadamard_kernel<false>);
+    const bool v8 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
+    const bool lin = ld == k && (batch == 1 || bstride == rows * k);
+    const void *kern = nullptr;
+    auto pick = [&](auto b16, auto vec) {
+        constexpr bool B = decltype(b16)::value, V = decltype(vec)::value;
+        kern = lin ? reinterpret_cast<const void *>(&hadamard_kernel<B, V, true>)
+                   : reinterpret_cast<const void *>(&hadamard_kernel<B, V, false>);
+    };
+    using T_ = std::true_type;
+    using F_ = std::false_type;
+    if (bf16)
+        v8 ? pick(T_{}, T_{}) : pick(T_{}, F_{});
+    else
+        v8 ? pick(F_{}, T_{}) : pick(F_{}, F_{});
     return cudaLaunchKernelExC(&cfg, kern, args);
 }
 

@@ -506,6 +506,12 @@ def test_hadamard_matches_oracle(ss, b):
     got = ss.hadamard(wide[:, :512], b)
     torch.cuda.synchronize()
     assert_same(to_np(got), oracle.hadamard(xh, b), "rot ld > k")
+    # an output 16 but not 32 bytes aligned (the two-store path)
+    buf = torch.empty(9 * 512 + 4, dtype=torch.float32, device="cuda")
+    got = ss.hadamard(to_dev(xh), b, out=buf[4:].view(9, 512))
+    torch.cuda.synchronize()
+    assert got.data_ptr() % 32 == 16
+    assert_same(to_np(got), oracle.hadamard(xh, b), "rot out 16-byte aligned")
     xs = [synth.sweep_operand(6, 256, seed=83 + i) for i in range(3)]
     got = ss.hadamard(torch.stack([to_dev(v) for v in xs]), b)
     torch.cuda.synchronize()
