@@ -427,22 +427,29 @@ __device__ __forceinline__ float quant_nvfp4(const float (&v)[VPC], float vmax, 
                                              const NvBlock *blk = nullptr)
 {
     constexpr int kLanes = 16 / VPC;
-    const float amax = gamax >= 0.0f ? gamax : group_amax(vmax, kLanes);
     uint32_t sb = 0;
     Recip rd;
+    bool fast;
     if (blk) {
+        // the block's owner took quot_fast once: a non-positive reciprocal
+        // marks a block for the IEEE division
         rd.b = blk->den;
         rd.y = blk->inv;
+        rd.nb = -rd.b;
+        rd.fast = true;
+        fast = blk->inv > 0.0f;
     } else {
+        const float amax = gamax >= 0.0f ? gamax : group_amax(vmax, kLanes);
         sb = nv_block_code(amax, rst);
         rd.b = tb.den[sb];
         rd.y = tb.inv[sb];
+        rd.nb = -rd.b;
+        rd.fast = rd.b >= 0x1p-60f && rd.b <= 0x1p60f;
+        fast = quot_fast(rd, amax);
     }
-    rd.nb = -rd.b;
-    rd.fast = rd.b >= 0x1p-60f && rd.b <= 0x1p60f;
     const float denom = rd.b;
     float qn[VPC], d[VPC];
-    neg_quotients<VPC>(v, rd, quot_fast(rd, amax), qn);
+    neg_quotients<VPC>(v, rd, fast, qn);
     const uint32_t codes = pack_e2m1<VPC>(qn) ^ (VPC == 4 ? 0x8888u : 0x88888888u);
     unpack_e2m1<VPC>(codes, denom, d);
     store_fp4<VPC, STORE>(codes, o);
@@ -1378,26 +1385,53 @@ __device__ __forceinline__ void stream_unit(const PassParams &p, const PassConst
         // and its reciprocal. (Full-width units: one row per slot, so block
         // j's scale byte is j - lane / 4 bytes from this lane's own.)
         constexpr int VPC = PAT == kDense ? 8 : 4;
+        // bf16 2:4 by magnitude: the block maxima on packed kept pairs (one
+        // conversion per block instead of one per chunk)
+        constexpr bool kPk = sizeof(T) == 2 && PAT == kSparse24 && SCORE == kMag;
         Sel<VPC> sl[4];
-        float g[4];
+        const int bs_ = lane >> 3, bj = lane & 7;
+        float am;
+        if constexpr (kPk) {
+            uint32_t g2[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            sl[i] = select_chunk<T, PAT, SCORE>(raw[i], out_i(i));
-            g[i] = sl[i].vmax;
-        }
+            for (int i = 0; i < 4; ++i) {
+                sl[i] = select_chunk<T, PAT, SCORE>(raw[i], out_i(i));
+                g2[i] = bf16x2_maxabs(sl[i].k0, sl[i].k1);
+            }
 #pragma unroll
-        for (int off = 1; off < 4; off <<= 1)
+            for (int off = 1; off < 4; off <<= 1)
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    g2[i] = bf16x2_maxabs(g2[i], __shfl_xor_sync(kFull, g2[i], off));
+            uint32_t t2[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                g[i] = fmaxf(g[i], __shfl_xor_sync(kFull, g[i], off));
-        const int bs_ = lane >> 3, bj = lane & 7;
-        float t[4];
+                t2[i] = __shfl_sync(kFull, g2[i], 4 * bj);
+            am = bf16x2_hmax(bs_ == 0 ? t2[0] : bs_ == 1 ? t2[1] : bs_ == 2 ? t2[2] : t2[3]);
+        } else {
+            float g[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            t[i] = __shfl_sync(kFull, g[i], 4 * bj);
-        const float am = bs_ == 0 ? t[0] : bs_ == 1 ? t[1] : bs_ == 2 ? t[2] : t[3];
+            for (int i = 0; i < 4; ++i) {
+                sl[i] = select_chunk<T, PAT, SCORE>(raw[i], out_i(i));
+                g[i] = sl[i].vmax;
+            }
+#pragma unroll
+            for (int off = 1; off < 4; off <<= 1)
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    g[i] = fmaxf(g[i], __shfl_xor_sync(kFull, g[i], off));
+            float t[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                t[i] = __shfl_sync(kFull, g[i], 4 * bj);
+            am = bs_ == 0 ? t[0] : bs_ == 1 ? t[1] : bs_ == 2 ? t[2] : t[3];
+        }
         const uint32_t sb = nv_block_code(am, c.rst);
-        const float den = c.tb.den[sb], inv = c.tb.inv[sb];
+        const float den = c.tb.den[sb];
+        // quot_fast for the block, once: its chunks' lanes read the verdict
+        // from the reciprocal's sign
+        const bool bfast = den >= 0x1p-60f && den <= 0x1p60f && __fmul_rn(am, c.tb.inv[sb]) < 0x1p126f;
+        const float inv = bfast ? c.tb.inv[sb] : -1.0f;
         {
             // the block's scale byte: block bj of chunk bs_, 8 bytes per chunk slot
             const ChunkOut ob_ = out_i(bs_);
@@ -1411,7 +1445,7 @@ __device__ __forceinline__ void stream_unit(const PassParams &p, const PassConst
             const int src = 8 * i + (lane >> 2);
             b.den = __shfl_sync(kFull, den, src);
             b.inv = __shfl_sync(kFull, inv, src);
-            finish_chunk<T, PAT, SCORE, FMT>(p, raw[i], sl[i], out_i(i), c, acc, -1.0f, nullptr, g[i], &b);
+            finish_chunk<T, PAT, SCORE, FMT>(p, raw[i], sl[i], out_i(i), c, acc, -1.0f, nullptr, 0.0f, &b);
         }
     } else {
 #pragma unroll
