@@ -58,14 +58,20 @@ def algorithmic_bytes(m=M, k=K):
     }
 
 
+# The sources the step's kernels are built from: the stream kernel (its
+# template, helpers, dispatch and bf16 instantiations), the ratio kernel and the
+# launch code. The ncu traffic figures are valid while these hash the same.
+STEP_KERNEL_SOURCES = ("device.cuh", "internal.cuh", "pass_impl.cuh", "pass_dispatch.cuh", "pass_bf16.cu",
+                       "misc.cu", "abi.cu")
+
+
 def kernel_source_sha():
-    """Hash of the CUDA sources (the ncu traffic figures are valid for one)."""
-    import glob
+    """Hash of the step kernels' CUDA sources (the ncu traffic figures are valid for one)."""
     import hashlib
     h = hashlib.sha256()
     src = os.path.join(ROOT, "semi_structured_sparsity_online_b200", "csrc")
-    for f in sorted(glob.glob(os.path.join(src, "*.cu")) + glob.glob(os.path.join(src, "*.cuh"))):
-        with open(f, "rb") as fh:
+    for name in STEP_KERNEL_SOURCES:
+        with open(os.path.join(src, name), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
@@ -519,7 +525,7 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ss24", "reference"], default="ss24")
-    ap.add_argument("--cpu-rows", type=int, default=96)
+    ap.add_argument("--cpu-rows", type=int, default=4096)
     ap.add_argument("--ref-rows", type=int, default=8, help="rows of one operand per reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
