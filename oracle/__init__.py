@@ -74,6 +74,11 @@ def lib():
         _lib.oracle_hadamard.restype = ctypes.c_int
         _lib.oracle_hadamard.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                          ctypes.c_int32, ctypes.c_void_p]
+        _lib.oracle_exp_ss.restype = ctypes.c_float
+        _lib.oracle_exp_ss.argtypes = [ctypes.c_float]
+        _lib.oracle_softmax_bf16.restype = ctypes.c_int
+        _lib.oracle_softmax_bf16.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                             ctypes.c_float, ctypes.c_void_p]
         _lib.oracle_amax.argtypes = [ctypes.POINTER(_Args)]
         _lib.oracle_tensor_scale.restype = ctypes.c_float
         _lib.oracle_tensor_scale.argtypes = [ctypes.POINTER(_Args)]
@@ -251,6 +256,20 @@ def hadamard(x, block):
     out = np.empty_like(f)
     if f.size and lib().oracle_hadamard(f.ctypes.data, rows, k, k, int(block), out.ctypes.data) != 0:
         raise ValueError("oracle_hadamard rejected its arguments")
+    return out
+
+
+def softmax_bf16(s, alpha):
+    """P = softmax(alpha * s) per row as bf16 bits (see oracle_softmax_bf16) of
+    logits given as bf16 bits (uint16) or float32, [rows, k] or [batch, rows, k]."""
+    a = np.asarray(s)
+    f = (a.astype(np.uint32) << 16).view(np.float32) if a.dtype == np.uint16 else a.astype(np.float32)
+    f = np.ascontiguousarray(f, dtype=np.float32)
+    k = f.shape[-1]
+    rows = f.size // k
+    out = np.empty(f.shape, dtype=np.uint16)
+    if lib().oracle_softmax_bf16(f.ctypes.data, rows, k, k, float(alpha), out.ctypes.data) != 0:
+        raise ValueError("oracle_softmax_bf16 rejected its arguments")
     return out
 
 

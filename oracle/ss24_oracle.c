@@ -832,3 +832,105 @@ int oracle_hadamard(const float *x, int64_t rows, int64_t k, int64_t ld, int32_t
     }
     return 0;
 }
+
+/* ---- attention probabilities: P = softmax(alpha * s) per row ----------------
+ * The producer of an attention operand (§3: "P" pruned along the key axis;
+ * the pages build it as softmax(N(0, 3) logits / sqrt(128))). A fused
+ * producer computes P and prunes it in the same pass; for its results to be
+ * reproducible bit for bit, the exponential and the order of the row sum are
+ * fixed here (the pages leave both open):
+ *   v_j = RN(alpha * s_j); m = max_j v_j; e_j = exp_ss(RN(v_j - m));
+ *   S = sum of the 256-element slices' sums, left to right, each slice summed
+ *       pairwise in index order (adjacent pairs, then adjacent pairs of pairs);
+ *   p_j = RN(e_j / S), then rounded to bf16 (nearest even): the bf16 operand
+ *   the pass prunes.
+ * exp_ss(x), x <= 0, binary32: Cody and Waite's argument reduction (W. J. Cody,
+ * W. Waite, "Software Manual for the Elementary Functions", 1980) with
+ * n = rint(RN(x * log2 e)), r = fma(-n, ln2_hi, x), r = fma(-n, ln2_lo, r)
+ * (ln2_hi = 0.693145751953125 exactly, ln2_lo = RN(ln 2 - ln2_hi)); e^r by the
+ * Taylor polynomial of degree 7 in Horner form with fused multiply-adds
+ * (coefficients RN(1/k!)); then times 2^n (one rounding where the result is
+ * subnormal). x < -103 gives 0 (e^-103 is below 2^-148). */
+float oracle_exp_ss(float x)
+{
+    if (x < -103.0f)
+        return 0.0f;
+    const float log2e = 1.44269502162933349609375f; /* RN(log2 e), 0x3fb8aa3b */
+    const float ln2_hi = 0.693145751953125f;          /* 0x3f317200 */
+    const float ln2_lo = 1.428606765330187e-06f;      /* 0x35bfbe8e */
+    float t = x * log2e;
+    float n = rintf(t);
+    float r = fmaf(-n, ln2_hi, x);
+    r = fmaf(-n, ln2_lo, r);
+    const float c7 = 1.98412701138295233249664306640625e-04f; /* RN(1/5040) */
+    const float c6 = 1.38888892251998186111450195312500e-03f; /* RN(1/720) */
+    const float c5 = 8.33333376795053482055664062500000e-03f; /* RN(1/120) */
+    const float c4 = 4.16666679084300994873046875000000e-02f; /* RN(1/24) */
+    const float c3 = 1.66666671633720397949218750000000e-01f; /* RN(1/6) */
+    float p = c7;
+    p = fmaf(p, r, c6);
+    p = fmaf(p, r, c5);
+    p = fmaf(p, r, c4);
+    p = fmaf(p, r, c3);
+    p = fmaf(p, r, 0.5f);
+    p = fmaf(p, r, 1.0f);
+    p = fmaf(p, r, 1.0f);
+    int ni = (int)n;
+    union {
+        uint32_t u;
+        float f;
+    } s2;
+    if (ni >= -126)
+        s2.u = (uint32_t)(ni + 127) << 23;
+    else
+        s2.u = 1u << (ni + 149);
+    return p * s2.f;
+}
+
+static uint16_t f32_to_bf16_rne(float f)
+{
+    union {
+        float f;
+        uint32_t u;
+    } v;
+    v.f = f;
+    return (uint16_t)((v.u + 0x7fffu + ((v.u >> 16) & 1u)) >> 16); /* finite inputs */
+}
+
+/* s: rows x k logits (row stride ld), fp32 values (a bf16 operand widened
+ * exactly); k a multiple of 256. p_bits: rows x k bf16 bit patterns. */
+int oracle_softmax_bf16(const float *s, int64_t rows, int64_t k, int64_t ld, float alpha, uint16_t *p_bits)
+{
+    if (!s || !p_bits || rows < 0 || k <= 0 || k % 256 != 0 || ld < k)
+        return -1;
+    float *e = (float *)malloc((size_t)k * sizeof(float));
+    if (!e)
+        return -1;
+    for (int64_t r = 0; r < rows; ++r) {
+        const float *row = s + r * ld;
+        float m = alpha * row[0];
+        for (int64_t j = 1; j < k; ++j) {
+            float v = alpha * row[j];
+            if (v > m)
+                m = v;
+        }
+        for (int64_t j = 0; j < k; ++j) {
+            float v = alpha * row[j];
+            e[j] = oracle_exp_ss(v - m);
+        }
+        float total = 0.0f;
+        for (int64_t t0 = 0; t0 < k; t0 += 256) {
+            float buf[256];
+            for (int i = 0; i < 256; ++i)
+                buf[i] = e[t0 + i];
+            for (int w = 256; w > 1; w /= 2) /* pairwise: adjacent pairs first */
+                for (int i = 0; i < w / 2; ++i)
+                    buf[i] = buf[2 * i] + buf[2 * i + 1];
+            total = t0 == 0 ? buf[0] : total + buf[0];
+        }
+        for (int64_t j = 0; j < k; ++j)
+            p_bits[r * k + j] = f32_to_bf16_rne(e[j] / total);
+    }
+    free(e);
+    return 0;
+}

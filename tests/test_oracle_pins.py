@@ -641,3 +641,43 @@ def test_hadamard_is_an_involution_and_rejects_bad_blocks():
             oracle.hadamard(xf, b)
     with pytest.raises(ValueError):
         oracle.hadamard(synth.gaussian_f32(2, 24, seed=1), 16)   # k not a multiple of b
+
+
+def test_exp_ss_within_one_ulp_of_libm():
+    """The softmax exponential (Cody-Waite reduction, degree-7 Taylor
+    polynomial) against libm's exp in binary64: at most 1 ulp of the binary32
+    result where it is normal, one subnormal unit below; exact at 0; zero
+    below -103."""
+    L = oracle.lib()
+    rng = np.random.default_rng(0)
+    xs = np.concatenate([np.linspace(-103, 0, 20001, dtype=np.float32), -rng.exponential(4, 20000).astype(np.float32),
+                         np.float32([-1e-30, -1e-8, -0.34657359, -0.34657362, -87.0, -102.99])])
+    for x in xs[xs >= -103]:
+        f, ref = L.oracle_exp_ss(float(x)), math.exp(float(x))
+        if ref >= 2.0 ** -126:
+            assert abs(f - ref) <= 2.0 ** (math.floor(math.log2(f)) - 23), x
+        else:
+            assert abs(f - ref) <= 2.0 ** -149, x
+    assert L.oracle_exp_ss(0.0) == 1.0 and L.oracle_exp_ss(-103.5) == 0.0
+
+
+def test_softmax_bf16_against_library_and_closed_forms():
+    """P against scipy's softmax in binary64 (within bf16 rounding plus the
+    binary32 steps), rows summing to 1, and two closed forms: a constant row
+    gives exactly 1/k, and a row with one logit far above the rest gives 1 there."""
+    from scipy.special import softmax
+    rng = np.random.default_rng(3)
+    s = (rng.standard_normal((6, 512)) * 3).astype(np.float32)
+    alpha = 1.0 / math.sqrt(128)
+    p = ((oracle.softmax_bf16(s, alpha).astype(np.uint32) << 16).view(np.float32)).astype(np.float64)
+    ref = softmax(s.astype(np.float64) * np.float32(alpha), axis=1)
+    assert np.all(np.abs(p - ref) <= 2.0 ** -8 * ref + 1e-38)
+    assert np.all(np.abs(p.sum(axis=1) - 1) < 512 * 2.0 ** -9 * ref.max())
+    const = oracle.softmax_bf16(np.full((2, 1024), 0.7, dtype=np.float32), 1.0)
+    assert np.all(const == 0x3A80)                                 # 1/1024 = 2^-10 in bf16
+    spike = np.zeros((1, 256), dtype=np.float32)
+    spike[0, 77] = 200.0
+    ps = (oracle.softmax_bf16(spike, 1.0).astype(np.uint32) << 16).view(np.float32)[0]
+    assert ps[77] == 1.0 and np.count_nonzero(ps) == 1
+    with pytest.raises(ValueError):
+        oracle.softmax_bf16(np.zeros((2, 200), dtype=np.float32), 1.0)   # k not a multiple of 256
