@@ -844,47 +844,48 @@ int oracle_hadamard(const float *x, int64_t rows, int64_t k, int64_t ld, int32_t
  *       pairwise in index order (adjacent pairs, then adjacent pairs of pairs);
  *   p_j = RN(e_j / S), then rounded to bf16 (nearest even): the bf16 operand
  *   the pass prunes.
- * exp_ss(x), x <= 0, binary32: Cody and Waite's argument reduction (W. J. Cody,
- * W. Waite, "Software Manual for the Elementary Functions", 1980) with
- * n = rint(RN(x * log2 e)), r = fma(-n, ln2_hi, x), r = fma(-n, ln2_lo, r)
- * (ln2_hi = 0.693145751953125 exactly, ln2_lo = RN(ln 2 - ln2_hi)); e^r by the
- * Taylor polynomial of degree 7 in Horner form with fused multiply-adds
- * (coefficients RN(1/k!)); then times 2^n (one rounding where the result is
- * subnormal). x < -103 gives 0 (e^-103 is below 2^-148). */
+ * exp_ss(x), x <= 0, binary32, after Cody and Waite's argument reduction
+ * (W. J. Cody, W. Waite, "Software Manual for the Elementary Functions", 1980):
+ *   x' = max(x, -104); t = RN(x' log2e); n = RN(RN(t + 1.5 * 2^23) - 1.5 * 2^23)
+ *   (t rounded to an integer, ties to even); r = fma(-n, ln2_hi, x'),
+ *   r = fma(-n, ln2_lo, r) (ln2_hi = 0.693145751953125 exactly,
+ *   ln2_lo = RN(ln 2 - ln2_hi)); q = the Taylor polynomial of e^r of degree 7
+ *   in Horner form with fused multiply-adds (coefficients RN(1/k!));
+ *   exp_ss = RN(RN(q * 2^(n + 64)) * 2^-64), i.e. q * 2^n rounded once (the
+ *   first product is exact). At x' = -104 the result rounds to 0. */
 float oracle_exp_ss(float x)
 {
-    if (x < -103.0f)
-        return 0.0f;
+    const float xc = x < -104.0f ? -104.0f : x;
     const float log2e = 1.44269502162933349609375f; /* RN(log2 e), 0x3fb8aa3b */
     const float ln2_hi = 0.693145751953125f;          /* 0x3f317200 */
     const float ln2_lo = 1.428606765330187e-06f;      /* 0x35bfbe8e */
-    float t = x * log2e;
-    float n = rintf(t);
-    float r = fmaf(-n, ln2_hi, x);
+    const float magic = 12582912.0f;                  /* 1.5 * 2^23 */
+    float t = xc * log2e;
+    float tm = t + magic;
+    float n = tm - magic;
+    float r = fmaf(-n, ln2_hi, xc);
     r = fmaf(-n, ln2_lo, r);
     const float c7 = 1.98412701138295233249664306640625e-04f; /* RN(1/5040) */
     const float c6 = 1.38888892251998186111450195312500e-03f; /* RN(1/720) */
     const float c5 = 8.33333376795053482055664062500000e-03f; /* RN(1/120) */
     const float c4 = 4.16666679084300994873046875000000e-02f; /* RN(1/24) */
     const float c3 = 1.66666671633720397949218750000000e-01f; /* RN(1/6) */
-    float p = c7;
-    p = fmaf(p, r, c6);
-    p = fmaf(p, r, c5);
-    p = fmaf(p, r, c4);
-    p = fmaf(p, r, c3);
-    p = fmaf(p, r, 0.5f);
-    p = fmaf(p, r, 1.0f);
-    p = fmaf(p, r, 1.0f);
-    int ni = (int)n;
+    float q = c7;
+    q = fmaf(q, r, c6);
+    q = fmaf(q, r, c5);
+    q = fmaf(q, r, c4);
+    q = fmaf(q, r, c3);
+    q = fmaf(q, r, 0.5f);
+    q = fmaf(q, r, 1.0f);
+    q = fmaf(q, r, 1.0f);
+    const int ni = (int)n; /* in [-150, 0] */
     union {
         uint32_t u;
         float f;
     } s2;
-    if (ni >= -126)
-        s2.u = (uint32_t)(ni + 127) << 23;
-    else
-        s2.u = 1u << (ni + 149);
-    return p * s2.f;
+    s2.u = (uint32_t)(ni + 64 + 127) << 23; /* 2^(n + 64), normal */
+    float up = q * s2.f;
+    return up * 0x1p-64f;
 }
 
 static uint16_t f32_to_bf16_rne(float f)

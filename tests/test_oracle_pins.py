@@ -646,19 +646,19 @@ def test_hadamard_is_an_involution_and_rejects_bad_blocks():
 def test_exp_ss_within_one_ulp_of_libm():
     """The softmax exponential (Cody-Waite reduction, degree-7 Taylor
     polynomial) against libm's exp in binary64: at most 1 ulp of the binary32
-    result where it is normal, one subnormal unit below; exact at 0; zero
-    below -103."""
+    result where it is normal, one subnormal unit below; exact at 0; zero at
+    and below -104."""
     L = oracle.lib()
     rng = np.random.default_rng(0)
-    xs = np.concatenate([np.linspace(-103, 0, 20001, dtype=np.float32), -rng.exponential(4, 20000).astype(np.float32),
-                         np.float32([-1e-30, -1e-8, -0.34657359, -0.34657362, -87.0, -102.99])])
-    for x in xs[xs >= -103]:
+    xs = np.concatenate([np.linspace(-104, 0, 20001, dtype=np.float32), -rng.exponential(4, 20000).astype(np.float32),
+                         np.float32([-1e-30, -1e-8, -0.34657359, -0.34657362, -86.9, -87.0, -102.99, -103.5])])
+    for x in xs[xs >= -104]:
         f, ref = L.oracle_exp_ss(float(x)), math.exp(float(x))
         if ref >= 2.0 ** -126:
             assert abs(f - ref) <= 2.0 ** (math.floor(math.log2(f)) - 23), x
         else:
             assert abs(f - ref) <= 2.0 ** -149, x
-    assert L.oracle_exp_ss(0.0) == 1.0 and L.oracle_exp_ss(-103.5) == 0.0
+    assert L.oracle_exp_ss(0.0) == 1.0 and L.oracle_exp_ss(-104.0) == 0.0 and L.oracle_exp_ss(-1e30) == 0.0
 
 
 def test_softmax_bf16_against_library_and_closed_forms():
