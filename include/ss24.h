@@ -440,6 +440,33 @@ ss24_status ss24_selfcheck_division(int32_t mode, uint32_t b_first, uint32_t b_c
 ss24_status ss24_selfcheck_encoder(int32_t kind, const uint32_t *bounds, int32_t n_bounds, uint32_t hi_first,
                                    uint32_t hi_count, unsigned long long *result, ss24_stream stream);
 
+/* ---- pruning in the producer: attention probabilities ------------------------ */
+
+/* P = softmax(alpha * s) per row, pruned and compressed along the key axis in
+ * the same pass (§3: P pruned along the key axis; §1: an operand computed on
+ * the fly is pruned before every GEMM): P is never stored. s: logits, bf16 or
+ * fp32, axis 1 (keys contiguous), k (keys) a multiple of 256, ld and batch as
+ * for the passes. The arithmetic, fixed so that results reproduce bit for bit
+ * (the pages leave it open): v = RN(alpha s); m = the row max; e = exp_ss(RN(v -
+ * m)); S = the row's 256-key slice sums added left to right, each slice summed
+ * pairwise in index order; p = RN(e / S) rounded to bf16 (nearest even).
+ * exp_ss: arguments below -104 taken as -104; Cody-Waite reduction (n = t
+ * rounded to an integer, ties to even; ln 2 split into an exact high part and
+ * a rounded low part), the degree-7 Taylor polynomial with coefficients
+ * RN(1/k!) in fused multiply-add Horner form, times 2^n rounded once. The
+ * bf16 P then goes through exactly what ss24_prune24_quant_fused (2:4), the
+ * pairwise 4:8 pass or a dense quantization does to a bf16 operand by
+ * magnitude: same outputs (layouts of ss24_outputs), same energies. Formats:
+ * NONE (sparse patterns), FP8 and NVFP4 with the tensor scale GIVEN
+ * (tensor_scale_in, device, one per operand; P <= 1, so 1/448 suits FP8),
+ * MXFP4, INT with groups. Errors: the operand and output checks of the passes,
+ * SS24_ERR_ARG (axis 0, alpha not finite), SS24_ERR_SHAPE (k not a multiple of
+ * 256), SS24_ERR_FORMAT (INT with one scale per row), SS24_ERR_NULL (no
+ * tensor scale for FP8 / NVFP4). */
+ss24_status ss24_softmax_prune(const ss24_operand *s, float alpha, ss24_pattern pattern, ss24_format fmt,
+                               const float *tensor_scale_in, ss24_outputs *out, ss24_energy *energy, void *ws,
+                               size_t ws_bytes, ss24_stream stream);
+
 /* ---- rotation ----------------------------------------------------------------- */
 
 /* Block Hadamard rotation along k (§4: a Hadamard matrix, orthogonal with

@@ -973,6 +973,75 @@ ss24_status ss24_dequantize(const ss24_operand *x, ss24_pattern pattern, ss24_fo
                                       in->meta, xhat, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+ss24_status ss24_softmax_prune(const ss24_operand *s, float alpha, ss24_pattern pattern, ss24_format fmt,
+                               const float *tensor_scale_in, ss24_outputs *out, ss24_energy *energy, void *ws,
+                               size_t ws_bytes, ss24_stream stream)
+{
+    ss24_status st = check_operand(s);
+    if (st != SS24_OK)
+        return st;
+    if (s->axis != 1 || !std::isfinite(alpha))
+        return SS24_ERR_ARG;
+    if ((st = check_pattern_k(pattern, s->k)) != SS24_OK)
+        return st;
+    if (s->k % 256 != 0)
+        return SS24_ERR_SHAPE;
+    if ((st = check_ws(ws, ws_bytes)) != SS24_OK)
+        return st;
+    Resolved r;
+    if ((st = resolve_format(fmt, pattern, s->k, true, &r)) != SS24_OK)
+        return st;
+    if (r.row_mode)
+        return SS24_ERR_FORMAT; // one INT scale per row is not offered here
+    if (!out)
+        return SS24_ERR_NULL;
+    if (per_tensor(fmt.kind) && !tensor_scale_in)
+        return SS24_ERR_NULL; // the tensor scale of P must be given
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    if (s->rows == 0)
+        return empty_operand(s, energy, out, per_tensor(fmt.kind) ? tensor_scale_in : nullptr, cs);
+    const bool needs_scales = fmt.kind == SS24_FMT_INT || fmt.kind == SS24_FMT_NVFP4 || fmt.kind == SS24_FMT_MXFP4;
+    if (!out->values || (needs_scales && !out->scales) || (per_tensor(fmt.kind) && !out->tensor_scale) ||
+        (pattern != SS24_DENSE && !out->meta))
+        return SS24_ERR_NULL;
+    if (!aligned16(out->values) || (needs_scales && !aligned16(out->scales)) ||
+        (pattern != SS24_DENSE && !aligned16(out->meta)))
+        return SS24_ERR_ALIGN;
+    PassParams p = base_params(s, stream_geometry(s), ws, energy);
+    output_strides(s, pattern, fmt, &p);
+    p.values = out->values;
+    p.scales = out->scales;
+    p.meta = out->meta;
+    p.q = r.q;
+    if (per_tensor(fmt.kind)) {
+        p.q.scale_in = tensor_scale_in;
+        p.q.scale_out = out->tensor_scale;
+    }
+    const bool smem = s->k <= kSoftmaxSmemKeys;
+    const size_t smem_bytes = smem ? static_cast<size_t>(kStreamWarps) * s->k * sizeof(float) : 0;
+    const void *k = softmax_prune_kernel_ptr(s->dtype == SS24_BF16 ? 1 : 0, pattern, fmt.kind, smem);
+    if (!k)
+        return SS24_ERR_FORMAT;
+    KernelInfo info;
+    // (the dynamic shared memory of the largest row, set once per kernel)
+    cudaError_t e = kernel_info(k, smem ? static_cast<size_t>(kStreamWarps) * kSoftmaxSmemKeys * sizeof(float) : 0,
+                                &info, kStreamThreads);
+    if (e != cudaSuccess)
+        return SS24_ERR_CUDA;
+    if (smem) {
+        int per_sm = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kStreamThreads, smem_bytes);
+        if (e != cudaSuccess)
+            return SS24_ERR_CUDA;
+        info.blocks_per_sm = per_sm;
+    }
+    p.ctas_per_op = static_cast<int32_t>(ctas_per_operand(info, p.batch, (s->rows + kStreamWarps - 1) / kStreamWarps));
+    float a = alpha;
+    void *args[2] = {&p, &a};
+    return cuda_status(
+        launch_pdl(k, static_cast<unsigned>(p.batch * p.ctas_per_op), kStreamThreads, smem_bytes, cs, args));
+}
+
 ss24_status ss24_hadamard(const ss24_operand *x, int32_t block, float *out, ss24_stream stream)
 {
     ss24_status st = check_operand(x);

@@ -126,6 +126,9 @@ cudaError_t launch_dequant(int pattern, int fmt, int32_t store, int32_t lg, int3
                            const uint8_t *meta, float *xhat, cudaStream_t stream);
 cudaError_t launch_hadamard(const void *x, int bf16, int64_t rows, int64_t k, int64_t ld, int64_t bstride,
                             int64_t batch, int32_t block, float *out, cudaStream_t stream);
+// Rows of up to this many keys keep their values in shared memory.
+constexpr int64_t kSoftmaxSmemKeys = 2048;
+const void *softmax_prune_kernel_ptr(int bf16, int pattern, int fmt, bool smem);
 int64_t scale_tiles_bytes(int64_t rows, int64_t cols);
 cudaError_t launch_scale_tiles(const uint8_t *in, int64_t rows, int64_t cols, int64_t batch, uint8_t *out,
                                cudaStream_t stream);

@@ -46,6 +46,8 @@ def pass_bytes(name, m, k):
         return 2 * n
     if name == "hadamard128":
         return 2 * n + 4 * n
+    if name == "softmax_24_fp8":
+        return 2 * n + n // 2 + n // 8     # read the logits; write FP8 codes + metadata of P
     if name == "amax_rows":
         return 2 * n + 4 * m
     if name == "dense_int8_given_rows":
@@ -68,7 +70,7 @@ def pass_bytes(name, m, k):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--pass", dest="name", default="fused_24_fp8", choices=sorted(PASSES) + ["tensor_scale", "error_energy", "amax_rows", "hadamard128",
+    ap.add_argument("--pass", dest="name", default="fused_24_fp8", choices=sorted(PASSES) + ["tensor_scale", "error_energy", "amax_rows", "hadamard128", "softmax_24_fp8",
                                                                        "dense_int8_given_rows"])
     ap.add_argument("--m", type=int, default=4096)
     ap.add_argument("--k", type=int, default=4096)
@@ -105,12 +107,20 @@ def main():
                                   lead)
 
     rot = torch.empty(x.shape, dtype=torch.float32, device="cuda") if args.name == "hadamard128" else None
+    alpha = float(np.float32(1.0 / np.sqrt(128.0)))
+    p_scale = torch.full((nb,), 1.0 / 448.0, device="cuda")
+    if args.name == "softmax_24_fp8":
+        out = ss24._alloc_outputs(args.m, args.k, ss24.SPARSE_24, ss24.make_format("fp8"), torch.bfloat16, "cuda",
+                                  lead)
 
     def once():
         if args.name == "amax_rows":
             ss24.amax_rows(x, scale_fmt="fp8", ws=ws, out=row_amax, scale_out=scale)
         elif args.name == "dense_int8_given_rows":
             ss24.run_int_rows(x, row_amax, bits=8, energy=e, ws=ws, out=out)
+        elif args.name == "softmax_24_fp8":
+            ss24.softmax_prune(x, alpha, pattern=ss24.SPARSE_24, fmt="fp8", tensor_scale=p_scale, energy=e, ws=ws,
+                               out=out)
         elif args.name == "hadamard128":
             ss24.hadamard(x, 128, out=rot)
         elif args.name == "tensor_scale":

@@ -87,6 +87,8 @@ _SIGNATURES = {
                                               _P]),
     "ss24_dequantize": (ctypes.c_int, [_OP, ctypes.c_int, Format, _OUT, _P, _P]),
     "ss24_hadamard": (ctypes.c_int, [_OP, ctypes.c_int32, _P, _P]),
+    "ss24_softmax_prune": (ctypes.c_int, [_OP, ctypes.c_float, ctypes.c_int, Format, _P, _OUT, _P, _P,
+                                          ctypes.c_size_t, _P]),
     "ss24_scale_tiles_bytes": (ctypes.c_int64, [ctypes.c_int64, ctypes.c_int64]),
     "ss24_scale_tiles": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, _P, _P]),
     "ss24_selfcheck_encoder": (ctypes.c_int, [ctypes.c_int32, _P, ctypes.c_int32, ctypes.c_uint32, ctypes.c_uint32,
@@ -364,6 +366,28 @@ def dequantize(out, rows, k, pattern=SPARSE_24, fmt="none", bits=8, group=0, pac
     _check(lib().ss24_dequantize(ctypes.byref(op), pattern, f, ctypes.byref(o), _ptr(xhat), _stream(stream)),
            "ss24_dequantize")
     return xhat
+
+
+def softmax_prune(s: torch.Tensor, alpha: float, pattern=SPARSE_24, fmt="fp8", bits=8, group=0, pack4=False,
+                  tensor_scale=None, energy=True, ws=None, stream=None, out=None):
+    """P = softmax(alpha * s) per row, pruned / quantized in the same pass
+    (ss24_softmax_prune): the same dict as run() for the bf16 operand P, which
+    is never stored. s: logits [rows, keys] or [B, rows, keys], bf16 or fp32."""
+    f = make_format(fmt, bits, group, pack4)
+    op = make_operand(s, 1)
+    if out is None:
+        out = _alloc_outputs(op.rows, op.k, pattern, f, torch.bfloat16, s.device, _lead(op))
+    e = _energy(op, s.device) if energy is True else energy
+    if e is not None and e is not False:
+        out["energy"] = e
+    else:
+        e = None
+    ws = ws or default_workspace(s.device)
+    o = Outputs(*(_ptr(out.get(key)) for key in ("values", "scales", "tensor_scale", "meta")))
+    _check(lib().ss24_softmax_prune(ctypes.byref(op), float(alpha), pattern, f, _ptr(tensor_scale), ctypes.byref(o),
+                                    _ptr(e), ws.ptr, ws.nbytes, _stream(stream)),
+           "ss24_softmax_prune")
+    return out
 
 
 def hadamard(x: torch.Tensor, block: int, out=None, stream=None):

@@ -233,3 +233,24 @@ def test_hadamard_validation():
     assert call(op(), 16, None) == 1                                               # SS24_ERR_NULL
     assert call(op(), 16, MISALIGNED) == 3                                         # SS24_ERR_ALIGN
     assert call(op(rows=0, ptr=None), 16, None) == 0                               # empty operand
+
+
+def test_softmax_prune_validation():
+    L = ss24.lib()
+    ws = ctypes.c_void_p(ALIGNED)
+
+    def op(rows=4, k=512, ld=None, axis=1, ptr=ALIGNED, dtype=ss24.BF16):
+        return ss24.Operand(ptr, dtype, axis, rows, k, ld or k, 0, 0)
+    outs = ss24.Outputs(ALIGNED, ALIGNED, ALIGNED, ALIGNED)
+
+    def call(o, alpha=0.1, pattern=ss24.SPARSE_24, fmt=("fp8",), scale=ALIGNED, wsb=None):
+        f = ss24.make_format(*fmt)
+        return L.ss24_softmax_prune(ctypes.byref(o), alpha, pattern, f, scale, ctypes.byref(outs), None, ws,
+                                    wsb if wsb is not None else _ws_bytes(), None)
+    assert call(op(axis=0, ld=8)) == 8                           # SS24_ERR_ARG: axis 0
+    assert call(op(), alpha=float("nan")) == 8                   # alpha not finite
+    assert call(op(k=264)) == 2                                  # SS24_ERR_SHAPE: keys % 256
+    assert call(op(), fmt=("int", 8, 0)) == 5                    # SS24_ERR_FORMAT: one INT scale per row
+    assert call(op(), fmt=("fp8",), scale=None) == 1             # SS24_ERR_NULL: FP8 needs the given scale
+    assert call(op(), fmt=("none",), pattern=ss24.DENSE) == 5    # dense needs a quantization format
+    assert call(op(), wsb=16) == 6                               # SS24_ERR_WORKSPACE

@@ -2,6 +2,8 @@
 same seeded inputs. Codes, scales, metadata and kept values must match bit for
 bit; energies to 1e-6 relative (the bound the library states for its binary32
 per-element terms summed in binary64)."""
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -555,6 +557,79 @@ def test_rotation_raises_predicted_ratio(ss, ws):
             ed = ss.run(inp, pattern=0, fmt="int", bits=5, ws=ws)["energy"]
             r.append(ss.predicted_ratio(es, ed)[3].item())
         assert abs(r[1] / r[0] - 1) < 0.02, r
+
+
+SOFTMAX_CASES = [(24, "none", 8, 0), (24, "fp8", 8, 0), (24, "nvfp4", 4, 0), (24, "mxfp4", 4, 0),
+                 (24, "int", 8, 32), (48, "nvfp4", 4, 0), (48, "fp8", 8, 0), (0, "fp8", 8, 0), (0, "mxfp4", 4, 0),
+                 (0, "int", 4, 64)]
+
+
+def _logits(rows, keys, seed):
+    return (np.random.default_rng(seed).standard_normal((rows, keys)) * 3.0).astype(np.float32)
+
+
+def _p_scale(fmt):
+    # P <= 1: the FP8 scale 1/448 and the NVFP4 tensor scale 1 / (6 * 448)
+    return {"fp8": np.float32(1.0 / 448.0), "nvfp4": np.float32(1.0 / 2688.0)}.get(fmt)
+
+
+@pytest.mark.parametrize("pattern,fmt,bits,group", SOFTMAX_CASES)
+@pytest.mark.parametrize("logits", ["bf16", "f32"])
+def test_softmax_prune_matches_oracle(ss, ws, pattern, fmt, bits, group, logits):
+    """P = softmax(alpha s) pruned in its producer, against the oracle's softmax
+    followed by the oracle's pass on that bf16 P: outputs bit for bit,
+    energies within 1e-6 (5 slices of 256 keys: a ragged last unit)."""
+    rows, keys, alpha = 37, 1280, float(np.float32(1.0 / math.sqrt(128)))
+    s = _logits(rows, keys, 90 + pattern)
+    sh = synth.bf16_bits(s) if logits == "bf16" else s
+    ts = _p_scale(fmt)
+    tsd = torch.tensor([ts], device="cuda") if ts is not None else None
+    out = ss.softmax_prune(to_dev(sh), alpha, pattern=pattern, fmt=fmt, bits=bits, group=group, tensor_scale=tsd,
+                           ws=ws)
+    torch.cuda.synchronize()
+    P = oracle.softmax_bf16(sh, alpha)
+    opat = {0: oracle.DENSE, 24: oracle.SPARSE_24, 48: oracle.SPARSE_48}[pattern]
+    ref = oracle.run(P, pattern=opat, fmt=fmt, bits=bits, group=group,
+                     **({"tensor_scale": float(ts)} if ts is not None else {}))
+    assert_same(to_np(out["values"]), ref["values"], "values")
+    if pattern:
+        assert_same(to_np(out["meta"]), ref["meta"], "meta")
+    if "scales" in ref and ref["scales"] is not None and out.get("scales") is not None:
+        assert_same(to_np(out["scales"]), ref["scales"], "scales")
+    assert_energy(out["energy"], ref["energy"], atol=1e-30)
+    assert ws.error() == 0
+
+
+def test_softmax_prune_batch_and_shapes(ss, ws):
+    """A batch of three operands, one slice per row, and a long row of 8192 keys."""
+    alpha = float(np.float32(1.0 / math.sqrt(128)))
+    xs = [synth.bf16_bits(_logits(8, 512, 95 + b)) for b in range(3)]
+    ts = torch.full((3,), 1.0 / 448.0, device="cuda")
+    out = ss.softmax_prune(torch.stack([to_dev(v) for v in xs]), alpha, pattern=24, fmt="fp8", tensor_scale=ts, ws=ws)
+    torch.cuda.synchronize()
+    for b, sh in enumerate(xs):
+        ref = oracle.run(oracle.softmax_bf16(sh, alpha), pattern=oracle.SPARSE_24, fmt="fp8",
+                         tensor_scale=float(np.float32(1.0 / 448.0)))
+        assert_same(to_np(out["values"][b]), ref["values"], f"values[{b}]")
+        assert_same(to_np(out["meta"][b]), ref["meta"], f"meta[{b}]")
+        assert_energy(out["energy"][b], ref["energy"], atol=1e-30)
+    # wide logits: arguments below -104 (clamped), subnormal e, quotients below
+    # 2^-40 (the IEEE-division chunks)
+    wide = (np.random.default_rng(98).standard_normal((16, 512)) * 40.0).astype(np.float32)
+    for a in (1.0, alpha):
+        out = ss.softmax_prune(to_dev(wide), a, pattern=24, fmt="fp8", tensor_scale=ts[:1], ws=ws)
+        torch.cuda.synchronize()
+        ref = oracle.run(oracle.softmax_bf16(wide, a), pattern=oracle.SPARSE_24, fmt="fp8",
+                         tensor_scale=float(np.float32(1.0 / 448.0)))
+        assert_same(to_np(out["values"]), ref["values"], f"wide values alpha={a}")
+        assert_same(to_np(out["meta"]), ref["meta"], f"wide meta alpha={a}")
+    for rows, keys in ((3, 256), (2, 8192)):
+        sh = synth.bf16_bits(_logits(rows, keys, 97))
+        out = ss.softmax_prune(to_dev(sh), alpha, pattern=24, fmt="none", ws=ws)
+        torch.cuda.synchronize()
+        ref = oracle.run(oracle.softmax_bf16(sh, alpha), pattern=oracle.SPARSE_24, fmt="none")
+        assert_same(to_np(out["values"]), ref["values"], f"values {rows}x{keys}")
+        assert_same(to_np(out["meta"]), ref["meta"], f"meta {rows}x{keys}")
 
 
 @pytest.mark.parametrize("sparse,dense", [(("fp8",), ("int", 5, 128)), (("nvfp4",), ("mxfp4",)),
