@@ -85,6 +85,18 @@ def attention_probs(heads: int = 32, seq: int = 2048, d: int = 128, seed: int = 
     return out
 
 
+def attention_logits(heads: int = 32, seq: int = 2048, seed: int = 9, logit_std: float = 3.0) -> np.ndarray:
+    """Attention logits [heads * seq, seq] ~ N(0, logit_std^2) in bf16 (the
+    1/sqrt(d) scale is left to the consumer)."""
+    rng = np.random.default_rng(seed)
+    out = np.empty((heads * seq, seq), dtype=np.uint16)
+    step = 4096
+    for r0 in range(0, heads * seq, step):
+        rr = min(step, heads * seq - r0)
+        out[r0:r0 + rr] = bf16_bits(rng.standard_normal((rr, seq), dtype=np.float32) * np.float32(logit_std))
+    return out
+
+
 def sweep_operand(tokens: int, k: int, seed: int = 8, outlier_frac: float = 0.001,
                   outlier_factor: float = 100.0) -> np.ndarray:
     """Throughput-sweep operand [tokens, k]: N(0, 1) with ``outlier_frac`` of the

@@ -876,6 +876,29 @@ def test_full_attention_operands(ss, ws):
     sampled_check(ss, ws, p, pattern=24, fmt="fp8", n_rows=16)
 
 
+def test_full_attention_softmax_prune(ss, ws):
+    """P = softmax(logits / sqrt(128)) for 32 heads x 2048 x 2048 keys, pruned
+    2:4 + FP8 in its producer: sampled rows against the oracle's softmax and
+    pass, bit for bit; energies by properties."""
+    s = synth.attention_logits(seed=9)
+    alpha = float(np.float32(1.0 / math.sqrt(128)))
+    ts = torch.tensor([1.0 / 448.0], device="cuda")
+    out = ss.softmax_prune(to_dev(s), alpha, pattern=24, fmt="fp8", tensor_scale=ts, ws=ws)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(10)
+    rows = np.unique(np.concatenate([[0, s.shape[0] - 1], rng.integers(0, s.shape[0], 16)]))
+    ref = oracle.run(oracle.softmax_bf16(s[rows], alpha), pattern=oracle.SPARSE_24, fmt="fp8",
+                     tensor_scale=float(np.float32(1.0 / 448.0)))
+    sel = torch.from_numpy(rows).cuda()
+    assert_same(to_np(out["values"][sel]), ref["values"], "values")
+    assert_same(to_np(out["meta"][sel]), ref["meta"], "meta")
+    e = out["energy"].cpu().numpy()
+    # each row of P sums to ~1 with 2048 near-equal entries: E_total ~ rows / 2048
+    assert 0.5 * s.shape[0] / 2048 < e[0] < 2.0 * s.shape[0] / 2048
+    assert 0.0 < e[1] / e[0] < 0.5 and 0.0 < e[2] < e[1]
+    assert ws.error() == 0
+
+
 @pytest.mark.parametrize("tokens,k", [(2048, 4096), (16384, 14336)])
 def test_full_sweep_nvfp4(ss, ws, tokens, k):
     xh = synth.sweep_operand(tokens, k, seed=8)
