@@ -79,6 +79,9 @@ def lib():
         _lib.oracle_softmax_bf16.restype = ctypes.c_int
         _lib.oracle_softmax_bf16.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                              ctypes.c_float, ctypes.c_void_p]
+        _lib.oracle_hadamard_bf16.restype = ctypes.c_int
+        _lib.oracle_hadamard_bf16.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                              ctypes.c_int32, ctypes.c_void_p]
         _lib.oracle_amax.argtypes = [ctypes.POINTER(_Args)]
         _lib.oracle_tensor_scale.restype = ctypes.c_float
         _lib.oracle_tensor_scale.argtypes = [ctypes.POINTER(_Args)]
@@ -256,6 +259,19 @@ def hadamard(x, block):
     out = np.empty_like(f)
     if f.size and lib().oracle_hadamard(f.ctypes.data, rows, k, k, int(block), out.ctypes.data) != 0:
         raise ValueError("oracle_hadamard rejected its arguments")
+    return out
+
+
+def hadamard_bf16(x, block):
+    """The rotation as a fused pass applies it (see oracle_hadamard_bf16): bf16
+    bits of the same shape as x (bf16 bits or float32, [rows, k] or [B, rows, k])."""
+    a = np.asarray(x)
+    f = (a.astype(np.uint32) << 16).view(np.float32) if a.dtype == np.uint16 else a.astype(np.float32)
+    f = np.ascontiguousarray(f, dtype=np.float32)
+    k = f.shape[-1]
+    out = np.empty(f.shape, dtype=np.uint16)
+    if f.size and lib().oracle_hadamard_bf16(f.ctypes.data, f.size // k, k, k, int(block), out.ctypes.data) != 0:
+        raise ValueError("oracle_hadamard_bf16 rejected its arguments")
     return out
 
 

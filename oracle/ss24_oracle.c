@@ -935,3 +935,22 @@ int oracle_softmax_bf16(const float *s, int64_t rows, int64_t k, int64_t ld, flo
     free(e);
     return 0;
 }
+
+/* The rotation as a fused pass applies it: oracle_hadamard's binary32 result
+ * rounded to bf16 (nearest even), the operand dtype the pass then prunes and
+ * quantizes (an online rotation feeding a bf16 GEMM stores bf16). out_bits:
+ * rows x k bf16 bit patterns. Returns 0, or -1 as oracle_hadamard. */
+int oracle_hadamard_bf16(const float *x, int64_t rows, int64_t k, int64_t ld, int32_t b, uint16_t *out_bits)
+{
+    if (!x || !out_bits || rows < 0)
+        return -1;
+    float *tmp = (float *)malloc((size_t)(rows > 0 ? rows : 1) * (size_t)k * sizeof(float));
+    if (!tmp)
+        return -1;
+    int rc = oracle_hadamard(x, rows, k, ld, b, tmp);
+    if (rc == 0)
+        for (int64_t i = 0; i < rows * k; ++i)
+            out_bits[i] = f32_to_bf16_rne(tmp[i]);
+    free(tmp);
+    return rc;
+}

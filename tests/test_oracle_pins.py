@@ -681,3 +681,24 @@ def test_softmax_bf16_against_library_and_closed_forms():
     assert ps[77] == 1.0 and np.count_nonzero(ps) == 1
     with pytest.raises(ValueError):
         oracle.softmax_bf16(np.zeros((2, 200), dtype=np.float32), 1.0)   # k not a multiple of 256
+
+
+def test_hadamard_bf16_is_the_nearest_bf16_of_the_rotation():
+    """The fused pass's rotation: each output is the bf16 nearest to the binary32
+    rotation (ties to even), checked against both bf16 neighbours; exact where
+    the rotation is itself a bf16 value (unit vectors, b a power of 4)."""
+    xh = synth.sweep_operand(8, 512, seed=73)
+    for b in (16, 32, 128):
+        rot = oracle.hadamard(xh, b).astype(np.float64)
+        got = ((oracle.hadamard_bf16(xh, b).astype(np.uint32) << 16).view(np.float32)).astype(np.float64)
+        bits = (oracle.hadamard(xh, b).view(np.uint32) >> 16).astype(np.uint32)
+        lo = ((bits << 16).view(np.float32)).astype(np.float64)                  # truncation toward zero
+        hi = (((bits + 1) << 16).view(np.float32)).astype(np.float64)            # next bf16 away from zero
+        d_got, d_lo, d_hi = np.abs(got - rot), np.abs(lo - rot), np.abs(hi - rot)
+        assert np.all(d_got <= np.minimum(d_lo, d_hi))
+        tie = d_lo == d_hi
+        assert np.all(((oracle.hadamard_bf16(xh, b)[tie] & 1) == 0))
+    e = np.zeros((1, 64), dtype=np.float32)
+    e[0, 5] = 1.0
+    got = (oracle.hadamard_bf16(e, 16).astype(np.uint32) << 16).view(np.float32)[0]
+    assert np.array_equal(np.abs(got[:16]), np.full(16, 0.25, dtype=np.float32)) and not got[16:].any()
