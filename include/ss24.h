@@ -168,6 +168,15 @@ typedef struct {
     int64_t batch;        /* operands in the call: 0 or 1 for one, up to 1024      */
     int64_t batch_stride; /* elements from one operand to the next (batch > 1);
                              at least rows * ld (axis 1) or k * ld (axis 0)       */
+    int32_t hadamard;     /* 0, or a block size b (a power of two, 2..256, dividing
+                             k): the pass takes the operand rotated along k, each
+                             block of b elements times the Sylvester matrix H_b and
+                             RN(1/sqrt(b)) as ss24_hadamard computes it, then
+                             rounded to bf16 (nearest even); §4 (rotation before
+                             quantization). bf16, axis 1, magnitude score only,
+                             and not the row-block INT pass (one scale per row
+                             without a given row amax): SS24_ERR_ARG otherwise. */
+    int32_t reserved;     /* 0                                                     */
 } ss24_operand;
 
 typedef struct {

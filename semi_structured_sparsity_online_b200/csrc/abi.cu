@@ -14,6 +14,7 @@
 namespace ss24 {
 const void *stream_kernel_bf16(int pattern, int score, int fmt, bool fw);
 const void *stream_kernel_f32(int pattern, int score, int fmt, bool fw);
+const void *stream_kernel_bf16_rot(int pattern, int fmt, bool fw);
 const void *rowsweep_kernel_bf16(int pattern, int score);
 const void *rowsweep_kernel_f32(int pattern, int score);
 const void *rowblock_kernel_bf16(int pattern, int score, int cpt);
@@ -268,6 +269,14 @@ ss24_status check_operand(const ss24_operand *x)
         return SS24_ERR_ALIGN;
     if (x->batch < 0 || x->batch > kMaxGrid)
         return SS24_ERR_SHAPE;
+    if (x->hadamard != 0) {
+        // the rotated pass: bf16 along k, a power-of-two block of 2..256 dividing k
+        const int32_t b = x->hadamard;
+        if (b < 2 || b > 256 || (b & (b - 1)) != 0 || x->axis != 1 || x->dtype != SS24_BF16)
+            return SS24_ERR_ARG;
+        if (x->k % b != 0)
+            return SS24_ERR_SHAPE;
+    }
     if (x->batch > 1) {
         // operands must not overlap
         if (x->batch_stride < (x->axis == 1 ? x->rows : x->k) * x->ld)
@@ -467,6 +476,13 @@ PassParams base_params(const ss24_operand *x, const Geometry &g, void *ws, ss24_
     p.energy_out = reinterpret_cast<double *>(energy);
     p.batch = static_cast<int32_t>(nbatch(x));
     p.x_bstride = bstride_elems(x);
+    if (x->hadamard != 0) {
+        int l = 0;
+        while ((1 << l) < x->hadamard)
+            ++l;
+        p.rot_log2b = l;
+        p.rot_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(x->hadamard)));
+    }
     return p;
 }
 
@@ -519,7 +535,11 @@ bool plan_tile(const ss24_operand *x, int pattern, int score, int mode, TilePlan
     if (x->axis == 1) {
         t->g = stream_geometry(x);
         // full width: W = 256 with four segments per unit
-        t->kernel = stream_kernel(x->dtype, pattern, score, mode, t->g.W == 256 && t->g.step_cols == 256);
+        const bool fw = t->g.W == 256 && t->g.step_cols == 256;
+        if (x->hadamard != 0)
+            t->kernel = score == SS24_SCORE_MAG ? stream_kernel_bf16_rot(pattern, mode, fw) : nullptr;
+        else
+            t->kernel = stream_kernel(x->dtype, pattern, score, mode, fw);
         t->smem = 0;
         return t->kernel != nullptr;
     }
@@ -530,13 +550,14 @@ bool plan_tile(const ss24_operand *x, int pattern, int score, int mode, TilePlan
 }
 
 // The read-only amax pass; leaves {amax of kept, amax of all} in the workspace.
-// For the magnitude score the kept amax equals the amax of all values, so the
-// cheaper dense form is used.
+// For 2:4 by magnitude the kept amax equals the amax of all values (a group's
+// largest value is always kept), so the cheaper dense form is used; pairwise
+// 4:8 can drop the largest value (its pair may rank third) and takes its own.
 cudaError_t run_amax(const ss24_operand *x, int pattern, int score, const float *norms, void *ws,
                      cudaStream_t stream, float *scale_out = nullptr, float divisor = 1.0f,
                      float *amax_user = nullptr, float *row_amax = nullptr)
 {
-    const int pat = score == SS24_SCORE_MAG ? SS24_DENSE : pattern;
+    const int pat = score == SS24_SCORE_MAG && pattern != SS24_SPARSE_48 ? SS24_DENSE : pattern;
     TilePlan t;
     if (!plan_tile(x, pat, score, kAmax, &t))
         return cudaErrorInvalidValue;
@@ -578,6 +599,8 @@ ss24_status run_pass(const ss24_operand *x, int pattern, int score, const float 
         return st;
     if (score != SS24_SCORE_MAG && score != SS24_SCORE_WANDA)
         return SS24_ERR_ARG;
+    if (x->hadamard != 0 && score != SS24_SCORE_MAG)
+        return SS24_ERR_ARG; // a rotated pass selects by magnitude
     if (score == SS24_SCORE_WANDA && pattern != SS24_DENSE && (!norms || !aligned16(norms)))
         return norms ? SS24_ERR_ALIGN : SS24_ERR_NULL;
     if ((st = check_ws(ws, ws_bytes)) != SS24_OK)
@@ -635,6 +658,8 @@ ss24_status run_pass(const ss24_operand *x, int pattern, int score, const float 
             p.q.amax_reduced = p.amax_out; // [0] = amax of the quantized values
         }
     }
+    if (r.row_mode && x->hadamard != 0)
+        return SS24_ERR_ARG; // one INT scale per row over a rotated operand: amax_rows + quantize_int_rows
     cudaError_t e;
     int cpt = 0, log2_tpr = 0;
     if (r.row_mode && rowblock_plan(x->k, &cpt, &log2_tpr)) {
@@ -795,6 +820,8 @@ ss24_status ss24_error_energy(const ss24_operand *x, ss24_pattern pattern, ss24_
         return st;
     if (score != SS24_SCORE_MAG && score != SS24_SCORE_WANDA)
         return SS24_ERR_ARG;
+    if (x->hadamard != 0 && score != SS24_SCORE_MAG)
+        return SS24_ERR_ARG; // a rotated pass selects by magnitude
     if (score == SS24_SCORE_WANDA && (!col_norms || !aligned16(col_norms)))
         return col_norms ? SS24_ERR_ALIGN : SS24_ERR_NULL;
     if ((st = check_ws(ws, ws_bytes)) != SS24_OK)
@@ -843,6 +870,8 @@ ss24_status ss24_amax(const ss24_operand *x, ss24_pattern pattern, ss24_score sc
         return st;
     if (score != SS24_SCORE_MAG && score != SS24_SCORE_WANDA)
         return SS24_ERR_ARG;
+    if (x->hadamard != 0 && score != SS24_SCORE_MAG)
+        return SS24_ERR_ARG; // a rotated pass selects by magnitude
     if (score == SS24_SCORE_WANDA && pattern != SS24_DENSE && (!col_norms || !aligned16(col_norms)))
         return col_norms ? SS24_ERR_ALIGN : SS24_ERR_NULL;
     if ((st = check_ws(ws, ws_bytes)) != SS24_OK)
@@ -868,6 +897,8 @@ ss24_status ss24_amax_rows(const ss24_operand *x, ss24_pattern pattern, ss24_sco
         return st;
     if (score != SS24_SCORE_MAG && score != SS24_SCORE_WANDA)
         return SS24_ERR_ARG;
+    if (x->hadamard != 0 && score != SS24_SCORE_MAG)
+        return SS24_ERR_ARG; // a rotated pass selects by magnitude
     if (score == SS24_SCORE_WANDA && pattern != SS24_DENSE && (!col_norms || !aligned16(col_norms)))
         return col_norms ? SS24_ERR_ALIGN : SS24_ERR_NULL;
     if (scale_out && !per_tensor(kind))
@@ -924,6 +955,8 @@ ss24_status ss24_tensor_scale(const ss24_operand *x, ss24_pattern pattern, ss24_
         return st;
     if (score != SS24_SCORE_MAG && score != SS24_SCORE_WANDA)
         return SS24_ERR_ARG;
+    if (x->hadamard != 0 && score != SS24_SCORE_MAG)
+        return SS24_ERR_ARG; // a rotated pass selects by magnitude
     if (score == SS24_SCORE_WANDA && pattern != SS24_DENSE && (!col_norms || !aligned16(col_norms)))
         return col_norms ? SS24_ERR_ALIGN : SS24_ERR_NULL;
     if (!per_tensor(kind))
@@ -980,7 +1013,7 @@ ss24_status ss24_softmax_prune(const ss24_operand *s, float alpha, ss24_pattern 
     ss24_status st = check_operand(s);
     if (st != SS24_OK)
         return st;
-    if (s->axis != 1 || !std::isfinite(alpha))
+    if (s->axis != 1 || !std::isfinite(alpha) || s->hadamard != 0)
         return SS24_ERR_ARG;
     if ((st = check_pattern_k(pattern, s->k)) != SS24_OK)
         return st;
@@ -1047,6 +1080,8 @@ ss24_status ss24_hadamard(const ss24_operand *x, int32_t block, float *out, ss24
     ss24_status st = check_operand(x);
     if (st != SS24_OK)
         return st;
+    if (x->hadamard != 0)
+        return SS24_ERR_ARG; // (the rotation is this call's own block)
     if (x->axis != 1)
         return SS24_ERR_ARG;
     if (block < 2 || block > 256 || (block & (block - 1)) != 0)

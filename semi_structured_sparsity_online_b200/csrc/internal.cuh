@@ -10,6 +10,9 @@ namespace ss24 {
 
 enum Pattern { kDense = 0, kSparse24 = 24, kSparse48 = 48 };
 enum Score { kMag = 0, kWanda = 1 };
+// A stream kernel's score parameter with this bit set: the magnitude score on
+// the operand rotated along k (block Hadamard, rounded to bf16) in registers.
+constexpr int kRotated = 2;
 // Formats of the pass; kAmax is the read-only amax pass; kEnergy the
 // read-only two-format energy pass; kIntRows is INT with one scale per row
 // from a given per-row amax (the stream kernel).
@@ -114,6 +117,9 @@ struct PassParams {
     // set per CTA by operand_view(): the operand served and the CTA's index
     // among that operand's CTAs
     int32_t op, cta;
+    // rotated kernels: log2 of the Hadamard block and RN(1/sqrt(block))
+    int32_t rot_log2b;
+    float rot_scale;
 };
 
 cudaError_t launch_ratio(const double *sparse_side, const double *dense_side, double *out, int64_t count,

@@ -170,14 +170,27 @@ __device__ __forceinline__ void neg_quotients(const float (&v)[VPC], const Recip
     }
 }
 
+// A packed product rounded once, as fma(a, b, -0): RN(a b), sign of zero
+// included. Products that feed an add or a subtract are written this way so
+// that no code generator can contract them into the following operation (the
+// readings round every product and every sum separately).
+__device__ __forceinline__ f32x2 mul2_rn(f32x2 a, f32x2 b, float z)
+{
+    // z: a zero the code generator cannot see as a constant (it is computed
+    // from run-time data), so the fused multiply-add is not rewritten as a
+    // multiply and then merged with its consumer
+    return fma2(a, b, pack2(z, z));
+}
+
 // Dequantized values code_value * s of a chunk (binary32 products).
 template <int VPC>
 __device__ __forceinline__ void scale_values(const float (&c)[VPC], float s, float (&d)[VPC])
 {
     const f32x2 s2 = pack2(s, s);
+    const float z = __fmul_rn(-0.0f, s); // -0 for the scales (s >= 0)
 #pragma unroll
     for (int i = 0; i < VPC / 2; ++i) {
-        const f32x2 r = mul2(pack2(c[2 * i], c[2 * i + 1]), s2);
+        const f32x2 r = mul2_rn(pack2(c[2 * i], c[2 * i + 1]), s2, z);
         d[2 * i] = lo2(r);
         d[2 * i + 1] = hi2(r);
     }
@@ -650,22 +663,23 @@ __device__ __forceinline__ Sel<PAT == kDense ? 8 : 4> select_chunk(const typenam
         // pairwise 4:8: pair p ranked by s_2p^2 + s_2p+1^2 (each product and
         // the sum rounded); for the magnitude score these are also the
         // pairs' energies
-        f32x2 a = mul2(pack2(x[0], x[2]), pack2(x[0], x[2]));
-        f32x2 b = mul2(pack2(x[1], x[3]), pack2(x[1], x[3]));
+        const float zq = __fmul_rn(-0.0f, fabsf(x[0])); // a run-time -0 (see mul2_rn)
+        f32x2 a = mul2_rn(pack2(x[0], x[2]), pack2(x[0], x[2]), zq);
+        f32x2 b = mul2_rn(pack2(x[1], x[3]), pack2(x[1], x[3]), zq);
         const f32x2 e01 = add2(a, b);
-        a = mul2(pack2(x[4], x[6]), pack2(x[4], x[6]));
-        b = mul2(pack2(x[5], x[7]), pack2(x[5], x[7]));
+        a = mul2_rn(pack2(x[4], x[6]), pack2(x[4], x[6]), zq);
+        b = mul2_rn(pack2(x[5], x[7]), pack2(x[5], x[7]), zq);
         const f32x2 e23 = add2(a, b);
         float e[4] = {lo2(e01), hi2(e01), lo2(e23), hi2(e23)};
         float rank[4] = {e[0], e[1], e[2], e[3]};
         if constexpr (SCORE == kWanda) {
             float s[8];
             scores<SCORE>(x, o, s);
-            a = mul2(pack2(s[0], s[2]), pack2(s[0], s[2]));
-            b = mul2(pack2(s[1], s[3]), pack2(s[1], s[3]));
+            a = mul2_rn(pack2(s[0], s[2]), pack2(s[0], s[2]), zq);
+            b = mul2_rn(pack2(s[1], s[3]), pack2(s[1], s[3]), zq);
             const f32x2 r01 = add2(a, b);
-            a = mul2(pack2(s[4], s[6]), pack2(s[4], s[6]));
-            b = mul2(pack2(s[5], s[7]), pack2(s[5], s[7]));
+            a = mul2_rn(pack2(s[4], s[6]), pack2(s[4], s[6]), zq);
+            b = mul2_rn(pack2(s[5], s[7]), pack2(s[5], s[7]), zq);
             const f32x2 r23 = add2(a, b);
             rank[0] = lo2(r01);
             rank[1] = hi2(r01);
@@ -820,7 +834,7 @@ __device__ __forceinline__ void dense_int_chunk(const typename Elem<T>::Raw &raw
             qn = pack2(fminf(fmaxf(a, -qmax), qmax), fminf(fmaxf(b, -qmax), qmax));
         }
         tt[i] = sub2(m2, qn);
-        const f32x2 d = mul2(sub2(tt[i], m2), s2);
+        const f32x2 d = mul2_rn(sub2(tt[i], m2), s2, __fmul_rn(-0.0f, rs.scale));
         e[i] = sub2(x2[i], d);
     }
     acc.eqd += sq_sum2<4>(e);
@@ -1194,13 +1208,70 @@ template <> struct Stream<float> {
 
 // Resident CTAs per SM the stream kernel is compiled for (register budget).
 // (Four CTAs where the kernel fits 64 registers without spilling, else three.)
-template <typename T, int PAT, int SCORE, int FMT, bool FW> struct StreamOcc {
-    // (INT holds four selected chunks across its group reduction)
+template <typename T, int PAT, int SCORE, int FMT, bool FW, bool ROT = false> struct StreamOcc {
+    // (INT holds four selected chunks across its group reduction; a rotated
+    // pass holds its rotation's temporaries)
     static constexpr bool light =
-        FMT == kAmax || (sizeof(T) == 2 && SCORE == kMag && PAT != kSparse48 &&
-                         (FMT == kNone || FMT == kMxfp4 || (FMT == kFp8 && (FW || PAT == kDense))));
+        !ROT && (FMT == kAmax || (sizeof(T) == 2 && SCORE == kMag && PAT != kSparse48 &&
+                                  (FMT == kNone || FMT == kMxfp4 || (FMT == kFp8 && (FW || PAT == kDense)))));
     static constexpr int value = light ? 4 : 3;
 };
+
+// Block Hadamard rotation, in place, of the bf16 chunk a lane holds, for
+// rotated passes. The lanes of a warp hold consecutive chunks of a row
+// segment, so the partner of a butterfly of stride h >= 8 is lane ^ (h / 8).
+// Binary32 arithmetic in stage order h = 1, 2, 4, ..., b/2: inside the lane
+// packed adds and subtracts of the pairs (y_i, y_i+h); across lanes
+// own * (+-1) + partner, which is exactly the rounded y_i + y_i+h (lower lane)
+// or y_i - y_i+h (upper lane); then times RN(1/sqrt(b)) and rounded to bf16
+// (nearest even). The whole warp calls it.
+__device__ __forceinline__ void rotate_chunk(uint4 &w, int log2b, float cb, int lane)
+{
+    float y[8];
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        y[2 * i] = __uint_as_float(ws[i] << 16);
+        y[2 * i + 1] = __uint_as_float(ws[i] & 0xffff0000u);
+    }
+#pragma unroll
+    for (int s = 0; s < 3; ++s) {
+        if (s >= log2b)
+            break;
+        const int h = 1 << s;
+#pragma unroll
+        for (int i0 = 0; i0 < 8; i0 += 2 * h) {
+            if (h == 1 && (i0 & 2))
+                continue; // (stride 1 pairs two butterflies 2 apart)
+#pragma unroll
+            for (int j = 0; j < (h == 1 ? 1 : h); j += 2) {
+                const int a = h == 1 ? i0 : i0 + j, b = h == 1 ? i0 + 2 : i0 + j + 1;
+                const f32x2 lo = pack2(y[a], y[b]), hi = pack2(y[a + h], y[b + h]);
+                const f32x2 sm = add2(lo, hi), df = sub2(lo, hi);
+                y[a] = lo2(sm), y[b] = hi2(sm), y[a + h] = lo2(df), y[b + h] = hi2(df);
+            }
+        }
+    }
+    for (int s = 3; s < log2b; ++s) {
+        const int m = 1 << (s - 3);
+        const float sg = (lane & m) ? -1.0f : 1.0f;
+        const f32x2 sg2 = pack2(sg, sg);
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) {
+            const float o0 = __shfl_xor_sync(kFull, y[i], m);
+            const float o1 = __shfl_xor_sync(kFull, y[i + 1], m);
+            const f32x2 r = fma2(pack2(y[i], y[i + 1]), sg2, pack2(o0, o1));
+            y[i] = lo2(r), y[i + 1] = hi2(r);
+        }
+    }
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(__fmul_rn(y[2 * i], cb), __fmul_rn(y[2 * i + 1], cb));
+        o[i] = *reinterpret_cast<const uint32_t *>(&h2);
+    }
+    w = make_uint4(o[0], o[1], o[2], o[3]);
+}
 
 // Byte advance of each output between consecutive slots of a full-width unit
 // (slots 256 input columns apart); -1 where it depends on runtime fields (INT
@@ -1220,7 +1291,7 @@ template <typename T, int PAT, int FMT> struct FwStep {
 template <typename T, int PAT, int SCORE>
 __device__ __forceinline__ float quantized_amax(const typename Elem<T>::Raw &raw, const ChunkOut &o)
 {
-    if constexpr (PAT == kDense || SCORE == kMag) {
+    if constexpr (PAT == kDense || (PAT == kSparse24 && SCORE == kMag)) {
         float xv[8];
         Elem<T>::unpack(raw, xv);
         return chunk_amax<T>(raw, xv);
@@ -1232,13 +1303,18 @@ __device__ __forceinline__ float quantized_amax(const typename Elem<T>::Raw &raw
 // A full-width unit of the amax pass, wholly inside the operand: the amax of
 // all values and of the kept values into acc, and the lane's largest
 // quantized magnitude returned (for the row amax).
-template <typename T, int PAT, int SCORE>
-__device__ __forceinline__ float amax_unit_fw(const T *xp, const ChunkOut &o, Acc &acc)
+template <typename T, int PAT, int SCORE, bool ROT = false>
+__device__ __forceinline__ float amax_unit_fw(const PassParams &p, const T *xp, const ChunkOut &o, Acc &acc)
 {
     typename Elem<T>::Raw raw[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
         raw[i] = Stream<T>::load(xp + i * 256, true);
+    if constexpr (ROT) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            rotate_chunk(raw[i].v, p.rot_log2b, p.rot_scale, static_cast<int>(threadIdx.x & 31));
+    }
     float m = 0.0f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -1252,7 +1328,9 @@ __device__ __forceinline__ float amax_unit_fw(const T *xp, const ChunkOut &o, Ac
             ChunkOut oi = o;
             if constexpr (SCORE == kWanda)
                 oi.norms = o.norms + i * 256;
-            const float kept = SCORE == kMag ? all : select_chunk<T, PAT, SCORE>(raw[i], oi).vmax;
+            // (2:4 by magnitude keeps every group's largest value; pairwise 4:8
+            // can drop it: its pair may rank third)
+            const float kept = (PAT == kSparse24 && SCORE == kMag) ? all : select_chunk<T, PAT, SCORE>(raw[i], oi).vmax;
             acc.amax_kept = fmaxf(acc.amax_kept, kept);
             m = fmaxf(m, kept);
         }
@@ -1262,7 +1340,7 @@ __device__ __forceinline__ float amax_unit_fw(const T *xp, const ChunkOut &o, Ac
 
 // One unit: four 16-byte loads per lane first, then the four chunks. FULL:
 // every chunk of the unit lies inside the operand (no per-chunk checks).
-template <typename T, int PAT, int SCORE, int FMT, bool FULL>
+template <typename T, int PAT, int SCORE, int FMT, bool FULL, bool ROT = false>
 __device__ __forceinline__ void stream_unit(const PassParams &p, const PassConsts &c, const T *xp, int64_t step_x,
                                             int64_t step_c, const ChunkOut &o, int64_t dval, int64_t dscale,
                                             int64_t dmeta, int64_t row0, int64_t col0, Acc &acc,
@@ -1276,6 +1354,13 @@ __device__ __forceinline__ void stream_unit(const PassParams &p, const PassConst
     for (int i = 0; i < 4; ++i) {
         ok[i] = FULL || (row0 + i * p.step_rows < p.rows && col0 + i * p.step_cols < p.k);
         raw[i] = Stream<T>::load(xp + i * step_x, ok[i]);
+    }
+    if constexpr (ROT) {
+        // (a chunk outside the operand is zero, and so is its whole block: k is
+        // a multiple of the block and blocks never straddle rows)
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            rotate_chunk(raw[i].v, p.rot_log2b, p.rot_scale, static_cast<int>(threadIdx.x & 31));
     }
     auto out_i = [&](int i) {
         ChunkOut oi = o;
@@ -1492,10 +1577,14 @@ __device__ __forceinline__ void stream_unit(const PassParams &p, const PassConst
 // are chosen by the host. FW: the full-width case W = 256 with four segments
 // per unit, where the slot offsets are compile-time constants and a unit
 // wholly inside the operand skips the per-chunk checks.
-template <typename T, int PAT, int SCORE, int FMT, bool FW>
-__global__ void __launch_bounds__(kStreamThreads, (StreamOcc<T, PAT, SCORE, FMT, FW>::value))
+template <typename T, int PAT, int SC, int FMT, bool FW>
+__global__ void __launch_bounds__(kStreamThreads, (StreamOcc<T, PAT, (SC & 1), FMT, FW, (SC & kRotated) != 0>::value))
     stream_kernel(const __grid_constant__ PassParams pk)
 {
+    // SC: the score, with kRotated set for a pass over the rotated operand
+    constexpr int SCORE = SC & 1;
+    constexpr bool ROT = (SC & kRotated) != 0;
+    static_assert(!ROT || (sizeof(T) == 2 && SCORE == kMag), "rotated passes: bf16, magnitude score");
     // the loop reads the (operand-independent) parameters in place and keeps
     // only this operand's output bases; the operand's full view is built for
     // the constants and again for the final reductions
@@ -1551,11 +1640,11 @@ __global__ void __launch_bounds__(kStreamThreads, (StreamOcc<T, PAT, SCORE, FMT,
                     const T *xp = x + row * p.ld + col0;
                     const ChunkOut o = make_out<T, PAT, FMT>(p, ob, row, col0, true, lane);
                     if (static_cast<int64_t>(b + 1) * 1024 <= p.k) {
-                        rm = fmaxf(rm, amax_unit_fw<T, PAT, SCORE>(xp, o, acc));
+                        rm = fmaxf(rm, amax_unit_fw<T, PAT, SCORE, ROT>(p, xp, o, acc));
                     } else {
                         Acc a{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                        stream_unit<T, PAT, SCORE, FMT, false>(p, c, xp, step_x, step_c, o, dval, dscale, dmeta, row,
-                                                               col0, a);
+                        stream_unit<T, PAT, SCORE, FMT, false, ROT>(p, c, xp, step_x, step_c, o, dval, dscale, dmeta,
+                                                                    row, col0, a);
                         acc.amax_all = fmaxf(acc.amax_all, a.amax_all);
                         acc.amax_kept = fmaxf(acc.amax_kept, a.amax_kept);
                         rm = fmaxf(rm, PAT == kDense ? a.amax_all : a.amax_kept);
@@ -1577,10 +1666,10 @@ __global__ void __launch_bounds__(kStreamThreads, (StreamOcc<T, PAT, SCORE, FMT,
         // full-width units lie inside the operand except in the last quad
         // of a row (rows are whole: one row per unit)
         if (FW && static_cast<int64_t>(ub + 1) * 1024 <= p.k)
-            stream_unit<T, PAT, SCORE, FMT, true>(p, c, xp, step_x, step_c, o, dval, dscale, dmeta, row0, col0,
+            stream_unit<T, PAT, SCORE, FMT, true, ROT>(p, c, xp, step_x, step_c, o, dval, dscale, dmeta, row0, col0,
                                                   acc, rowa, rowa_in, rscales);
         else
-            stream_unit<T, PAT, SCORE, FMT, false>(p, c, xp, step_x, step_c, o, dval, dscale, dmeta, row0, col0,
+            stream_unit<T, PAT, SCORE, FMT, false, ROT>(p, c, xp, step_x, step_c, o, dval, dscale, dmeta, row0, col0,
                                                    acc, rowa, rowa_in, rscales);
         // only the energies this pass produces (the others stay zero)
         if constexpr (FMT != kAmax)
@@ -1658,8 +1747,8 @@ __global__ void __launch_bounds__(kRowThreads) rowsweep_kernel(const T *__restri
     for (int64_t row = static_cast<int64_t>(p.cta) * kConsumerWarps + warp; row < p.rows;
          row += static_cast<int64_t>(p.ctas_per_op) * kConsumerWarps) {
         const T *xr = x + p.op * p.x_bstride + row * ld;
-        // sweep 1: the row amax of the values to quantize (for the magnitude
-        // score the kept amax equals the amax of all values)
+        // sweep 1: the row amax of the values to quantize (for 2:4 by
+        // magnitude the kept amax equals the amax of all values)
         float amax = 0.0f;
         for (int c0 = 0; c0 < nchunks; c0 += 256) {
             typename Elem<T>::Raw buf[8];
@@ -1670,7 +1759,7 @@ __global__ void __launch_bounds__(kRowThreads) rowsweep_kernel(const T *__restri
             for (int u = 0; u < 8; ++u) {
                 const int c = c0 + 32 * u + lane;
                 if (c < nchunks) {
-                    if constexpr (PAT == kDense || SCORE == kMag) {
+                    if constexpr (PAT == kDense || (PAT == kSparse24 && SCORE == kMag)) {
                         float xv[8];
                         Elem<T>::unpack(buf[u], xv);
                         amax = fmaxf(amax, chunk_amax<T>(buf[u], xv));
@@ -1780,12 +1869,12 @@ __global__ void __launch_bounds__(kRowThreads, (RowblockOcc<T, PAT, SCORE, CPT>:
             raw[j] = Stream<T>::load(xr + 8 * c, rv && c < nchunks);
         }
         const ChunkOut o = make_out<T, PAT, kInt>(p, ob, row, 8 * t, rv, lane);
-        // the row amax of the values to quantize (for the magnitude score the
+        // the row amax of the values to quantize (for 2:4 by magnitude the
         // kept amax equals the amax of all values)
         float m = 0.0f;
 #pragma unroll
         for (int j = 0; j < CPT; ++j) {
-            if constexpr (PAT == kDense || SCORE == kMag) {
+            if constexpr (PAT == kDense || (PAT == kSparse24 && SCORE == kMag)) {
                 float xv[8];
                 Elem<T>::unpack(raw[j], xv);
                 m = fmaxf(m, chunk_amax<T>(raw[j], xv));

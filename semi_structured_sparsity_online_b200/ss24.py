@@ -41,7 +41,8 @@ class Format(ctypes.Structure):
 class Operand(ctypes.Structure):
     _fields_ = [("x", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("axis", ctypes.c_int32),
                 ("rows", ctypes.c_int64), ("k", ctypes.c_int64), ("ld", ctypes.c_int64),
-                ("batch", ctypes.c_int64), ("batch_stride", ctypes.c_int64)]
+                ("batch", ctypes.c_int64), ("batch_stride", ctypes.c_int64),
+                ("hadamard", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 class Outputs(ctypes.Structure):
@@ -135,10 +136,11 @@ def make_format(fmt="none", bits=8, group=0, pack4=False) -> Format:
     return Format(kind, int(bits), int(group), int(bool(pack4)))
 
 
-def make_operand(x: torch.Tensor, axis: int = 1, rows=None, k=None) -> Operand:
+def make_operand(x: torch.Tensor, axis: int = 1, rows=None, k=None, hadamard: int = 0) -> Operand:
     """Operand descriptor of a CUDA tensor. 2-D: one operand; axis 1: x is
     [rows, ld] with k contiguous; axis 0: x is [k, ld] holding A[r][c] at
-    x[c][r]. 3-D [B, ., .]: a batch of B such operands (x.stride(0) apart)."""
+    x[c][r]. 3-D [B, ., .]: a batch of B such operands (x.stride(0) apart).
+    hadamard: 0, or the block of the rotation the pass applies along k first."""
     if x.dtype == torch.bfloat16:
         dt = BF16
     elif x.dtype == torch.float32:
@@ -155,7 +157,7 @@ def make_operand(x: torch.Tensor, axis: int = 1, rows=None, k=None) -> Operand:
     else:
         kk = m.shape[0] if k is None else k
         r = m.shape[1] if rows is None else rows
-    return Operand(x.data_ptr(), dt, axis, r, kk, m.stride(0), batch, bstride)
+    return Operand(x.data_ptr(), dt, axis, r, kk, m.stride(0), batch, bstride, int(hadamard), 0)
 
 
 class Workspace:
@@ -233,13 +235,13 @@ def _energy(op, device):
 
 
 def run(x: torch.Tensor, pattern=SPARSE_24, fmt="none", bits=8, group=0, pack4=False, score="mag",
-        col_norms=None, tensor_scale=None, energy=True, axis=1, ws=None, stream=None, out=None):
+        col_norms=None, tensor_scale=None, energy=True, axis=1, ws=None, stream=None, out=None, hadamard=0):
     """One pass through the matching C entry point. Returns a dict of output
     tensors (``values``, ``scales``, ``tensor_scale``, ``meta``) and ``energy``
     (float64[4] on the device: e_total, e_prune, e_quant, e_quant_dense). A
     3-D x is a batch: every output and the energies get a leading [B]."""
     f = make_format(fmt, bits, group, pack4)
-    op = make_operand(x, axis)
+    op = make_operand(x, axis, hadamard=hadamard)
     sc = _SCORE[score] if isinstance(score, str) else int(score)
     if out is None:
         out = _alloc_outputs(op.rows, op.k, pattern, f, x.dtype, x.device, _lead(op))
@@ -277,11 +279,11 @@ def run(x: torch.Tensor, pattern=SPARSE_24, fmt="none", bits=8, group=0, pack4=F
 
 
 def error_energy(x, pattern=SPARSE_24, sparse_fmt=("none",), dense_fmt=("int", 8, 0), score="mag",
-                 col_norms=None, sparse_scale=None, dense_scale=None, axis=1, ws=None, stream=None, energy=None):
+                 col_norms=None, sparse_scale=None, dense_scale=None, axis=1, ws=None, stream=None, energy=None, hadamard=0):
     """Read-only energy pass; returns float64[4] (or [B, 4]) on the device."""
     sf = make_format(*sparse_fmt) if isinstance(sparse_fmt, tuple) else sparse_fmt
     df = make_format(*dense_fmt) if isinstance(dense_fmt, tuple) else dense_fmt
-    op = make_operand(x, axis)
+    op = make_operand(x, axis, hadamard=hadamard)
     e = energy if energy is not None else _energy(op, x.device)
     ws = ws or default_workspace(x.device)
     _check(lib().ss24_error_energy(ctypes.byref(op), pattern, _SCORE[score] if isinstance(score, str) else score,
@@ -290,8 +292,8 @@ def error_energy(x, pattern=SPARSE_24, sparse_fmt=("none",), dense_fmt=("int", 8
     return e
 
 
-def amax(x, pattern=SPARSE_24, score="mag", col_norms=None, axis=1, ws=None, stream=None):
-    op = make_operand(x, axis)
+def amax(x, pattern=SPARSE_24, score="mag", col_norms=None, axis=1, ws=None, stream=None, hadamard=0):
+    op = make_operand(x, axis, hadamard=hadamard)
     out = torch.empty(max(op.batch, 1), dtype=torch.float32, device=x.device)
     ws = ws or default_workspace(x.device)
     _check(lib().ss24_amax(ctypes.byref(op), pattern, _SCORE[score] if isinstance(score, str) else score,
@@ -300,10 +302,10 @@ def amax(x, pattern=SPARSE_24, score="mag", col_norms=None, axis=1, ws=None, str
 
 
 def tensor_scale(x, fmt="fp8", pattern=SPARSE_24, score="mag", col_norms=None, axis=1, ws=None, stream=None,
-                 out=None):
+                 out=None, hadamard=0):
     """The per-tensor scale (FP8: amax / 448, NVFP4: amax / 2688) as a device
     float32[1] (float32[B] for a batch)."""
-    op = make_operand(x, axis)
+    op = make_operand(x, axis, hadamard=hadamard)
     out = out if out is not None else torch.empty(max(op.batch, 1), dtype=torch.float32, device=x.device)
     ws = ws or default_workspace(x.device)
     _check(lib().ss24_tensor_scale(ctypes.byref(op), pattern, _SCORE[score] if isinstance(score, str) else score,
@@ -313,11 +315,11 @@ def tensor_scale(x, fmt="fp8", pattern=SPARSE_24, score="mag", col_norms=None, a
 
 
 def amax_rows(x, pattern=DENSE, score="mag", col_norms=None, scale_fmt=None, ws=None, stream=None, out=None,
-              scale_out=None):
+              scale_out=None, hadamard=0):
     """Per-row amax of the values a pass with this pattern / score quantizes,
     float32 [rows] (or [B, rows]) on the device, and, with scale_fmt ("fp8" or
     "nvfp4"), the per-tensor scale from the same read: returns (rows, scale)."""
-    op = make_operand(x, 1)
+    op = make_operand(x, 1, hadamard=hadamard)
     lead = _lead(op)
     shape = (op.rows,) if lead is None else (lead, op.rows)
     out = out if out is not None else torch.empty(shape, dtype=torch.float32, device=x.device)
@@ -332,11 +334,11 @@ def amax_rows(x, pattern=DENSE, score="mag", col_norms=None, scale_fmt=None, ws=
 
 
 def run_int_rows(x, row_amax, pattern=DENSE, bits=8, pack4=False, score="mag", col_norms=None, energy=True,
-                 ws=None, stream=None, out=None):
+                 ws=None, stream=None, out=None, hadamard=0):
     """INT-b with one scale per row from a given per-row amax (ss24_quantize_int_rows);
     returns the same dict as run()."""
     f = make_format("int", bits, 0, pack4)
-    op = make_operand(x, 1)
+    op = make_operand(x, 1, hadamard=hadamard)
     if out is None:
         out = _alloc_outputs(op.rows, op.k, pattern, f, x.dtype, x.device, _lead(op))
     e = _energy(op, x.device) if energy is True else energy

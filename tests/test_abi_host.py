@@ -254,3 +254,27 @@ def test_softmax_prune_validation():
     assert call(op(), fmt=("fp8",), scale=None) == 1             # SS24_ERR_NULL: FP8 needs the given scale
     assert call(op(), fmt=("none",), pattern=ss24.DENSE) == 5    # dense needs a quantization format
     assert call(op(), wsb=16) == 6                               # SS24_ERR_WORKSPACE
+
+
+def test_rotated_operand_validation():
+    """The operand's hadamard field: checked before anything is launched."""
+    L = ss24.lib()
+    ws = ctypes.c_void_p(ALIGNED)
+    outs = ss24.Outputs(ALIGNED, ALIGNED, ALIGNED, ALIGNED)
+
+    def op(rows=4, k=1024, ld=None, axis=1, dtype=ss24.BF16, had=16):
+        return ss24.Operand(ALIGNED, dtype, axis, rows, k, ld or k, 0, 0, had, 0)
+
+    def fused(o, score=ss24._SCORE["mag"], fmt=("fp8",)):
+        return L.ss24_prune24_quant_fused(ctypes.byref(o), score, ALIGNED, ss24.make_format(*fmt), ALIGNED,
+                                          ctypes.byref(outs), None, ws, _ws_bytes(), None)
+    assert fused(op(had=3)) == 8 and fused(op(had=512)) == 8 and fused(op(had=1)) == 8   # SS24_ERR_ARG
+    assert fused(op(dtype=ss24.F32)) == 8                                                # bf16 only
+    assert fused(op(axis=0, ld=8)) == 8                                                  # axis 1 only
+    assert fused(op(k=1040, had=32)) == 2                                                # SS24_ERR_SHAPE: k % block
+    assert fused(op(), score=ss24._SCORE["wanda"]) == 8                                  # magnitude only
+    assert L.ss24_quantize_int(ctypes.byref(op(k=4096)), ss24.make_format("int", 8, 0), ctypes.byref(outs), None,
+                               ws, _ws_bytes(), None) == 8                               # the row-block INT pass
+    assert L.ss24_hadamard(ctypes.byref(op()), 16, ALIGNED, None) == 8                   # no second rotation
+    assert L.ss24_softmax_prune(ctypes.byref(op(k=1024)), 0.1, ss24.SPARSE_24, ss24.make_format("fp8"), ALIGNED,
+                                ctypes.byref(outs), None, ws, _ws_bytes(), None) == 8

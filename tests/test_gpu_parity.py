@@ -559,6 +559,84 @@ def test_rotation_raises_predicted_ratio(ss, ws):
         assert abs(r[1] / r[0] - 1) < 0.02, r
 
 
+def test_pairwise48_drops_the_largest_value(ss, ws):
+    """Pairwise 4:8 ranks pairs by energy, so a tensor's or row's largest value
+    can be dropped (pairs (0.8, 0.8) and (0.75, 0.75) outrank (1.0, 0)): the
+    derived tensor scales and the per-row INT scales take the kept amax."""
+    pat8 = synth.bf16_bits(np.array([0.8, 0.8, 0.75, 0.75, 1.0, 0.0, 0.1, 0.1], dtype=np.float32))
+    for rows, k in ((16, 2048), (3, 20480), (5, 256)):
+        xh = np.tile(pat8, (rows, k // 8))
+        for fmt, bits in (("fp8", 8), ("nvfp4", 4), ("int", 8)):
+            compare(ss, ws, xh, pattern=48, fmt=fmt, bits=bits, group=0)
+    xh = np.tile(pat8, (8, 1024 // 8))
+    ra, _ = ss.amax_rows(to_dev(xh), pattern=48, ws=ws)
+    torch.cuda.synchronize()
+    assert np.all(ra.cpu().numpy() == np.float32(synth.bf16_to_f32(pat8)[0]))   # 0.8 in bf16, not 1.0
+
+
+ROT_CASES = [(24, "none", 8, 0), (24, "fp8", 8, 0), (24, "nvfp4", 4, 0), (24, "mxfp4", 4, 0), (24, "int", 8, 64),
+             (48, "nvfp4", 4, 0), (48, "fp8", 8, 0), (0, "fp8", 8, 0), (0, "nvfp4", 4, 0), (0, "int", 5, 128)]
+
+
+@pytest.mark.parametrize("pattern,fmt,bits,group", ROT_CASES)
+@pytest.mark.parametrize("b", [16, 128, 256])
+def test_rotated_pass_fused_matches_oracle(ss, ws, pattern, fmt, bits, group, b):
+    """The rotation inside the pass (operand field hadamard = b) against the
+    oracle's rotation rounded to bf16 followed by the oracle's pass: full-width
+    rows, a partial last unit and narrow rows; FP8 / NVFP4 with the derived
+    tensor scale (the amax pass rotates too) and FP8 with a given one."""
+    opat = {0: oracle.DENSE, 24: oracle.SPARSE_24, 48: oracle.SPARSE_48}[pattern]
+    for rows, k in ((37, 1024), (5, 1280), (9, 512), (6, 256)):
+        if k % b:
+            continue
+        xh = synth.sweep_operand(rows, k, seed=100 + b)
+        rot = oracle.hadamard_bf16(xh, b)
+        out = ss.run(to_dev(xh), pattern=pattern, fmt=fmt, bits=bits, group=group, ws=ws, hadamard=b)
+        torch.cuda.synchronize()
+        ts = oracle.tensor_scale(rot, fmt, pattern=opat) if fmt in ("fp8", "nvfp4") else None
+        ref = oracle.run(rot, pattern=opat, fmt=fmt, bits=bits, group=group,
+                         **({"tensor_scale": ts} if ts is not None else {}))
+        for key in ("values", "scales", "meta"):
+            if key in ref and out.get(key) is not None:
+                assert_same(to_np(out[key]), ref[key], f"{key} {rows}x{k}")
+        assert_energy(out["energy"], ref["energy"], atol=1e-30)
+        if fmt == "fp8":
+            given = torch.tensor([np.float32(0.05)], device="cuda")
+            out = ss.run(to_dev(xh), pattern=pattern, fmt=fmt, tensor_scale=given, ws=ws, hadamard=b)
+            torch.cuda.synchronize()
+            ref = oracle.run(rot, pattern=opat, fmt=fmt, tensor_scale=float(np.float32(0.05)))
+            assert_same(to_np(out["values"]), ref["values"], f"values given scale {rows}x{k}")
+    assert ws.error() == 0
+
+
+def test_rotated_rows_energy_and_batch(ss, ws):
+    """Rotated per-row INT (the row amax pass and the INT pass from it), the
+    rotated energy pass, and a rotated batch."""
+    b = 64
+    xh = synth.linear_input(40, 2048, seed=105)[0]
+    rot = oracle.hadamard_bf16(xh, b)
+    x = to_dev(xh)
+    ra, _ = ss.amax_rows(x, ws=ws, hadamard=b)
+    out = ss.run_int_rows(x, ra, bits=8, ws=ws, hadamard=b)
+    torch.cuda.synchronize()
+    ref = oracle.run(rot, pattern=oracle.DENSE, fmt="int", bits=8, group=0)
+    assert_same(to_np(out["values"]), ref["values"], "int rows values")
+    assert_same(to_np(out["scales"]), ref["scales"], "int rows scales")
+    e = ss.error_energy(x, pattern=24, sparse_fmt=("fp8",), dense_fmt=("int", 5, 128), ws=ws, hadamard=b)
+    torch.cuda.synchronize()
+    ts = oracle.tensor_scale(rot, "fp8", pattern=oracle.SPARSE_24)
+    sp = oracle.run(rot, pattern=oracle.SPARSE_24, fmt="fp8", tensor_scale=ts)["energy"]
+    de = oracle.run(rot, pattern=oracle.DENSE, fmt="int", bits=5, group=128)["energy"]
+    assert_energy(e, np.array([sp[0], sp[1], sp[2], de[3]]), atol=1e-30)
+    xs = [synth.sweep_operand(7, 1024, seed=106 + i) for i in range(3)]
+    out = ss.run(torch.stack([to_dev(v) for v in xs]), pattern=24, fmt="mxfp4", ws=ws, hadamard=32)
+    torch.cuda.synchronize()
+    for i, v in enumerate(xs):
+        ref = oracle.run(oracle.hadamard_bf16(v, 32), pattern=oracle.SPARSE_24, fmt="mxfp4")
+        assert_same(to_np(out["values"][i]), ref["values"], f"batch values {i}")
+        assert_energy(out["energy"][i], ref["energy"], atol=1e-30)
+
+
 SOFTMAX_CASES = [(24, "none", 8, 0), (24, "fp8", 8, 0), (24, "nvfp4", 4, 0), (24, "mxfp4", 4, 0),
                  (24, "int", 8, 32), (48, "nvfp4", 4, 0), (48, "fp8", 8, 0), (0, "fp8", 8, 0), (0, "mxfp4", 4, 0),
                  (0, "int", 4, 64)]
