@@ -77,6 +77,8 @@ def main():
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--seed", type=int, default=8)
     ap.add_argument("--batch", type=int, default=0, help="0: one 2-D operand; B: one launch over B operands")
+    ap.add_argument("--hadamard", type=int, default=0,
+                    help="passes in PASSES: rotate the operand along k in the pass (block size)")
     ap.add_argument("--dequant", action="store_true",
                     help="time the reconstruction of the pass's outputs (ss24_dequantize) instead of the pass")
     ap.add_argument("--derive-scale", action="store_true",
@@ -92,14 +94,15 @@ def main():
     e = torch.zeros((nb, 4), dtype=torch.float64, device="cuda")
     if args.batch == 0:
         e = e[0]
-    scale = ss24.tensor_scale(x, "fp8", ss24.SPARSE_24, ws=ws)
+    scale = ss24.tensor_scale(x, "fp8", ss24.SPARSE_24, ws=ws, hadamard=args.hadamard)
     out = None
     if args.name in PASSES:
         pattern, fmt, bits, group = PASSES[args.name]
         out = ss24._alloc_outputs(args.m, args.k, pattern, ss24.make_format(fmt, bits, group), torch.bfloat16, "cuda",
                                   lead)
         if fmt == "nvfp4":
-            scale = ss24.tensor_scale(x, "nvfp4", pattern if pattern != ss24.DENSE else ss24.DENSE, ws=ws)
+            scale = ss24.tensor_scale(x, "nvfp4", pattern if pattern != ss24.DENSE else ss24.DENSE, ws=ws,
+                                      hadamard=args.hadamard)
 
     row_amax = ss24.amax_rows(x, ws=ws)[0] if args.name in ("amax_rows", "dense_int8_given_rows") else None
     if args.name == "dense_int8_given_rows":
@@ -131,7 +134,8 @@ def main():
         else:
             pattern, fmt, bits, group = PASSES[args.name]
             ts = scale if fmt in ("fp8", "nvfp4") and not args.derive_scale else None
-            ss24.run(x, pattern=pattern, fmt=fmt, bits=bits, group=group, tensor_scale=ts, energy=e, ws=ws, out=out)
+            ss24.run(x, pattern=pattern, fmt=fmt, bits=bits, group=group, tensor_scale=ts, energy=e, ws=ws, out=out,
+                     hadamard=args.hadamard)
 
     once()
     torch.cuda.synchronize()
@@ -156,7 +160,7 @@ def main():
     t.synchronize()
     us = s.elapsed_time(t) / args.iters * 1e3
     assert ws.error() == 0
-    print(f"{args.name}{' dequant' if args.dequant else ''} m={args.m} k={args.k} batch={args.batch}: {us:.2f} us/launch, {gb / us / 1e3:.1f} GB/s "
+    print(f"{args.name}{' dequant' if args.dequant else ''}{f' hadamard {args.hadamard}' if args.hadamard else ''} m={args.m} k={args.k} batch={args.batch}: {us:.2f} us/launch, {gb / us / 1e3:.1f} GB/s "
           f"({gb} algorithmic bytes per launch; warm L2 between launches)")
 
 
