@@ -70,8 +70,8 @@ def pass_bytes(name, m, k):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--pass", dest="name", default="fused_24_fp8", choices=sorted(PASSES) + ["tensor_scale", "error_energy", "amax_rows", "hadamard128", "softmax_24_fp8",
-                                                                       "dense_int8_given_rows"])
+    extra = ["tensor_scale", "error_energy", "amax_rows", "hadamard128", "softmax_24_fp8", "dense_int8_given_rows"]
+    ap.add_argument("--pass", dest="name", default="fused_24_fp8", choices=sorted(PASSES) + extra)
     ap.add_argument("--m", type=int, default=4096)
     ap.add_argument("--k", type=int, default=4096)
     ap.add_argument("--iters", type=int, default=3)
@@ -160,7 +160,8 @@ def main():
     t.synchronize()
     us = s.elapsed_time(t) / args.iters * 1e3
     assert ws.error() == 0
-    print(f"{args.name}{' dequant' if args.dequant else ''}{f' hadamard {args.hadamard}' if args.hadamard else ''} m={args.m} k={args.k} batch={args.batch}: {us:.2f} us/launch, {gb / us / 1e3:.1f} GB/s "
+    tag = (" dequant" if args.dequant else "") + (f" hadamard {args.hadamard}" if args.hadamard else "")
+    print(f"{args.name}{tag} m={args.m} k={args.k} batch={args.batch}: {us:.2f} us/launch, {gb / us / 1e3:.1f} GB/s "
           f"({gb} algorithmic bytes per launch; warm L2 between launches)")
 
 

@@ -279,7 +279,8 @@ def run(x: torch.Tensor, pattern=SPARSE_24, fmt="none", bits=8, group=0, pack4=F
 
 
 def error_energy(x, pattern=SPARSE_24, sparse_fmt=("none",), dense_fmt=("int", 8, 0), score="mag",
-                 col_norms=None, sparse_scale=None, dense_scale=None, axis=1, ws=None, stream=None, energy=None, hadamard=0):
+                 col_norms=None, sparse_scale=None, dense_scale=None, axis=1, ws=None, stream=None, energy=None,
+                 hadamard=0):
     """Read-only energy pass; returns float64[4] (or [B, 4]) on the device."""
     sf = make_format(*sparse_fmt) if isinstance(sparse_fmt, tuple) else sparse_fmt
     df = make_format(*dense_fmt) if isinstance(dense_fmt, tuple) else dense_fmt
