@@ -278,3 +278,29 @@ def test_rotated_operand_validation():
     assert L.ss24_hadamard(ctypes.byref(op()), 16, ALIGNED, None) == 8                   # no second rotation
     assert L.ss24_softmax_prune(ctypes.byref(op(k=1024)), 0.1, ss24.SPARSE_24, ss24.make_format("fp8"), ALIGNED,
                                 ctypes.byref(outs), None, ws, _ws_bytes(), None) == 8
+
+
+def test_algorithmic_bytes_match_the_stored_layouts():
+    """The bytes the benchmark and run_case count per launch, from the layouts:
+    input 2 bytes per bf16 element; FP8 codes 1 byte per stored value; metadata
+    1/8 byte per element (2:4) or 1/16 (4:8); E4M3 block scales 1 byte per 16
+    stored values, E8M0 per 32; INT scales 4 bytes per group or row."""
+    import bench
+    from semi_structured_sparsity_online_b200 import run_case
+    m = k = 4096
+    n = m * k
+    ab = bench.algorithmic_bytes(m, k)
+    assert ab["fused_24_fp8"] == 2 * n + n // 2 + n // 8 == 44_040_192
+    assert ab["dense_fp8"] == 3 * n == 50_331_648
+    assert ab["tensor_scale"] == 2 * n + 4 * m
+    assert ab["dense_int8_row"] == 2 * n + 4 * m + n + 4 * m
+    pb = run_case.pass_bytes
+    assert pb("fused_24_fp8", m, k) == ab["fused_24_fp8"]
+    assert pb("fused_24_none", m, k) == 2 * n + n + n // 8 == 52_428_800
+    assert pb("fused_24_nvfp4", m, k) == 2 * n + n // 4 + n // 32 + n // 8 == 40_370_176
+    assert pb("fused_24_mxfp4", m, k) == 2 * n + n // 4 + n // 64 + n // 8 == 40_108_032
+    assert pb("fused_48_nvfp4", m, k) == 2 * n + n // 4 + n // 32 + n // 16 == 39_321_600
+    assert pb("fused_24_int8g128", m, k) == 2 * n + n // 2 + 4 * (n // 2 // 128) + n // 8 == 44_302_336
+    assert pb("dense_nvfp4", m, k) == 2 * n + n // 2 + n // 16 == 42_991_616
+    assert pb("hadamard128", m, k) == 6 * n
+    assert pb("softmax_24_fp8", m, k) == ab["fused_24_fp8"]
