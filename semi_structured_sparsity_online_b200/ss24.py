@@ -239,7 +239,10 @@ def run(x: torch.Tensor, pattern=SPARSE_24, fmt="none", bits=8, group=0, pack4=F
     """One pass through the matching C entry point. Returns a dict of output
     tensors (``values``, ``scales``, ``tensor_scale``, ``meta``) and ``energy``
     (float64[4] on the device: e_total, e_prune, e_quant, e_quant_dense). A
-    3-D x is a batch: every output and the energies get a leading [B]."""
+    3-D x is a batch: every output and the energies get a leading [B].
+    hadamard=b rotates x along k in the pass first (block Hadamard of b, the
+    result rounded to bf16; bf16 input, magnitude score), and so do the amax
+    passes behind a derived tensor scale."""
     f = make_format(fmt, bits, group, pack4)
     op = make_operand(x, axis, hadamard=hadamard)
     sc = _SCORE[score] if isinstance(score, str) else int(score)
