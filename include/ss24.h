@@ -230,8 +230,8 @@ ss24_status ss24_quantize_fp8(const ss24_operand *x, const float *tensor_scale_i
                               ss24_outputs *out, ss24_energy *energy, void *ws, size_t ws_bytes,
                               ss24_stream stream);
 
-/* Dense symmetric INT-b with per-group or per-row scales (§3 "INT8 with a
- * single scale per row"; §2 equal-bit partners INT3 ... INT9). fmt.kind must be
+/* Dense symmetric INT-b with per-group or per-row scales (§3: INT8 with one
+ * scale per row; §2 equal-bit partners INT3 ... INT9). fmt.kind must be
  * SS24_FMT_INT. energy receives e_total and e_quant_dense. */
 ss24_status ss24_quantize_int(const ss24_operand *x, ss24_format fmt, ss24_outputs *out,
                               ss24_energy *energy, void *ws, size_t ws_bytes, ss24_stream stream);
@@ -334,26 +334,31 @@ ss24_status ss24_predicted_ratio(const ss24_energy *sparse_side, const ss24_ener
 
 /* ---- without caller-supplied scratch ----------------------------------------- */
 
-/* The fused 2:4 pass of ss24_prune24_quant_fused (same arguments, same results)
- * for callers that cannot allocate device memory: code that runs where
- * cudaMalloc is not allowed (inside a caching allocator's own callbacks, or a
- * host that hands the library only the operand and the output buffers) and so
- * cannot provide a workspace. No counterpart in the paper: it exists for such
- * callers only.
+/* The fused 2:4 pass of ss24_prune24_quant_fused (same arguments, same results,
+ * axis 1 only) for callers that cannot allocate device memory: code that runs
+ * where cudaMalloc is not allowed (inside a caching allocator's own callbacks,
+ * or a host that hands the library only the operand and the output buffers)
+ * and so cannot provide a workspace. No counterpart in the paper: it exists for
+ * such callers only.
  *
  * Scratch. The pass's scratch (per-CTA partial sums, two ticket counters and
  * an error word, 57,600 bytes: enough for the at most 1024 CTAs the pass
  * launches, whatever the operand size) lives in a device array owned by the
  * library: one copy on every GPU that loads the library, kept until the
- * process exits. The entry point allocates nothing and frees nothing. If the
- * pass ever needed more scratch than the array holds it returns
- * SS24_ERR_WORKSPACE. Errors recorded by a timed-out kernel wait are cleared at
- * the next call and are not reported through this entry point.
+ * process exits. The entry point allocates nothing and frees nothing.
+ *
+ * Errors. Every argument is checked before anything is enqueued, as for the
+ * other entry points: a rejected call enqueues nothing, and leaves the array
+ * as it was. An operand with axis 0 is rejected (SS24_ERR_ARG): the strided-
+ * axis kernel waits on its tile copies with a time limit and records a wait
+ * that gave up in the array, where the caller could not see it; the axis-1
+ * kernels this entry point launches contain no such wait.
  *
  * First call on a device: it looks up the array's device address (once per
- * device, with that device current); make that first call before any stream
- * capture. Every call then clears the array's counters with a stream-ordered
- * memset before launching.
+ * device and context, with that device current; a context created after a
+ * device reset gets a fresh lookup); make that first call before any stream
+ * capture. Every accepted call then clears the array's counters with a
+ * stream-ordered memset before its first launch.
  *
  * Concurrency. All calls on a device share the one array, which keeps the
  * last call's contents: calls that overlap on the GPU (on different streams,

@@ -99,9 +99,14 @@ bool make_map(CUtensorMap *map, const ss24_operand *x, int64_t inner, int64_t ou
     return r == CUDA_SUCCESS;
 }
 
-// Kernel attributes (dynamic shared memory) and occupancy, once per kernel.
+bool current_ctx_id(unsigned long long *id);
+
+// Kernel attributes (dynamic shared memory) and occupancy, once per kernel and
+// context (a context created after a device reset starts without the
+// attributes).
 struct KernelInfo {
     int blocks_per_sm = 0;
+    unsigned long long ctx_id = 0;
 };
 
 std::mutex g_mu;
@@ -110,9 +115,11 @@ int g_sms = 0;
 
 cudaError_t kernel_info(const void *k, size_t smem, KernelInfo *out, int threads = kThreads)
 {
+    unsigned long long id = 0;
+    const bool have_id = current_ctx_id(&id);
     std::lock_guard<std::mutex> lock(g_mu);
     auto it = g_info.find(k);
-    if (it != g_info.end()) {
+    if (it != g_info.end() && have_id && it->second.ctx_id == id) {
         *out = it->second;
         return cudaSuccess;
     }
@@ -131,6 +138,7 @@ cudaError_t kernel_info(const void *k, size_t smem, KernelInfo *out, int threads
         if (e != cudaSuccess)
             return e;
     }
+    info.ctx_id = current_ctx_id(&id) ? id : 0;
     g_info[k] = info;
     *out = info;
     return cudaSuccess;
@@ -588,9 +596,12 @@ ss24_status empty_operand(const ss24_operand *x, ss24_energy *energy, const ss24
 }
 
 // The storing pass shared by the quantize / prune entry points.
+// With launch false it only validates: it returns the status the call would
+// return before enqueueing anything, and enqueues nothing.
 ss24_status run_pass(const ss24_operand *x, int pattern, int score, const float *norms, ss24_format fmt,
                      bool allow_none, const float *scale_in, const ss24_outputs *out, ss24_energy *energy,
-                     void *ws, size_t ws_bytes, cudaStream_t stream, const float *row_amax_in = nullptr)
+                     void *ws, size_t ws_bytes, cudaStream_t stream, const float *row_amax_in = nullptr,
+                     bool launch_it = true)
 {
     ss24_status st = check_operand(x);
     if (st != SS24_OK)
@@ -620,7 +631,8 @@ ss24_status run_pass(const ss24_operand *x, int pattern, int score, const float 
         g = stream_geometry(x); // (row mode uses only rows / k of it)
     }
     if (x->rows == 0)
-        return empty_operand(x, energy, out, per_tensor(fmt.kind) ? scale_in : nullptr, stream);
+        return launch_it ? empty_operand(x, energy, out, per_tensor(fmt.kind) ? scale_in : nullptr, stream)
+                         : SS24_OK;
     if (!out->values)
         return SS24_ERR_NULL;
     if (!aligned16(out->values))
@@ -636,6 +648,10 @@ ss24_status run_pass(const ss24_operand *x, int pattern, int score, const float 
         return SS24_ERR_NULL;
     if (pattern != SS24_DENSE && !aligned16(out->meta))
         return SS24_ERR_ALIGN;
+    if (r.row_mode && x->hadamard != 0 && !row_amax_in)
+        return SS24_ERR_ARG; // one INT scale per row over a rotated operand: amax_rows + quantize_int_rows
+    if (!launch_it)
+        return SS24_OK;
 
     // ---- launches ----
     PassParams p = base_params(x, g, ws, energy);
@@ -658,8 +674,6 @@ ss24_status run_pass(const ss24_operand *x, int pattern, int score, const float 
             p.q.amax_reduced = p.amax_out; // [0] = amax of the quantized values
         }
     }
-    if (r.row_mode && x->hadamard != 0)
-        return SS24_ERR_ARG; // one INT scale per row over a rotated operand: amax_rows + quantize_int_rows
     cudaError_t e;
     int cpt = 0, log2_tpr = 0;
     if (r.row_mode && rowblock_plan(x->k, &cpt, &log2_tpr)) {
@@ -688,15 +702,49 @@ ss24_status run_pass(const ss24_operand *x, int pattern, int score, const float 
 // loads the library, held until the process exits. The pass needs the same
 // fixed amount whatever the operand size (partials for at most kMaxGrid CTAs).
 constexpr size_t kStaticScratchBytes = kWsBytes;
+static_assert(kStaticScratchBytes >= kWsBytes, "the array must hold the pass's whole workspace");
 static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_static_mu;
-void *g_static_ptr[kMaxDevices] = {};
+struct StaticScratch {
+    unsigned long long ctx_id = 0; // context the address belongs to (0: none yet)
+    void *ptr = nullptr;
+};
+StaticScratch g_static[kMaxDevices];
 
-// Device address of the array on the current device. Host code must not use
-// the symbol's host-side name as a pointer; the address comes from
-// cudaGetSymbolAddress, taken once per device with that device current.
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+// Process-unique ID of the current context (cuCtxGetId), through the driver
+// entry points the runtime exposes; false if it cannot be read.
+bool current_ctx_id(unsigned long long *id)
+{
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+    });
+    CUcontext ctx = nullptr;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx)
+        return false;
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of the array in the current device's context. Host code must
+// not use the symbol's host-side name as a pointer; the address comes from
+// cudaGetSymbolAddress, taken with the device current, once per device and
+// context: a context created after a device reset loads the module again, so
+// the address is looked up again when the context's ID changes.
 cudaError_t static_scratch(void **ptr)
 {
     int dev = 0;
@@ -705,15 +753,21 @@ cudaError_t static_scratch(void **ptr)
         return e;
     if (dev < 0 || dev >= kMaxDevices)
         return cudaErrorInvalidDevice;
+    // (no current context yet, e.g. on a fresh thread: the lookup below makes
+    // the device's primary context current, and the ID is read after it)
+    unsigned long long id = 0;
+    const bool have_id = current_ctx_id(&id);
     std::lock_guard<std::mutex> lock(g_static_mu);
-    if (!g_static_ptr[dev]) {
+    StaticScratch &s = g_static[dev];
+    if (!s.ptr || !have_id || s.ctx_id != id) {
         void *p = nullptr;
         e = cudaGetSymbolAddress(&p, g_static_scratch);
         if (e != cudaSuccess)
             return e;
-        g_static_ptr[dev] = p;
+        s.ptr = p;
+        s.ctx_id = current_ctx_id(&id) ? id : 0;
     }
-    *ptr = g_static_ptr[dev];
+    *ptr = s.ptr;
     return cudaSuccess;
 }
 
@@ -1273,11 +1327,19 @@ ss24_status ss24_prune24_quant_fused_noalloc(const ss24_operand *x, ss24_score s
                                              ss24_energy *energy, ss24_stream stream)
 {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (ss24_workspace_bytes() > kStaticScratchBytes)
-        return SS24_ERR_WORKSPACE; // the pass would need more scratch than the array holds
+    // the strided-axis kernel waits on its copies with a time limit and records
+    // a wait that gave up in the scratch's error word, which a caller of this
+    // entry point cannot read: only the axis-1 kernels (no such waits) run here
+    if (x && x->axis != 1)
+        return SS24_ERR_ARG;
     void *scratch = nullptr;
     if (static_scratch(&scratch) != cudaSuccess)
         return SS24_ERR_CUDA;
+    // every check first: a rejected call enqueues nothing, not even the clear
+    ss24_status st = run_pass(x, SS24_SPARSE_24, score, col_norms, fmt, true, tensor_scale_in, out, energy, scratch,
+                              kStaticScratchBytes, s, nullptr, false);
+    if (st != SS24_OK)
+        return st;
     // the error word and the ticket counters must start at zero for this call
     if (cudaMemsetAsync(scratch, 0, kWsClearBytes, s) != cudaSuccess)
         return SS24_ERR_CUDA;

@@ -25,6 +25,7 @@ OK = 0
 STATUS_NAMES = {0: "SS24_OK", 1: "SS24_ERR_NULL", 2: "SS24_ERR_SHAPE", 3: "SS24_ERR_ALIGN",
                 4: "SS24_ERR_DTYPE", 5: "SS24_ERR_FORMAT", 6: "SS24_ERR_WORKSPACE", 7: "SS24_ERR_CUDA",
                 8: "SS24_ERR_ARG"}
+STATUS_NAMES_INV = {v: k for k, v in STATUS_NAMES.items()}
 BF16, F32 = 0, 1
 MAG, WANDA = 0, 1
 DENSE, SPARSE_24, SPARSE_48 = 0, 24, 48
