@@ -79,12 +79,17 @@ def lib():
         _lib.oracle_softmax_bf16.restype = ctypes.c_int
         _lib.oracle_softmax_bf16.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                              ctypes.c_float, ctypes.c_void_p]
+        _lib.oracle_softmax_f64_bf16.restype = ctypes.c_int
+        _lib.oracle_softmax_f64_bf16.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                                 ctypes.c_float, ctypes.c_void_p]
         _lib.oracle_hadamard_bf16.restype = ctypes.c_int
         _lib.oracle_hadamard_bf16.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                               ctypes.c_int32, ctypes.c_void_p]
         _lib.oracle_amax.argtypes = [ctypes.POINTER(_Args)]
         _lib.oracle_tensor_scale.restype = ctypes.c_float
         _lib.oracle_tensor_scale.argtypes = [ctypes.POINTER(_Args)]
+        _lib.oracle_scale_of_amax.restype = ctypes.c_float
+        _lib.oracle_scale_of_amax.argtypes = [ctypes.c_float, ctypes.c_int32]
         _lib.oracle_select24.restype = ctypes.c_int
         _lib.oracle_select24.argtypes = [ctypes.c_void_p]
         _lib.oracle_select48.restype = ctypes.c_int
@@ -214,6 +219,67 @@ def tensor_scale(x, fmt, *, pattern=SPARSE_24, score=MAG, norms=None, axis=1, ro
     return float(lib().oracle_tensor_scale(ctypes.byref(args)))
 
 
+def host_threads():
+    """Host cores this process may run on (the thread count of run_parallel)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        return os.cpu_count() or 1
+
+
+def _row_blocks(rows, threads, block_rows):
+    if block_rows is None:
+        block_rows = max(1, -(-rows // (4 * threads)))
+    return [(r0, min(rows, r0 + block_rows)) for r0 in range(0, rows, block_rows)]
+
+
+def run_parallel(x, *, threads=None, block_rows=None, pattern=SPARSE_24, score=MAG, norms=None, fmt="none",
+                 bits=8, group=0, pack4=False, tensor_scale=None):
+    """run() on host threads: the rows of an axis-1 operand x [rows][k] cut into
+    contiguous blocks, each block one run() call (the C oracle, which releases
+    the interpreter lock while it runs). Each row's outputs depend on that row
+    alone once the tensor scale is fixed, so the blocks' outputs, concatenated,
+    are run()'s outputs on the whole operand. A per-tensor scale that is not
+    given is derived first, exactly as run() derives it: the amax of every
+    block (amax(), an exact maximum), their maximum, then scale_of_amax. The
+    energies are the blocks' binary64 sums added in block order (run() adds
+    the same terms in row order: equal up to the order of binary64 additions).
+    Returns run()'s dict."""
+    from concurrent.futures import ThreadPoolExecutor
+    x = np.ascontiguousarray(x)
+    rows = x.shape[0]
+    threads = threads or host_threads()
+    blocks = _row_blocks(rows, threads, block_rows)
+    fmt_id = _FMT_NAMES[fmt] if isinstance(fmt, str) else fmt
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        if fmt_id in (FMT_FP8, FMT_NVFP4) and tensor_scale is None:
+            am = list(ex.map(lambda b: amax(x[b[0]:b[1]], pattern=pattern, score=score, norms=norms), blocks))
+            tensor_scale = float(lib().oracle_scale_of_amax(max(am) if am else 0.0, fmt_id))
+        parts = list(ex.map(lambda b: run(x[b[0]:b[1]], pattern=pattern, score=score, norms=norms, fmt=fmt,
+                                          bits=bits, group=group, pack4=pack4, tensor_scale=tensor_scale),
+                            blocks))
+    if not parts:
+        return run(x, pattern=pattern, score=score, norms=norms, fmt=fmt, bits=bits, group=group, pack4=pack4,
+                   tensor_scale=tensor_scale)
+    out = {}
+    for key in parts[0]:
+        if key == "energy":
+            e = np.zeros(4, dtype=np.float64)
+            for p in parts:
+                e += p["energy"]
+            out[key] = e
+        elif key == "tensor_scale":
+            out[key] = parts[0][key]
+        else:
+            out[key] = np.concatenate([p[key] for p in parts], axis=0)
+    return out
+
+
+def scale_of_amax(a, fmt):
+    """The per-tensor scale of an amax (FP8: a / 448, NVFP4: a / 2688)."""
+    return float(lib().oracle_scale_of_amax(float(a), _FMT_NAMES[fmt] if isinstance(fmt, str) else fmt))
+
+
 def select24(s):
     s = np.ascontiguousarray(s, dtype=np.float32)
     return lib().oracle_select24(s.ctypes.data)
@@ -286,6 +352,37 @@ def softmax_bf16(s, alpha):
     out = np.empty(f.shape, dtype=np.uint16)
     if lib().oracle_softmax_bf16(f.ctypes.data, rows, k, k, float(alpha), out.ctypes.data) != 0:
         raise ValueError("oracle_softmax_bf16 rejected its arguments")
+    return out
+
+
+def softmax_f64_bf16(s, alpha, threads=1):
+    """P = softmax(alpha * s) per row from the plain definition in binary64
+    (libm exp, index-order sum), rounded once to bf16 (see
+    oracle_softmax_f64_bf16): bf16 bits of the same shape as the logits (bf16
+    bits or float32, [rows, k] or [batch, rows, k]). threads > 1 runs row
+    blocks on host threads (each row depends on itself alone)."""
+    a = np.asarray(s)
+    f = (a.astype(np.uint32) << 16).view(np.float32) if a.dtype == np.uint16 else a.astype(np.float32)
+    f = np.ascontiguousarray(f, dtype=np.float32)
+    k = f.shape[-1]
+    rows = f.size // k
+    out = np.empty(f.shape, dtype=np.uint16)
+    f2, o2 = f.reshape(rows, k), out.reshape(rows, k)
+
+    def block(b):
+        r0, r1 = b
+        if lib().oracle_softmax_f64_bf16(f2[r0:r1].ctypes.data, r1 - r0, k, k, float(alpha),
+                                         o2[r0:r1].ctypes.data) != 0:
+            raise ValueError("oracle_softmax_f64_bf16 rejected its arguments")
+
+    blocks = _row_blocks(rows, threads, None)
+    if threads > 1:
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(max_workers=threads) as ex:
+            list(ex.map(block, blocks))
+    else:
+        for b in blocks:
+            block(b)
     return out
 
 

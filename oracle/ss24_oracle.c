@@ -295,7 +295,7 @@ static int64_t quantized_row(const oracle_args *a, int64_t r, float *xr, float *
 }
 
 /* ------------------------------------------------------------------------- */
-/* Quantizers (round to nearest; §2 "plain round-to-nearest", §3 formats).    */
+/* Quantizers (round to nearest, §2; the formats, §3).                        */
 /* Each writes codes for one row vector v[n] and its dequantized values.      */
 /* ------------------------------------------------------------------------- */
 
@@ -356,7 +356,7 @@ static void quant_int_row(const qctx *q, int64_t r, const float *v, float *deq)
     }
 }
 
-/* FP8 E4M3 with one scale per tensor (§3 "FP8"; the pages fix no granularity,
+/* FP8 E4M3 with one scale per tensor (§3 names FP8; the pages fix no granularity,
  * per-tensor is the reading): s = amax / 448; code = E4M3(v / s);
  * deq = decode(code) * s; s == 0 gives zero codes. */
 static void quant_fp8_row(const qctx *q, int64_t r, const float *v, float *deq)
@@ -651,10 +651,14 @@ double oracle_bits_per_element(int32_t fmt, int32_t bits, int32_t group, int32_t
  * s = amax / 448, NVFP4 s_t = amax / (6 * 448), over the values that get
  * quantized. Lets a test check sampled rows of a large operand with the scale
  * of the whole tensor. */
+float oracle_scale_of_amax(float amax, int32_t fmt)
+{
+    return fmt == OR_FMT_FP8 ? amax / 448.0f : amax / 2688.0f;
+}
+
 float oracle_tensor_scale(const oracle_args *a)
 {
-    float amax = oracle_amax(a);
-    return a->fmt == OR_FMT_FP8 ? amax / 448.0f : amax / 2688.0f;
+    return oracle_scale_of_amax(oracle_amax(a), a->fmt);
 }
 
 /* ------------------------------------------------------------------------- */
@@ -834,7 +838,7 @@ int oracle_hadamard(const float *x, int64_t rows, int64_t k, int64_t ld, int32_t
 }
 
 /* ---- attention probabilities: P = softmax(alpha * s) per row ----------------
- * The producer of an attention operand (§3: "P" pruned along the key axis;
+ * The producer of an attention operand (§3: P pruned along the key axis;
  * the pages build it as softmax(N(0, 3) logits / sqrt(128))). A fused
  * producer computes P and prunes it in the same pass; for its results to be
  * reproducible bit for bit, the exponential and the order of the row sum are
@@ -931,6 +935,65 @@ int oracle_softmax_bf16(const float *s, int64_t rows, int64_t k, int64_t ld, flo
         }
         for (int64_t j = 0; j < k; ++j)
             p_bits[r * k + j] = f32_to_bf16_rne(e[j] / total);
+    }
+    free(e);
+    return 0;
+}
+
+/* The same probabilities as the plain definition, without the fixed choices
+ * above: v_j = RN(alpha * s_j) (the binary32 scaling of the logits), then in
+ * binary64 e_j = exp(v_j - m) with libm's exp, S = sum of e_j in index order,
+ * p_j = e_j / S, and p_j rounded once from binary64 to bf16 (nearest, ties to
+ * even). An exponential within an ulp of e^x and any accurate order of the row
+ * sum give a binary32 p within a few binary32 ulps of this p_j, so their bf16
+ * roundings differ by at most one bf16 ulp from the bf16 p_j here. Same
+ * arguments and layout as oracle_softmax_bf16 (k a multiple of 256 is not
+ * required). */
+static uint16_t f64_to_bf16_rne(double d)
+{
+    /* d >= 0 finite. bf16 has an 8-bit significand; below 2^-126 its steps
+     * are 2^-133 (subnormal). q = d / step is exact (a power-of-two scaling);
+     * nearbyint rounds it to an integer, ties to even. */
+    if (d == 0.0)
+        return 0;
+    int e;
+    (void)frexp(d, &e); /* d = f * 2^e, f in [0.5, 1) */
+    int step_exp = e - 8;
+    if (step_exp < -133)
+        step_exp = -133;
+    const double q = ldexp(d, -step_exp);
+    const double r = ldexp(nearbyint(q), step_exp); /* exactly a bf16 value */
+    union {
+        float f;
+        uint32_t u;
+    } v;
+    v.f = (float)r; /* exact */
+    return (uint16_t)(v.u >> 16);
+}
+
+int oracle_softmax_f64_bf16(const float *s, int64_t rows, int64_t k, int64_t ld, float alpha, uint16_t *p_bits)
+{
+    if (!s || !p_bits || rows < 0 || k <= 0 || ld < k)
+        return -1;
+    double *e = (double *)malloc((size_t)k * sizeof(double));
+    if (!e)
+        return -1;
+    for (int64_t r = 0; r < rows; ++r) {
+        const float *row = s + r * ld;
+        float m = alpha * row[0];
+        for (int64_t j = 1; j < k; ++j) {
+            float v = alpha * row[j];
+            if (v > m)
+                m = v;
+        }
+        double total = 0.0;
+        for (int64_t j = 0; j < k; ++j) {
+            float v = alpha * row[j];
+            e[j] = exp((double)v - (double)m);
+            total += e[j];
+        }
+        for (int64_t j = 0; j < k; ++j)
+            p_bits[r * k + j] = f64_to_bf16_rne(e[j] / total);
     }
     free(e);
     return 0;

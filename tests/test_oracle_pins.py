@@ -702,3 +702,58 @@ def test_hadamard_bf16_is_the_nearest_bf16_of_the_rotation():
     e[0, 5] = 1.0
     got = (oracle.hadamard_bf16(e, 16).astype(np.uint32) << 16).view(np.float32)[0]
     assert np.array_equal(np.abs(got[:16]), np.full(16, 0.25, dtype=np.float32)) and not got[16:].any()
+
+
+@pytest.mark.parametrize("pattern,fmt,bits,group,score", [
+    (oracle.SPARSE_24, "nvfp4", 4, 0, "mag"), (oracle.SPARSE_48, "nvfp4", 4, 0, "mag"),
+    (oracle.SPARSE_24, "fp8", 8, 0, "mag"), (oracle.DENSE, "fp8", 8, 0, "mag"),
+    (oracle.DENSE, "int", 8, 0, "mag"), (oracle.SPARSE_24, "int", 4, 128, "wanda"),
+    (oracle.SPARSE_48, "fp8", 8, 0, "wanda"), (oracle.DENSE, "mxfp4", 4, 0, "mag"),
+    (oracle.SPARSE_24, "none", 8, 0, "mag")])
+def test_threaded_driver_equals_the_plain_oracle(pattern, fmt, bits, group, score):
+    """run_parallel (row blocks on host threads; the tensor scale from the
+    blocks' amax) against one plain run() over the whole operand: outputs bit
+    for bit, energies equal up to the order of the binary64 additions. Ragged
+    blocks of 37 rows, and one block per row."""
+    xh = synth.sweep_operand(300, 1024, seed=81)
+    norms = synth.linear_weight(4, 1024, seed=82)[1] if score == "wanda" else None
+    kw = dict(pattern=pattern, fmt=fmt, bits=bits, group=group, norms=norms,
+              score=oracle.WANDA if score == "wanda" else oracle.MAG)
+    ref = oracle.run(xh, **kw)
+    for block_rows in (37, 1):
+        got = oracle.run_parallel(xh, block_rows=block_rows, threads=4, **kw)
+        assert set(got) == set(ref)
+        for key in ref:
+            if key == "energy":
+                np.testing.assert_allclose(got[key], ref[key], rtol=1e-10, atol=0.0)
+            else:
+                assert np.array_equal(np.ascontiguousarray(got[key]).view(np.uint8),
+                                      np.ascontiguousarray(ref[key]).view(np.uint8)), key
+
+
+def test_binary64_softmax_is_the_nearest_bf16_of_the_library_softmax():
+    """oracle.softmax_f64_bf16 against scipy's softmax in binary64 of the same
+    binary32 scaled logits: every output is the nearer of the two bf16 values
+    around scipy's (ties, to within 1e-12, may go either way; an exact tie goes
+    to the even pattern); a constant row gives exactly 1/k; a row with one
+    dominant logit gives 1 there and 0 elsewhere; row blocks on threads give
+    the same bits."""
+    rng = np.random.default_rng(61)
+    s = (rng.standard_normal((48, 1024)) * 3.0).astype(np.float32)
+    alpha = np.float32(1.0 / math.sqrt(128.0))
+    got = oracle.softmax_f64_bf16(s, float(alpha))
+    assert np.array_equal(got, oracle.softmax_f64_bf16(s, float(alpha), threads=4))
+    ref = special.softmax((s * alpha).astype(np.float32).astype(np.float64), axis=1)
+    g = (got.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    t = (ref.astype(np.float32).view(np.uint32) >> 16).astype(np.uint32)      # a bf16 pattern near ref
+    cands = [((np.clip(t.astype(np.int64) + d, 0, 0x7f7f).astype(np.uint32) << 16).view(np.float32))
+             .astype(np.float64) for d in (-1, 0, 1)]
+    dist = np.stack([np.abs(c - ref) for c in cands])
+    best = dist.min(axis=0)
+    assert np.all(np.abs(g - ref) <= best * (1 + 1e-12) + 1e-300)
+    const = oracle.softmax_f64_bf16(np.full((2, 1024), -1.25, dtype=np.float32), 1.0)
+    assert np.all(const == 0x3A80)                                   # 2^-10, exactly
+    spike = np.zeros((1, 256), dtype=np.float32)
+    spike[0, 9] = 900.0
+    ps = (oracle.softmax_f64_bf16(spike, 1.0).astype(np.uint32) << 16).view(np.float32)[0]
+    assert ps[9] == 1.0 and np.count_nonzero(ps) == 1
