@@ -898,60 +898,64 @@ def test_repeated_calls_are_deterministic(ss, ws):
 
 
 # --------------------------------------------------------------------------
-# full-size configurations: sampled rows against the oracle, energies by
-# properties that hold at any size
+# full-size configurations: every output of the whole tensor against the
+# oracle (run on all host cores, row blocks), all four energies to 1e-6
 # --------------------------------------------------------------------------
 
-def sampled_check(ss, ws, xh, *, pattern, fmt, bits=8, group=0, score="mag", norms=None, n_rows=48, seed=0):
+def full_check(ss, ws, xh, *, pattern, fmt, bits=8, group=0, pack4=False, score="mag", norms=None):
+    """One pass over the whole operand on the GPU (tensor scale derived by the
+    library when the format has one) against oracle.run_parallel on the same
+    bytes: codes, scales, metadata and tensor scale bit for bit, the four
+    energies within 1e-6 relative."""
     x = to_dev(xh)
     nd = to_dev(norms) if norms is not None else None
-    out = ss.run(x, pattern=pattern, fmt=fmt, bits=bits, group=group, score=score, col_norms=nd, ws=ws)
+    out = ss.run(x, pattern=pattern, fmt=fmt, bits=bits, group=group, pack4=pack4, score=score, col_norms=nd, ws=ws)
     torch.cuda.synchronize()
+    assert ws.error() == 0
+    got = {key: to_np(t) for key, t in out.items() if key != "energy"}
+    energy = out["energy"]
+    del out, x
     sc = oracle.WANDA if score == "wanda" else oracle.MAG
     opat = {0: oracle.DENSE, 24: oracle.SPARSE_24, 48: oracle.SPARSE_48}[pattern]
-    ts = None
-    if fmt in ("fp8", "nvfp4"):
-        ts = oracle.tensor_scale(xh, fmt, pattern=opat, score=sc, norms=norms)
-        assert out["tensor_scale"].item() == np.float32(ts)
-    rng = np.random.default_rng(seed)
-    rows = np.unique(np.concatenate([[0, xh.shape[0] - 1], rng.integers(0, xh.shape[0], n_rows)]))
-    ref = oracle.run(xh[rows], pattern=opat, fmt=fmt, bits=bits, group=group, score=sc, norms=norms,
-                     tensor_scale=ts)
-    for key in ("values", "scales", "meta"):
+    ref = oracle.run_parallel(xh, pattern=opat, fmt=fmt, bits=bits, group=group, pack4=pack4, score=sc,
+                              norms=norms)
+    for key in ("values", "scales", "meta", "tensor_scale"):
         if key in ref:
-            assert_same(to_np(out[key][torch.from_numpy(rows).cuda()]), ref[key], key)
-    # E_total of the whole tensor, summed independently in binary64
-    xf = synth.bf16_to_f32(xh).astype(np.float64) if xh.dtype == np.uint16 else xh.astype(np.float64)
-    e = out["energy"].cpu().numpy()
-    et = float(np.einsum("ij,ij->", xf, xf))
-    assert abs(e[0] - et) <= RTOL * et
-    assert ws.error() == 0
-    return e
+            assert_same(got[key], ref[key], key)
+    assert_energy(energy, ref["energy"], atol=1e-30)
+    return energy.cpu().numpy()
 
 
 def test_full_linear_input_fp8_and_int8_per_row(ss, ws):
+    """Linear input X 4096 x 4096 (Student-t, 8 outlier channels x50): fused
+    2:4 + FP8 and its dense FP8 and INT8-per-row partners."""
     xh, _ = synth.linear_input(4096, 4096, seed=1)
-    e = sampled_check(ss, ws, xh, pattern=24, fmt="fp8")
+    e = full_check(ss, ws, xh, pattern=24, fmt="fp8")
     assert 0.0 < e[1] / e[0] < 0.5
-    sampled_check(ss, ws, xh, pattern=0, fmt="fp8")
-    sampled_check(ss, ws, xh, pattern=0, fmt="int", bits=8, group=0)
+    full_check(ss, ws, xh, pattern=0, fmt="fp8")
+    full_check(ss, ws, xh, pattern=0, fmt="int", bits=8, group=0)
 
 
 def test_full_weight_wanda_int(ss, ws):
+    """Linear weight W 14336 x 4096 with Wanda scores: 2:4 + INT(2m) g128 against
+    dense INT(m+1) g128, m = 2, 4, 8 (INT4 packed, INT8, INT16; INT3 packed,
+    INT5, INT9)."""
     w, norms = synth.linear_weight(14336, 4096, seed=2)
     for m in (2, 4, 8):
-        sampled_check(ss, ws, w, pattern=24, fmt="int", bits=2 * m, group=128, score="wanda", norms=norms,
-                      n_rows=16, seed=m)
-        sampled_check(ss, ws, w, pattern=0, fmt="int", bits=m + 1, group=128, n_rows=16, seed=m)
+        full_check(ss, ws, w, pattern=24, fmt="int", bits=2 * m, group=128, pack4=m == 2, score="wanda",
+                   norms=norms)
+        full_check(ss, ws, w, pattern=0, fmt="int", bits=m + 1, group=128, pack4=m == 2)
 
 
 def test_full_attention_operands(ss, ws):
+    """Q (32 heads x 8192 x 128) pruned along d: 2:4 + FP8 against dense NVFP4
+    and MXFP4; P (32 x 2048 x 2048) pruned along the keys: 2:4 + FP8."""
     q = synth.attention_qkv(seed=4)
-    sampled_check(ss, ws, q, pattern=24, fmt="fp8")
-    sampled_check(ss, ws, q, pattern=0, fmt="nvfp4")
-    sampled_check(ss, ws, q, pattern=0, fmt="mxfp4")
+    full_check(ss, ws, q, pattern=24, fmt="fp8")
+    full_check(ss, ws, q, pattern=0, fmt="nvfp4")
+    full_check(ss, ws, q, pattern=0, fmt="mxfp4")
     p = synth.attention_probs(seed=7)
-    sampled_check(ss, ws, p, pattern=24, fmt="fp8", n_rows=16)
+    full_check(ss, ws, p, pattern=24, fmt="fp8")
 
 
 def test_full_attention_softmax_prune(ss, ws):
@@ -977,9 +981,81 @@ def test_full_attention_softmax_prune(ss, ws):
     assert ws.error() == 0
 
 
+def _bf16_ulp(v):
+    """Spacing of bf16 values at |v| (2^-133 below the normal range)."""
+    e = np.floor(np.log2(np.maximum(np.abs(v), 2.0 ** -126)))
+    return np.exp2(e - 7.0)
+
+
+def _meta24_of(p):
+    """Metadata of 2:4 selection by magnitude on p [rows, k] (ties keep the lower
+    index): one nibble i0 | i1 << 2 per group, two groups per byte."""
+    g = np.abs(p.reshape(p.shape[0], -1, 4))
+    beaten = np.zeros(g.shape, dtype=np.int32)
+    for i in range(4):
+        for j in range(4):
+            if i != j:
+                beaten[..., i] += (g[..., j] > g[..., i]) | ((g[..., j] == g[..., i]) & (j < i))
+    kept = beaten < 2
+    idx = np.argsort(~kept, axis=-1, kind="stable")[..., :2]            # kept positions, ascending
+    nib = (idx[..., 0] | (idx[..., 1] << 2)).astype(np.uint8)
+    return (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8)
+
+
+def test_full_softmax_prune_against_binary64_softmax(ss, ws):
+    """The softmax producer checked against the plain definition, independently
+    of the exponential and summation order it fixes: P for 32 heads x 2048 x
+    2048 keys (logits N(0, 3^2), alpha = 1/sqrt(128)) pruned 2:4 with bf16
+    kept values, against softmax in binary64 (libm exp, index-order sum)
+    rounded once to bf16:
+      - every kept value within one bf16 ulp of the binary64 P at its position;
+      - the metadata equal to the selection on the binary64 P in every group
+        whose second and third largest values are further apart than the sum
+        of their ulps (where one ulp of error each cannot swap them);
+      - E_total within 2^-6 relative of the binary64 P's energy."""
+    import oracle as orc
+    s = synth.attention_logits(seed=9)
+    alpha = float(np.float32(1.0 / math.sqrt(128)))
+    out = ss.softmax_prune(to_dev(s), alpha, pattern=24, fmt="none", ws=ws)
+    torch.cuda.synchronize()
+    assert ws.error() == 0
+    kept = (to_np(out["values"]).astype(np.uint32) << 16).view(np.float32)
+    meta = to_np(out["meta"])
+    e_total = out["energy"].cpu().numpy()[0]
+    del out
+    pref = orc.softmax_f64_bf16(s, alpha, threads=orc.host_threads())
+    rows, k = pref.shape
+    checked = total = 0
+    e_ref = 0.0
+    for r0 in range(0, rows, 4096):
+        r1 = min(rows, r0 + 4096)
+        p = (pref[r0:r1].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        e_ref += float(np.einsum("ij,ij->", p, p))
+        m = meta[r0:r1]
+        nib = np.stack([m & 0xF, m >> 4], axis=-1).reshape(r1 - r0, -1)      # [rows, groups]
+        i0, i1 = nib & 3, nib >> 2
+        g = p.reshape(r1 - r0, -1, 4)
+        at = np.stack([np.take_along_axis(g, i0[..., None], -1)[..., 0],
+                       np.take_along_axis(g, i1[..., None], -1)[..., 0]], axis=-1).reshape(r1 - r0, -1)
+        kv = kept[r0:r1].astype(np.float64)
+        assert np.all(np.abs(kv - at) <= _bf16_ulp(at)), "a kept value is more than one bf16 ulp off"
+        srt = -np.sort(-g, axis=-1)
+        sep = (srt[..., 1] - srt[..., 2]) > _bf16_ulp(srt[..., 1]) + _bf16_ulp(srt[..., 2])
+        ref_meta = _meta24_of(p)
+        ref_nib = np.stack([ref_meta & 0xF, ref_meta >> 4], axis=-1).reshape(r1 - r0, -1)
+        assert np.array_equal(nib[sep], ref_nib[sep]), "selection differs where the order is not in doubt"
+        checked += int(sep.sum())
+        total += sep.size
+    assert checked > 0.9 * total
+    assert abs(e_total - e_ref) <= 2.0 ** -6 * e_ref
+
+
 @pytest.mark.parametrize("tokens,k", [(2048, 4096), (16384, 14336)])
 def test_full_sweep_nvfp4(ss, ws, tokens, k):
+    """The throughput sweep's smallest and largest shapes (0.1% outliers x100):
+    2:4 + NVFP4, pairwise 4:8 + NVFP4 and 2:4 with bf16 kept values, whole
+    tensors."""
     xh = synth.sweep_operand(tokens, k, seed=8)
-    sampled_check(ss, ws, xh, pattern=24, fmt="nvfp4", n_rows=12)
-    sampled_check(ss, ws, xh, pattern=48, fmt="nvfp4", n_rows=12)
-    sampled_check(ss, ws, xh, pattern=24, fmt="none", n_rows=12)
+    full_check(ss, ws, xh, pattern=24, fmt="nvfp4")
+    full_check(ss, ws, xh, pattern=48, fmt="nvfp4")
+    full_check(ss, ws, xh, pattern=24, fmt="none")
