@@ -1,26 +1,44 @@
 """Benchmark of the online 2:4 prune + compress + quantize + error-energy path.
 
-Workload (one step): a batch of B = 8 linear-layer inputs X, each bf16
-4096 x 4096, Student-t (nu = 4, unit variance) with 8 outlier channels x50.
-A step runs every row of the hot path once over the batch, pass by pass; each
-pass is one batched call over all 8 operands (one kernel launch), so each
-pass reads its operands from HBM (the batch is 256 MiB, twice the L2):
-  1. per-tensor FP8 scale and per-row amax of each X       ss24_amax_rows
-  2. fused 2:4 magnitude prune + compress + FP8 E4M3 of the
-     kept values + energies (E_total, E_prune, E_q)        ss24_prune24_quant_fused
-  3. dense FP8 E4M3 partner (same scale) + energy          ss24_quantize_fp8
-  4. dense INT8, one scale per row (from the row amax),
-     partner + energy                                      ss24_quantize_int_rows
-  5. predicted R against both partners (one launch each)   ss24_predicted_ratio
-The whole step is one CUDA graph, the passes chained by programmatic dependent
-launch. Every 8th step of the timed region instead replays a copy of that graph
-with an event-record node at every pass boundary, the nodes pointed at that
-step's own events: the per-kernel durations are CUDA events on the launching
-stream inside the timed region (an event node ends the overlap of the launches
-it separates, so those steps are a little slower, and are counted).
+The headline is the fused pass of the throughput sweep's largest shape: one
+bf16 operand X of 16384 tokens x 14336 (N(0,1) with 0.1% of the elements x100),
+2:4 magnitude prune + compress + NVFP4 of the kept values + energies, the
+tensor scale given. `value` is that pass's own GB/s of algorithmic bytes,
+timed with CUDA events on its launching stream inside the timed region.
+
+One step runs every row of the hot path once, each pass one launch (batched
+operands share a launch), in this order:
+  throughput sweep X, 16384 x 14336 bf16 (448 MiB)
+    sweep_scale          NVFP4 tensor scale (amax pass)            ss24_tensor_scale
+    sweep_fused_24_nvfp4 2:4 + NVFP4, scale given, energies (HEADLINE) ss24_prune24_quant_fused
+    sweep_fused_48_nvfp4 pairwise 4:8 + NVFP4, scale given, energies ss24_prune48_pairwise_quant_fused
+    sweep_compress_24    2:4 prune + compress, bf16 kept values      ss24_prune24_compress
+    sweep_dense_nvfp4    dense NVFP4 partner, scale given, energy    ss24_quantize_nvfp4
+    sweep_ratio          R of 2:4 and of 4:8 against dense NVFP4     ss24_predicted_ratio (2 launches)
+  linear inputs, 8 x 4096 x 4096 bf16 (Student-t, 8 outlier channels x50)
+    linear_scale_rows    FP8 tensor scale + per-row amax             ss24_amax_rows
+    linear_fused_24_fp8  2:4 + FP8, energies                         ss24_prune24_quant_fused
+    linear_dense_fp8     dense FP8 partner, energy                   ss24_quantize_fp8
+    linear_dense_int8_row dense INT8 one scale per row, energy       ss24_quantize_int_rows
+    linear_ratio         R against both partners                     ss24_predicted_ratio (2 launches)
+  linear weight W, 14336 x 4096 bf16, Wanda score (lognormal column norms)
+    weight_wanda_24_int4 Wanda 2:4 + INT4 g128 (packed), energies    ss24_prune24_quant_fused
+    weight_dense_int3    dense INT3 g128 equal-bit partner (packed)  ss24_quantize_int
+    weight_ratio         R                                           ss24_predicted_ratio
+  attention V, 32 heads x 8192 keys x 128 bf16, pruned along the keys
+    v_keys_24_fp8        strided axis: FP8 scale pass + 2:4 + FP8    ss24_prune24_quant_fused (2 launches)
+Every operand is larger than the L2 or each pass starts where the previous
+one's reads are no longer cached (each pass reads its operand from HBM).
+
+The step is one CUDA graph, with an event-record node at every pass boundary;
+before each replay the nodes are pointed at that step's own events, so every
+pass of every timed step is timed by CUDA events on the launching stream.
+The contract's timed region is exactly --steps steps. When it is shorter than
+a second, a sustained region of the same evented steps follows (at least one
+second) and reports the same per-pass statistics.
 
 Prints ONE JSON line (rank 0). ``--impl reference`` times the CPU oracle on a
-bounded sample of the same workload instead.
+bounded sample of the headline workload instead.
 """
 from __future__ import annotations
 
@@ -38,47 +56,67 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "fused 2:4 prune+compress+quant HBM GB/s and % of peak/memcpy; Gelem/s"
-WORKLOAD = ("linear-input X bf16 4096x4096 (Student-t nu=4 /sqrt2, 8 outlier channels x50), batch of 8 per step: "
-            "FP8 tensor scale, fused 2:4 magnitude prune+compress+FP8 E4M3 kept values, dense FP8 and dense INT8 "
-            "per-row partners, energies, predicted R")
-M = K = 4096
-BATCH = 8
-EVENT_EVERY = 8   # steps per evented step in the timed region
+HEADLINE = "sweep_fused_24_nvfp4"
+SWEEP_M, SWEEP_K = 16384, 14336
+LIN_B, LIN_M, LIN_K = 8, 4096, 4096
+W_M, W_K = 14336, 4096
+V_H, V_KEYS, V_D = 32, 8192, 128
+WORKLOAD = (f"throughput sweep operand X bf16 {SWEEP_M}x{SWEEP_K} (N(0,1), 0.1% of elements x100): fused 2:4 "
+            "magnitude prune+compress+NVFP4 (16-value E4M3 block scales + fp32 tensor scale, given) of the kept "
+            "values with error energies; the step also runs the hot path's other rows (tensor scale, pairwise "
+            "4:8+NVFP4, bf16 compression, dense NVFP4 partner, R; FP8 / INT8-per-row on 8 linear inputs "
+            "4096x4096; Wanda 2:4+INT4 g128 vs dense INT3 on a 14336x4096 weight; V 32x8192x128 along the keys)")
+SUSTAIN_S = 1.0
 
 
-def algorithmic_bytes(m=M, k=K):
-    """Bytes each pass must move per operand (bf16 in; see the DESIGN notes)."""
-    n = m * k
+def _n(m, k):
+    return m * k
+
+
+def pass_bytes():
+    """Algorithmic bytes of each pass of the step: every input element read once
+    (2 bytes, bf16) and every output byte written once (codes, scales,
+    metadata); the energy records, tensor scales and workspace partials (a few
+    hundred bytes) are not counted."""
+    ns = _n(SWEEP_M, SWEEP_K)
+    nl = _n(LIN_M, LIN_K)
+    nw = _n(W_M, W_K)
+    nv = V_H * V_KEYS * V_D
     return {
-        "tensor_scale": 2 * n + 4 * m,                 # read X; write the row amax
-        "fused_24_fp8": 2 * n + n // 2 + n // 8,       # read X; write FP8 codes (k/2) + metadata (k/8)
-        "dense_fp8": 2 * n + n,                        # read X; write FP8 codes
-        "dense_int8_row": 2 * n + 4 * m + n + 4 * m,   # read X and the row amax; write INT8 codes + row scales
-        "ratio": 0,
+        "sweep_scale": 2 * ns,
+        # codes (k/2 kept values, 4 bits), E4M3 scales (one per 16 kept), metadata (4 bits per 4)
+        "sweep_fused_24_nvfp4": 2 * ns + ns // 4 + ns // 32 + ns // 8,
+        "sweep_fused_48_nvfp4": 2 * ns + ns // 4 + ns // 32 + ns // 16,
+        "sweep_compress_24": 2 * ns + ns + ns // 8,
+        "sweep_dense_nvfp4": 2 * ns + ns // 2 + ns // 16,
+        "sweep_ratio": 0,
+        "linear_scale_rows": LIN_B * (2 * nl + 4 * LIN_M),
+        "linear_fused_24_fp8": LIN_B * (2 * nl + nl // 2 + nl // 8),
+        "linear_dense_fp8": LIN_B * (2 * nl + nl),
+        "linear_dense_int8_row": LIN_B * (2 * nl + 4 * LIN_M + nl + 4 * LIN_M),
+        "linear_ratio": 0,
+        # packed INT4 codes of k/2 kept values, fp32 scale per 128 kept, metadata
+        "weight_wanda_24_int4": 2 * nw + 4 * W_K + nw // 4 + 4 * (nw // 2 // 128) + nw // 8,
+        "weight_dense_int3": 2 * nw + nw // 2 + 4 * (nw // 128),
+        "weight_ratio": 0,
+        # an amax read, then the fused pass: read, FP8 codes, metadata
+        "v_keys_24_fp8": 2 * nv + (2 * nv + nv // 2 + nv // 8),
     }
 
 
-# The sources the step's kernels are built from: the stream kernel (its
-# template, helpers, dispatch and bf16 instantiations), the ratio kernel and the
-# launch code. The ncu traffic figures are valid while these hash the same.
-STEP_KERNEL_SOURCES = ("device.cuh", "internal.cuh", "pass_impl.cuh", "pass_dispatch.cuh", "pass_bf16.cu",
-                       "misc.cu", "abi.cu")
-
-
-def kernel_source_sha():
-    """Hash of the step kernels' CUDA sources (the ncu traffic figures are valid for one)."""
-    import hashlib
-    h = hashlib.sha256()
-    src = os.path.join(ROOT, "semi_structured_sparsity_online_b200", "csrc")
-    for name in STEP_KERNEL_SOURCES:
-        with open(os.path.join(src, name), "rb") as fh:
-            h.update(fh.read())
-    return h.hexdigest()[:16]
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
 
 
 def measured_traffic(pass_name):
-    """DRAM bytes per launch of a pass from the committed ncu capture, or None
-    when the kernels changed since it was taken."""
+    """DRAM bytes per launch of a step pass from the committed ncu capture
+    (profiles/traffic.json), or None when the kernels changed since it was
+    taken (the file records the hash of the kernel sources it belongs to)."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             t = json.load(f)
@@ -89,13 +127,16 @@ def measured_traffic(pass_name):
     return t.get(pass_name)
 
 
-def load_peaks():
-    try:
-        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            p = json.load(f)
-        return float(p["hbm_gbs"]), "measured"
-    except Exception:
-        return 6650.0, "fallback"
+def kernel_source_sha():
+    """Hash of the CUDA sources the step's kernels are built from."""
+    import hashlib
+    h = hashlib.sha256()
+    src = os.path.join(ROOT, "semi_structured_sparsity_online_b200", "csrc")
+    for name in sorted(os.listdir(src)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(src, name), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()[:16]
 
 
 # ---------------------------------------------------------------------------
@@ -120,20 +161,24 @@ class ClockSampler:
         except Exception:
             self.max_mhz = None
 
+    def _sample(self):
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            for bit, name in self.REASONS.items():
+                if r & bit and name != "gpu_idle":
+                    self.reasons.add(name)
+        except Exception:
+            pass
+
     def _run(self):
         while not self._stop.is_set():
-            try:
-                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
-                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                for bit, name in self.REASONS.items():
-                    if r & bit and name != "gpu_idle":
-                        self.reasons.add(name)
-            except Exception:
-                pass
-            time.sleep(0.02)
+            self._sample()
+            time.sleep(0.01)
 
     def __enter__(self):
         if self.ok:
+            self._sample()
             self.t = threading.Thread(target=self._run, daemon=True)
             self.t.start()
         return self
@@ -153,15 +198,6 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # the CUDA path
 # ---------------------------------------------------------------------------
-
-def make_batch(seed0=1):
-    from semi_structured_sparsity_online_b200 import synth
-    xs = []
-    for b in range(BATCH):
-        x, _ = synth.linear_input(M, K, seed=seed0 + b)
-        xs.append(x)
-    return xs
-
 
 class Cudart:
     """The few runtime calls torch does not expose: event-record nodes in a
@@ -216,64 +252,127 @@ class Cudart:
                    "cudaGraphExecEventRecordNodeSetEvent")
 
 
-class Step:
-    """Device buffers and per-pass CUDA graphs for one step over the batch.
-    Each pass is one batched call (one kernel launch over all 8 operands)."""
+def host_inputs(seed_offset=0):
+    """The step's operands on the host (numpy bf16 bits / fp32), seeded."""
+    from semi_structured_sparsity_online_b200 import synth
+    so = seed_offset
+    sweep = synth.sweep_operand(SWEEP_M, SWEEP_K, seed=8 + so)
+    lin = np.stack([synth.linear_input(LIN_M, LIN_K, seed=1 + b + so)[0] for b in range(LIN_B)])
+    w, norms = synth.linear_weight(W_M, W_K, seed=2 + so)
+    # V of every head stored [keys][d]: the operand pruned along the keys is
+    # A[r = d][c = key] at v[key * 128 + d] (axis 0)
+    v = synth.attention_qkv(V_H, V_KEYS, V_D, seed=6 + so).reshape(V_H, V_KEYS, V_D)
+    return {"sweep": sweep, "lin": lin, "w": w, "norms": norms, "v": v}
 
-    def __init__(self, ss, x_dev, stream):
+
+class Step:
+    """Device buffers and the step's passes (each one launch, or two where noted)."""
+
+    def __init__(self, ss, dev, stream, hx):
         import torch
-        self.ss, self.torch, self.stream = ss, torch, stream
-        self.x = x_dev                                                # [BATCH, M, K]
-        dev = x_dev.device
+        self.ss, self.torch, self.stream, self.dev = ss, torch, stream, dev
+        bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)  # noqa: E731
+        self.h = {"sweep": bf(hx["sweep"]).pin_memory(), "lin": bf(hx["lin"]), "w": bf(hx["w"]),
+                  "v": bf(hx["v"])}
+        self.x = {key: t.to(dev) for key, t in self.h.items()}
+        self.norms = torch.from_numpy(hx["norms"]).to(dev)
         self.ws = ss.Workspace(dev, stream)
-        self.scale = torch.empty(BATCH, dtype=torch.float32, device=dev)
-        self.row_amax = torch.empty((BATCH, M), dtype=torch.float32, device=dev)
-        self.sp = ss._alloc_outputs(M, K, ss.SPARSE_24, ss.make_format("fp8"), torch.bfloat16, dev, BATCH)
-        self.d8 = ss._alloc_outputs(M, K, ss.DENSE, ss.make_format("fp8"), torch.bfloat16, dev, BATCH)
-        self.di = ss._alloc_outputs(M, K, ss.DENSE, ss.make_format("int", 8, 0), torch.bfloat16, dev, BATCH)
-        self.e = torch.zeros((3, BATCH, 4), dtype=torch.float64, device=dev)   # sparse, dense fp8, dense int8
-        self.r = torch.zeros((2, BATCH, 4), dtype=torch.float64, device=dev)   # R vs fp8, R vs int8
-        self.passes = ["tensor_scale", "fused_24_fp8", "dense_fp8", "dense_int8_row", "ratio"]
-        self.launches_per_step = 4 + 2
+        f = ss.make_format
+        self.s_scale = torch.empty(1, dtype=torch.float32, device=dev)
+        self.s24 = ss._alloc_outputs(SWEEP_M, SWEEP_K, ss.SPARSE_24, f("nvfp4"), torch.bfloat16, dev)
+        self.s48 = ss._alloc_outputs(SWEEP_M, SWEEP_K, ss.SPARSE_48, f("nvfp4"), torch.bfloat16, dev)
+        self.s24n = ss._alloc_outputs(SWEEP_M, SWEEP_K, ss.SPARSE_24, f("none"), torch.bfloat16, dev)
+        self.sd = ss._alloc_outputs(SWEEP_M, SWEEP_K, ss.DENSE, f("nvfp4"), torch.bfloat16, dev)
+        self.se = torch.zeros((4, 4), dtype=torch.float64, device=dev)      # 2:4, 4:8, compress, dense
+        self.sr = torch.zeros((2, 4), dtype=torch.float64, device=dev)
+        self.l_scale = torch.empty(LIN_B, dtype=torch.float32, device=dev)
+        self.l_rows = torch.empty((LIN_B, LIN_M), dtype=torch.float32, device=dev)
+        self.l24 = ss._alloc_outputs(LIN_M, LIN_K, ss.SPARSE_24, f("fp8"), torch.bfloat16, dev, LIN_B)
+        self.ld8 = ss._alloc_outputs(LIN_M, LIN_K, ss.DENSE, f("fp8"), torch.bfloat16, dev, LIN_B)
+        self.ldi = ss._alloc_outputs(LIN_M, LIN_K, ss.DENSE, f("int", 8, 0), torch.bfloat16, dev, LIN_B)
+        self.le = torch.zeros((3, LIN_B, 4), dtype=torch.float64, device=dev)
+        self.lr = torch.zeros((2, LIN_B, 4), dtype=torch.float64, device=dev)
+        self.w24 = ss._alloc_outputs(W_M, W_K, ss.SPARSE_24, f("int", 4, 128, True), torch.bfloat16, dev)
+        self.wd = ss._alloc_outputs(W_M, W_K, ss.DENSE, f("int", 3, 128, True), torch.bfloat16, dev)
+        self.we = torch.zeros((2, 4), dtype=torch.float64, device=dev)
+        self.wr = torch.zeros(4, dtype=torch.float64, device=dev)
+        self.v24 = ss._alloc_outputs(V_D, V_KEYS, ss.SPARSE_24, f("fp8"), torch.bfloat16, dev, V_H)
+        self.ve = torch.zeros((V_H, 4), dtype=torch.float64, device=dev)
+        # (name, launches)
+        self.passes = [("sweep_scale", 1), ("sweep_fused_24_nvfp4", 1), ("sweep_fused_48_nvfp4", 1),
+                       ("sweep_compress_24", 1), ("sweep_dense_nvfp4", 1), ("sweep_ratio", 2),
+                       ("linear_scale_rows", 1), ("linear_fused_24_fp8", 1), ("linear_dense_fp8", 1),
+                       ("linear_dense_int8_row", 1), ("linear_ratio", 2),
+                       ("weight_wanda_24_int4", 1), ("weight_dense_int3", 1), ("weight_ratio", 1),
+                       ("v_keys_24_fp8", 2)]
+        self.names = [p for p, _ in self.passes]
+        self.launches_per_step = sum(n for _, n in self.passes)
 
     def run_pass(self, name):
-        ss, s, x = self.ss, self.stream, self.x
-        if name == "tensor_scale":
-            # the FP8 tensor scale and the per-row amax of the INT8 partner in
-            # one read (magnitude score: the kept amax equals the amax of all)
-            ss.amax_rows(x, pattern=ss.DENSE, scale_fmt="fp8", ws=self.ws, stream=s, out=self.row_amax,
-                         scale_out=self.scale)
-        elif name == "fused_24_fp8":
-            ss.run(x, pattern=ss.SPARSE_24, fmt="fp8", tensor_scale=self.scale, energy=self.e[0], ws=self.ws,
-                   stream=s, out=self.sp)
-        elif name == "dense_fp8":
-            # for the magnitude score the kept amax equals the amax of all values,
-            # so the 2:4 scales are the dense FP8 scales too
-            ss.run(x, pattern=ss.DENSE, fmt="fp8", tensor_scale=self.scale, energy=self.e[1], ws=self.ws,
-                   stream=s, out=self.d8)
-        elif name == "dense_int8_row":
-            ss.run_int_rows(x, self.row_amax, pattern=ss.DENSE, bits=8, energy=self.e[2], ws=self.ws, stream=s,
-                            out=self.di)
-        elif name == "ratio":
-            ss.predicted_ratio(self.e[0], self.e[1], out=self.r[0], stream=s)
-            ss.predicted_ratio(self.e[0], self.e[2], out=self.r[1], stream=s)
+        ss, s, ws = self.ss, self.stream, self.ws
+        xs, xl, xw = self.x["sweep"], self.x["lin"], self.x["w"]
+        if name == "sweep_scale":
+            # 2:4 by magnitude keeps every group's largest value: the kept amax is
+            # the amax of all values, and one scale serves the three NVFP4 passes
+            ss.tensor_scale(xs, "nvfp4", ss.SPARSE_24, ws=ws, stream=s, out=self.s_scale)
+        elif name == "sweep_fused_24_nvfp4":
+            ss.run(xs, pattern=ss.SPARSE_24, fmt="nvfp4", tensor_scale=self.s_scale, energy=self.se[0], ws=ws,
+                   stream=s, out=self.s24)
+        elif name == "sweep_fused_48_nvfp4":
+            ss.run(xs, pattern=ss.SPARSE_48, fmt="nvfp4", tensor_scale=self.s_scale, energy=self.se[1], ws=ws,
+                   stream=s, out=self.s48)
+        elif name == "sweep_compress_24":
+            ss.run(xs, pattern=ss.SPARSE_24, fmt="none", energy=self.se[2], ws=ws, stream=s, out=self.s24n)
+        elif name == "sweep_dense_nvfp4":
+            ss.run(xs, pattern=ss.DENSE, fmt="nvfp4", tensor_scale=self.s_scale, energy=self.se[3], ws=ws,
+                   stream=s, out=self.sd)
+        elif name == "sweep_ratio":
+            ss.predicted_ratio(self.se[0], self.se[3], out=self.sr[0], stream=s)
+            ss.predicted_ratio(self.se[1], self.se[3], out=self.sr[1], stream=s)
+        elif name == "linear_scale_rows":
+            ss.amax_rows(xl, pattern=ss.DENSE, scale_fmt="fp8", ws=ws, stream=s, out=self.l_rows,
+                         scale_out=self.l_scale)
+        elif name == "linear_fused_24_fp8":
+            ss.run(xl, pattern=ss.SPARSE_24, fmt="fp8", tensor_scale=self.l_scale, energy=self.le[0], ws=ws,
+                   stream=s, out=self.l24)
+        elif name == "linear_dense_fp8":
+            ss.run(xl, pattern=ss.DENSE, fmt="fp8", tensor_scale=self.l_scale, energy=self.le[1], ws=ws, stream=s,
+                   out=self.ld8)
+        elif name == "linear_dense_int8_row":
+            ss.run_int_rows(xl, self.l_rows, pattern=ss.DENSE, bits=8, energy=self.le[2], ws=ws, stream=s,
+                            out=self.ldi)
+        elif name == "linear_ratio":
+            ss.predicted_ratio(self.le[0], self.le[1], out=self.lr[0], stream=s)
+            ss.predicted_ratio(self.le[0], self.le[2], out=self.lr[1], stream=s)
+        elif name == "weight_wanda_24_int4":
+            ss.run(xw, pattern=ss.SPARSE_24, fmt="int", bits=4, group=128, pack4=True, score="wanda",
+                   col_norms=self.norms, energy=self.we[0], ws=ws, stream=s, out=self.w24)
+        elif name == "weight_dense_int3":
+            ss.run(xw, pattern=ss.DENSE, fmt="int", bits=3, group=128, pack4=True, energy=self.we[1], ws=ws,
+                   stream=s, out=self.wd)
+        elif name == "weight_ratio":
+            ss.predicted_ratio(self.we[0], self.we[1], out=self.wr, stream=s)
+        elif name == "v_keys_24_fp8":
+            # V [head][key][d] pruned along the keys: axis 0 (a 3-D batch of 32 heads)
+            ss.run(self.x["v"], pattern=ss.SPARSE_24, fmt="fp8", energy=self.ve, ws=ws, stream=s, out=self.v24,
+                   axis=0)
+        else:
+            raise KeyError(name)
 
     def run_eager(self):
-        for p in self.passes:
+        for p in self.names:
             self.run_pass(p)
 
     def capture(self, rt):
-        """The whole step as one CUDA graph (the passes chained by
-        programmatic dependent launch), with an event-record node before each
-        pass and after the last one. Before each replay the nodes are pointed
-        at that step's own events, so every step's pass boundaries are timed
-        with CUDA events on the launching stream."""
+        """The whole step as one CUDA graph, with an event-record node before
+        each pass and after the last one; before each replay the nodes are
+        pointed at that step's own events."""
         torch = self.torch
         self.rt = rt
-        marks = [rt.event_create() for _ in range(len(self.passes) + 1)]
+        marks = [rt.event_create() for _ in range(len(self.names) + 1)]
         self.graph = torch.cuda.CUDAGraph(keep_graph=True)
         with torch.cuda.graph(self.graph, stream=self.stream):
-            for i, p in enumerate(self.passes):
+            for i, p in enumerate(self.names):
                 rt.record_external(marks[i], self.stream.cuda_stream)
                 self.run_pass(p)
             rt.record_external(marks[-1], self.stream.cuda_stream)
@@ -281,24 +380,15 @@ class Step:
         self.nodes = [nodes[m.value] for m in marks]
         self.graph.instantiate()
         self.exec = self.graph.raw_cuda_graph_exec()
-        # the same step without event nodes: every pass boundary stays a
-        # programmatic (overlapping) launch
-        self.plain = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(self.plain, stream=self.stream):
-            self.run_eager()
 
-    def replay(self, events=None):
-        """One step. With events (len(passes) + 1 fresh events) the evented
-        graph runs and records the pass boundaries; else the plain graph."""
-        if events is None:
-            self.plain.replay()
-            return
+    def replay(self, events):
         for node, ev in zip(self.nodes, events):
             self.rt.set_node_event(self.exec, node, ev)
         self.graph.replay()
 
 
 def memcpy_gbps(torch, dev, nbytes=1 << 30, iters=10):
+    """Device-to-device copy of nbytes (read + write bytes counted), best of iters."""
     a = torch.empty(nbytes // 2, dtype=torch.bfloat16, device=dev)
     b = torch.empty_like(a)
     b.copy_(a)
@@ -316,23 +406,32 @@ def memcpy_gbps(torch, dev, nbytes=1 << 30, iters=10):
     return 2 * nbytes / best / 1e9
 
 
-def cpu_baseline_sample(xs_host, rows=96):
-    """The oracle, as it stands, on a bounded sample: the first `rows` rows of
-    every operand of the batch through the same passes (each sample treated as
-    its own operand). Returns (GB/s of algorithmic bytes, seconds, cores)."""
+def oracle_fused_gbps(x_host, rows, threads):
+    """The oracle, as it stands, on the headline pass (2:4 + NVFP4 with the
+    tensor scale given, energies) over the first `rows` rows of the operand,
+    on `threads` host threads. Returns (GB/s of algorithmic bytes, seconds)."""
     import oracle
+    xs = np.ascontiguousarray(x_host[:rows])
+    scale = oracle.scale_of_amax(float(np.abs(_bf16_f32(xs)).max()), "nvfp4")
     t0 = time.perf_counter()
-    for x in xs_host:
-        xs = np.ascontiguousarray(x[:rows])
-        ts = oracle.tensor_scale(xs, "fp8")
-        sp = oracle.run(xs, pattern=oracle.SPARSE_24, fmt="fp8", tensor_scale=ts)["energy"]
-        d8 = oracle.run(xs, pattern=oracle.DENSE, fmt="fp8", tensor_scale=ts)["energy"]
-        di = oracle.run(xs, pattern=oracle.DENSE, fmt="int", bits=8, group=0)["energy"]
-        oracle.ratio(sp, d8)
-        oracle.ratio(sp, di)
+    if threads == 1:
+        oracle.run(xs, pattern=oracle.SPARSE_24, fmt="nvfp4", tensor_scale=scale)
+    else:
+        oracle.run_parallel(xs, pattern=oracle.SPARSE_24, fmt="nvfp4", tensor_scale=scale, threads=threads)
     dt = time.perf_counter() - t0
-    nbytes = sum(algorithmic_bytes(rows, K).values()) * len(xs_host)
-    return nbytes / dt / 1e9, dt, 1
+    n = rows * x_host.shape[1]
+    nbytes = 2 * n + n // 4 + n // 32 + n // 8
+    return nbytes / dt / 1e9, dt
+
+
+def _bf16_f32(a):
+    return (a.astype(np.uint32) << 16).view(np.float32)
+
+
+def stats_us(samples_s):
+    a = np.asarray(samples_s) * 1e6
+    return {"median": round(float(np.median(a)), 3), "p10": round(float(np.percentile(a, 10)), 3),
+            "p90": round(float(np.percentile(a, 90)), 3), "n": int(a.size)}
 
 
 def run_cuda(args):
@@ -344,6 +443,9 @@ def run_cuda(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        sys.exit(f"bench.py --gpus {args.gpus}: this process sees WORLD_SIZE={world}; launch {args.gpus} ranks with "
+                 f"python -m torch.distributed.run --nproc-per-node {args.gpus} bench.py --gpus {args.gpus}")
     if world > 1:
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
@@ -352,75 +454,141 @@ def run_cuda(args):
     ss.lib()
     stream = torch.cuda.Stream(device=dev)
 
-    # each rank draws its own batch (independent problems: weak scaling)
-    xs_host = make_batch(seed0=1 + 100 * rank)
-    x_pinned = torch.from_numpy(np.stack(xs_host).view(np.int16)).view(torch.bfloat16).pin_memory()
-    x_dev = torch.empty((BATCH, M, K), dtype=torch.bfloat16, device=dev)
-    with torch.cuda.stream(stream):
-        x_dev.copy_(x_pinned, non_blocking=True)
-    stream.synchronize()
-
-    step = Step(ss, x_dev, stream)
+    # each rank draws its own inputs (independent problems: weak scaling)
+    hx = host_inputs(seed_offset=100 * rank)
+    step = Step(ss, dev, stream, hx)
+    torch.cuda.synchronize()
     with torch.cuda.stream(stream):
         step.run_eager()          # first launches: kernel attributes, tensor-map entry point
     stream.synchronize()
+    if step.ws.error(stream) != 0:
+        raise RuntimeError("a kernel wait timed out")
     rt = Cudart()
     step.capture(rt)
-    with torch.cuda.stream(stream):       # graph replays launch on the current stream
-        for _ in range(args.warmup):
-            step.replay()
-        step.replay([rt.event_create() for _ in range(len(step.passes) + 1)])   # the evented graph too
-    stream.synchronize()
-    if step.ws.error(stream) != 0:
-        raise RuntimeError("a kernel wait timed out during warm-up")
-
-    # ---- timed region: K steps; every EVENT_EVERY-th step runs the evented
-    # graph (its pass boundaries timed by CUDA events), the others the plain one ----
-    n_ev = len(step.passes) + 1
-    timed = [i for i in range(args.steps) if i % EVENT_EVERY == 0]
-    evs = {i: [rt.event_create() for _ in range(n_ev)] for i in timed}
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(dev.index)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    with clocks, torch.cuda.stream(stream):
-        start.record(stream)
-        for i in range(args.steps):
-            step.replay(evs.get(i))
-        end.record(stream)
-        end.synchronize()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    elapsed_s = start.elapsed_time(end) / 1e3
-    per_pass = {p: 0.0 for p in step.passes}
-    for i in timed:
-        for j, p in enumerate(step.passes):
-            per_pass[p] += rt.elapsed_ms(evs[i][j], evs[i][j + 1]) / 1e3
-    if world > 1:
-        t = torch.tensor([elapsed_s], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_s = t.item()
-    err = step.ws.error(stream)
-    if err != 0:
-        raise RuntimeError(f"a kernel wait timed out (code {err})")
-
-    ab = algorithmic_bytes()
-    step_bytes = BATCH * sum(ab.values())
-    ms_per_step = elapsed_s / args.steps * 1e3
-    value = world * step_bytes * args.steps / elapsed_s / 1e9
-    elems = world * BATCH * M * K * args.steps / elapsed_s / 1e9
-
-    # ---- end to end through the public API with host buffers ----
-    e2e_steps = max(3, min(20, args.steps // 10))
-    r_host = torch.empty((2, BATCH, 4), dtype=torch.float64).pin_memory()
-    h2d = BATCH * M * K * 2
-    d2h = r_host.numel() * 8
+    n_ev = len(step.names) + 1
+    warm = [rt.event_create() for _ in range(n_ev)]
     with torch.cuda.stream(stream):
-        x_dev.copy_(x_pinned, non_blocking=True)     # warm-up of the copy path
-        step.replay()
-        r_host.copy_(step.r, non_blocking=True)
+        for _ in range(max(args.warmup, 3)):
+            step.replay(warm)
+    stream.synchronize()
+
+    def timed_region(nsteps, clocks):
+        evs = [[rt.event_create() for _ in range(n_ev)] for _ in range(nsteps)]
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        with clocks, torch.cuda.stream(stream):
+            start.record(stream)
+            for i in range(nsteps):
+                step.replay(evs[i])
+            end.record(stream)
+            end.synchronize()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        per = {p: [rt.elapsed_ms(evs[i][j], evs[i][j + 1]) / 1e3 for i in range(nsteps)]
+               for j, p in enumerate(step.names)}
+        return start.elapsed_time(end) / 1e3, per
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return t.item()
+
+    # ---- the contract's timed region: exactly --steps steps ----
+    clocks = ClockSampler(dev.index)
+    elapsed_s, per = timed_region(args.steps, clocks)
+    elapsed_s = max_over_ranks(elapsed_s)
+    head_s = max_over_ranks(float(np.sum(per[HEADLINE])))
+    if step.ws.error(stream) != 0:
+        raise RuntimeError("a kernel wait timed out")
+    # ---- sustained region when the contract's region is under a second ----
+    sustained = None
+    if elapsed_s < SUSTAIN_S and not args.no_sustain:
+        n2 = int(np.ceil(SUSTAIN_S / (elapsed_s / args.steps)))
+        clocks2 = ClockSampler(dev.index)
+        el2, per2 = timed_region(n2, clocks2)
+        el2 = max_over_ranks(el2)
+        sustained = {"steps": n2, "seconds": round(el2, 3), "clocks": clocks2.summary(), "per": per2}
+
+    ab = pass_bytes()
+    head_bytes = ab[HEADLINE]
+    value = world * head_bytes * args.steps / head_s / 1e9
+    step_bytes = sum(ab.values())
+    ms_per_step = elapsed_s / args.steps * 1e3
+    peak, peak_kind = load_peaks()
+    mc = memcpy_gbps(torch, dev)
+
+    def pass_table(per_pass):
+        out = {}
+        for p in step.names:
+            st = stats_us(per_pass[p])
+            out[p] = {"us": st, "bytes_per_launch": ab[p],
+                      "gbps_median": round(ab[p] / (st["median"] * 1e-6) / 1e9, 1) if ab[p] else None}
+        return out
+
+    passes = pass_table(per)
+    head_us = float(np.mean(per[HEADLINE])) * 1e6
+    achieved = head_bytes / (head_us * 1e-6) / 1e9
+    # "+amax": the same pass when it derives its tensor scale (an amax read first)
+    plus_amax_s = float(np.sum(per["sweep_scale"]) + np.sum(per[HEADLINE]))
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "headline_pass": HEADLINE, "m": SWEEP_M, "k": SWEEP_K,
+                   "input_dtype": "bf16", "tensor_scale": "given (computed by the step's amax pass)",
+                   "l2": "inputs larger than L2 (headline operand 448 MiB; linear batch 256 MiB); every pass reads "
+                         "its operand from HBM",
+                   "parallelism": f"dp{world} (independent operands per rank)"},
+        "headline": {"pass": HEADLINE, "gbps_mean": round(achieved, 1),
+                     "us": stats_us(per[HEADLINE]), "gelem_per_s": round(SWEEP_M * SWEEP_K / head_us / 1e3, 2),
+                     "frac_of_peak": round(achieved / peak, 4), "frac_of_memcpy": round(achieved / mc, 4),
+                     "plus_amax_gbps": round(head_bytes * args.steps / plus_amax_s / 1e9, 1)},
+        "step_gbps": round(world * step_bytes * args.steps / elapsed_s / 1e9, 1),
+        "memcpy_gbps": round(mc, 1),
+        "roofline": {"bound": "hbm", "kernel": HEADLINE, "achieved": round(achieved, 1), "peak": peak,
+                     "peak_source": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": measured_traffic(HEADLINE), "algorithmic_bytes_per_launch": head_bytes},
+        "passes": passes,
+        "gpu_launches": step.launches_per_step * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if sustained is not None:
+        ps = pass_table(sustained.pop("per"))
+        result["sustained"] = dict(sustained, headline_us=ps[HEADLINE]["us"],
+                                   headline_gbps_median=ps[HEADLINE]["gbps_median"],
+                                   passes={p: ps[p]["us"]["median"] for p in step.names})
+
+    sr = step.sr.cpu().numpy()
+    lr = step.lr.cpu().numpy()
+    result["predicted_r"] = {"sweep_24_nvfp4_vs_dense_nvfp4": round(float(sr[0, 3]), 4),
+                             "sweep_48_nvfp4_vs_dense_nvfp4": round(float(sr[1, 3]), 4),
+                             "linear_24_fp8_vs_dense_fp8": round(float(lr[0, 0, 3]), 4),
+                             "linear_24_fp8_vs_dense_int8_row": round(float(lr[1, 0, 3]), 4),
+                             "weight_wanda_24_int4_vs_dense_int3": round(float(step.wr[3].item()), 4),
+                             "energy_loss_24_sweep": round(float(sr[0, 0]), 5)}
+
+    # ---- end to end through the public API with host buffers: the headline
+    # operand copied in from pinned memory, the user's call (tensor scale derived
+    # by the library: an amax read, then the fused pass), energies read back ----
+    e2e_steps = max(3, min(10, args.steps // 2))
+    xin = step.h["sweep"]
+    e_host = torch.empty(4, dtype=torch.float64).pin_memory()
+    s_host = torch.empty(1, dtype=torch.float32).pin_memory()
+    xs = step.x["sweep"]
+
+    def e2e_once():
+        xs.copy_(xin, non_blocking=True)
+        ss.run(xs, pattern=ss.SPARSE_24, fmt="nvfp4", energy=step.se[0], ws=step.ws, stream=stream, out=step.s24)
+        e_host.copy_(step.se[0], non_blocking=True)
+        s_host.copy_(step.s24["tensor_scale"], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        e2e_once()
     stream.synchronize()
     if world > 1:
         dist.barrier()
@@ -428,62 +596,28 @@ def run_cuda(args):
     with torch.cuda.stream(stream):
         e0.record(stream)
         for _ in range(e2e_steps):
-            x_dev.copy_(x_pinned, non_blocking=True)
-            step.replay()
-            r_host.copy_(step.r, non_blocking=True)
+            e2e_once()
         e1.record(stream)
     e1.synchronize()
-    e2e_s = e0.elapsed_time(e1) / 1e3
-    if world > 1:
-        t = torch.tensor([e2e_s], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_s = t.item()
-    e2e_value = world * step_bytes * e2e_steps / e2e_s / 1e9
+    e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3)
+    result["e2e"] = {"value": round(world * head_bytes * e2e_steps / e2e_s / 1e9, 1), "unit": "GB/s",
+                     "h2d_bytes_per_step": int(xin.numel() * 2), "d2h_bytes_per_step": 8 * 4 + 4,
+                     "steps": e2e_steps, "call": "ss24.run -> ss24_prune24_quant_fused (tensor scale derived)"}
+    if step.ws.error(stream) != 0:
+        raise RuntimeError("a kernel wait timed out")
 
-    peak, peak_kind = load_peaks()
-    mc = memcpy_gbps(torch, dev)
-
-    # dominant kernel: the pass with the largest device time
-    dom = max((p for p in step.passes if ab[p] > 0), key=lambda p: per_pass[p])
-    # one launch per pass covers the whole batch (the ratio pass is two tiny launches)
-    dom_us = per_pass[dom] / len(timed) * 1e6
-    achieved = BATCH * ab[dom] / (dom_us * 1e-6) / 1e9
-    passes = {}
-    for p in step.passes:
-        us = per_pass[p] / len(timed) * 1e6
-        passes[p] = {"us_per_step": round(us, 3),
-                     "gbps": round(BATCH * ab[p] / (us * 1e-6) / 1e9, 1) if ab[p] else None,
-                     "bytes_per_launch": BATCH * ab[p]}
-    traffic = measured_traffic(dom)
-
-    r = step.r.cpu().numpy()
-    result = {
-        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "operands_per_step": BATCH, "m": M, "k": K, "input_dtype": "bf16",
-                   "l2": "inputs larger than L2: 8 x 32 MiB per step; each pass is one launch over all 8 "
-                         "operands before the next pass", "parallelism": f"dp{world} (independent batches)"},
-        "gelem_per_s": round(elems, 2),
-        "frac_of_peak": round(value / world / peak, 4),
-        "memcpy_gbps": round(mc, 1),
-        "frac_of_memcpy": round(value / world / mc, 4),
-        "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peak,
-                     "peak_source": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
-                     "traffic": traffic, "algorithmic_bytes_per_launch": BATCH * ab[dom]},
-        "passes": passes,
-        "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
-        "gpu_launches": step.launches_per_step * args.steps,
-        "clocks": clocks.summary(),
-        "predicted_r": {"vs_dense_fp8": round(float(r[0, 0, 3]), 4), "vs_dense_int8_row": round(float(r[1, 0, 3]), 4),
-                        "energy_loss_24": round(float(r[0, 0, 0]), 5)},
-    }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        gbps, dt, cores = cpu_baseline_sample(xs_host, rows=args.cpu_rows)
-        result["cpu_baseline"] = {"value": round(gbps, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-                                  "sample": f"first {args.cpu_rows} rows of each of the 8 operands, all passes "
-                                            f"({dt:.1f} s of CPU work)"}
+        import oracle
+        threads = oracle.host_threads()
+        g1, t1 = oracle_fused_gbps(hx["sweep"], args.cpu_rows_1, 1)
+        gn, tn = oracle_fused_gbps(hx["sweep"], SWEEP_M, threads)
+        result["cpu_baseline"] = {
+            "value": round(gn, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"the headline pass (2:4 + NVFP4, scale given, energies) over the whole {SWEEP_M}x{SWEEP_K} "
+                      f"operand on {threads} host threads (row blocks): {tn:.1f} s",
+            "host_cpus": os.cpu_count(),
+            "single_core": {"value": round(g1, 4), "unit": "GB/s", "cores": 1,
+                            "sample": f"first {args.cpu_rows_1} rows, one thread: {t1:.1f} s"}}
     if world > 1:
         del step
         dist.barrier()
@@ -493,28 +627,34 @@ def run_cuda(args):
 
 
 def run_reference(args):
-    """The oracle on the host cores, per step a bounded sample of the workload."""
+    """The oracle on the host cores, per step a bounded sample of the headline
+    workload (the first --ref-rows rows of the operand through the headline pass)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    xs_host = make_batch()
+    import oracle
+    from semi_structured_sparsity_online_b200 import synth
+    x = synth.sweep_operand(SWEEP_M, SWEEP_K, seed=8)
     rows = args.ref_rows
+    threads = oracle.host_threads()
     for _ in range(args.warmup):
-        cpu_baseline_sample(xs_host[:1], rows=rows)
-    t0 = time.perf_counter()
+        oracle_fused_gbps(x, rows, threads)
+    t = 0.0
     for _ in range(args.steps):
-        cpu_baseline_sample(xs_host[:1], rows=rows)
-    dt = time.perf_counter() - t0
-    nbytes = sum(algorithmic_bytes(rows, K).values()) * args.steps
-    value = nbytes / dt / 1e9
-    sample = f"per step: first {rows} rows of one 4096x4096 operand through all passes"
+        t += oracle_fused_gbps(x, rows, threads)[1]
+    n = rows * SWEEP_K
+    nbytes = (2 * n + n // 4 + n // 32 + n // 8) * args.steps
+    value = nbytes / t / 1e9
+    sample = (f"per step: the first {rows} rows of the {SWEEP_M}x{SWEEP_K} operand through the headline pass "
+              f"(2:4 + NVFP4, scale given, energies) on {threads} host threads")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "sample": sample},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "config": {"workload": WORKLOAD, "headline_pass": HEADLINE, "sample": sample},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }))
 
@@ -522,13 +662,16 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ss24", "reference"], default="ss24")
-    ap.add_argument("--cpu-rows", type=int, default=4096)
-    ap.add_argument("--ref-rows", type=int, default=8, help="rows of one operand per reference step")
+    ap.add_argument("--cpu-rows-1", type=int, default=1024, help="rows of the single-thread CPU baseline")
+    ap.add_argument("--ref-rows", type=int, default=1024, help="rows of the operand per reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sustain", action="store_true", help="skip the sustained region")
     args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
     if args.impl == "reference":
         run_reference(args)
     else:

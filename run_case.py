@@ -3,7 +3,7 @@
 A small, self-contained driver for profiling a single kernel (for example under
 Nsight Compute) or for a quick timing of one configuration:
 
-    python -m semi_structured_sparsity_online_b200.run_case --pass fused_24_fp8 --m 4096 --k 4096 --iters 3
+    python run_case.py --pass fused_24_fp8 --m 4096 --k 4096 --iters 3
 
 With --batch B the pass runs as one batched launch over B operands of that
 shape (a [B, m, k] tensor).
@@ -17,11 +17,17 @@ time per launch and the GB/s of the pass's algorithmic bytes.
 from __future__ import annotations
 
 import argparse
+import os
+import sys
 
 import numpy as np
 import torch
 
-from semi_structured_sparsity_online_b200 import ss24, synth
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from semi_structured_sparsity_online_b200 import ss24, synth  # noqa: E402
 
 # (pattern, format, bits, group): the stored format of each pass
 PASSES = {

@@ -284,18 +284,15 @@ def test_algorithmic_bytes_match_the_stored_layouts():
     """The bytes the benchmark and run_case count per launch, from the layouts:
     input 2 bytes per bf16 element; FP8 codes 1 byte per stored value; metadata
     1/8 byte per element (2:4) or 1/16 (4:8); E4M3 block scales 1 byte per 16
-    stored values, E8M0 per 32; INT scales 4 bytes per group or row."""
+    stored values, E8M0 per 32; INT scales 4 bytes per group or row; packed
+    INT4 / INT3 codes half a byte per stored value."""
     import bench
-    from semi_structured_sparsity_online_b200 import run_case
+    import run_case
     m = k = 4096
     n = m * k
-    ab = bench.algorithmic_bytes(m, k)
-    assert ab["fused_24_fp8"] == 2 * n + n // 2 + n // 8 == 44_040_192
-    assert ab["dense_fp8"] == 3 * n == 50_331_648
-    assert ab["tensor_scale"] == 2 * n + 4 * m
-    assert ab["dense_int8_row"] == 2 * n + 4 * m + n + 4 * m
     pb = run_case.pass_bytes
-    assert pb("fused_24_fp8", m, k) == ab["fused_24_fp8"]
+    assert pb("fused_24_fp8", m, k) == 2 * n + n // 2 + n // 8 == 44_040_192
+    assert pb("dense_fp8", m, k) == 3 * n == 50_331_648
     assert pb("fused_24_none", m, k) == 2 * n + n + n // 8 == 52_428_800
     assert pb("fused_24_nvfp4", m, k) == 2 * n + n // 4 + n // 32 + n // 8 == 40_370_176
     assert pb("fused_24_mxfp4", m, k) == 2 * n + n // 4 + n // 64 + n // 8 == 40_108_032
@@ -303,4 +300,17 @@ def test_algorithmic_bytes_match_the_stored_layouts():
     assert pb("fused_24_int8g128", m, k) == 2 * n + n // 2 + 4 * (n // 2 // 128) + n // 8 == 44_302_336
     assert pb("dense_nvfp4", m, k) == 2 * n + n // 2 + n // 16 == 42_991_616
     assert pb("hadamard128", m, k) == 6 * n
-    assert pb("softmax_24_fp8", m, k) == ab["fused_24_fp8"]
+    assert pb("softmax_24_fp8", m, k) == pb("fused_24_fp8", m, k)
+    ab = bench.pass_bytes()
+    ns = bench.SWEEP_M * bench.SWEEP_K
+    assert ab["sweep_fused_24_nvfp4"] == pb("fused_24_nvfp4", bench.SWEEP_M, bench.SWEEP_K) == 565_182_464
+    assert ab["sweep_fused_48_nvfp4"] == pb("fused_48_nvfp4", bench.SWEEP_M, bench.SWEEP_K)
+    assert ab["sweep_compress_24"] == pb("fused_24_none", bench.SWEEP_M, bench.SWEEP_K)
+    assert ab["sweep_dense_nvfp4"] == pb("dense_nvfp4", bench.SWEEP_M, bench.SWEEP_K)
+    assert ab["sweep_scale"] == 2 * ns
+    assert ab["linear_fused_24_fp8"] == 8 * pb("fused_24_fp8", m, k)
+    assert ab["linear_dense_fp8"] == 8 * pb("dense_fp8", m, k)
+    assert ab["linear_dense_int8_row"] == 8 * (2 * n + 4 * m + n + 4 * m)
+    nw = bench.W_M * bench.W_K
+    assert ab["weight_wanda_24_int4"] == 2 * nw + 4 * bench.W_K + nw // 4 + 4 * (nw // 256) + nw // 8
+    assert ab["weight_dense_int3"] == 2 * nw + nw // 2 + 4 * (nw // 128)
