@@ -108,7 +108,15 @@
  * stream) and returns SS24_OK, or SS24_ERR_CUDA if a launch failed. Results
  * are valid once the stream is synchronized. Kernels never trap: an internal
  * wait that exceeds about two seconds records a nonzero code in the
- * workspace (read with ss24_workspace_error) and the kernel returns.
+ * workspace (read with ss24_workspace_error) and the kernel returns; its
+ * outputs and energies are then incomplete. The only kernels with such waits
+ * are those of the strided axis (axis 0), which wait on their tile copies.
+ *
+ * Test hook. When the environment variable SS24_TEST_SKIP_TILE holds a
+ * number t >= 0 at the time of a call, the first CTA of that call's
+ * strided-axis kernel does not copy its t-th tile and every wait of the
+ * kernel gives up after 10 ms instead of two seconds: a wait runs out on
+ * purpose, and the error word shows it. For tests of that path only.
  */
 #ifndef SS24_H
 #define SS24_H

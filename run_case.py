@@ -37,6 +37,9 @@ PASSES = {
     "fused_24_mxfp4": (ss24.SPARSE_24, "mxfp4", 4, 0),
     "fused_24_int8g128": (ss24.SPARSE_24, "int", 8, 128),
     "fused_48_nvfp4": (ss24.SPARSE_48, "nvfp4", 4, 0),
+    "fused_48_fp8": (ss24.SPARSE_48, "fp8", 8, 0),
+    "fused_24_int4g128": (ss24.SPARSE_24, "int", 4, 128),
+    "dense_int3g128": (ss24.DENSE, "int", 3, 128),
     "dense_fp8": (ss24.DENSE, "fp8", 8, 0),
     "dense_nvfp4": (ss24.DENSE, "nvfp4", 4, 0),
     "dense_mxfp4": (ss24.DENSE, "mxfp4", 4, 0),
@@ -66,7 +69,9 @@ def pass_bytes(name, m, k):
     elif fmt == "fp8":
         vals, scales = q, 0
     elif fmt == "int":
-        vals, scales = q * (2 if bits > 8 else 1), 4 * (m if group == 0 else q // group)
+        # int8 / int16 containers; INT4 and narrower packed two codes per byte
+        vals = q // 2 if bits <= 4 else q * (2 if bits > 8 else 1)
+        scales = 4 * (m if group == 0 else q // group)
     elif fmt == "nvfp4":
         vals, scales = q // 2, q // 16
     else:
@@ -87,6 +92,8 @@ def main():
                     help="passes in PASSES: rotate the operand along k in the pass (block size)")
     ap.add_argument("--dequant", action="store_true",
                     help="time the reconstruction of the pass's outputs (ss24_dequantize) instead of the pass")
+    ap.add_argument("--score", default="mag", choices=["mag", "wanda"],
+                    help="passes in PASSES: the selection score (wanda: column norms exp(N(0,1)))")
     ap.add_argument("--derive-scale", action="store_true",
                     help="FP8 / NVFP4: let the pass compute its tensor scale (an amax launch precedes it)")
     args = ap.parse_args()
@@ -102,10 +109,13 @@ def main():
         e = e[0]
     scale = ss24.tensor_scale(x, "fp8", ss24.SPARSE_24, ws=ws, hadamard=args.hadamard)
     out = None
+    norms = None
+    if args.score == "wanda":
+        norms = torch.from_numpy(np.exp(np.random.default_rng(3).standard_normal(args.k)).astype(np.float32)).cuda()
     if args.name in PASSES:
         pattern, fmt, bits, group = PASSES[args.name]
-        out = ss24._alloc_outputs(args.m, args.k, pattern, ss24.make_format(fmt, bits, group), torch.bfloat16, "cuda",
-                                  lead)
+        out = ss24._alloc_outputs(args.m, args.k, pattern, ss24.make_format(fmt, bits, group, fmt == "int" and bits <= 4),
+                                  torch.bfloat16, "cuda", lead)
         if fmt == "nvfp4":
             scale = ss24.tensor_scale(x, "nvfp4", pattern if pattern != ss24.DENSE else ss24.DENSE, ws=ws,
                                       hadamard=args.hadamard)
@@ -140,8 +150,9 @@ def main():
         else:
             pattern, fmt, bits, group = PASSES[args.name]
             ts = scale if fmt in ("fp8", "nvfp4") and not args.derive_scale else None
-            ss24.run(x, pattern=pattern, fmt=fmt, bits=bits, group=group, tensor_scale=ts, energy=e, ws=ws, out=out,
-                     hadamard=args.hadamard)
+            ss24.run(x, pattern=pattern, fmt=fmt, bits=bits, group=group, pack4=fmt == "int" and bits <= 4,
+                     tensor_scale=ts, energy=e, ws=ws, out=out, hadamard=args.hadamard, score=args.score,
+                     col_norms=norms)
 
     once()
     torch.cuda.synchronize()

@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <unordered_map>
@@ -15,6 +16,7 @@ namespace ss24 {
 const void *stream_kernel_bf16(int pattern, int score, int fmt, bool fw);
 const void *stream_kernel_f32(int pattern, int score, int fmt, bool fw);
 const void *stream_kernel_bf16_rot(int pattern, int fmt, bool fw);
+const void *stream_lb_kernel_bf16(int pattern, int score, int fmt);
 const void *rowsweep_kernel_bf16(int pattern, int score);
 const void *rowsweep_kernel_f32(int pattern, int score);
 const void *rowblock_kernel_bf16(int pattern, int score, int cpt);
@@ -32,6 +34,7 @@ namespace {
 // ---------------------------------------------------------------------------
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned32(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 bool pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
 int64_t next_pow2(int64_t v)
 {
@@ -482,6 +485,16 @@ PassParams base_params(const ss24_operand *x, const Geometry &g, void *ws, ss24_
     p.amax_partials = reinterpret_cast<float *>(w + kWsAmaxOff);
     p.amax_out = reinterpret_cast<float *>(w + kWsAmaxReducedOff);
     p.energy_out = reinterpret_cast<double *>(energy);
+    p.wait_limit_ns = kWaitLimitNs;
+    p.test_skip_tile = -1;
+    if (const char *t = std::getenv("SS24_TEST_SKIP_TILE")) {
+        // test hook (ss24.h): one tile copy skipped, waits limited to 10 ms
+        const long v = std::strtol(t, nullptr, 10);
+        if (v >= 0 && v < INT32_MAX) {
+            p.test_skip_tile = static_cast<int32_t>(v);
+            p.wait_limit_ns = kTestWaitLimitNs;
+        }
+    }
     p.batch = static_cast<int32_t>(nbatch(x));
     p.x_bstride = bstride_elems(x);
     if (x->hadamard != 0) {
@@ -544,10 +557,17 @@ bool plan_tile(const ss24_operand *x, int pattern, int score, int mode, TilePlan
         t->g = stream_geometry(x);
         // full width: W = 256 with four segments per unit
         const bool fw = t->g.W == 256 && t->g.step_cols == 256;
-        if (x->hadamard != 0)
+        if (x->hadamard != 0) {
             t->kernel = score == SS24_SCORE_MAG ? stream_kernel_bf16_rot(pattern, mode, fw) : nullptr;
-        else
-            t->kernel = stream_kernel(x->dtype, pattern, score, mode, fw);
+        } else {
+            // bf16 with rows a multiple of 64: one lane per 32 consecutive
+            // elements (where that kernel has the format)
+            t->kernel = nullptr;
+            if (fw && x->dtype == SS24_BF16 && x->k % 64 == 0)
+                t->kernel = stream_lb_kernel_bf16(pattern, score, mode);
+            if (!t->kernel)
+                t->kernel = stream_kernel(x->dtype, pattern, score, mode, fw);
+        }
         t->smem = 0;
         return t->kernel != nullptr;
     }
@@ -656,6 +676,15 @@ ss24_status run_pass(const ss24_operand *x, int pattern, int score, const float 
     // ---- launches ----
     PassParams p = base_params(x, g, ws, energy);
     output_strides(x, pattern, fmt, &p);
+    {
+        // lane-block kernel: 32-byte loads measured faster for pairwise 4:8
+        // only; 32-byte stores wherever the values are aligned for them
+        const int64_t es = static_cast<int64_t>(esize(x->dtype));
+        const bool in32 = aligned32(x->x) && (x->ld * es) % 32 == 0 &&
+                          (nbatch(x) == 1 || (x->batch_stride * es) % 32 == 0);
+        const bool out32 = aligned32(out->values) && p.values_bstride % 32 == 0;
+        p.lb_wide = (in32 && pattern == SS24_SPARSE_48 ? 1 : 0) | (out32 ? 2 : 0);
+    }
     p.values = out->values;
     p.scales = out->scales;
     p.meta = out->meta;

@@ -65,13 +65,10 @@ __device__ __forceinline__ uint64_t global_timer_ns()
     return t;
 }
 
-// A wait gives up after this long; the kernel then records an error code and
-// returns instead of spinning forever.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
-
 // Waits until the barrier phase with the given parity has completed.
-// Returns false (without having waited forever) if that takes over ~2 s.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
+// Returns false (without having waited forever) if that takes longer than
+// limit_ns; the kernel then records an error code and returns.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns)
 {
     if (mbar_try_wait(bar, parity))
         return true;
@@ -80,7 +77,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
         for (int i = 0; i < 32; ++i)
             if (mbar_try_wait(bar, parity))
                 return true;
-        if (global_timer_ns() - t0 > kWaitLimitNs)
+        if (global_timer_ns() - t0 > limit_ns)
             return false;
     }
 }

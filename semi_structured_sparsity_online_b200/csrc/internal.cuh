@@ -19,6 +19,12 @@ constexpr int kRotated = 2;
 enum Fmt { kNone = 0, kFp8 = 1, kInt = 2, kNvfp4 = 3, kMxfp4 = 4, kAmax = 5, kEnergy = 6, kIntRows = 7 };
 enum IntStore { kInt8 = 0, kInt16 = 1, kPack4 = 2 };
 
+// How long a kernel's wait on a barrier may take before the kernel gives up,
+// records an error code in the workspace and returns (instead of spinning
+// forever); and the shorter limit of the test hook (see ss24.h).
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr uint64_t kTestWaitLimitNs = 10000000ull;
+
 // Consumer warps per CTA and the TMA stage ring (each stage 16 KiB).
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumers = kConsumerWarps * 32;
@@ -120,6 +126,15 @@ struct PassParams {
     // rotated kernels: log2 of the Hadamard block and RN(1/sqrt(block))
     int32_t rot_log2b;
     float rot_scale;
+    // the time limit of every barrier wait (ns); and a test hook: with
+    // test_skip_tile = t >= 0 the first CTA of operand 0 of the strided-axis
+    // kernel does not copy its t-th tile, so that its consumers' wait runs out
+    uint64_t wait_limit_ns;
+    int32_t test_skip_tile;
+    // lane-block kernel: bit 0, a lane's 64 input bytes are read with two
+    // 32-byte loads (the operand's rows 32-byte aligned); bit 1, its 32-byte
+    // runs of output are written with one store (the values 32-byte aligned)
+    int32_t lb_wide;
 };
 
 cudaError_t launch_ratio(const double *sparse_side, const double *dense_side, double *out, int64_t count,

@@ -1057,7 +1057,14 @@ __device__ __forceinline__ void producer(const CUtensorMap *map, const PassParam
     for (int64_t t = p.cta; t < p.n_tiles; t += p.ctas_per_op, ++it) {
         const int s = it % kStages;
         const uint32_t use = it / kStages;
-        if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1)) {
+        if (p.test_skip_tile >= 0 && p.op == 0 && p.cta == 0 && it == static_cast<uint32_t>(p.test_skip_tile)) {
+            // test hook: this tile is never copied, so its consumers' wait runs
+            // out; nothing more is issued, and the copies already issued are
+            // drained below
+            failed = true;
+            break;
+        }
+        if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1, p.wait_limit_ns)) {
             record_error(p.err, 1);
             failed = true;
             break;
@@ -1075,7 +1082,7 @@ __device__ __forceinline__ void producer(const CUtensorMap *map, const PassParam
         // let the copies already issued land before the CTA can exit
         for (int s = 0; s < kStages && s < static_cast<int>(it); ++s) {
             const uint32_t last_use = (it - 1 - ((it - 1 - s) % kStages)) / kStages;
-            (void)mbar_wait(&full[s], last_use & 1);
+            (void)mbar_wait(&full[s], last_use & 1, p.wait_limit_ns);
         }
     }
 }
@@ -1183,6 +1190,31 @@ __device__ __forceinline__ uint4 ld_stream(const void *p, bool ok)
                  : "+r"(r.x), "+r"(r.y), "+r"(r.z), "+r"(r.w)
                  : "l"(p), "r"(static_cast<int>(ok)));
     return r;
+}
+
+// 32-byte global load (two 16-byte halves) that bypasses L1, predicated like
+// ld_stream; p must be 32-byte aligned. A warp's 32 loads then cover whole
+// 32-byte sectors, where 16-byte loads 32 or 64 bytes apart would fetch each
+// sector twice.
+__device__ __forceinline__ void ld_stream32(const void *p, bool ok, uint4 &a, uint4 &b)
+{
+    a = make_uint4(0u, 0u, 0u, 0u);
+    b = a;
+    asm volatile("{\n"
+                 " .reg .pred q;\n"
+                 " setp.ne.b32 q, %9, 0;\n"
+                 " @q ld.global.nc.L1::no_allocate.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n"
+                 "}\n"
+                 : "+r"(a.x), "+r"(a.y), "+r"(a.z), "+r"(a.w), "+r"(b.x), "+r"(b.y), "+r"(b.z), "+r"(b.w)
+                 : "l"(p), "r"(static_cast<int>(ok)));
+}
+
+// 32-byte global store; p must be 32-byte aligned.
+__device__ __forceinline__ void st32(void *p, const uint4 &a, const uint4 &b)
+{
+    asm volatile("st.global.v8.u32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a.x), "r"(a.y), "r"(a.z),
+                 "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+                 : "memory");
 }
 
 template <typename T> struct Stream;
@@ -2085,7 +2117,7 @@ __global__ void __launch_bounds__(kThreads, 1) axis0_kernel(const __grid_constan
         // one thread waits for the stage and tells the others, so that every
         // consumer leaves the loop together if the wait gives up
         if (tid == 0) {
-            const bool ok = mbar_wait(&full[s], (it / kStages) & 1);
+            const bool ok = mbar_wait(&full[s], (it / kStages) & 1, p.wait_limit_ns);
             if (!ok)
                 record_error(p.err, 5);
             *ready = ok;

@@ -191,6 +191,20 @@ def test_dense_pass_full_width(ss, ws, fmt, bits, group, pack4, k):
     compare(ss, ws, xh, pattern=0, fmt=fmt, bits=bits, group=group, pack4=pack4)
 
 
+@pytest.mark.parametrize("pattern", [0, 24, 48])
+@pytest.mark.parametrize("fmt,bits,group,pack4", [("none", 8, 0, False), ("fp8", 8, 0, False), ("nvfp4", 4, 0, False),
+                                                  ("int", 3, 16, False), ("mxfp4", 4, 0, False)])
+def test_full_width_rows_not_a_multiple_of_64(ss, ws, pattern, fmt, bits, group, pack4):
+    """bf16 by magnitude with k = 4128 (a multiple of 32, not of 64; a ragged
+    last unit of 32 columns): the full-width stream kernel with a chunk per
+    lane and segment, where k = 2048 / 4608 take one lane per 32 elements."""
+    k = 4128
+    if (pattern == 0 and fmt == "none") or (pattern and fmt == "mxfp4"):
+        pytest.skip("format not defined for this pattern / k")
+    xh = synth.sweep_operand(23, k, seed=12 + pattern)
+    compare(ss, ws, xh, pattern=pattern, fmt=fmt, bits=bits, group=group, pack4=pack4)
+
+
 @pytest.mark.parametrize("fmt,bits,group,pack4", FORMATS)
 def test_sparse_pass_fp32(ss, ws, fmt, bits, group, pack4):
     xh = synth.gaussian_f32(37, 1024, seed=0)
@@ -270,6 +284,40 @@ def test_strided_axis_limits_and_energy_pass(ss, ws):
 # --------------------------------------------------------------------------
 # batches: B same-shaped operands in one call, each exactly as alone
 # --------------------------------------------------------------------------
+
+def test_bounded_wait_runs_out_and_is_reported(ss, monkeypatch):
+    """A wait that runs out, made on purpose (the SS24_TEST_SKIP_TILE hook: the
+    first CTA of the strided-axis kernel skips its third tile copy, and waits
+    give up after 10 ms): the call returns, the kernel ends without hanging,
+    the workspace's error word is set; after ss24_workspace_init the same call
+    is exact against the oracle again."""
+    import time
+    xh = synth.sweep_operand(4096, 4096, seed=31)      # A[r][c] at xh[c][r]: k = 4096 positions x 4096 rows
+    ts = oracle.tensor_scale(xh, "fp8", pattern=oracle.SPARSE_24, axis=0)
+    sd = torch.tensor([ts], dtype=torch.float32, device="cuda")
+    x = to_dev(xh)
+    ws = ss.Workspace()
+    ss.run(x, pattern=24, fmt="fp8", tensor_scale=sd, ws=ws, axis=0)      # first call: module and attributes
+    torch.cuda.synchronize()
+    assert ws.error() == 0
+    monkeypatch.setenv("SS24_TEST_SKIP_TILE", "2")
+    t0 = time.perf_counter()
+    ss.run(x, pattern=24, fmt="fp8", tensor_scale=sd, ws=ws, axis=0)
+    code = ws.error()                                   # synchronizes the stream
+    elapsed = time.perf_counter() - t0
+    assert code != 0, "the skipped tile did not make a wait run out"
+    assert elapsed < 1.5, elapsed                       # the 10 ms limit, not two seconds
+    monkeypatch.delenv("SS24_TEST_SKIP_TILE")
+    assert ss.lib().ss24_workspace_init(ws.ptr, ws.nbytes, None) == 0
+    assert ws.error() == 0
+    out = ss.run(x, pattern=24, fmt="fp8", tensor_scale=sd, ws=ws, axis=0)
+    torch.cuda.synchronize()
+    ref = oracle.run(xh, pattern=oracle.SPARSE_24, fmt="fp8", tensor_scale=ts, axis=0)
+    for key in ("values", "meta"):
+        assert_same(to_np(out[key]), ref[key], key)
+    assert_energy(out["energy"], ref["energy"], atol=1e-30)
+    assert ws.error() == 0
+
 
 def compare_batch(ss, ws, xs, *, pattern, fmt, bits=8, group=0, pack4=False, axis=1, pad_rows=0, tensor_scale=None):
     """xs: host arrays of one shape; they are placed pad_rows apart (a strided
