@@ -508,6 +508,27 @@ ss24_status ss24_softmax_prune(const ss24_operand *s, float alpha, ss24_pattern 
  * multiple of 8 and of block), SS24_ERR_NULL, SS24_ERR_ALIGN. */
 ss24_status ss24_hadamard(const ss24_operand *x, int32_t block, float *out, ss24_stream stream);
 
+/* ---- the consumer: 2:4-sparse GEMM on the tensor cores ---------------------- */
+
+/* Y = s_a s_b A B^T on the 2:4-sparse FP8 MMA of the 5th-generation tensor
+ * cores (§1: an operand computed on the fly is pruned and compressed before
+ * every GEMM; §3: the sparse GEMM reads the kept values and their indices). A
+ * is the 2:4 operand as ss24_prune24_quant_fused writes it with FP8: a_values
+ * the E4M3 kept values u8 [m][k/2], a_meta the metadata u8 [m][k/8] (the
+ * pass's layout is the one the sparse MMA takes, read in 128-row x 16-byte
+ * tiles), a_scale its tensor scale (device fp32). B is a dense E4M3 operand u8
+ * [n][k] (k contiguous; e.g. a weight through ss24_quantize_fp8) with tensor
+ * scale b_scale (device fp32). y (device fp32 [m][n], row major) receives
+ * RN(acc * RN(s_a * s_b)), acc the binary32 accumulation of the products.
+ * Shapes: m and n multiples of 128, k a multiple of 256 (a zero m or n is an
+ * empty product: nothing is launched). Pointers 16-byte aligned. The workspace
+ * carries the error word of the kernel's bounded waits (ss24_workspace_error).
+ * Errors: SS24_ERR_SHAPE, SS24_ERR_NULL, SS24_ERR_ALIGN, SS24_ERR_WORKSPACE,
+ * SS24_ERR_CUDA. */
+ss24_status ss24_sparse_gemm_fp8(const uint8_t *a_values, const uint8_t *a_meta, const float *a_scale,
+                                 const uint8_t *b, const float *b_scale, int64_t m, int64_t n, int64_t k, float *y,
+                                 void *ws, size_t ws_bytes, ss24_stream stream);
+
 /* ---- consumer layouts ------------------------------------------------------ */
 
 /* Bytes of the block-scale tiles of a rows x cols scale matrix (one operand):

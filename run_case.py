@@ -94,11 +94,14 @@ def main():
                     help="time the reconstruction of the pass's outputs (ss24_dequantize) instead of the pass")
     ap.add_argument("--score", default="mag", choices=["mag", "wanda"],
                     help="passes in PASSES: the selection score (wanda: column norms exp(N(0,1)))")
+    ap.add_argument("--axis", type=int, default=1, choices=[0, 1],
+                    help="1: k contiguous; 0: the operand stored [k][m] (rows contiguous), pruned along k")
     ap.add_argument("--derive-scale", action="store_true",
                     help="FP8 / NVFP4: let the pass compute its tensor scale (an amax launch precedes it)")
     args = ap.parse_args()
     nb = max(args.batch, 1)
-    xb = np.stack([synth.sweep_operand(args.m, args.k, seed=args.seed + i) for i in range(nb)])
+    shape = (args.m, args.k) if args.axis == 1 else (args.k, args.m)
+    xb = np.stack([synth.sweep_operand(*shape, seed=args.seed + i) for i in range(nb)])
     x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).cuda()
     if args.batch == 0:
         x = x[0]
@@ -107,7 +110,7 @@ def main():
     e = torch.zeros((nb, 4), dtype=torch.float64, device="cuda")
     if args.batch == 0:
         e = e[0]
-    scale = ss24.tensor_scale(x, "fp8", ss24.SPARSE_24, ws=ws, hadamard=args.hadamard)
+    scale = ss24.tensor_scale(x, "fp8", ss24.SPARSE_24, ws=ws, hadamard=args.hadamard, axis=args.axis)
     out = None
     norms = None
     if args.score == "wanda":
@@ -118,7 +121,7 @@ def main():
                                   torch.bfloat16, "cuda", lead)
         if fmt == "nvfp4":
             scale = ss24.tensor_scale(x, "nvfp4", pattern if pattern != ss24.DENSE else ss24.DENSE, ws=ws,
-                                      hadamard=args.hadamard)
+                                      hadamard=args.hadamard, axis=args.axis)
 
     row_amax = ss24.amax_rows(x, ws=ws)[0] if args.name in ("amax_rows", "dense_int8_given_rows") else None
     if args.name == "dense_int8_given_rows":
@@ -146,13 +149,13 @@ def main():
             ss24.tensor_scale(x, "fp8", ss24.SPARSE_24, ws=ws, out=scale)
         elif args.name == "error_energy":
             ss24.error_energy(x, ss24.SPARSE_24, ("fp8",), ("int", 5, 128), sparse_scale=scale, dense_scale=None,
-                              ws=ws, energy=e)
+                              ws=ws, energy=e, axis=args.axis)
         else:
             pattern, fmt, bits, group = PASSES[args.name]
             ts = scale if fmt in ("fp8", "nvfp4") and not args.derive_scale else None
             ss24.run(x, pattern=pattern, fmt=fmt, bits=bits, group=group, pack4=fmt == "int" and bits <= 4,
                      tensor_scale=ts, energy=e, ws=ws, out=out, hadamard=args.hadamard, score=args.score,
-                     col_norms=norms)
+                     col_norms=norms, axis=args.axis)
 
     once()
     torch.cuda.synchronize()
@@ -177,7 +180,8 @@ def main():
     t.synchronize()
     us = s.elapsed_time(t) / args.iters * 1e3
     assert ws.error() == 0
-    tag = (" dequant" if args.dequant else "") + (f" hadamard {args.hadamard}" if args.hadamard else "")
+    tag = ((" dequant" if args.dequant else "") + (f" hadamard {args.hadamard}" if args.hadamard else "")
+           + (" axis 0" if args.axis == 0 else ""))
     print(f"{args.name}{tag} m={args.m} k={args.k} batch={args.batch}: {us:.2f} us/launch, {gb / us / 1e3:.1f} GB/s "
           f"({gb} algorithmic bytes per launch; warm L2 between launches)")
 

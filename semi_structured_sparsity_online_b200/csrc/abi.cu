@@ -1351,6 +1351,27 @@ ss24_status ss24_decode_e2m1(const uint8_t *in, float *out, int64_t n, ss24_stre
     return cuda_status(launch_convert(3, in, out, n, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+ss24_status ss24_sparse_gemm_fp8(const uint8_t *a_values, const uint8_t *a_meta, const float *a_scale,
+                                 const uint8_t *b, const float *b_scale, int64_t m, int64_t n, int64_t k, float *y,
+                                 void *ws, size_t ws_bytes, ss24_stream stream)
+{
+    if (m < 0 || n < 0 || k <= 0 || m % 128 != 0 || n % 128 != 0 || k % 256 != 0 || m > INT32_MAX ||
+        n > INT32_MAX || k > INT32_MAX)
+        return SS24_ERR_SHAPE;
+    ss24_status st = check_ws(ws, ws_bytes);
+    if (st != SS24_OK)
+        return st;
+    if (m == 0 || n == 0)
+        return SS24_OK;
+    if (!a_values || !a_meta || !a_scale || !b || !b_scale || !y)
+        return SS24_ERR_NULL;
+    if (!aligned16(a_values) || !aligned16(a_meta) || !aligned16(b) || !aligned16(y))
+        return SS24_ERR_ALIGN;
+    int32_t *err = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + kWsErrOff);
+    return cuda_status(launch_sparse_gemm_fp8(a_values, a_meta, a_scale, b, b_scale, m, n, k, y, err, kWaitLimitNs,
+                                              reinterpret_cast<cudaStream_t>(stream)));
+}
+
 ss24_status ss24_prune24_quant_fused_noalloc(const ss24_operand *x, ss24_score score, const float *col_norms,
                                              ss24_format fmt, const float *tensor_scale_in, ss24_outputs *out,
                                              ss24_energy *energy, ss24_stream stream)

@@ -155,5 +155,9 @@ cudaError_t launch_scale_tiles(const uint8_t *in, int64_t rows, int64_t cols, in
                                cudaStream_t stream);
 cudaError_t launch_selfcheck_encoder(int e2m1, const uint32_t *bounds, int n_bounds, uint32_t hi_first,
                                      uint32_t hi_count, unsigned long long *result, cudaStream_t stream);
+size_t sparse_gemm_smem_bytes();
+cudaError_t launch_sparse_gemm_fp8(const uint8_t *a_values, const uint8_t *a_meta, const float *a_scale,
+                                   const uint8_t *b, const float *b_scale, int64_t m, int64_t n, int64_t k, float *y,
+                                   int32_t *err, uint64_t wait_limit_ns, cudaStream_t stream);
 
 } // namespace ss24

@@ -95,6 +95,8 @@ _SIGNATURES = {
     "ss24_scale_tiles": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, _P, _P]),
     "ss24_selfcheck_encoder": (ctypes.c_int, [ctypes.c_int32, _P, ctypes.c_int32, ctypes.c_uint32, ctypes.c_uint32,
                                               _P, _P]),
+    "ss24_sparse_gemm_fp8": (ctypes.c_int, [_P, _P, _P, _P, _P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                            _P, _P, _S, _P]),
     "ss24_encode_e4m3": (ctypes.c_int, [_P, _P, ctypes.c_int64, _P]),
     "ss24_decode_e4m3": (ctypes.c_int, [_P, _P, ctypes.c_int64, _P]),
     "ss24_encode_e2m1": (ctypes.c_int, [_P, _P, ctypes.c_int64, _P]),
@@ -428,6 +430,21 @@ def predicted_ratio(sparse_energy, dense_energy, out=None, stream=None):
     _check(lib().ss24_predicted_ratio(_ptr(sparse_energy), _ptr(dense_energy), _ptr(r), count, _stream(stream)),
            "ss24_predicted_ratio")
     return r
+
+
+def sparse_gemm_fp8(a, b, y=None, ws=None, stream=None):
+    """Y = s_a s_b A B^T on the tensor cores' 2:4-sparse FP8 MMA
+    (ss24_sparse_gemm_fp8). a: the dict of a 2:4 + FP8 pass over [m, k]
+    (``values`` [m, k/2], ``meta`` [m, k/8], ``tensor_scale``); b: the dict of a
+    dense FP8 pass over [n, k] (``values`` [n, k], ``tensor_scale``). Returns
+    float32 [m, n] on the device."""
+    m, n, k = a["values"].shape[0], b["values"].shape[0], b["values"].shape[1]
+    y = y if y is not None else torch.empty((m, n), dtype=torch.float32, device=a["values"].device)
+    ws = ws or default_workspace(a["values"].device)
+    _check(lib().ss24_sparse_gemm_fp8(_ptr(a["values"]), _ptr(a["meta"]), _ptr(a["tensor_scale"]),
+                                      _ptr(b["values"]), _ptr(b["tensor_scale"]), m, n, k, _ptr(y), ws.ptr,
+                                      ws.nbytes, _stream(stream)), "ss24_sparse_gemm_fp8")
+    return y
 
 
 def bits_per_element(fmt="none", bits=8, group=0, pattern=SPARSE_24, k=4096, with_scales=False) -> float:
