@@ -61,6 +61,8 @@ def pass_bytes(name, m, k):
         return 2 * n + 4 * m
     if name == "dense_int8_given_rows":
         return 2 * n + 8 * m + n
+    if name == "sparse_gemm_fp8":
+        raise ValueError("the GEMM is counted in FLOPs (see main)")
     pattern, fmt, bits, group = PASSES[name]
     q = n // 2 if pattern != ss24.DENSE else n
     meta = n // 8 if pattern == ss24.SPARSE_24 else (n // 16 if pattern == ss24.SPARSE_48 else 0)
@@ -81,10 +83,12 @@ def pass_bytes(name, m, k):
 
 def main():
     ap = argparse.ArgumentParser()
-    extra = ["tensor_scale", "error_energy", "amax_rows", "hadamard128", "softmax_24_fp8", "dense_int8_given_rows"]
+    extra = ["tensor_scale", "error_energy", "amax_rows", "hadamard128", "softmax_24_fp8", "dense_int8_given_rows",
+             "sparse_gemm_fp8"]
     ap.add_argument("--pass", dest="name", default="fused_24_fp8", choices=sorted(PASSES) + extra)
     ap.add_argument("--m", type=int, default=4096)
     ap.add_argument("--k", type=int, default=4096)
+    ap.add_argument("--n", type=int, default=4096, help="sparse_gemm_fp8: columns of the product (rows of B)")
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--seed", type=int, default=8)
     ap.add_argument("--batch", type=int, default=0, help="0: one 2-D operand; B: one launch over B operands")
@@ -99,6 +103,8 @@ def main():
     ap.add_argument("--derive-scale", action="store_true",
                     help="FP8 / NVFP4: let the pass compute its tensor scale (an amax launch precedes it)")
     args = ap.parse_args()
+    if args.name == "sparse_gemm_fp8":
+        return gemm_case(args)
     nb = max(args.batch, 1)
     shape = (args.m, args.k) if args.axis == 1 else (args.k, args.m)
     xb = np.stack([synth.sweep_operand(*shape, seed=args.seed + i) for i in range(nb)])
@@ -184,6 +190,29 @@ def main():
            + (" axis 0" if args.axis == 0 else ""))
     print(f"{args.name}{tag} m={args.m} k={args.k} batch={args.batch}: {us:.2f} us/launch, {gb / us / 1e3:.1f} GB/s "
           f"({gb} algorithmic bytes per launch; warm L2 between launches)")
+
+
+def gemm_case(args):
+    """The consumer: A = 2:4 + FP8 of an [m, k] sweep operand, B = dense FP8 of
+    an [n, k] N(0, 0.02^2) operand, Y = A B^T on the sparse tensor cores."""
+    x = torch.from_numpy(synth.sweep_operand(args.m, args.k, seed=args.seed).view(np.int16)).view(torch.bfloat16)
+    w = torch.from_numpy(synth.gaussian_bf16(args.n, args.k, seed=args.seed + 1, std=0.02).view(np.int16))
+    ws = ss24.Workspace()
+    a = ss24.run(x.cuda(), pattern=ss24.SPARSE_24, fmt="fp8", ws=ws)
+    b = ss24.run(w.view(torch.bfloat16).cuda(), pattern=ss24.DENSE, fmt="fp8", ws=ws)
+    y = ss24.sparse_gemm_fp8(a, b, ws=ws)
+    torch.cuda.synchronize()
+    s, t = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(args.iters):
+        ss24.sparse_gemm_fp8(a, b, y=y, ws=ws)
+    t.record()
+    t.synchronize()
+    us = s.elapsed_time(t) / args.iters * 1e3
+    assert ws.error() == 0
+    flops = 2 * args.m * args.n * args.k
+    print(f"sparse_gemm_fp8 m={args.m} n={args.n} k={args.k}: {us:.2f} us/launch, {flops / us / 1e6:.1f} "
+          f"dense-equivalent TFLOP/s ({flops // 2} multiply-adds of kept values)")
 
 
 if __name__ == "__main__":
