@@ -433,8 +433,9 @@ ss24_status ss24_dequantize(const ss24_operand *x, ss24_pattern pattern, ss24_fo
  * kernels divide with the correction). mode 1: 2^23 pseudo-random pairs per
  * unit of b_count, exponents across the corrected range. mode 2 checks the
  * packed bf16 operations the 2:4 selection and the amax use (magnitude
- * comparison through a rounded bf16 difference, magnitude maximum, bf16 to
- * binary32 conversion and squares on the multiply-add unit) for the magnitude
+ * comparison through a rounded bf16 difference, magnitude maximum and its
+ * test against a limit, bf16 to binary32 conversion and squares on the
+ * multiply-add unit) for the magnitude
  * bits a = b_first + j, j < b_count (b_first + b_count <= 2^15), against every
  * magnitude b < 2^15, finite values only, both signs; a mismatch is reported as
  * (a << 32 | b). Adds the number of

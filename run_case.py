@@ -102,6 +102,9 @@ def main():
                     help="1: k contiguous; 0: the operand stored [k][m] (rows contiguous), pruned along k")
     ap.add_argument("--derive-scale", action="store_true",
                     help="FP8 / NVFP4: let the pass compute its tensor scale (an amax launch precedes it)")
+    ap.add_argument("--energy", default="fp8/int:5:128",
+                    help="error_energy: the 2:4 side's and the dense side's formats, e.g. nvfp4/int:3:64 or nvfp4/int,3,64 "
+                         "(FP8 and NVFP4 take the given tensor scale)")
     args = ap.parse_args()
     if args.name == "sparse_gemm_fp8":
         return gemm_case(args)
@@ -129,6 +132,13 @@ def main():
             scale = ss24.tensor_scale(x, "nvfp4", pattern if pattern != ss24.DENSE else ss24.DENSE, ws=ws,
                                       hadamard=args.hadamard, axis=args.axis)
 
+    if args.name == "error_energy":
+        def _parse(f):
+            t = f.replace(",", ":").split(":")
+            return (t[0],) + tuple(int(v) for v in t[1:])
+        e_fmt = tuple(_parse(f) for f in args.energy.split("/"))
+        e_scale = tuple(ss24.tensor_scale(x, f[0], ss24.SPARSE_24 if i == 0 else ss24.DENSE, ws=ws, axis=args.axis)
+                        if f[0] in ("fp8", "nvfp4") else None for i, f in enumerate(e_fmt))
     row_amax = ss24.amax_rows(x, ws=ws)[0] if args.name in ("amax_rows", "dense_int8_given_rows") else None
     if args.name == "dense_int8_given_rows":
         out = ss24._alloc_outputs(args.m, args.k, ss24.DENSE, ss24.make_format("int", 8, 0), torch.bfloat16, "cuda",
@@ -154,7 +164,7 @@ def main():
         elif args.name == "tensor_scale":
             ss24.tensor_scale(x, "fp8", ss24.SPARSE_24, ws=ws, out=scale)
         elif args.name == "error_energy":
-            ss24.error_energy(x, ss24.SPARSE_24, ("fp8",), ("int", 5, 128), sparse_scale=scale, dense_scale=None,
+            ss24.error_energy(x, ss24.SPARSE_24, e_fmt[0], e_fmt[1], sparse_scale=e_scale[0], dense_scale=e_scale[1],
                               ws=ws, energy=e, axis=args.axis)
         else:
             pattern, fmt, bits, group = PASSES[args.name]

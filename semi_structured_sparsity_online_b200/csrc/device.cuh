@@ -160,13 +160,15 @@ __device__ __forceinline__ float2 f16x2_to_f32(uint32_t h2)
     return make_float2(lo, hi);
 }
 
-// Two E4M3 codes in a 16-bit register -> two binary32 (exact).
-__device__ __forceinline__ float2 e4m3x2h_to_f32(uint16_t h)
+// Two E4M3 codes in a 16-bit register -> their values as f16x2 (exact).
+__device__ __forceinline__ uint32_t e4m3x2h_to_f16x2(uint16_t h)
 {
     uint32_t h2;
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(h));
-    return f16x2_to_f32(h2);
+    return h2;
 }
+// Two E4M3 codes in a 16-bit register -> two binary32 (exact).
+__device__ __forceinline__ float2 e4m3x2h_to_f32(uint16_t h) { return f16x2_to_f32(e4m3x2h_to_f16x2(h)); }
 // Two binary32 -> two E4M3 codes (lo in the low byte), saturating, in a 16-bit register.
 __device__ __forceinline__ uint16_t cvt_e4m3x2h(float lo, float hi)
 {
@@ -199,6 +201,25 @@ __device__ __forceinline__ uint32_t cvt_e2m1x4(float v0, float v1, float v2, flo
         " mov.b16 %0, {b0, b1};\n"
         "}\n"
         : "=h"(r)
+        : "f"(v0), "f"(v1), "f"(v2), "f"(v3));
+    return r;
+}
+
+// cvt_e2m1x4 that also gives the code values it writes, decoded exactly as
+// f16x2 words (values 0 and 1 in d01, 2 and 3 in d23; the low lane first).
+__device__ __forceinline__ uint32_t cvt_e2m1x4_dec(float v0, float v1, float v2, float v3, uint32_t &d01,
+                                                   uint32_t &d23)
+{
+    uint16_t r;
+    asm("{\n"
+        " .reg .b8 b0, b1;\n"
+        " cvt.rn.satfinite.e2m1x2.f32 b0, %4, %3;\n"
+        " cvt.rn.satfinite.e2m1x2.f32 b1, %6, %5;\n"
+        " mov.b16 %0, {b0, b1};\n"
+        " cvt.rn.f16x2.e2m1x2 %1, b0;\n"
+        " cvt.rn.f16x2.e2m1x2 %2, b1;\n"
+        "}\n"
+        : "=h"(r), "=r"(d01), "=r"(d23)
         : "f"(v0), "f"(v1), "f"(v2), "f"(v3));
     return r;
 }
@@ -267,6 +288,19 @@ __device__ __forceinline__ f32x2 sub2(f32x2 a, f32x2 b)
     asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
 }
+
+// (h.lo - a, h.hi - b) for the f16 lanes of h: mixed-precision subtractions,
+// the f16 operand taken exactly and each difference rounded once.
+__device__ __forceinline__ f32x2 f16x2_sub_f32(uint32_t h, float a, float b)
+{
+    float lo, hi;
+    asm("{ .reg .b16 l, h; mov.b32 {l, h}, %2;\n"
+        " sub.rn.f32.f16 %0, l, %3;\n"
+        " sub.rn.f32.f16 %1, h, %4; }"
+        : "=f"(lo), "=f"(hi)
+        : "r"(h), "f"(a), "f"(b));
+    return pack2(lo, hi);
+}
 __device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c)
 {
     f32x2 d;
@@ -334,6 +368,19 @@ __device__ __forceinline__ uint32_t bf16x2_gt_abs(uint32_t b, uint32_t a)
     return m;
 }
 __device__ __forceinline__ uint32_t sel_mask(uint32_t m, uint32_t a, uint32_t b) { return (a & m) | (b & ~m); }
+
+// True when the larger magnitude of some lane of a and b is >= the bf16 value
+// lim (both lanes of lim2 hold it): bf16x2_any_ge_abs from one packed maximum
+// of the magnitudes and one comparison.
+__device__ __forceinline__ bool bf16x2_max_ge_abs(uint32_t a, uint32_t b, uint32_t lim2)
+{
+    uint32_t m;
+    asm("{ .reg .b32 mx; max.xorsign.abs.bf16x2 mx, %1, %2; and.b32 mx, mx, 0x7fff7fff;\n"
+        " set.ge.u32.bf16x2 %0, mx, %3; }"
+        : "=r"(m)
+        : "r"(a), "r"(b), "r"(lim2));
+    return m != 0u;
+}
 
 // True when some lane of a or b has a magnitude >= the bf16 value lim (both
 // lanes of lim2 hold it): two packed comparisons.

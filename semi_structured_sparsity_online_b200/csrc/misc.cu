@@ -127,8 +127,11 @@ __global__ void selfcheck_division_kernel(int mode, uint32_t b_first, unsigned l
             const uint32_t u = ha | (hb << 16), v = hb | (ha << 16);   // lanes (a, b) and (b, a)
             const uint32_t gt = bf16x2_gt_abs(v, u);                    // lane 0: |b| > |a|; lane 1: |a| > |b|
             const uint32_t mx = bf16x2_maxabs(u, v);
+            // the FP8 overflow guard's test of a larger magnitude against a limit
+            const bool ge = bf16x2_max_ge_abs(hb | (hb << 16), 0u, a | (a << 16));
             const float fa = __uint_as_float(ha << 16), fb = __uint_as_float(hb << 16);
             bool ok = gt == ((b > a ? 0xffffu : 0u) | (a > b ? 0xffff0000u : 0u));
+            ok = ok && ge == (b >= a);
             ok = ok && (mx & 0x7fffu) == max(a, b) && ((mx >> 16) & 0x7fffu) == max(a, b);
             ok = ok && bf16x2_hmax(u) == fmaxf(fabsf(fa), fabsf(fb));
             ok = ok && __float_as_uint(bf16_lo(u)) == __float_as_uint(fa) &&

@@ -1,0 +1,22 @@
+// Instantiations of the lane-block energy pass (2:4 by magnitude, bf16,
+// full-width rows with k a multiple of 64; both sides' formats fixed).
+#include "pass_lane_energy.cuh"
+
+namespace ss24 {
+const void *stream_lb_energy_kernel_bf16(int sparse_fmt, int dense_fmt)
+{
+    switch (sparse_fmt) {
+    case kNone:
+        return stream_lb_energy_for_dense<kNone>(dense_fmt);
+    case kFp8:
+        return stream_lb_energy_for_dense<kFp8>(dense_fmt);
+    case kNvfp4:
+        return stream_lb_energy_for_dense<kNvfp4>(dense_fmt);
+    case kMxfp4:
+        return stream_lb_energy_for_dense<kMxfp4>(dense_fmt);
+    case kInt:
+        return stream_lb_energy_for_dense<kInt>(dense_fmt);
+    }
+    return nullptr;
+}
+} // namespace ss24

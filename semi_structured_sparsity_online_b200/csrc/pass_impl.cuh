@@ -776,7 +776,7 @@ __device__ __forceinline__ void finish_chunk(const PassParams &p, const typename
         if constexpr (kPair) {
             // the overflow guard as two packed comparisons of the kept values
             // with the CTA's limit (equivalent to quot_fast on their maximum)
-            const bool fast = c.rst.fast && !(c.guard && bf16x2_any_ge_abs(sl.k0, sl.k1, c.lim2));
+            const bool fast = c.rst.fast && !(c.guard && bf16x2_max_ge_abs(sl.k0, sl.k1, c.lim2));
             eq = quant_fp8_as<VPC, true>(v, fast, c.rst, o);
         } else {
             eq = quant_fp8<VPC, true>(v, vmax, c.rst, c.guard, o);

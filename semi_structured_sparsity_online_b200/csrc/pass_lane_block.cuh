@@ -64,7 +64,9 @@ __device__ __forceinline__ uint32_t fp8_codes4(const float (&v)[4], const Recip 
 
 // E2M1 codes of four values of an NVFP4 block with divisor den and its
 // reciprocal inv (bits 0..15); FAST as above. The operations are
-// quant_nvfp4's.
+// quant_nvfp4's: the codes are formed for the negated quotients and their sign
+// bits flipped, the code values come decoded from the same conversion (-c),
+// and the squared errors of v - RN(c den) are added to eq.
 template <bool FAST>
 __device__ __forceinline__ uint32_t nv_codes4(const float (&v)[4], float den, float inv, float &eq)
 {
@@ -73,23 +75,33 @@ __device__ __forceinline__ uint32_t nv_codes4(const float (&v)[4], float den, fl
     rd.y = inv;
     rd.nb = -den;
     rd.fast = true;
-    float qn[4], d[4];
+    float qn[4], dn[4];
     neg_quotients<4>(v, rd, FAST, qn);
-    const uint32_t codes = pack_e2m1<4>(qn) ^ 0x8888u;
-    unpack_e2m1<4>(codes, den, d);
-    eq += err_energy<4>(v, d);
-    return codes;
+    uint32_t d01, d23;
+    const uint32_t codes = cvt_e2m1x4_dec(qn[0], qn[1], qn[2], qn[3], d01, d23);
+    const float2 c01 = f16x2_to_f32(d01), c23 = f16x2_to_f32(d23);
+    const float cn[4] = {c01.x, c01.y, c23.x, c23.y};
+    scale_values<4>(cn, den, dn); // -RN(c den)
+    eq += err_energy_neg<4>(v, dn);
+    return codes ^ 0x8888u;
 }
 
-// E2M1 codes of four values of an MXFP4 block (times inv = 2^-e, decoded
-// times mult = 2^e); the operations are quant_mxfp4's.
-__device__ __forceinline__ uint32_t mx_codes4(const float (&v)[4], float inv, float mult, float &eq)
+// The sum of a block's squared errors from the sum rs of its squared
+// quotient-unit errors (q - c)^2, for a power-of-two scale f: v - c f = f (q -
+// c) and every step scales exactly (normal range).
+__device__ __forceinline__ float block_err(f32x2 rs, float f) { return f * (f * (lo2(rs) + hi2(rs))); }
+
+// E2M1 codes of four values of an MXFP4 block (quotients v inv, inv = 2^-e,
+// exact), adding (c - q)^2 to rs: the block's squared error is 2^2e times the
+// sum, as v - c 2^e = 2^e (q - c) exactly. The codes are quant_mxfp4's.
+__device__ __forceinline__ uint32_t mx_codes4(const float (&v)[4], float inv, f32x2 &rs)
 {
-    float q[4], d[4];
+    float q[4];
     scale_values<4>(v, inv, q);
-    const uint32_t codes = pack_e2m1<4>(q);
-    unpack_e2m1<4>(codes, mult, d);
-    eq += err_energy<4>(v, d);
+    uint32_t d01, d23;
+    const uint32_t codes = cvt_e2m1x4_dec(q[0], q[1], q[2], q[3], d01, d23);
+    const f32x2 r01 = f16x2_sub_f32(d01, q[0], q[1]), r23 = f16x2_sub_f32(d23, q[2], q[3]);
+    rs = fma2(r23, r23, fma2(r01, r01, rs));
     return codes;
 }
 
@@ -181,9 +193,10 @@ __device__ __forceinline__ void int_codes4(const float (&v)[4], const IntScale &
 // (the kept values of four chunks: NQ = 4); values(j, v) gives quad j, qm[j]
 // its largest magnitude. A group of g values spans g / 4 quads: inside the
 // lane when that is at most NQ, else over g / (4 NQ) lanes (an xor reduction
-// of their maxima). Codes are stored contiguously per lane (int8, int16 or
-// packed nibbles); a group's scale by the lane holding its first quad.
-template <int NQ, typename Values>
+// of their maxima). With STORE, codes are stored contiguously per lane (int8,
+// int16 or packed nibbles) and a group's scale by the lane holding its first
+// quad; without, only the energy is formed.
+template <int NQ, bool STORE, typename Values>
 __device__ __forceinline__ void lb_int(const QuantSpec &q, const Values &values, const float (&qm)[NQ], bool valid,
                                        bool wide, const ChunkOut &o, float &eq)
 {
@@ -236,7 +249,7 @@ __device__ __forceinline__ void lb_int(const QuantSpec &q, const Values &values,
                 int_codes4<false>(v, sc[j], q.qmax, b[j], eq);
         }
     }
-    if (!valid)
+    if (!STORE || !valid)
         return;
     if (q.store == kInt8) {
         uint32_t wd[NQ];
@@ -382,7 +395,7 @@ __device__ __forceinline__ void lb_unit(const PassConsts &c, const QuantSpec &q,
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 if constexpr (kPk)
-                    bad |= c.guard && bf16x2_any_ge_abs(k0[i], k1[i], c.lim2);
+                    bad |= c.guard && bf16x2_max_ge_abs(k0[i], k1[i], c.lim2);
                 else
                     bad |= c.guard && !(__fmul_rn(cmax[i], c.rst.y) < 0x1p126f);
             }
@@ -401,7 +414,7 @@ __device__ __forceinline__ void lb_unit(const PassConsts &c, const QuantSpec &q,
                     values(i, v);
                     bool fi;
                     if constexpr (kPk)
-                        fi = c.rst.fast && !(c.guard && bf16x2_any_ge_abs(k0[i], k1[i], c.lim2));
+                        fi = c.rst.fast && !(c.guard && bf16x2_max_ge_abs(k0[i], k1[i], c.lim2));
                     else
                         fi = c.guard ? quot_fast(c.rst, cmax[i]) : c.rst.fast;
                     codes[i] = fi ? fp8_codes4<true>(v, c.rst, eq) : fp8_codes4<false>(v, c.rst, eq);
@@ -439,12 +452,14 @@ __device__ __forceinline__ void lb_unit(const PassConsts &c, const QuantSpec &q,
             am = fmaxf(am, __shfl_xor_sync(kFull, am, 1));
             const MxScale s = mx_scale(am);
             uint32_t codes[4];
+            f32x2 rs = pack2(0.0f, 0.0f);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 float v[4];
                 values(i, v);
-                codes[i] = mx_codes4(v, s.inv, s.mult, eq);
+                codes[i] = mx_codes4(v, s.inv, rs);
             }
+            eq = block_err(rs, s.mult);
             if (valid) {
                 *reinterpret_cast<uint2 *>(o.val) =
                     make_uint2(codes[0] | (codes[1] << 16), codes[2] | (codes[3] << 16));
@@ -460,7 +475,7 @@ __device__ __forceinline__ void lb_unit(const PassConsts &c, const QuantSpec &q,
                 else
                     qm[i] = cmax[i];
             }
-            lb_int<4>(q, values, qm, valid, wide, o, eq);
+            lb_int<4, true>(q, values, qm, valid, wide, o, eq);
         }
         // (a lane outside the operand holds zeros; its scale may be zero and
         // its quotients then not finite: it contributes no energy)
@@ -557,13 +572,15 @@ __device__ __forceinline__ void lb_unit(const PassConsts &c, const QuantSpec &q,
             const MxScale s = mx_scale(bf16x2_hmax(
                 bf16x2_maxabs(bf16x2_maxabs(chunk_max2(0), chunk_max2(1)), bf16x2_maxabs(chunk_max2(2), chunk_max2(3)))));
             uint32_t codes[4];
+            f32x2 rs = pack2(0.0f, 0.0f);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 float v[4], u[4];
                 values(i, 0, v);
                 values(i, 1, u);
-                codes[i] = mx_codes4(v, s.inv, s.mult, eq) | (mx_codes4(u, s.inv, s.mult, eq) << 16);
+                codes[i] = mx_codes4(v, s.inv, rs) | (mx_codes4(u, s.inv, rs) << 16);
             }
+            eq = block_err(rs, s.mult);
             if (valid) {
                 *reinterpret_cast<uint4 *>(o.val) = make_uint4(codes[0], codes[1], codes[2], codes[3]);
                 *o.scale = static_cast<uint8_t>(s.byte);
@@ -600,20 +617,26 @@ __global__ void __launch_bounds__(kStreamThreads, (LbOcc<PAT, FMT>::value))
     const int sa = tw / p.units_b, sb = tw - sa * p.units_b;
     double e_total = 0.0, e_prune = 0.0, e_q = 0.0, e_qd = 0.0;
     Acc acc{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    while (ua < p.units_a) {
-        const int64_t row = ua;
-        const int64_t col = static_cast<int64_t>(ub) * 1024 + 32 * lane;
-        const bool valid = col < p.k; // (k is a multiple of 64: a lane is wholly in or out)
-        const T *xp = x + row * p.ld + col;
-        uint4 w[4];
+    // a unit's loads (k is a multiple of 64: a lane is wholly in or out)
+    auto load = [&](int a, int b, uint4 (&w)[4]) {
+        const int64_t col = static_cast<int64_t>(b) * 1024 + 32 * lane;
+        const bool ok = a < p.units_a && col < p.k;
+        const T *xp = x + static_cast<int64_t>(a) * p.ld + col;
         if (PAT == kSparse48 && (p.lb_wide & 1)) {
-            ld_stream32(xp, valid, w[0], w[1]);
-            ld_stream32(xp + 16, valid, w[2], w[3]);
+            ld_stream32(xp, ok, w[0], w[1]);
+            ld_stream32(xp + 16, ok, w[2], w[3]);
         } else {
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                w[i] = ld_stream(xp + 8 * i, valid);
+                w[i] = ld_stream(xp + 8 * i, ok);
         }
+    };
+    while (ua < p.units_a) {
+        const int64_t row = ua;
+        const int64_t col = static_cast<int64_t>(ub) * 1024 + 32 * lane;
+        const bool valid = col < p.k;
+        uint4 w[4];
+        load(ua, ub, w);
         const ChunkOut o = make_out<T, PAT, FMT>(p, ob, row, col, valid, lane);
         acc.et = acc.ep = acc.eq = acc.eqd = 0.0f;
         lb_unit<PAT, FMT>(c, p.q, w, valid, (p.lb_wide & 2) != 0, o, acc);

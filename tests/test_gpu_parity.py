@@ -935,6 +935,41 @@ def test_amax_and_error_energy_and_ratio(ss, ws):
     assert ws.error() == 0
 
 
+# the read-only energy pass on bf16 full-width rows (k >= 1024, a multiple of
+# 64): every pair of a 2:4 side's format and a dense side's format, with INT
+# groups inside one lane and across lanes, a ragged last unit (k = 4608) and
+# given per-tensor scales, one of them small enough that the quotients leave
+# the fast division's range
+LB_SPARSE = [("none",), ("fp8",), ("nvfp4",), ("mxfp4",), ("int", 8, 4), ("int", 8, 128), ("int", 4, 16, True),
+             ("int", 12, 64)]
+LB_DENSE = [("fp8",), ("nvfp4",), ("mxfp4",), ("int", 8, 8), ("int", 5, 256), ("int", 3, 32), ("int", 16, 64)]
+
+
+def _fmt_kw(f):
+    return dict(fmt=f[0], bits=(f[1] if len(f) > 1 else 8), group=(f[2] if len(f) > 2 else 0),
+                pack4=(len(f) > 3 and f[3]))
+
+
+@pytest.mark.parametrize("k", [1024, 4608, 5120])
+def test_error_energy_every_format_pair_full_width(ss, ws, k):
+    xh, _ = synth.linear_input(24, k, seed=90 + k, n_outlier=16)
+    x = to_dev(xh)
+    sp = {f: oracle.run(xh, **_fmt_kw(f))["energy"] for f in LB_SPARSE}
+    de = {f: oracle.run(xh, pattern=oracle.DENSE, **_fmt_kw(f))["energy"] for f in LB_DENSE}
+    for sf in LB_SPARSE:
+        for df in LB_DENSE:
+            e = ss.error_energy(x, pattern=24, sparse_fmt=sf, dense_fmt=df, ws=ws)
+            assert_energy(e, [sp[sf][0], sp[sf][1], sp[sf][2], de[df][3]])
+    for s_given in (0.37, 2.0 ** -120):
+        ts = torch.tensor([s_given], dtype=torch.float32, device="cuda")
+        for sf, df in ((("fp8",), ("fp8",)), (("nvfp4",), ("nvfp4",)), (("fp8",), ("nvfp4",))):
+            e = ss.error_energy(x, pattern=24, sparse_fmt=sf, dense_fmt=df, sparse_scale=ts, dense_scale=ts, ws=ws)
+            a = oracle.run(xh, fmt=sf[0], tensor_scale=np.float32(s_given))["energy"]
+            b = oracle.run(xh, pattern=oracle.DENSE, fmt=df[0], tensor_scale=np.float32(s_given))["energy"]
+            assert_energy(e, [a[0], a[1], a[2], b[3]])
+    assert ws.error() == 0
+
+
 def test_repeated_calls_are_deterministic(ss, ws):
     xh, _ = synth.linear_input(300, 1024, seed=1)
     x = to_dev(xh)
