@@ -25,9 +25,17 @@
 
 namespace ss24 {
 
-// Resident CTAs per SM (register budget of 64 per thread).
+// Whether a unit's loads are issued one unit ahead (a software pipeline, 16
+// more registers), and the resident CTAs per SM that the register budget then
+// allows: 3 (80 registers) with the pipeline, else 4 (64). The pipeline
+// measured faster for the NVFP4 and MXFP4 passes of the 2:4 and dense
+// patterns, slower for 4:8 and for INT (whose group reductions need the
+// registers).
+template <int PAT, int FMT> struct LbPipe {
+    static constexpr bool value = (PAT == kSparse24 || PAT == kDense) && (FMT == kNvfp4 || FMT == kMxfp4);
+};
 template <int PAT, int FMT> struct LbOcc {
-    static constexpr int value = 4;
+    static constexpr int value = LbPipe<PAT, FMT>::value ? 3 : 4;
 };
 
 // The four values of a packed 2:4 selection in output order (group 0's kept
@@ -631,12 +639,30 @@ __global__ void __launch_bounds__(kStreamThreads, (LbOcc<PAT, FMT>::value))
                 w[i] = ld_stream(xp + 8 * i, ok);
         }
     };
+    // with the pipeline, the next unit's loads are issued before this unit's
+    // arithmetic
+    constexpr bool kPipe = LbPipe<PAT, FMT>::value;
+    uint4 wn[4];
+    if constexpr (kPipe)
+        load(ua, ub, wn);
     while (ua < p.units_a) {
         const int64_t row = ua;
         const int64_t col = static_cast<int64_t>(ub) * 1024 + 32 * lane;
         const bool valid = col < p.k;
         uint4 w[4];
-        load(ua, ub, w);
+        if constexpr (kPipe) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                w[i] = wn[i];
+            int na = ua + sa, nb = ub + sb;
+            if (nb >= p.units_b) {
+                nb -= p.units_b;
+                ++na;
+            }
+            load(na, nb, wn); // (a unit past the end loads nothing)
+        } else {
+            load(ua, ub, w);
+        }
         const ChunkOut o = make_out<T, PAT, FMT>(p, ob, row, col, valid, lane);
         acc.et = acc.ep = acc.eq = acc.eqd = 0.0f;
         lb_unit<PAT, FMT>(c, p.q, w, valid, (p.lb_wide & 2) != 0, o, acc);
@@ -667,9 +693,12 @@ __global__ void __launch_bounds__(kStreamThreads, (LbOcc<PAT, FMT>::value))
 // kept values, and 2:4 INT with groups, all by magnitude. The others stay with
 // the stream kernel: bf16 and FP8 of 2:4 and of the dense pattern (few
 // instructions per chunk: bound by memory, where the stream kernel's loads of
-// 512 contiguous bytes per warp instruction are faster), dense INT and INT
-// with one scale per row (more registers than the four-CTA budget), and the
-// Wanda score (a lane's 32 column norms are 128 scattered bytes per load).
+// 512 contiguous bytes per warp instruction are faster), dense INT (its eight
+// quads per lane need more than 64 registers; at 3 CTAs per SM it measured 8%
+// slower), INT with one scale per row, and the Wanda score (a lane's 32 column
+// norms are 128 scattered bytes per load; staged in shared memory instead,
+// with conflict-free reads, the 2:4 Wanda passes still measured 9 - 40%
+// slower).
 template <int PAT> const void *stream_lb_for_fmt(int fmt)
 {
     switch (fmt) {

@@ -191,6 +191,16 @@ def test_dense_pass_full_width(ss, ws, fmt, bits, group, pack4, k):
     compare(ss, ws, xh, pattern=0, fmt=fmt, bits=bits, group=group, pack4=pack4)
 
 
+@pytest.mark.parametrize("k", [1024, 4608])
+@pytest.mark.parametrize("bits,group,pack4", [(8, 8, False), (5, 256, False), (4, 256, True), (2, 8, True),
+                                              (16, 32, False), (7, 128, False)])
+def test_dense_int_every_group_span_full_width(ss, ws, bits, group, pack4, k):
+    """Dense INT on full-width bf16 rows: groups of 8 (four per lane of 32
+    values) up to 256 (eight lanes), every code width and storage."""
+    xh = synth.linear_input(21, k, seed=19 + bits, n_outlier=8)[0]
+    compare(ss, ws, xh, pattern=0, fmt="int", bits=bits, group=group, pack4=pack4)
+
+
 @pytest.mark.parametrize("pattern", [0, 24, 48])
 @pytest.mark.parametrize("fmt,bits,group,pack4", [("none", 8, 0, False), ("fp8", 8, 0, False), ("nvfp4", 4, 0, False),
                                                   ("int", 3, 16, False), ("mxfp4", 4, 0, False)])
