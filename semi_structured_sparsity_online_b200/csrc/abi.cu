@@ -18,6 +18,7 @@ const void *stream_kernel_f32(int pattern, int score, int fmt, bool fw);
 const void *stream_kernel_bf16_rot(int pattern, int fmt, bool fw);
 const void *stream_lb_kernel_bf16(int pattern, int score, int fmt);
 const void *stream_lb_energy_kernel_bf16(int sparse_fmt, int dense_fmt);
+const void *stream_lb_kernel_bf16_rot(int pattern, int fmt);
 const void *rowsweep_kernel_bf16(int pattern, int score);
 const void *rowsweep_kernel_f32(int pattern, int score);
 const void *rowblock_kernel_bf16(int pattern, int score, int cpt);
@@ -559,7 +560,13 @@ bool plan_tile(const ss24_operand *x, int pattern, int score, int mode, TilePlan
         // full width: W = 256 with four segments per unit
         const bool fw = t->g.W == 256 && t->g.step_cols == 256;
         if (x->hadamard != 0) {
-            t->kernel = score == SS24_SCORE_MAG ? stream_kernel_bf16_rot(pattern, mode, fw) : nullptr;
+            t->kernel = nullptr;
+            if (score == SS24_SCORE_MAG) {
+                if (fw && x->k % 64 == 0)
+                    t->kernel = stream_lb_kernel_bf16_rot(pattern, mode);
+                if (!t->kernel)
+                    t->kernel = stream_kernel_bf16_rot(pattern, mode, fw);
+            }
         } else {
             // bf16 with rows a multiple of 64: one lane per 32 consecutive
             // elements (where that kernel has the format)

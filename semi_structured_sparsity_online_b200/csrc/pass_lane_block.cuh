@@ -31,12 +31,97 @@ namespace ss24 {
 // measured faster for the NVFP4 and MXFP4 passes of the 2:4 and dense
 // patterns, slower for 4:8 and for INT (whose group reductions need the
 // registers).
-template <int PAT, int FMT> struct LbPipe {
-    static constexpr bool value = (PAT == kSparse24 || PAT == kDense) && (FMT == kNvfp4 || FMT == kMxfp4);
+template <int PAT, int FMT, bool ROT = false> struct LbPipe {
+    static constexpr bool value = !ROT && (PAT == kSparse24 || PAT == kDense) && (FMT == kNvfp4 || FMT == kMxfp4);
 };
-template <int PAT, int FMT> struct LbOcc {
-    static constexpr int value = LbPipe<PAT, FMT>::value ? 3 : 4;
+// (the rotated passes hold a lane's 32 values as binary32 during the
+// rotation: 3 CTAs)
+template <int PAT, int FMT, bool ROT = false> struct LbOcc {
+    static constexpr int value = (LbPipe<PAT, FMT, ROT>::value || ROT) ? 3 : 4;
 };
+
+// Block Hadamard rotation (block b = 2^log2b, 2 <= b <= 256), in place, of
+// the 32 consecutive bf16 values a lane holds: the stream kernel's
+// rotate_chunk for the lane-block layout. Binary32 arithmetic in stage order
+// h = 1, 2, 4, ..., b/2 on the pairs (y_i, y_i+h): inside the lane for h <= 16
+// (packed adds and subtracts), across lanes for h >= 32 with the partner lane
+// ^ (h / 32), own * (+-1) + partner (exactly the rounded y_i + y_i+h in the
+// lower lane, y_i - y_i+h in the upper); then times RN(1/sqrt(b)) and rounded
+// to bf16 (nearest even). The same operations as rotate_chunk, value by
+// value. The whole warp calls it.
+// The in-lane stages h = 1 .. 2^(NS-1) of rotate_lane32 (NS <= 5), fully
+// unrolled so that every index is a constant.
+template <int NS> __device__ __forceinline__ void rotate_in_lane(float (&y)[32])
+{
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+        const int h = 1 << s;
+        // the 16 butterflies (i, i + h) with bit h of i clear, two per packed
+        // add and subtract: the t-th such i is (t & (h - 1)) | ((t & ~(h - 1)) << 1)
+#pragma unroll
+        for (int t = 0; t < 16; t += 2) {
+            const int a = (t & (h - 1)) | ((t & ~(h - 1)) << 1);
+            const int b = ((t + 1) & (h - 1)) | (((t + 1) & ~(h - 1)) << 1);
+            const f32x2 lo = pack2(y[a], y[b]), hi = pack2(y[a + h], y[b + h]);
+            const f32x2 sm = add2(lo, hi), df = sub2(lo, hi);
+            y[a] = lo2(sm), y[b] = hi2(sm), y[a + h] = lo2(df), y[b + h] = hi2(df);
+        }
+    }
+}
+
+__device__ __forceinline__ void rotate_lane32(uint4 (&w)[4], int log2b, float cb, int lane)
+{
+    float y[32];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t ws[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            y[8 * i + 2 * j] = __uint_as_float(ws[j] << 16);
+            y[8 * i + 2 * j + 1] = __uint_as_float(ws[j] & 0xffff0000u);
+        }
+    }
+    switch (log2b < 5 ? log2b : 5) {
+    case 1:
+        rotate_in_lane<1>(y);
+        break;
+    case 2:
+        rotate_in_lane<2>(y);
+        break;
+    case 3:
+        rotate_in_lane<3>(y);
+        break;
+    case 4:
+        rotate_in_lane<4>(y);
+        break;
+    default:
+        rotate_in_lane<5>(y);
+        break;
+    }
+    for (int s = 5; s < log2b; ++s) {
+        const int m = 1 << (s - 5);
+        const float sg = (lane & m) ? -1.0f : 1.0f;
+        const f32x2 sg2 = pack2(sg, sg);
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+            const float o0 = __shfl_xor_sync(kFull, y[i], m);
+            const float o1 = __shfl_xor_sync(kFull, y[i + 1], m);
+            const f32x2 r = fma2(pack2(y[i], y[i + 1]), sg2, pack2(o0, o1));
+            y[i] = lo2(r), y[i + 1] = hi2(r);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const __nv_bfloat162 h2 =
+                __floats2bfloat162_rn(__fmul_rn(y[8 * i + 2 * j], cb), __fmul_rn(y[8 * i + 2 * j + 1], cb));
+            o[j] = *reinterpret_cast<const uint32_t *>(&h2);
+        }
+        w[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
 
 // The four values of a packed 2:4 selection in output order (group 0's kept
 // values, then group 1's), as binary32.
@@ -601,8 +686,11 @@ __device__ __forceinline__ void lb_unit(const PassConsts &c, const QuantSpec &q,
 // The kernel: persistent, 8 warps per CTA, a warp per unit (1024 columns of
 // one row), units u = warp index, warp index + number of warps, ... among the
 // CTAs serving one operand of a batch; energies reduced as in stream_kernel.
-template <int PAT, int FMT>
-__global__ void __launch_bounds__(kStreamThreads, (LbOcc<PAT, FMT>::value))
+//
+// ROT: the pass over the operand rotated along k (rotate_lane32 right after
+// the loads).
+template <int PAT, int FMT, bool ROT = false>
+__global__ void __launch_bounds__(kStreamThreads, (LbOcc<PAT, FMT, ROT>::value))
     stream_lb_kernel(const __grid_constant__ PassParams pk)
 {
     using T = __nv_bfloat16;
@@ -641,7 +729,7 @@ __global__ void __launch_bounds__(kStreamThreads, (LbOcc<PAT, FMT>::value))
     };
     // with the pipeline, the next unit's loads are issued before this unit's
     // arithmetic
-    constexpr bool kPipe = LbPipe<PAT, FMT>::value;
+    constexpr bool kPipe = LbPipe<PAT, FMT, ROT>::value;
     uint4 wn[4];
     if constexpr (kPipe)
         load(ua, ub, wn);
@@ -663,6 +751,8 @@ __global__ void __launch_bounds__(kStreamThreads, (LbOcc<PAT, FMT>::value))
         } else {
             load(ua, ub, w);
         }
+        if constexpr (ROT)
+            rotate_lane32(w, p.rot_log2b, p.rot_scale, lane);
         const ChunkOut o = make_out<T, PAT, FMT>(p, ob, row, col, valid, lane);
         acc.et = acc.ep = acc.eq = acc.eqd = 0.0f;
         lb_unit<PAT, FMT>(c, p.q, w, valid, (p.lb_wide & 2) != 0, o, acc);
@@ -699,22 +789,22 @@ __global__ void __launch_bounds__(kStreamThreads, (LbOcc<PAT, FMT>::value))
 // norms are 128 scattered bytes per load; staged in shared memory instead,
 // with conflict-free reads, the 2:4 Wanda passes still measured 9 - 40%
 // slower).
-template <int PAT> const void *stream_lb_for_fmt(int fmt)
+template <int PAT, bool ROT = false> const void *stream_lb_for_fmt(int fmt)
 {
     switch (fmt) {
     case kNone:
     case kFp8:
         if constexpr (PAT == kSparse48)
-            return fmt == kNone ? reinterpret_cast<const void *>(&stream_lb_kernel<PAT, kNone>)
-                                : reinterpret_cast<const void *>(&stream_lb_kernel<PAT, kFp8>);
+            return fmt == kNone ? reinterpret_cast<const void *>(&stream_lb_kernel<PAT, kNone, ROT>)
+                                : reinterpret_cast<const void *>(&stream_lb_kernel<PAT, kFp8, ROT>);
         break;
     case kNvfp4:
-        return reinterpret_cast<const void *>(&stream_lb_kernel<PAT, kNvfp4>);
+        return reinterpret_cast<const void *>(&stream_lb_kernel<PAT, kNvfp4, ROT>);
     case kMxfp4:
-        return reinterpret_cast<const void *>(&stream_lb_kernel<PAT, kMxfp4>);
+        return reinterpret_cast<const void *>(&stream_lb_kernel<PAT, kMxfp4, ROT>);
     case kInt:
         if constexpr (PAT == kSparse24)
-            return reinterpret_cast<const void *>(&stream_lb_kernel<PAT, kInt>);
+            return reinterpret_cast<const void *>(&stream_lb_kernel<PAT, kInt, ROT>);
         break;
     }
     return nullptr;

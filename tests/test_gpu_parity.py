@@ -667,6 +667,30 @@ def test_rotated_pass_fused_matches_oracle(ss, ws, pattern, fmt, bits, group, b)
     assert ws.error() == 0
 
 
+@pytest.mark.parametrize("pattern,fmt,bits,group", [(24, "fp8", 8, 0), (24, "nvfp4", 4, 0), (24, "int", 4, 32),
+                                                    (24, "none", 8, 0), (48, "mxfp4", 4, 0), (0, "mxfp4", 4, 0),
+                                                    (0, "fp8", 8, 0)])
+@pytest.mark.parametrize("b", [2, 4, 8, 32, 64])
+def test_rotated_pass_every_block_full_width(ss, ws, pattern, fmt, bits, group, b):
+    """The rotation inside the pass on full-width rows (k = 4608: four whole
+    units and a ragged fifth) for blocks inside one lane's 32 values (b <= 32)
+    and across two lanes (b = 64), against the oracle's rotation rounded to
+    bf16 and its pass."""
+    opat = {0: oracle.DENSE, 24: oracle.SPARSE_24, 48: oracle.SPARSE_48}[pattern]
+    xh = synth.sweep_operand(11, 4608, seed=130 + b)
+    rot = oracle.hadamard_bf16(xh, b)
+    out = ss.run(to_dev(xh), pattern=pattern, fmt=fmt, bits=bits, group=group, ws=ws, hadamard=b)
+    torch.cuda.synchronize()
+    ts = oracle.tensor_scale(rot, fmt, pattern=opat) if fmt in ("fp8", "nvfp4") else None
+    ref = oracle.run(rot, pattern=opat, fmt=fmt, bits=bits, group=group,
+                     **({"tensor_scale": ts} if ts is not None else {}))
+    for key in ("values", "scales", "meta"):
+        if key in ref and out.get(key) is not None:
+            assert_same(to_np(out[key]), ref[key], key)
+    assert_energy(out["energy"], ref["energy"], atol=1e-30)
+    assert ws.error() == 0
+
+
 def test_rotated_rows_energy_and_batch(ss, ws):
     """Rotated per-row INT (the row amax pass and the INT pass from it), the
     rotated energy pass, and a rotated batch."""
