@@ -19,6 +19,7 @@ const void *stream_kernel_bf16_rot(int pattern, int fmt, bool fw);
 const void *stream_lb_kernel_bf16(int pattern, int score, int fmt);
 const void *stream_lb_energy_kernel_bf16(int sparse_fmt, int dense_fmt);
 const void *stream_lb_kernel_bf16_rot(int pattern, int fmt);
+const void *stream_lb_energy_kernel_bf16_rot(int sparse_fmt, int dense_fmt);
 const void *rowsweep_kernel_bf16(int pattern, int score);
 const void *rowsweep_kernel_f32(int pattern, int score);
 const void *rowblock_kernel_bf16(int pattern, int score, int cpt);
@@ -934,10 +935,12 @@ ss24_status ss24_error_energy(const ss24_operand *x, ss24_pattern pattern, ss24_
     if (!plan_tile(x, pattern, score, kEnergy, &t))
         return SS24_ERR_CUDA;
     // 2:4 by magnitude on bf16 full-width rows with k a multiple of 64: the
-    // lane-block form with both formats fixed at compile time
-    if (x->axis == 1 && x->hadamard == 0 && x->dtype == SS24_BF16 && score == SS24_SCORE_MAG &&
-        pattern == SS24_SPARSE_24 && t.g.W == 256 && t.g.step_cols == 256 && x->k % 64 == 0) {
-        if (const void *kl = stream_lb_energy_kernel_bf16(rs.q.fmt, rd.q.fmt))
+    // lane-block form with both formats fixed at compile time (rotated or not)
+    if (x->axis == 1 && x->dtype == SS24_BF16 && score == SS24_SCORE_MAG && pattern == SS24_SPARSE_24 &&
+        t.g.W == 256 && t.g.step_cols == 256 && x->k % 64 == 0) {
+        const void *kl = x->hadamard != 0 ? stream_lb_energy_kernel_bf16_rot(rs.q.fmt, rd.q.fmt)
+                                          : stream_lb_energy_kernel_bf16(rs.q.fmt, rd.q.fmt);
+        if (kl)
             t.kernel = kl;
     }
     PassParams p = base_params(x, t.g, ws, energy);

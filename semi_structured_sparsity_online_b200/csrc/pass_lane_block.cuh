@@ -30,14 +30,18 @@ namespace ss24 {
 // allows: 3 (80 registers) with the pipeline, else 4 (64). The pipeline
 // measured faster for the NVFP4 and MXFP4 passes of the 2:4 and dense
 // patterns, slower for 4:8 and for INT (whose group reductions need the
-// registers).
+// registers). Value 1: the next unit's words are copied into the current
+// unit's registers each step; 2: two register buffers used in turn (the loop
+// body twice), faster for NVFP4 (dense 146.2 -> 141.3 us on 16384 x 14336),
+// slower for MXFP4 (dense 107.8 -> 112.1 us).
 template <int PAT, int FMT, bool ROT = false> struct LbPipe {
-    static constexpr bool value = !ROT && (PAT == kSparse24 || PAT == kDense) && (FMT == kNvfp4 || FMT == kMxfp4);
+    static constexpr int value =
+        ROT || !(PAT == kSparse24 || PAT == kDense) ? 0 : FMT == kNvfp4 ? 2 : FMT == kMxfp4 ? 1 : 0;
 };
 // (the rotated passes hold a lane's 32 values as binary32 during the
 // rotation: 3 CTAs)
 template <int PAT, int FMT, bool ROT = false> struct LbOcc {
-    static constexpr int value = (LbPipe<PAT, FMT, ROT>::value || ROT) ? 3 : 4;
+    static constexpr int value = (LbPipe<PAT, FMT, ROT>::value != 0 || ROT) ? 3 : 4;
 };
 
 // Block Hadamard rotation (block b = 2^log2b, 2 <= b <= 256), in place, of
@@ -727,30 +731,11 @@ __global__ void __launch_bounds__(kStreamThreads, (LbOcc<PAT, FMT, ROT>::value))
                 w[i] = ld_stream(xp + 8 * i, ok);
         }
     };
-    // with the pipeline, the next unit's loads are issued before this unit's
-    // arithmetic
-    constexpr bool kPipe = LbPipe<PAT, FMT, ROT>::value;
-    uint4 wn[4];
-    if constexpr (kPipe)
-        load(ua, ub, wn);
-    while (ua < p.units_a) {
-        const int64_t row = ua;
-        const int64_t col = static_cast<int64_t>(ub) * 1024 + 32 * lane;
+    // one unit: its arithmetic and stores, and its energies added up
+    auto unit = [&](uint4 (&w)[4], int a, int b) {
+        const int64_t row = a;
+        const int64_t col = static_cast<int64_t>(b) * 1024 + 32 * lane;
         const bool valid = col < p.k;
-        uint4 w[4];
-        if constexpr (kPipe) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                w[i] = wn[i];
-            int na = ua + sa, nb = ub + sb;
-            if (nb >= p.units_b) {
-                nb -= p.units_b;
-                ++na;
-            }
-            load(na, nb, wn); // (a unit past the end loads nothing)
-        } else {
-            load(ua, ub, w);
-        }
         if constexpr (ROT)
             rotate_lane32(w, p.rot_log2b, p.rot_scale, lane);
         const ChunkOut o = make_out<T, PAT, FMT>(p, ob, row, col, valid, lane);
@@ -763,11 +748,56 @@ __global__ void __launch_bounds__(kStreamThreads, (LbOcc<PAT, FMT, ROT>::value))
             e_q += acc.eq;
         if constexpr (FMT != kNone && PAT == kDense)
             e_qd += acc.eqd;
-        ua += sa;
-        ub += sb;
-        if (ub >= p.units_b) {
-            ub -= p.units_b;
-            ++ua;
+    };
+    auto advance = [&](int &a, int &b) {
+        a += sa;
+        b += sb;
+        if (b >= p.units_b) {
+            b -= p.units_b;
+            ++a;
+        }
+    };
+    // (with the pipeline, a unit past the end loads nothing)
+    constexpr int kPipe = LbPipe<PAT, FMT, ROT>::value;
+    if constexpr (kPipe == 2) {
+        uint4 wa[4], wb[4];
+        load(ua, ub, wa);
+        while (ua < p.units_a) {
+            int na = ua, nb = ub;
+            advance(na, nb);
+            load(na, nb, wb);
+            unit(wa, ua, ub);
+            ua = na;
+            ub = nb;
+            if (ua >= p.units_a)
+                break;
+            advance(na, nb);
+            load(na, nb, wa);
+            unit(wb, ua, ub);
+            ua = na;
+            ub = nb;
+        }
+    } else if constexpr (kPipe == 1) {
+        uint4 wn[4];
+        load(ua, ub, wn);
+        while (ua < p.units_a) {
+            uint4 w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                w[i] = wn[i];
+            int na = ua, nb = ub;
+            advance(na, nb);
+            load(na, nb, wn);
+            unit(w, ua, ub);
+            ua = na;
+            ub = nb;
+        }
+    } else {
+        while (ua < p.units_a) {
+            uint4 w[4];
+            load(ua, ub, w);
+            unit(w, ua, ub);
+            advance(ua, ub);
         }
     }
     const PassParams v = operand_view(pk);

@@ -192,7 +192,8 @@ __device__ __forceinline__ float lb_dense_energy(const PassConsts &c, const Quan
     return eq;
 }
 
-template <int SF, int DF>
+// ROT: over the operand rotated along k (rotate_lane32 right after the loads).
+template <int SF, int DF, bool ROT = false>
 __global__ void __launch_bounds__(kStreamThreads, 3) stream_lb_energy_kernel(const __grid_constant__ PassParams pk)
 {
     using T = __nv_bfloat16;
@@ -220,6 +221,8 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_lb_energy_kernel(con
 #pragma unroll
         for (int i = 0; i < 4; ++i)
             w[i] = ld_stream(xp + 8 * i, valid);
+        if constexpr (ROT)
+            rotate_lane32(w, p.rot_log2b, p.rot_scale, lane);
         uint32_t k0[4], k1[4];
         float et = 0.0f, ep = 0.0f;
 #pragma unroll
@@ -254,17 +257,17 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_lb_energy_kernel(con
 // The lane-block energy kernel for 2:4 by magnitude with the 2:4 side's format
 // sf (NONE, FP8, NVFP4, MXFP4, INT) and the dense side's format df (FP8,
 // NVFP4, MXFP4, INT), or nullptr.
-template <int SF> const void *stream_lb_energy_for_dense(int df)
+template <int SF, bool ROT = false> const void *stream_lb_energy_for_dense(int df)
 {
     switch (df) {
     case kFp8:
-        return reinterpret_cast<const void *>(&stream_lb_energy_kernel<SF, kFp8>);
+        return reinterpret_cast<const void *>(&stream_lb_energy_kernel<SF, kFp8, ROT>);
     case kNvfp4:
-        return reinterpret_cast<const void *>(&stream_lb_energy_kernel<SF, kNvfp4>);
+        return reinterpret_cast<const void *>(&stream_lb_energy_kernel<SF, kNvfp4, ROT>);
     case kMxfp4:
-        return reinterpret_cast<const void *>(&stream_lb_energy_kernel<SF, kMxfp4>);
+        return reinterpret_cast<const void *>(&stream_lb_energy_kernel<SF, kMxfp4, ROT>);
     case kInt:
-        return reinterpret_cast<const void *>(&stream_lb_energy_kernel<SF, kInt>);
+        return reinterpret_cast<const void *>(&stream_lb_energy_kernel<SF, kInt, ROT>);
     }
     return nullptr;
 }

@@ -691,6 +691,21 @@ def test_rotated_pass_every_block_full_width(ss, ws, pattern, fmt, bits, group, 
     assert ws.error() == 0
 
 
+@pytest.mark.parametrize("b", [8, 32, 128])
+def test_rotated_error_energy_format_pairs(ss, ws, b):
+    """The read-only energy pass over the operand rotated in registers (full-
+    width rows, k = 4608), against the oracle's passes on its own rotation."""
+    xh = synth.sweep_operand(9, 4608, seed=140 + b)
+    rot = oracle.hadamard_bf16(xh, b)
+    x = to_dev(xh)
+    for sf, df in ((("nvfp4",), ("mxfp4",)), (("mxfp4",), ("int", 3, 64)), (("int", 4, 16, True), ("fp8",))):
+        e = ss.error_energy(x, pattern=24, sparse_fmt=sf, dense_fmt=df, ws=ws, hadamard=b)
+        sp = oracle.run(rot, **_fmt_kw(sf))["energy"]
+        de = oracle.run(rot, pattern=oracle.DENSE, **_fmt_kw(df))["energy"]
+        assert_energy(e, [sp[0], sp[1], sp[2], de[3]])
+    assert ws.error() == 0
+
+
 def test_rotated_rows_energy_and_batch(ss, ws):
     """Rotated per-row INT (the row amax pass and the INT pass from it), the
     rotated energy pass, and a rotated batch."""
