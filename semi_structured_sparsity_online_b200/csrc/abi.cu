@@ -19,6 +19,7 @@ const void *stream_kernel_bf16_rot(int pattern, int fmt, bool fw);
 const void *stream_lb_kernel_bf16(int pattern, int score, int fmt);
 const void *stream_lb_energy_kernel_bf16(int sparse_fmt, int dense_fmt);
 const void *stream_lb_kernel_bf16_rot(int pattern, int fmt);
+const void *stream_lb_amax_kernel_bf16_rot(int pattern);
 const void *stream_lb_energy_kernel_bf16_rot(int sparse_fmt, int dense_fmt);
 const void *rowsweep_kernel_bf16(int pattern, int score);
 const void *rowsweep_kernel_f32(int pattern, int score);
@@ -598,6 +599,15 @@ cudaError_t run_amax(const ss24_operand *x, int pattern, int score, const float 
     TilePlan t;
     if (!plan_tile(x, pat, score, kAmax, &t))
         return cudaErrorInvalidValue;
+    // over the rotated operand on bf16 full-width rows (k a multiple of 64),
+    // without per-row output: the lane-block amax kernel
+    if (x->axis == 1 && x->hadamard != 0 && score == SS24_SCORE_MAG && !row_amax && t.g.W == 256 &&
+        t.g.step_cols == 256 && x->k % 64 == 0) {
+        if (const void *kl = stream_lb_amax_kernel_bf16_rot(pat)) {
+            t.kernel = kl;
+            t.smem = 0;
+        }
+    }
     PassParams p = base_params(x, t.g, ws, nullptr);
     p.norms = norms;
     p.q.scale_out = scale_out;

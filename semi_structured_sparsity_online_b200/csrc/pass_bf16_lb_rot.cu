@@ -31,6 +31,17 @@ template <int PAT> const void *rot_for_fmt(int fmt)
 
 } // namespace
 
+const void *stream_lb_amax_kernel_bf16_rot(int pattern)
+{
+    if (pattern == kDense)
+        return reinterpret_cast<const void *>(&stream_lb_amax_rot_kernel<kDense>);
+    if (pattern == kSparse24)
+        return reinterpret_cast<const void *>(&stream_lb_amax_rot_kernel<kSparse24>);
+    if (pattern == kSparse48)
+        return reinterpret_cast<const void *>(&stream_lb_amax_rot_kernel<kSparse48>);
+    return nullptr;
+}
+
 const void *stream_lb_kernel_bf16_rot(int pattern, int fmt)
 {
     if (pattern == kDense)

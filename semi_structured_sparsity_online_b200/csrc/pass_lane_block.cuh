@@ -32,11 +32,14 @@ namespace ss24 {
 // patterns, slower for 4:8 and for INT (whose group reductions need the
 // registers). Value 1: the next unit's words are copied into the current
 // unit's registers each step; 2: two register buffers used in turn (the loop
-// body twice), faster for NVFP4 (dense 146.2 -> 141.3 us on 16384 x 14336),
-// slower for MXFP4 (dense 107.8 -> 112.1 us).
+// body twice), faster for NVFP4 (dense 146.2 -> 141.3 us on 16384 x 14336)
+// and for 2:4 INT (INT8 g128 on 8 x 4096^2: 115.1 -> 112.4 us), slower for
+// MXFP4 (dense 107.8 -> 112.1 us) and for 4:8 (NVFP4 154.6 -> 159.8 us).
 template <int PAT, int FMT, bool ROT = false> struct LbPipe {
-    static constexpr int value =
-        ROT || !(PAT == kSparse24 || PAT == kDense) ? 0 : FMT == kNvfp4 ? 2 : FMT == kMxfp4 ? 1 : 0;
+    static constexpr int value = ROT || !(PAT == kSparse24 || PAT == kDense) ? 0
+                                 : (FMT == kNvfp4 || FMT == kInt)            ? 2
+                                 : FMT == kMxfp4                             ? 1
+                                                                             : 0;
 };
 // (the rotated passes hold a lane's 32 values as binary32 during the
 // rotation: 3 CTAs)
@@ -804,6 +807,68 @@ __global__ void __launch_bounds__(kStreamThreads, (LbOcc<PAT, FMT, ROT>::value))
     if (!v.energy_out)
         return;
     grid_reduce_energy(v, e_total, e_prune, e_q, e_qd, red, &flag, tid, lane, warp);
+}
+
+// The amax pass over the rotated operand in the lane-block layout (bf16, by
+// magnitude, full-width rows with k a multiple of 64, no per-row output): the
+// largest magnitude of all rotated values and of the kept ones (2:4 keeps
+// every group's largest value; pairwise 4:8 can drop it and takes the
+// selection's own maximum), reduced over the grid as the stream kernel's amax
+// mode does (grid_reduce_amax: the operand's two maxima, the tensor scale or
+// the caller's amax).
+template <int PAT>
+__global__ void __launch_bounds__(kStreamThreads, 3) stream_lb_amax_rot_kernel(const __grid_constant__ PassParams pk)
+{
+    using T = __nv_bfloat16;
+    const PassParams &p = pk;
+    const int op = static_cast<int>(blockIdx.x) / pk.ctas_per_op;
+    const int cta = static_cast<int>(blockIdx.x) - op * pk.ctas_per_op;
+    __shared__ float fred[kStreamWarps * 2];
+    __shared__ uint32_t flag;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    grid_dependency_wait();
+    grid_dependents_launch();
+    const T *x = static_cast<const T *>(p.x) + op * p.x_bstride;
+    const int tw = p.ctas_per_op * kStreamWarps;
+    const int u0 = cta * kStreamWarps + warp;
+    int ua = u0 / p.units_b, ub = u0 - ua * p.units_b;
+    const int sa = tw / p.units_b, sb = tw - sa * p.units_b;
+    float amax_all = 0.0f, amax_kept = 0.0f;
+    while (ua < p.units_a) {
+        const int64_t col = static_cast<int64_t>(ub) * 1024 + 32 * lane;
+        const bool valid = col < p.k; // (a lane outside the row holds zeros)
+        const T *xp = x + static_cast<int64_t>(ua) * p.ld + col;
+        uint4 w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            w[i] = ld_stream(xp + 8 * i, valid);
+        rotate_lane32(w, p.rot_log2b, p.rot_scale, lane);
+        uint32_t m2 = bf16x2_maxabs(bf16x2_maxabs(w[0].x, w[0].y), bf16x2_maxabs(w[0].z, w[0].w));
+#pragma unroll
+        for (int i = 1; i < 4; ++i)
+            m2 = bf16x2_maxabs(m2, bf16x2_maxabs(bf16x2_maxabs(w[i].x, w[i].y), bf16x2_maxabs(w[i].z, w[i].w)));
+        const float all = bf16x2_hmax(m2);
+        amax_all = fmaxf(amax_all, all);
+        if constexpr (PAT == kSparse48) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                Elem<T>::Raw raw;
+                raw.v = w[i];
+                const ChunkOut none{nullptr, nullptr, nullptr, nullptr, false, 0};
+                amax_kept = fmaxf(amax_kept, select_chunk<T, PAT, kMag>(raw, none).vmax);
+            }
+        } else {
+            amax_kept = fmaxf(amax_kept, all);
+        }
+        ua += sa;
+        ub += sb;
+        if (ub >= p.units_b) {
+            ub -= p.units_b;
+            ++ua;
+        }
+    }
+    const PassParams v = operand_view(pk);
+    grid_reduce_amax<PAT>(v, amax_kept, amax_all, fred, &flag, tid, lane, warp);
 }
 
 // The lane-block kernel for (pattern, format), or nullptr where it has none.

@@ -376,6 +376,21 @@ def test_batch_given_scales_axis0_and_long_rows(ss, ws):
     compare_batch(ss, ws, xl, pattern=24, fmt="int", bits=8, group=0, pad_rows=3)
 
 
+@pytest.mark.parametrize("pattern,fmt,bits,group", [(24, "nvfp4", 4, 0), (0, "nvfp4", 4, 0), (24, "mxfp4", 4, 0),
+                                                    (0, "mxfp4", 4, 0), (48, "nvfp4", 4, 0), (24, "int", 8, 128),
+                                                    (48, "fp8", 8, 0)])
+@pytest.mark.parametrize("rows,k,batch,pad", [(1, 1024, 1, 0), (2, 4160, 3, 2), (5, 2048, 4, 0)])
+def test_lane_block_few_units_and_batches(ss, ws, pattern, fmt, bits, group, rows, k, batch, pad):
+    """The lane-block kernels (with and without their one-unit-ahead loads) on
+    operands with fewer units than warps, a last unit with two lanes inside
+    the row (k = 4160), and strided batches: every output and energy of every
+    operand against the oracle."""
+    if fmt == "int" and (k // 2) % group:
+        pytest.skip("the rows hold no whole number of groups")
+    xs = [synth.sweep_operand(rows, k, seed=150 + 7 * b + rows) for b in range(batch)]
+    compare_batch(ss, ws, xs, pattern=pattern, fmt=fmt, bits=bits, group=group, pad_rows=pad)
+
+
 def test_batch_amax_scale_energy_and_empty(ss, ws):
     xs = [synth.gaussian_bf16(40, 256, seed=80 + b, std=1.0 + b) for b in range(5)]
     xd = to_dev(np.stack(xs))
