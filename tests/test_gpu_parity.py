@@ -1206,3 +1206,21 @@ def test_full_sweep_nvfp4(ss, ws, tokens, k):
     full_check(ss, ws, xh, pattern=24, fmt="nvfp4")
     full_check(ss, ws, xh, pattern=48, fmt="nvfp4")
     full_check(ss, ws, xh, pattern=24, fmt="none")
+    full_check(ss, ws, xh, pattern=0, fmt="nvfp4")
+    full_check(ss, ws, xh, pattern=24, fmt="mxfp4")
+    full_check(ss, ws, xh, pattern=0, fmt="mxfp4")
+
+
+def test_full_sweep_error_energy(ss, ws):
+    """The read-only energy pass over the largest sweep operand (16384 x
+    14336) for two format pairs, against the oracle's sparse and dense passes
+    over the whole tensor: all four energies within 1e-6 relative."""
+    xh = synth.sweep_operand(16384, 14336, seed=9)
+    x = to_dev(xh)
+    for sf, df in ((("nvfp4",), ("nvfp4",)), (("fp8",), ("int", 5, 128))):
+        e = ss.error_energy(x, pattern=24, sparse_fmt=sf, dense_fmt=df, ws=ws)
+        torch.cuda.synchronize()
+        sp = oracle.run_parallel(xh, pattern=oracle.SPARSE_24, **_fmt_kw(sf))["energy"]
+        de = oracle.run_parallel(xh, pattern=oracle.DENSE, **_fmt_kw(df))["energy"]
+        assert_energy(e, [sp[0], sp[1], sp[2], de[3]])
+    assert ws.error() == 0
