@@ -16,15 +16,19 @@
 // steps) per copy. A 2-D TMA box of 16 bytes x 128 rows cuts them out of the
 // row-major array; no reordering pass is needed.
 //
-// Kernel. One CTA per 128 x 128 output tile, 128 threads. Lane 0 of warp 0
-// streams k tiles of 256 (A: 128 rows x 128 bytes, B: 128 rows x 256 bytes,
-// both with 128-byte swizzle; metadata: 128 rows x 32 bytes) into a ring of
-// stages by TMA; lane 0 of warp 1 copies each stage's metadata into tensor
-// memory and issues four sparse MMAs (k = 64 each) per stage, releasing the
-// stage with a commit; the four warps then read the accumulator (warp w: rows
-// 32w .. 32w + 31) and write Y. Every barrier wait is bounded: a wait that
-// gives up records an error code in the workspace, and the kernel still drains
-// its copies and frees its tensor memory.
+// Kernel. One CTA per 128 x BN output tile, 128 threads. Lane 0 of warp 0
+// streams k tiles of BK into a ring of stages by TMA (A: 128 rows x BK/2
+// bytes with 128- or 64-byte swizzle, B: BN rows x BK bytes as boxes of 128
+// bytes with 128-byte swizzle; metadata: 128 rows x BK/8 bytes); lane 0 of
+// warp 1 copies each stage's metadata into tensor memory and issues BK/64
+// sparse MMAs (k = 64 each, N = BN) per stage, releasing the stage with a
+// commit; the four warps then read the accumulator (warp w: rows 32w .. 32w +
+// 31) and write Y. Two shapes: BN = 256 with BK = 128 and five stages where n
+// is a multiple of 256 (each A and B byte brought to the SM serves twice the
+// products of the other shape), else BN = 128 with BK = 256 and four stages.
+// Every barrier wait is bounded: a wait that gives up records an error code
+// in the workspace, and the kernel still drains its copies and frees its
+// tensor memory.
 #include <cudaTypedefs.h>
 
 #include "device.cuh"
@@ -34,14 +38,24 @@ namespace ss24 {
 
 namespace {
 
-constexpr int kGemmBM = 128, kGemmBN = 128, kGemmBK = 256; // logical k per stage
-constexpr int kGemmStages = 4;
-constexpr uint32_t kGemmABytes = kGemmBM * kGemmBK / 2;   // 16 KiB (compressed)
-constexpr uint32_t kGemmBBytes = kGemmBN * kGemmBK;       // 32 KiB (two 128-byte boxes)
-constexpr uint32_t kGemmEBytes = kGemmBM * kGemmBK / 8;   // 4 KiB (two 16-byte boxes)
-constexpr uint32_t kGemmStageBytes = kGemmABytes + kGemmBBytes + kGemmEBytes;
-constexpr uint32_t kGemmTmemCols = 256; // accumulator 128 columns, metadata 8 per stage
+constexpr int kGemmBM = 128;
 constexpr int kGemmThreads = 128;
+
+// A tile shape: BN output columns, BK logical k per stage, STAGES stages.
+template <int BN, int BK, int STAGES> struct GemmShape {
+    static constexpr uint32_t kABytes = kGemmBM * BK / 2; // compressed A: 128 rows x BK/2 bytes
+    static constexpr uint32_t kBBytes = BN * BK;          // BK/128 boxes of BN rows x 128 bytes
+    static constexpr uint32_t kEBytes = kGemmBM * BK / 8; // BK/128 boxes of 128 rows x 16 bytes
+    static constexpr uint32_t kStageBytes = kABytes + kBBytes + kEBytes;
+    static constexpr int kBoxes = BK / 128;               // B and metadata boxes per stage
+    static constexpr int kSteps = BK / 64;                // MMAs per stage
+    static constexpr uint32_t kMetaCols = BK / 32;        // tensor-memory columns of a stage's metadata
+    // accumulator BN columns + the stages' metadata, rounded up to a power of two
+    static constexpr uint32_t kTmemCols = BN + STAGES * kMetaCols <= 256 ? 256 : 512;
+    static constexpr size_t kSmemBytes = STAGES * kStageBytes + 1024 + 256;
+    static_assert(kStageBytes % 1024 == 0, "stages on 1024-byte boundaries");
+    static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+};
 
 // Shared-memory matrix descriptor (tcgen05): start address, leading and stride
 // byte offsets (in 16-byte units), version 1, layout type.
@@ -57,16 +71,22 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
 }
 constexpr uint32_t kLayoutNone = 0, kLayoutSw128 = 2;
 
+constexpr uint32_t kLayoutSw64 = 4;
+
 // K-major operand with 128-byte swizzle: rows of 128 bytes, 8-row groups
 // 1024 bytes apart.
 __device__ __forceinline__ uint64_t desc_sw128(uint32_t addr) { return smem_desc(addr, 1, 64, kLayoutSw128); }
+// K-major operand with 64-byte swizzle: rows of 64 bytes, 8-row groups 512
+// bytes apart.
+__device__ __forceinline__ uint64_t desc_sw64(uint32_t addr) { return smem_desc(addr, 1, 32, kLayoutSw64); }
 
 // Instruction descriptor: sparse, binary32 accumulator, E4M3 x E4M3, both
-// K-major, N = 128, M = 128.
+// K-major, N = BN, M = 128.
+template <int BN>
 constexpr uint32_t kGemmIdesc = (1u << 2)                                     // sparse
                                 | (1u << 4)                                   // D: f32
                                 | (0u << 7) | (0u << 10)                      // A, B: e4m3
-                                | (static_cast<uint32_t>(kGemmBN >> 3) << 17) // N / 8
+                                | (static_cast<uint32_t>(BN >> 3) << 17)      // N / 8
                                 | (static_cast<uint32_t>(kGemmBM >> 4) << 24); // M / 16
 
 __device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t cols)
@@ -135,25 +155,27 @@ struct GemmParams {
     uint64_t wait_limit_ns;
 };
 
+template <int BN, int BK, int STAGES>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     sparse_gemm_fp8_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                            const __grid_constant__ CUtensorMap map_e, const GemmParams p)
 {
+    using S = GemmShape<BN, BK, STAGES>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    // stages start on a 1024-byte boundary (128-byte swizzle atoms)
+    // stages start on a 1024-byte boundary (swizzle atoms)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *stages = smem;
-    uint64_t *full = reinterpret_cast<uint64_t *>(stages + kGemmStages * kGemmStageBytes);
-    uint64_t *empty = full + kGemmStages;
-    uint64_t *accbar = empty + kGemmStages;
+    uint64_t *full = reinterpret_cast<uint64_t *>(stages + STAGES * S::kStageBytes);
+    uint64_t *empty = full + STAGES;
+    uint64_t *accbar = empty + STAGES;
     uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(accbar + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kGemmBN, m0 = static_cast<int64_t>(blockIdx.y) * kGemmBM;
-    const int nk = static_cast<int>(p.k / kGemmBK);
+    const int64_t n0 = static_cast<int64_t>(blockIdx.x) * BN, m0 = static_cast<int64_t>(blockIdx.y) * kGemmBM;
+    const int nk = static_cast<int>(p.k / BK);
 
     if (tid == 0) {
-        for (int s = 0; s < kGemmStages; ++s) {
+        for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
@@ -161,7 +183,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         fence_barrier_init();
     }
     if (warp == 0) {
-        tmem_alloc(tmem_base_smem, kGemmTmemCols);
+        tmem_alloc(tmem_base_smem, S::kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -175,47 +197,50 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int issued = 0;
         bool failed = false;
         for (int kt = 0; kt < nk; ++kt) {
-            const int s = kt % kGemmStages;
-            if (kt >= kGemmStages && !mbar_wait(&empty[s], ((kt / kGemmStages) - 1) & 1, p.wait_limit_ns)) {
+            const int s = kt % STAGES;
+            if (kt >= STAGES && !mbar_wait(&empty[s], ((kt / STAGES) - 1) & 1, p.wait_limit_ns)) {
                 atomicCAS(p.err, 0, 11);
                 failed = true;
                 break;
             }
-            uint8_t *sa = stages + s * kGemmStageBytes, *sb = sa + kGemmABytes, *se = sb + kGemmBBytes;
-            mbar_arrive_expect_tx(&full[s], kGemmStageBytes);
-            const int32_t ka = static_cast<int32_t>(kt * (kGemmBK / 2)), kb = kt * kGemmBK, ke = kt * (kGemmBK / 8);
+            uint8_t *sa = stages + s * S::kStageBytes, *sb = sa + S::kABytes, *se = sb + S::kBBytes;
+            mbar_arrive_expect_tx(&full[s], S::kStageBytes);
+            const int32_t ka = static_cast<int32_t>(kt * (BK / 2)), kb = kt * BK, ke = kt * (BK / 8);
             tma_box(sa, &map_a, ka, static_cast<int32_t>(m0), &full[s]);
-            tma_box(sb, &map_b, kb, static_cast<int32_t>(n0), &full[s]);
-            tma_box(sb + kGemmBBytes / 2, &map_b, kb + 128, static_cast<int32_t>(n0), &full[s]);
-            tma_box(se, &map_e, ke, static_cast<int32_t>(m0), &full[s]);
-            tma_box(se + kGemmEBytes / 2, &map_e, ke + 16, static_cast<int32_t>(m0), &full[s]);
+#pragma unroll
+            for (int h = 0; h < S::kBoxes; ++h) {
+                tma_box(sb + h * (BN * 128), &map_b, kb + 128 * h, static_cast<int32_t>(n0), &full[s]);
+                tma_box(se + h * (kGemmBM * 16), &map_e, ke + 16 * h, static_cast<int32_t>(m0), &full[s]);
+            }
             ++issued;
         }
         if (failed) {
             // the copies already issued land before the CTA can exit
-            for (int kt = issued > kGemmStages ? issued - kGemmStages : 0; kt < issued; ++kt)
-                (void)mbar_wait(&full[kt % kGemmStages], (kt / kGemmStages) & 1, p.wait_limit_ns);
+            for (int kt = issued > STAGES ? issued - STAGES : 0; kt < issued; ++kt)
+                (void)mbar_wait(&full[kt % STAGES], (kt / STAGES) & 1, p.wait_limit_ns);
         }
     } else if (warp == 1 && lane == 0) {
         // MMA issuer
         const uint32_t acc = tmem;
         for (int kt = 0; kt < nk; ++kt) {
-            const int s = kt % kGemmStages;
-            if (!mbar_wait(&full[s], (kt / kGemmStages) & 1, p.wait_limit_ns)) {
+            const int s = kt % STAGES;
+            if (!mbar_wait(&full[s], (kt / STAGES) & 1, p.wait_limit_ns)) {
                 atomicCAS(p.err, 0, 12);
                 break;
             }
             tc_fence_after();
-            uint8_t *sa = stages + s * kGemmStageBytes, *sb = sa + kGemmABytes, *se = sb + kGemmBBytes;
-            // metadata: two 128-row x 16-byte tiles into this stage's 8 columns
-            const uint32_t ecol = kGemmBN + 8 * s;
-            for (int h = 0; h < 2; ++h)
-                tc_cp_128x128b(tmem + ecol + 4 * h, smem_desc(smem_u32(se + h * (kGemmEBytes / 2)), 128, 8, kLayoutNone));
-            for (int j = 0; j < 4; ++j) {
+            uint8_t *sa = stages + s * S::kStageBytes, *sb = sa + S::kABytes, *se = sb + S::kBBytes;
+            // metadata: 128-row x 16-byte tiles into this stage's columns
+            const uint32_t ecol = BN + S::kMetaCols * s;
+#pragma unroll
+            for (int h = 0; h < S::kBoxes; ++h)
+                tc_cp_128x128b(tmem + ecol + 4 * h, smem_desc(smem_u32(se + h * (kGemmBM * 16)), 128, 8, kLayoutNone));
+#pragma unroll
+            for (int j = 0; j < S::kSteps; ++j) {
                 // k step j: 64 values of k = 32 bytes of compressed A, 64 bytes of B
-                const uint64_t ad = desc_sw128(smem_u32(sa) + 32 * j);
-                const uint64_t bd = desc_sw128(smem_u32(sb) + (j >> 1) * (kGemmBBytes / 2) + 64 * (j & 1));
-                tc_mma_sp(acc, ad, bd, tmem + ecol + 2 * j, kGemmIdesc, (kt | j) != 0 ? 1u : 0u);
+                const uint64_t ad = BK == 256 ? desc_sw128(smem_u32(sa) + 32 * j) : desc_sw64(smem_u32(sa) + 32 * j);
+                const uint64_t bd = desc_sw128(smem_u32(sb) + (j >> 1) * (BN * 128) + 64 * (j & 1));
+                tc_mma_sp(acc, ad, bd, tmem + ecol + 2 * j, kGemmIdesc<BN>, (kt | j) != 0 ? 1u : 0u);
             }
             tc_commit(&empty[s]); // the stage is free once these MMAs have read it
         }
@@ -232,7 +257,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int64_t row = m0 + 32 * warp + lane;
     float *yr = p.y + row * p.n + n0;
 #pragma unroll 1
-    for (int c0 = 0; c0 < kGemmBN; c0 += 32) {
+    for (int c0 = 0; c0 < BN; c0 += 32) {
         uint32_t v[32];
         tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + c0, v);
 #pragma unroll
@@ -245,7 +270,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, kGemmTmemCols);
+        tmem_dealloc(tmem, S::kTmemCols);
     }
 }
 
@@ -267,36 +292,52 @@ bool encode_u8(CUtensorMap *map, const void *base, uint64_t inner, uint64_t oute
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-} // namespace
+using GemmWide = GemmShape<256, 128, 5>;
+using GemmNarrow = GemmShape<128, 256, 4>;
 
-size_t sparse_gemm_smem_bytes() { return kGemmStages * kGemmStageBytes + 1024 + 256; }
-
-cudaError_t launch_sparse_gemm_fp8(const uint8_t *a_values, const uint8_t *a_meta, const float *a_scale,
-                                   const uint8_t *b, const float *b_scale, int64_t m, int64_t n, int64_t k, float *y,
-                                   int32_t *err, uint64_t wait_limit_ns, cudaStream_t stream)
+template <int BN, int BK, int STAGES>
+cudaError_t launch_shape(const uint8_t *a_values, const uint8_t *a_meta, const float *a_scale, const uint8_t *b,
+                         const float *b_scale, int64_t m, int64_t n, int64_t k, float *y, int32_t *err,
+                         uint64_t wait_limit_ns, cudaStream_t stream)
 {
+    using S = GemmShape<BN, BK, STAGES>;
     CUtensorMap ma, mb, me;
-    if (!encode_u8(&ma, a_values, k / 2, m, k / 2, 128, kGemmBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_u8(&mb, b, k, n, k, 128, kGemmBN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+    if (!encode_u8(&ma, a_values, k / 2, m, k / 2, BK / 2, kGemmBM,
+                   BK == 256 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !encode_u8(&mb, b, k, n, k, 128, BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_u8(&me, a_meta, k / 8, m, k / 8, 16, kGemmBM, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    const size_t smem = sparse_gemm_smem_bytes();
-    cudaError_t e = cudaFuncSetAttribute(sparse_gemm_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    auto kern = sparse_gemm_fp8_kernel<BN, BK, STAGES>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(S::kSmemBytes));
     if (e != cudaSuccess)
         return e;
     GemmParams p{m, n, k, a_scale, b_scale, y, err, wait_limit_ns};
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(n / kGemmBN), static_cast<unsigned>(m / kGemmBM));
+    cfg.gridDim = dim3(static_cast<unsigned>(n / BN), static_cast<unsigned>(m / kGemmBM));
     cfg.blockDim = dim3(kGemmThreads);
-    cfg.dynamicSmemBytes = smem;
+    cfg.dynamicSmemBytes = S::kSmemBytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, sparse_gemm_fp8_kernel, ma, mb, me, p);
+    return cudaLaunchKernelEx(&cfg, kern, ma, mb, me, p);
+}
+
+} // namespace
+
+size_t sparse_gemm_smem_bytes() { return GemmWide::kSmemBytes > GemmNarrow::kSmemBytes ? GemmWide::kSmemBytes : GemmNarrow::kSmemBytes; }
+
+cudaError_t launch_sparse_gemm_fp8(const uint8_t *a_values, const uint8_t *a_meta, const float *a_scale,
+                                   const uint8_t *b, const float *b_scale, int64_t m, int64_t n, int64_t k, float *y,
+                                   int32_t *err, uint64_t wait_limit_ns, cudaStream_t stream)
+{
+    if (n % 256 == 0)
+        return launch_shape<256, 128, 5>(a_values, a_meta, a_scale, b, b_scale, m, n, k, y, err, wait_limit_ns,
+                                         stream);
+    return launch_shape<128, 256, 4>(a_values, a_meta, a_scale, b, b_scale, m, n, k, y, err, wait_limit_ns, stream);
 }
 
 } // namespace ss24
