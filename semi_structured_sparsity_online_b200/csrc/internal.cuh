@@ -48,7 +48,8 @@ constexpr int kRowThreads = 256;
 // 272 / 528 bytes) and process it like an axis-1 tile of width 128.
 constexpr int kAxis0K = 128;
 constexpr size_t kAxis0TBytes = 64 * 136 * 2; // >= 32 * 132 * 4
-constexpr size_t kAxis0SmemBytes = kStages * kStageBytes + kAxis0TBytes + 4096;
+// (two transpose buffers, used by alternate tiles)
+constexpr size_t kAxis0SmemBytes = kStages * kStageBytes + 2 * kAxis0TBytes + 4096;
 
 // Workspace layout (bytes):
 //   [0, 256)                 header: the error word at 0

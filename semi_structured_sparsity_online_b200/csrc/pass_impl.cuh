@@ -2084,8 +2084,8 @@ __global__ void __launch_bounds__(kThreads, 2) axis0_kernel(const __grid_constan
     const PassParams p = operand_view(pk);
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t *stages = smem;
-    uint8_t *Tb = smem + kStages * kStageBytes;
-    uint64_t *full = reinterpret_cast<uint64_t *>(Tb + kAxis0TBytes);
+    uint8_t *Tb = smem + kStages * kStageBytes; // two transpose buffers
+    uint64_t *full = reinterpret_cast<uint64_t *>(Tb + 2 * kAxis0TBytes);
     uint64_t *empty = full + kStages;
     double *red = reinterpret_cast<double *>(empty + kStages);
     float *fred = reinterpret_cast<float *>(red + kConsumerWarps * 4);
@@ -2128,7 +2128,12 @@ __global__ void __launch_bounds__(kThreads, 2) axis0_kernel(const __grid_constan
         named_barrier_sync(1, kConsumers);
         if (!*ready)
             break;
-        A0::transpose(stages + s * kStageBytes, Tb, tid);
+        // this tile's transpose buffer: the other one may still be read by
+        // threads finishing the previous tile; a buffer is written again only
+        // two tiles later, after every thread has passed the next tile's
+        // first barrier (and so has read it)
+        uint8_t *Tc = Tb + (it & 1) * kAxis0TBytes;
+        A0::transpose(stages + s * kStageBytes, Tc, tid);
         named_barrier_sync(1, kConsumers); // S is read, T is written
         if (lane == 0)
             mbar_arrive(&empty[s]);
@@ -2137,9 +2142,8 @@ __global__ void __launch_bounds__(kThreads, 2) axis0_kernel(const __grid_constan
         for (int i = 0; i < 4; ++i)
             if (i < p.cpt) {
                 const int j = tid + i * kConsumers;
-                raw[i] = A0::load(Tb, j >> 4, j & 15);
+                raw[i] = A0::load(Tc, j >> 4, j & 15);
             }
-        named_barrier_sync(1, kConsumers); // T is read: the next tile may overwrite it
         const int64_t rt = t / p.n_col_tiles, ct = t - rt * p.n_col_tiles;
         const int64_t row0 = rt * A0::kRows, col0 = ct * kAxis0K;
         acc.et = acc.ep = acc.eq = acc.eqd = 0.0f;
