@@ -242,6 +242,41 @@ __device__ __forceinline__ float quant_fp8_as(const float (&v)[VPC], bool fast, 
     return err_energy_neg<VPC>(v, dn);
 }
 
+// quant_fp8_as (STORE, fast division decided by the caller) that adds the
+// squared errors to the packed chains acc2 instead of returning their sum:
+// the same terms, summed in two chains across the tile's chunks.
+template <int VPC>
+__device__ __forceinline__ void quant_fp8_acc(const float (&v)[VPC], bool fast, const Recip &rc, const ChunkOut &o,
+                                              f32x2 &acc2)
+{
+    float qn[VPC], decn[VPC], dn[VPC];
+    neg_quotients<VPC>(v, rc, fast, qn);
+    uint16_t h[VPC / 2];
+#pragma unroll
+    for (int t = 0; t < VPC / 2; ++t) {
+        h[t] = cvt_e4m3x2h(qn[2 * t], qn[2 * t + 1]);
+        const float2 f = e4m3x2h_to_f32(h[t]);
+        decn[2 * t] = f.x;
+        decn[2 * t + 1] = f.y;
+    }
+    scale_values<VPC>(decn, rc.b, dn);
+    uint32_t c[VPC / 4];
+#pragma unroll
+    for (int t = 0; t < VPC / 4; ++t)
+        c[t] = (static_cast<uint32_t>(h[2 * t]) | (static_cast<uint32_t>(h[2 * t + 1]) << 16)) ^ 0x80808080u;
+    if (o.valid) {
+        if constexpr (VPC == 4)
+            *reinterpret_cast<uint32_t *>(o.val) = c[0];
+        else
+            *reinterpret_cast<uint2 *>(o.val) = make_uint2(c[0], c[1]);
+    }
+#pragma unroll
+    for (int i = 0; i < VPC / 2; ++i) {
+        const f32x2 e = add2(pack2(v[2 * i], v[2 * i + 1]), pack2(dn[2 * i], dn[2 * i + 1]));
+        acc2 = fma2(e, e, acc2);
+    }
+}
+
 // Integer rounding by the magic constant 1.5 * 2^23: for |q| < 2^22 the sum
 // q + M rounds q to the nearest integer (ties to even) in its low mantissa
 // bits, and (q + M) - M is that integer exactly.
@@ -525,6 +560,9 @@ __device__ __forceinline__ float quant_energy_only(const float (&v)[VPC], float 
 struct Acc {
     float et, ep, eq, eqd; // energies of the current tile (binary32)
     float amax_kept, amax_all;
+    // FP8 of a packed 2:4 selection: the squared errors' two packed chains
+    // over the tile (added to eq where the tile's energies are taken)
+    f32x2 eq2 = 0ull;
 };
 
 // Per-CTA constants of a pass: the tensor scales (as reciprocals), the NVFP4
@@ -777,7 +815,7 @@ __device__ __forceinline__ void finish_chunk(const PassParams &p, const typename
             // the overflow guard as two packed comparisons of the kept values
             // with the CTA's limit (equivalent to quot_fast on their maximum)
             const bool fast = c.rst.fast && !(c.guard && bf16x2_max_ge_abs(sl.k0, sl.k1, c.lim2));
-            eq = quant_fp8_as<VPC, true>(v, fast, c.rst, o);
+            quant_fp8_acc<VPC>(v, fast, c.rst, o, acc.eq2);
         } else {
             eq = quant_fp8<VPC, true>(v, vmax, c.rst, c.guard, o);
         }
@@ -1710,6 +1748,10 @@ __global__ void __launch_bounds__(kStreamThreads, (StreamOcc<T, PAT, (SC & 1), F
             e_prune += acc.ep;
         if constexpr (FMT != kAmax && FMT != kNone && PAT != kDense)
             e_q += acc.eq;
+        if constexpr (FMT == kFp8 && PAT == kSparse24) {
+            e_q += lo2(acc.eq2) + hi2(acc.eq2);
+            acc.eq2 = 0ull;
+        }
         if constexpr (FMT != kAmax && FMT != kNone && (PAT == kDense || FMT == kEnergy))
             e_qd += acc.eqd;
         ua += sa;
@@ -2161,6 +2203,10 @@ __global__ void __launch_bounds__(kThreads, 2) axis0_kernel(const __grid_constan
             e_prune += acc.ep;
             e_q += acc.eq;
             e_qd += acc.eqd;
+        }
+        if constexpr (FMT == kFp8 && PAT == kSparse24) {
+            e_q += lo2(acc.eq2) + hi2(acc.eq2);
+            acc.eq2 = 0ull;
         }
     }
     if constexpr (FMT == kAmax) {

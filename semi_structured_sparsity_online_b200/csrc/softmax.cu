@@ -229,6 +229,10 @@ __global__ void __launch_bounds__(kStreamThreads) softmax_prune_kernel(const __g
                 e_prune += acc.ep;
             if constexpr (FMT != kNone && PAT != kDense)
                 e_q += acc.eq;
+            if constexpr (FMT == kFp8 && PAT == kSparse24) {
+                e_q += lo2(acc.eq2) + hi2(acc.eq2);
+                acc.eq2 = 0ull;
+            }
             if constexpr (FMT != kNone && PAT == kDense)
                 e_qd += acc.eqd;
         }
