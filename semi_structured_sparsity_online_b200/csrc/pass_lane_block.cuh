@@ -7,7 +7,12 @@
 // (magnitude score, round-to-nearest), §3 (formats; one read of the input, the
 // kept values and indices written once), §4 (error energies), §6 (pairwise
 // 4:8). The arithmetic of every value is that of the stream kernel
-// (pass_impl.cuh); only the assignment of elements to lanes differs.
+// (pass_impl.cuh); only the assignment of elements to lanes differs (MXFP4
+// forms its error terms in quotient units and scales them by 2^2e, the same
+// values in the normal range). The same kernel serves the passes over the
+// operand rotated along k (rotate_lane32, the stream kernel's rotation value
+// by value), and its loads run one unit ahead for the formats where that
+// measured faster (LbPipe).
 //
 // Layout. A unit is 1024 consecutive columns of one row, served by one warp;
 // lane L holds columns 32L .. 32L + 31 of it (four consecutive 16-byte
