@@ -82,18 +82,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64
     }
 }
 
-// 2-D tiled TMA load of one box into shared memory, completing on `bar`.
-// Coordinates are {inner (contiguous) element index, outer index}.
-__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int32_t c_inner,
-                                            int32_t c_outer, uint64_t *bar, uint64_t policy)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
-        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(c_inner), "r"(c_outer), "r"(smem_u32(bar)), "l"(policy)
-        : "memory");
-}
-
 // 3-D tiled TMA load: {inner, outer, operand of a batch}.
 __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int32_t c0, int32_t c1, int32_t c2,
                                             uint64_t *bar, uint64_t policy)
@@ -442,16 +430,6 @@ __device__ __forceinline__ float div_fast(float a, const Recip &r)
     return with_sign_of(__fmaf_rn(res, r.y, q0), a);
 }
 
-// Two quotients with packed arithmetic (the sign is restored by the caller
-// through with_sign_of on each half).
-__device__ __forceinline__ f32x2 div_fast2(f32x2 a, const Recip &r)
-{
-    const f32x2 y2 = pack2(r.y, r.y), nb2 = pack2(r.nb, r.nb);
-    const f32x2 q0 = mul2(a, y2);
-    const f32x2 res = fma2(q0, nb2, a);
-    return fma2(res, y2, q0);
-}
-
 // Negated quotients -(a / b) of two values: Markstein's correction run with
 // -y in place of y (q0 = RN(a (-y)), r = a + q0 b exact, RN(q0 + r (-y))).
 // Because rounding to nearest is symmetric this is exactly -RN(a / b) where
@@ -474,30 +452,7 @@ __device__ __forceinline__ f32x2 neg_div_fast2(f32x2 a, const Recip &r)
 // (2,3)'s winner, (2,3) when (2,3)'s loser beats (0,1)'s winner, and the two
 // winners otherwise: four comparisons in all. A later index wins a comparison
 // only when its score is strictly larger.
-struct Pick {
-    bool p;     // winner of (0,1) is 1
-    bool q;     // winner of (2,3) is 3
-    bool both01; // both kept elements are 0 and 1
-    bool both23; // both kept elements are 2 and 3
-    uint32_t nib;
-};
-
-__device__ __forceinline__ Pick top2_of_4(float s0, float s1, float s2, float s3)
-{
-    Pick k;
-    k.p = s1 > s0;
-    k.q = s3 > s2;
-    const float w01 = k.p ? s1 : s0, l01 = k.p ? s0 : s1;
-    const float w23 = k.q ? s3 : s2, l23 = k.q ? s2 : s3;
-    const bool ta = w23 > l01;  // (0,1)'s loser does not beat (2,3)'s winner
-    const bool tb = l23 > w01;  // (2,3)'s loser beats (0,1)'s winner
-    k.both01 = !ta;
-    k.both23 = tb;
-    const uint32_t mixed = static_cast<uint32_t>(k.p) | ((2u + static_cast<uint32_t>(k.q)) << 2);
-    k.nib = k.both01 ? 0x4u : (k.both23 ? 0xEu : mixed);
-    return k;
-}
-
+//
 // One 2:4 group: the kept values in index order, the dropped values, the
 // group's energy, the energy of its dropped pair and the metadata nibble. With
 // kAbs the scores are the magnitudes of the values themselves (compared

@@ -74,8 +74,6 @@ template <> struct Elem<float> {
     }
 };
 
-__device__ __forceinline__ float sq(float a) { return a * a; }
-
 // ---------------------------------------------------------------------------
 // quantizers of one chunk's values (VPC = 4 kept or 8 dense values); every
 // lane of the warp calls them (group reductions shuffle across lanes)
