@@ -314,3 +314,28 @@ def test_algorithmic_bytes_match_the_stored_layouts():
     nw = bench.W_M * bench.W_K
     assert ab["weight_wanda_24_int4"] == 2 * nw + 4 * bench.W_K + nw // 4 + 4 * (nw // 256) + nw // 8
     assert ab["weight_dense_int3"] == 2 * nw + nw // 2 + 4 * (nw // 128)
+
+
+def test_bench_traffic_is_tied_to_the_kernel_sources(tmp_path, monkeypatch):
+    """The bench reports a kernel's ncu DRAM bytes only while the kernel
+    sources hash to the value recorded beside them: any change to a source
+    makes the figure stale, and the bench reports none."""
+    import json
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    src = tmp_path / "semi_structured_sparsity_online_b200" / "csrc"
+    src.mkdir(parents=True)
+    (src / "a.cu").write_text("kernel a")
+    (src / "b.cuh").write_text("header b")
+    (src / "notes.txt").write_text("not a source")
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    sha = bench.kernel_source_sha()
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps({"source_sha": sha, "sweep_fused_24_nvfp4": 123}))
+    assert bench.measured_traffic("sweep_fused_24_nvfp4") == 123
+    assert bench.measured_traffic("sweep_dense_nvfp4") is None
+    (src / "notes.txt").write_text("edited, still not a source")
+    assert bench.measured_traffic("sweep_fused_24_nvfp4") == 123
+    (src / "b.cuh").write_text("header b, changed")
+    assert bench.measured_traffic("sweep_fused_24_nvfp4") is None
