@@ -7,7 +7,9 @@
 // values), E_q of the kept values quantized to the 2:4 side's format (2m
 // bits), E_q,dense of every value quantized to the dense side's format (m + 1
 // bits). Nothing but the energies is written. The arithmetic of every value is
-// that of the stream kernel's energy pass; a lane holds 32 consecutive
+// that of the stream kernel's energy pass (MXFP4's error terms formed in
+// quotient units and scaled by 2^2e, the same values in the normal range); it
+// also serves the operand rotated along k (ROT). A lane holds 32 consecutive
 // elements as in the lane-block pass (pass_lane_block.cuh), so each side's
 // blocks and groups are reduced inside the lane or over a few lanes, and
 // each side's division path is voted once per unit.
